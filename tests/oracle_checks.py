@@ -1,0 +1,347 @@
+"""Checks that pin the fp64 oracle to things other than itself.
+
+Each ``check_*`` function raises AssertionError when the oracle currently
+routed by ``oracle`` (the default build, or a planted-mistake build selected
+with ``oracle.using_library``) disagrees with:
+
+* closed forms (dt -> 0 gives y = D x; scalar geometric series; a hand-worked
+  case with softplus(0) = ln 2 and exp(-ln 2) = 1/2; SiLU through an identity
+  conv tap);
+* library routines for special cases (``np.convolve`` for the causal conv,
+  ``np.logaddexp`` for softplus);
+* the brute-force L x L state-space-duality matrix M[t,s] = (C_t.B_s)
+  exp(sum_{r=s+1..t} dt_r A) dt_s ("Hybrid Architectures ..." summary page,
+  section 2: state space duality recasts the scan as a matrix product;
+  appendix O: Mamba's implicit attention matrix);
+* an independent chunked evaluation of the same operator at several chunk
+  lengths (chunk-size invariance; chunk length 1 is the recurrence itself and
+  chunk length L is the full matrix);
+* invariants: linearity of y - D x in x, causality, state hand-off between
+  calls, prefill(L) + one decode step = prefill(L + 1), conv-state hand-off;
+* the Mamba cache-size formula of the same page's appendix C, which fixes the
+  element counts of the conv state and the SSM state.
+
+All inputs are small and seeded so the whole set runs in seconds on a CPU.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+import oracle
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _close(a, b, tol, what):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, f"{what}: shape {a.shape} vs {b.shape}"
+    scale = max(1.0, float(np.max(np.abs(b))) if b.size else 1.0)
+    err = float(np.max(np.abs(a - b))) if a.size else 0.0
+    assert err <= tol * scale, f"{what}: max abs err {err:.3e} > {tol:.1e} * {scale:.3e}"
+
+
+def _random_scan_inputs(rng, b=2, L=48, H=4, P=5, N=6, G=2, init=True, a_lo=0.05, a_hi=2.0):
+    x = rng.standard_normal((b, L, H, P))
+    B = rng.standard_normal((b, L, G, N)) / math.sqrt(N)
+    C = rng.standard_normal((b, L, G, N)) / math.sqrt(N)
+    dt_raw = rng.uniform(-4.0, 1.0, (b, L, H))
+    dt_bias = rng.standard_normal(H) * 0.5
+    A = -np.exp(rng.uniform(math.log(a_lo), math.log(a_hi), H))
+    D = rng.standard_normal(H)
+    h0 = rng.standard_normal((b, H, P, N)) * 0.3 if init else None
+    return dict(x=x, B=B, C=C, dt_raw=dt_raw, dt_bias=dt_bias, A=A, D=D, init_state=h0)
+
+
+def _scan(inp):
+    return oracle.selective_scan(inp["x"], inp["B"], inp["C"], inp["dt_raw"], inp["A"],
+                                 inp["dt_bias"], inp["D"], inp["init_state"], nthreads=2)
+
+
+# ----------------------------------------------------------------------------
+# closed forms
+# ----------------------------------------------------------------------------
+
+def check_dt_to_zero():
+    """dt_raw -> -40 makes dt = softplus(-40) ~ 4e-18: the state keeps its
+    initial value and y_t = C_t.h0 + D x_t (with h0 = 0: y = D x)."""
+    inp = _random_scan_inputs(_rng(1))
+    inp["dt_raw"] = np.full_like(inp["dt_raw"], -40.0)
+    inp["dt_bias"] = np.zeros_like(inp["dt_bias"])
+    y, fs = _scan(inp)
+    _close(fs, inp["init_state"], 1e-14, "dt->0 final state")
+    H, G = inp["x"].shape[2], inp["B"].shape[2]
+    g_of_h = np.arange(H) // (H // G)
+    Cg = inp["C"][:, :, g_of_h, :]                               # [b,L,H,N]
+    expect = np.einsum("blhn,bhpn->blhp", Cg, inp["init_state"]) + inp["D"][None, None, :, None] * inp["x"]
+    _close(y, expect, 1e-13, "dt->0 output")
+    inp["init_state"] = None
+    y0, fs0 = _scan(inp)
+    _close(y0, inp["D"][None, None, :, None] * inp["x"], 1e-15, "dt->0, zero state: y = D x")
+    assert np.all(np.abs(fs0) < 1e-15), "dt->0, zero state: final state must stay 0"
+
+
+def check_geometric_series():
+    """Constant dt, B, C, x and one head: h_t = a h_{t-1} + dt x B gives
+    h_t = a^{t+1} h0 + dt x B (1 - a^{t+1}) / (1 - a), a = exp(dt A)."""
+    L, P, N = 40, 3, 4
+    rng = _rng(2)
+    Bv = rng.standard_normal(N)
+    Cv = rng.standard_normal(N)
+    xv = rng.standard_normal(P)
+    h0 = rng.standard_normal((P, N))
+    v, A, D = -0.7, -0.9, 0.25
+    dt = math.log1p(math.exp(v))
+    a = math.exp(dt * A)
+    x = np.broadcast_to(xv, (1, L, 1, P)).copy()
+    B = np.broadcast_to(Bv, (1, L, 1, N)).copy()
+    C = np.broadcast_to(Cv, (1, L, 1, N)).copy()
+    y, fs = oracle.selective_scan(x, B, C, np.full((1, L, 1), v), np.array([A]),
+                                  None, np.array([D]), h0[None, None])
+    t = np.arange(L)[:, None]
+    geo = (1.0 - a ** (t + 1)) / (1.0 - a)                       # [L,1]
+    expect = (a ** (t + 1)) * (h0 @ Cv)[None, :] + dt * (Cv @ Bv) * geo * xv[None, :] + D * xv[None, :]
+    _close(y[0, :, 0, :], expect, 1e-13, "geometric series y")
+    fs_expect = a ** L * h0 + dt * np.outer(xv, Bv) * (1.0 - a ** L) / (1.0 - a)
+    _close(fs[0, 0], fs_expect, 1e-13, "geometric series final state")
+
+
+def check_hand_worked():
+    """dt_raw = 0, A = -1, B = C = x = 1, D = 3, one state: dt = softplus(0) =
+    ln 2 and exp(dt A) = 1/2, so h_t = ln2 (2 - 2^-t) and y_t = h_t + 3."""
+    L = 12
+    ones = np.ones((1, L, 1, 1))
+    y, fs = oracle.selective_scan(ones, ones, ones, np.zeros((1, L, 1)), np.array([-1.0]),
+                                  None, np.array([3.0]))
+    expect = [math.log(2.0) * (2.0 - 2.0 ** (-t)) + 3.0 for t in range(L)]
+    _close(y[0, :, 0, 0], expect, 1e-15, "hand-worked y")
+    _close(fs.reshape(-1), [math.log(2.0) * (2.0 - 2.0 ** (-(L - 1)))], 1e-15, "hand-worked state")
+
+
+def check_conv_identity_tap():
+    """Taps (0,..,0,1) and no bias reduce the conv to the identity, so
+    u = SiLU(xBC) = xBC / (1 + exp(-xBC)); SiLU(0) = 0."""
+    rng = _rng(3)
+    xbc = rng.standard_normal((2, 9, 7)) * 3.0
+    xbc[0, 0, 0] = 0.0
+    k = 4
+    w = np.zeros((7, k))
+    w[:, k - 1] = 1.0
+    st = rng.standard_normal((2, 7, k))
+    u, _ = oracle.conv1d_silu(xbc, w, None, st)
+    _close(u, xbc / (1.0 + np.exp(-xbc)), 1e-15, "identity tap = SiLU")
+    assert u[0, 0, 0] == 0.0
+
+
+# ----------------------------------------------------------------------------
+# library routines for special cases
+# ----------------------------------------------------------------------------
+
+def check_conv_matches_np_convolve():
+    """Causal depthwise conv with a cached left context equals np.convolve of
+    the extended sequence with the reversed taps (valid part), then SiLU;
+    the new cache is the last k inputs of the extended sequence."""
+    rng = _rng(4)
+    for (b, L, cd, k) in [(2, 11, 5, 4), (1, 2, 3, 4), (3, 1, 4, 4), (1, 7, 2, 3)]:
+        xbc = rng.standard_normal((b, L, cd))
+        w = rng.standard_normal((cd, k)) * 0.5
+        bias = rng.standard_normal(cd) * 0.3
+        st = rng.standard_normal((b, cd, k))
+        u, st2 = oracle.conv1d_silu(xbc, w, bias, st)
+        for bi in range(b):
+            for c in range(cd):
+                ext = np.concatenate([st[bi, c, :], xbc[bi, :, c]])           # times -k .. L-1
+                pre = np.convolve(ext[1:], w[c, ::-1], mode="valid") + bias[c]  # starts at time -k+1
+                _close(u[bi, :, c], pre / (1.0 + np.exp(-pre)), 1e-14, f"conv vs np.convolve {b,L,cd,k}")
+                _close(st2[bi, c, :], ext[-k:], 0.0, "conv new cache")
+        u0, none = oracle.conv1d_silu(xbc, w, bias, None)
+        assert none is None
+        for bi in range(b):
+            for c in range(cd):
+                ext = np.concatenate([np.zeros(k - 1), xbc[bi, :, c]])
+                pre = np.convolve(ext, w[c, ::-1], mode="valid") + bias[c]
+                _close(u0[bi, :, c], pre / (1.0 + np.exp(-pre)), 1e-14, "conv, zero left context")
+
+
+def _softplus(v):
+    return np.logaddexp(0.0, v)
+
+
+def check_matrix_form():
+    """Brute-force L x L SSD matrix with the initial-state term:
+    y_t = sum_{s<=t} (C_t.B_s) exp(sum_{r=s+1..t} dt_r A) dt_s x_s
+          + exp(sum_{r=0..t} dt_r A) C_t.h0 + D x_t,
+    with dt = np.logaddexp(0, dt_raw + dt_bias) and head h on group h/(H/G)."""
+    inp = _random_scan_inputs(_rng(5), b=2, L=37, H=4, P=3, N=5, G=2)
+    y, fs = _scan(inp)
+    x, B, C = inp["x"], inp["B"], inp["C"]
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    for bi in range(b):
+        for h in range(H):
+            g = h // (H // G)
+            dt = _softplus(inp["dt_raw"][bi, :, h] + inp["dt_bias"][h])
+            lg = dt * inp["A"][h]
+            M = np.zeros((L, L))
+            for t in range(L):
+                for s in range(t + 1):
+                    M[t, s] = (C[bi, t, g] @ B[bi, s, g]) * math.exp(lg[s + 1: t + 1].sum()) * dt[s]
+            h0 = inp["init_state"][bi, h]
+            decay0 = np.exp(np.cumsum(lg))                                   # exp(sum_{r<=t})
+            y_ref = M @ x[bi, :, h, :] + decay0[:, None] * (C[bi, :, g, :] @ h0.T) + inp["D"][h] * x[bi, :, h, :]
+            _close(y[bi, :, h, :], y_ref, 1e-12, f"matrix form y (b={bi}, h={h})")
+            # final state: h_L = exp(sum lg) h0 + sum_s exp(sum_{r>s} lg) dt_s x_s B_s^T
+            w_s = np.array([math.exp(lg[s + 1:].sum()) * dt[s] for s in range(L)])
+            fs_ref = decay0[-1] * h0 + (x[bi, :, h, :] * w_s[:, None]).T @ B[bi, :, g, :]
+            _close(fs[bi, h], fs_ref, 1e-12, f"matrix form final state (b={bi}, h={h})")
+
+
+def chunked_ssd(inp, Q):
+    """Chunked evaluation of the same operator (independent of the oracle):
+    intra-chunk masked (C B^T o L) X, inter-chunk state passing, C.h_prev."""
+    x, B, C = inp["x"], inp["B"], inp["C"]
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    y = np.zeros_like(x)
+    fs = np.zeros((b, H, P, N))
+    for bi in range(b):
+        for h in range(H):
+            g = h // (H // G)
+            dt = _softplus(inp["dt_raw"][bi, :, h] + inp["dt_bias"][h])
+            a = dt * inp["A"][h]
+            hs = np.zeros((P, N)) if inp["init_state"] is None else inp["init_state"][bi, h].copy()
+            for s0 in range(0, L, Q):
+                s1 = min(L, s0 + Q)
+                cum = np.cumsum(a[s0:s1])
+                seg = cum[:, None] - cum[None, :]
+                Lm = np.where(np.tril(np.ones_like(seg)) > 0, np.exp(np.minimum(seg, 0.0)), 0.0)
+                Xc, Bc, Cc = x[bi, s0:s1, h, :], B[bi, s0:s1, g, :], C[bi, s0:s1, g, :]
+                Gm = Cc @ Bc.T
+                y_diag = (Gm * Lm * dt[None, s0:s1]) @ Xc
+                y_off = np.exp(cum)[:, None] * (Cc @ hs.T)
+                y[bi, s0:s1, h, :] = y_diag + y_off + inp["D"][h] * Xc
+                wj = np.exp(cum[-1] - cum) * dt[s0:s1]
+                hs = math.exp(cum[-1]) * hs + (Xc * wj[:, None]).T @ Bc
+            fs[bi, h] = hs
+    return y, fs
+
+
+def check_chunk_size_invariance():
+    """The chunked form at chunk 1, 8, 64 and L (incl. a ragged last chunk)
+    equals the oracle's token-by-token recurrence to rounding."""
+    inp = _random_scan_inputs(_rng(6), b=1, L=200, H=2, P=4, N=8, G=1)
+    y, fs = _scan(inp)
+    for Q in (1, 8, 64, 200, 256):
+        yc, fc = chunked_ssd(inp, Q)
+        _close(y, yc, 1e-11, f"chunked Q={Q} y")
+        _close(fs, fc, 1e-11, f"chunked Q={Q} final state")
+
+
+# ----------------------------------------------------------------------------
+# invariants
+# ----------------------------------------------------------------------------
+
+def check_linearity_in_x():
+    """For fixed dt, B, C and zero initial state, y - D x is linear in x."""
+    rng = _rng(7)
+    inp = _random_scan_inputs(rng, init=False)
+    x1 = inp["x"]
+    x2 = rng.standard_normal(x1.shape)
+    Dx = lambda x: inp["D"][None, None, :, None] * x
+    f = lambda x: _scan(dict(inp, x=x))[0] - Dx(x)
+    _close(f(x1 + 2.5 * x2), f(x1) + 2.5 * f(x2), 1e-12, "linearity")
+
+
+def check_causality():
+    """Changing any input at time >= t0 leaves y[:t0] bit-identical."""
+    rng = _rng(8)
+    inp = _random_scan_inputs(rng)
+    y, _ = _scan(inp)
+    t0 = 21
+    pert = {k: (v.copy() if isinstance(v, np.ndarray) else v) for k, v in inp.items()}
+    for key in ("x", "B", "C", "dt_raw"):
+        pert[key][:, t0:] += rng.standard_normal(pert[key][:, t0:].shape)
+    y2, _ = _scan(pert)
+    assert np.array_equal(y[:, :t0], y2[:, :t0]), "causality"
+    assert not np.allclose(y[:, t0:], y2[:, t0:]), "later outputs must change"
+
+
+def check_state_handoff():
+    """scan(0..L) equals scan(0..t) followed by scan(t..L) started from the
+    first call's final state."""
+    inp = _random_scan_inputs(_rng(9), L=50)
+    y, fs = _scan(inp)
+    t = 17
+    first = {k: (v[:, :t] if k in ("x", "B", "C", "dt_raw") else v) for k, v in inp.items()}
+    ya, fa = _scan(first)
+    second = {k: (v[:, t:] if k in ("x", "B", "C", "dt_raw") else v) for k, v in inp.items()}
+    second["init_state"] = fa
+    yb, fb = _scan(second)
+    _close(np.concatenate([ya, yb], axis=1), y, 1e-13, "hand-off y")
+    _close(fb, fs, 1e-13, "hand-off final state")
+
+
+def check_decode_step_extends_prefill():
+    """prefill(L) then one decode step equals prefill(L+1)."""
+    inp = _random_scan_inputs(_rng(10), L=30)
+    y, fs = _scan(inp)
+    L = 29
+    pre = {k: (v[:, :L] if k in ("x", "B", "C", "dt_raw") else v) for k, v in inp.items()}
+    _, f_pre = _scan(pre)
+    yd, fd = oracle.state_update(f_pre, inp["x"][:, L], inp["B"][:, L], inp["C"][:, L],
+                                 inp["dt_raw"][:, L], inp["A"], inp["dt_bias"], inp["D"])
+    _close(yd, y[:, L], 1e-13, "decode y")
+    _close(fd, fs, 1e-13, "decode state")
+
+
+def check_conv_state_handoff():
+    """conv over [0, L) equals conv over [0, t) then [t, L) carrying the cache,
+    including calls shorter than the conv width."""
+    rng = _rng(11)
+    b, L, cd, k = 2, 13, 6, 4
+    xbc = rng.standard_normal((b, L, cd))
+    w = rng.standard_normal((cd, k))
+    bias = rng.standard_normal(cd)
+    st0 = rng.standard_normal((b, cd, k))
+    u, st = oracle.conv1d_silu(xbc, w, bias, st0)
+    cur = st0
+    pieces = []
+    for (s0, s1) in [(0, 2), (2, 3), (3, 9), (9, 13)]:
+        part, cur = oracle.conv1d_silu(xbc[:, s0:s1], w, bias, cur)
+        pieces.append(part)
+    _close(np.concatenate(pieces, axis=1), u, 1e-15, "conv hand-off output")
+    _close(cur, st, 0.0, "conv hand-off cache")
+
+
+def check_cache_size_formula():
+    """Appendix C: a Mamba layer caches d_ssm*d_state + N_conv*(2*d_state + d_ssm)
+    values (one group).  The oracle's SSM state [H,P,N] and conv cache
+    [conv_dim, k] per sequence must hold exactly that many."""
+    H, P, N, G, k = 3, 4, 5, 1, 4
+    inp = _random_scan_inputs(_rng(12), b=1, L=3, H=H, P=P, N=N, G=G)
+    _, fs = _scan(inp)
+    cd = H * P + 2 * G * N
+    _, cs = oracle.conv1d_silu(np.zeros((1, 2, cd)), np.zeros((cd, k)), None, np.zeros((1, cd, k)))
+    d_ssm, d_state = H * P, N
+    assert fs[0].size + cs[0].size == d_ssm * d_state + k * (2 * d_state + d_ssm)
+
+
+ALL_CHECKS = [
+    check_dt_to_zero,
+    check_geometric_series,
+    check_hand_worked,
+    check_conv_identity_tap,
+    check_conv_matches_np_convolve,
+    check_matrix_form,
+    check_chunk_size_invariance,
+    check_linearity_in_x,
+    check_causality,
+    check_state_handoff,
+    check_decode_step_extends_prefill,
+    check_conv_state_handoff,
+    check_cache_size_formula,
+]

@@ -1,0 +1,61 @@
+"""Plant plausible mistakes in a copy of the oracle's C source and check that
+the pins catch every one of them (CPU only).
+
+Each mutant is a one-token edit of the kind a careful reader could still miss:
+a dropped term, a wrong sign, a wrong index, operands swapped.  The edited
+copy is compiled into a temporary directory and routed to with
+``oracle.using_library``; the default oracle build is never touched.
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+import oracle_checks
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "ssd_oracle.c")
+
+MUTANTS = {
+    "drop_D_term": ("yt[p] = acc + Dh * xt[p];", "yt[p] = acc;"),
+    "decay_sign": ("const double a = exp(dt * A);", "const double a = exp(-dt * A);"),
+    "decay_missing_dt": ("const double a = exp(dt * A);", "const double a = exp(A);"),
+    "input_missing_dt": ("row[n] = a * row[n] + dt * xt[p] * Bt[n];", "row[n] = a * row[n] + xt[p] * Bt[n];"),
+    "output_before_update": (
+        "row[n] = a * row[n] + dt * xt[p] * Bt[n];\n                acc += Ct[n] * row[n];",
+        "acc += Ct[n] * row[n];\n                row[n] = a * row[n] + dt * xt[p] * Bt[n];"),
+    "B_C_swapped": ("acc += Ct[n] * row[n];", "acc += Bt[n] * row[n];"),
+    "group_map_modulo": ("const int64_t g = h / (H / G);", "const int64_t g = h % G;"),
+    "softplus_no_abs": ("log1p(exp(-fabs(v)))", "log1p(exp(-v))"),
+    "dt_bias_ignored": ("J->dt_raw[(bi * L + t) * H + h] + bias", "J->dt_raw[(bi * L + t) * H + h]"),
+    "init_state_ignored": ("if (J->init_state) memcpy", "if (0) memcpy"),
+    "silu_sign": ("return v / (1.0 + exp(-v));", "return v / (1.0 + exp(v));"),
+    "conv_taps_reversed": ("acc += w[c * k + j] * hist[(t - k + 1 + j) + k];",
+                           "acc += w[c * k + (k - 1 - j)] * hist[(t - k + 1 + j) + k];"),
+    "conv_off_by_one": ("acc += w[c * k + j] * hist[(t - k + 1 + j) + k];",
+                        "acc += w[c * k + j] * hist[(t - k + j) + k];"),
+    "conv_cache_shift": ("conv_state[(bi * conv_dim + c) * k + j] = hist[L + j];",
+                         "conv_state[(bi * conv_dim + c) * k + j] = hist[L + j - (j > 0)];"),
+    "conv_bias_dropped": ("double acc = bias ? bias[c] : 0.0;", "double acc = 0.0;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not unique in oracle source"
+    mutated = tmp_path / "mutant.c"
+    mutated.write_text(src.replace(old, new))
+    lib_path = str(tmp_path / "libmutant.so")
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+                           str(mutated), "-o", lib_path, "-lm"])
+    lib = oracle.open_library(lib_path)
+    caught = []
+    with oracle.using_library(lib):
+        for check in oracle_checks.ALL_CHECKS:
+            try:
+                check()
+            except AssertionError:
+                caught.append(check.__name__)
+    assert caught, f"planted mistake {name!r} passed every pin"
