@@ -1,0 +1,476 @@
+"""Benchmark of the Mamba-2 layer hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one prefill layer call over one batch of the FRANKENSTALLM-H 3B
+layer shape (batch 8 x 2048 tokens, 40 heads x 64, d_state 128, 8 groups,
+chunk 128, conv 4, bf16 I/O, fp32 state): causal conv1d+SiLU, then the
+chunked SSD scan (dt softplus, chunk cumsum, C.B^T o L times X, chunk states,
+state passing, C.h + D.x), with inputs resident in HBM.  Rank 0 prints one
+JSON line.  Next to the headline prefill number the line carries:
+  roofline      the scan kernel's achieved HBM GB/s (algorithmic bytes per
+                launch / its CUDA-event duration) against the measured peak;
+  scan_only     tokens/s of the scan kernel alone;
+  decode        one decode step of the 256-sequence, 128-head workload
+                (conv-cache roll + state update), state-update GB/s;
+  e2e           the same prefill step through the public API with the step's
+                inputs copied from pinned host memory and y + final state
+                copied back, inside the timed region;
+  cpu_baseline  the fp64 oracle timed on this host's cores on a bounded sample.
+Multi-GPU: one process per GPU (torchrun); each rank runs its own batch
+(independent sequences, no data-path collective): weak scaling.
+``--impl reference`` times the fp64 CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from ssd_selective_scan_b200 import synth  # noqa: E402
+
+METRIC = "SSD prefill scan tokens/s/layer & % roofline; decode state-update HBM GB/s"
+PREFILL = synth.CONFIGS[1]
+DECODE = synth.CONFIGS[4]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+# ----------------------------------------------------------------------------
+# algorithmic work (bytes the method must move; FLOPs of the causal tiles)
+# ----------------------------------------------------------------------------
+
+def scan_bytes_per_token(s) -> int:
+    """x, B, C, dt read and y written once: e * (2*H*P + 2*G*N + H)."""
+    return s.elem_bytes * (2 * s.H * s.P + 2 * s.G * s.N + s.H)
+
+
+def scan_flops_per_token(s) -> int:
+    """causal C.B^T (G*Q*N) + causal (..)X (H*Q*P) + chunk state and C.h (4*H*P*N)."""
+    return s.G * s.Q * s.N + s.H * s.Q * s.P + 4 * s.H * s.P * s.N
+
+
+def conv_bytes_per_token(s) -> int:
+    return 2 * s.elem_bytes * s.conv_dim
+
+
+def decode_state_update_bytes(s) -> int:
+    """fp32 state read + written, x/B/C/dt read, y written."""
+    return 8 * s.b * s.H * s.P * s.N + s.elem_bytes * s.b * (s.H * s.P + 2 * s.G * s.N + s.H + s.H * s.P)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return dict(FALLBACK_PEAKS, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def scan_kernel_traffic(kernel_tag: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d.get(kernel_tag)
+        if e and e.get("source_sha") == source_digest():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def source_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "ssd_selective_scan_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: torch.device):
+        # nvidia-smi ignores CUDA_VISIBLE_DEVICES: address the GPU by UUID
+        try:
+            self.gpu = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            self.gpu = str(device.index or 0)
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100", "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.path) as f:
+                for r in csv.reader(f):
+                    if len(r) >= 9:
+                        rows.append([c.strip() for c in r])
+            os.unlink(self.path)
+        except Exception:
+            pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------
+# the prefill step, the decode step, and their timing
+# ----------------------------------------------------------------------------
+
+class PrefillStep:
+    def __init__(self, s, seed, dev):
+        from ssd_selective_scan_b200 import layer
+        self.layer = layer
+        self.s = s
+        inp = synth.layer_inputs(s, seed)
+        self.host = inp
+        self.d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+        self.conv_state = torch.zeros(s.b, s.conv_dim, s.k, dtype=s.torch_dtype, device=dev)
+        self.u = torch.empty(s.b, s.L, s.conv_dim, dtype=s.torch_dtype, device=dev)
+        self.y = torch.empty(s.b, s.L, s.H, s.P, dtype=s.torch_dtype, device=dev)
+        self.fs = torch.empty(s.b, s.H, s.P, s.N, dtype=torch.float32, device=dev)
+        self.views = layer.split_channels(self.u, s.H, s.P, s.G, s.N)
+
+    def conv(self):
+        d = self.d
+        self.layer.conv1d_silu(d["xBC"], d["w"], d["bias"], self.conv_state, out=self.u)
+
+    def scan(self):
+        d, s = self.d, self.s
+        x, B, C = self.views
+        self.layer.chunk_scan_fwd(x, B, C, d["dt_raw"], d["A"], d["dt_bias"], d["D"], None,
+                                  Q=s.Q, y=self.y, final_state=self.fs)
+
+    def __call__(self):
+        self.conv()
+        self.scan()
+
+
+class DecodeStep:
+    def __init__(self, s, seed, dev):
+        from ssd_selective_scan_b200 import layer
+        self.layer = layer
+        self.s = s
+        inp = synth.decode_inputs(s, seed)
+        self.d = {k: v.to(dev) for k, v in inp.items()}
+        self.u = torch.empty(s.b, s.conv_dim, dtype=s.torch_dtype, device=dev)
+        self.y = torch.empty(s.b, s.H, s.P, dtype=s.torch_dtype, device=dev)
+        self.views = layer.split_channels(self.u, s.H, s.P, s.G, s.N)
+
+    def conv(self):
+        d, s = self.d, self.s
+        self.layer.conv1d_silu(d["xBC"].view(s.b, 1, s.conv_dim), d["w"], None, d["conv_state"],
+                               out=self.u.view(s.b, 1, s.conv_dim))
+
+    def update(self):
+        d = self.d
+        x, B, C = self.views
+        self.layer.state_update(d["state"], x, B, C, d["dt_raw"], d["A"], d["dt_bias"], d["D"],
+                                y=self.y)
+
+
+def _events(n):
+    return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+
+def run_ours(args, rank, world, dev):
+    import torch.distributed as dist
+    s = PREFILL
+    step = PrefillStep(s, synth.config_seed(1) + rank, dev)
+    dec = DecodeStep(DECODE, synth.config_seed(4) + rank, dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    K = args.steps
+    ev_scan = _events(2 * K)
+    ev_conv = _events(2 * K)
+    t0, t1 = _events(2)
+    barrier()
+    with ClockSampler(dev) as clk:
+        t0.record()
+        for i in range(K):
+            ev_conv[2 * i].record()
+            step.conv()
+            ev_conv[2 * i + 1].record()
+            ev_scan[2 * i].record()
+            step.scan()
+            ev_scan[2 * i + 1].record()
+        t1.record()
+        barrier()
+        # keep the sampler alive over a longer stretch of identical work so the
+        # clock record has enough samples (not part of the timed number)
+        t_end = time.time() + max(0.0, 1.5 - t0.elapsed_time(t1) / 1e3)
+        while time.time() < t_end:
+            for _ in range(20):
+                step()
+            torch.cuda.synchronize()
+    clocks = clk.summary()
+    ms_total = max_over_ranks(t0.elapsed_time(t1))
+    ms_step = ms_total / K
+    scan_ms = statistics.mean(ev_scan[2 * i].elapsed_time(ev_scan[2 * i + 1]) for i in range(K))
+    conv_ms = statistics.mean(ev_conv[2 * i].elapsed_time(ev_conv[2 * i + 1]) for i in range(K))
+    scan_ms = max_over_ranks(scan_ms)
+    conv_ms = max_over_ranks(conv_ms)
+    tokens = s.b * s.L
+
+    # decode: conv-cache roll + state update, one token per sequence
+    for _ in range(max(3, args.warmup)):
+        dec.conv(); dec.update()
+    KD = max(10, K)
+    ev_u = _events(2 * KD)
+    d0, d1 = _events(2)
+    barrier()
+    d0.record()
+    for i in range(KD):
+        dec.conv()
+        ev_u[2 * i].record()
+        dec.update()
+        ev_u[2 * i + 1].record()
+    d1.record()
+    barrier()
+    dec_ms = max_over_ranks(d0.elapsed_time(d1) / KD)
+    upd_ms = max_over_ranks(statistics.mean(ev_u[2 * i].elapsed_time(ev_u[2 * i + 1]) for i in range(KD)))
+
+    # end to end through the public API: H2D inputs, the layer, D2H results
+    pin_x = step.host["xBC"].pin_memory()
+    pin_dt = step.host["dt_raw"].pin_memory()
+    out_y = torch.empty(step.y.shape, dtype=step.y.dtype, pin_memory=True)
+    out_fs = torch.empty(step.fs.shape, dtype=torch.float32, pin_memory=True)
+    KE = max(3, K // 4)
+
+    def e2e_step():
+        step.d["xBC"].copy_(pin_x, non_blocking=True)
+        step.d["dt_raw"].copy_(pin_dt, non_blocking=True)
+        step()
+        out_y.copy_(step.y, non_blocking=True)
+        out_fs.copy_(step.fs, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    e0, e1 = _events(2)
+    barrier()
+    e0.record()
+    for _ in range(KE):
+        e2e_step()
+    e1.record()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / KE)
+    h2d = pin_x.numel() * pin_x.element_size() + pin_dt.numel() * pin_dt.element_size()
+    d2h = out_y.numel() * out_y.element_size() + out_fs.numel() * 4
+
+    if rank != 0:
+        return None
+    peaks = load_peaks()
+    scan_bytes = scan_bytes_per_token(s) * tokens
+    achieved = scan_bytes / (scan_ms * 1e-3) / 1e9
+    traffic = scan_kernel_traffic("chunk_scan")
+    line = {
+        "metric": METRIC,
+        "value": world * tokens / (ms_step * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": s.name, "batch": s.b, "seq_len": s.L, "heads": s.H,
+                   "head_dim": s.P, "d_state": s.N, "groups": s.G, "chunk": s.Q, "conv": s.k,
+                   "state_dtype": "f32", "per_rank_batch": s.b,
+                   "l2": "inputs larger than L2 (xBC 151 MB, conv output 151 MB per step)",
+                   "step": "conv1d+SiLU then chunked SSD scan (one prefill layer)"},
+        "roofline": {"bound": "hbm", "kernel": "chunk_scan", "achieved": achieved,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                     "algorithmic_bytes_per_launch": scan_bytes,
+                     "algorithmic_flops_per_launch": scan_flops_per_token(s) * tokens,
+                     "tensor_frac": scan_flops_per_token(s) * tokens / (scan_ms * 1e-3) / 1e12 /
+                                    peaks["bf16_tflops"],
+                     "peak_source": peaks["source"], "launch_ms": scan_ms},
+        "scan_only": {"tokens_per_s": tokens / (scan_ms * 1e-3), "ms": scan_ms},
+        "conv": {"ms": conv_ms, "GB/s": conv_bytes_per_token(s) * tokens / (conv_ms * 1e-3) / 1e9,
+                 "frac_hbm": conv_bytes_per_token(s) * tokens / (conv_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "decode": {"workload": DECODE.name, "ms_per_step": dec_ms, "state_update_ms": upd_ms,
+                   "state_update_GB/s": decode_state_update_bytes(DECODE) / (upd_ms * 1e-3) / 1e9,
+                   "frac_hbm": decode_state_update_bytes(DECODE) / (upd_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                   "tokens_per_s": world * DECODE.b / (dec_ms * 1e-3)},
+        "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+    }
+    return line
+
+
+# ----------------------------------------------------------------------------
+# the fp64 oracle on the host (cpu_baseline and the reference arm)
+# ----------------------------------------------------------------------------
+
+def oracle_sample(seqs: int = 1):
+    """One oracle prefill-layer call on `seqs` sequences of the bench workload."""
+    import numpy as np
+    import oracle
+    s = PREFILL.with_(b=seqs)
+    inp = synth.layer_inputs(s, synth.config_seed(1))
+    f = lambda t: None if t is None else t.to(torch.float64).numpy()
+    args = (f(inp["xBC"]), f(inp["w"]), f(inp["bias"]), None, f(inp["dt_raw"]), f(inp["A"]),
+            f(inp["dt_bias"]), f(inp["D"]), None, s.H, s.P, s.G, s.N)
+    threads = min(oracle.default_threads(), s.b * s.H)
+
+    def run():
+        t = time.perf_counter()
+        oracle.layer_prefill(*args, nthreads=threads)
+        return time.perf_counter() - t
+    return s, run, threads
+
+
+def cpu_baseline(seqs: int = 1):
+    s, run, threads = oracle_sample(seqs)
+    run()  # warm (compile, page in)
+    secs = run()
+    return {"value": s.b * s.L / secs, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{s.b} of {PREFILL.b} sequences x {s.L} tokens of the bench workload, "
+                      f"conv1d+SiLU and token-by-token scan in fp64, {threads} threads",
+            "seconds": secs}
+
+
+def run_reference(args):
+    s, run, threads = oracle_sample(1)
+    for _ in range(args.warmup):
+        run()
+    secs = [run() for _ in range(args.steps)]
+    total = sum(secs)
+    v = args.steps * s.b * s.L / total
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": PREFILL.name, "batch": PREFILL.b, "seq_len": PREFILL.L,
+                   "heads": PREFILL.H, "head_dim": PREFILL.P, "d_state": PREFILL.N,
+                   "groups": PREFILL.G, "chunk": PREFILL.Q, "conv": PREFILL.k,
+                   "step": "fp64 oracle: conv1d+SiLU then token-by-token recurrence, one sequence"},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"1 of {PREFILL.b} sequences x {PREFILL.L} tokens per step"},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    import datetime
+    import torch.distributed as dist
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    from ssd_selective_scan_b200 import binding
+    binding.load()
+    line = run_ours(args, rank, world, dev)
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(1)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,194 @@
+/*
+ * ssd.h -- C ABI of libssd: the data-parallel hot path of the Mamba-2
+ * selective state-space layer on NVIDIA B200 (sm_100a).
+ *
+ * Operations (sources are the pages this library implements):
+ *   - causal depthwise conv1d + SiLU over the x | B | C channels, with a
+ *     k-column rolling cache ("Hybrid Architectures for Language Models:
+ *     Systematic Analysis and Design Insights", summary page, appendix C:
+ *     the Mamba cache holds N_conv * (2*d_state + d_ssm) conv entries and
+ *     d_ssm * d_state state entries per layer; Nemotron feasibility report,
+ *     section 1.4: conv kernel 4, SiLU);
+ *   - the chunked state-space-duality (SSD) scan: the recurrence
+ *     h_t = Abar h_{t-1} + Bbar x_t, y_t = C h_t + D x_t (summary page,
+ *     section 2 Background) evaluated chunk by chunk as matrix products
+ *     (same section: state space duality recasts the scan as hardware-
+ *     efficient matrix multiplication; chunk length 128 in the feasibility
+ *     report, sections 1.4 and 2.6);
+ *   - the single-token decode update of the same recurrence.
+ * Discretisation (the pages leave it open; this is the Mamba-2 reading):
+ *   dt = softplus(dt_raw + dt_bias), Abar = exp(dt * A), Bbar = dt * B.
+ *
+ * Notation: b batch, L tokens, H heads, P head dim, N state size (d_state),
+ * G groups of B/C (head h uses group h / (H / G)), Q chunk length,
+ * k conv width, conv_dim = H*P + 2*G*N.
+ *
+ * Conventions shared by every call:
+ *   - Every tensor argument is a DEVICE pointer owned by the caller.  The
+ *     library never allocates or frees device memory, never synchronises the
+ *     device or the stream, and keeps no mutable global state; calls are
+ *     thread-safe.  All work is enqueued on `stream` (0 = legacy default).
+ *   - I/O tensors (xBC, x, B, C, dt_raw, y, conv_state) have the element
+ *     type given by `dtype`; parameters (w, bias, A, D, dt_bias) and SSM
+ *     states are float32.  Accumulation is float32; bf16 outputs are
+ *     rounded to nearest even.
+ *   - Tensors are dense row-major in the layouts stated below, except where
+ *     a row stride is taken.  Pointers must be 16-byte aligned and inner
+ *     sizes must allow 16-byte vector access where stated.
+ *   - Return value: SSD_OK when the work was enqueued;
+ *     SSD_ERR_INVALID_ARG for a NULL required pointer, a negative or
+ *     inconsistent size, a misaligned pointer or stride, or overlapping
+ *     input/output buffers -- nothing is launched;
+ *     SSD_ERR_UNSUPPORTED for a valid combination this build has no kernel
+ *     for -- nothing is launched;
+ *     SSD_ERR_CUDA when a launch failed (cudaGetLastError was not
+ *     cudaSuccess; the error is cleared).  Asynchronous faults surface at the
+ *     caller's next synchronisation, as for any CUDA work.
+ *   - Empty work (b == 0 or L == 0) returns SSD_OK and launches no kernel;
+ *     the token tensors are then never touched and may be NULL.  The one
+ *     exception is ssd_chunk_scan_fwd with b > 0, L == 0 and a final_state:
+ *     it enqueues a copy of init_state (or zeros) into final_state.
+ */
+#ifndef SSD_H_
+#define SSD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SSD_ABI_VERSION 1
+
+/* Entry points are the library's only exported symbols. */
+#if defined(__GNUC__)
+#define SSD_API __attribute__((visibility("default")))
+#else
+#define SSD_API
+#endif
+
+typedef enum ssd_status {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1,
+    SSD_ERR_UNSUPPORTED = 2,
+    SSD_ERR_CUDA = 3,
+    SSD_ERR_TIMEOUT = 4
+} ssd_status_t;
+
+typedef enum ssd_dtype {
+    SSD_F32 = 0,
+    SSD_BF16 = 1
+} ssd_dtype_t;
+
+/* Human-readable name of a status code (static storage; never NULL). */
+SSD_API const char* ssd_status_string(ssd_status_t status);
+
+/* SSD_ABI_VERSION of the loaded library. */
+SSD_API int ssd_abi_version(void);
+
+/*
+ * Causal depthwise conv1d + SiLU.
+ *
+ *   u[t][c] = SiLU(bias[c] + sum_{j<k} w[c][j] * e[t-k+1+j][c])
+ *
+ * where e[tau] = xBC[tau] for tau >= 0 and, for tau < 0, the cached input
+ * conv_state[c][tau+k] (or 0 when conv_state is NULL).
+ *
+ *   xBC        [b][L][conv_dim]  dtype, read only
+ *   out        [b][L][conv_dim]  dtype, written; must not overlap xBC
+ *   w          [conv_dim][k]     float32 taps; tap k-1 multiplies token t
+ *   bias       [conv_dim]        float32, may be NULL (zero)
+ *   conv_state [b][conv_dim][k]  dtype, may be NULL.  On entry column j holds
+ *                                the input at time j-k before this call's
+ *                                first token; on exit it holds the last k
+ *                                inputs of (old cache | xBC), oldest first.
+ *                                With L == 1 this is the decode-step roll.
+ * Requirements: 2 <= k <= 4 (else SSD_ERR_UNSUPPORTED); conv_dim a multiple
+ * of 8 (bf16) or 4 (f32); xBC, out, conv_state 16-byte aligned.
+ */
+SSD_API ssd_status_t ssd_conv1d_silu(const void* xBC, void* out, const float* w,
+                             const float* bias, void* conv_state, int b, int L,
+                             int conv_dim, int k, ssd_dtype_t dtype,
+                             cudaStream_t stream);
+
+/*
+ * Bytes of device workspace ssd_chunk_scan_fwd needs for these sizes
+ * (0 when none).  Pure host function; depends only on its arguments and
+ * the device properties of the current device.
+ */
+SSD_API size_t ssd_chunk_scan_workspace_bytes(int b, int L, int H, int P, int N, int G,
+                                      int Q, ssd_dtype_t dtype);
+
+/*
+ * Chunked SSD scan (prefill).  For every (batch, head), with
+ * dt_t = softplus(dt_raw[t] + dt_bias), a_t = dt_t * A:
+ *
+ *   h_t = exp(a_t) h_{t-1} + dt_t x_t B_t^T        (h: P x N, h_{-1} = init)
+ *   y_t = h_t C_t + D x_t
+ *
+ * evaluated in chunks of Q tokens: intra-chunk (C B^T o L) X with the decay
+ * mask L[i][j] = exp(cum_i - cum_j) dt_j (j <= i), chunk states, inter-chunk
+ * state passing and the C . h_prev term.  The result does not depend on Q
+ * beyond rounding.
+ *
+ *   x          token t, head h, p at x[(b*L + t)*row_stride + h*P + p]
+ *   B, C       token t, group g, n at B[(b*L + t)*row_stride + g*N + n]
+ *              (x, B, C may be the three channel ranges of the conv output,
+ *              row_stride = conv_dim)                         dtype, read only
+ *   dt_raw     [b][L][H]          dtype
+ *   dt_bias    [H]                float32, may be NULL (zero)
+ *   A          [H]                float32, expected <= 0 (a decaying state)
+ *   D          [H]                float32, may be NULL (zero)
+ *   init_state [b][H][P][N]       float32, may be NULL (zero state)
+ *   y          [b][L][H][P]       dtype, written; must not overlap inputs
+ *   final_state[b][H][P][N]       float32, may be NULL; may alias init_state
+ *   workspace  device scratch of at least ssd_chunk_scan_workspace_bytes()
+ *              bytes (may be NULL when that is 0); contents on entry are
+ *              ignored; only this call uses it while it runs
+ *   status     optional device int32: set to SSD_ERR_TIMEOUT by the kernels
+ *              if a bounded wait gave up (the results are then invalid);
+ *              never cleared by the library
+ * Requirements: P a multiple of 8, N a multiple of 8, H % G == 0, Q in
+ * {64, 128}; row_stride a multiple of 8 elements (16 bytes); all pointers
+ * 16-byte aligned.
+ */
+SSD_API ssd_status_t ssd_chunk_scan_fwd(const void* x, const void* B, const void* C,
+                                int64_t row_stride, const void* dt_raw,
+                                const float* dt_bias, const float* A,
+                                const float* D, const float* init_state,
+                                void* y, float* final_state, int b, int L,
+                                int H, int P, int N, int G, int Q,
+                                ssd_dtype_t dtype, void* workspace,
+                                size_t workspace_bytes, int32_t* status,
+                                cudaStream_t stream);
+
+/*
+ * Single-token decode update, in place on the float32 state:
+ *
+ *   dt = softplus(dt_raw + dt_bias); h <- exp(dt*A) h + dt x B^T;
+ *   y = h C + D x
+ *
+ *   state   [b][H][P][N]  float32, read and rewritten in place
+ *   x       [b][.][H][P]  x[bi*row_stride + h*P + p]        dtype
+ *   B, C    [b][.][G][N]  B[bi*row_stride + g*N + n]        dtype
+ *           (row_stride = conv_dim when reading the conv output)
+ *   dt_raw  [b][H]        dtype
+ *   dt_bias [H], A [H], D [H]  float32 (dt_bias and D may be NULL)
+ *   y       [b][H][P]     dtype, written
+ * Requirements: N a multiple of 4 with N <= 256; P >= 1; H % G == 0;
+ * state 16-byte aligned.
+ */
+SSD_API ssd_status_t ssd_state_update(float* state, const void* x, const void* B,
+                              const void* C, int64_t row_stride,
+                              const void* dt_raw, const float* dt_bias,
+                              const float* A, const float* D, void* y, int b,
+                              int H, int P, int N, int G, ssd_dtype_t dtype,
+                              cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_H_ */

@@ -1,0 +1,188 @@
+// api.cu -- the extern "C" entry points of libssd (declared in include/ssd.h):
+// argument validation, kernel selection and launch.  No allocation, no
+// synchronisation, no global mutable state.
+#include "ssd.h"
+
+#include "kernels.h"
+
+namespace {
+
+using ssd::ScanArgs;
+
+struct Range {
+    uintptr_t lo, hi;   // [lo, hi)
+};
+
+Range span(const void* p, int64_t bytes)
+{
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return Range{a, a + (uintptr_t)(bytes > 0 ? bytes : 0)};
+}
+
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi && a.hi > a.lo && b.hi > b.lo; }
+
+bool aligned(const void* p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
+
+bool valid_dtype(ssd_dtype_t d) { return d == SSD_F32 || d == SSD_BF16; }
+
+int elem_bytes(ssd_dtype_t d) { return d == SSD_F32 ? 4 : 2; }
+
+ssd_status_t from_cuda(cudaError_t e)
+{
+    if (e == cudaSuccess) return SSD_OK;
+    (void)cudaGetLastError();
+    return SSD_ERR_CUDA;
+}
+
+int max_optin_smem()
+{
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return 0;
+    return v;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ssd_status_string(ssd_status_t s)
+{
+    switch (s) {
+        case SSD_OK: return "SSD_OK";
+        case SSD_ERR_INVALID_ARG: return "SSD_ERR_INVALID_ARG: invalid argument (nothing launched)";
+        case SSD_ERR_UNSUPPORTED: return "SSD_ERR_UNSUPPORTED: no kernel for this combination (nothing launched)";
+        case SSD_ERR_CUDA: return "SSD_ERR_CUDA: kernel launch failed";
+        case SSD_ERR_TIMEOUT: return "SSD_ERR_TIMEOUT: a bounded device wait gave up";
+    }
+    return "SSD_ERR_UNKNOWN";
+}
+
+int ssd_abi_version(void) { return SSD_ABI_VERSION; }
+
+ssd_status_t ssd_conv1d_silu(const void* xBC, void* out, const float* w, const float* bias,
+                             void* conv_state, int b, int L, int conv_dim, int k,
+                             ssd_dtype_t dtype, cudaStream_t stream)
+{
+    if (!valid_dtype(dtype) || b < 0 || L < 0 || conv_dim <= 0 || k <= 0) return SSD_ERR_INVALID_ARG;
+    if (b == 0 || L == 0) return SSD_OK;   // empty work: nothing is read or written
+    if (!xBC || !out || !w) return SSD_ERR_INVALID_ARG;
+    const int e = elem_bytes(dtype);
+    const int vec = 16 / e;
+    if (conv_dim % vec) return SSD_ERR_INVALID_ARG;
+    if (!aligned(xBC, 16) || !aligned(out, 16) || !aligned(w, 4) || (bias && !aligned(bias, 4)) ||
+        (conv_state && !aligned(conv_state, 16)))
+        return SSD_ERR_INVALID_ARG;
+    const int64_t io_bytes = (int64_t)b * L * conv_dim * e;
+    const Range rx = span(xBC, io_bytes), ro = span(out, io_bytes);
+    const Range rs = span(conv_state, conv_state ? (int64_t)b * conv_dim * k * e : 0);
+    if (overlap(rx, ro) || overlap(rs, rx) || overlap(rs, ro)) return SSD_ERR_INVALID_ARG;
+    if (k < 2 || k > 4) return SSD_ERR_UNSUPPORTED;
+    if (b > 65535 || (L + 31) / 32 > 65535) return SSD_ERR_UNSUPPORTED;
+    return from_cuda(ssd::launch_conv1d_silu(xBC, out, w, bias, conv_state, b, L, conv_dim, k,
+                                             dtype == SSD_BF16, stream));
+}
+
+size_t ssd_chunk_scan_workspace_bytes(int b, int L, int H, int P, int N, int G, int Q,
+                                      ssd_dtype_t dtype)
+{
+    (void)b; (void)L; (void)H; (void)P; (void)N; (void)G; (void)Q; (void)dtype;
+    return 0;
+}
+
+ssd_status_t ssd_chunk_scan_fwd(const void* x, const void* B, const void* C, int64_t row_stride,
+                                const void* dt_raw, const float* dt_bias, const float* A,
+                                const float* D, const float* init_state, void* y,
+                                float* final_state, int b, int L, int H, int P, int N, int G,
+                                int Q, ssd_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                                int32_t* status, cudaStream_t stream)
+{
+    if (!valid_dtype(dtype) || b < 0 || L < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0)
+        return SSD_ERR_INVALID_ARG;
+    if (H % G || P % 8 || N % 8 || (Q != 64 && Q != 128)) return SSD_ERR_INVALID_ARG;
+    // With no tokens the token tensors are never touched and may be NULL.
+    const bool tokens = b > 0 && L > 0;
+    if (!A || (tokens && (!x || !B || !C || !dt_raw || !y))) return SSD_ERR_INVALID_ARG;
+    if (row_stride % 8 || row_stride < (int64_t)H * P || row_stride < (int64_t)G * N)
+        return SSD_ERR_INVALID_ARG;
+    const void* ptrs16[] = {x, B, C, dt_raw, y, init_state, final_state};
+    for (const void* p : ptrs16)
+        if (p && !aligned(p, 16)) return SSD_ERR_INVALID_ARG;
+    if (!aligned(A, 4) || (dt_bias && !aligned(dt_bias, 4)) || (D && !aligned(D, 4)) ||
+        (status && !aligned(status, 4)))
+        return SSD_ERR_INVALID_ARG;
+    const size_t need_ws = ssd_chunk_scan_workspace_bytes(b, L, H, P, N, G, Q, dtype);
+    if (workspace_bytes < need_ws || (need_ws && !workspace)) return SSD_ERR_INVALID_ARG;
+
+    const int e = elem_bytes(dtype);
+    const int64_t rows = (int64_t)b * L;
+    const int64_t row_bytes = row_stride * e;
+    // Conservative extents of the strided inputs: from the pointer to the end
+    // of the last row's channel range.
+    const Range rx = span(x, rows ? (rows - 1) * row_bytes + (int64_t)H * P * e : 0);
+    const Range rB = span(B, rows ? (rows - 1) * row_bytes + (int64_t)G * N * e : 0);
+    const Range rC = span(C, rows ? (rows - 1) * row_bytes + (int64_t)G * N * e : 0);
+    const Range rdt = span(dt_raw, rows * H * e);
+    const Range ry = span(y, rows * H * P * e);
+    const int64_t st_bytes = (int64_t)b * H * P * N * 4;
+    const Range ri = span(init_state, init_state ? st_bytes : 0);
+    const Range rf = span(final_state, final_state ? st_bytes : 0);
+    const Range rw = span(workspace, (int64_t)workspace_bytes);
+    for (Range in : {rx, rB, rC, rdt, ri})
+        if (overlap(ry, in)) return SSD_ERR_INVALID_ARG;
+    for (Range in : {rx, rB, rC, rdt, ry})
+        if (overlap(rf, in)) return SSD_ERR_INVALID_ARG;
+    if (final_state && init_state && final_state != init_state && overlap(rf, ri))
+        return SSD_ERR_INVALID_ARG;
+    for (Range in : {rx, rB, rC, rdt, ry, ri, rf})
+        if (overlap(rw, in)) return SSD_ERR_INVALID_ARG;
+
+    if (b == 0) return SSD_OK;
+    if (L == 0) {
+        // No tokens: the final state is the initial state.
+        if (!final_state || final_state == init_state) return SSD_OK;
+        return from_cuda(init_state ? cudaMemcpyAsync(final_state, init_state, (size_t)st_bytes,
+                                                      cudaMemcpyDeviceToDevice, stream)
+                                    : cudaMemsetAsync(final_state, 0, (size_t)st_bytes, stream));
+    }
+    if ((int64_t)b * H > 0x7fffffffLL) return SSD_ERR_UNSUPPORTED;
+
+    ScanArgs a{x, B, C, row_stride, dt_raw, dt_bias, A, D, init_state, y, final_state,
+               b, L, H, P, N, G, Q, dtype == SSD_BF16, workspace, workspace_bytes, status};
+    if (ssd::chunk_scan_simt_smem_bytes(P, N) > (size_t)max_optin_smem()) return SSD_ERR_UNSUPPORTED;
+    return from_cuda(ssd::launch_chunk_scan_simt(a, stream));
+}
+
+ssd_status_t ssd_state_update(float* state, const void* x, const void* B, const void* C,
+                              int64_t row_stride, const void* dt_raw, const float* dt_bias,
+                              const float* A, const float* D, void* y, int b, int H, int P, int N,
+                              int G, ssd_dtype_t dtype, cudaStream_t stream)
+{
+    if (!valid_dtype(dtype) || b < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || H % G)
+        return SSD_ERR_INVALID_ARG;
+    if (!state || !x || !B || !C || !dt_raw || !A || !y) return SSD_ERR_INVALID_ARG;
+    if (N % 4 || row_stride < (int64_t)H * P || row_stride < (int64_t)G * N) return SSD_ERR_INVALID_ARG;
+    const int e = elem_bytes(dtype);
+    if (!aligned(state, 16) || !aligned(x, e) || !aligned(B, e) || !aligned(C, e) ||
+        !aligned(dt_raw, e) || !aligned(y, e) || !aligned(A, 4) || (dt_bias && !aligned(dt_bias, 4)) ||
+        (D && !aligned(D, 4)))
+        return SSD_ERR_INVALID_ARG;
+    const Range rs = span(state, (int64_t)b * H * P * N * 4);
+    const Range ry = span(y, (int64_t)b * H * P * e);
+    const int64_t last = b ? (int64_t)(b - 1) * row_stride * e : 0;
+    const Range rx = span(x, b ? last + (int64_t)H * P * e : 0);
+    const Range rB = span(B, b ? last + (int64_t)G * N * e : 0);
+    const Range rC = span(C, b ? last + (int64_t)G * N * e : 0);
+    const Range rdt = span(dt_raw, (int64_t)b * H * e);
+    for (Range in : {rx, rB, rC, rdt, ry})
+        if (overlap(rs, in)) return SSD_ERR_INVALID_ARG;
+    for (Range in : {rx, rB, rC, rdt})
+        if (overlap(ry, in)) return SSD_ERR_INVALID_ARG;
+    if (!ssd::state_update_supports_n(N)) return SSD_ERR_UNSUPPORTED;
+    if ((int64_t)b * H > 0x7fffffffLL) return SSD_ERR_UNSUPPORTED;
+    if (b == 0) return SSD_OK;
+    return from_cuda(ssd::launch_state_update(state, x, B, C, row_stride, dt_raw, dt_bias, A, D, y,
+                                              b, H, P, N, G, dtype == SSD_BF16, stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,64 @@
+// common.cuh -- small device helpers shared by the libssd kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssd {
+
+// ---------------------------------------------------------------------------
+// Element access for the two I/O types.  Vectors are 16 bytes: 8 bf16 or
+// 4 float.
+// ---------------------------------------------------------------------------
+template <typename T> struct io;
+
+template <> struct io<float> {
+    static constexpr int kVec = 4;
+    __device__ static inline float to_f(float v) { return v; }
+    __device__ static inline float from_f(float v) { return v; }
+    __device__ static inline void load_vec(const float* p, float (&v)[4]) {
+        float4 q = *reinterpret_cast<const float4*>(p);
+        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+    }
+    __device__ static inline void store_vec(float* p, const float (&v)[4]) {
+        *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    }
+};
+
+template <> struct io<__nv_bfloat16> {
+    static constexpr int kVec = 8;
+    __device__ static inline float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+    __device__ static inline __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
+    __device__ static inline void load_vec(const __nv_bfloat16* p, float (&v)[8]) {
+        uint4 q = *reinterpret_cast<const uint4*>(p);
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+    __device__ static inline void store_vec(__nv_bfloat16* p, const float (&v)[8]) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+            w[i] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+};
+
+template <typename T>
+__device__ inline float ld_f(const T* p) { return io<T>::to_f(*p); }
+
+// softplus(v) = log(1 + e^v), evaluated without overflow as
+// max(v, 0) + log1p(exp(-|v|)).
+__device__ inline float softplus_f(float v) {
+    return fmaxf(v, 0.0f) + log1pf(expf(-fabsf(v)));
+}
+
+__device__ inline float silu_f(float v) { return v / (1.0f + expf(-v)); }
+
+}  // namespace ssd

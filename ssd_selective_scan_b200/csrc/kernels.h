@@ -1,0 +1,44 @@
+// kernels.h -- internal launch interface between the C ABI (api.cu) and the
+// kernels.  Not installed; the public interface is include/ssd.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace ssd {
+
+// Arguments of one chunked-scan call, already validated by the ABI layer.
+struct ScanArgs {
+    const void* x;
+    const void* B;
+    const void* C;
+    int64_t row_stride;
+    const void* dt_raw;
+    const float* dt_bias;
+    const float* A;
+    const float* D;
+    const float* init_state;
+    void* y;
+    float* final_state;
+    int b, L, H, P, N, G, Q;
+    bool bf16;
+    void* workspace;
+    size_t workspace_bytes;
+    int32_t* status;
+};
+
+cudaError_t launch_conv1d_silu(const void* xBC, void* out, const float* w, const float* bias,
+                               void* conv_state, int b, int L, int conv_dim, int k, bool bf16,
+                               cudaStream_t s);
+
+bool state_update_supports_n(int N);
+cudaError_t launch_state_update(float* state, const void* x, const void* B, const void* C,
+                                int64_t row_stride, const void* dt_raw, const float* dt_bias,
+                                const float* A, const float* D, void* y, int b, int H, int P,
+                                int N, int G, bool bf16, cudaStream_t s);
+
+size_t chunk_scan_simt_smem_bytes(int P, int N);
+cudaError_t launch_chunk_scan_simt(const ScanArgs& a, cudaStream_t s);
+
+}  // namespace ssd

@@ -1,0 +1,142 @@
+// state_update.cu -- single-token selective state update (decode step).
+//
+// The recurrence of "Hybrid Architectures for Language Models" (summary page,
+// section 2 Background), h = Abar h + Bbar x, y = C h + D x, run once per
+// (sequence, head) with Abar = exp(dt*A), Bbar = dt*B and
+// dt = softplus(dt_raw + dt_bias).  The state is float32 [b][H][P][N] and is
+// rewritten in place; it stays a constant size however long the context is
+// (the Mamba cache of the same page's appendix C).
+//
+// HBM-bound: each state element is read once and written once (8 bytes) for
+// ~4 flops.  One CTA per (sequence, head); each warp takes rows p of the
+// head's P x N state, with TPR lanes per row each holding N/TPR contiguous
+// floats as 128-bit vectors.  All of a thread's rows are loaded before any is
+// used, so every thread keeps ROWS x 16 bytes of streaming loads in flight.
+// The y reduction over N is a butterfly over the TPR lanes of a row.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ssd {
+
+constexpr int kSuThreads = 128;
+
+template <typename T, int N>
+__global__ void __launch_bounds__(kSuThreads)
+state_update_kernel(float* __restrict__ state, const T* __restrict__ x,
+                    const T* __restrict__ B, const T* __restrict__ C, int64_t row_stride,
+                    const T* __restrict__ dt_raw, const float* __restrict__ dt_bias,
+                    const float* __restrict__ A, const float* __restrict__ D,
+                    T* __restrict__ y, int H, int P, int G)
+{
+    constexpr int NV = N / 4;                      // float4 per state row
+    constexpr int TPR = NV < 32 ? NV : 32;         // lanes per row
+    constexpr int VPL = NV / TPR;                  // float4 per lane per row
+    constexpr int RPW = 32 / TPR;                  // rows per warp pass
+    constexpr int ROWS = 8;                        // passes loaded together
+
+    const int h = blockIdx.x % H;
+    const int bi = blockIdx.x / H;
+    const int g = h / (H / G);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sub = lane / TPR, li = lane % TPR;
+    constexpr int kWarps = kSuThreads / 32;
+
+    const float dt = softplus_f(ld_f(dt_raw + (size_t)bi * H + h) + (dt_bias ? dt_bias[h] : 0.0f));
+    const float dA = expf(dt * A[h]);
+    const float Dh = D ? D[h] : 0.0f;
+
+    const T* xr = x + (size_t)bi * row_stride + (size_t)h * P;
+    const T* Br = B + (size_t)bi * row_stride + (size_t)g * N;
+    const T* Cr = C + (size_t)bi * row_stride + (size_t)g * N;
+    float bv[VPL][4], cvv[VPL][4];
+#pragma unroll
+    for (int v = 0; v < VPL; ++v)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int n = (v * TPR + li) * 4 + e;
+            bv[v][e] = ld_f(Br + n);
+            cvv[v][e] = ld_f(Cr + n);
+        }
+
+    float* sh = state + ((size_t)bi * H + h) * (size_t)P * N;
+    T* yr = y + ((size_t)bi * H + h) * P;
+    const int rows_per_iter = kWarps * RPW * ROWS;
+    for (int p0 = 0; p0 < P; p0 += rows_per_iter) {
+        float4 st[ROWS][VPL];
+        int prow[ROWS];
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) {
+            prow[r] = p0 + (r * kWarps + warp) * RPW + sub;
+            if (prow[r] < P) {
+#pragma unroll
+                for (int v = 0; v < VPL; ++v)
+                    st[r][v] = __ldcs(reinterpret_cast<const float4*>(sh + (size_t)prow[r] * N) + v * TPR + li);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) {
+            const bool ok = prow[r] < P;
+            const float xp = ok ? ld_f(xr + prow[r]) : 0.0f;
+            const float dtx = dt * xp;
+            float acc = 0.0f;
+            if (ok) {
+#pragma unroll
+                for (int v = 0; v < VPL; ++v) {
+                    float4 s = st[r][v];
+                    s.x = fmaf(dA, s.x, dtx * bv[v][0]);
+                    s.y = fmaf(dA, s.y, dtx * bv[v][1]);
+                    s.z = fmaf(dA, s.z, dtx * bv[v][2]);
+                    s.w = fmaf(dA, s.w, dtx * bv[v][3]);
+                    acc = fmaf(cvv[v][0], s.x, acc);
+                    acc = fmaf(cvv[v][1], s.y, acc);
+                    acc = fmaf(cvv[v][2], s.z, acc);
+                    acc = fmaf(cvv[v][3], s.w, acc);
+                    __stcs(reinterpret_cast<float4*>(sh + (size_t)prow[r] * N) + v * TPR + li, s);
+                }
+            }
+#pragma unroll
+            for (int o = TPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (ok && li == 0) yr[prow[r]] = io<T>::from_f(fmaf(Dh, xp, acc));
+        }
+    }
+}
+
+template <typename T>
+static cudaError_t launch_su_t(float* state, const void* x, const void* B, const void* C,
+                               int64_t rs, const void* dt_raw, const float* dt_bias, const float* A,
+                               const float* D, void* y, int b, int H, int P, int N, int G,
+                               cudaStream_t s)
+{
+    const dim3 grid((unsigned)((int64_t)b * H));
+#define SSD_SU_CASE(NN)                                                                        \
+    case NN:                                                                                   \
+        state_update_kernel<T, NN><<<grid, kSuThreads, 0, s>>>(                                \
+            state, static_cast<const T*>(x), static_cast<const T*>(B), static_cast<const T*>(C), \
+            rs, static_cast<const T*>(dt_raw), dt_bias, A, D, static_cast<T*>(y), H, P, G);    \
+        break;
+    switch (N) {
+        SSD_SU_CASE(4) SSD_SU_CASE(8) SSD_SU_CASE(16) SSD_SU_CASE(32)
+        SSD_SU_CASE(64) SSD_SU_CASE(128) SSD_SU_CASE(256)
+        default: return cudaErrorInvalidValue;
+    }
+#undef SSD_SU_CASE
+    return cudaGetLastError();
+}
+
+bool state_update_supports_n(int N)
+{
+    return N == 4 || N == 8 || N == 16 || N == 32 || N == 64 || N == 128 || N == 256;
+}
+
+cudaError_t launch_state_update(float* state, const void* x, const void* B, const void* C,
+                                int64_t row_stride, const void* dt_raw, const float* dt_bias,
+                                const float* A, const float* D, void* y, int b, int H, int P,
+                                int N, int G, bool bf16, cudaStream_t s)
+{
+    return bf16 ? launch_su_t<__nv_bfloat16>(state, x, B, C, row_stride, dt_raw, dt_bias, A, D, y,
+                                             b, H, P, N, G, s)
+                : launch_su_t<float>(state, x, B, C, row_stride, dt_raw, dt_bias, A, D, y, b, H,
+                                     P, N, G, s);
+}
+
+}  // namespace ssd

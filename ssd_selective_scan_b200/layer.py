@@ -1,0 +1,168 @@
+"""Torch-facing calls over the libssd C ABI.
+
+PyTorch is plumbing here: it allocates device memory and supplies the current
+CUDA stream.  Each function checks tensor shapes, allocates the outputs,
+passes raw pointers to the C entry point of the same name (``libssd``) and
+raises ``SsdError`` on any non-OK status.  All arithmetic runs in the CUDA
+kernels of libssd.so.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import binding as libssd
+
+_DT = {torch.float32: libssd.SSD_F32, torch.bfloat16: libssd.SSD_BF16}
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype not in _DT:
+        raise TypeError(f"unsupported I/O dtype {t.dtype}; use float32 or bfloat16")
+    return _DT[t.dtype]
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _f32(t, name):
+    if t is None:
+        return None
+    if t.dtype != torch.float32 or not t.is_contiguous() or not t.is_cuda:
+        raise ValueError(f"{name} must be a contiguous float32 CUDA tensor")
+    return t
+
+
+def conv1d_silu(xBC: torch.Tensor, w: torch.Tensor, bias: torch.Tensor | None = None,
+                conv_state: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
+    """Causal depthwise conv1d + SiLU.  xBC [b, L, conv_dim]; w [conv_dim, k] f32;
+    conv_state [b, conv_dim, k] (updated in place).  Returns out."""
+    if xBC.dim() != 3 or not xBC.is_contiguous():
+        raise ValueError("xBC must be a contiguous [b, L, conv_dim] tensor")
+    b, L, cd = xBC.shape
+    k = w.shape[1]
+    if out is None:
+        out = torch.empty_like(xBC)
+    if conv_state is not None and (conv_state.shape != (b, cd, k) or conv_state.dtype != xBC.dtype
+                                   or not conv_state.is_contiguous()):
+        raise ValueError("conv_state must be a contiguous [b, conv_dim, k] tensor of xBC's dtype")
+    st = libssd.ssd_conv1d_silu(_ptr(xBC), _ptr(out), _ptr(_f32(w, "w")), _ptr(_f32(bias, "bias")),
+                                _ptr(conv_state), b, L, cd, k, _dtype_code(xBC), _stream(stream))
+    libssd.check("ssd_conv1d_silu", st)
+    return out
+
+
+def _row_view_stride(t: torch.Tensor, name: str) -> int:
+    """Row stride (elements between consecutive tokens) of a [b, L, heads, dim]
+    view whose tokens are evenly spaced and whose inner dims are dense."""
+    b, L, nh, d = t.shape
+    s = t.stride()
+    if s[3] != 1 or s[2] != d or (b > 1 and s[0] != L * s[1]):
+        raise ValueError(f"{name}: expected inner-dense [b, L, {nh}, {d}] with uniform token stride")
+    return s[1]
+
+
+def chunk_scan_workspace_bytes(b, L, H, P, N, G, Q, dtype: torch.dtype) -> int:
+    return int(libssd.ssd_chunk_scan_workspace_bytes(b, L, H, P, N, G, Q, _DT[dtype]))
+
+
+def chunk_scan_fwd(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor, dt_raw: torch.Tensor,
+                   A: torch.Tensor, dt_bias: torch.Tensor | None = None,
+                   D: torch.Tensor | None = None, init_state: torch.Tensor | None = None,
+                   Q: int = 128, y: torch.Tensor | None = None,
+                   final_state: torch.Tensor | bool | None = True,
+                   workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                   stream=None):
+    """Chunked SSD scan.  x [b, L, H, P], B/C [b, L, G, N] (views sharing one
+    token stride, e.g. channel ranges of the conv output), dt_raw [b, L, H].
+    Returns (y [b, L, H, P], final_state [b, H, P, N] f32 or None)."""
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    if b * L == 0:
+        # no tokens: strides of empty views are meaningless; any valid one will do
+        rs = -(-max(H * P, G * N) // 8) * 8
+    else:
+        rs = _row_view_stride(x, "x")
+        if _row_view_stride(B, "B") != rs or _row_view_stride(C, "C") != rs:
+            raise ValueError("x, B and C must share one token stride")
+    if B.dtype != x.dtype or C.dtype != x.dtype or dt_raw.dtype != x.dtype:
+        raise ValueError("x, B, C, dt_raw must share the I/O dtype")
+    if dt_raw.shape != (b, L, H) or not dt_raw.is_contiguous():
+        raise ValueError("dt_raw must be a contiguous [b, L, H] tensor")
+    if y is None:
+        y = torch.empty((b, L, H, P), dtype=x.dtype, device=x.device)
+    if final_state is True:
+        final_state = torch.empty((b, H, P, N), dtype=torch.float32, device=x.device)
+    elif final_state is False:
+        final_state = None
+    need = chunk_scan_workspace_bytes(b, L, H, P, N, G, Q, x.dtype)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = libssd.ssd_chunk_scan_fwd(
+        _ptr(x), _ptr(B), _ptr(C), rs, _ptr(dt_raw), _ptr(_f32(dt_bias, "dt_bias")),
+        _ptr(_f32(A, "A")), _ptr(_f32(D, "D")), _ptr(_f32(init_state, "init_state")), _ptr(y),
+        _ptr(final_state), b, L, H, P, N, G, Q, _dtype_code(x), _ptr(workspace), ws_bytes,
+        _ptr(status), _stream(stream))
+    libssd.check("ssd_chunk_scan_fwd", st)
+    return y, final_state
+
+
+def state_update(state: torch.Tensor, x: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
+                 dt_raw: torch.Tensor, A: torch.Tensor, dt_bias: torch.Tensor | None = None,
+                 D: torch.Tensor | None = None, y: torch.Tensor | None = None, stream=None):
+    """One decode token, state [b, H, P, N] f32 updated in place.  x [b, H, P],
+    B/C [b, G, N] views sharing one batch stride (e.g. channel ranges of the
+    conv output), dt_raw [b, H].  Returns y [b, H, P]."""
+    b, H, P, N = state.shape
+    G = B.shape[1]
+    _f32(state, "state")
+    rs = x.stride(0)
+    for t, nm, d in ((x, "x", P), (B, "B", N), (C, "C", N)):
+        if t.stride(-1) != 1 or t.stride(-2) != d or (b > 1 and t.stride(0) != rs):
+            raise ValueError(f"{nm}: inner-dense view with the shared batch stride expected")
+    if y is None:
+        y = torch.empty((b, H, P), dtype=x.dtype, device=x.device)
+    st = libssd.ssd_state_update(_ptr(state), _ptr(x), _ptr(B), _ptr(C), rs, _ptr(dt_raw),
+                                 _ptr(_f32(dt_bias, "dt_bias")), _ptr(_f32(A, "A")),
+                                 _ptr(_f32(D, "D")), _ptr(y), b, H, P, N, G, _dtype_code(x),
+                                 _stream(stream))
+    libssd.check("ssd_state_update", st)
+    return y
+
+
+def split_channels(u: torch.Tensor, H: int, P: int, G: int, N: int):
+    """[.., conv_dim] -> views x [.., H, P], B [.., G, N], C [.., G, N]."""
+    lead = u.shape[:-1]
+    x = u[..., : H * P].unflatten(-1, (H, P))
+    B = u[..., H * P: H * P + G * N].unflatten(-1, (G, N))
+    C = u[..., H * P + G * N:].unflatten(-1, (G, N))
+    assert x.shape[:-2] == lead
+    return x, B, C
+
+
+def layer_prefill(xBC, w, dt_raw, A, H, P, G, N, *, bias=None, conv_state=None, dt_bias=None,
+                  D=None, init_state=None, Q=128, u=None, y=None, final_state=True, stream=None):
+    """conv1d+SiLU then the chunked scan on the same stream.
+    Returns (y, final_state); conv_state, if given, is updated in place."""
+    u = conv1d_silu(xBC, w, bias, conv_state, out=u, stream=stream)
+    x, B, C = split_channels(u, H, P, G, N)
+    return chunk_scan_fwd(x, B, C, dt_raw, A, dt_bias, D, init_state, Q=Q, y=y,
+                          final_state=final_state, stream=stream)
+
+
+def decode_step(xBC, w, conv_state, state, dt_raw, A, H, P, G, N, *, bias=None, dt_bias=None,
+                D=None, u=None, y=None, stream=None):
+    """One token per sequence: conv-cache roll + conv + SiLU, then the state
+    update.  xBC [b, conv_dim]; conv_state and state updated in place.  Returns y."""
+    b, cd = xBC.shape
+    u = conv1d_silu(xBC.view(b, 1, cd), w, bias, conv_state,
+                    out=None if u is None else u.view(b, 1, cd), stream=stream).view(b, cd)
+    x, B, C = split_channels(u, H, P, G, N)
+    return state_update(state, x, B, C, dt_raw, A, dt_bias, D, y=y, stream=stream)

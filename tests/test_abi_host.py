@@ -1,0 +1,142 @@
+"""C-ABI boundary on the host (no GPU needed): libssd.so loads, exports every
+entry point include/ssd.h declares (and the binding covers exactly those), and
+argument validation rejects bad calls before anything reaches the device.
+
+Pointer arguments here are fake addresses that are never dereferenced: every
+call below fails validation (or is empty work) before any CUDA call."""
+import os
+import re
+import subprocess
+
+import pytest
+
+from ssd_selective_scan_b200 import build as ssd_build
+from ssd_selective_scan_b200 import binding as libssd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssd.h")
+
+OK, INV, UNS = libssd.SSD_OK, libssd.SSD_ERR_INVALID_ARG, libssd.SSD_ERR_UNSUPPORTED
+F32, BF16 = libssd.SSD_F32, libssd.SSD_BF16
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    ssd_build.build()
+    libssd.load()
+
+
+def declared_entry_points():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"SSD_API\s+[\w\s\*]+?\b(ssd_\w+)\s*\(", txt)))
+
+
+def test_header_declares_the_entry_points():
+    assert declared_entry_points() == sorted([
+        "ssd_abi_version", "ssd_chunk_scan_fwd", "ssd_chunk_scan_workspace_bytes",
+        "ssd_conv1d_silu", "ssd_state_update", "ssd_status_string"])
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.check_output(["nm", "-D", "--defined-only", libssd.LIB_PATH], text=True)
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    missing = set(declared_entry_points()) - exported
+    assert not missing, f"declared but not exported: {missing}"
+    assert set(libssd.SIGNATURES) == set(declared_entry_points())
+    lib = libssd.load()
+    for name in declared_entry_points():
+        assert hasattr(lib, name)
+
+
+def test_version_and_status_strings():
+    assert libssd.ssd_abi_version() == 1
+    assert libssd.status_string(OK) == "SSD_OK"
+    for s in (INV, UNS, libssd.SSD_ERR_CUDA, libssd.SSD_ERR_TIMEOUT):
+        assert libssd.status_string(s).startswith("SSD_ERR_")
+    assert libssd.status_string(99) == "SSD_ERR_UNKNOWN"
+
+
+# fake, well-separated, 256-byte aligned device addresses (never dereferenced)
+def fake(i, off=0):
+    return 0x7f0000000000 + i * (1 << 32) + off
+
+
+def conv(**kw):
+    a = dict(xBC=fake(1), out=fake(2), w=fake(3), bias=None, conv_state=fake(4), b=2, L=16,
+             conv_dim=64, k=4, dtype=BF16, stream=None)
+    a.update(kw)
+    return libssd.ssd_conv1d_silu(**a)
+
+
+def test_conv_validation():
+    assert conv(b=0) == OK and conv(L=0) == OK                      # empty work, no launch
+    assert conv(xBC=None) == INV and conv(out=None) == INV and conv(w=None) == INV
+    assert conv(b=0, xBC=None, out=None) == OK                       # empty work takes NULL
+    assert conv(b=-1) == INV and conv(L=-1) == INV and conv(conv_dim=0) == INV
+    assert conv(dtype=7) == INV
+    assert conv(conv_dim=60) == INV                                  # not a multiple of 8 (bf16)
+    assert conv(conv_dim=60, dtype=F32, b=0) == OK                   # multiple of 4 is fine for f32
+    assert conv(xBC=fake(1, 8)) == INV and conv(conv_state=fake(4, 4)) == INV   # misaligned
+    assert conv(out=fake(1, 64)) == INV                              # out overlaps xBC
+    assert conv(conv_state=fake(2, 16)) == INV                       # cache overlaps out
+    assert conv(k=5) == UNS and conv(k=1) == UNS
+
+
+def scan(**kw):
+    a = dict(x=fake(1), B=fake(1, 2560 * 2), C=fake(1, (2560 + 1024) * 2), row_stride=4608,
+             dt_raw=fake(2), dt_bias=None, A=fake(3), D=fake(4), init_state=None, y=fake(5),
+             final_state=fake(6), b=2, L=256, H=40, P=64, N=128, G=8, Q=128, dtype=BF16,
+             workspace=None, workspace_bytes=0, status=None, stream=None)
+    a.update(kw)
+    if a["workspace"] is None and a["workspace_bytes"] == 0 and "workspace_bytes" not in kw:
+        need = libssd.ssd_chunk_scan_workspace_bytes(a["b"], a["L"], a["H"], a["P"], a["N"],
+                                                     a["G"], a["Q"], a["dtype"])
+        if need:
+            a["workspace"], a["workspace_bytes"] = fake(7), need
+    return libssd.ssd_chunk_scan_fwd(**a)
+
+
+def test_scan_validation():
+    assert scan(b=0) == OK and scan(b=0, x=None, y=None, B=None, C=None, dt_raw=None) == OK
+    for k in ("x", "B", "C", "dt_raw", "A", "y"):
+        assert scan(**{k: None}) == INV, k
+    assert scan(H=40, G=7) == INV                                    # H % G
+    assert scan(P=60) == INV and scan(N=100) == INV                  # multiples of 8
+    assert scan(Q=96) == INV and scan(Q=256) == INV
+    assert scan(row_stride=4604) == INV                              # not a multiple of 8
+    assert scan(row_stride=2048) == INV                              # shorter than H*P
+    assert scan(x=fake(1, 2)) == INV and scan(y=fake(5, 8)) == INV   # misaligned
+    assert scan(y=fake(1, 4096)) == INV                              # y overlaps x
+    assert scan(final_state=fake(5, 1024)) == INV                    # final state overlaps y
+    assert scan(init_state=fake(6, 512)) == INV                      # partial alias of final state
+    assert scan(dtype=3) == INV and scan(L=-1) == INV and scan(H=0) == INV
+
+
+def test_scan_workspace_query_and_check():
+    need = libssd.ssd_chunk_scan_workspace_bytes(8, 2048, 40, 64, 128, 8, 128, BF16)
+    assert need >= 0
+    if need:
+        assert scan(workspace=None, workspace_bytes=need) == INV
+        assert scan(workspace=fake(7), workspace_bytes=need - 1) == INV
+        assert scan(workspace=fake(1, 64), workspace_bytes=need) == INV    # overlaps x
+
+
+def su(**kw):
+    a = dict(state=fake(1), x=fake(2), B=fake(2, 16384 * 2), C=fake(2, (16384 + 1024) * 2),
+             row_stride=10240, dt_raw=fake(3), dt_bias=None, A=fake(4), D=fake(5), y=fake(6),
+             b=4, H=128, P=64, N=128, G=8, dtype=BF16, stream=None)
+    a.update(kw)
+    return libssd.ssd_state_update(**a)
+
+
+def test_state_update_validation():
+    assert su(b=0) == OK
+    for k in ("state", "x", "B", "C", "dt_raw", "A", "y"):
+        assert su(**{k: None}) == INV, k
+    assert su(G=3) == INV and su(N=6) == INV and su(P=0) == INV
+    assert su(row_stride=100) == INV
+    assert su(state=fake(1, 8)) == INV                               # state not 16-byte aligned
+    assert su(x=fake(2, 1)) == INV                                   # x not element aligned
+    assert su(y=fake(1, 64)) == INV                                  # y overlaps state
+    assert su(state=fake(2, 64)) == INV                              # state overlaps x
+    assert su(N=512) == UNS and su(N=12) == UNS                      # no kernel for these N
