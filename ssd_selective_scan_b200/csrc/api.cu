@@ -149,6 +149,7 @@ ssd_status_t ssd_chunk_scan_fwd(const void* x, const void* B, const void* C, int
 
     ScanArgs a{x, B, C, row_stride, dt_raw, dt_bias, A, D, init_state, y, final_state,
                b, L, H, P, N, G, Q, dtype == SSD_BF16, workspace, workspace_bytes, status};
+    if (ssd::chunk_scan_tc_supported(a)) return from_cuda(ssd::launch_chunk_scan_tc(a, stream));
     if (ssd::chunk_scan_simt_smem_bytes(P, N) > (size_t)max_optin_smem()) return SSD_ERR_UNSUPPORTED;
     return from_cuda(ssd::launch_chunk_scan_simt(a, stream));
 }

@@ -38,6 +38,9 @@ cudaError_t launch_state_update(float* state, const void* x, const void* B, cons
                                 const float* A, const float* D, void* y, int b, int H, int P,
                                 int N, int G, bool bf16, cudaStream_t s);
 
+bool chunk_scan_tc_supported(const ScanArgs& a);
+cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t s);
+
 size_t chunk_scan_simt_smem_bytes(int P, int N);
 cudaError_t launch_chunk_scan_simt(const ScanArgs& a, cudaStream_t s);
 
