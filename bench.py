@@ -192,6 +192,8 @@ class PrefillStep:
         self.y = torch.empty(s.b, s.L, s.H, s.P, dtype=s.torch_dtype, device=dev)
         self.fs = torch.empty(s.b, s.H, s.P, s.N, dtype=torch.float32, device=dev)
         self.views = layer.split_channels(self.u, s.H, s.P, s.G, s.N)
+        need = layer.chunk_scan_workspace_bytes(s.b, s.L, s.H, s.P, s.N, s.G, s.Q, s.torch_dtype)
+        self.ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev) if need else None
 
     def conv(self):
         d = self.d
@@ -201,7 +203,7 @@ class PrefillStep:
         d, s = self.d, self.s
         x, B, C = self.views
         self.layer.chunk_scan_fwd(x, B, C, d["dt_raw"], d["A"], d["dt_bias"], d["D"], None,
-                                  Q=s.Q, y=self.y, final_state=self.fs)
+                                  Q=s.Q, y=self.y, final_state=self.fs, workspace=self.ws)
 
     def __call__(self):
         self.conv()
@@ -433,6 +435,29 @@ def run_reference(args):
     }
 
 
+def run_one_kernel(args, dev):
+    """Launch one kernel of the bench workloads alone (for ncu captures)."""
+    if args.kernel == "decode":
+        st = DecodeStep(DECODE, synth.config_seed(4), dev)
+        st.conv()
+        fn = st.update
+    else:
+        st = PrefillStep(PREFILL, synth.config_seed(1), dev)
+        st.conv()
+        fn = st.scan if args.kernel == "scan" else st.conv
+    for _ in range(args.warmup):
+        fn()
+    e0, e1 = _events(2)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"kernel": args.kernel, "launches": args.steps,
+                      "ms_per_launch": e0.elapsed_time(e1) / args.steps}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -440,6 +465,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", choices=["scan", "conv", "decode"],
+                    help="launch only this kernel (warmup + steps launches on the bench "
+                         "workload) and print its mean CUDA-event time; for profiler captures")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -461,6 +489,9 @@ def main():
                                 device_id=dev)
     from ssd_selective_scan_b200 import binding
     binding.load()
+    if args.kernel:
+        run_one_kernel(args, dev)
+        return 0
     line = run_ours(args, rank, world, dev)
     if rank == 0:
         if not args.no_cpu_baseline:

@@ -106,7 +106,7 @@ SSD_API int ssd_abi_version(void);
  *                                inputs of (old cache | xBC), oldest first.
  *                                With L == 1 this is the decode-step roll.
  * Requirements: 2 <= k <= 4 (else SSD_ERR_UNSUPPORTED); conv_dim a multiple
- * of 8 (bf16) or 4 (f32); xBC, out, conv_state 16-byte aligned.
+ * of 8 (bf16) or 4 (f32); xBC, out, w, conv_state 16-byte aligned.
  */
 SSD_API ssd_status_t ssd_conv1d_silu(const void* xBC, void* out, const float* w,
                              const float* bias, void* conv_state, int b, int L,

@@ -70,7 +70,7 @@ ssd_status_t ssd_conv1d_silu(const void* xBC, void* out, const float* w, const f
     const int e = elem_bytes(dtype);
     const int vec = 16 / e;
     if (conv_dim % vec) return SSD_ERR_INVALID_ARG;
-    if (!aligned(xBC, 16) || !aligned(out, 16) || !aligned(w, 4) || (bias && !aligned(bias, 4)) ||
+    if (!aligned(xBC, 16) || !aligned(out, 16) || !aligned(w, 16) || (bias && !aligned(bias, 4)) ||
         (conv_state && !aligned(conv_state, 16)))
         return SSD_ERR_INVALID_ARG;
     const int64_t io_bytes = (int64_t)b * L * conv_dim * e;
@@ -86,8 +86,11 @@ ssd_status_t ssd_conv1d_silu(const void* xBC, void* out, const float* w, const f
 size_t ssd_chunk_scan_workspace_bytes(int b, int L, int H, int P, int N, int G, int Q,
                                       ssd_dtype_t dtype)
 {
-    (void)b; (void)L; (void)H; (void)P; (void)N; (void)G; (void)Q; (void)dtype;
-    return 0;
+    if (b <= 0 || L <= 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || !valid_dtype(dtype)) return 0;
+    ScanArgs a{};
+    a.b = b; a.L = L; a.H = H; a.P = P; a.N = N; a.G = G; a.Q = Q;
+    a.bf16 = dtype == SSD_BF16;
+    return ssd::chunk_scan_tc_supported(a) ? ssd::chunk_scan_tc_workspace_bytes(a) : 0;
 }
 
 ssd_status_t ssd_chunk_scan_fwd(const void* x, const void* B, const void* C, int64_t row_stride,

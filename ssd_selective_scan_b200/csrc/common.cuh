@@ -24,6 +24,13 @@ template <> struct io<float> {
     __device__ static inline void store_vec(float* p, const float (&v)[4]) {
         *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
     }
+    __device__ static inline void decode(uint4 q, float (&v)[4]) {
+        v[0] = __uint_as_float(q.x); v[1] = __uint_as_float(q.y);
+        v[2] = __uint_as_float(q.z); v[3] = __uint_as_float(q.w);
+    }
+    // element e of a packed word array
+    __device__ static inline float word_get(const uint32_t* w, int e) { return __uint_as_float(w[e]); }
+    __device__ static inline void word_set(uint32_t* w, int e, float v) { w[e] = __float_as_uint(v); }
 };
 
 template <> struct io<__nv_bfloat16> {
@@ -38,6 +45,21 @@ template <> struct io<__nv_bfloat16> {
             v[2 * i] = __uint_as_float(w[i] << 16);
             v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
         }
+    }
+    __device__ static inline void decode(uint4 q, float (&v)[8]) {
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+    __device__ static inline float word_get(const uint32_t* w, int e) {
+        return __uint_as_float((e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16));
+    }
+    __device__ static inline void word_set(uint32_t* w, int e, float v) {
+        const uint32_t b = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v));
+        w[e >> 1] = (e & 1) ? ((w[e >> 1] & 0x0000ffffu) | (b << 16)) : ((w[e >> 1] & 0xffff0000u) | b);
     }
     __device__ static inline void store_vec(__nv_bfloat16* p, const float (&v)[8]) {
         uint32_t w[4];
@@ -59,6 +81,9 @@ __device__ inline float softplus_f(float v) {
     return fmaxf(v, 0.0f) + log1pf(expf(-fabsf(v)));
 }
 
-__device__ inline float silu_f(float v) { return v / (1.0f + expf(-v)); }
+// SiLU(v) = v / (1 + e^-v) with the hardware exp and approximate divide
+// (a few ulp, well inside the float32 parity bound).  For v -> -inf the
+// denominator overflows to inf and the result is -0.
+__device__ inline float silu_f(float v) { return __fdividef(v, 1.0f + __expf(-v)); }
 
 }  // namespace ssd

@@ -39,6 +39,7 @@ cudaError_t launch_state_update(float* state, const void* x, const void* B, cons
                                 int N, int G, bool bf16, cudaStream_t s);
 
 bool chunk_scan_tc_supported(const ScanArgs& a);
+size_t chunk_scan_tc_workspace_bytes(const ScanArgs& a);
 cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t s);
 
 size_t chunk_scan_simt_smem_bytes(int P, int N);

@@ -58,6 +58,11 @@ CASES = {
                          dict(a_range=(0.01, 2.0), init_state=True)),
     "bf16_short_L": (synth.CONFIGS[1].with_(b=3, L=5, H=4, G=2), dict(init_state=True)),
     "bf16_n16": (synth.CONFIGS[1].with_(b=1, L=130, H=4, N=16, G=1), {}),
+    # more (sequence, head) chains than the persistent grid has CTAs: chains
+    # are cut between CTAs and finished from a handed-over state
+    "bf16_many_chains_handoff": (synth.CONFIGS[1].with_(b=3, L=300, H=128, G=8), dict(init_state=True)),
+    "bf16_many_chains_long_memory": (synth.CONFIGS[1].with_(b=5, L=520, H=64, G=8),
+                                     dict(a_range=(0.01, 2.0))),
 }
 
 
