@@ -33,8 +33,9 @@ def declared_entry_points():
 
 def test_header_declares_the_entry_points():
     assert declared_entry_points() == sorted([
-        "ssd_abi_version", "ssd_chunk_scan_fwd", "ssd_chunk_scan_workspace_bytes",
-        "ssd_conv1d_silu", "ssd_state_update", "ssd_status_string"])
+        "ssd_abi_version", "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_static",
+        "ssd_chunk_scan_workspace_bytes", "ssd_conv1d_silu", "ssd_state_update",
+        "ssd_status_string"])
 
 
 def test_library_exports_every_declared_symbol():
@@ -113,8 +114,11 @@ def test_scan_validation():
 
 
 def test_scan_workspace_query_and_check():
-    need = libssd.ssd_chunk_scan_workspace_bytes(8, 2048, 40, 64, 128, 8, 128, BF16)
-    assert need >= 0
+    # the shape of scan()'s defaults: every call below must fail validation
+    need = libssd.ssd_chunk_scan_workspace_bytes(2, 256, 40, 64, 128, 8, 128, BF16)
+    assert need > 0                                   # the tensor-core path takes scratch
+    assert libssd.ssd_chunk_scan_workspace_bytes(2, 256, 4, 64, 16, 1, 64, F32) == 0
+    assert libssd.ssd_chunk_scan_workspace_bytes(0, 256, 40, 64, 128, 8, 128, BF16) == 0
     if need:
         assert scan(workspace=None, workspace_bytes=need) == INV
         assert scan(workspace=fake(7), workspace_bytes=need - 1) == INV
