@@ -165,6 +165,39 @@ SSD_API ssd_status_t ssd_chunk_scan_fwd(const void* x, const void* B, const void
                                 cudaStream_t stream);
 
 /*
+ * ssd_chunk_scan_fwd without a caller-provided workspace, for callers that
+ * cannot allocate device memory on their call path (a host framework that
+ * owns every device allocation and forbids raw cudaMalloc, a serving loop
+ * that must not allocate per request, a runtime with a fixed memory budget).
+ * The pages have no counterpart: this is a deployment convenience.
+ *
+ * Same arguments, semantics and requirements as ssd_chunk_scan_fwd, minus
+ * `workspace` / `workspace_bytes`.  The scratch memory comes from a 10 MiB
+ * array compiled into the library, which every GPU that loads the library
+ * holds until the process exits.  Nothing is allocated.
+ *   - The first call on a device looks the array's device address up
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - A call whose scratch need (ssd_chunk_scan_workspace_bytes) exceeds
+ *     10 MiB returns SSD_ERR_UNSUPPORTED and launches nothing.  The
+ *     tensor-core scan needs at most 2 x SMs x 32 KiB plus a small control
+ *     block, about 9.3 MiB on a 148-SM B200.
+ *   - All calls on a device share the array; the parts that must start at
+ *     zero are cleared on the call's stream.  Calls whose executions overlap
+ *     on the GPU (unordered streams) race on the array: order them.
+ * Unlike the rest of the library, this entry point keeps global state: the
+ * array and the cached per-device addresses.
+ */
+SSD_API ssd_status_t ssd_chunk_scan_fwd_static(const void* x, const void* B, const void* C,
+                                       int64_t row_stride, const void* dt_raw,
+                                       const float* dt_bias, const float* A,
+                                       const float* D, const float* init_state,
+                                       void* y, float* final_state, int b, int L,
+                                       int H, int P, int N, int G, int Q,
+                                       ssd_dtype_t dtype, int32_t* status,
+                                       cudaStream_t stream);
+
+/*
  * Single-token decode update, in place on the float32 state:
  *
  *   dt = softplus(dt_raw + dt_bias); h <- exp(dt*A) h + dt x B^T;

@@ -35,6 +35,8 @@ SIGNATURES = {
                                 _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp, _vp]),
     "ssd_state_update": (_i, [_vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp,
                               _i, _i, _i, _i, _i, _i, _vp]),
+    "ssd_chunk_scan_fwd_static": (_i, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                       _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp]),
 }
 
 _lock = threading.Lock()
@@ -86,6 +88,13 @@ def ssd_chunk_scan_fwd(x, B, C, row_stride, dt_raw, dt_bias, A, D, init_state, y
     return load().ssd_chunk_scan_fwd(x, B, C, row_stride, dt_raw, dt_bias, A, D, init_state, y,
                                      final_state, b, L, H, P, N, G, Q, dtype, workspace,
                                      workspace_bytes, status, stream)
+
+
+def ssd_chunk_scan_fwd_static(x, B, C, row_stride, dt_raw, dt_bias, A, D, init_state, y,
+                              final_state, b, L, H, P, N, G, Q, dtype, status, stream) -> int:
+    return load().ssd_chunk_scan_fwd_static(x, B, C, row_stride, dt_raw, dt_bias, A, D, init_state,
+                                            y, final_state, b, L, H, P, N, G, Q, dtype, status,
+                                            stream)
 
 
 def ssd_state_update(state, x, B, C, row_stride, dt_raw, dt_bias, A, D, y, b, H, P, N, G, dtype,
