@@ -62,6 +62,7 @@ constexpr int kCtlWarp = kEwThreads / 32;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr int kEwBarrier = 1;    // named barrier among the elementwise warps
+constexpr int kVecBarrier = 2;   // named barrier among elementwise warps 0-3
 
 // Shared-memory layout, offsets from a 1024-byte aligned base.  Tiles are
 // 128-byte swizzled: 128-byte rows, 16-byte chunk c of row r at r*128 +
@@ -72,7 +73,7 @@ constexpr int kOffC = 32768;          // C tile  [128 tok][128 n]   (2 halves), 
 constexpr int kOffX = 65536;          // X tile  [128 tok][64 p]
 constexpr int kOffHX = 81920;         // bf16 state [128 n][64 p], then w o X [128 tok][64 p]
 constexpr int kOffVec = 98304;        // per chunk parity: cl, dt, v  (3 x float[128]) x 2
-constexpr int kOffBar = kOffVec + 3072;  // 6 mbarriers
+constexpr int kOffBar = kOffVec + 3072 + 32;  // (4 warp totals before it) 6 mbarriers
 constexpr int kOffMisc = kOffBar + 64;   // tmem slot, abort flag, ticket
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
 
@@ -235,7 +236,6 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     uint64_t* bar_ld = reinterpret_cast<uint64_t*>(smem + kOffBar);   // TMA B, C, X landed
     uint64_t* bar_m1 = bar_ld + 1;      // G and Yo done
     uint64_t* bar_m2 = bar_ld + 2;      // Yd and the state update done
-    uint64_t* bar_vec = bar_ld + 3;     // chunk vectors written (control warp)
     uint64_t* bar_mready = bar_ld + 4;  // M, w o X, scaled state ready (elementwise warps)
     uint64_t* bar_hx = bar_ld + 5;      // bf16 state in smem, Yd / Yo consumed (elementwise warps)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
@@ -253,7 +253,6 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         mbar_init(bar_ld, 1);
         mbar_init(bar_m1, 1);
         mbar_init(bar_m2, 1);
-        mbar_init(bar_vec, 1);
         mbar_init(bar_mready, kEwThreads);
         mbar_init(bar_hx, kEwThreads);
         fence_mbar_init();
@@ -286,91 +285,34 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             tma_load_3d(sC + kTileHalf, &tmC, g * kN + 64, t0, bi, bar_ld);
             tma_load_3d(sX, &tmX, h * kP, t0, bi, bar_ld);
         };
-        // dt_raw of tokens 4*lane .. 4*lane+3 of an item's chunk
-        auto load_dt = [&](const Item& it, float (&d)[4]) {
-            const int bi = it.chain / H, h = it.chain % H;
-            const __nv_bfloat16* p = prm.dt_raw + (size_t)bi * L * H + h;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int t = it.chunk * kQ + lane * 4 + k;
-                d[k] = t < L ? __bfloat162float(p[(size_t)t * H]) : 0.0f;
-            }
-        };
-        auto write_vecs = [&](const Item& it, const float (&d)[4], int parity) {
-            const int h = it.chain % H;
-            const float A2 = prm.A[h] * 1.4426950408889634f;   // A * log2(e)
-            const float bias = prm.dt_bias ? prm.dt_bias[h] : 0.0f;
-            float dt[4], cl[4], run = 0.0f;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int t = it.chunk * kQ + lane * 4 + k;
-                dt[k] = t < L ? softplus_f(d[k] + bias) : 0.0f;
-                run += dt[k] * A2;
-                cl[k] = run;
-            }
-            float incl = run;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float v = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += v;
-            }
-            const float excl = incl - run;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) cl[k] += excl;
-            const float cl_e = __shfl_sync(0xffffffffu, cl[3], lane | 7);   // last token of the 32-block
-            const ChunkVecs cv = chunk_vecs(smem, parity);
-            float v[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) v[k] = ex2_approx(cl_e - cl[k]) * dt[k];
-            reinterpret_cast<float4*>(cv.cl)[lane] = make_float4(cl[0], cl[1], cl[2], cl[3]);
-            reinterpret_cast<float4*>(cv.dt)[lane] = make_float4(dt[0], dt[1], dt[2], dt[3]);
-            reinterpret_cast<float4*>(cv.v)[lane] = make_float4(v[0], v[1], v[2], v[3]);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_vec);
-        };
-
-        if (rg.count > 0) {
-            float dtr[4];
-            const Item it0 = item_at(rg, 0, nc);
-            if (lane == 0) issue_loads(it0);
-            load_dt(it0, dtr);
-            write_vecs(it0, dtr, 0);
-            if (rg.count > 1) load_dt(item_at(rg, 1, nc), dtr);
+        if (rg.count > 0 && lane == 0) {
+            issue_loads(item_at(rg, 0, nc));
             for (int idx = 0; idx < rg.count; ++idx) {
                 const uint32_t ph = (uint32_t)idx & 1u;
-                if (lane == 0) {
-                    mbar_wait_bounded(bar_ld, ph, kWaitNs, aborted, prm.status);
-                    mbar_wait_bounded(bar_hx, ph, kWaitNs, aborted, prm.status);
-                    tc_fence_after_sync();
+                mbar_wait_bounded(bar_ld, ph, kWaitNs, aborted, prm.status);
+                mbar_wait_bounded(bar_hx, ph, kWaitNs, aborted, prm.status);
+                tc_fence_after_sync();
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)   // G = C B^T
-                        umma_bf16(tmem + kColG, desc_kmajor(aC, k), desc_kmajor(aB, k), kIdG, k > 0);
+                for (int k = 0; k < 8; ++k)   // G = C B^T
+                    umma_bf16(tmem + kColG, desc_kmajor(aC, k), desc_kmajor(aB, k), kIdG, k > 0);
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)   // Yo = C h^T
-                        umma_bf16(tmem + kColYo, desc_kmajor(aC, k), desc_mnmajor(aHX, k), kIdYo, k > 0);
-                    umma_commit(bar_m1);
-                }
-                __syncwarp();
-                if (idx + 1 < rg.count) {
-                    write_vecs(item_at(rg, idx + 1, nc), dtr, (idx + 1) & 1);
-                    if (idx + 2 < rg.count) load_dt(item_at(rg, idx + 2, nc), dtr);
-                }
-                if (lane == 0) {
-                    mbar_wait_bounded(bar_mready, ph, kWaitNs, aborted, prm.status);
-                    tc_fence_after_sync();
+                for (int k = 0; k < 8; ++k)   // Yo = C h^T
+                    umma_bf16(tmem + kColYo, desc_kmajor(aC, k), desc_mnmajor(aHX, k), kIdYo, k > 0);
+                umma_commit(bar_m1);
+                mbar_wait_bounded(bar_mready, ph, kWaitNs, aborted, prm.status);
+                tc_fence_after_sync();
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)   // Yd = M X
-                        umma_bf16(tmem + kColG, desc_kmajor(aC, k), desc_mnmajor(aX, k), kIdYd, k > 0);
+                for (int k = 0; k < 8; ++k)   // Yd = M X
+                    umma_bf16(tmem + kColG, desc_kmajor(aC, k), desc_mnmajor(aX, k), kIdYd, k > 0);
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)   // h += B^T (w o X)   (h already decayed)
-                        umma_bf16(tmem + kColH, desc_mnmajor(aB, k), desc_mnmajor(aHX, k), kIdS, 1);
-                    umma_commit(bar_m2);
-                    mbar_wait_bounded(bar_m2, ph, kWaitNs, aborted, prm.status);
-                    if (idx + 1 < rg.count) issue_loads(item_at(rg, idx + 1, nc));
-                }
-                __syncwarp();
+                for (int k = 0; k < 8; ++k)   // h += B^T (w o X)   (h already decayed)
+                    umma_bf16(tmem + kColH, desc_mnmajor(aB, k), desc_mnmajor(aHX, k), kIdS, 1);
+                umma_commit(bar_m2);
+                mbar_wait_bounded(bar_m2, ph, kWaitNs, aborted, prm.status);
+                if (idx + 1 < rg.count) issue_loads(item_at(rg, idx + 1, nc));
             }
         }
+        __syncwarp();
     } else {
         // ------------------------------------------------------------------
         // elementwise warps
@@ -383,13 +325,56 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         const uint32_t tH = tmem + kColH + (uint32_t)half * 32 + lane_off;
 
         // start of a segment: fp32 state into TMEM, bf16 copy into smem
+        float* sWs = reinterpret_cast<float*>(smem + kOffBar) - 8;   // 4 warp totals
+        // dt_raw of token `row` of an item's chunk (warps 0-3)
+        auto load_dt = [&](const Item& it) -> float {
+            const int t = it.chunk * kQ + row;
+            if (half != 0 || t >= L) return 0.0f;
+            const int bi = it.chain / H, h = it.chain % H;
+            return __bfloat162float(prm.dt_raw[((size_t)bi * L + t) * H + h]);
+        };
+        // Chunk vectors of an item (warps 0-3, one token each): dt, the
+        // inclusive cumulative log2 decay and the off-diagonal column factor.
+        // Stage 1 scans within each warp; stage 2, after a barrier among the
+        // four warps, adds the preceding warps' totals and writes the vectors.
+        float vec_a = 0.0f, vec_dt = 0.0f;
+        auto vecs_stage1 = [&](const Item& it, float dtr) {
+            const int h = it.chain % H;
+            const int t = it.chunk * kQ + row;
+            const float bias = prm.dt_bias ? prm.dt_bias[h] : 0.0f;
+            vec_dt = t < L ? softplus_f(dtr + bias) : 0.0f;
+            vec_a = vec_dt * (prm.A[h] * 1.4426950408889634f);   // dt * A * log2(e)
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float v = __shfl_up_sync(0xffffffffu, vec_a, o);
+                if (lane >= o) vec_a += v;
+            }
+            if (lane == 31) sWs[quad] = vec_a;
+        };
+        auto vecs_stage2 = [&](int parity) {
+            float pre = 0.0f;
+            for (int w = 0; w < quad; ++w) pre += sWs[w];
+            const float cl = vec_a + pre;
+            const float cl_e = __shfl_sync(0xffffffffu, cl, 31);
+            const ChunkVecs cv = chunk_vecs(smem, parity);
+            cv.cl[row] = cl;
+            cv.dt[row] = vec_dt;
+            cv.v[row] = ex2_approx(cl_e - cl) * vec_dt;
+        };
+        auto make_vecs = [&](const Item& it, float dtr, int parity) {   // warps 0-3 only
+            vecs_stage1(it, dtr);
+            named_bar_sync(kVecBarrier, 128);
+            vecs_stage2(parity);
+        };
+
         // Hand chunk `idx` over to the MMA side (bf16 state in smem, Yd / Yo of
-        // the previous chunk consumed).  Waiting for the chunk's vectors first
-        // keeps the control warp at most one vector phase ahead of this side.
+        // the previous chunk consumed); the barrier also publishes the chunk's
+        // vectors, written by warps 0-3, to all elementwise warps.
         auto hand_over = [&](int idx) {
-            mbar_wait_bounded(bar_vec, (uint32_t)idx & 1u, kWaitNs, aborted, prm.status);
+            (void)idx;
             fence_proxy_async_smem();
             tc_fence_before_sync();
+            named_bar_sync(kEwBarrier, kEwThreads);
             mbar_arrive(bar_hx);
         };
         auto begin_segment = [&](const Item& it, int idx) {
@@ -432,6 +417,11 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             hand_over(idx);
         };
 
+        float dtr_next = 0.0f;
+        if (rg.count > 0 && half == 0) {
+            make_vecs(item_at(rg, 0, nc), load_dt(item_at(rg, 0, nc)), 0);
+            if (rg.count > 1) dtr_next = load_dt(item_at(rg, 1, nc));
+        }
         for (int idx = 0; idx < rg.count; ++idx) {
             const uint32_t ph = (uint32_t)idx & 1u;
             const Item it = item_at(rg, idx, nc);
@@ -529,6 +519,12 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             fence_proxy_async_smem();
             tc_fence_before_sync();
             mbar_arrive(bar_mready);
+            // the next chunk's vectors while the tensor cores run (its parity
+            // buffer was last read in chunk idx-1, which every warp has left)
+            if (half == 0 && idx + 1 < rg.count) {
+                make_vecs(item_at(rg, idx + 1, nc), dtr_next, (idx + 1) & 1);
+                if (idx + 2 < rg.count) dtr_next = load_dt(item_at(rg, idx + 2, nc));
+            }
 
             mbar_wait_bounded(bar_m2, ph, kWaitNs, aborted, prm.status);
             tc_fence_after_sync();
