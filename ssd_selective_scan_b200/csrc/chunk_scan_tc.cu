@@ -21,12 +21,15 @@
 // with e the last token of J, both factors <= 1 (the decay never grows), so
 // only the 32 x 32 diagonal blocks need one exponential per element.
 //
-// CTA = 8 elementwise warps + 1 control warp; two CTAs per SM.  The control
-// warp issues the TMA loads (128-byte swizzle, no multicast) and the
-// tcgen05.mma batches, and computes the next chunk's dt / cumulative decay
-// while the elementwise warps work; the two sides meet only on mbarriers.
+// CTA = 16 elementwise warps + 1 control warp, one CTA per SM, software-
+// pipelined across chunks.  The control warp issues the TMA loads (128-byte
+// swizzle, no multicast) into two stages, one chunk ahead, and the tcgen05.mma
+// batches; C B^T of the next chunk runs into a second TMEM buffer while the
+// elementwise warps build the current chunk's decay-masked tile, so the
+// tensor cores and the CUDA cores overlap.  The two sides meet only on
+// mbarriers, each producer at most one phase ahead of its consumers.
 // Elementwise warp w serves TMEM lanes 32*(w%4).. (token rows, or state
-// columns n) and column half w/4.  The fp32 state lives in TMEM and never
+// columns n) and column quarter w/4.  The fp32 state lives in TMEM and never
 // leaves the chip inside a sequence.
 //
 // Scheduling is persistent and balanced: the (sequence x head) chains times
@@ -56,34 +59,38 @@ using namespace sm100;
 constexpr int kQ = 128;          // chunk length
 constexpr int kP = 64;           // head dim
 constexpr int kN = 128;          // state size
-constexpr int kEwThreads = 256;  // 8 elementwise warps: 4 lane quadrants x 2 column halves
+constexpr int kEwWarps = 16;     // elementwise warps: 4 lane quadrants x 4 column quarters
+constexpr int kEwThreads = kEwWarps * 32;
 constexpr int kThreads = kEwThreads + 32;
-constexpr int kCtlWarp = kEwThreads / 32;
-constexpr uint32_t kTmemCols = 256;
+constexpr int kCtlWarp = kEwWarps;
+constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr int kEwBarrier = 1;    // named barrier among the elementwise warps
-constexpr int kVecBarrier = 2;   // named barrier among elementwise warps 0-3
+constexpr int kVecBarrier = 2;   // named barrier among the vector warps (lane quadrant 1)
 
 // Shared-memory layout, offsets from a 1024-byte aligned base.  Tiles are
 // 128-byte swizzled: 128-byte rows, 16-byte chunk c of row r at r*128 +
 // ((c ^ (r & 7)) * 16).  Tiles 128 elements wide along their contiguous
 // dimension are stored as two 16 KB halves (64 elements each).
-constexpr int kOffB = 0;              // B tile  [128 tok][128 n]   (2 halves)
-constexpr int kOffC = 32768;          // C tile  [128 tok][128 n]   (2 halves), then M [128 i][128 j]
-constexpr int kOffX = 65536;          // X tile  [128 tok][64 p]
-constexpr int kOffHX = 81920;         // bf16 state [128 n][64 p], then w o X [128 tok][64 p]
-constexpr int kOffVec = 98304;        // per chunk parity: cl, dt, v  (3 x float[128]) x 2
-constexpr int kOffBar = kOffVec + 3072 + 32;  // (4 warp totals before it) 6 mbarriers
-constexpr int kOffMisc = kOffBar + 64;   // tmem slot, abort flag, ticket
+constexpr int kStageBytes = 81920;    // B [128 tok][128 n], C [128 tok][128 n], X [128 tok][64 p]
+constexpr int kOffStage = 0;          // 2 stages
+constexpr int kStB = 0, kStC = 32768, kStX = 65536;
+constexpr int kOffM = 2 * kStageBytes;          // masked tile M [128 i][128 j]
+constexpr int kOffHX = kOffM + 32768;           // bf16 state [128 n][64 p], then w o X [128 tok][64 p]
+constexpr int kOffVec = kOffHX + 16384;         // per chunk parity: cl, dt, v  (3 x float[128]) x 2
+constexpr int kOffWs = kOffVec + 3072;          // float[8] scan totals
+constexpr int kOffBar = kOffWs + 32;            // mbarriers
+constexpr int kOffMisc = kOffBar + 96;          // tmem slot, abort flag, ticket
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
 
 constexpr uint32_t kTileHalf = 16384;
 constexpr uint32_t kBytesLoad = 5 * 16384;   // B, C (two halves each) and X
 
 // TMEM columns
-constexpr uint32_t kColG = 0;     // G [0,128), then Yd [0,64)
-constexpr uint32_t kColYo = 128;  // Yo [128,192)
-constexpr uint32_t kColH = 192;   // fp32 state [192,256): lane n, column p
+constexpr uint32_t kColG = 0;     // G, two buffers [0,128) and [128,256)
+constexpr uint32_t kColYd = 256;  // Yd [256,320)
+constexpr uint32_t kColYo = 320;  // Yo [320,384)
+constexpr uint32_t kColH = 384;   // fp32 state [384,448): lane n, column p
 
 // instruction descriptors
 constexpr uint32_t kIdG = umma_idesc_bf16(128, 128, false, false);   // C (K-maj) x B (K-maj)
@@ -95,6 +102,14 @@ constexpr uint32_t kIdS = umma_idesc_bf16(128, 64, true, true);      // B^T (MN-
 // fp32 state [P][N] per range boundary.
 constexpr size_t kWsCtrlBytes(int slots) { return ((size_t)(64 + 4 * slots) + 255) / 256 * 256; }
 constexpr size_t kStateBytes = (size_t)kP * kN * 4;
+
+// softplus(v) = max(v, 0) + log(1 + e^-|v|) with the hardware exp and log
+// (bf16 outputs: well inside their rounding; for v < -17 the log term
+// rounds to 0, i.e. dt below 4e-8 becomes 0).
+__device__ inline float softplus_fast(float v)
+{
+    return fmaxf(v, 0.0f) + __logf(1.0f + __expf(-fabsf(v)));
+}
 
 __device__ inline uint32_t sw128(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
 
@@ -145,6 +160,23 @@ __device__ inline ChunkVecs chunk_vecs(uint8_t* smem, int parity)
     return ChunkVecs{base, base + kQ, base + 2 * kQ};
 }
 
+// Division by a runtime constant d (1 <= d < 2^31) as a multiply-high and
+// a shift (round-up reciprocal method for 32-bit unsigned division).
+struct FastDiv {
+    uint32_t d, m, s;
+    __host__ static FastDiv make(uint32_t d)
+    {
+        FastDiv f;
+        f.d = d;
+        f.s = 0;
+        while ((1ull << f.s) < d) ++f.s;
+        f.m = (uint32_t)((((1ull << 32) * ((1ull << f.s) - d)) / d) + 1);
+        return f;
+    }
+    __device__ uint32_t div(uint32_t n) const { return (__umulhi(n, m) + n) >> s; }
+    __device__ uint32_t mod(uint32_t n) const { return n - div(n) * d; }
+};
+
 // A CTA's contiguous range of the unit list (chain-major, nc chunks per
 // chain), in processing order: A = the head of the last chain (published at
 // its end), B = whole chains, C = the tail of the first chain (starts from
@@ -177,7 +209,7 @@ struct Item {
     bool seg_start, seg_end, publish, depend;
 };
 
-__device__ inline Item item_at(const Range& r, int idx, int nc)
+__device__ inline Item item_at(const Range& r, int idx, int nc, const FastDiv& fnc)
 {
     Item it;
     if (idx < r.lenA) {
@@ -192,8 +224,9 @@ __device__ inline Item item_at(const Range& r, int idx, int nc)
     idx -= r.lenA;
     const int nb = (r.chB1 - r.chB0) * nc;
     if (idx < nb) {
-        it.chain = r.chB0 + idx / nc;
-        it.chunk = idx % nc;
+        const uint32_t q = fnc.div((uint32_t)idx);
+        it.chain = r.chB0 + (int)q;
+        it.chunk = idx - (int)q * nc;
         it.seg_start = it.chunk == 0;
         it.seg_end = it.chunk == nc - 1;
         it.publish = false;
@@ -220,12 +253,25 @@ struct Params {
     float* final_state;
     int L, H, G, nc, nslots;
     long long units;
+    FastDiv fnc, fH, fHG;   // division by nc, H, H / G
     int* ws_ctrl;        // [0] ticket, [16 + t] hand-off flag of boundary t
     float* ws_states;    // [nslots][P][N]
     int32_t* status;
 };
 
-__global__ void __launch_bounds__(kThreads, 2)
+__device__ inline void tmem_ld8(uint32_t taddr, float (&v)[8])
+{
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7])
+                 : "r"(taddr)
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
 chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const Params prm)
 {
@@ -233,28 +279,31 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(smem + kOffBar);   // TMA B, C, X landed
-    uint64_t* bar_m1 = bar_ld + 1;      // G and Yo done
-    uint64_t* bar_m2 = bar_ld + 2;      // Yd and the state update done
-    uint64_t* bar_mready = bar_ld + 4;  // M, w o X, scaled state ready (elementwise warps)
-    uint64_t* bar_hx = bar_ld + 5;      // bf16 state in smem, Yd / Yo consumed (elementwise warps)
+    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(smem + kOffBar);   // [2]: TMA stage landed
+    uint64_t* bar_m1 = bar_ld + 2;      // G ready
+    uint64_t* bar_m3 = bar_ld + 3;      // Yo ready (bf16 state read)
+    uint64_t* bar_m2 = bar_ld + 4;      // Yd and the state update done
+    uint64_t* bar_mready = bar_ld + 5;  // masked tile M ready (elementwise warps)
+    uint64_t* bar_hx = bar_ld + 6;      // bf16 state in smem, Yd / Yo consumed (elementwise warps)
+    uint64_t* bar_sready = bar_ld + 7;  // w o X and decayed state ready (elementwise warps)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* aborted = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
     int* ticket_slot = reinterpret_cast<int*>(smem + kOffMisc + 8);
-    uint8_t* sB = smem + kOffB;
-    uint8_t* sC = smem + kOffC;   // C, then M
-    uint8_t* sX = smem + kOffX;
-    uint8_t* sHX = smem + kOffHX; // bf16 state, then w o X
-    const uint32_t aB = smem_u32(sB), aC = smem_u32(sC), aX = smem_u32(sX), aHX = smem_u32(sHX);
+    uint8_t* sM = smem + kOffM;
+    uint8_t* sHX = smem + kOffHX;  // bf16 state, then w o X
+    const uint32_t aM = smem_u32(sM), aHX = smem_u32(sHX);
     const int H = prm.H, nc = prm.nc, L = prm.L;
 
     if (tid == 0) {
         *aborted = 0;
         mbar_init(bar_ld, 1);
+        mbar_init(bar_ld + 1, 1);
         mbar_init(bar_m1, 1);
+        mbar_init(bar_m3, 1);
         mbar_init(bar_m2, 1);
         mbar_init(bar_mready, kEwThreads);
         mbar_init(bar_hx, kEwThreads);
+        mbar_init(bar_sready, kEwThreads);
         fence_mbar_init();
         *ticket_slot = atomicAdd(prm.ws_ctrl, 1);
     }
@@ -268,48 +317,102 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
 
     if (warp == kCtlWarp) {
         // ------------------------------------------------------------------
-        // control warp: TMA, MMA issue, chunk vectors
+        // control warp (one thread): TMA and MMA issue
         // ------------------------------------------------------------------
-        if (lane == 0) {
+        if (lane == 0 && rg.count > 0) {
             prefetch_tensormap(&tmX);
             prefetch_tensormap(&tmB);
             prefetch_tensormap(&tmC);
-        }
-        auto issue_loads = [&](const Item& it) {
-            const int bi = it.chain / H, h = it.chain % H, g = h / (H / prm.G);
-            const int t0 = it.chunk * kQ;
-            mbar_arrive_expect_tx(bar_ld, kBytesLoad);
-            tma_load_3d(sB, &tmB, g * kN, t0, bi, bar_ld);
-            tma_load_3d(sB + kTileHalf, &tmB, g * kN + 64, t0, bi, bar_ld);
-            tma_load_3d(sC, &tmC, g * kN, t0, bi, bar_ld);
-            tma_load_3d(sC + kTileHalf, &tmC, g * kN + 64, t0, bi, bar_ld);
-            tma_load_3d(sX, &tmX, h * kP, t0, bi, bar_ld);
-        };
-        if (rg.count > 0 && lane == 0) {
-            issue_loads(item_at(rg, 0, nc));
+            auto stage = [&](int idx) { return smem + kOffStage + (idx & 1) * kStageBytes; };
+            auto coords = [&](const Item& it, int& bi, int& h, int& g) {
+                bi = (int)prm.fH.div((uint32_t)it.chain);
+                h = it.chain - bi * H;
+                g = (int)prm.fHG.div((uint32_t)h);
+            };
+            auto issue_loads = [&](int idx) {
+                const Item it = item_at(rg, idx, nc, prm.fnc);
+                int bi, h, g;
+                coords(it, bi, h, g);
+                const int t0 = it.chunk * kQ;
+                uint8_t* st = stage(idx);
+                uint64_t* bar = bar_ld + (idx & 1);
+                mbar_arrive_expect_tx(bar, kBytesLoad);
+                tma_load_3d(st + kStB, &tmB, g * kN, t0, bi, bar);
+                tma_load_3d(st + kStB + kTileHalf, &tmB, g * kN + 64, t0, bi, bar);
+                tma_load_3d(st + kStC, &tmC, g * kN, t0, bi, bar);
+                tma_load_3d(st + kStC + kTileHalf, &tmC, g * kN + 64, t0, bi, bar);
+                tma_load_3d(st + kStX, &tmX, h * kP, t0, bi, bar);
+            };
+            auto prefetch_l2 = [&](int idx) {
+                const Item it = item_at(rg, idx, nc, prm.fnc);
+                int bi, h, g;
+                coords(it, bi, h, g);
+                const int t0 = it.chunk * kQ;
+                tma_prefetch_l2_3d(&tmB, g * kN, t0, bi);
+                tma_prefetch_l2_3d(&tmB, g * kN + 64, t0, bi);
+                tma_prefetch_l2_3d(&tmC, g * kN, t0, bi);
+                tma_prefetch_l2_3d(&tmC, g * kN + 64, t0, bi);
+                tma_prefetch_l2_3d(&tmX, h * kP, t0, bi);
+            };
+            auto wait_ld = [&](int idx) {
+                mbar_wait_bounded(bar_ld + (idx & 1), (uint32_t)(idx >> 1) & 1u, kWaitNs, aborted, prm.status);
+            };
+            // Matrix descriptors of K-step 0 for every operand; K-step k adds
+            // a constant to the start-address field (no carry: shared-memory
+            // addresses stay below 256 KB).
+            // Stage 1 is kStageBytes after stage 0, so its descriptors are
+            // stage 0's plus a constant; selected without indexing.
+            const uint32_t st0 = smem_u32(smem + kOffStage);
+            const uint64_t dCk0 = desc_kmajor(st0 + kStC, 0), dBk0 = desc_kmajor(st0 + kStB, 0);
+            const uint64_t dBmn0 = desc_mnmajor(st0 + kStB, 0), dXmn0 = desc_mnmajor(st0 + kStX, 0);
+            const uint64_t dMk = desc_kmajor(aM, 0), dHXmn = desc_mnmajor(aHX, 0);
+            constexpr uint64_t kStageStep = (uint64_t)(kStageBytes >> 4);
+            auto kstep_k = [](int k) -> uint64_t { return (uint64_t)(((k >> 2) * kTileHalf + (k & 3) * 32u) >> 4); };
+            auto kstep_mn = [](int k) -> uint64_t { return (uint64_t)((k * 2048u) >> 4); };
+            auto mma_G = [&](int idx) {   // G = C B^T into buffer idx & 1
+                const uint64_t so = (idx & 1) ? kStageStep : 0;
+                const uint64_t dC = dCk0 + so, dB = dBk0 + so;
+                const uint32_t d = tmem + kColG + (uint32_t)(idx & 1) * 128u;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) umma_bf16(d, dC + kstep_k(k), dB + kstep_k(k), kIdG, k > 0);
+                umma_commit(bar_m1);
+            };
+
+            issue_loads(0);
+            if (rg.count > 1) issue_loads(1);
+            if (rg.count > 2) prefetch_l2(2);
+            wait_ld(0);
+            tc_fence_after_sync();
+            mma_G(0);
             for (int idx = 0; idx < rg.count; ++idx) {
                 const uint32_t ph = (uint32_t)idx & 1u;
-                mbar_wait_bounded(bar_ld, ph, kWaitNs, aborted, prm.status);
+                const uint64_t so = (idx & 1) ? kStageStep : 0;
+                const uint64_t dC = dCk0 + so, dBmn = dBmn0 + so, dXmn = dXmn0 + so;
                 mbar_wait_bounded(bar_hx, ph, kWaitNs, aborted, prm.status);
                 tc_fence_after_sync();
 #pragma unroll
-                for (int k = 0; k < 8; ++k)   // G = C B^T
-                    umma_bf16(tmem + kColG, desc_kmajor(aC, k), desc_kmajor(aB, k), kIdG, k > 0);
-#pragma unroll
                 for (int k = 0; k < 8; ++k)   // Yo = C h^T
-                    umma_bf16(tmem + kColYo, desc_kmajor(aC, k), desc_mnmajor(aHX, k), kIdYo, k > 0);
-                umma_commit(bar_m1);
+                    umma_bf16(tmem + kColYo, dC + kstep_k(k), dHXmn + kstep_mn(k), kIdYo, k > 0);
+                umma_commit(bar_m3);
+                if (idx + 1 < rg.count) {
+                    wait_ld(idx + 1);
+                    tc_fence_after_sync();
+                    mma_G(idx + 1);
+                }
+                mbar_wait_bounded(bar_sready, ph, kWaitNs, aborted, prm.status);
+                tc_fence_after_sync();
+#pragma unroll
+                for (int k = 0; k < 8; ++k)   // h += B^T (w o X)   (h already decayed)
+                    umma_bf16(tmem + kColH, dBmn + kstep_mn(k), dHXmn + kstep_mn(k), kIdS, 1);
                 mbar_wait_bounded(bar_mready, ph, kWaitNs, aborted, prm.status);
                 tc_fence_after_sync();
 #pragma unroll
                 for (int k = 0; k < 8; ++k)   // Yd = M X
-                    umma_bf16(tmem + kColG, desc_kmajor(aC, k), desc_mnmajor(aX, k), kIdYd, k > 0);
-#pragma unroll
-                for (int k = 0; k < 8; ++k)   // h += B^T (w o X)   (h already decayed)
-                    umma_bf16(tmem + kColH, desc_mnmajor(aB, k), desc_mnmajor(aHX, k), kIdS, 1);
+                    umma_bf16(tmem + kColYd, dMk + kstep_k(k), dXmn + kstep_mn(k), kIdYd, k > 0);
                 umma_commit(bar_m2);
                 mbar_wait_bounded(bar_m2, ph, kWaitNs, aborted, prm.status);
-                if (idx + 1 < rg.count) issue_loads(item_at(rg, idx + 1, nc));
+                if (idx + 2 < rg.count) issue_loads(idx + 2);
+                if (idx + 3 < rg.count) prefetch_l2(idx + 3);
             }
         }
         __syncwarp();
@@ -318,67 +421,75 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         // elementwise warps
         // ------------------------------------------------------------------
         const int quad = warp & 3;          // TMEM lane quadrant
-        const int half = warp >> 2;         // column half
+        const int quarter = warp >> 2;      // column quarter
         const int row = quad * 32 + lane;   // token row i / state column n
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const uint32_t tG = tmem + kColG, tYd = tmem + kColG, tYo = tmem + kColYo;
-        const uint32_t tH = tmem + kColH + (uint32_t)half * 32 + lane_off;
+        const uint32_t tH = tmem + kColH + (uint32_t)quarter * 16 + lane_off;
+        // warps 1, 5, 9, 13 compute the chunk vectors (their sub-partition
+        // does not host the control warp)
+        const bool vec_warp = quad == 1;
+        const int vrow = quarter * 32 + lane;   // their token
+        float* sWs = reinterpret_cast<float*>(smem + kOffWs);
 
-        // start of a segment: fp32 state into TMEM, bf16 copy into smem
-        float* sWs = reinterpret_cast<float*>(smem + kOffBar) - 8;   // 4 warp totals
-        // dt_raw of token `row` of an item's chunk (warps 0-3)
-        auto load_dt = [&](const Item& it) -> float {
-            const int t = it.chunk * kQ + row;
-            if (half != 0 || t >= L) return 0.0f;
-            const int bi = it.chain / H, h = it.chain % H;
-            return __bfloat162float(prm.dt_raw[((size_t)bi * L + t) * H + h]);
+        // Inputs of an item's chunk vectors for token `vrow`: raw dt,
+        // A * log2(e), dt_bias.  Loaded a chunk ahead of use.
+        // The loads are only issued here; their values are first used a
+        // chunk later, so the vector warps never wait on them.
+        struct VecIn {
+            float a, bias;
+            unsigned short dtr;   // raw bf16 bits
+            bool valid;
         };
-        // Chunk vectors of an item (warps 0-3, one token each): dt, the
-        // inclusive cumulative log2 decay and the off-diagonal column factor.
-        // Stage 1 scans within each warp; stage 2, after a barrier among the
-        // four warps, adds the preceding warps' totals and writes the vectors.
-        float vec_a = 0.0f, vec_dt = 0.0f;
-        auto vecs_stage1 = [&](const Item& it, float dtr) {
-            const int h = it.chain % H;
-            const int t = it.chunk * kQ + row;
-            const float bias = prm.dt_bias ? prm.dt_bias[h] : 0.0f;
-            vec_dt = t < L ? softplus_f(dtr + bias) : 0.0f;
-            vec_a = vec_dt * (prm.A[h] * 1.4426950408889634f);   // dt * A * log2(e)
+        auto load_vec_in = [&](const Item& it) -> VecIn {
+            VecIn v{0.0f, 0.0f, 0, false};
+            const int t = it.chunk * kQ + vrow;
+            const int bi = (int)prm.fH.div((uint32_t)it.chain), h = it.chain - bi * H;
+            v.a = prm.A[h];
+            v.bias = prm.dt_bias ? prm.dt_bias[h] : 0.0f;
+            v.valid = t < L;
+            const unsigned short* dp = reinterpret_cast<const unsigned short*>(prm.dt_raw);
+            v.dtr = v.valid ? dp[((size_t)bi * L + t) * H + h] : (unsigned short)0;
+            return v;
+        };
+        // Chunk vectors (vector warps, one token each): dt, the inclusive
+        // cumulative log2 decay and the off-diagonal column factor.  A scan
+        // within each warp, a barrier among the four, then the prefix.
+        auto make_vecs = [&](const VecIn& in, int parity) {
+            const float dtr = __uint_as_float((uint32_t)in.dtr << 16);
+            const float dt = in.valid ? softplus_fast(dtr + in.bias) : 0.0f;
+            float a = dt * (in.a * 1.4426950408889634f);   // dt * A * log2(e)
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const float v = __shfl_up_sync(0xffffffffu, vec_a, o);
-                if (lane >= o) vec_a += v;
+                const float v = __shfl_up_sync(0xffffffffu, a, o);
+                if (lane >= o) a += v;
             }
-            if (lane == 31) sWs[quad] = vec_a;
-        };
-        auto vecs_stage2 = [&](int parity) {
+            if (lane == 31) sWs[quarter] = a;
+            named_bar_sync(kVecBarrier, 128);
             float pre = 0.0f;
-            for (int w = 0; w < quad; ++w) pre += sWs[w];
-            const float cl = vec_a + pre;
+            for (int w = 0; w < quarter; ++w) pre += sWs[w];
+            const float cl = a + pre;
             const float cl_e = __shfl_sync(0xffffffffu, cl, 31);
             const ChunkVecs cv = chunk_vecs(smem, parity);
-            cv.cl[row] = cl;
-            cv.dt[row] = vec_dt;
-            cv.v[row] = ex2_approx(cl_e - cl) * vec_dt;
-        };
-        auto make_vecs = [&](const Item& it, float dtr, int parity) {   // warps 0-3 only
-            vecs_stage1(it, dtr);
-            named_bar_sync(kVecBarrier, 128);
-            vecs_stage2(parity);
+            cv.cl[vrow] = cl;
+            cv.dt[vrow] = dt;
+            cv.v[vrow] = ex2_approx(cl_e - cl) * dt;
+            named_bar_sync(kVecBarrier, 128);   // totals read before the next scan overwrites them
         };
 
-        // Hand chunk `idx` over to the MMA side (bf16 state in smem, Yd / Yo of
-        // the previous chunk consumed); the barrier also publishes the chunk's
-        // vectors, written by warps 0-3, to all elementwise warps.
-        auto hand_over = [&](int idx) {
-            (void)idx;
+        // Hand chunk k over to the MMA side: its G is ready (waited here, so
+        // the G barrier never runs two phases ahead), the bf16 state is in
+        // smem and the previous chunk's Yd / Yo are consumed.  The barrier
+        // also publishes chunk k's vectors to every elementwise warp.
+        auto hand_over = [&](int k) {
+            mbar_wait_bounded(bar_m1, (uint32_t)k & 1u, kWaitNs, aborted, prm.status);
             fence_proxy_async_smem();
             tc_fence_before_sync();
             named_bar_sync(kEwBarrier, kEwThreads);
             mbar_arrive(bar_hx);
         };
+        // start of a segment: fp32 state into TMEM, bf16 copy into smem
         auto begin_segment = [&](const Item& it, int idx) {
-            const int bi = it.chain / H, h = it.chain % H;
+            const int bi = (int)prm.fH.div((uint32_t)it.chain), h = it.chain - bi * H;
             const float* src = nullptr;
             bool cg = false;
             if (it.depend) {
@@ -399,142 +510,140 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             } else if (prm.init_state) {
                 src = prm.init_state + ((size_t)bi * H + h) * (size_t)(kP * kN);
             }
+            const int p0 = quarter * 16;
+            float hv[16];
 #pragma unroll
-            for (int pc = 0; pc < 2; ++pc) {
-                const int p0 = half * 32 + pc * 16;
-                float hv[16];
-#pragma unroll
-                for (int p = 0; p < 16; ++p) {
-                    const float* q = src + (size_t)(p0 + p) * kN + row;
-                    hv[p] = src ? (cg ? __ldcg(q) : *q) : 0.0f;
-                }
-                tmem_st16(tH + pc * 16, hv);
-#pragma unroll
-                for (int q = 0; q < 2; ++q)
-                    *reinterpret_cast<uint4*>(sHX + sw128(row, (p0 >> 3) + q)) = pack_bf16x8(&hv[q * 8]);
+            for (int p = 0; p < 16; ++p) {
+                const float* q = src + (size_t)(p0 + p) * kN + row;
+                hv[p] = src ? (cg ? __ldcg(q) : *q) : 0.0f;
             }
+            tmem_st16(tH, hv);
+#pragma unroll
+            for (int q = 0; q < 2; ++q)
+                *reinterpret_cast<uint4*>(sHX + sw128(row, (p0 >> 3) + q)) = pack_bf16x8(&hv[q * 8]);
             tmem_wait_st();
             hand_over(idx);
         };
 
-        float dtr_next = 0.0f;
-        if (rg.count > 0 && half == 0) {
-            make_vecs(item_at(rg, 0, nc), load_dt(item_at(rg, 0, nc)), 0);
-            if (rg.count > 1) dtr_next = load_dt(item_at(rg, 1, nc));
+        VecIn vin_next{0.0f, 0.0f, 0, false};
+        if (rg.count > 0) {
+            if (vec_warp) {
+                make_vecs(load_vec_in(item_at(rg, 0, nc, prm.fnc)), 0);
+                if (rg.count > 1) vin_next = load_vec_in(item_at(rg, 1, nc, prm.fnc));
+            }
         }
         for (int idx = 0; idx < rg.count; ++idx) {
             const uint32_t ph = (uint32_t)idx & 1u;
-            const Item it = item_at(rg, idx, nc);
-            const int bi = it.chain / H, h = it.chain % H;
+            const Item it = item_at(rg, idx, nc, prm.fnc);
+            const int bi = (int)prm.fH.div((uint32_t)it.chain), h = it.chain - bi * H;
             const float Dh = prm.D ? prm.D[h] : 0.0f;
+            uint8_t* st = smem + kOffStage + (idx & 1) * kStageBytes;
             if (it.seg_start) begin_segment(it, idx);
-
-            mbar_wait_bounded(bar_m1, ph, kWaitNs, aborted, prm.status);
-            mbar_wait_bounded(bar_ld, ph, kWaitNs, aborted, prm.status);
             tc_fence_after_sync();
+
             const ChunkVecs cv = chunk_vecs(smem, (int)ph);
             const float cl_i = cv.cl[row];
             const float cl_last = cv.cl[kQ - 1];
 
-            // x of this thread's row and column half (kept for D x)
-            uint4 xraw[4];
+            // M = G o L for row `row` (G in buffer idx & 1).  Column block jb
+            // (32 tokens) is zero above the row quadrant's diagonal block; of
+            // every other block, column quarter `quarter` takes 8 columns.
+            const uint32_t tG = tmem + kColG + (uint32_t)(idx & 1) * 128u + lane_off;
+            // Block jb (32 tokens) of the masked tile: zero above the row
+            // quadrant's diagonal block; of every other block, column quarter
+            // `quarter` takes 8 columns.
+            auto m_block = [&](int jb) {
+                const int j0 = jb * 32 + quarter * 8;
+                uint4 packed = make_uint4(0, 0, 0, 0);
+                if (jb <= quad) {
+                    float gv[8];
+                    tmem_ld8(tG + j0, gv);
+                    tmem_wait_ld();
+                    float m[8];
+                    if (jb < quad) {
+                        const float u = ex2_approx(cl_i - cv.cl[jb * 32 + 31]);
+                        const float4 va = reinterpret_cast<const float4*>(cv.v + j0)[0];
+                        const float4 vb = reinterpret_cast<const float4*>(cv.v + j0)[1];
+                        const float vv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
-            for (int q = 0; q < 4; ++q) xraw[q] = *reinterpret_cast<const uint4*>(sX + sw128(row, half * 4 + q));
-
-            // M = G o L: row `row`, column blocks {0,3} (half 0) or {1,2} (half 1),
-            // written over C (both MMAs reading C are done); 16 columns at a time
-#pragma unroll
-            for (int s2 = 0; s2 < 2; ++s2) {
-                const int jb = half == 0 ? (s2 == 0 ? 0 : 3) : (s2 == 0 ? 1 : 2);
-                const float u = ex2_approx(cl_i - cv.cl[jb * 32 + 31]);
-#pragma unroll
-                for (int pc = 0; pc < 2; ++pc) {
-                    const int j0 = jb * 32 + pc * 16;
-                    uint4 packed[2];
-                    if (jb <= quad) {
-                        float gv[16];
-                        tmem_ld16(tG + lane_off + j0, gv);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int q = 0; q < 2; ++q) {
-                            float m[8];
-                            if (jb < quad) {
-                                const float4 va = reinterpret_cast<const float4*>(cv.v + j0 + q * 8)[0];
-                                const float4 vb = reinterpret_cast<const float4*>(cv.v + j0 + q * 8)[1];
-                                const float vv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
-#pragma unroll
-                                for (int e = 0; e < 8; ++e) m[e] = gv[q * 8 + e] * u * vv[e];
-                            } else {
-                                const float4 ca = reinterpret_cast<const float4*>(cv.cl + j0 + q * 8)[0];
-                                const float4 cb = reinterpret_cast<const float4*>(cv.cl + j0 + q * 8)[1];
-                                const float4 da = reinterpret_cast<const float4*>(cv.dt + j0 + q * 8)[0];
-                                const float4 db = reinterpret_cast<const float4*>(cv.dt + j0 + q * 8)[1];
-                                const float cc[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
-                                const float dd[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
-#pragma unroll
-                                for (int e = 0; e < 8; ++e) {
-                                    const int j = j0 + q * 8 + e;
-                                    const float v = gv[q * 8 + e] * ex2_approx(cl_i - cc[e]) * dd[e];
-                                    m[e] = (j <= row) ? v : 0.0f;
-                                }
-                            }
-                            packed[q] = pack_bf16x8(m);
-                        }
+                        for (int e = 0; e < 8; ++e) m[e] = gv[e] * u * vv[e];
                     } else {
-                        packed[0] = packed[1] = make_uint4(0, 0, 0, 0);
-                    }
+                        const float4 ca = reinterpret_cast<const float4*>(cv.cl + j0)[0];
+                        const float4 cb = reinterpret_cast<const float4*>(cv.cl + j0)[1];
+                        const float4 da = reinterpret_cast<const float4*>(cv.dt + j0)[0];
+                        const float4 db = reinterpret_cast<const float4*>(cv.dt + j0)[1];
+                        const float cc[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+                        const float dd[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
 #pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const int jq = j0 + q * 8;
-                        *reinterpret_cast<uint4*>(sC + (jq >> 6) * kTileHalf + sw128(row, (jq & 63) >> 3)) = packed[q];
+                        for (int e = 0; e < 8; ++e) {
+                            const int j = j0 + e;
+                            const float v = gv[e] * ex2_approx(cl_i - cc[e]) * dd[e];
+                            m[e] = (j <= row) ? v : 0.0f;
+                        }
                     }
+                    packed = pack_bf16x8(m);
                 }
-            }
-            // w o X over the bf16 state copy (C h^T, its reader, is done)
+                *reinterpret_cast<uint4*>(sM + (j0 >> 6) * kTileHalf + sw128(row, (j0 & 63) >> 3)) = packed;
+            };
+            // first half of the masked tile while C h^T reads the bf16 state
+            m_block(0);
+            m_block(1);
+
+            // x of this thread's row and column quarter (kept for D x)
+            mbar_wait_bounded(bar_ld + (idx & 1), (uint32_t)(idx >> 1) & 1u, kWaitNs, aborted, prm.status);
+            uint4 xraw[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q)
+                xraw[q] = *reinterpret_cast<const uint4*>(st + kStX + sw128(row, quarter * 2 + q));
+
+            // w o X over the bf16 state copy once C h^T has read it
+            mbar_wait_bounded(bar_m3, ph, kWaitNs, aborted, prm.status);
             {
                 const float wj = ex2_approx(cl_last - cl_i) * cv.dt[row];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < 2; ++q) {
                     float v[8];
                     unpack_bf16x8(xraw[q], v);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) v[e] *= wj;
-                    *reinterpret_cast<uint4*>(sHX + sw128(row, half * 4 + q)) = pack_bf16x8(v);
+                    *reinterpret_cast<uint4*>(sHX + sw128(row, quarter * 2 + q)) = pack_bf16x8(v);
                 }
             }
             // decay the fp32 state in place; the chunk-state product accumulates onto it
             {
                 const float decay = ex2_approx(cl_last);
+                float hv[16];
+                tmem_ld16(tH, hv);
+                tmem_wait_ld();
 #pragma unroll
-                for (int pc = 0; pc < 2; ++pc) {
-                    float hv[16];
-                    tmem_ld16(tH + pc * 16, hv);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int p = 0; p < 16; ++p) hv[p] *= decay;
-                    tmem_st16(tH + pc * 16, hv);
-                }
+                for (int p = 0; p < 16; ++p) hv[p] *= decay;
+                tmem_st16(tH, hv);
                 tmem_wait_st();
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
+            mbar_arrive(bar_sready);   // the chunk-state product can start
+
+            m_block(2);
+            m_block(3);
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
             mbar_arrive(bar_mready);
-            // the next chunk's vectors while the tensor cores run (its parity
-            // buffer was last read in chunk idx-1, which every warp has left)
-            if (half == 0 && idx + 1 < rg.count) {
-                make_vecs(item_at(rg, idx + 1, nc), dtr_next, (idx + 1) & 1);
-                if (idx + 2 < rg.count) dtr_next = load_dt(item_at(rg, idx + 2, nc));
+
+            // the next chunk's vectors while the tensor cores run
+            if (vec_warp && idx + 1 < rg.count) {
+                make_vecs(vin_next, (idx + 1) & 1);
+                if (idx + 2 < rg.count) vin_next = load_vec_in(item_at(rg, idx + 2, nc, prm.fnc));
             }
 
             mbar_wait_bounded(bar_m2, ph, kWaitNs, aborted, prm.status);
             tc_fence_after_sync();
             // new state: bf16 copy for the next chunk, or out at the end of a segment
-#pragma unroll
-            for (int pc = 0; pc < 2; ++pc) {
+            {
                 float hv[16];
-                tmem_ld16(tH + pc * 16, hv);
+                tmem_ld16(tH, hv);
                 tmem_wait_ld();
-                const int p0 = half * 32 + pc * 16;
+                const int p0 = quarter * 16;
                 if (!it.seg_end) {
 #pragma unroll
                     for (int q = 0; q < 2; ++q)
@@ -543,41 +652,43 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                     float* dst = prm.ws_states + (size_t)ticket * (kP * kN);
 #pragma unroll
                     for (int p = 0; p < 16; ++p) __stcg(dst + (size_t)(p0 + p) * kN + row, hv[p]);
+                    __threadfence();
+                    named_bar_sync(kEwBarrier, kEwThreads);
+                    if (tid == 0) st_release_gpu(prm.ws_ctrl + 16 + ticket, 1);
                 } else if (prm.final_state) {
                     float* dst = prm.final_state + ((size_t)bi * H + h) * (size_t)(kP * kN);
 #pragma unroll
                     for (int p = 0; p < 16; ++p) dst[(size_t)(p0 + p) * kN + row] = hv[p];
                 }
             }
-            if (it.seg_end && it.publish) {
-                __threadfence();
-                named_bar_sync(kEwBarrier, kEwThreads);
-                if (tid == 0) st_release_gpu(prm.ws_ctrl + 16 + ticket, 1);
-            }
-            // output: y = Yd + 2^cl Yo + D x, token row `row`, p of this half
+            // output: y = Yd + 2^cl Yo + D x, token row `row`, p of this quarter.
+            // Yd / Yo are read and y packed first; the next chunk is then
+            // handed over so its MMAs start while the stores drain.
+            uint4 ypk[2];
             {
-                const int t = it.chunk * kQ + row;
                 const float sc = ex2_approx(cl_i);
-                __nv_bfloat16* yrow = prm.y + (((size_t)bi * L + t) * H + h) * kP + half * 32;
+                float yd[16], yo[16];
+                tmem_ld16(tmem + kColYd + lane_off + quarter * 16, yd);
+                tmem_ld16(tmem + kColYo + lane_off + quarter * 16, yo);
+                tmem_wait_ld();
 #pragma unroll
-                for (int pc = 0; pc < 2; ++pc) {
-                    float yd[16], yo[16];
-                    tmem_ld16(tYd + lane_off + half * 32 + pc * 16, yd);
-                    tmem_ld16(tYo + lane_off + half * 32 + pc * 16, yo);
-                    tmem_wait_ld();
+                for (int q = 0; q < 2; ++q) {
+                    float xv[8], o[8];
+                    unpack_bf16x8(xraw[q], xv);
 #pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        float xv[8], o[8];
-                        unpack_bf16x8(xraw[pc * 2 + q], xv);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) o[e] = yd[q * 8 + e] + sc * yo[q * 8 + e] + Dh * xv[e];
-                        if (t < L) *reinterpret_cast<uint4*>(yrow + pc * 16 + q * 8) = pack_bf16x8(o);
-                    }
+                    for (int e = 0; e < 8; ++e) o[e] = yd[q * 8 + e] + sc * yo[q * 8 + e] + Dh * xv[e];
+                    ypk[q] = pack_bf16x8(o);
                 }
             }
-            // hand Yd / Yo and the bf16 state over to the next chunk's MMAs;
-            // a new segment hands over after loading its initial state
             if (idx + 1 < rg.count && !it.seg_end) hand_over(idx + 1);
+            {
+                const int t = it.chunk * kQ + row;
+                if (t < L) {
+                    __nv_bfloat16* yrow = prm.y + (((size_t)bi * L + t) * H + h) * kP + quarter * 16;
+                    __stcs(reinterpret_cast<uint4*>(yrow), ypk[0]);
+                    __stcs(reinterpret_cast<uint4*>(yrow + 8), ypk[1]);
+                }
+            }
         }
     }
 
@@ -628,7 +739,7 @@ int tc_slots(const ScanArgs& a)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
         sms = 148;
     const long long chains = (long long)a.b * a.H;
-    const long long slots = 2LL * sms;   // two CTAs per SM
+    const long long slots = sms;   // one CTA per SM
     return (int)(chains < slots ? chains : slots);
 }
 
@@ -675,6 +786,9 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t s)
     prm.nc = (a.L + kQ - 1) / kQ;
     prm.nslots = slots;
     prm.units = (long long)a.b * a.H * prm.nc;
+    prm.fnc = FastDiv::make((uint32_t)prm.nc);
+    prm.fH = FastDiv::make((uint32_t)a.H);
+    prm.fHG = FastDiv::make((uint32_t)(a.H / a.G));
     prm.ws_ctrl = static_cast<int*>(a.workspace);
     prm.ws_states = reinterpret_cast<float*>(static_cast<uint8_t*>(a.workspace) + ctrl);
     prm.status = a.status;

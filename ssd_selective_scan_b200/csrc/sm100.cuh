@@ -47,15 +47,20 @@ __device__ inline void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes)
                  : "memory");
 }
 
+// One wait attempt.  The thread is suspended until the phase completes or
+// about kSuspendNs elapse, so a waiting warp does not take issue slots from
+// the warps that are working.
+constexpr uint32_t kSuspendNs = 100000;
+
 __device__ inline bool mbar_try_wait(uint64_t* bar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
         : "memory");
     return ok != 0;
 }
@@ -92,6 +97,15 @@ __device__ inline void tma_load_3d(void* smem_dst, const CUtensorMap* map, int c
         " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
         : "memory");
+}
+
+// Prefetch a tile of a tensor into L2 (no shared memory, no completion).
+__device__ inline void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
 }
 
 __device__ inline void prefetch_tensormap(const CUtensorMap* map)
