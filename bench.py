@@ -98,14 +98,17 @@ def scan_kernel_traffic(kernel_tag: str):
     return None
 
 
+# The sources the tensor-core scan kernel is compiled from.
+SCAN_SOURCES = ("chunk_scan_tc.cu", "sm100.cuh", "common.cuh", "kernels.h")
+
+
 def source_digest() -> str:
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "ssd_selective_scan_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in SCAN_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 

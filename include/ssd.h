@@ -180,8 +180,8 @@ SSD_API ssd_status_t ssd_chunk_scan_fwd(const void* x, const void* B, const void
  *     before any stream capture.
  *   - A call whose scratch need (ssd_chunk_scan_workspace_bytes) exceeds
  *     10 MiB returns SSD_ERR_UNSUPPORTED and launches nothing.  The
- *     tensor-core scan needs at most 2 x SMs x 32 KiB plus a small control
- *     block, about 9.3 MiB on a 148-SM B200.
+ *     tensor-core scan needs at most (SM count) x 32 KiB plus a small
+ *     control block, about 4.6 MiB on a 148-SM B200.
  *   - All calls on a device share the array; the parts that must start at
  *     zero are cleared on the call's stream.  Calls whose executions overlap
  *     on the GPU (unordered streams) race on the array: order them.

@@ -11,8 +11,8 @@
 //
 // The array is kStaticScratchBytes (10 MiB) of file-scope __device__ memory:
 // every GPU that loads this library holds it until the process exits.  The
-// tensor-core scan needs at most 2 x (SM count) x 32 KiB + a small control
-// block (about 9.3 MiB on a 148-SM B200), so every call it can serve fits;
+// tensor-core scan needs at most (SM count) x 32 KiB + a small control
+// block (about 4.6 MiB on a 148-SM B200), so every call it can serve fits;
 // a call whose scratch need (ssd_chunk_scan_workspace_bytes) exceeds the
 // array is refused with SSD_ERR_UNSUPPORTED before anything is launched.
 //
