@@ -3,14 +3,18 @@
 // Architectures for Language Models", summary page, appendix C; conv width 4
 // and SiLU from the Nemotron feasibility report, section 1.4).
 //
-// HBM-bound streaming kernel.  Each thread owns one 16-byte vector of
-// channels (8 bf16 or 4 float) and walks a tile of TT tokens, keeping the
-// k-1 previous inputs in registers; the k-1 halo tokens before its tile are
-// re-read (they were just read by the neighbouring tile, so they come from
-// L2).  Loads and stores are 128-bit and coalesced along channels.
+// HBM-bound streaming kernel.  Each thread owns 4 adjacent channels (an
+// 8-byte bf16 or 16-byte float vector) and walks a tile of 32 tokens,
+// keeping the k-1 previous inputs in registers; the k-1 halo tokens before
+// its tile are re-read (they were just read by the neighbouring tile, so
+// they come from L2).  Tokens move in groups of 8 whose loads are all issued
+// before any is used.  A warp covers 128 consecutive channels, so every load
+// and store instruction is coalesced along channels.  Four channels per
+// thread keep the register count low enough for many resident warps (the
+// bytes in flight per SM are what saturates HBM).
 //
 // The cache is read and rewritten by the thread that owns token tile 0 of a
-// channel vector, so an in-place cache update never races with a reader.
+// channel group, so an in-place cache update never races with a reader.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -19,26 +23,65 @@ namespace ssd {
 constexpr int kConvThreads = 128;
 constexpr int kConvTile = 32;   // tokens per thread
 constexpr int kGroup = 8;       // tokens loaded together
+constexpr int kCpt = 4;         // channels per thread
 
-// The V channels x K columns of one thread's cache block are contiguous and
-// 16*K bytes long (V * sizeof(T) = 16), so they move as K 16-byte vectors.
-// Elements are addressed with compile-time indices only (unrolled loops), so
-// the block stays in registers.
+// 4 channels of type T as one vector register group.
+template <typename T> struct Vec4;
+
+template <> struct Vec4<float> {
+    using raw = uint4;
+    __device__ static raw load(const float* p) { return __ldcs(reinterpret_cast<const uint4*>(p)); }
+    __device__ static void decode(raw q, float (&v)[4]) {
+        v[0] = __uint_as_float(q.x); v[1] = __uint_as_float(q.y);
+        v[2] = __uint_as_float(q.z); v[3] = __uint_as_float(q.w);
+    }
+    __device__ static void store(float* p, const float (&v)[4]) {
+        *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    }
+    __device__ static float act(float v) { return silu_f(v); }
+};
+
+template <> struct Vec4<__nv_bfloat16> {
+    using raw = uint2;
+    __device__ static raw load(const __nv_bfloat16* p) { return __ldcs(reinterpret_cast<const uint2*>(p)); }
+    __device__ static void decode(raw q, float (&v)[4]) {
+        v[0] = __uint_as_float(q.x << 16); v[1] = __uint_as_float(q.x & 0xffff0000u);
+        v[2] = __uint_as_float(q.y << 16); v[3] = __uint_as_float(q.y & 0xffff0000u);
+    }
+    __device__ static void store(__nv_bfloat16* p, const float (&v)[4]) {
+        __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
+        __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
+        *reinterpret_cast<uint2*>(p) = make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
+    }
+    __device__ static float act(float v) { return silu_tanh(v); }
+};
+
+// One thread's cache block: 4 channels x K columns of type T, contiguous
+// (channel-major), moved as K vectors of 4 * sizeof(T) bytes.  Elements are
+// addressed with compile-time indices only, so the block stays in registers.
 template <typename T, int K>
 struct CacheBlock {
-    static constexpr int kWords = 4 * K;
-    uint32_t w[kWords];
+    using R = typename Vec4<T>::raw;
+    static constexpr int kWordsPerVec = sizeof(R) / 4;
+    uint32_t w[K * kWordsPerVec];
     __device__ void load(const T* p) {
 #pragma unroll
         for (int i = 0; i < K; ++i) {
-            const uint4 q = reinterpret_cast<const uint4*>(p)[i];
-            w[4 * i] = q.x; w[4 * i + 1] = q.y; w[4 * i + 2] = q.z; w[4 * i + 3] = q.w;
+            const R q = reinterpret_cast<const R*>(p)[i];
+            const uint32_t* qw = reinterpret_cast<const uint32_t*>(&q);
+#pragma unroll
+            for (int k = 0; k < kWordsPerVec; ++k) w[i * kWordsPerVec + k] = qw[k];
         }
     }
     __device__ void store(T* p) const {
 #pragma unroll
-        for (int i = 0; i < K; ++i)
-            reinterpret_cast<uint4*>(p)[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        for (int i = 0; i < K; ++i) {
+            R q;
+            uint32_t* qw = reinterpret_cast<uint32_t*>(&q);
+#pragma unroll
+            for (int k = 0; k < kWordsPerVec; ++k) qw[k] = w[i * kWordsPerVec + k];
+            reinterpret_cast<R*>(p)[i] = q;
+        }
     }
     __device__ float get(int c, int j) const { return io<T>::word_get(w, c * K + j); }
     __device__ void set(int c, int j, float v) { io<T>::word_set(w, c * K + j, v); }
@@ -50,19 +93,18 @@ struct CacheBlock {
 template <typename T, int K, int S>
 __device__ inline void roll_cache(T* cs, const T* xb, int L, int conv_dim)
 {
-    constexpr int V = io<T>::kVec;
     CacheBlock<T, K> blk;
     if (S < K) blk.load(cs);
 #pragma unroll
     for (int j = 0; j < K; ++j) {
         if (j < K - S) {
 #pragma unroll
-            for (int c = 0; c < V; ++c) blk.set(c, j, blk.get(c, j + S));
+            for (int c = 0; c < kCpt; ++c) blk.set(c, j, blk.get(c, j + S));
         } else {
-            float v[V];
-            io<T>::load_vec(xb + (size_t)(L - K + j) * conv_dim, v);
+            float v[kCpt];
+            Vec4<T>::decode(Vec4<T>::load(xb + (size_t)(L - K + j) * conv_dim), v);
 #pragma unroll
-            for (int c = 0; c < V; ++c) blk.set(c, j, v[c]);
+            for (int c = 0; c < kCpt; ++c) blk.set(c, j, v[c]);
         }
     }
     blk.store(cs);
@@ -74,83 +116,80 @@ conv1d_silu_kernel(const T* __restrict__ xBC, T* __restrict__ out,
                    const float* __restrict__ w, const float* __restrict__ bias,
                    T* __restrict__ conv_state, int L, int conv_dim)
 {
-    constexpr int V = io<T>::kVec;
-    const int nvec = conv_dim / V;
-    const int cv = blockIdx.x * kConvThreads + threadIdx.x;
-    if (cv >= nvec) return;
-    const int c0 = cv * V;
+    using V4 = Vec4<T>;
+    const int ngroups = conv_dim / kCpt;
+    const int cg = blockIdx.x * kConvThreads + threadIdx.x;
+    if (cg >= ngroups) return;
+    const int c0 = cg * kCpt;
     const int t0 = blockIdx.y * kConvTile;
     const int bi = blockIdx.z;
     const T* xb = xBC + (size_t)bi * L * conv_dim + c0;
     T* ob = out + (size_t)bi * L * conv_dim + c0;
 
-    float wt[K][V];
+    // taps of the thread's 4 channels: 4*K contiguous floats
+    float wt[K][kCpt];
     {
-        // the thread's V channels x K taps are V*K contiguous floats
         const float4* w4 = reinterpret_cast<const float4*>(w + (size_t)c0 * K);
-        float wl[V * K];
+        float wl[kCpt * K];
 #pragma unroll
-        for (int i = 0; i < V * K / 4; ++i) {
+        for (int i = 0; i < K; ++i) {
             const float4 q = __ldg(w4 + i);
             wl[4 * i] = q.x; wl[4 * i + 1] = q.y; wl[4 * i + 2] = q.z; wl[4 * i + 3] = q.w;
         }
 #pragma unroll
-        for (int c = 0; c < V; ++c)
+        for (int c = 0; c < kCpt; ++c)
 #pragma unroll
             for (int j = 0; j < K; ++j) wt[j][c] = wl[c * K + j];
     }
-    float bs[V];
+    float bs[kCpt];
 #pragma unroll
-    for (int c = 0; c < V; ++c) bs[c] = bias ? bias[c0 + c] : 0.0f;
+    for (int c = 0; c < kCpt; ++c) bs[c] = bias ? bias[c0 + c] : 0.0f;
 
     // hist[j] holds the input at time t0 - (K-1) + j for j < K-1.
-    float hist[K][V];
+    float hist[K][kCpt];
     if (t0 == 0) {
         if (conv_state) {
             // cache layout [b][conv_dim][K]: column j = time j - K
             CacheBlock<T, K> blk;
             blk.load(conv_state + ((size_t)bi * conv_dim + c0) * K);
 #pragma unroll
-            for (int c = 0; c < V; ++c)
+            for (int c = 0; c < kCpt; ++c)
 #pragma unroll
                 for (int j = 1; j < K; ++j) hist[j - 1][c] = blk.get(c, j);
         } else {
 #pragma unroll
             for (int j = 0; j < K - 1; ++j)
 #pragma unroll
-                for (int c = 0; c < V; ++c) hist[j][c] = 0.0f;
+                for (int c = 0; c < kCpt; ++c) hist[j][c] = 0.0f;
         }
     } else {
 #pragma unroll
-        for (int j = 0; j < K - 1; ++j)
-            io<T>::load_vec(xb + (size_t)(t0 - (K - 1) + j) * conv_dim, hist[j]);
+        for (int j = 0; j < K - 1; ++j) V4::decode(V4::load(xb + (size_t)(t0 - (K - 1) + j) * conv_dim), hist[j]);
     }
 
-    // Tokens move in groups of kGroup: all loads of a group are issued before
-    // any is used, so each thread keeps kGroup x 16 bytes in flight.
     const int t1 = min(L, t0 + kConvTile);
     for (int tb = t0; tb < t1; tb += kGroup) {
-        uint4 raw[kGroup];
+        typename V4::raw raw[kGroup];
 #pragma unroll
         for (int u = 0; u < kGroup; ++u)
-            if (tb + u < t1) raw[u] = __ldcs(reinterpret_cast<const uint4*>(xb + (size_t)(tb + u) * conv_dim));
+            if (tb + u < t1) raw[u] = V4::load(xb + (size_t)(tb + u) * conv_dim);
 #pragma unroll
         for (int u = 0; u < kGroup; ++u) {
             if (tb + u < t1) {
-                io<T>::decode(raw[u], hist[K - 1]);
-                float o[V];
+                V4::decode(raw[u], hist[K - 1]);
+                float o[kCpt];
 #pragma unroll
-                for (int c = 0; c < V; ++c) {
+                for (int c = 0; c < kCpt; ++c) {
                     float acc = bs[c];
 #pragma unroll
                     for (int j = 0; j < K; ++j) acc = fmaf(wt[j][c], hist[j][c], acc);
-                    o[c] = silu_f(acc);
+                    o[c] = V4::act(acc);
                 }
-                io<T>::store_vec(ob + (size_t)(tb + u) * conv_dim, o);
+                V4::store(ob + (size_t)(tb + u) * conv_dim, o);
 #pragma unroll
                 for (int j = 0; j < K - 1; ++j)
 #pragma unroll
-                    for (int c = 0; c < V; ++c) hist[j][c] = hist[j + 1][c];
+                    for (int c = 0; c < kCpt; ++c) hist[j][c] = hist[j + 1][c];
             }
         }
     }
@@ -172,9 +211,8 @@ template <typename T, int K>
 static cudaError_t launch_conv_k(const void* xBC, void* out, const float* w, const float* bias,
                                  void* conv_state, int b, int L, int conv_dim, cudaStream_t s)
 {
-    constexpr int V = io<T>::kVec;
-    const int nvec = conv_dim / V;
-    dim3 grid((nvec + kConvThreads - 1) / kConvThreads, (L + kConvTile - 1) / kConvTile, b);
+    const int ngroups = conv_dim / kCpt;
+    dim3 grid((ngroups + kConvThreads - 1) / kConvThreads, (L + kConvTile - 1) / kConvTile, b);
     conv1d_silu_kernel<T, K><<<grid, kConvThreads, 0, s>>>(
         static_cast<const T*>(xBC), static_cast<T*>(out), w, bias, static_cast<T*>(conv_state),
         L, conv_dim);
