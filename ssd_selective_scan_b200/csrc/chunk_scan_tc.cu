@@ -21,13 +21,17 @@
 // with e the last token of J, both factors <= 1 (the decay never grows), so
 // only the 32 x 32 diagonal blocks need one exponential per element.
 //
-// CTA = 16 elementwise warps + 1 control warp, one CTA per SM, software-
-// pipelined across chunks.  The control warp issues the TMA loads (128-byte
-// swizzle, no multicast) into two stages, one chunk ahead, and the tcgen05.mma
-// batches; C B^T of the next chunk runs into a second TMEM buffer while the
-// elementwise warps build the current chunk's decay-masked tile, so the
-// tensor cores and the CUDA cores overlap.  The two sides meet only on
-// mbarriers, each producer at most one phase ahead of its consumers.
+// CTA = 16 elementwise warps + an MMA warp + a producer warp + a vector
+// warp, one CTA per SM, software-pipelined across chunks.  The producer warp
+// issues the TMA loads (128-byte swizzle, no multicast) into two stages one
+// chunk ahead and stores each chunk's y tile by TMA; the vector warp computes
+// the next chunk's dt / cumulative decay vectors, its dt loads issued a chunk
+// earlier still.  The MMA warp only waits and issues tcgen05.mma (issue
+// blocks until the tensor core accepts the instruction, so nothing else may
+// sit on that thread); C B^T of the next chunk runs into a second TMEM buffer
+// while the elementwise warps build the current chunk's decay-masked tile.
+// The warps meet only on mbarriers, each producer at most one phase ahead of
+// its consumers.
 // Elementwise warp w serves TMEM lanes 32*(w%4).. (token rows, or state
 // columns n) and column quarter w/4.  The fp32 state lives in TMEM and never
 // leaves the chip inside a sequence.
@@ -61,12 +65,13 @@ constexpr int kP = 64;           // head dim
 constexpr int kN = 128;          // state size
 constexpr int kEwWarps = 16;     // elementwise warps: 4 lane quadrants x 4 column quarters
 constexpr int kEwThreads = kEwWarps * 32;
-constexpr int kThreads = kEwThreads + 32;
-constexpr int kCtlWarp = kEwWarps;
+constexpr int kMmaWarp = kEwWarps;       // issues tcgen05.mma
+constexpr int kProdWarp = kEwWarps + 1;  // TMA loads / stores
+constexpr int kVecWarp = kEwWarps + 2;   // chunk vectors (dt, cumulative decay)
+constexpr int kThreads = kEwThreads + 96;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr int kEwBarrier = 1;    // named barrier among the elementwise warps
-constexpr int kVecBarrier = 2;   // named barrier among the vector warps (lane quadrant 1)
 
 // Shared-memory layout, offsets from a 1024-byte aligned base.  Tiles are
 // 128-byte swizzled: 128-byte rows, 16-byte chunk c of row r at r*128 +
@@ -80,11 +85,12 @@ constexpr int kOffHX = kOffM + 32768;           // bf16 state [128 n][64 p], the
 constexpr int kOffVec = kOffHX + 16384;         // per chunk parity: cl, dt, v  (3 x float[128]) x 2
 constexpr int kOffWs = kOffVec + 3072;          // float[8] scan totals
 constexpr int kOffBar = kOffWs + 32;            // mbarriers
-constexpr int kOffMisc = kOffBar + 96;          // tmem slot, abort flag, ticket
+constexpr int kOffMisc = kOffBar + 96;          // tmem slot, abort flag, ticket (12 mbarriers above)
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
 
 constexpr uint32_t kTileHalf = 16384;
-constexpr uint32_t kBytesLoad = 5 * 16384;   // B, C (two halves each) and X
+constexpr uint32_t kBytesBC = 4 * 16384;   // B and C, two halves each
+constexpr uint32_t kBytesX = 16384;
 
 // TMEM columns
 constexpr uint32_t kColG = 0;     // G, two buffers [0,128) and [128,256)
@@ -174,7 +180,6 @@ struct FastDiv {
         return f;
     }
     __device__ uint32_t div(uint32_t n) const { return (__umulhi(n, m) + n) >> s; }
-    __device__ uint32_t mod(uint32_t n) const { return n - div(n) * d; }
 };
 
 // A CTA's contiguous range of the unit list (chain-major, nc chunks per
@@ -273,19 +278,23 @@ __device__ inline void tmem_ld8(uint32_t taddr, float (&v)[8])
 
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmC, const Params prm)
+                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY,
+                     const Params prm)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(smem + kOffBar);   // [2]: TMA stage landed
+    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(smem + kOffBar);   // [2]: stage's B and C landed
     uint64_t* bar_m1 = bar_ld + 2;      // G ready
     uint64_t* bar_m3 = bar_ld + 3;      // Yo ready (bf16 state read)
     uint64_t* bar_m2 = bar_ld + 4;      // Yd and the state update done
     uint64_t* bar_mready = bar_ld + 5;  // masked tile M ready (elementwise warps)
     uint64_t* bar_hx = bar_ld + 6;      // bf16 state in smem, Yd / Yo consumed (elementwise warps)
     uint64_t* bar_sready = bar_ld + 7;  // w o X and decayed state ready (elementwise warps)
+    uint64_t* bar_ystaged = bar_ld + 8; // y tile staged in the chunk's X buffer (elementwise warps)
+    uint64_t* bar_vec = bar_ld + 9;     // chunk vectors published (producer warp)
+    uint64_t* bar_ldx = bar_ld + 10;    // [2]: stage's X landed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* aborted = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
     int* ticket_slot = reinterpret_cast<int*>(smem + kOffMisc + 8);
@@ -304,6 +313,10 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         mbar_init(bar_mready, kEwThreads);
         mbar_init(bar_hx, kEwThreads);
         mbar_init(bar_sready, kEwThreads);
+        mbar_init(bar_ystaged, kEwThreads);
+        mbar_init(bar_vec, 1);
+        mbar_init(bar_ldx, 1);
+        mbar_init(bar_ldx + 1, 1);
         fence_mbar_init();
         *ticket_slot = atomicAdd(prm.ws_ctrl, 1);
     }
@@ -315,51 +328,18 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     const int ticket = *ticket_slot;
     const Range rg = make_range(ticket, prm.nslots, prm.units, nc);
 
-    if (warp == kCtlWarp) {
+    auto coords = [&](const Item& it, int& bi, int& h, int& g) {
+        bi = (int)prm.fH.div((uint32_t)it.chain);
+        h = it.chain - bi * H;
+        g = (int)prm.fHG.div((uint32_t)h);
+    };
+    auto stage = [&](int idx) { return smem + kOffStage + (idx & 1) * kStageBytes; };
+
+    if (warp == kMmaWarp) {
         // ------------------------------------------------------------------
-        // control warp (one thread): TMA and MMA issue
+        // MMA warp (one thread): waits and tcgen05.mma issue only
         // ------------------------------------------------------------------
         if (lane == 0 && rg.count > 0) {
-            prefetch_tensormap(&tmX);
-            prefetch_tensormap(&tmB);
-            prefetch_tensormap(&tmC);
-            auto stage = [&](int idx) { return smem + kOffStage + (idx & 1) * kStageBytes; };
-            auto coords = [&](const Item& it, int& bi, int& h, int& g) {
-                bi = (int)prm.fH.div((uint32_t)it.chain);
-                h = it.chain - bi * H;
-                g = (int)prm.fHG.div((uint32_t)h);
-            };
-            auto issue_loads = [&](int idx) {
-                const Item it = item_at(rg, idx, nc, prm.fnc);
-                int bi, h, g;
-                coords(it, bi, h, g);
-                const int t0 = it.chunk * kQ;
-                uint8_t* st = stage(idx);
-                uint64_t* bar = bar_ld + (idx & 1);
-                mbar_arrive_expect_tx(bar, kBytesLoad);
-                tma_load_3d(st + kStB, &tmB, g * kN, t0, bi, bar);
-                tma_load_3d(st + kStB + kTileHalf, &tmB, g * kN + 64, t0, bi, bar);
-                tma_load_3d(st + kStC, &tmC, g * kN, t0, bi, bar);
-                tma_load_3d(st + kStC + kTileHalf, &tmC, g * kN + 64, t0, bi, bar);
-                tma_load_3d(st + kStX, &tmX, h * kP, t0, bi, bar);
-            };
-            auto prefetch_l2 = [&](int idx) {
-                const Item it = item_at(rg, idx, nc, prm.fnc);
-                int bi, h, g;
-                coords(it, bi, h, g);
-                const int t0 = it.chunk * kQ;
-                tma_prefetch_l2_3d(&tmB, g * kN, t0, bi);
-                tma_prefetch_l2_3d(&tmB, g * kN + 64, t0, bi);
-                tma_prefetch_l2_3d(&tmC, g * kN, t0, bi);
-                tma_prefetch_l2_3d(&tmC, g * kN + 64, t0, bi);
-                tma_prefetch_l2_3d(&tmX, h * kP, t0, bi);
-            };
-            auto wait_ld = [&](int idx) {
-                mbar_wait_bounded(bar_ld + (idx & 1), (uint32_t)(idx >> 1) & 1u, kWaitNs, aborted, prm.status);
-            };
-            // Matrix descriptors of K-step 0 for every operand; K-step k adds
-            // a constant to the start-address field (no carry: shared-memory
-            // addresses stay below 256 KB).
             // Stage 1 is kStageBytes after stage 0, so its descriptors are
             // stage 0's plus a constant; selected without indexing.
             const uint32_t st0 = smem_u32(smem + kOffStage);
@@ -369,6 +349,9 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             constexpr uint64_t kStageStep = (uint64_t)(kStageBytes >> 4);
             auto kstep_k = [](int k) -> uint64_t { return (uint64_t)(((k >> 2) * kTileHalf + (k & 3) * 32u) >> 4); };
             auto kstep_mn = [](int k) -> uint64_t { return (uint64_t)((k * 2048u) >> 4); };
+            auto wait_ld = [&](int idx) {
+                mbar_wait_bounded(bar_ld + (idx & 1), (uint32_t)(idx >> 1) & 1u, kWaitNs, aborted, prm.status);
+            };
             auto mma_G = [&](int idx) {   // G = C B^T into buffer idx & 1
                 const uint64_t so = (idx & 1) ? kStageStep : 0;
                 const uint64_t dC = dCk0 + so, dB = dBk0 + so;
@@ -378,9 +361,6 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 umma_commit(bar_m1);
             };
 
-            issue_loads(0);
-            if (rg.count > 1) issue_loads(1);
-            if (rg.count > 2) prefetch_l2(2);
             wait_ld(0);
             tc_fence_after_sync();
             mma_G(0);
@@ -394,11 +374,6 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 for (int k = 0; k < 8; ++k)   // Yo = C h^T
                     umma_bf16(tmem + kColYo, dC + kstep_k(k), dHXmn + kstep_mn(k), kIdYo, k > 0);
                 umma_commit(bar_m3);
-                if (idx + 1 < rg.count) {
-                    wait_ld(idx + 1);
-                    tc_fence_after_sync();
-                    mma_G(idx + 1);
-                }
                 mbar_wait_bounded(bar_sready, ph, kWaitNs, aborted, prm.status);
                 tc_fence_after_sync();
 #pragma unroll
@@ -410,9 +385,165 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 for (int k = 0; k < 8; ++k)   // Yd = M X
                     umma_bf16(tmem + kColYd, dMk + kstep_k(k), dXmn + kstep_mn(k), kIdYd, k > 0);
                 umma_commit(bar_m2);
+                // the next chunk's C B^T last: its loads may still be landing
+                if (idx + 1 < rg.count) {
+                    wait_ld(idx + 1);
+                    tc_fence_after_sync();
+                    mma_G(idx + 1);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == kProdWarp) {
+        // ------------------------------------------------------------------
+        // producer warp (one thread): TMA loads, L2 prefetches and y stores
+        // ------------------------------------------------------------------
+        if (lane == 0 && rg.count > 0) {
+            // B and C of item idx into its stage (G = C B^T needs only these)
+            auto issue_bc = [&](int idx) {
+                const Item it = item_at(rg, idx, nc, prm.fnc);
+                int bi, h, g;
+                coords(it, bi, h, g);
+                const int t0 = it.chunk * kQ;
+                uint8_t* st = stage(idx);
+                uint64_t* bar = bar_ld + (idx & 1);
+                mbar_arrive_expect_tx(bar, kBytesBC);
+                tma_load_3d(st + kStB, &tmB, g * kN, t0, bi, bar);
+                tma_load_3d(st + kStB + kTileHalf, &tmB, g * kN + 64, t0, bi, bar);
+                tma_load_3d(st + kStC, &tmC, g * kN, t0, bi, bar);
+                tma_load_3d(st + kStC + kTileHalf, &tmC, g * kN + 64, t0, bi, bar);
+            };
+            // X of item idx into its stage (the buffer that held y of item idx - 2)
+            auto issue_x = [&](int idx) {
+                const Item it = item_at(rg, idx, nc, prm.fnc);
+                int bi, h, g;
+                coords(it, bi, h, g);
+                uint64_t* bar = bar_ldx + (idx & 1);
+                mbar_arrive_expect_tx(bar, kBytesX);
+                tma_load_3d(stage(idx) + kStX, &tmX, h * kP, it.chunk * kQ, bi, bar);
+            };
+            auto prefetch_l2 = [&](int idx) {
+                const Item it = item_at(rg, idx, nc, prm.fnc);
+                int bi, h, g;
+                coords(it, bi, h, g);
+                const int t0 = it.chunk * kQ;
+                tma_prefetch_l2_3d(&tmB, g * kN, t0, bi);
+                tma_prefetch_l2_3d(&tmB, g * kN + 64, t0, bi);
+                tma_prefetch_l2_3d(&tmC, g * kN, t0, bi);
+                tma_prefetch_l2_3d(&tmC, g * kN + 64, t0, bi);
+                tma_prefetch_l2_3d(&tmX, h * kP, t0, bi);
+            };
+            prefetch_tensormap(&tmX);
+            prefetch_tensormap(&tmB);
+            prefetch_tensormap(&tmC);
+            prefetch_tensormap(&tmY);
+            issue_bc(0);
+            issue_x(0);
+            if (rg.count > 1) {
+                issue_bc(1);
+                issue_x(1);
+            }
+            if (rg.count > 2) prefetch_l2(2);
+            for (int idx = 0; idx < rg.count; ++idx) {
+                const uint32_t ph = (uint32_t)idx & 1u;
+                // all MMAs of item idx are done: its B and C buffers are free
                 mbar_wait_bounded(bar_m2, ph, kWaitNs, aborted, prm.status);
-                if (idx + 2 < rg.count) issue_loads(idx + 2);
+                if (idx + 2 < rg.count) issue_bc(idx + 2);
+                // y of item idx is staged in its X buffer: store it, then
+                // reload the buffer once the store has read it
+                mbar_wait_bounded(bar_ystaged, ph, kWaitNs, aborted, prm.status);
+                const Item it = item_at(rg, idx, nc, prm.fnc);
+                int bi, h, g;
+                coords(it, bi, h, g);
+                tma_store_3d(&tmY, stage(idx) + kStX, h * kP, it.chunk * kQ, bi);
+                bulk_commit_group();
+                bulk_wait_group_read0();
+                if (idx + 2 < rg.count) issue_x(idx + 2);
                 if (idx + 3 < rg.count) prefetch_l2(idx + 3);
+            }
+            bulk_wait_group0();   // all y stores complete before the CTA exits
+        }
+        __syncwarp();
+    } else if (warp == kVecWarp) {
+        // ------------------------------------------------------------------
+        // vector warp: dt, cumulative decay and the off-diagonal column
+        // factors of each chunk, published one chunk ahead.  The strided dt
+        // loads of item idx + 1 are issued before item idx is computed, so
+        // their latency is hidden behind a whole chunk.
+        // ------------------------------------------------------------------
+        struct DtIn {
+            float a2, bias;
+            int nvalid;   // tokens 4*lane + k with k < nvalid lie inside the sequence
+            __nv_bfloat16 dt[4];
+        };
+        // raw inputs of item idx for tokens 4*lane .. 4*lane+3
+        auto load_dt = [&](int idx) {
+            DtIn in;
+            const Item it = item_at(rg, idx, nc, prm.fnc);
+            int bi, h, g;
+            coords(it, bi, h, g);
+            in.a2 = prm.A[h] * 1.4426950408889634f;   // A * log2(e)
+            in.bias = prm.dt_bias ? prm.dt_bias[h] : 0.0f;
+            const __nv_bfloat16* dp = prm.dt_raw + (size_t)bi * L * H + h;
+            const int t0 = it.chunk * kQ + lane * 4;
+            in.nvalid = L - t0;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) in.dt[k] = k < in.nvalid ? dp[(size_t)(t0 + k) * H] : __float2bfloat16_rn(0.0f);
+            return in;
+        };
+        // dt (0 past the sequence end), the inclusive cumulative log2 decay
+        // (local sums, then a warp scan) and the off-diagonal column factor
+        // 2^(cl_e - cl) dt, e the last token of the 32-token block.
+        float vcl[4], vdt[4], vv[4];
+        auto compute_vecs = [&](const DtIn& in) {
+            float run = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                vdt[k] = k < in.nvalid ? softplus_fast(__bfloat162float(in.dt[k]) + in.bias) : 0.0f;
+                run += vdt[k] * in.a2;
+                vcl[k] = run;
+            }
+            float incl = run;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            const float excl = incl - run;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) vcl[k] += excl;
+            const float cl_e = __shfl_sync(0xffffffffu, vcl[3], lane | 7);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) vv[k] = ex2_approx(cl_e - vcl[k]) * vdt[k];
+        };
+        auto publish_vecs = [&](int idx) {
+            const ChunkVecs cv = chunk_vecs(smem, idx & 1);
+            reinterpret_cast<float4*>(cv.cl)[lane] = make_float4(vcl[0], vcl[1], vcl[2], vcl[3]);
+            reinterpret_cast<float4*>(cv.dt)[lane] = make_float4(vdt[0], vdt[1], vdt[2], vdt[3]);
+            reinterpret_cast<float4*>(cv.v)[lane] = make_float4(vv[0], vv[1], vv[2], vv[3]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_vec);
+        };
+
+        if (rg.count > 0) {
+            DtIn in = load_dt(0);
+            compute_vecs(in);
+            publish_vecs(0);
+            if (rg.count > 1) {
+                in = load_dt(1);
+                compute_vecs(in);
+            }
+            if (rg.count > 2) in = load_dt(2);
+            for (int idx = 0; idx + 1 < rg.count; ++idx) {
+                // the elementwise warps finished reading vectors idx - 1
+                // before arriving for MMA2(idx), so buffer (idx + 1) & 1 is free
+                if (lane == 0) mbar_wait_bounded(bar_m2, (uint32_t)idx & 1u, kWaitNs, aborted, prm.status);
+                __syncwarp();
+                publish_vecs(idx + 1);
+                if (idx + 2 < rg.count) {
+                    compute_vecs(in);
+                    if (idx + 3 < rg.count) in = load_dt(idx + 3);
+                }
             }
         }
         __syncwarp();
@@ -425,62 +556,12 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         const int row = quad * 32 + lane;   // token row i / state column n
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const uint32_t tH = tmem + kColH + (uint32_t)quarter * 16 + lane_off;
-        // warps 1, 5, 9, 13 compute the chunk vectors (their sub-partition
-        // does not host the control warp)
-        const bool vec_warp = quad == 1;
-        const int vrow = quarter * 32 + lane;   // their token
-        float* sWs = reinterpret_cast<float*>(smem + kOffWs);
-
-        // Inputs of an item's chunk vectors for token `vrow`: raw dt,
-        // A * log2(e), dt_bias.  Loaded a chunk ahead of use.
-        // The loads are only issued here; their values are first used a
-        // chunk later, so the vector warps never wait on them.
-        struct VecIn {
-            float a, bias;
-            unsigned short dtr;   // raw bf16 bits
-            bool valid;
-        };
-        auto load_vec_in = [&](const Item& it) -> VecIn {
-            VecIn v{0.0f, 0.0f, 0, false};
-            const int t = it.chunk * kQ + vrow;
-            const int bi = (int)prm.fH.div((uint32_t)it.chain), h = it.chain - bi * H;
-            v.a = prm.A[h];
-            v.bias = prm.dt_bias ? prm.dt_bias[h] : 0.0f;
-            v.valid = t < L;
-            const unsigned short* dp = reinterpret_cast<const unsigned short*>(prm.dt_raw);
-            v.dtr = v.valid ? dp[((size_t)bi * L + t) * H + h] : (unsigned short)0;
-            return v;
-        };
-        // Chunk vectors (vector warps, one token each): dt, the inclusive
-        // cumulative log2 decay and the off-diagonal column factor.  A scan
-        // within each warp, a barrier among the four, then the prefix.
-        auto make_vecs = [&](const VecIn& in, int parity) {
-            const float dtr = __uint_as_float((uint32_t)in.dtr << 16);
-            const float dt = in.valid ? softplus_fast(dtr + in.bias) : 0.0f;
-            float a = dt * (in.a * 1.4426950408889634f);   // dt * A * log2(e)
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float v = __shfl_up_sync(0xffffffffu, a, o);
-                if (lane >= o) a += v;
-            }
-            if (lane == 31) sWs[quarter] = a;
-            named_bar_sync(kVecBarrier, 128);
-            float pre = 0.0f;
-            for (int w = 0; w < quarter; ++w) pre += sWs[w];
-            const float cl = a + pre;
-            const float cl_e = __shfl_sync(0xffffffffu, cl, 31);
-            const ChunkVecs cv = chunk_vecs(smem, parity);
-            cv.cl[vrow] = cl;
-            cv.dt[vrow] = dt;
-            cv.v[vrow] = ex2_approx(cl_e - cl) * dt;
-            named_bar_sync(kVecBarrier, 128);   // totals read before the next scan overwrites them
-        };
-
-        // Hand chunk k over to the MMA side: its G is ready (waited here, so
-        // the G barrier never runs two phases ahead), the bf16 state is in
-        // smem and the previous chunk's Yd / Yo are consumed.  The barrier
-        // also publishes chunk k's vectors to every elementwise warp.
+        // Hand chunk k over to the MMA side: its vectors are published and
+        // its G is ready (both waited here, before the arrival, so neither
+        // barrier runs two phases ahead of this side), the bf16 state is in
+        // smem and the previous chunk's Yd / Yo are consumed.
         auto hand_over = [&](int k) {
+            mbar_wait_bounded(bar_vec, (uint32_t)k & 1u, kWaitNs, aborted, prm.status);
             mbar_wait_bounded(bar_m1, (uint32_t)k & 1u, kWaitNs, aborted, prm.status);
             fence_proxy_async_smem();
             tc_fence_before_sync();
@@ -525,13 +606,6 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             hand_over(idx);
         };
 
-        VecIn vin_next{0.0f, 0.0f, 0, false};
-        if (rg.count > 0) {
-            if (vec_warp) {
-                make_vecs(load_vec_in(item_at(rg, 0, nc, prm.fnc)), 0);
-                if (rg.count > 1) vin_next = load_vec_in(item_at(rg, 1, nc, prm.fnc));
-            }
-        }
         for (int idx = 0; idx < rg.count; ++idx) {
             const uint32_t ph = (uint32_t)idx & 1u;
             const Item it = item_at(rg, idx, nc, prm.fnc);
@@ -590,7 +664,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             m_block(1);
 
             // x of this thread's row and column quarter (kept for D x)
-            mbar_wait_bounded(bar_ld + (idx & 1), (uint32_t)(idx >> 1) & 1u, kWaitNs, aborted, prm.status);
+            mbar_wait_bounded(bar_ldx + (idx & 1), (uint32_t)(idx >> 1) & 1u, kWaitNs, aborted, prm.status);
             uint4 xraw[2];
 #pragma unroll
             for (int q = 0; q < 2; ++q)
@@ -630,11 +704,6 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             tc_fence_before_sync();
             mbar_arrive(bar_mready);
 
-            // the next chunk's vectors while the tensor cores run
-            if (vec_warp && idx + 1 < rg.count) {
-                make_vecs(vin_next, (idx + 1) & 1);
-                if (idx + 2 < rg.count) vin_next = load_vec_in(item_at(rg, idx + 2, nc, prm.fnc));
-            }
 
             mbar_wait_bounded(bar_m2, ph, kWaitNs, aborted, prm.status);
             tc_fence_after_sync();
@@ -680,15 +749,14 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                     ypk[q] = pack_bf16x8(o);
                 }
             }
+            // y tile into this chunk's X buffer (M X, its last reader, is done;
+            // the x values are in registers); the control warp stores it by TMA
+#pragma unroll
+            for (int q = 0; q < 2; ++q)
+                *reinterpret_cast<uint4*>(st + kStX + sw128(row, quarter * 2 + q)) = ypk[q];
+            fence_proxy_async_smem();
+            mbar_arrive(bar_ystaged);
             if (idx + 1 < rg.count && !it.seg_end) hand_over(idx + 1);
-            {
-                const int t = it.chunk * kQ + row;
-                if (t < L) {
-                    __nv_bfloat16* yrow = prm.y + (((size_t)bi * L + t) * H + h) * kP + quarter * 16;
-                    __stcs(reinterpret_cast<uint4*>(yrow), ypk[0]);
-                    __stcs(reinterpret_cast<uint4*>(yrow + 8), ypk[1]);
-                }
-            }
         }
     }
 
@@ -765,6 +833,8 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t s)
     if ((e = make_map(&tmX, a.x, (uint64_t)a.H * a.P, a.L, a.b, rb)) != cudaSuccess) return e;
     if ((e = make_map(&tmB, a.B, (uint64_t)a.G * a.N, a.L, a.b, rb)) != cudaSuccess) return e;
     if ((e = make_map(&tmC, a.C, (uint64_t)a.G * a.N, a.L, a.b, rb)) != cudaSuccess) return e;
+    CUtensorMap tmY;
+    if ((e = make_map(&tmY, a.y, (uint64_t)a.H * a.P, a.L, a.b, (uint64_t)a.H * a.P * 2)) != cudaSuccess) return e;
     e = cudaFuncSetAttribute(chunk_scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     const int slots = tc_slots(a);
@@ -792,7 +862,7 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t s)
     prm.ws_ctrl = static_cast<int*>(a.workspace);
     prm.ws_states = reinterpret_cast<float*>(static_cast<uint8_t*>(a.workspace) + ctrl);
     prm.status = a.status;
-    chunk_scan_tc_kernel<<<slots, kThreads, kSmemBytes, s>>>(tmX, tmB, tmC, prm);
+    chunk_scan_tc_kernel<<<slots, kThreads, kSmemBytes, s>>>(tmX, tmB, tmC, tmY, prm);
     return cudaGetLastError();
 }
 

@@ -99,6 +99,24 @@ __device__ inline void tma_load_3d(void* smem_dst, const CUtensorMap* map, int c
         : "memory");
 }
 
+// TMA: tiled tensor store from shared memory (bulk-group completion).
+// Rows outside the tensor are not written.
+__device__ inline void tma_store_3d(const CUtensorMap* map, const void* smem_src, int c0, int c1, int c2)
+{
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+
+__device__ inline void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Wait until every committed bulk store has finished reading shared memory.
+__device__ inline void bulk_wait_group_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+// Wait until every committed bulk store has completed.
+__device__ inline void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Prefetch a tile of a tensor into L2 (no shared memory, no completion).
 __device__ inline void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2)
 {
