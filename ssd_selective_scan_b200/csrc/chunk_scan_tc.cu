@@ -80,12 +80,12 @@ constexpr int kEwBarrier = 1;    // named barrier among the elementwise warps
 constexpr int kStageBytes = 81920;    // B [128 tok][128 n], C [128 tok][128 n], X [128 tok][64 p]
 constexpr int kOffStage = 0;          // 2 stages
 constexpr int kStB = 0, kStC = 32768, kStX = 65536;
-constexpr int kOffM = 2 * kStageBytes;          // masked tile M [128 i][128 j]
-constexpr int kOffHX = kOffM + 32768;           // bf16 state [128 n][64 p], then w o X [128 tok][64 p]
-constexpr int kOffVec = kOffHX + 16384;         // per chunk parity: cl, dt, v  (3 x float[128]) x 2
-constexpr int kOffWs = kOffVec + 3072;          // float[8] scan totals
-constexpr int kOffBar = kOffWs + 32;            // mbarriers
-constexpr int kOffMisc = kOffBar + 96;          // tmem slot, abort flag, ticket (12 mbarriers above)
+constexpr int kOffHB = 2 * kStageBytes;         // bf16 state entering the item [128 n][64 p]
+constexpr int kOffWX = kOffHB + 16384;          // w o X [128 tok][64 p]
+constexpr int kOffVec = kOffWX + 16384;         // per chunk parity: cl, dt, v  (3 x float[128]) x 2
+constexpr int kOffBar = kOffVec + 3072;         // mbarriers
+constexpr int kNumBars = 13;
+constexpr int kOffMisc = kOffBar + 8 * kNumBars;   // tmem slot, abort flag, ticket
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
 
 constexpr uint32_t kTileHalf = 16384;
@@ -93,15 +93,16 @@ constexpr uint32_t kBytesBC = 4 * 16384;   // B and C, two halves each
 constexpr uint32_t kBytesX = 16384;
 
 // TMEM columns
-constexpr uint32_t kColG = 0;     // G, two buffers [0,128) and [128,256)
-constexpr uint32_t kColYd = 256;  // Yd [256,320)
-constexpr uint32_t kColYo = 320;  // Yo [320,384)
+constexpr uint32_t kColG = 0;     // G [0,128)
+constexpr uint32_t kColM = 128;   // masked tile M, bf16 pairs along j [128,192)
+constexpr uint32_t kColYd = 192;  // Yd [192,256)
+constexpr uint32_t kColYo = 256;  // Yo, two buffers [256,320) and [320,384)
 constexpr uint32_t kColH = 384;   // fp32 state [384,448): lane n, column p
 
 // instruction descriptors
 constexpr uint32_t kIdG = umma_idesc_bf16(128, 128, false, false);   // C (K-maj) x B (K-maj)
 constexpr uint32_t kIdYo = umma_idesc_bf16(128, 64, false, true);    // C (K-maj) x h (MN-maj)
-constexpr uint32_t kIdYd = umma_idesc_bf16(128, 64, false, true);    // M (K-maj) x X (MN-maj)
+constexpr uint32_t kIdYd = umma_idesc_bf16(128, 64, false, true);    // M (TMEM, K-maj) x X (MN-maj)
 constexpr uint32_t kIdS = umma_idesc_bf16(128, 64, true, true);      // B^T (MN-maj) x wX (MN-maj)
 
 // Workspace: control block (ticket, hand-off flags), then one published
@@ -285,22 +286,23 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(smem + kOffBar);   // [2]: stage's B and C landed
-    uint64_t* bar_m1 = bar_ld + 2;      // G ready
-    uint64_t* bar_m3 = bar_ld + 3;      // Yo ready (bf16 state read)
-    uint64_t* bar_m2 = bar_ld + 4;      // Yd and the state update done
-    uint64_t* bar_mready = bar_ld + 5;  // masked tile M ready (elementwise warps)
-    uint64_t* bar_hx = bar_ld + 6;      // bf16 state in smem, Yd / Yo consumed (elementwise warps)
-    uint64_t* bar_sready = bar_ld + 7;  // w o X and decayed state ready (elementwise warps)
-    uint64_t* bar_ystaged = bar_ld + 8; // y tile staged in the chunk's X buffer (elementwise warps)
-    uint64_t* bar_vec = bar_ld + 9;     // chunk vectors published (producer warp)
-    uint64_t* bar_ldx = bar_ld + 10;    // [2]: stage's X landed
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+    uint64_t* bar_ld = bars + 0;        // [2]: stage's B and C landed (TMA)
+    uint64_t* bar_m1 = bars + 2;        // G ready
+    uint64_t* bar_m2 = bars + 3;        // Yd ready (all MMAs of the item done)
+    uint64_t* bar_sready = bars + 4;    // bf16 state, w o X and decayed state ready (elementwise warps)
+    uint64_t* bar_mready = bars + 5;    // masked tile M in TMEM; G, Yd, Yo of earlier items read (elementwise warps)
+    uint64_t* bar_vec = bars + 6;       // chunk vectors published (vector warp)
+    uint64_t* bar_ldx = bars + 7;       // [2]: stage's X landed (TMA)
+    // Per stage, so that the producer warp, which nothing else waits for,
+    // can never fall two phases behind them:
+    uint64_t* bar_ystaged = bars + 9;   // [2]: y tile staged in the stage's X buffer (elementwise warps)
+    uint64_t* bar_m4 = bars + 11;       // [2]: C h^T and the state update done; stage's B and C free
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* aborted = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
     int* ticket_slot = reinterpret_cast<int*>(smem + kOffMisc + 8);
-    uint8_t* sM = smem + kOffM;
-    uint8_t* sHX = smem + kOffHX;  // bf16 state, then w o X
-    const uint32_t aM = smem_u32(sM), aHX = smem_u32(sHX);
+    uint8_t* sHB = smem + kOffHB;
+    uint8_t* sWX = smem + kOffWX;
     const int H = prm.H, nc = prm.nc, L = prm.L;
 
     if (tid == 0) {
@@ -308,15 +310,16 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         mbar_init(bar_ld, 1);
         mbar_init(bar_ld + 1, 1);
         mbar_init(bar_m1, 1);
-        mbar_init(bar_m3, 1);
         mbar_init(bar_m2, 1);
-        mbar_init(bar_mready, kEwThreads);
-        mbar_init(bar_hx, kEwThreads);
         mbar_init(bar_sready, kEwThreads);
-        mbar_init(bar_ystaged, kEwThreads);
+        mbar_init(bar_mready, kEwThreads);
         mbar_init(bar_vec, 1);
         mbar_init(bar_ldx, 1);
         mbar_init(bar_ldx + 1, 1);
+        mbar_init(bar_ystaged, kEwThreads);
+        mbar_init(bar_ystaged + 1, kEwThreads);
+        mbar_init(bar_m4, 1);
+        mbar_init(bar_m4 + 1, 1);
         fence_mbar_init();
         *ticket_slot = atomicAdd(prm.ws_ctrl, 1);
     }
@@ -345,19 +348,18 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             const uint32_t st0 = smem_u32(smem + kOffStage);
             const uint64_t dCk0 = desc_kmajor(st0 + kStC, 0), dBk0 = desc_kmajor(st0 + kStB, 0);
             const uint64_t dBmn0 = desc_mnmajor(st0 + kStB, 0), dXmn0 = desc_mnmajor(st0 + kStX, 0);
-            const uint64_t dMk = desc_kmajor(aM, 0), dHXmn = desc_mnmajor(aHX, 0);
+            const uint64_t dHB = desc_mnmajor(smem_u32(sHB), 0), dWX = desc_mnmajor(smem_u32(sWX), 0);
             constexpr uint64_t kStageStep = (uint64_t)(kStageBytes >> 4);
             auto kstep_k = [](int k) -> uint64_t { return (uint64_t)(((k >> 2) * kTileHalf + (k & 3) * 32u) >> 4); };
             auto kstep_mn = [](int k) -> uint64_t { return (uint64_t)((k * 2048u) >> 4); };
             auto wait_ld = [&](int idx) {
                 mbar_wait_bounded(bar_ld + (idx & 1), (uint32_t)(idx >> 1) & 1u, kWaitNs, aborted, prm.status);
             };
-            auto mma_G = [&](int idx) {   // G = C B^T into buffer idx & 1
+            auto mma_G = [&](int idx) {   // G = C B^T
                 const uint64_t so = (idx & 1) ? kStageStep : 0;
                 const uint64_t dC = dCk0 + so, dB = dBk0 + so;
-                const uint32_t d = tmem + kColG + (uint32_t)(idx & 1) * 128u;
 #pragma unroll
-                for (int k = 0; k < 8; ++k) umma_bf16(d, dC + kstep_k(k), dB + kstep_k(k), kIdG, k > 0);
+                for (int k = 0; k < 8; ++k) umma_bf16(tmem + kColG, dC + kstep_k(k), dB + kstep_k(k), kIdG, k > 0);
                 umma_commit(bar_m1);
             };
 
@@ -368,25 +370,23 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 const uint32_t ph = (uint32_t)idx & 1u;
                 const uint64_t so = (idx & 1) ? kStageStep : 0;
                 const uint64_t dC = dCk0 + so, dBmn = dBmn0 + so, dXmn = dXmn0 + so;
-                mbar_wait_bounded(bar_hx, ph, kWaitNs, aborted, prm.status);
-                tc_fence_after_sync();
-#pragma unroll
-                for (int k = 0; k < 8; ++k)   // Yo = C h^T
-                    umma_bf16(tmem + kColYo, dC + kstep_k(k), dHXmn + kstep_mn(k), kIdYo, k > 0);
-                umma_commit(bar_m3);
                 mbar_wait_bounded(bar_sready, ph, kWaitNs, aborted, prm.status);
                 tc_fence_after_sync();
+                const uint32_t dYo = tmem + kColYo + (uint32_t)(idx & 1) * 64u;
+#pragma unroll
+                for (int k = 0; k < 8; ++k)   // Yo = C h^T
+                    umma_bf16(dYo, dC + kstep_k(k), dHB + kstep_mn(k), kIdYo, k > 0);
 #pragma unroll
                 for (int k = 0; k < 8; ++k)   // h += B^T (w o X)   (h already decayed)
-                    umma_bf16(tmem + kColH, dBmn + kstep_mn(k), dHXmn + kstep_mn(k), kIdS, 1);
+                    umma_bf16(tmem + kColH, dBmn + kstep_mn(k), dWX + kstep_mn(k), kIdS, 1);
+                umma_commit(bar_m4 + (idx & 1));
                 mbar_wait_bounded(bar_mready, ph, kWaitNs, aborted, prm.status);
                 tc_fence_after_sync();
 #pragma unroll
-                for (int k = 0; k < 8; ++k)   // Yd = M X
-                    umma_bf16(tmem + kColYd, dMk + kstep_k(k), dXmn + kstep_mn(k), kIdYd, k > 0);
+                for (int k = 0; k < 8; ++k)   // Yd = M X, M from TMEM
+                    umma_bf16_tmem_a(tmem + kColYd, tmem + kColM + (uint32_t)k * 8u, dXmn + kstep_mn(k), kIdYd, k > 0);
                 umma_commit(bar_m2);
-                // the next chunk's C B^T last: its loads may still be landing
-                if (idx + 1 < rg.count) {
+                if (idx + 1 < rg.count) {   // the next item's C B^T (G was read: mready)
                     wait_ld(idx + 1);
                     tc_fence_after_sync();
                     mma_G(idx + 1);
@@ -445,13 +445,13 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             }
             if (rg.count > 2) prefetch_l2(2);
             for (int idx = 0; idx < rg.count; ++idx) {
-                const uint32_t ph = (uint32_t)idx & 1u;
-                // all MMAs of item idx are done: its B and C buffers are free
-                mbar_wait_bounded(bar_m2, ph, kWaitNs, aborted, prm.status);
+                const uint32_t sph = (uint32_t)(idx >> 1) & 1u;   // per-stage barrier parity
+                // the state update, the last MMA reading B and C of item idx, is done
+                mbar_wait_bounded(bar_m4 + (idx & 1), sph, kWaitNs, aborted, prm.status);
                 if (idx + 2 < rg.count) issue_bc(idx + 2);
                 // y of item idx is staged in its X buffer: store it, then
                 // reload the buffer once the store has read it
-                mbar_wait_bounded(bar_ystaged, ph, kWaitNs, aborted, prm.status);
+                mbar_wait_bounded(bar_ystaged + (idx & 1), sph, kWaitNs, aborted, prm.status);
                 const Item it = item_at(rg, idx, nc, prm.fnc);
                 int bi, h, g;
                 coords(it, bi, h, g);
@@ -535,9 +535,11 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             }
             if (rg.count > 2) in = load_dt(2);
             for (int idx = 0; idx + 1 < rg.count; ++idx) {
-                // the elementwise warps finished reading vectors idx - 1
-                // before arriving for MMA2(idx), so buffer (idx + 1) & 1 is free
-                if (lane == 0) mbar_wait_bounded(bar_m2, (uint32_t)idx & 1u, kWaitNs, aborted, prm.status);
+                // The elementwise warps waited for vectors idx before arriving
+                // for item idx's state products, and read vectors idx - 1 only
+                // before the masked tile of item idx - 1 was ready (earlier
+                // still), so buffer (idx + 1) & 1 is free.
+                if (lane == 0) mbar_wait_bounded(bar_sready, (uint32_t)idx & 1u, kWaitNs, aborted, prm.status);
                 __syncwarp();
                 publish_vecs(idx + 1);
                 if (idx + 2 < rg.count) {
@@ -554,22 +556,13 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         const int quad = warp & 3;          // TMEM lane quadrant
         const int quarter = warp >> 2;      // column quarter
         const int row = quad * 32 + lane;   // token row i / state column n
+        const int p0 = quarter * 16;        // this thread's 16 columns p
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const uint32_t tH = tmem + kColH + (uint32_t)quarter * 16 + lane_off;
-        // Hand chunk k over to the MMA side: its vectors are published and
-        // its G is ready (both waited here, before the arrival, so neither
-        // barrier runs two phases ahead of this side), the bf16 state is in
-        // smem and the previous chunk's Yd / Yo are consumed.
-        auto hand_over = [&](int k) {
-            mbar_wait_bounded(bar_vec, (uint32_t)k & 1u, kWaitNs, aborted, prm.status);
-            mbar_wait_bounded(bar_m1, (uint32_t)k & 1u, kWaitNs, aborted, prm.status);
-            fence_proxy_async_smem();
-            tc_fence_before_sync();
-            named_bar_sync(kEwBarrier, kEwThreads);
-            mbar_arrive(bar_hx);
-        };
-        // start of a segment: fp32 state into TMEM, bf16 copy into smem
-        auto begin_segment = [&](const Item& it, int idx) {
+        const uint32_t tH = tmem + kColH + (uint32_t)p0 + lane_off;
+
+        // state entering a segment: the initial state, the predecessor
+        // CTA's published state (a dependent segment), or zero
+        auto segment_state = [&](const Item& it, float (&hv)[16]) {
             const int bi = (int)prm.fH.div((uint32_t)it.chain), h = it.chain - bi * H;
             const float* src = nullptr;
             bool cg = false;
@@ -591,133 +584,172 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             } else if (prm.init_state) {
                 src = prm.init_state + ((size_t)bi * H + h) * (size_t)(kP * kN);
             }
-            const int p0 = quarter * 16;
-            float hv[16];
 #pragma unroll
             for (int p = 0; p < 16; ++p) {
                 const float* q = src + (size_t)(p0 + p) * kN + row;
                 hv[p] = src ? (cg ? __ldcg(q) : *q) : 0.0f;
             }
-            tmem_st16(tH, hv);
-#pragma unroll
-            for (int q = 0; q < 2; ++q)
-                *reinterpret_cast<uint4*>(sHX + sw128(row, (p0 >> 3) + q)) = pack_bf16x8(&hv[q * 8]);
-            tmem_wait_st();
-            hand_over(idx);
         };
 
+        // y of item j = Yd + 2^cl Yo (token row `row`, this quarter's p; D x
+        // is in Yd through M's diagonal), written over x in the item's X
+        // buffer for the producer's TMA store.  M X of item j (the X
+        // buffer's last reader) is done once bar_m2 has completed for it.
+        auto y_epilogue = [&](int j, float cl_i) {
+            mbar_wait_bounded(bar_m2, (uint32_t)j & 1u, kWaitNs, aborted, prm.status);
+            tc_fence_after_sync();
+            uint8_t* xs = stage(j) + kStX;
+            const float sc = ex2_approx(cl_i);
+            float yd[16], yo[16];
+            tmem_ld16(tmem + kColYd + lane_off + (uint32_t)p0, yd);
+            tmem_ld16(tmem + kColYo + (uint32_t)(j & 1) * 64u + lane_off + (uint32_t)p0, yo);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                float o[8];
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    const float2 r = fma2(make_float2(sc, sc), make_float2(yo[q * 8 + e], yo[q * 8 + e + 1]),
+                                          make_float2(yd[q * 8 + e], yd[q * 8 + e + 1]));
+                    o[e] = r.x;
+                    o[e + 1] = r.y;
+                }
+                *reinterpret_cast<uint4*>(xs + sw128(row, quarter * 2 + q)) = pack_bf16x8(o);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(bar_ystaged + (j & 1));
+        };
+
+        float prev_cl_i = 0.0f;
         for (int idx = 0; idx < rg.count; ++idx) {
-            const uint32_t ph = (uint32_t)idx & 1u;
             const Item it = item_at(rg, idx, nc, prm.fnc);
             const int bi = (int)prm.fH.div((uint32_t)it.chain), h = it.chain - bi * H;
             const float Dh = prm.D ? prm.D[h] : 0.0f;
-            uint8_t* st = smem + kOffStage + (idx & 1) * kStageBytes;
-            if (it.seg_start) begin_segment(it, idx);
-            tc_fence_after_sync();
+            uint8_t* st = stage(idx);
 
-            const ChunkVecs cv = chunk_vecs(smem, (int)ph);
+            // 1. the state entering item idx (fp32, state column n = row)
+            float hv[16];
+            if (it.seg_start) {
+                segment_state(it, hv);
+            } else {
+                // the previous item's C h^T and state update are done, so
+                // the state, its bf16 copy and w o X buffers are free
+                mbar_wait_bounded(bar_m4 + ((idx - 1) & 1), (uint32_t)((idx - 1) >> 1) & 1u, kWaitNs, aborted,
+                                  prm.status);
+                tc_fence_after_sync();
+                tmem_ld16(tH, hv);
+                tmem_wait_ld();
+            }
+            // 2. its bf16 copy for C h^T
+#pragma unroll
+            for (int q = 0; q < 2; ++q)
+                *reinterpret_cast<uint4*>(sHB + sw128(row, (p0 >> 3) + q)) = pack_bf16x8(&hv[q * 8]);
+
+            // 3. the decayed state back into TMEM (the state product
+            //    accumulates onto it) and w o X, w_j = 2^(cl_last - cl_j) dt_j
+            mbar_wait_bounded(bar_vec, (uint32_t)idx & 1u, kWaitNs, aborted, prm.status);
+            const ChunkVecs cv = chunk_vecs(smem, idx & 1);
             const float cl_i = cv.cl[row];
             const float cl_last = cv.cl[kQ - 1];
+            {
+                const float decay = ex2_approx(cl_last);
+#pragma unroll
+                for (int p = 0; p < 16; p += 2) {
+                    const float2 r = mul2(make_float2(hv[p], hv[p + 1]), make_float2(decay, decay));
+                    hv[p] = r.x;
+                    hv[p + 1] = r.y;
+                }
+                tmem_st16(tH, hv);
+            }
+            mbar_wait_bounded(bar_ldx + (idx & 1), (uint32_t)(idx >> 1) & 1u, kWaitNs, aborted, prm.status);
+            {
+                const float wj = ex2_approx(cl_last - cl_i) * cv.dt[row];
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    float v[8];
+                    unpack_bf16x8(*reinterpret_cast<const uint4*>(st + kStX + sw128(row, quarter * 2 + q)), v);
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) {
+                        const float2 r = mul2(make_float2(v[e], v[e + 1]), make_float2(wj, wj));
+                        v[e] = r.x;
+                        v[e + 1] = r.y;
+                    }
+                    *reinterpret_cast<uint4*>(sWX + sw128(row, quarter * 2 + q)) = pack_bf16x8(v);
+                }
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            mbar_arrive(bar_sready);   // C h^T and the state update can start
 
-            // M = G o L for row `row` (G in buffer idx & 1).  Column block jb
-            // (32 tokens) is zero above the row quadrant's diagonal block; of
-            // every other block, column quarter `quarter` takes 8 columns.
-            const uint32_t tG = tmem + kColG + (uint32_t)(idx & 1) * 128u + lane_off;
-            // Block jb (32 tokens) of the masked tile: zero above the row
-            // quadrant's diagonal block; of every other block, column quarter
-            // `quarter` takes 8 columns.
-            auto m_block = [&](int jb) {
-                const int j0 = jb * 32 + quarter * 8;
-                uint4 packed = make_uint4(0, 0, 0, 0);
-                if (jb <= quad) {
-                    float gv[8];
-                    tmem_ld8(tG + j0, gv);
-                    tmem_wait_ld();
-                    float m[8];
+            // 4. y of the previous item, whose M X ran meanwhile
+            if (idx > 0) y_epilogue(idx - 1, prev_cl_i);
+
+            // 5. the masked tile M = G o L of item idx into TMEM (bf16
+            //    pairs), the A operand of M X.  Column block jb (32 tokens)
+            //    is zero above the row quadrant's diagonal block; of every
+            //    block, column quarter `quarter` takes 8 columns.
+            mbar_wait_bounded(bar_m1, (uint32_t)idx & 1u, kWaitNs, aborted, prm.status);
+            tc_fence_after_sync();
+            {
+                float gv[4][8];
+#pragma unroll
+                for (int jb = 0; jb < 4; ++jb)
+                    if (jb <= quad) tmem_ld8(tmem + kColG + lane_off + (uint32_t)(jb * 32 + quarter * 8), gv[jb]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int jb = 0; jb < 4; ++jb) {
+                    const int j0 = jb * 32 + quarter * 8;
+                    uint32_t w[4] = {0u, 0u, 0u, 0u};
                     if (jb < quad) {
                         const float u = ex2_approx(cl_i - cv.cl[jb * 32 + 31]);
                         const float4 va = reinterpret_cast<const float4*>(cv.v + j0)[0];
                         const float4 vb = reinterpret_cast<const float4*>(cv.v + j0)[1];
                         const float vv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) m[e] = gv[e] * u * vv[e];
-                    } else {
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 uv = mul2(make_float2(u, u), make_float2(vv[2 * e], vv[2 * e + 1]));
+                            const float2 m = mul2(make_float2(gv[jb][2 * e], gv[jb][2 * e + 1]), uv);
+                            __nv_bfloat162 b2 = __floats2bfloat162_rn(m.x, m.y);
+                            w[e] = *reinterpret_cast<uint32_t*>(&b2);
+                        }
+                    } else if (jb == quad) {
                         const float4 ca = reinterpret_cast<const float4*>(cv.cl + j0)[0];
                         const float4 cb = reinterpret_cast<const float4*>(cv.cl + j0)[1];
                         const float4 da = reinterpret_cast<const float4*>(cv.dt + j0)[0];
                         const float4 db = reinterpret_cast<const float4*>(cv.dt + j0)[1];
                         const float cc[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
                         const float dd[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+                        // diagonal element: + D (so that M X includes D x)
+                        float m[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int j = j0 + e;
-                            const float v = gv[e] * ex2_approx(cl_i - cc[e]) * dd[e];
-                            m[e] = (j <= row) ? v : 0.0f;
+                        for (int e = 0; e < 8; e += 2) {
+                            const float2 f = mul2(make_float2(ex2_approx(cl_i - cc[e]), ex2_approx(cl_i - cc[e + 1])),
+                                                  make_float2(dd[e], dd[e + 1]));
+                            const float2 v = mul2(make_float2(gv[jb][e], gv[jb][e + 1]), f);
+                            m[e] = (j0 + e < row) ? v.x : (j0 + e == row ? v.x + Dh : 0.0f);
+                            m[e + 1] = (j0 + e + 1 < row) ? v.y : (j0 + e + 1 == row ? v.y + Dh : 0.0f);
+                        }
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            __nv_bfloat162 b2 = __floats2bfloat162_rn(m[2 * e], m[2 * e + 1]);
+                            w[e] = *reinterpret_cast<uint32_t*>(&b2);
                         }
                     }
-                    packed = pack_bf16x8(m);
-                }
-                *reinterpret_cast<uint4*>(sM + (j0 >> 6) * kTileHalf + sw128(row, (j0 & 63) >> 3)) = packed;
-            };
-            // first half of the masked tile while C h^T reads the bf16 state
-            m_block(0);
-            m_block(1);
-
-            // x of this thread's row and column quarter (kept for D x)
-            mbar_wait_bounded(bar_ldx + (idx & 1), (uint32_t)(idx >> 1) & 1u, kWaitNs, aborted, prm.status);
-            uint4 xraw[2];
-#pragma unroll
-            for (int q = 0; q < 2; ++q)
-                xraw[q] = *reinterpret_cast<const uint4*>(st + kStX + sw128(row, quarter * 2 + q));
-
-            // w o X over the bf16 state copy once C h^T has read it
-            mbar_wait_bounded(bar_m3, ph, kWaitNs, aborted, prm.status);
-            {
-                const float wj = ex2_approx(cl_last - cl_i) * cv.dt[row];
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    float v[8];
-                    unpack_bf16x8(xraw[q], v);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) v[e] *= wj;
-                    *reinterpret_cast<uint4*>(sHX + sw128(row, quarter * 2 + q)) = pack_bf16x8(v);
+                    tmem_st4(tmem + kColM + lane_off + (uint32_t)(j0 >> 1), w[0], w[1], w[2], w[3]);
                 }
             }
-            // decay the fp32 state in place; the chunk-state product accumulates onto it
-            {
-                const float decay = ex2_approx(cl_last);
-                float hv[16];
+            tmem_wait_st();
+            tc_fence_before_sync();
+            mbar_arrive(bar_mready);   // M X can start
+
+            // 6. end of a segment: the state leaves the chip
+            if (it.seg_end) {
+                mbar_wait_bounded(bar_m4 + (idx & 1), (uint32_t)(idx >> 1) & 1u, kWaitNs, aborted, prm.status);
+                tc_fence_after_sync();
                 tmem_ld16(tH, hv);
                 tmem_wait_ld();
-#pragma unroll
-                for (int p = 0; p < 16; ++p) hv[p] *= decay;
-                tmem_st16(tH, hv);
-                tmem_wait_st();
-            }
-            fence_proxy_async_smem();
-            tc_fence_before_sync();
-            mbar_arrive(bar_sready);   // the chunk-state product can start
-
-            m_block(2);
-            m_block(3);
-            fence_proxy_async_smem();
-            tc_fence_before_sync();
-            mbar_arrive(bar_mready);
-
-
-            mbar_wait_bounded(bar_m2, ph, kWaitNs, aborted, prm.status);
-            tc_fence_after_sync();
-            // new state: bf16 copy for the next chunk, or out at the end of a segment
-            {
-                float hv[16];
-                tmem_ld16(tH, hv);
-                tmem_wait_ld();
-                const int p0 = quarter * 16;
-                if (!it.seg_end) {
-#pragma unroll
-                    for (int q = 0; q < 2; ++q)
-                        *reinterpret_cast<uint4*>(sHX + sw128(row, (p0 >> 3) + q)) = pack_bf16x8(&hv[q * 8]);
-                } else if (it.publish) {
+                if (it.publish) {
                     float* dst = prm.ws_states + (size_t)ticket * (kP * kN);
 #pragma unroll
                     for (int p = 0; p < 16; ++p) __stcg(dst + (size_t)(p0 + p) * kN + row, hv[p]);
@@ -730,34 +762,9 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                     for (int p = 0; p < 16; ++p) dst[(size_t)(p0 + p) * kN + row] = hv[p];
                 }
             }
-            // output: y = Yd + 2^cl Yo + D x, token row `row`, p of this quarter.
-            // Yd / Yo are read and y packed first; the next chunk is then
-            // handed over so its MMAs start while the stores drain.
-            uint4 ypk[2];
-            {
-                const float sc = ex2_approx(cl_i);
-                float yd[16], yo[16];
-                tmem_ld16(tmem + kColYd + lane_off + quarter * 16, yd);
-                tmem_ld16(tmem + kColYo + lane_off + quarter * 16, yo);
-                tmem_wait_ld();
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    float xv[8], o[8];
-                    unpack_bf16x8(xraw[q], xv);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) o[e] = yd[q * 8 + e] + sc * yo[q * 8 + e] + Dh * xv[e];
-                    ypk[q] = pack_bf16x8(o);
-                }
-            }
-            // y tile into this chunk's X buffer (M X, its last reader, is done;
-            // the x values are in registers); the control warp stores it by TMA
-#pragma unroll
-            for (int q = 0; q < 2; ++q)
-                *reinterpret_cast<uint4*>(st + kStX + sw128(row, quarter * 2 + q)) = ypk[q];
-            fence_proxy_async_smem();
-            mbar_arrive(bar_ystaged);
-            if (idx + 1 < rg.count && !it.seg_end) hand_over(idx + 1);
+            prev_cl_i = cl_i;
         }
+        if (rg.count > 0) y_epilogue(rg.count - 1, prev_cl_i);
     }
 
     tc_fence_before_sync();

@@ -65,6 +65,20 @@ __device__ inline bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     return ok != 0;
 }
 
+// Non-blocking test: has the phase with the given parity completed?
+__device__ inline bool mbar_test(uint64_t* bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete, giving up after
 // limit_ns.  A CTA that gave up once (*aborted set) does not wait again, so a
 // failing kernel ends in bounded time; the give-up is reported in *status.
@@ -83,6 +97,33 @@ __device__ inline bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_
         }
     }
     return true;
+}
+
+// ---------------------------------------------------------------------------
+// Packed fp32 pair arithmetic (sm_100: one instruction for two lanes of
+// work, each rounded exactly as the scalar fp32 operation).
+// ---------------------------------------------------------------------------
+__device__ inline float2 mul2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// a * b + c
+__device__ inline float2 fma2(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
 }
 
 // ---------------------------------------------------------------------------
@@ -198,6 +239,14 @@ __device__ inline void tmem_ld16(uint32_t taddr, float (&v)[16])
 }
 
 // Whole warp: store 16 consecutive 32-bit columns of this warp's 32 lanes.
+// 4 consecutive 32-bit columns of the warp's 32 lanes
+__device__ inline void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(a), "r"(b),
+                 "r"(c), "r"(d)
+                 : "memory");
+}
+
 __device__ inline void tmem_st16(uint32_t taddr, const float (&v)[16])
 {
     asm volatile(
@@ -291,6 +340,19 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, bool a_mn_m
 }
 
 // Single thread: D[tmem] (+)= A[smem] * B[smem].
+// D (TMEM) (+)= A (TMEM, K-major: row m in lane m, two bf16 per 32-bit
+// column along K) x B (shared memory descriptor), bf16 in, fp32 out.
+__device__ inline void umma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 __device__ inline void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                  uint32_t accumulate)
 {
