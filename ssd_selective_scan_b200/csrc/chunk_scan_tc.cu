@@ -9,12 +9,14 @@
 // with dt_i = softplus(dt_raw_i + dt_bias) and cl_i = sum_{r<=i} dt_r A log2(e):
 //
 //   G      = C B^T                         (Q x Q, K = N)    tcgen05 -> TMEM
-//   M[i,j] = G[i,j] 2^(cl_i - cl_j) dt_j    (j <= i, else 0)  CUDA cores -> smem
-//   Yd     = M X                           (Q x P, K = Q)    tcgen05 -> TMEM
+//   M[i,j] = G[i,j] 2^(cl_i - cl_j) dt_j    (j < i)
+//          = G[i,i] dt_i + D                (j = i), 0 (j > i)  CUDA cores -> TMEM
+//   Yd     = M X                           (Q x P, K = Q)    tcgen05 (A from TMEM)
 //   Yo     = C h_prev^T                    (Q x P, K = N)    tcgen05 -> TMEM
 //   h      = 2^(cl_last) h_prev + B^T (w o X),  w_j = 2^(cl_last - cl_j) dt_j
 //            (the decay is applied to h in TMEM, then the product accumulates onto it)
-//   y_i    = Yd_i + 2^(cl_i) Yo_i + D x_i                    -> bf16
+//   y_i    = Yd_i + 2^(cl_i) Yo_i                            -> bf16
+// (D on M's diagonal makes M X include the skip term D x.)
 //
 // The decay mask is factored per 32-token block: for a column block J
 // strictly below row i's block, 2^(cl_i - cl_j) = 2^(cl_i - cl_e) 2^(cl_e - cl_j)
@@ -28,10 +30,12 @@
 // the next chunk's dt / cumulative decay vectors, its dt loads issued a chunk
 // earlier still.  The MMA warp only waits and issues tcgen05.mma (issue
 // blocks until the tensor core accepts the instruction, so nothing else may
-// sit on that thread); C B^T of the next chunk runs into a second TMEM buffer
-// while the elementwise warps build the current chunk's decay-masked tile.
-// The warps meet only on mbarriers, each producer at most one phase ahead of
-// its consumers.
+// sit on that thread).  Per chunk the elementwise warps first release the
+// state products (bf16 state copy, decayed state, w o X), then finish the
+// previous chunk's y while those run, then build the masked tile, after
+// which M X and the next chunk's C B^T run.  The warps meet only on
+// mbarriers, each waiter gated by what it waits for, so no barrier runs two
+// phases ahead of a waiter.
 // Elementwise warp w serves TMEM lanes 32*(w%4).. (token rows, or state
 // columns n) and column quarter w/4.  The fp32 state lives in TMEM and never
 // leaves the chip inside a sequence.
