@@ -25,6 +25,29 @@ constexpr int kConvTile = 32;   // tokens per thread
 constexpr int kGroup = 8;       // tokens loaded together
 constexpr int kCpt = 4;         // channels per thread
 
+// Packed fp32 pairs (sm_100: one instruction does two lanes of fp32 work,
+// each rounded as the scalar operation).
+__device__ inline float2 fma2(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ inline float2 mul2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
 // 4 channels of type T as one vector register group.
 template <typename T> struct Vec4;
 
@@ -38,7 +61,7 @@ template <> struct Vec4<float> {
     __device__ static void store(float* p, const float (&v)[4]) {
         *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
     }
-    __device__ static float act(float v) { return silu_f(v); }
+    __device__ static float2 act2(float2 v) { return make_float2(silu_f(v.x), silu_f(v.y)); }
 };
 
 template <> struct Vec4<__nv_bfloat16> {
@@ -53,7 +76,15 @@ template <> struct Vec4<__nv_bfloat16> {
         __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
         *reinterpret_cast<uint2*>(p) = make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
     }
-    __device__ static float act(float v) { return silu_tanh(v); }
+    // SiLU(v) = v/2 + (v/2) tanh(v/2), as in silu_tanh, on a pair
+    __device__ static float2 act2(float2 v)
+    {
+        const float2 hv = mul2(v, make_float2(0.5f, 0.5f));
+        float tx, ty;
+        asm("tanh.approx.f32 %0, %1;" : "=f"(tx) : "f"(hv.x));
+        asm("tanh.approx.f32 %0, %1;" : "=f"(ty) : "f"(hv.y));
+        return fma2(hv, make_float2(tx, ty), hv);
+    }
 };
 
 // One thread's cache block: 4 channels x K columns of type T, contiguous
@@ -177,14 +208,16 @@ conv1d_silu_kernel(const T* __restrict__ xBC, T* __restrict__ out,
         for (int u = 0; u < kGroup; ++u) {
             if (tb + u < t1) {
                 V4::decode(raw[u], hist[K - 1]);
-                float o[kCpt];
+                // the 4 channels as two fp32 pairs
+                float2 a01 = make_float2(bs[0], bs[1]), a23 = make_float2(bs[2], bs[3]);
 #pragma unroll
-                for (int c = 0; c < kCpt; ++c) {
-                    float acc = bs[c];
-#pragma unroll
-                    for (int j = 0; j < K; ++j) acc = fmaf(wt[j][c], hist[j][c], acc);
-                    o[c] = V4::act(acc);
+                for (int j = 0; j < K; ++j) {
+                    a01 = fma2(make_float2(wt[j][0], wt[j][1]), make_float2(hist[j][0], hist[j][1]), a01);
+                    a23 = fma2(make_float2(wt[j][2], wt[j][3]), make_float2(hist[j][2], hist[j][3]), a23);
                 }
+                a01 = V4::act2(a01);
+                a23 = V4::act2(a23);
+                const float o[kCpt] = {a01.x, a01.y, a23.x, a23.y};
                 V4::store(ob + (size_t)(tb + u) * conv_dim, o);
 #pragma unroll
                 for (int j = 0; j < K - 1; ++j)
