@@ -40,7 +40,7 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
-from ssd_selective_scan_b200 import synth  # noqa: E402
+from ssd_selective_scan_b200 import shard, synth  # noqa: E402
 
 METRIC = "SSD prefill scan tokens/s/layer & % roofline; decode state-update HBM GB/s"
 PREFILL = synth.CONFIGS[1]
@@ -249,8 +249,8 @@ def _events(n):
 def run_ours(args, rank, world, dev):
     import torch.distributed as dist
     s = PREFILL
-    step = PrefillStep(s, synth.config_seed(1) + rank, dev)
-    dec = DecodeStep(DECODE, synth.config_seed(4) + rank, dev)
+    step = PrefillStep(s, shard.rank_seed(synth.config_seed(1), rank), dev)
+    dec = DecodeStep(DECODE, shard.rank_seed(synth.config_seed(4), rank), dev)
 
     def barrier():
         if world > 1:
@@ -258,11 +258,7 @@ def run_ours(args, rank, world, dev):
         torch.cuda.synchronize()
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return shard.max_over_ranks(v, dev)
 
     for _ in range(args.warmup):
         step()
@@ -351,7 +347,7 @@ def run_ours(args, rank, world, dev):
     traffic = scan_kernel_traffic("chunk_scan")
     line = {
         "metric": METRIC,
-        "value": world * tokens / (ms_step * 1e-3),
+        "value": shard.aggregate_tokens_per_s(tokens, world, ms_step),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": K,
@@ -382,7 +378,7 @@ def run_ours(args, rank, world, dev):
                    "state_update_GB/s": decode_state_update_bytes(DECODE) / (upd_ms * 1e-3) / 1e9,
                    "frac_hbm": decode_state_update_bytes(DECODE) / (upd_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                    "tokens_per_s": world * DECODE.b / (dec_ms * 1e-3)},
-        "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": shard.aggregate_tokens_per_s(tokens, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": 2 * K,
         "clocks": clocks,
