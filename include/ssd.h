@@ -220,6 +220,24 @@ SSD_API ssd_status_t ssd_state_update(float* state, const void* x, const void* B
                               int H, int P, int N, int G, ssd_dtype_t dtype,
                               cudaStream_t stream);
 
+/*
+ * Self-test of the bounded device waits (failure detection without a fault).
+ * Every wait of the tensor-core scan gives up after a time limit, records
+ * SSD_ERR_TIMEOUT in the call's status word and lets the kernel run to its
+ * end, so that a lost arrival never hangs the GPU.  This call launches one
+ * thread that waits, through the same wait routine, on a barrier nothing
+ * arrives on, for limit_ns nanoseconds.
+ *
+ *   status    device int32, written: SSD_ERR_TIMEOUT (4) when the wait ran
+ *             out as designed; SSD_ERR_CUDA (3) if the routine misbehaved
+ *             (returned early, or waited again after giving up).  The caller
+ *             zeroes it before the call and reads it after synchronising.
+ *   limit_ns  1 .. 1e9 (else SSD_ERR_INVALID_ARG)
+ * Returns SSD_OK when the kernel was launched; the context stays usable.
+ */
+SSD_API ssd_status_t ssd_selftest_bounded_wait(int32_t* status, uint64_t limit_ns,
+                                               cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

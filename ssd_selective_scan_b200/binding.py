@@ -37,6 +37,7 @@ SIGNATURES = {
                               _i, _i, _i, _i, _i, _i, _vp]),
     "ssd_chunk_scan_fwd_static": (_i, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                        _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp]),
+    "ssd_selftest_bounded_wait": (_i, [_vp, ctypes.c_uint64, _vp]),
 }
 
 _lock = threading.Lock()
@@ -101,6 +102,10 @@ def ssd_state_update(state, x, B, C, row_stride, dt_raw, dt_bias, A, D, y, b, H,
                      stream) -> int:
     return load().ssd_state_update(state, x, B, C, row_stride, dt_raw, dt_bias, A, D, y, b, H, P,
                                    N, G, dtype, stream)
+
+
+def ssd_selftest_bounded_wait(status, limit_ns, stream) -> int:
+    return load().ssd_selftest_bounded_wait(status, limit_ns, stream)
 
 
 def check(fn: str, status: int) -> None:

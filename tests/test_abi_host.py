@@ -34,8 +34,8 @@ def declared_entry_points():
 def test_header_declares_the_entry_points():
     assert declared_entry_points() == sorted([
         "ssd_abi_version", "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_static",
-        "ssd_chunk_scan_workspace_bytes", "ssd_conv1d_silu", "ssd_state_update",
-        "ssd_status_string"])
+        "ssd_chunk_scan_workspace_bytes", "ssd_conv1d_silu", "ssd_selftest_bounded_wait",
+        "ssd_state_update", "ssd_status_string"])
 
 
 def test_library_exports_every_declared_symbol():
@@ -144,3 +144,10 @@ def test_state_update_validation():
     assert su(y=fake(1, 64)) == INV                                  # y overlaps state
     assert su(state=fake(2, 64)) == INV                              # state overlaps x
     assert su(N=512) == UNS and su(N=12) == UNS                      # no kernel for these N
+
+
+def test_selftest_validation():
+    # rejected before any launch: no status word, or a limit out of range
+    assert libssd.ssd_selftest_bounded_wait(None, 1000000, None) == libssd.SSD_ERR_INVALID_ARG
+    assert libssd.ssd_selftest_bounded_wait(fake(1), 0, None) == libssd.SSD_ERR_INVALID_ARG
+    assert libssd.ssd_selftest_bounded_wait(fake(1), 2_000_000_000, None) == libssd.SSD_ERR_INVALID_ARG
