@@ -198,6 +198,47 @@ SSD_API ssd_status_t ssd_chunk_scan_fwd_static(const void* x, const void* B, con
                                        cudaStream_t stream);
 
 /*
+ * Ragged prefill: the chunked scan of ssd_chunk_scan_fwd over several
+ * sequences of different lengths packed along one token dimension, each
+ * sequence from its own initial state ("Mamba-2 layer" serving: a prefill
+ * batch of unequal prompts, or a long prompt processed in pieces with the
+ * state handed from one call to the next).  Sequence s is the packed tokens
+ * cu_seqlens[s] .. cu_seqlens[s+1]-1; no token of one sequence affects
+ * another.
+ *
+ *   x          [T][.]   x[t*row_stride + h*P + p]           dtype
+ *   B, C       [T][.]   B[t*row_stride + g*N + n]           dtype
+ *   dt_raw     [T][H]                                       dtype
+ *   y          [T][H][P]                                    dtype, written
+ *   cu_seqlens [nseq+1] int32, DEVICE memory: cu_seqlens[0] = 0,
+ *              non-decreasing, cu_seqlens[nseq] = T.  It is read on the
+ *              device: if it breaks these rules, nothing is written and
+ *              SSD_ERR_INVALID_ARG is stored in *status.
+ *   init_state [nseq][H][P][N] float32 or NULL (zeros)
+ *   final_state[nseq][H][P][N] float32 or NULL; an empty sequence's final
+ *              state is its initial state (or zero)
+ *   status     device int32, REQUIRED (cu_seqlens errors and SSD_ERR_TIMEOUT
+ *              are reported there); the caller zeroes it before the call
+ *   workspace  ssd_chunk_scan_varlen_workspace_bytes(...) bytes, device,
+ *              caller-owned, no initial contents required
+ * Other arguments and requirements as for ssd_chunk_scan_fwd.  nseq = 0
+ * requires T = 0 and does nothing.
+ */
+SSD_API size_t ssd_chunk_scan_varlen_workspace_bytes(int nseq, int T, int H, int P, int N, int G,
+                                                     int Q, ssd_dtype_t dtype);
+
+SSD_API ssd_status_t ssd_chunk_scan_fwd_varlen(const void* x, const void* B, const void* C,
+                                               int64_t row_stride, const void* dt_raw,
+                                               const float* dt_bias, const float* A,
+                                               const float* D, const float* init_state,
+                                               void* y, float* final_state,
+                                               const int32_t* cu_seqlens, int nseq, int T,
+                                               int H, int P, int N, int G, int Q,
+                                               ssd_dtype_t dtype, void* workspace,
+                                               size_t workspace_bytes, int32_t* status,
+                                               cudaStream_t stream);
+
+/*
  * Single-token decode update, in place on the float32 state:
  *
  *   dt = softplus(dt_raw + dt_bias); h <- exp(dt*A) h + dt x B^T;

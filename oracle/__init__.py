@@ -148,6 +148,44 @@ def selective_scan(x, B, C, dt_raw, A, dt_bias=None, D=None, init_state=None,
     return y, fs
 
 
+def selective_scan_varlen(x, B, C, dt_raw, A, cu_seqlens, dt_bias=None, D=None, init_state=None,
+                          nthreads: int | None = None):
+    """The recurrence on a ragged batch packed along the token dimension:
+    sequence s is tokens cu_seqlens[s] .. cu_seqlens[s+1]-1, run from its own
+    initial state (the chunked-prefill reading of "Hybrid Architectures for
+    Language Models", section 2: each sequence is an independent recurrence).
+
+    x [T, H, P]; B, C [T, G, N]; dt_raw [T, H]; init_state [nseq, H, P, N]
+    or None.  Returns (y [T, H, P], final_state [nseq, H, P, N]); an empty
+    sequence's final state is its initial state (or zero).
+    """
+    x = _f64(x)
+    T, H, P = x.shape
+    B = _f64(B)
+    G, N = B.shape[1], B.shape[2]
+    C = _f64(C)
+    dt_raw = _f64(dt_raw, (T, H))
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    nseq = cu.size - 1
+    if nseq < 0 or cu[0] != 0 or cu[-1] != T or np.any(np.diff(cu) < 0):
+        raise ValueError("cu_seqlens must start at 0, not decrease and end at T")
+    init_state = _f64(init_state, (nseq, H, P, N))
+    y = np.zeros_like(x)
+    fs = np.zeros((nseq, H, P, N), dtype=np.float64)
+    for s in range(nseq):
+        a, b = int(cu[s]), int(cu[s + 1])
+        init = None if init_state is None else init_state[s:s + 1]
+        if a == b:
+            if init is not None:
+                fs[s] = init[0]
+            continue
+        ys, fss = selective_scan(x[None, a:b], B[None, a:b], C[None, a:b], dt_raw[None, a:b], A,
+                                 dt_bias, D, init, nthreads)
+        y[a:b] = ys[0]
+        fs[s] = fss[0]
+    return y, fs
+
+
 def state_update(state, x, B, C, dt_raw, A, dt_bias=None, D=None, nthreads: int | None = None):
     """One decode token.  state [b, H, P, N]; x [b, H, P]; B, C [b, G, N];
     dt_raw [b, H].  Returns (y [b, H, P], new_state); inputs are not modified."""

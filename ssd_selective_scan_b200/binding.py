@@ -38,6 +38,9 @@ SIGNATURES = {
     "ssd_chunk_scan_fwd_static": (_i, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                        _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp]),
     "ssd_selftest_bounded_wait": (_i, [_vp, ctypes.c_uint64, _vp]),
+    "ssd_chunk_scan_varlen_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i]),
+    "ssd_chunk_scan_fwd_varlen": (_i, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                       _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp, _vp]),
 }
 
 _lock = threading.Lock()
@@ -102,6 +105,18 @@ def ssd_state_update(state, x, B, C, row_stride, dt_raw, dt_bias, A, D, y, b, H,
                      stream) -> int:
     return load().ssd_state_update(state, x, B, C, row_stride, dt_raw, dt_bias, A, D, y, b, H, P,
                                    N, G, dtype, stream)
+
+
+def ssd_chunk_scan_varlen_workspace_bytes(nseq, T, H, P, N, G, Q, dtype) -> int:
+    return load().ssd_chunk_scan_varlen_workspace_bytes(nseq, T, H, P, N, G, Q, dtype)
+
+
+def ssd_chunk_scan_fwd_varlen(x, B, C, row_stride, dt_raw, dt_bias, A, D, init_state, y, final_state,
+                              cu_seqlens, nseq, T, H, P, N, G, Q, dtype, workspace, workspace_bytes,
+                              status, stream) -> int:
+    return load().ssd_chunk_scan_fwd_varlen(x, B, C, row_stride, dt_raw, dt_bias, A, D, init_state, y,
+                                            final_state, cu_seqlens, nseq, T, H, P, N, G, Q, dtype,
+                                            workspace, workspace_bytes, status, stream)
 
 
 def ssd_selftest_bounded_wait(status, limit_ns, stream) -> int:

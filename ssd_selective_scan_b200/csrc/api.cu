@@ -148,10 +148,87 @@ ssd_status_t ssd_chunk_scan_fwd(const void* x, const void* B, const void* C, int
                                                       cudaMemcpyDeviceToDevice, stream)
                                     : cudaMemsetAsync(final_state, 0, (size_t)st_bytes, stream));
     }
-    if ((int64_t)b * H > 0x7fffffffLL) return SSD_ERR_UNSUPPORTED;
+    // the unit list of the tensor-core path: b * H * chunks
+    if ((int64_t)b * H * ((L + Q - 1) / Q) > 0x7fffffffLL) return SSD_ERR_UNSUPPORTED;
 
     ScanArgs a{x, B, C, row_stride, dt_raw, dt_bias, A, D, init_state, y, final_state,
                b, L, H, P, N, G, Q, dtype == SSD_BF16, workspace, workspace_bytes, status};
+    if (ssd::chunk_scan_tc_supported(a)) return from_cuda(ssd::launch_chunk_scan_tc(a, stream));
+    if (ssd::chunk_scan_simt_smem_bytes(P, N) > (size_t)max_optin_smem()) return SSD_ERR_UNSUPPORTED;
+    return from_cuda(ssd::launch_chunk_scan_simt(a, stream));
+}
+
+size_t ssd_chunk_scan_varlen_workspace_bytes(int nseq, int T, int H, int P, int N, int G, int Q,
+                                             ssd_dtype_t dtype)
+{
+    if (nseq <= 0 || T < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || !valid_dtype(dtype)) return 0;
+    static const int kAnyPtr = 0;
+    ScanArgs a{};
+    a.b = 1; a.L = T; a.H = H; a.P = P; a.N = N; a.G = G; a.Q = Q;
+    a.bf16 = dtype == SSD_BF16;
+    a.cu_seqlens = &kAnyPtr;   // only its presence matters here
+    a.nseq = nseq;
+    return ssd::chunk_scan_tc_supported(a) ? ssd::chunk_scan_tc_workspace_bytes(a) : ssd::varlen_table_bytes(nseq);
+}
+
+ssd_status_t ssd_chunk_scan_fwd_varlen(const void* x, const void* B, const void* C, int64_t row_stride,
+                                       const void* dt_raw, const float* dt_bias, const float* A,
+                                       const float* D, const float* init_state, void* y,
+                                       float* final_state, const int32_t* cu_seqlens, int nseq, int T,
+                                       int H, int P, int N, int G, int Q, ssd_dtype_t dtype, void* workspace,
+                                       size_t workspace_bytes, int32_t* status, cudaStream_t stream)
+{
+    if (!valid_dtype(dtype) || nseq < 0 || T < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0)
+        return SSD_ERR_INVALID_ARG;
+    if (H % G || P % 8 || N % 8 || (Q != 64 && Q != 128)) return SSD_ERR_INVALID_ARG;
+    if (nseq == 0) return T == 0 ? SSD_OK : SSD_ERR_INVALID_ARG;   // tokens without sequences
+    // cu_seqlens is read on the device; a bad one is reported through status
+    if (!A || !cu_seqlens || !status) return SSD_ERR_INVALID_ARG;
+    const bool tokens = T > 0;
+    if (tokens && (!x || !B || !C || !dt_raw || !y)) return SSD_ERR_INVALID_ARG;
+    if (row_stride % 8 || row_stride < (int64_t)H * P || row_stride < (int64_t)G * N) return SSD_ERR_INVALID_ARG;
+    const void* ptrs16[] = {x, B, C, dt_raw, y, init_state, final_state};
+    for (const void* p : ptrs16)
+        if (p && !aligned(p, 16)) return SSD_ERR_INVALID_ARG;
+    if (!aligned(A, 4) || (dt_bias && !aligned(dt_bias, 4)) || (D && !aligned(D, 4)) || !aligned(status, 4) ||
+        !aligned(cu_seqlens, 4))
+        return SSD_ERR_INVALID_ARG;
+    // the unit list of the tensor-core path: H * (T / Q + nseq) bounds it
+    if ((int64_t)H * ((int64_t)T / Q + nseq + 1) > 0x7fffffffLL) return SSD_ERR_UNSUPPORTED;
+    const size_t need_ws = ssd_chunk_scan_varlen_workspace_bytes(nseq, T, H, P, N, G, Q, dtype);
+    if (workspace_bytes < need_ws || !workspace) return SSD_ERR_INVALID_ARG;
+
+    const int e = elem_bytes(dtype);
+    const int64_t rows = T;
+    const int64_t row_bytes = row_stride * e;
+    const Range rx = span(x, rows ? (rows - 1) * row_bytes + (int64_t)H * P * e : 0);
+    const Range rB = span(B, rows ? (rows - 1) * row_bytes + (int64_t)G * N * e : 0);
+    const Range rC = span(C, rows ? (rows - 1) * row_bytes + (int64_t)G * N * e : 0);
+    const Range rdt = span(dt_raw, rows * H * e);
+    const Range ry = span(y, rows * H * P * e);
+    const int64_t st_bytes = (int64_t)nseq * H * P * N * 4;
+    const Range ri = span(init_state, init_state ? st_bytes : 0);
+    const Range rf = span(final_state, final_state ? st_bytes : 0);
+    const Range rcu = span(cu_seqlens, (int64_t)(nseq + 1) * 4);
+    const Range rw = span(workspace, (int64_t)workspace_bytes);
+    for (Range in : {rx, rB, rC, rdt, ri, rcu})
+        if (overlap(ry, in)) return SSD_ERR_INVALID_ARG;
+    for (Range in : {rx, rB, rC, rdt, ry, rcu})
+        if (overlap(rf, in)) return SSD_ERR_INVALID_ARG;
+    if (final_state && init_state && final_state != init_state && overlap(rf, ri)) return SSD_ERR_INVALID_ARG;
+    for (Range in : {rx, rB, rC, rdt, ry, ri, rf, rcu})
+        if (overlap(rw, in)) return SSD_ERR_INVALID_ARG;
+
+    if (!tokens) {
+        // every sequence is empty: check cu_seqlens and set the final states
+        return from_cuda(ssd::launch_varlen_prep(reinterpret_cast<const int*>(cu_seqlens), nseq, 0, H, Q,
+                                                 static_cast<int*>(workspace), nullptr, nullptr, 0, init_state,
+                                                 final_state, (long long)H * P * N, status, stream));
+    }
+    ScanArgs a{x, B, C, row_stride, dt_raw, dt_bias, A, D, init_state, y, final_state,
+               1, T, H, P, N, G, Q, dtype == SSD_BF16, workspace, workspace_bytes, status};
+    a.cu_seqlens = reinterpret_cast<const int*>(cu_seqlens);
+    a.nseq = nseq;
     if (ssd::chunk_scan_tc_supported(a)) return from_cuda(ssd::launch_chunk_scan_tc(a, stream));
     if (ssd::chunk_scan_simt_smem_bytes(P, N) > (size_t)max_optin_smem()) return SSD_ERR_UNSUPPORTED;
     return from_cuda(ssd::launch_chunk_scan_simt(a, stream));

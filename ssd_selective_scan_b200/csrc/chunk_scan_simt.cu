@@ -39,7 +39,8 @@ chunk_scan_simt_kernel(const T* __restrict__ x, const T* __restrict__ B, const T
                        int64_t rs, const T* __restrict__ dt_raw, const float* __restrict__ dt_bias,
                        const float* __restrict__ A, const float* __restrict__ D,
                        const float* __restrict__ init_state, T* __restrict__ y,
-                       float* __restrict__ final_state, int L, int H, int P, int N, int G)
+                       float* __restrict__ final_state, int L, int H, int P, int N, int G,
+                       const int* __restrict__ cu_seqlens, const int* __restrict__ ws_hdr)
 {
     extern __shared__ float smem[];
     constexpr int QS = kSimtChunk;
@@ -54,7 +55,17 @@ chunk_scan_simt_kernel(const T* __restrict__ x, const T* __restrict__ B, const T
     float* sW = sDt + QS;                   // [QS]
 
     const int h = blockIdx.x % H;
-    const int bi = blockIdx.x / H;
+    const int bi = blockIdx.x / H;   // sequence
+    // tokens of the sequence: a dense batch's row bi, or a ragged batch's
+    // packed tokens cu_seqlens[bi] .. cu_seqlens[bi+1]-1 (nothing is done
+    // when the preparation kernel found cu_seqlens invalid)
+    size_t row_base = (size_t)bi * L;
+    int Ls = L;
+    if (cu_seqlens) {
+        if (ws_hdr[0]) return;
+        row_base = (size_t)cu_seqlens[bi];
+        Ls = cu_seqlens[bi + 1] - cu_seqlens[bi];
+    }
     const int g = h / (H / G);
     const int tid = threadIdx.x;
     const float Ah = A[h];
@@ -67,9 +78,9 @@ chunk_scan_simt_kernel(const T* __restrict__ x, const T* __restrict__ B, const T
         sH[p * ldN + n] = init_state ? init_state[sidx + e] : 0.0f;
     }
 
-    for (int t0 = 0; t0 < L; t0 += QS) {
-        const int Qc = min(QS, L - t0);
-        const size_t row0 = (size_t)bi * L + t0;
+    for (int t0 = 0; t0 < Ls; t0 += QS) {
+        const int Qc = min(QS, Ls - t0);
+        const size_t row0 = row_base + t0;
         for (int e = tid; e < Qc * N; e += kSimtThreads) {
             const int i = e / N, n = e % N;
             sB[i * ldN + n] = ld_f(B + (row0 + i) * rs + (size_t)g * N + n);
@@ -139,11 +150,21 @@ static cudaError_t launch_simt_t(const ScanArgs& a, cudaStream_t s)
     auto kern = chunk_scan_simt_kernel<T>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const dim3 grid((unsigned)((int64_t)a.b * a.H));
+    const bool ragged = a.cu_seqlens != nullptr;
+    const int* hdr = nullptr;
+    if (ragged) {   // validate cu_seqlens on the device first
+        if (!a.workspace || a.workspace_bytes < varlen_table_bytes(a.nseq)) return cudaErrorInvalidValue;
+        int* ws = static_cast<int*>(a.workspace);
+        e = launch_varlen_prep(a.cu_seqlens, a.nseq, a.L, a.H, kSimtChunk, ws, nullptr, nullptr, 0, a.init_state,
+                               a.final_state, (long long)a.H * a.P * a.N, a.status, s);
+        if (e != cudaSuccess) return e;
+        hdr = ws;
+    }
+    const dim3 grid((unsigned)((int64_t)(ragged ? a.nseq : a.b) * a.H));
     kern<<<grid, kSimtThreads, smem, s>>>(
         static_cast<const T*>(a.x), static_cast<const T*>(a.B), static_cast<const T*>(a.C),
         a.row_stride, static_cast<const T*>(a.dt_raw), a.dt_bias, a.A, a.D, a.init_state,
-        static_cast<T*>(a.y), a.final_state, a.L, a.H, a.P, a.N, a.G);
+        static_cast<T*>(a.y), a.final_state, a.L, a.H, a.P, a.N, a.G, a.cu_seqlens, hdr);
     return cudaGetLastError();
 }
 

@@ -187,39 +187,135 @@ struct FastDiv {
     __device__ uint32_t div(uint32_t n) const { return (__umulhi(n, m) + n) >> s; }
 };
 
-// A CTA's contiguous range of the unit list (chain-major, nc chunks per
-// chain), in processing order: A = the head of the last chain (published at
-// its end), B = whole chains, C = the tail of the first chain (starts from
-// the predecessor's published state).
+struct Params {
+    const __nv_bfloat16* dt_raw;
+    const float* dt_bias;
+    const float* A;
+    const float* D;
+    const float* init_state;
+    __nv_bfloat16* y;
+    float* final_state;
+    int L, H, G, nc, nslots;   // L: tokens per sequence (dense) or in the packed dimension (ragged)
+    int units;                 // dense batches: units in the list
+    FastDiv fnc, fH, fHG;      // division by nc, H, H / G
+    int* ws_ctrl;        // [0] ticket, [16 + t] hand-off flag of boundary t
+    float* ws_states;    // [nslots][P][N]
+    int32_t* status;
+    // Ragged batches (cu_seqlens != nullptr): sequence s is the packed tokens
+    // cu_seqlens[s] .. cu_seqlens[s+1] - 1; seq_units[s] = H times the chunk
+    // count of the sequences before s; ws_hdr[0] != 0 marks an invalid
+    // cu_seqlens (nothing is done), ws_hdr[1] = the number of units.
+    const int* cu_seqlens;
+    const int* seq_units;
+    const int* ws_hdr;
+    int nseq;
+};
+
+// The unit list: chains c = s * H + h (sequence-major), each the chunks of
+// its sequence in order.  Unit u -> (chain, chunk, chunks in that chain).
+struct Loc {
+    int chain, chunk, ncc;
+};
+
+// `hint` is a sequence at or before u's; callers that visit units in
+// increasing order keep it and the search costs O(1) per call.
+__device__ inline Loc locate(const Params& p, int u, int& hint)
+{
+    Loc l;
+    if (!p.cu_seqlens) {
+        const int ch = (int)p.fnc.div((uint32_t)u);
+        l.chain = ch;
+        l.chunk = u - ch * p.nc;
+        l.ncc = p.nc;
+        return l;
+    }
+    int s = hint;
+    while (s + 1 < p.nseq && __ldg(p.seq_units + s + 1) <= u) ++s;
+    hint = s;
+    const int base = __ldg(p.seq_units + s);
+    const int ncs = max(1, (__ldg(p.seq_units + s + 1) - base) / p.H);   // (never an empty sequence)
+    const int local = u - base;
+    const int h = local / ncs;
+    l.chain = s * p.H + h;
+    l.chunk = local - h * ncs;
+    l.ncc = ncs;
+    return l;
+}
+
+// The (non-empty) sequence holding unit u of a ragged batch: the last s
+// with seq_units[s] <= u (binary search).
+__device__ inline int seq_of_unit(const Params& p, int u)
+{
+    int lo = 0, hi = p.nseq - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(p.seq_units + mid) <= u) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+// A CTA's contiguous range of the unit list, in processing order:
+//   A = the head of the chain the range ends in (published at its end);
+//   B = whole chains;
+//   C = the tail of the chain the range starts in, from the predecessor's
+//       published state.
+// A range that starts and ends inside one chain is a single C segment that
+// is published at its end too.
 struct Range {
     int chA, lenA;
-    int chB0, chB1;
-    int chC, startC;
+    int uB0, nB, sB0;   // B: units [uB0, uB0 + nB); sB0 = sequence of uB0
+    int chC, startC, lenC;
+    bool pubC;
     int count;
 };
 
-__device__ inline Range make_range(int t, int nslots, long long units, int nc)
+__device__ inline Range make_range(const Params& p, int t, int units)
 {
-    const long long u0 = units * t / nslots, u1 = units * (t + 1) / nslots;
-    Range r;
-    const int ch0 = (int)(u0 / nc), c0 = (int)(u0 % nc);
-    const int ch1 = (int)(u1 / nc), c1 = (int)(u1 % nc);
-    r.chA = ch1;
-    r.lenA = c1;
-    r.chC = ch0;
-    r.startC = c0;
-    r.chB0 = c0 > 0 ? ch0 + 1 : ch0;
-    r.chB1 = ch1;
-    r.count = r.lenA + (r.chB1 - r.chB0) * nc + (c0 > 0 ? nc - c0 : 0);
+    Range r{};
+    const int u0 = (int)((long long)units * t / p.nslots);
+    const int u1 = (int)((long long)units * (t + 1) / p.nslots);
+    if (u1 <= u0) return r;
+    int hint0 = p.cu_seqlens ? seq_of_unit(p, u0) : 0;
+    const Loc a = locate(p, u0, hint0);
+    Loc b{-1, 0, 0};   // u1 == units: the end of the list
+    if (u1 < units) {
+        int hint1 = p.cu_seqlens ? seq_of_unit(p, u1) : 0;
+        b = locate(p, u1, hint1);
+    }
+    if (a.chunk > 0 && b.chain == a.chain) {   // inside one chain
+        r.chC = a.chain;
+        r.startC = a.chunk;
+        r.lenC = b.chunk - a.chunk;
+        r.pubC = true;
+        r.count = r.lenC;
+        return r;
+    }
+    r.chA = b.chain;
+    r.lenA = b.chunk;
+    if (a.chunk > 0) {
+        r.chC = a.chain;
+        r.startC = a.chunk;
+        r.lenC = a.ncc - a.chunk;
+    }
+    r.uB0 = a.chunk > 0 ? u0 + (a.ncc - a.chunk) : u0;
+    r.nB = (u1 - b.chunk) - r.uB0;
+    r.sB0 = p.cu_seqlens && r.nB > 0 ? seq_of_unit(p, r.uB0) : 0;
+    r.count = r.lenA + r.nB + r.lenC;
     return r;
 }
 
 struct Item {
     int chain, chunk;
+    int seq, h;        // chain = seq * H + h
+    int tok0;          // first token of the chunk along the token dimension
+    int nvalid;        // tokens of the sequence in the chunk (<= kQ)
+    int bi;            // coordinate along the batch dimension (0 for a ragged batch)
     bool seg_start, seg_end, publish, depend;
+    bool direct_y;     // y written row by row (a ragged batch's last, partial chunk)
 };
 
-__device__ inline Item item_at(const Range& r, int idx, int nc, const FastDiv& fnc)
+__device__ inline Item item_at(const Params& p, const Range& r, int idx, int& hint)
 {
     Item it;
     if (idx < r.lenA) {
@@ -229,45 +325,40 @@ __device__ inline Item item_at(const Range& r, int idx, int nc, const FastDiv& f
         it.seg_end = idx == r.lenA - 1;
         it.publish = it.seg_end;
         it.depend = false;
-        return it;
-    }
-    idx -= r.lenA;
-    const int nb = (r.chB1 - r.chB0) * nc;
-    if (idx < nb) {
-        const uint32_t q = fnc.div((uint32_t)idx);
-        it.chain = r.chB0 + (int)q;
-        it.chunk = idx - (int)q * nc;
-        it.seg_start = it.chunk == 0;
-        it.seg_end = it.chunk == nc - 1;
+    } else if (idx - r.lenA < r.nB) {
+        const Loc l = locate(p, r.uB0 + (idx - r.lenA), hint);
+        it.chain = l.chain;
+        it.chunk = l.chunk;
+        it.seg_start = l.chunk == 0;
+        it.seg_end = l.chunk == l.ncc - 1;
         it.publish = false;
         it.depend = false;
-        return it;
+    } else {
+        const int k = idx - r.lenA - r.nB;
+        it.chain = r.chC;
+        it.chunk = r.startC + k;
+        it.seg_start = k == 0;
+        it.depend = it.seg_start;
+        it.seg_end = k == r.lenC - 1;
+        it.publish = it.seg_end && r.pubC;
     }
-    idx -= nb;
-    it.chain = r.chC;
-    it.chunk = r.startC + idx;
-    it.seg_start = idx == 0;
-    it.seg_end = it.chunk == nc - 1;
-    it.publish = false;
-    it.depend = it.seg_start;
+    it.seq = (int)p.fH.div((uint32_t)it.chain);
+    it.h = it.chain - it.seq * p.H;
+    if (p.cu_seqlens) {
+        const int s0 = __ldg(p.cu_seqlens + it.seq);
+        const int len = __ldg(p.cu_seqlens + it.seq + 1) - s0;
+        it.tok0 = s0 + it.chunk * kQ;
+        it.nvalid = min(kQ, len - it.chunk * kQ);
+        it.bi = 0;
+        it.direct_y = it.nvalid < kQ;
+    } else {
+        it.tok0 = it.chunk * kQ;
+        it.nvalid = min(kQ, p.L - it.tok0);
+        it.bi = it.seq;
+        it.direct_y = false;
+    }
     return it;
 }
-
-struct Params {
-    const __nv_bfloat16* dt_raw;
-    const float* dt_bias;
-    const float* A;
-    const float* D;
-    const float* init_state;
-    __nv_bfloat16* y;
-    float* final_state;
-    int L, H, G, nc, nslots;
-    long long units;
-    FastDiv fnc, fH, fHG;   // division by nc, H, H / G
-    int* ws_ctrl;        // [0] ticket, [16 + t] hand-off flag of boundary t
-    float* ws_states;    // [nslots][P][N]
-    int32_t* status;
-};
 
 __device__ inline void tmem_ld8(uint32_t taddr, float (&v)[8])
 {
@@ -307,7 +398,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     int* ticket_slot = reinterpret_cast<int*>(smem + kOffMisc + 8);
     uint8_t* sHB = smem + kOffHB;
     uint8_t* sWX = smem + kOffWX;
-    const int H = prm.H, nc = prm.nc, L = prm.L;
+    const int H = prm.H, L = prm.L;
 
     if (tid == 0) {
         *aborted = 0;
@@ -333,13 +424,10 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     const int ticket = *ticket_slot;
-    const Range rg = make_range(ticket, prm.nslots, prm.units, nc);
-
-    auto coords = [&](const Item& it, int& bi, int& h, int& g) {
-        bi = (int)prm.fH.div((uint32_t)it.chain);
-        h = it.chain - bi * H;
-        g = (int)prm.fHG.div((uint32_t)h);
-    };
+    // a ragged batch reads its unit count (0 if cu_seqlens was invalid)
+    const int units = prm.cu_seqlens ? (prm.ws_hdr[0] ? 0 : prm.ws_hdr[1]) : prm.units;
+    const Range rg = make_range(prm, ticket, units);
+    auto group_of = [&](const Item& it) { return (int)prm.fHG.div((uint32_t)it.h); };
     auto stage = [&](int idx) { return smem + kOffStage + (idx & 1) * kStageBytes; };
 
     if (warp == kMmaWarp) {
@@ -404,38 +492,34 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         // ------------------------------------------------------------------
         if (lane == 0 && rg.count > 0) {
             // B and C of item idx into its stage (G = C B^T needs only these)
+            // each call site visits items in increasing order and keeps its own hint
+            int hint_bc = rg.sB0, hint_x = rg.sB0, hint_pf = rg.sB0, hint_st = rg.sB0;
             auto issue_bc = [&](int idx) {
-                const Item it = item_at(rg, idx, nc, prm.fnc);
-                int bi, h, g;
-                coords(it, bi, h, g);
-                const int t0 = it.chunk * kQ;
+                const Item it = item_at(prm, rg, idx, hint_bc);
+                const int g = group_of(it);
                 uint8_t* st = stage(idx);
                 uint64_t* bar = bar_ld + (idx & 1);
                 mbar_arrive_expect_tx(bar, kBytesBC);
-                tma_load_3d(st + kStB, &tmB, g * kN, t0, bi, bar);
-                tma_load_3d(st + kStB + kTileHalf, &tmB, g * kN + 64, t0, bi, bar);
-                tma_load_3d(st + kStC, &tmC, g * kN, t0, bi, bar);
-                tma_load_3d(st + kStC + kTileHalf, &tmC, g * kN + 64, t0, bi, bar);
+                tma_load_3d(st + kStB, &tmB, g * kN, it.tok0, it.bi, bar);
+                tma_load_3d(st + kStB + kTileHalf, &tmB, g * kN + 64, it.tok0, it.bi, bar);
+                tma_load_3d(st + kStC, &tmC, g * kN, it.tok0, it.bi, bar);
+                tma_load_3d(st + kStC + kTileHalf, &tmC, g * kN + 64, it.tok0, it.bi, bar);
             };
             // X of item idx into its stage (the buffer that held y of item idx - 2)
             auto issue_x = [&](int idx) {
-                const Item it = item_at(rg, idx, nc, prm.fnc);
-                int bi, h, g;
-                coords(it, bi, h, g);
+                const Item it = item_at(prm, rg, idx, hint_x);
                 uint64_t* bar = bar_ldx + (idx & 1);
                 mbar_arrive_expect_tx(bar, kBytesX);
-                tma_load_3d(stage(idx) + kStX, &tmX, h * kP, it.chunk * kQ, bi, bar);
+                tma_load_3d(stage(idx) + kStX, &tmX, it.h * kP, it.tok0, it.bi, bar);
             };
             auto prefetch_l2 = [&](int idx) {
-                const Item it = item_at(rg, idx, nc, prm.fnc);
-                int bi, h, g;
-                coords(it, bi, h, g);
-                const int t0 = it.chunk * kQ;
-                tma_prefetch_l2_3d(&tmB, g * kN, t0, bi);
-                tma_prefetch_l2_3d(&tmB, g * kN + 64, t0, bi);
-                tma_prefetch_l2_3d(&tmC, g * kN, t0, bi);
-                tma_prefetch_l2_3d(&tmC, g * kN + 64, t0, bi);
-                tma_prefetch_l2_3d(&tmX, h * kP, t0, bi);
+                const Item it = item_at(prm, rg, idx, hint_pf);
+                const int g = group_of(it);
+                tma_prefetch_l2_3d(&tmB, g * kN, it.tok0, it.bi);
+                tma_prefetch_l2_3d(&tmB, g * kN + 64, it.tok0, it.bi);
+                tma_prefetch_l2_3d(&tmC, g * kN, it.tok0, it.bi);
+                tma_prefetch_l2_3d(&tmC, g * kN + 64, it.tok0, it.bi);
+                tma_prefetch_l2_3d(&tmX, it.h * kP, it.tok0, it.bi);
             };
             prefetch_tensormap(&tmX);
             prefetch_tensormap(&tmB);
@@ -456,12 +540,12 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 // y of item idx is staged in its X buffer: store it, then
                 // reload the buffer once the store has read it
                 mbar_wait_bounded(bar_ystaged + (idx & 1), sph, kWaitNs, aborted, prm.status);
-                const Item it = item_at(rg, idx, nc, prm.fnc);
-                int bi, h, g;
-                coords(it, bi, h, g);
-                tma_store_3d(&tmY, stage(idx) + kStX, h * kP, it.chunk * kQ, bi);
-                bulk_commit_group();
-                bulk_wait_group_read0();
+                const Item it = item_at(prm, rg, idx, hint_st);
+                if (!it.direct_y) {   // (a partial ragged chunk's rows went out directly)
+                    tma_store_3d(&tmY, stage(idx) + kStX, it.h * kP, it.tok0, it.bi);
+                    bulk_commit_group();
+                    bulk_wait_group_read0();
+                }
                 if (idx + 2 < rg.count) issue_x(idx + 2);
                 if (idx + 3 < rg.count) prefetch_l2(idx + 3);
             }
@@ -481,18 +565,16 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             __nv_bfloat16 dt[4];
         };
         // raw inputs of item idx for tokens 4*lane .. 4*lane+3
+        int hint = rg.sB0;
         auto load_dt = [&](int idx) {
             DtIn in;
-            const Item it = item_at(rg, idx, nc, prm.fnc);
-            int bi, h, g;
-            coords(it, bi, h, g);
-            in.a2 = prm.A[h] * 1.4426950408889634f;   // A * log2(e)
-            in.bias = prm.dt_bias ? prm.dt_bias[h] : 0.0f;
-            const __nv_bfloat16* dp = prm.dt_raw + (size_t)bi * L * H + h;
-            const int t0 = it.chunk * kQ + lane * 4;
-            in.nvalid = L - t0;
+            const Item it = item_at(prm, rg, idx, hint);
+            in.a2 = prm.A[it.h] * 1.4426950408889634f;   // A * log2(e)
+            in.bias = prm.dt_bias ? prm.dt_bias[it.h] : 0.0f;
+            const __nv_bfloat16* dp = prm.dt_raw + ((size_t)it.bi * L + it.tok0 + lane * 4) * H + it.h;
+            in.nvalid = it.nvalid - lane * 4;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) in.dt[k] = k < in.nvalid ? dp[(size_t)(t0 + k) * H] : __float2bfloat16_rn(0.0f);
+            for (int k = 0; k < 4; ++k) in.dt[k] = k < in.nvalid ? dp[(size_t)k * H] : __float2bfloat16_rn(0.0f);
             return in;
         };
         // dt (0 past the sequence end), the inclusive cumulative log2 decay
@@ -599,7 +681,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         // is in Yd through M's diagonal), written over x in the item's X
         // buffer for the producer's TMA store.  M X of item j (the X
         // buffer's last reader) is done once bar_m2 has completed for it.
-        auto y_epilogue = [&](int j, float cl_i) {
+        auto y_epilogue = [&](int j, float cl_i, const Item& itj) {
             mbar_wait_bounded(bar_m2, (uint32_t)j & 1u, kWaitNs, aborted, prm.status);
             tc_fence_after_sync();
             uint8_t* xs = stage(j) + kStX;
@@ -618,16 +700,26 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                     o[e] = r.x;
                     o[e + 1] = r.y;
                 }
-                *reinterpret_cast<uint4*>(xs + sw128(row, quarter * 2 + q)) = pack_bf16x8(o);
+                if (!itj.direct_y) {
+                    *reinterpret_cast<uint4*>(xs + sw128(row, quarter * 2 + q)) = pack_bf16x8(o);
+                } else if (row < itj.nvalid) {
+                    // a ragged batch's partial last chunk: its rows past the
+                    // sequence's end belong to the next sequence, so the rows
+                    // go out one by one instead of as a 128-row TMA box
+                    __nv_bfloat16* yr = prm.y + ((size_t)(itj.tok0 + row) * H + itj.h) * kP + p0 + q * 8;
+                    *reinterpret_cast<uint4*>(yr) = pack_bf16x8(o);
+                }
             }
             fence_proxy_async_smem();
             mbar_arrive(bar_ystaged + (j & 1));
         };
 
         float prev_cl_i = 0.0f;
+        Item prev_it{};
+        int hint = rg.sB0;
         for (int idx = 0; idx < rg.count; ++idx) {
-            const Item it = item_at(rg, idx, nc, prm.fnc);
-            const int bi = (int)prm.fH.div((uint32_t)it.chain), h = it.chain - bi * H;
+            const Item it = item_at(prm, rg, idx, hint);
+            const int bi = it.seq, h = it.h;
             const float Dh = prm.D ? prm.D[h] : 0.0f;
             uint8_t* st = stage(idx);
 
@@ -687,7 +779,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             mbar_arrive(bar_sready);   // C h^T and the state update can start
 
             // 4. y of the previous item, whose M X ran meanwhile
-            if (idx > 0) y_epilogue(idx - 1, prev_cl_i);
+            if (idx > 0) y_epilogue(idx - 1, prev_cl_i, prev_it);
 
             // 5. the masked tile M = G o L of item idx into TMEM (bf16
             //    pairs), the A operand of M X.  Column block jb (32 tokens)
@@ -767,8 +859,9 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 }
             }
             prev_cl_i = cl_i;
+            prev_it = it;
         }
-        if (rg.count > 0) y_epilogue(rg.count - 1, prev_cl_i);
+        if (rg.count > 0) y_epilogue(rg.count - 1, prev_cl_i, prev_it);
     }
 
     tc_fence_before_sync();
@@ -817,7 +910,7 @@ int tc_slots(const ScanArgs& a)
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
         sms = 148;
-    const long long chains = (long long)a.b * a.H;
+    const long long chains = (long long)(a.cu_seqlens ? a.nseq : a.b) * a.H;
     const long long slots = sms;   // one CTA per SM
     return (int)(chains < slots ? chains : slots);
 }
@@ -831,6 +924,11 @@ bool chunk_scan_tc_supported(const ScanArgs& a)
 
 size_t chunk_scan_tc_workspace_bytes(const ScanArgs& a)
 {
+    if (a.cu_seqlens) {   // ragged: the unit table comes first
+        if (a.nseq <= 0) return 0;
+        const int slots = tc_slots(a);
+        return varlen_table_bytes(a.nseq) + kWsCtrlBytes(slots) + (size_t)slots * kStateBytes;
+    }
     if (a.b <= 0 || a.L <= 0) return 0;
     const int slots = tc_slots(a);
     return kWsCtrlBytes(slots) + (size_t)slots * kStateBytes;
@@ -850,9 +948,21 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t s)
     if (e != cudaSuccess) return e;
     const int slots = tc_slots(a);
     const size_t ctrl = kWsCtrlBytes(slots);
-    if (!a.workspace || a.workspace_bytes < ctrl + (size_t)slots * kStateBytes) return cudaErrorInvalidValue;
-    // ticket counter and hand-off flags start at zero on every call
-    if ((e = cudaMemsetAsync(a.workspace, 0, ctrl, s)) != cudaSuccess) return e;
+    const bool ragged = a.cu_seqlens != nullptr;
+    const size_t table = ragged ? varlen_table_bytes(a.nseq) : 0;
+    if (!a.workspace || a.workspace_bytes < table + ctrl + (size_t)slots * kStateBytes) return cudaErrorInvalidValue;
+    uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+    int* ws_ctrl = reinterpret_cast<int*>(ws + table);
+    // ticket counter and hand-off flags start at zero on every call (a
+    // ragged call's preparation kernel clears them with its other work)
+    if (ragged) {
+        e = launch_varlen_prep(a.cu_seqlens, a.nseq, a.L, a.H, kQ, reinterpret_cast<int*>(ws),
+                               reinterpret_cast<int*>(ws + kVarlenUnitsOffset), ws_ctrl, (int)(ctrl / 4),
+                               a.init_state, a.final_state, (long long)a.H * kP * kN, a.status, s);
+        if (e != cudaSuccess) return e;
+    } else if ((e = cudaMemsetAsync(ws_ctrl, 0, ctrl, s)) != cudaSuccess) {
+        return e;
+    }
     Params prm;
     prm.dt_raw = static_cast<const __nv_bfloat16*>(a.dt_raw);
     prm.dt_bias = a.dt_bias;
@@ -864,14 +974,18 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t s)
     prm.L = a.L;
     prm.H = a.H;
     prm.G = a.G;
-    prm.nc = (a.L + kQ - 1) / kQ;
+    prm.nc = ragged ? 1 : (a.L + kQ - 1) / kQ;   // (a ragged batch's chunk counts vary)
     prm.nslots = slots;
-    prm.units = (long long)a.b * a.H * prm.nc;
+    prm.units = ragged ? 0 : a.b * a.H * prm.nc;
     prm.fnc = FastDiv::make((uint32_t)prm.nc);
     prm.fH = FastDiv::make((uint32_t)a.H);
     prm.fHG = FastDiv::make((uint32_t)(a.H / a.G));
-    prm.ws_ctrl = static_cast<int*>(a.workspace);
-    prm.ws_states = reinterpret_cast<float*>(static_cast<uint8_t*>(a.workspace) + ctrl);
+    prm.ws_ctrl = ws_ctrl;
+    prm.ws_states = reinterpret_cast<float*>(ws + table + ctrl);
+    prm.cu_seqlens = a.cu_seqlens;
+    prm.seq_units = ragged ? reinterpret_cast<const int*>(ws + kVarlenUnitsOffset) : nullptr;
+    prm.ws_hdr = ragged ? reinterpret_cast<const int*>(ws) : nullptr;
+    prm.nseq = ragged ? a.nseq : a.b;
     prm.status = a.status;
     chunk_scan_tc_kernel<<<slots, kThreads, kSmemBytes, s>>>(tmX, tmB, tmC, tmY, prm);
     return cudaGetLastError();

@@ -26,7 +26,21 @@ struct ScanArgs {
     void* workspace;
     size_t workspace_bytes;
     int32_t* status;
+    // Ragged batches: sequence s is tokens cu_seqlens[s] .. cu_seqlens[s+1]-1
+    // of one packed token dimension of L tokens (b = 1 then); nseq sequences.
+    const int* cu_seqlens = nullptr;
+    int nseq = 0;
 };
+
+// Workspace of a ragged scan: a header (hdr[0] = invalid cu_seqlens flag,
+// hdr[1] = unit count) and the per-sequence unit prefix, then the path's own
+// workspace.
+inline size_t varlen_table_bytes(int nseq) { return ((size_t)256 + (size_t)(nseq + 1) * 4 + 255) / 256 * 256; }
+constexpr size_t kVarlenUnitsOffset = 256;   // seq_units after the 256-byte header
+
+cudaError_t launch_varlen_prep(const int* cu_seqlens, int nseq, int T, int H, int Q, int* hdr, int* seq_units,
+                               int* ctrl, int ctrl_ints, const float* init_state, float* final_state,
+                               long long state_elems_per_seq, int32_t* status, cudaStream_t s);
 
 cudaError_t launch_conv1d_silu(const void* xBC, void* out, const float* w, const float* bias,
                                void* conv_state, int b, int L, int conv_dim, int k, bool bf16,

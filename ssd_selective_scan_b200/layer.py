@@ -114,6 +114,63 @@ def chunk_scan_fwd(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor, dt_raw: to
     return y, final_state
 
 
+def chunk_scan_varlen_workspace_bytes(nseq, T, H, P, N, G, Q, dtype: torch.dtype) -> int:
+    return int(libssd.ssd_chunk_scan_varlen_workspace_bytes(nseq, T, H, P, N, G, Q, _DT[dtype]))
+
+
+def chunk_scan_fwd_varlen(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor, dt_raw: torch.Tensor,
+                          A: torch.Tensor, cu_seqlens: torch.Tensor, dt_bias: torch.Tensor | None = None,
+                          D: torch.Tensor | None = None, init_state: torch.Tensor | None = None,
+                          Q: int = 128, y: torch.Tensor | None = None,
+                          final_state: torch.Tensor | bool | None = True,
+                          workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                          stream=None):
+    """Chunked SSD scan of a ragged batch packed along the token dimension.
+    x [T, H, P], B/C [T, G, N] (views sharing one token stride), dt_raw
+    [T, H]; cu_seqlens int32 [nseq + 1] on the device (sequence s is tokens
+    cu_seqlens[s] .. cu_seqlens[s+1]-1); init_state [nseq, H, P, N] or None.
+    Returns (y [T, H, P], final_state [nseq, H, P, N] f32 or None).  A bad
+    cu_seqlens is reported in `status` (allocated here if not given), which
+    the caller reads after synchronising."""
+    T, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or not cu_seqlens.is_contiguous():
+        raise ValueError("cu_seqlens must be a contiguous int32 vector")
+    nseq = cu_seqlens.numel() - 1
+    if T == 0:
+        rs = -(-max(H * P, G * N) // 8) * 8
+    else:
+        rs = x.stride(0)
+        if x.stride(2) != 1 or x.stride(1) != P:
+            raise ValueError("x must be [T, H, P] with contiguous (H, P) rows")
+        for t, name in ((B, "B"), (C, "C")):
+            if t.stride(0) != rs or t.stride(2) != 1 or t.stride(1) != N:
+                raise ValueError(f"{name} must share x's token stride with contiguous (G, N) rows")
+    if B.dtype != x.dtype or C.dtype != x.dtype or dt_raw.dtype != x.dtype:
+        raise ValueError("x, B, C, dt_raw must share the I/O dtype")
+    if dt_raw.shape != (T, H) or not dt_raw.is_contiguous():
+        raise ValueError("dt_raw must be a contiguous [T, H] tensor")
+    if y is None:
+        y = torch.empty((T, H, P), dtype=x.dtype, device=x.device)
+    if final_state is True:
+        final_state = torch.empty((nseq, H, P, N), dtype=torch.float32, device=x.device)
+    elif final_state is False:
+        final_state = None
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=x.device)
+    need = chunk_scan_varlen_workspace_bytes(nseq, T, H, P, N, G, Q, x.dtype)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = libssd.ssd_chunk_scan_fwd_varlen(
+        _ptr(x), _ptr(B), _ptr(C), rs, _ptr(dt_raw), _ptr(_f32(dt_bias, "dt_bias")),
+        _ptr(_f32(A, "A")), _ptr(_f32(D, "D")), _ptr(_f32(init_state, "init_state")), _ptr(y),
+        _ptr(final_state), _ptr(cu_seqlens), nseq, T, H, P, N, G, Q, _dtype_code(x), _ptr(workspace),
+        ws_bytes, _ptr(status), _stream(stream))
+    libssd.check("ssd_chunk_scan_fwd_varlen", st)
+    return y, final_state
+
+
 def state_update(state: torch.Tensor, x: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
                  dt_raw: torch.Tensor, A: torch.Tensor, dt_bias: torch.Tensor | None = None,
                  D: torch.Tensor | None = None, y: torch.Tensor | None = None, stream=None):

@@ -330,6 +330,48 @@ def check_cache_size_formula():
     assert fs[0].size + cs[0].size == d_ssm * d_state + k * (2 * d_state + d_ssm)
 
 
+def check_varlen_matches_each_sequence_alone():
+    """A ragged batch (lengths 13, 0, 40, 1, 7, 0: empty sequences inside and
+    at the end) equals the independent chunked evaluation of each sequence
+    alone from its own initial state; an empty sequence's final state is its
+    initial state."""
+    rng = _rng(21)
+    lens = [13, 0, 40, 1, 7, 0]
+    T, H, P, N, G = sum(lens), 4, 3, 5, 2
+    inp = _random_scan_inputs(rng, b=1, L=T, H=H, P=P, N=N, G=G, init=False)
+    x, B, C, dt_raw = inp["x"][0], inp["B"][0], inp["C"][0], inp["dt_raw"][0]
+    h0 = rng.standard_normal((len(lens), H, P, N)) * 0.3
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    y, fs = oracle.selective_scan_varlen(x, B, C, dt_raw, inp["A"], cu, inp["dt_bias"], inp["D"], h0,
+                                         nthreads=2)
+    for s in range(len(lens)):
+        a, b = int(cu[s]), int(cu[s + 1])
+        if a == b:
+            assert np.array_equal(fs[s], h0[s]), f"empty sequence {s}: final state is not its initial state"
+            continue
+        one = dict(x=x[None, a:b], B=B[None, a:b], C=C[None, a:b], dt_raw=dt_raw[None, a:b],
+                   dt_bias=inp["dt_bias"], A=inp["A"], D=inp["D"], init_state=h0[s:s + 1])
+        yr, fr = chunked_ssd(one, Q=8)
+        _close(y[a:b], yr[0], 1e-12, f"ragged y (sequence {s})")
+        _close(fs[s], fr[0], 1e-12, f"ragged final state (sequence {s})")
+
+
+def check_varlen_chunked_prefill():
+    """A sequence prefilled as two ragged calls, the second from the first
+    call's final state, equals one call on the whole sequence."""
+    rng = _rng(22)
+    L, t = 50, 23
+    inp = _random_scan_inputs(rng, b=1, L=L)
+    x, B, C, dt_raw, h0 = inp["x"][0], inp["B"][0], inp["C"][0], inp["dt_raw"][0], inp["init_state"]
+    y, fs = oracle.selective_scan_varlen(x, B, C, dt_raw, inp["A"], [0, L], inp["dt_bias"], inp["D"], h0)
+    ya, fa = oracle.selective_scan_varlen(x[:t], B[:t], C[:t], dt_raw[:t], inp["A"], [0, t], inp["dt_bias"],
+                                          inp["D"], h0)
+    yb, fb = oracle.selective_scan_varlen(x[t:], B[t:], C[t:], dt_raw[t:], inp["A"], [0, L - t],
+                                          inp["dt_bias"], inp["D"], fa)
+    _close(np.concatenate([ya, yb]), y, 1e-13, "chunked prefill y")
+    _close(fb, fs, 1e-13, "chunked prefill final state")
+
+
 ALL_CHECKS = [
     check_dt_to_zero,
     check_geometric_series,
@@ -344,4 +386,6 @@ ALL_CHECKS = [
     check_decode_step_extends_prefill,
     check_conv_state_handoff,
     check_cache_size_formula,
+    check_varlen_matches_each_sequence_alone,
+    check_varlen_chunked_prefill,
 ]

@@ -34,6 +34,7 @@ def declared_entry_points():
 def test_header_declares_the_entry_points():
     assert declared_entry_points() == sorted([
         "ssd_abi_version", "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_static",
+        "ssd_chunk_scan_fwd_varlen", "ssd_chunk_scan_varlen_workspace_bytes",
         "ssd_chunk_scan_workspace_bytes", "ssd_conv1d_silu", "ssd_selftest_bounded_wait",
         "ssd_state_update", "ssd_status_string"])
 
@@ -151,3 +152,33 @@ def test_selftest_validation():
     assert libssd.ssd_selftest_bounded_wait(None, 1000000, None) == libssd.SSD_ERR_INVALID_ARG
     assert libssd.ssd_selftest_bounded_wait(fake(1), 0, None) == libssd.SSD_ERR_INVALID_ARG
     assert libssd.ssd_selftest_bounded_wait(fake(1), 2_000_000_000, None) == libssd.SSD_ERR_INVALID_ARG
+
+
+def varlen(**kw):
+    a = dict(x=fake(1), B=fake(1, 5120), C=fake(1, 7168), row_stride=4608, dt_raw=fake(2), dt_bias=None,
+             A=fake(3), D=None, init_state=None, y=fake(4), final_state=fake(5), cu_seqlens=fake(6), nseq=3,
+             T=500, H=40, P=64, N=128, G=8, Q=128, dtype=BF16, workspace=fake(7), workspace_bytes=1 << 30,
+             status=fake(8), stream=None)
+    a.update(kw)
+    return libssd.ssd_chunk_scan_fwd_varlen(**a)
+
+
+def test_varlen_validation():
+    # every call here fails validation (or does nothing) before any launch
+    assert varlen(nseq=0, T=0) == OK                 # nothing to do
+    assert varlen(nseq=0, T=10) == INV               # tokens without sequences
+    assert varlen(status=None) == INV                # cu_seqlens errors need a status word
+    assert varlen(cu_seqlens=None) == INV
+    assert varlen(A=None) == INV and varlen(x=None) == INV and varlen(y=None) == INV
+    assert varlen(dtype=7) == INV and varlen(G=7) == INV and varlen(Q=96) == INV
+    assert varlen(nseq=-1) == INV and varlen(T=-1) == INV
+    assert varlen(workspace_bytes=16) == INV and varlen(workspace=None) == INV
+    assert varlen(cu_seqlens=fake(6, 2)) == INV      # misaligned
+    assert varlen(y=fake(1, 64)) == INV              # y overlaps x
+    assert varlen(final_state=fake(6)) == INV        # final state overlaps cu_seqlens
+    assert varlen(H=256, row_stride=16384, T=(1 << 31) - 1) == UNS   # unit list would overflow
+    ws = libssd.ssd_chunk_scan_varlen_workspace_bytes(3, 500, 40, 64, 128, 8, 128, BF16)
+    assert ws > 0 and ws == libssd.ssd_chunk_scan_varlen_workspace_bytes(3, 500, 40, 64, 128, 8, 128, BF16)
+    # the fp32 path needs only the unit table
+    assert libssd.ssd_chunk_scan_varlen_workspace_bytes(3, 500, 4, 64, 16, 1, 64, F32) == 256 + 256 * 0 + 256
+    assert libssd.ssd_chunk_scan_varlen_workspace_bytes(0, 0, 4, 64, 16, 1, 64, F32) == 0

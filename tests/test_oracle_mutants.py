@@ -59,3 +59,31 @@ def test_pins_catch_planted_mistake(name, tmp_path):
             except AssertionError:
                 caught.append(check.__name__)
     assert caught, f"planted mistake {name!r} passed every pin"
+
+
+def _carry_state_across_sequences(x, B, C, dt_raw, A, cu_seqlens, dt_bias=None, D=None, init_state=None,
+                                  nthreads=None):
+    """Planted mistake: every sequence after the first starts from the
+    previous sequence's final state instead of its own initial state."""
+    import numpy as np
+    y, fs = _REAL_VARLEN(x, B, C, dt_raw, A, [0, int(cu_seqlens[-1])], dt_bias, D,
+                         None if init_state is None else init_state[:1], nthreads)
+    n = len(cu_seqlens) - 1
+    return y, np.repeat(fs, n, axis=0)
+
+
+def _ignore_initial_states(x, B, C, dt_raw, A, cu_seqlens, dt_bias=None, D=None, init_state=None,
+                           nthreads=None):
+    """Planted mistake: the per-sequence initial states are dropped."""
+    return _REAL_VARLEN(x, B, C, dt_raw, A, cu_seqlens, dt_bias, D, None, nthreads)
+
+
+_REAL_VARLEN = oracle.selective_scan_varlen
+
+
+@pytest.mark.parametrize("mutant", [_carry_state_across_sequences, _ignore_initial_states],
+                         ids=lambda f: f.__name__)
+def test_pins_catch_planted_ragged_mistake(mutant, monkeypatch):
+    monkeypatch.setattr(oracle, "selective_scan_varlen", mutant)
+    with pytest.raises(AssertionError):
+        oracle_checks.check_varlen_matches_each_sequence_alone()
