@@ -87,7 +87,9 @@ constexpr int kStB = 0, kStC = 32768, kStX = 65536;
 constexpr int kOffHB = 2 * kStageBytes;         // bf16 state entering the item [128 n][64 p]
 constexpr int kOffWX = kOffHB + 16384;          // w o X [128 tok][64 p]
 constexpr int kOffVec = kOffWX + 16384;         // per chunk parity: cl, dt, v  (3 x float[128]) x 2
-constexpr int kOffBar = kOffVec + 3072;         // mbarriers
+constexpr int kMaxSeqSmem = 1024;               // ragged batches: tables in shared memory up to this
+constexpr int kOffSeq = kOffVec + 3072;         // cu_seqlens, then seq_units (int[kMaxSeqSmem + 1] each)
+constexpr int kOffBar = kOffSeq + 8 * (kMaxSeqSmem + 1) + 8;   // mbarriers (8-byte aligned)
 constexpr int kNumBars = 13;
 constexpr int kOffMisc = kOffBar + 8 * kNumBars;   // tmem slot, abort flag, ticket
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
@@ -217,12 +219,20 @@ struct Loc {
     int chain, chunk, ncc;
 };
 
+// Ragged batches' tables, in shared memory when they fit (else global):
+// cu = cu_seqlens, su = seq_units.
+struct Tabs {
+    const int* cu;
+    const int* su;
+};
+
 // `hint` is a sequence at or before u's; callers that visit units in
 // increasing order keep it and the search costs O(1) per call.
-__device__ inline Loc locate(const Params& p, int u, int& hint)
+template <bool kRagged>
+__device__ inline Loc locate(const Params& p, const Tabs& tb, int u, int& hint)
 {
     Loc l;
-    if (!p.cu_seqlens) {
+    if constexpr (!kRagged) {
         const int ch = (int)p.fnc.div((uint32_t)u);
         l.chain = ch;
         l.chunk = u - ch * p.nc;
@@ -230,10 +240,10 @@ __device__ inline Loc locate(const Params& p, int u, int& hint)
         return l;
     }
     int s = hint;
-    while (s + 1 < p.nseq && __ldg(p.seq_units + s + 1) <= u) ++s;
+    while (s + 1 < p.nseq && tb.su[s + 1] <= u) ++s;
     hint = s;
-    const int base = __ldg(p.seq_units + s);
-    const int ncs = max(1, (__ldg(p.seq_units + s + 1) - base) / p.H);   // (never an empty sequence)
+    const int base = tb.su[s];
+    const int ncs = max(1, (tb.su[s + 1] - base) / p.H);   // (never an empty sequence)
     const int local = u - base;
     const int h = local / ncs;
     l.chain = s * p.H + h;
@@ -244,12 +254,12 @@ __device__ inline Loc locate(const Params& p, int u, int& hint)
 
 // The (non-empty) sequence holding unit u of a ragged batch: the last s
 // with seq_units[s] <= u (binary search).
-__device__ inline int seq_of_unit(const Params& p, int u)
+__device__ inline int seq_of_unit(const Params& p, const Tabs& tb, int u)
 {
     int lo = 0, hi = p.nseq - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (__ldg(p.seq_units + mid) <= u) lo = mid;
+        if (tb.su[mid] <= u) lo = mid;
         else hi = mid - 1;
     }
     return lo;
@@ -270,18 +280,19 @@ struct Range {
     int count;
 };
 
-__device__ inline Range make_range(const Params& p, int t, int units)
+template <bool kRagged>
+__device__ inline Range make_range(const Params& p, const Tabs& tb, int t, int units)
 {
     Range r{};
     const int u0 = (int)((long long)units * t / p.nslots);
     const int u1 = (int)((long long)units * (t + 1) / p.nslots);
     if (u1 <= u0) return r;
-    int hint0 = p.cu_seqlens ? seq_of_unit(p, u0) : 0;
-    const Loc a = locate(p, u0, hint0);
+    int hint0 = kRagged ? seq_of_unit(p, tb, u0) : 0;
+    const Loc a = locate<kRagged>(p, tb, u0, hint0);
     Loc b{-1, 0, 0};   // u1 == units: the end of the list
     if (u1 < units) {
-        int hint1 = p.cu_seqlens ? seq_of_unit(p, u1) : 0;
-        b = locate(p, u1, hint1);
+        int hint1 = kRagged ? seq_of_unit(p, tb, u1) : 0;
+        b = locate<kRagged>(p, tb, u1, hint1);
     }
     if (a.chunk > 0 && b.chain == a.chain) {   // inside one chain
         r.chC = a.chain;
@@ -300,7 +311,7 @@ __device__ inline Range make_range(const Params& p, int t, int units)
     }
     r.uB0 = a.chunk > 0 ? u0 + (a.ncc - a.chunk) : u0;
     r.nB = (u1 - b.chunk) - r.uB0;
-    r.sB0 = p.cu_seqlens && r.nB > 0 ? seq_of_unit(p, r.uB0) : 0;
+    r.sB0 = kRagged && r.nB > 0 ? seq_of_unit(p, tb, r.uB0) : 0;
     r.count = r.lenA + r.nB + r.lenC;
     return r;
 }
@@ -315,7 +326,8 @@ struct Item {
     bool direct_y;     // y written row by row (a ragged batch's last, partial chunk)
 };
 
-__device__ inline Item item_at(const Params& p, const Range& r, int idx, int& hint)
+template <bool kRagged>
+__device__ inline Item item_at(const Params& p, const Tabs& tb, const Range& r, int idx, int& hint)
 {
     Item it;
     if (idx < r.lenA) {
@@ -326,7 +338,7 @@ __device__ inline Item item_at(const Params& p, const Range& r, int idx, int& hi
         it.publish = it.seg_end;
         it.depend = false;
     } else if (idx - r.lenA < r.nB) {
-        const Loc l = locate(p, r.uB0 + (idx - r.lenA), hint);
+        const Loc l = locate<kRagged>(p, tb, r.uB0 + (idx - r.lenA), hint);
         it.chain = l.chain;
         it.chunk = l.chunk;
         it.seg_start = l.chunk == 0;
@@ -344,9 +356,9 @@ __device__ inline Item item_at(const Params& p, const Range& r, int idx, int& hi
     }
     it.seq = (int)p.fH.div((uint32_t)it.chain);
     it.h = it.chain - it.seq * p.H;
-    if (p.cu_seqlens) {
-        const int s0 = __ldg(p.cu_seqlens + it.seq);
-        const int len = __ldg(p.cu_seqlens + it.seq + 1) - s0;
+    if constexpr (kRagged) {
+        const int s0 = tb.cu[it.seq];
+        const int len = tb.cu[it.seq + 1] - s0;
         it.tok0 = s0 + it.chunk * kQ;
         it.nvalid = min(kQ, len - it.chunk * kQ);
         it.bi = 0;
@@ -372,6 +384,7 @@ __device__ inline void tmem_ld8(uint32_t taddr, float (&v)[8])
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+template <bool kRagged>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY,
@@ -425,8 +438,22 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     const uint32_t tmem = *tmem_slot;
     const int ticket = *ticket_slot;
     // a ragged batch reads its unit count (0 if cu_seqlens was invalid)
-    const int units = prm.cu_seqlens ? (prm.ws_hdr[0] ? 0 : prm.ws_hdr[1]) : prm.units;
-    const Range rg = make_range(prm, ticket, units);
+    const int units = kRagged ? (prm.ws_hdr[0] ? 0 : prm.ws_hdr[1]) : prm.units;
+    Tabs tabs{prm.cu_seqlens, prm.seq_units};
+    if constexpr (kRagged) {
+        // the ragged tables into shared memory when they fit
+        if (prm.nseq <= kMaxSeqSmem && units > 0) {
+            int* scu = reinterpret_cast<int*>(smem + kOffSeq);
+            int* ssu = scu + (kMaxSeqSmem + 1);
+            for (int i = tid; i <= prm.nseq; i += kThreads) {
+                scu[i] = prm.cu_seqlens[i];
+                ssu[i] = prm.seq_units[i];
+            }
+            __syncthreads();
+            tabs = Tabs{scu, ssu};
+        }
+    }
+    const Range rg = make_range<kRagged>(prm, tabs, ticket, units);
     auto group_of = [&](const Item& it) { return (int)prm.fHG.div((uint32_t)it.h); };
     auto stage = [&](int idx) { return smem + kOffStage + (idx & 1) * kStageBytes; };
 
@@ -495,7 +522,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             // each call site visits items in increasing order and keeps its own hint
             int hint_bc = rg.sB0, hint_x = rg.sB0, hint_pf = rg.sB0, hint_st = rg.sB0;
             auto issue_bc = [&](int idx) {
-                const Item it = item_at(prm, rg, idx, hint_bc);
+                const Item it = item_at<kRagged>(prm, tabs, rg, idx, hint_bc);
                 const int g = group_of(it);
                 uint8_t* st = stage(idx);
                 uint64_t* bar = bar_ld + (idx & 1);
@@ -507,13 +534,13 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             };
             // X of item idx into its stage (the buffer that held y of item idx - 2)
             auto issue_x = [&](int idx) {
-                const Item it = item_at(prm, rg, idx, hint_x);
+                const Item it = item_at<kRagged>(prm, tabs, rg, idx, hint_x);
                 uint64_t* bar = bar_ldx + (idx & 1);
                 mbar_arrive_expect_tx(bar, kBytesX);
                 tma_load_3d(stage(idx) + kStX, &tmX, it.h * kP, it.tok0, it.bi, bar);
             };
             auto prefetch_l2 = [&](int idx) {
-                const Item it = item_at(prm, rg, idx, hint_pf);
+                const Item it = item_at<kRagged>(prm, tabs, rg, idx, hint_pf);
                 const int g = group_of(it);
                 tma_prefetch_l2_3d(&tmB, g * kN, it.tok0, it.bi);
                 tma_prefetch_l2_3d(&tmB, g * kN + 64, it.tok0, it.bi);
@@ -540,7 +567,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 // y of item idx is staged in its X buffer: store it, then
                 // reload the buffer once the store has read it
                 mbar_wait_bounded(bar_ystaged + (idx & 1), sph, kWaitNs, aborted, prm.status);
-                const Item it = item_at(prm, rg, idx, hint_st);
+                const Item it = item_at<kRagged>(prm, tabs, rg, idx, hint_st);
                 if (!it.direct_y) {   // (a partial ragged chunk's rows went out directly)
                     tma_store_3d(&tmY, stage(idx) + kStX, it.h * kP, it.tok0, it.bi);
                     bulk_commit_group();
@@ -568,7 +595,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         int hint = rg.sB0;
         auto load_dt = [&](int idx) {
             DtIn in;
-            const Item it = item_at(prm, rg, idx, hint);
+            const Item it = item_at<kRagged>(prm, tabs, rg, idx, hint);
             in.a2 = prm.A[it.h] * 1.4426950408889634f;   // A * log2(e)
             in.bias = prm.dt_bias ? prm.dt_bias[it.h] : 0.0f;
             const __nv_bfloat16* dp = prm.dt_raw + ((size_t)it.bi * L + it.tok0 + lane * 4) * H + it.h;
@@ -681,7 +708,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         // is in Yd through M's diagonal), written over x in the item's X
         // buffer for the producer's TMA store.  M X of item j (the X
         // buffer's last reader) is done once bar_m2 has completed for it.
-        auto y_epilogue = [&](int j, float cl_i, const Item& itj) {
+        int hint_y = rg.sB0;   // the epilogue visits items in increasing order too
+        auto y_epilogue = [&](int j, float cl_i) {
             mbar_wait_bounded(bar_m2, (uint32_t)j & 1u, kWaitNs, aborted, prm.status);
             tc_fence_after_sync();
             uint8_t* xs = stage(j) + kStX;
@@ -690,6 +718,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             tmem_ld16(tmem + kColYd + lane_off + (uint32_t)p0, yd);
             tmem_ld16(tmem + kColYo + (uint32_t)(j & 1) * 64u + lane_off + (uint32_t)p0, yo);
             tmem_wait_ld();
+            uint4 packed[2];
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
                 float o[8];
@@ -700,25 +729,35 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                     o[e] = r.x;
                     o[e + 1] = r.y;
                 }
-                if (!itj.direct_y) {
-                    *reinterpret_cast<uint4*>(xs + sw128(row, quarter * 2 + q)) = pack_bf16x8(o);
-                } else if (row < itj.nvalid) {
+                packed[q] = pack_bf16x8(o);
+            }
+            bool staged = true;
+            if constexpr (kRagged) {
+                const Item itj = item_at<kRagged>(prm, tabs, rg, j, hint_y);
+                if (itj.direct_y) {
                     // a ragged batch's partial last chunk: its rows past the
                     // sequence's end belong to the next sequence, so the rows
                     // go out one by one instead of as a 128-row TMA box
-                    __nv_bfloat16* yr = prm.y + ((size_t)(itj.tok0 + row) * H + itj.h) * kP + p0 + q * 8;
-                    *reinterpret_cast<uint4*>(yr) = pack_bf16x8(o);
+                    staged = false;
+                    if (row < itj.nvalid) {
+                        __nv_bfloat16* yr = prm.y + ((size_t)(itj.tok0 + row) * H + itj.h) * kP + p0;
+                        reinterpret_cast<uint4*>(yr)[0] = packed[0];
+                        reinterpret_cast<uint4*>(yr)[1] = packed[1];
+                    }
                 }
+            }
+            if (staged) {
+#pragma unroll
+                for (int q = 0; q < 2; ++q) *reinterpret_cast<uint4*>(xs + sw128(row, quarter * 2 + q)) = packed[q];
             }
             fence_proxy_async_smem();
             mbar_arrive(bar_ystaged + (j & 1));
         };
 
         float prev_cl_i = 0.0f;
-        Item prev_it{};
         int hint = rg.sB0;
         for (int idx = 0; idx < rg.count; ++idx) {
-            const Item it = item_at(prm, rg, idx, hint);
+            const Item it = item_at<kRagged>(prm, tabs, rg, idx, hint);
             const int bi = it.seq, h = it.h;
             const float Dh = prm.D ? prm.D[h] : 0.0f;
             uint8_t* st = stage(idx);
@@ -779,7 +818,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             mbar_arrive(bar_sready);   // C h^T and the state update can start
 
             // 4. y of the previous item, whose M X ran meanwhile
-            if (idx > 0) y_epilogue(idx - 1, prev_cl_i, prev_it);
+            if (idx > 0) y_epilogue(idx - 1, prev_cl_i);
 
             // 5. the masked tile M = G o L of item idx into TMEM (bf16
             //    pairs), the A operand of M X.  Column block jb (32 tokens)
@@ -859,9 +898,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 }
             }
             prev_cl_i = cl_i;
-            prev_it = it;
         }
-        if (rg.count > 0) y_epilogue(rg.count - 1, prev_cl_i, prev_it);
+        if (rg.count > 0) y_epilogue(rg.count - 1, prev_cl_i);
     }
 
     tc_fence_before_sync();
@@ -944,7 +982,8 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t s)
     if ((e = make_map(&tmC, a.C, (uint64_t)a.G * a.N, a.L, a.b, rb)) != cudaSuccess) return e;
     CUtensorMap tmY;
     if ((e = make_map(&tmY, a.y, (uint64_t)a.H * a.P, a.L, a.b, (uint64_t)a.H * a.P * 2)) != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(chunk_scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    auto kernel = a.cu_seqlens ? chunk_scan_tc_kernel<true> : chunk_scan_tc_kernel<false>;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     const int slots = tc_slots(a);
     const size_t ctrl = kWsCtrlBytes(slots);
@@ -987,7 +1026,7 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t s)
     prm.ws_hdr = ragged ? reinterpret_cast<const int*>(ws) : nullptr;
     prm.nseq = ragged ? a.nseq : a.b;
     prm.status = a.status;
-    chunk_scan_tc_kernel<<<slots, kThreads, kSmemBytes, s>>>(tmX, tmB, tmC, tmY, prm);
+    kernel<<<slots, kThreads, kSmemBytes, s>>>(tmX, tmB, tmC, tmY, prm);
     return cudaGetLastError();
 }
 
