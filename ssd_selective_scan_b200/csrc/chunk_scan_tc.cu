@@ -518,63 +518,75 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         // producer warp (one thread): TMA loads, L2 prefetches and y stores
         // ------------------------------------------------------------------
         if (lane == 0 && rg.count > 0) {
+            // The coordinates of an item, computed once (for its L2
+            // prefetch) and passed along a rotation of items idx .. idx + 3.
+            struct Co {
+                int g, h, tok0, bi;
+                bool direct_y;
+            };
+            int hint = rg.sB0;   // items are visited in increasing order
+            auto coord = [&](int idx) {
+                Co c{0, 0, 0, 0, false};
+                if (idx < rg.count) {
+                    const Item it = item_at<kRagged>(prm, tabs, rg, idx, hint);
+                    c = Co{group_of(it), it.h, it.tok0, it.bi, it.direct_y};
+                }
+                return c;
+            };
             // B and C of item idx into its stage (G = C B^T needs only these)
-            // each call site visits items in increasing order and keeps its own hint
-            int hint_bc = rg.sB0, hint_x = rg.sB0, hint_pf = rg.sB0, hint_st = rg.sB0;
-            auto issue_bc = [&](int idx) {
-                const Item it = item_at<kRagged>(prm, tabs, rg, idx, hint_bc);
-                const int g = group_of(it);
+            auto issue_bc = [&](int idx, const Co& c) {
                 uint8_t* st = stage(idx);
                 uint64_t* bar = bar_ld + (idx & 1);
                 mbar_arrive_expect_tx(bar, kBytesBC);
-                tma_load_3d(st + kStB, &tmB, g * kN, it.tok0, it.bi, bar);
-                tma_load_3d(st + kStB + kTileHalf, &tmB, g * kN + 64, it.tok0, it.bi, bar);
-                tma_load_3d(st + kStC, &tmC, g * kN, it.tok0, it.bi, bar);
-                tma_load_3d(st + kStC + kTileHalf, &tmC, g * kN + 64, it.tok0, it.bi, bar);
+                tma_load_3d(st + kStB, &tmB, c.g * kN, c.tok0, c.bi, bar);
+                tma_load_3d(st + kStB + kTileHalf, &tmB, c.g * kN + 64, c.tok0, c.bi, bar);
+                tma_load_3d(st + kStC, &tmC, c.g * kN, c.tok0, c.bi, bar);
+                tma_load_3d(st + kStC + kTileHalf, &tmC, c.g * kN + 64, c.tok0, c.bi, bar);
             };
             // X of item idx into its stage (the buffer that held y of item idx - 2)
-            auto issue_x = [&](int idx) {
-                const Item it = item_at<kRagged>(prm, tabs, rg, idx, hint_x);
+            auto issue_x = [&](int idx, const Co& c) {
                 uint64_t* bar = bar_ldx + (idx & 1);
                 mbar_arrive_expect_tx(bar, kBytesX);
-                tma_load_3d(stage(idx) + kStX, &tmX, it.h * kP, it.tok0, it.bi, bar);
+                tma_load_3d(stage(idx) + kStX, &tmX, c.h * kP, c.tok0, c.bi, bar);
             };
-            auto prefetch_l2 = [&](int idx) {
-                const Item it = item_at<kRagged>(prm, tabs, rg, idx, hint_pf);
-                const int g = group_of(it);
-                tma_prefetch_l2_3d(&tmB, g * kN, it.tok0, it.bi);
-                tma_prefetch_l2_3d(&tmB, g * kN + 64, it.tok0, it.bi);
-                tma_prefetch_l2_3d(&tmC, g * kN, it.tok0, it.bi);
-                tma_prefetch_l2_3d(&tmC, g * kN + 64, it.tok0, it.bi);
-                tma_prefetch_l2_3d(&tmX, it.h * kP, it.tok0, it.bi);
+            auto prefetch_l2 = [&](const Co& c) {
+                tma_prefetch_l2_3d(&tmB, c.g * kN, c.tok0, c.bi);
+                tma_prefetch_l2_3d(&tmB, c.g * kN + 64, c.tok0, c.bi);
+                tma_prefetch_l2_3d(&tmC, c.g * kN, c.tok0, c.bi);
+                tma_prefetch_l2_3d(&tmC, c.g * kN + 64, c.tok0, c.bi);
+                tma_prefetch_l2_3d(&tmX, c.h * kP, c.tok0, c.bi);
             };
             prefetch_tensormap(&tmX);
             prefetch_tensormap(&tmB);
             prefetch_tensormap(&tmC);
             prefetch_tensormap(&tmY);
-            issue_bc(0);
-            issue_x(0);
+            Co c0 = coord(0), c1 = coord(1), c2 = coord(2), c3 = coord(3);   // items idx .. idx + 3
+            issue_bc(0, c0);
+            issue_x(0, c0);
             if (rg.count > 1) {
-                issue_bc(1);
-                issue_x(1);
+                issue_bc(1, c1);
+                issue_x(1, c1);
             }
-            if (rg.count > 2) prefetch_l2(2);
+            if (rg.count > 2) prefetch_l2(c2);
             for (int idx = 0; idx < rg.count; ++idx) {
                 const uint32_t sph = (uint32_t)(idx >> 1) & 1u;   // per-stage barrier parity
                 // the state update, the last MMA reading B and C of item idx, is done
                 mbar_wait_bounded(bar_m4 + (idx & 1), sph, kWaitNs, aborted, prm.status);
-                if (idx + 2 < rg.count) issue_bc(idx + 2);
+                if (idx + 2 < rg.count) issue_bc(idx + 2, c2);
                 // y of item idx is staged in its X buffer: store it, then
                 // reload the buffer once the store has read it
                 mbar_wait_bounded(bar_ystaged + (idx & 1), sph, kWaitNs, aborted, prm.status);
-                const Item it = item_at<kRagged>(prm, tabs, rg, idx, hint_st);
-                if (!it.direct_y) {   // (a partial ragged chunk's rows went out directly)
-                    tma_store_3d(&tmY, stage(idx) + kStX, it.h * kP, it.tok0, it.bi);
+                if (!c0.direct_y) {   // (a partial ragged chunk's rows went out directly)
+                    tma_store_3d(&tmY, stage(idx) + kStX, c0.h * kP, c0.tok0, c0.bi);
                     bulk_commit_group();
                     bulk_wait_group_read0();
                 }
-                if (idx + 2 < rg.count) issue_x(idx + 2);
-                if (idx + 3 < rg.count) prefetch_l2(idx + 3);
+                if (idx + 2 < rg.count) issue_x(idx + 2, c2);
+                if (idx + 3 < rg.count) prefetch_l2(c3);
+                c0 = c1;
+                c1 = c2;
+                c2 = c3;
+                c3 = coord(idx + 4);
             }
             bulk_wait_group0();   // all y stores complete before the CTA exits
         }
@@ -708,7 +720,9 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         // is in Yd through M's diagonal), written over x in the item's X
         // buffer for the producer's TMA store.  M X of item j (the X
         // buffer's last reader) is done once bar_m2 has completed for it.
-        int hint_y = rg.sB0;   // the epilogue visits items in increasing order too
+        // the previous item's row placement (ragged batches only)
+        int prev_tok0 = 0, prev_nvalid = 0, prev_h = 0;
+        bool prev_direct = false;
         auto y_epilogue = [&](int j, float cl_i) {
             mbar_wait_bounded(bar_m2, (uint32_t)j & 1u, kWaitNs, aborted, prm.status);
             tc_fence_after_sync();
@@ -733,14 +747,13 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             }
             bool staged = true;
             if constexpr (kRagged) {
-                const Item itj = item_at<kRagged>(prm, tabs, rg, j, hint_y);
-                if (itj.direct_y) {
+                if (prev_direct) {
                     // a ragged batch's partial last chunk: its rows past the
                     // sequence's end belong to the next sequence, so the rows
                     // go out one by one instead of as a 128-row TMA box
                     staged = false;
-                    if (row < itj.nvalid) {
-                        __nv_bfloat16* yr = prm.y + ((size_t)(itj.tok0 + row) * H + itj.h) * kP + p0;
+                    if (row < prev_nvalid) {
+                        __nv_bfloat16* yr = prm.y + ((size_t)(prev_tok0 + row) * H + prev_h) * kP + p0;
                         reinterpret_cast<uint4*>(yr)[0] = packed[0];
                         reinterpret_cast<uint4*>(yr)[1] = packed[1];
                     }
@@ -898,6 +911,12 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 }
             }
             prev_cl_i = cl_i;
+            if constexpr (kRagged) {
+                prev_tok0 = it.tok0;
+                prev_nvalid = it.nvalid;
+                prev_h = it.h;
+                prev_direct = it.direct_y;
+            }
         }
         if (rg.count > 0) y_epilogue(rg.count - 1, prev_cl_i);
     }
