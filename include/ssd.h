@@ -239,6 +239,43 @@ SSD_API ssd_status_t ssd_chunk_scan_fwd_varlen(const void* x, const void* B, con
                                                cudaStream_t stream);
 
 /*
+ * Fused prefill: ssd_conv1d_silu, then ssd_chunk_scan_fwd on its output, as
+ * one call that does not write the conv output to memory.  In the Mamba-2
+ * layer the conv (width 4, SiLU) feeds the scan directly (Nemotron
+ * feasibility report, section 1.4; the conv cache of "Hybrid Architectures
+ * for Language Models", summary page, appendix C).  Results equal those of
+ * the two calls; on the tensor-core path bit for bit.
+ *
+ *   xBC        [b][L][conv_dim]   dtype, conv_dim = H*P + 2*G*N, channels
+ *                                 x | B | C; read only
+ *   w, bias, conv_state           as for ssd_conv1d_silu (conv_state, if
+ *                                 given, is read and rewritten in place)
+ *   dt_raw, dt_bias, A, D, init_state, y, final_state, status
+ *                                 as for ssd_chunk_scan_fwd
+ *   workspace  at least ssd_conv_scan_workspace_bytes(...) bytes of device
+ *              scratch, caller-owned, no initial contents required
+ * Paths: with bf16, P = 64, N = 128, Q = 128 and k = 4 the conv of the B
+ * and C channels goes to the workspace (2*G*N elements per token) and the x
+ * channels are convolved inside the tensor-core scan kernel as their tiles
+ * arrive (two launches, the conv output of x never leaves the chip).  Other
+ * shapes run the conv into the workspace (conv_dim elements per token), then
+ * the scan.
+ * Requirements: those of both calls; y must not overlap xBC, conv_state or
+ * the workspace.
+ */
+SSD_API size_t ssd_conv_scan_workspace_bytes(int b, int L, int H, int P, int N, int G, int Q,
+                                             int k, ssd_dtype_t dtype);
+
+SSD_API ssd_status_t ssd_conv_scan_fwd(const void* xBC, const float* w, const float* bias,
+                                       void* conv_state, const void* dt_raw,
+                                       const float* dt_bias, const float* A, const float* D,
+                                       const float* init_state, void* y, float* final_state,
+                                       int b, int L, int H, int P, int N, int G, int Q, int k,
+                                       ssd_dtype_t dtype, void* workspace,
+                                       size_t workspace_bytes, int32_t* status,
+                                       cudaStream_t stream);
+
+/*
  * Single-token decode update, in place on the float32 state:
  *
  *   dt = softplus(dt_raw + dt_bias); h <- exp(dt*A) h + dt x B^T;

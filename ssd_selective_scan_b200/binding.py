@@ -41,6 +41,9 @@ SIGNATURES = {
     "ssd_chunk_scan_varlen_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i]),
     "ssd_chunk_scan_fwd_varlen": (_i, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                        _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp, _vp]),
+    "ssd_conv_scan_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),
+    "ssd_conv_scan_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                               _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp, _vp]),
 }
 
 _lock = threading.Lock()
@@ -117,6 +120,17 @@ def ssd_chunk_scan_fwd_varlen(x, B, C, row_stride, dt_raw, dt_bias, A, D, init_s
     return load().ssd_chunk_scan_fwd_varlen(x, B, C, row_stride, dt_raw, dt_bias, A, D, init_state, y,
                                             final_state, cu_seqlens, nseq, T, H, P, N, G, Q, dtype,
                                             workspace, workspace_bytes, status, stream)
+
+
+def ssd_conv_scan_workspace_bytes(b, L, H, P, N, G, Q, k, dtype) -> int:
+    return load().ssd_conv_scan_workspace_bytes(b, L, H, P, N, G, Q, k, dtype)
+
+
+def ssd_conv_scan_fwd(xBC, w, bias, conv_state, dt_raw, dt_bias, A, D, init_state, y, final_state,
+                      b, L, H, P, N, G, Q, k, dtype, workspace, workspace_bytes, status, stream) -> int:
+    return load().ssd_conv_scan_fwd(xBC, w, bias, conv_state, dt_raw, dt_bias, A, D, init_state, y,
+                                    final_state, b, L, H, P, N, G, Q, k, dtype, workspace,
+                                    workspace_bytes, status, stream)
 
 
 def ssd_selftest_bounded_wait(status, limit_ns, stream) -> int:

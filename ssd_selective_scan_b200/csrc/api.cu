@@ -42,6 +42,17 @@ int max_optin_smem()
     return v;
 }
 
+size_t round_up_256(size_t n) { return (n + 255) / 256 * 256; }
+
+// the fused tensor-core path: bf16, P = 64, N = 128, Q = 128, conv width 4
+bool conv_scan_fused(int H, int P, int N, int G, int Q, int k, ssd_dtype_t dtype)
+{
+    ScanArgs a{};
+    a.b = 1; a.L = 1; a.H = H; a.P = P; a.N = N; a.G = G; a.Q = Q;
+    a.bf16 = dtype == SSD_BF16;
+    return k == 4 && ssd::chunk_scan_tc_supported(a);
+}
+
 }  // namespace
 
 extern "C" {
@@ -232,6 +243,103 @@ ssd_status_t ssd_chunk_scan_fwd_varlen(const void* x, const void* B, const void*
     if (ssd::chunk_scan_tc_supported(a)) return from_cuda(ssd::launch_chunk_scan_tc(a, stream));
     if (ssd::chunk_scan_simt_smem_bytes(P, N) > (size_t)max_optin_smem()) return SSD_ERR_UNSUPPORTED;
     return from_cuda(ssd::launch_chunk_scan_simt(a, stream));
+}
+
+size_t ssd_conv_scan_workspace_bytes(int b, int L, int H, int P, int N, int G, int Q, int k,
+                                     ssd_dtype_t dtype)
+{
+    if (b <= 0 || L <= 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || k <= 0 || !valid_dtype(dtype)) return 0;
+    const size_t per_token = conv_scan_fused(H, P, N, G, Q, k, dtype) ? (size_t)2 * G * N : (size_t)H * P + 2 * (size_t)G * N;
+    return round_up_256((size_t)b * L * per_token * elem_bytes(dtype)) +
+           ssd_chunk_scan_workspace_bytes(b, L, H, P, N, G, Q, dtype);
+}
+
+ssd_status_t ssd_conv_scan_fwd(const void* xBC, const float* w, const float* bias, void* conv_state,
+                               const void* dt_raw, const float* dt_bias, const float* A, const float* D,
+                               const float* init_state, void* y, float* final_state, int b, int L, int H,
+                               int P, int N, int G, int Q, int k, ssd_dtype_t dtype, void* workspace,
+                               size_t workspace_bytes, int32_t* status, cudaStream_t stream)
+{
+    if (!valid_dtype(dtype) || b < 0 || L < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || k <= 0)
+        return SSD_ERR_INVALID_ARG;
+    if (H % G || P % 8 || N % 8 || (Q != 64 && Q != 128)) return SSD_ERR_INVALID_ARG;
+    if ((int64_t)H * P + 2 * (int64_t)G * N > 0x7fffffffLL) return SSD_ERR_INVALID_ARG;
+    const int conv_dim = H * P + 2 * G * N;   // a multiple of 8: 16-byte rows for either dtype
+    if (b == 0 || L == 0) {
+        // no tokens: the conv cache is unchanged and the scan's rule for
+        // empty sequences applies (final state = initial state)
+        if (k > 4 || k < 2) return SSD_ERR_UNSUPPORTED;
+        return ssd_chunk_scan_fwd(nullptr, nullptr, nullptr, conv_dim, nullptr, dt_bias, A, D, init_state, nullptr,
+                                  final_state, b, L, H, P, N, G, Q, dtype, nullptr, 0, status, stream);
+    }
+    if (!xBC || !w || !dt_raw || !A || !y) return SSD_ERR_INVALID_ARG;
+    const void* ptrs16[] = {xBC, w, conv_state, dt_raw, y, init_state, final_state, workspace};
+    for (const void* p : ptrs16)
+        if (p && !aligned(p, 16)) return SSD_ERR_INVALID_ARG;
+    if (!aligned(A, 4) || (bias && !aligned(bias, 4)) || (dt_bias && !aligned(dt_bias, 4)) || (D && !aligned(D, 4)) ||
+        (status && !aligned(status, 4)))
+        return SSD_ERR_INVALID_ARG;
+    const size_t need_ws = ssd_conv_scan_workspace_bytes(b, L, H, P, N, G, Q, k, dtype);
+    if (workspace_bytes < need_ws || !workspace) return SSD_ERR_INVALID_ARG;
+
+    const int e = elem_bytes(dtype);
+    const int64_t rows = (int64_t)b * L;
+    const Range rx = span(xBC, rows * conv_dim * e);
+    const Range rw = span(w, (int64_t)conv_dim * k * 4);
+    const Range rcs = span(conv_state, conv_state ? (int64_t)b * conv_dim * k * e : 0);
+    const Range rdt = span(dt_raw, rows * H * e);
+    const Range ry = span(y, rows * H * P * e);
+    const int64_t st_bytes = (int64_t)b * H * P * N * 4;
+    const Range ri = span(init_state, init_state ? st_bytes : 0);
+    const Range rf = span(final_state, final_state ? st_bytes : 0);
+    const Range rws = span(workspace, (int64_t)workspace_bytes);
+    for (Range in : {rx, rw, rcs, rdt, ri})
+        if (overlap(ry, in)) return SSD_ERR_INVALID_ARG;
+    for (Range in : {rx, rw, rcs, rdt, ry})
+        if (overlap(rf, in)) return SSD_ERR_INVALID_ARG;
+    if (final_state && init_state && final_state != init_state && overlap(rf, ri)) return SSD_ERR_INVALID_ARG;
+    for (Range in : {rx, rw, rdt, ry, ri, rf})
+        if (overlap(rcs, in)) return SSD_ERR_INVALID_ARG;
+    for (Range in : {rx, rw, rcs, rdt, ry, ri, rf})
+        if (overlap(rws, in)) return SSD_ERR_INVALID_ARG;
+    if (k < 2 || k > 4) return SSD_ERR_UNSUPPORTED;
+    if (b > 65535 || (L + 31) / 32 > 65535) return SSD_ERR_UNSUPPORTED;
+    if ((int64_t)b * H * ((L + Q - 1) / Q) > 0x7fffffffLL) return SSD_ERR_UNSUPPORTED;
+
+    const bool bf16 = dtype == SSD_BF16;
+    const int GN = G * N, HP = H * P;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const uint8_t* xb = static_cast<const uint8_t*>(xBC);
+    if (conv_scan_fused(H, P, N, G, Q, k, dtype)) {
+        // B and C convolved into the workspace, x inside the scan kernel
+        const size_t bc_bytes = round_up_256((size_t)rows * 2 * GN * e);
+        ssd::ConvSlice c{xb + (size_t)HP * e, conv_dim, ws, 2 * GN, w + (size_t)HP * k, bias ? bias + HP : nullptr,
+                         conv_state ? static_cast<uint8_t*>(conv_state) + (size_t)HP * k * e : nullptr,
+                         (int64_t)conv_dim * k, b, L, 2 * GN, k, bf16};
+        const ssd_status_t st = from_cuda(ssd::launch_conv1d_silu_slice(c, stream));
+        if (st != SSD_OK) return st;
+        ScanArgs a{xBC, ws, ws + (size_t)GN * e, conv_dim, dt_raw, dt_bias, A, D, init_state, y, final_state,
+                   b, L, H, P, N, G, Q, bf16, ws + bc_bytes, workspace_bytes - bc_bytes, status};
+        a.bc_row_stride = 2 * GN;
+        a.conv_w = w;
+        a.conv_bias = bias;
+        a.conv_state = conv_state;
+        return from_cuda(ssd::launch_chunk_scan_tc(a, stream));
+    }
+    // the conv output into the workspace, then the scan on its channel ranges
+    ScanArgs a{nullptr, nullptr, nullptr, conv_dim, dt_raw, dt_bias, A, D, init_state, y, final_state,
+               b, L, H, P, N, G, Q, bf16, nullptr, 0, status};
+    const bool tc = ssd::chunk_scan_tc_supported(a);
+    if (!tc && ssd::chunk_scan_simt_smem_bytes(P, N) > (size_t)max_optin_smem()) return SSD_ERR_UNSUPPORTED;
+    const size_t u_bytes = round_up_256((size_t)rows * conv_dim * e);
+    const ssd_status_t st = from_cuda(ssd::launch_conv1d_silu(xBC, ws, w, bias, conv_state, b, L, conv_dim, k, bf16, stream));
+    if (st != SSD_OK) return st;
+    a.x = ws;
+    a.B = ws + (size_t)HP * e;
+    a.C = ws + (size_t)(HP + GN) * e;
+    a.workspace = ws + u_bytes;
+    a.workspace_bytes = workspace_bytes - u_bytes;
+    return from_cuda(tc ? ssd::launch_chunk_scan_tc(a, stream) : ssd::launch_chunk_scan_simt(a, stream));
 }
 
 ssd_status_t ssd_state_update(float* state, const void* x, const void* B, const void* C,

@@ -204,14 +204,63 @@ def split_channels(u: torch.Tensor, H: int, P: int, G: int, N: int):
     return x, B, C
 
 
+def conv_scan_workspace_bytes(b, L, H, P, N, G, Q, k, dtype: torch.dtype) -> int:
+    return int(libssd.ssd_conv_scan_workspace_bytes(b, L, H, P, N, G, Q, k, _DT[dtype]))
+
+
+def conv_scan_fwd(xBC: torch.Tensor, w: torch.Tensor, dt_raw: torch.Tensor, A: torch.Tensor,
+                  H: int, P: int, G: int, N: int, *, bias: torch.Tensor | None = None,
+                  conv_state: torch.Tensor | None = None, dt_bias: torch.Tensor | None = None,
+                  D: torch.Tensor | None = None, init_state: torch.Tensor | None = None,
+                  Q: int = 128, y: torch.Tensor | None = None,
+                  final_state: torch.Tensor | bool | None = True,
+                  workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                  stream=None):
+    """Fused prefill: conv1d+SiLU of xBC [b, L, conv_dim], then the chunked
+    scan of its x | B | C channels, without writing the conv output.  w
+    [conv_dim, k] f32; conv_state [b, conv_dim, k] (I/O dtype) is updated in
+    place.  Returns (y [b, L, H, P], final_state [b, H, P, N] f32 or None)."""
+    if xBC.dim() != 3 or not xBC.is_contiguous():
+        raise ValueError("xBC must be a contiguous [b, L, conv_dim] tensor")
+    b, L, cd = xBC.shape
+    if cd != H * P + 2 * G * N:
+        raise ValueError(f"xBC has {cd} channels, expected H*P + 2*G*N = {H * P + 2 * G * N}")
+    k = w.shape[1]
+    if w.shape != (cd, k):
+        raise ValueError("w must be [conv_dim, k]")
+    if conv_state is not None and (conv_state.shape != (b, cd, k) or conv_state.dtype != xBC.dtype
+                                   or not conv_state.is_contiguous()):
+        raise ValueError("conv_state must be a contiguous [b, conv_dim, k] tensor of xBC's dtype")
+    if dt_raw.dtype != xBC.dtype or dt_raw.shape != (b, L, H) or not dt_raw.is_contiguous():
+        raise ValueError("dt_raw must be a contiguous [b, L, H] tensor of xBC's dtype")
+    if y is None:
+        y = torch.empty((b, L, H, P), dtype=xBC.dtype, device=xBC.device)
+    if final_state is True:
+        final_state = torch.empty((b, H, P, N), dtype=torch.float32, device=xBC.device)
+    elif final_state is False:
+        final_state = None
+    need = conv_scan_workspace_bytes(b, L, H, P, N, G, Q, k, xBC.dtype)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=xBC.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = libssd.ssd_conv_scan_fwd(
+        _ptr(xBC), _ptr(_f32(w, "w")), _ptr(_f32(bias, "bias")), _ptr(conv_state), _ptr(dt_raw),
+        _ptr(_f32(dt_bias, "dt_bias")), _ptr(_f32(A, "A")), _ptr(_f32(D, "D")),
+        _ptr(_f32(init_state, "init_state")), _ptr(y), _ptr(final_state), b, L, H, P, N, G, Q, k,
+        _dtype_code(xBC), _ptr(workspace), ws_bytes, _ptr(status), _stream(stream))
+    libssd.check("ssd_conv_scan_fwd", st)
+    return y, final_state
+
+
 def layer_prefill(xBC, w, dt_raw, A, H, P, G, N, *, bias=None, conv_state=None, dt_bias=None,
-                  D=None, init_state=None, Q=128, u=None, y=None, final_state=True, stream=None):
-    """conv1d+SiLU then the chunked scan on the same stream.
-    Returns (y, final_state); conv_state, if given, is updated in place."""
-    u = conv1d_silu(xBC, w, bias, conv_state, out=u, stream=stream)
-    x, B, C = split_channels(u, H, P, G, N)
-    return chunk_scan_fwd(x, B, C, dt_raw, A, dt_bias, D, init_state, Q=Q, y=y,
-                          final_state=final_state, stream=stream)
+                  D=None, init_state=None, Q=128, y=None, final_state=True, workspace=None,
+                  stream=None):
+    """The prefill layer (conv1d+SiLU, then the chunked scan) through the
+    fused call.  Returns (y, final_state); conv_state, if given, is updated
+    in place."""
+    return conv_scan_fwd(xBC, w, dt_raw, A, H, P, G, N, bias=bias, conv_state=conv_state,
+                         dt_bias=dt_bias, D=D, init_state=init_state, Q=Q, y=y,
+                         final_state=final_state, workspace=workspace, stream=stream)
 
 
 def decode_step(xBC, w, conv_state, state, dt_raw, A, H, P, G, N, *, bias=None, dt_bias=None,

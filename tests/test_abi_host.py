@@ -35,7 +35,8 @@ def test_header_declares_the_entry_points():
     assert declared_entry_points() == sorted([
         "ssd_abi_version", "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_static",
         "ssd_chunk_scan_fwd_varlen", "ssd_chunk_scan_varlen_workspace_bytes",
-        "ssd_chunk_scan_workspace_bytes", "ssd_conv1d_silu", "ssd_selftest_bounded_wait",
+        "ssd_chunk_scan_workspace_bytes", "ssd_conv1d_silu", "ssd_conv_scan_fwd",
+        "ssd_conv_scan_workspace_bytes", "ssd_selftest_bounded_wait",
         "ssd_state_update", "ssd_status_string"])
 
 
@@ -182,3 +183,35 @@ def test_varlen_validation():
     # the fp32 path needs only the unit table
     assert libssd.ssd_chunk_scan_varlen_workspace_bytes(3, 500, 4, 64, 16, 1, 64, F32) == 256 + 256 * 0 + 256
     assert libssd.ssd_chunk_scan_varlen_workspace_bytes(0, 0, 4, 64, 16, 1, 64, F32) == 0
+
+
+def cs(**kw):
+    a = dict(xBC=fake(1), w=fake(2), bias=None, conv_state=None, dt_raw=fake(3), dt_bias=None,
+             A=fake(4), D=None, init_state=None, y=fake(5), final_state=fake(6), b=2, L=256, H=40,
+             P=64, N=128, G=8, Q=128, k=4, dtype=BF16, workspace=fake(7), workspace_bytes=1 << 30,
+             status=None, stream=None)
+    a.update(kw)
+    return libssd.ssd_conv_scan_fwd(**a)
+
+
+def test_conv_scan_validation():
+    # every call here fails validation (or is empty work) before any launch
+    assert cs(b=0, xBC=None, y=None, dt_raw=None, final_state=None) == OK   # nothing to do
+    for k in ("xBC", "w", "dt_raw", "A", "y"):
+        assert cs(**{k: None}) == INV, k
+    assert cs(workspace=None) == INV and cs(workspace_bytes=16) == INV
+    assert cs(H=40, G=7) == INV and cs(P=60) == INV and cs(Q=96) == INV and cs(dtype=5) == INV
+    assert cs(xBC=fake(1, 8)) == INV and cs(conv_state=fake(8, 4)) == INV   # misaligned
+    assert cs(y=fake(1, 64)) == INV                                    # y overlaps xBC
+    assert cs(conv_state=fake(5, 16)) == INV                           # cache overlaps y
+    assert cs(workspace=fake(6)) == INV                                # workspace overlaps final state
+    assert cs(final_state=fake(3, 64)) == INV                          # final state overlaps dt_raw
+    assert cs(k=5) == UNS and cs(k=1) == UNS
+    # the fused tensor-core path keeps B and C only (2 G N per token); others the whole conv output
+    fused = libssd.ssd_conv_scan_workspace_bytes(2, 256, 40, 64, 128, 8, 128, 4, BF16)
+    scan = libssd.ssd_chunk_scan_workspace_bytes(2, 256, 40, 64, 128, 8, 128, BF16)
+    assert fused == 2 * 256 * 2 * 8 * 128 * 2 + scan
+    assert libssd.ssd_conv_scan_workspace_bytes(2, 256, 40, 64, 128, 8, 128, 3, BF16) == \
+        2 * 256 * 4608 * 2 + scan
+    assert libssd.ssd_conv_scan_workspace_bytes(1, 256, 4, 64, 16, 1, 64, 4, F32) == 256 * 288 * 4
+    assert libssd.ssd_conv_scan_workspace_bytes(0, 256, 4, 64, 16, 1, 64, 4, F32) == 0
