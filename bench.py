@@ -13,9 +13,10 @@ JSON line.  Next to the headline prefill number the line carries:
   scan_only     tokens/s of the scan kernel alone;
   decode        one decode step of the 256-sequence, 128-head workload
                 (conv-cache roll + state update), state-update GB/s;
-  e2e           the same prefill step through the public API with the step's
-                inputs copied from pinned host memory and y + final state
-                copied back, inside the timed region;
+  e2e           the same prefill step through the public one-call entry point
+                (ssd_conv_scan_fwd) with the step's inputs copied from pinned
+                host memory and y + final state copied back, inside the timed
+                region;
   cpu_baseline  the fp64 oracle timed on this host's cores on a bounded sample.
 Multi-GPU: one process per GPU (torchrun); each rank runs its own batch
 (independent sequences, no data-path collective): weak scaling.
@@ -203,6 +204,8 @@ class PrefillStep:
         self.views = layer.split_channels(self.u, s.H, s.P, s.G, s.N)
         need = layer.chunk_scan_workspace_bytes(s.b, s.L, s.H, s.P, s.N, s.G, s.Q, s.torch_dtype)
         self.ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev) if need else None
+        need = layer.conv_scan_workspace_bytes(s.b, s.L, s.H, s.P, s.N, s.G, s.Q, s.k, s.torch_dtype)
+        self.ws_layer = torch.empty(need, dtype=torch.uint8, device=dev)
 
     def conv(self):
         d = self.d
@@ -217,6 +220,14 @@ class PrefillStep:
     def __call__(self):
         self.conv()
         self.scan()
+
+    def layer_call(self):
+        """The same two kernels through the one-call prefill entry point."""
+        d, s = self.d, self.s
+        self.layer.conv_scan_fwd(d["xBC"], d["w"], d["dt_raw"], d["A"], s.H, s.P, s.G, s.N,
+                                 bias=d["bias"], conv_state=self.conv_state, dt_bias=d["dt_bias"],
+                                 D=d["D"], Q=s.Q, y=self.y, final_state=self.fs,
+                                 workspace=self.ws_layer)
 
 
 class DecodeStep:
@@ -322,7 +333,7 @@ def run_ours(args, rank, world, dev):
     def e2e_step():
         step.d["xBC"].copy_(pin_x, non_blocking=True)
         step.d["dt_raw"].copy_(pin_dt, non_blocking=True)
-        step()
+        step.layer_call()
         out_y.copy_(step.y, non_blocking=True)
         out_fs.copy_(step.fs, non_blocking=True)
 

@@ -239,12 +239,12 @@ SSD_API ssd_status_t ssd_chunk_scan_fwd_varlen(const void* x, const void* B, con
                                                cudaStream_t stream);
 
 /*
- * Fused prefill: ssd_conv1d_silu, then ssd_chunk_scan_fwd on its output, as
- * one call that does not write the conv output to memory.  In the Mamba-2
- * layer the conv (width 4, SiLU) feeds the scan directly (Nemotron
- * feasibility report, section 1.4; the conv cache of "Hybrid Architectures
- * for Language Models", summary page, appendix C).  Results equal those of
- * the two calls; on the tensor-core path bit for bit.
+ * The prefill layer in one call: ssd_conv1d_silu, then ssd_chunk_scan_fwd on
+ * its output (in the Mamba-2 layer the conv, width 4 with SiLU, feeds the
+ * scan directly: Nemotron feasibility report, section 1.4; the conv cache of
+ * "Hybrid Architectures for Language Models", summary page, appendix C).
+ * The conv output goes to the caller's workspace; the results are those of
+ * the two calls, bit for bit.
  *
  *   xBC        [b][L][conv_dim]   dtype, conv_dim = H*P + 2*G*N, channels
  *                                 x | B | C; read only
@@ -253,15 +253,10 @@ SSD_API ssd_status_t ssd_chunk_scan_fwd_varlen(const void* x, const void* B, con
  *   dt_raw, dt_bias, A, D, init_state, y, final_state, status
  *                                 as for ssd_chunk_scan_fwd
  *   workspace  at least ssd_conv_scan_workspace_bytes(...) bytes of device
- *              scratch, caller-owned, no initial contents required
- * Paths: with bf16, P = 64, N = 128, Q = 128 and k = 4 the conv of the B
- * and C channels goes to the workspace (2*G*N elements per token) and the x
- * channels are convolved inside the tensor-core scan kernel as their tiles
- * arrive (two launches, the conv output of x never leaves the chip).  Other
- * shapes run the conv into the workspace (conv_dim elements per token), then
- * the scan.
- * Requirements: those of both calls; y must not overlap xBC, conv_state or
- * the workspace.
+ *              scratch (the conv output, b*L*conv_dim elements, then the
+ *              scan's workspace), caller-owned, no initial contents required
+ * Requirements: those of both calls; no output may overlap an input or the
+ * workspace.
  */
 SSD_API size_t ssd_conv_scan_workspace_bytes(int b, int L, int H, int P, int N, int G, int Q,
                                              int k, ssd_dtype_t dtype);

@@ -44,15 +44,6 @@ int max_optin_smem()
 
 size_t round_up_256(size_t n) { return (n + 255) / 256 * 256; }
 
-// the fused tensor-core path: bf16, P = 64, N = 128, Q = 128, conv width 4
-bool conv_scan_fused(int H, int P, int N, int G, int Q, int k, ssd_dtype_t dtype)
-{
-    ScanArgs a{};
-    a.b = 1; a.L = 1; a.H = H; a.P = P; a.N = N; a.G = G; a.Q = Q;
-    a.bf16 = dtype == SSD_BF16;
-    return k == 4 && ssd::chunk_scan_tc_supported(a);
-}
-
 }  // namespace
 
 extern "C" {
@@ -249,8 +240,8 @@ size_t ssd_conv_scan_workspace_bytes(int b, int L, int H, int P, int N, int G, i
                                      ssd_dtype_t dtype)
 {
     if (b <= 0 || L <= 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || k <= 0 || !valid_dtype(dtype)) return 0;
-    const size_t per_token = conv_scan_fused(H, P, N, G, Q, k, dtype) ? (size_t)2 * G * N : (size_t)H * P + 2 * (size_t)G * N;
-    return round_up_256((size_t)b * L * per_token * elem_bytes(dtype)) +
+    const size_t conv_dim = (size_t)H * P + 2 * (size_t)G * N;
+    return round_up_256((size_t)b * L * conv_dim * elem_bytes(dtype)) +
            ssd_chunk_scan_workspace_bytes(b, L, H, P, N, G, Q, dtype);
 }
 
@@ -306,27 +297,11 @@ ssd_status_t ssd_conv_scan_fwd(const void* xBC, const float* w, const float* bia
     if (b > 65535 || (L + 31) / 32 > 65535) return SSD_ERR_UNSUPPORTED;
     if ((int64_t)b * H * ((L + Q - 1) / Q) > 0x7fffffffLL) return SSD_ERR_UNSUPPORTED;
 
+    // the conv output u into the workspace, then the scan on its x | B | C
+    // channel ranges (row stride conv_dim)
     const bool bf16 = dtype == SSD_BF16;
     const int GN = G * N, HP = H * P;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    const uint8_t* xb = static_cast<const uint8_t*>(xBC);
-    if (conv_scan_fused(H, P, N, G, Q, k, dtype)) {
-        // B and C convolved into the workspace, x inside the scan kernel
-        const size_t bc_bytes = round_up_256((size_t)rows * 2 * GN * e);
-        ssd::ConvSlice c{xb + (size_t)HP * e, conv_dim, ws, 2 * GN, w + (size_t)HP * k, bias ? bias + HP : nullptr,
-                         conv_state ? static_cast<uint8_t*>(conv_state) + (size_t)HP * k * e : nullptr,
-                         (int64_t)conv_dim * k, b, L, 2 * GN, k, bf16};
-        const ssd_status_t st = from_cuda(ssd::launch_conv1d_silu_slice(c, stream));
-        if (st != SSD_OK) return st;
-        ScanArgs a{xBC, ws, ws + (size_t)GN * e, conv_dim, dt_raw, dt_bias, A, D, init_state, y, final_state,
-                   b, L, H, P, N, G, Q, bf16, ws + bc_bytes, workspace_bytes - bc_bytes, status};
-        a.bc_row_stride = 2 * GN;
-        a.conv_w = w;
-        a.conv_bias = bias;
-        a.conv_state = conv_state;
-        return from_cuda(ssd::launch_chunk_scan_tc(a, stream));
-    }
-    // the conv output into the workspace, then the scan on its channel ranges
     ScanArgs a{nullptr, nullptr, nullptr, conv_dim, dt_raw, dt_bias, A, D, init_state, y, final_state,
                b, L, H, P, N, G, Q, bf16, nullptr, 0, status};
     const bool tc = ssd::chunk_scan_tc_supported(a);

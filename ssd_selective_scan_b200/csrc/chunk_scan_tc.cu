@@ -53,17 +53,6 @@
 //
 // Token rows past the end of the sequence are zero-filled by TMA and get
 // dt = 0, so a ragged last chunk needs no special case.
-//
-// Fused prefill (kConv): the x tiles are loaded raw from the conv input xBC
-// and the elementwise warps apply the causal depthwise conv1d (width 4) and
-// SiLU to them in shared memory before anything reads them, with the same
-// arithmetic as the stand-alone conv kernel, so the result equals the
-// two-launch path bit for bit.  The 3 tokens before a chunk come from xBC
-// (L2-resident: the previous chunk just loaded them), from the conv cache at
-// a sequence's start, or are zero.  The cache's x columns are rewritten at
-// the end of each chain; B and C arrive already convolved (by the conv
-// kernel over their channels, into a compact buffer), since each group's B
-// and C serve H / G heads and convolving them once is cheaper.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -104,13 +93,6 @@ constexpr int kOffBar = kOffSeq + 8 * (kMaxSeqSmem + 1) + 8;   // mbarriers (8-b
 constexpr int kNumBars = 13;
 constexpr int kOffMisc = kOffBar + 8 * kNumBars;   // tmem slot, abort flag, ticket
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
-// The fused-conv kernel also keeps the head's conv taps and bias, and the
-// last 3 raw tokens of each chunk (the next chunk's left context).
-constexpr int kOffConvW = (kOffMisc + 16 + 15) / 16 * 16;   // float4 taps [64 p], then float bias [64 p]
-constexpr int kOffHalo = kOffConvW + 64 * 16 + 64 * 4;       // bf16 [3 tok][64 p]
-constexpr int kSmemBytesConv = kOffHalo + 3 * 128 + 1024;
-static_assert(kOffConvW % 16 == 0 && kOffHalo % 16 == 0, "vector access to the conv taps and left context");
-static_assert(kSmemBytesConv <= 232448, "shared memory per block");
 
 constexpr uint32_t kTileHalf = 16384;
 constexpr uint32_t kBytesBC = 4 * 16384;   // B and C, two halves each
@@ -229,14 +211,6 @@ struct Params {
     const int* seq_units;
     const int* ws_hdr;
     int nseq;
-    // Fused conv1d+SiLU of the x channels (dense batches): xin is the conv
-    // input xBC [b][L][conv_ld] (bf16), conv_w [conv_dim][4] and conv_bias
-    // [conv_dim] (or null) in float32, conv_state [b][conv_dim][4] (or null).
-    const __nv_bfloat16* xin;
-    int64_t conv_ld;
-    const float* conv_w;
-    const float* conv_bias;
-    __nv_bfloat16* conv_state;
 };
 
 // The unit list: chains c = s * H + h (sequence-major), each the chunks of
@@ -410,39 +384,7 @@ __device__ inline void tmem_ld8(uint32_t taddr, float (&v)[8])
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// SiLU(v) = v/2 + (v/2) tanh(v/2): the stand-alone conv kernel's bf16-output
-// form (there on packed pairs, each lane the same IEEE operations), so the
-// fused path rounds identically.
-__device__ inline float silu_half_tanh(float v)
-{
-    const float hv = v * 0.5f;
-    float t;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(hv));
-    return fmaf(hv, t, hv);
-}
-
-__device__ inline uint2 ld_shared_u2(uint32_t addr)
-{
-    uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
-    return v;
-}
-
-__device__ inline void st_shared_u2(uint32_t addr, uint2 v)
-{
-    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(v.x), "r"(v.y) : "memory");
-}
-
-__device__ inline uint32_t pack_bf16x2(float2 v)
-{
-    __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
-    return *reinterpret_cast<uint32_t*>(&h);
-}
-
-// bf16 element i (0..3) of 4 packed in a uint2, as its 16 bits
-__device__ inline uint32_t bf16_bits(uint2 q, int i) { return ((i < 2 ? q.x : q.y) >> ((i & 1) * 16)) & 0xffffu; }
-
-template <bool kRagged, bool kConv>
+template <bool kRagged>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY,
@@ -825,127 +767,6 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             mbar_arrive(bar_ystaged + (j & 1));
         };
 
-        // Fused conv1d+SiLU of an item's x tile in its stage buffer, in
-        // place.  Thread t takes tokens 4 (t / 16) .. + 3 and channels
-        // 4 (t % 16) .. + 3 of the 128 x 64 tile and needs the 3 tokens
-        // before them; all raw tokens are read before any is overwritten.
-        const int ctg = tid >> 4, ccg = tid & 15;
-        float4* sConvW = reinterpret_cast<float4*>(smem + kOffConvW);        // taps of the head's channels
-        float* sConvB = reinterpret_cast<float*>(smem + kOffConvW + 64 * 16);  // bias
-        auto conv_x = [&](const Item& it, uint8_t* xs) {
-            const int ch = it.h * kP + ccg * 4;
-            if (it.seg_start) {
-                // a new chain (head): its taps and bias into shared memory
-                // (the previous item's readers are past its last barrier)
-                if (tid < kP) {
-                    sConvW[tid] = __ldg(reinterpret_cast<const float4*>(prm.conv_w) + (size_t)it.h * kP + tid);
-                    sConvB[tid] = prm.conv_bias ? __ldg(prm.conv_bias + (size_t)it.h * kP + tid) : 0.0f;
-                }
-                named_bar_sync(kEwBarrier, kEwThreads);
-            }
-            // Row r's 8 bytes for channels 4 ccg .. + 3 sit at r * 128 +
-            // ((ccg * 8) ^ ((r & 7) * 16)).  With r = 4 ctg - 3 + j, r & 7 =
-            // ((j + 1) & 7) ^ (4 if ctg is even), so the address of row j is
-            // a per-thread base xor a constant, plus j * 128.
-            const uint32_t xbase = smem_u32(xs) + (uint32_t)(ctg * 4 - 3) * 128u;
-            const uint32_t xk = (uint32_t)(ccg * 8) ^ ((ctg & 1) ? 0u : 64u);
-            uint2 raw[7];   // tokens 4 ctg - 3 .. 4 ctg + 3, 4 channels each
-#pragma unroll
-            for (int j = 0; j < 7; ++j) {
-                if (j >= 3 || ctg > 0)
-                    raw[j] = ld_shared_u2(xbase + (uint32_t)j * 128u + (xk ^ ((uint32_t)((j + 1) & 7) << 4)));
-            }
-            uint8_t* halo = smem + kOffHalo;   // [3 tok][64 p]
-            if (ctg == 0) {
-                if (!it.seg_start) {
-                    // the previous item was this chain's previous chunk: its
-                    // last 3 raw tokens were kept
-#pragma unroll
-                    for (int j = 0; j < 3; ++j) raw[j] = *reinterpret_cast<const uint2*>(halo + j * 128 + ccg * 8);
-                } else if (it.tok0 > 0) {
-                    const __nv_bfloat16* src = prm.xin + ((size_t)it.bi * L + it.tok0 - 3) * prm.conv_ld + ch;
-#pragma unroll
-                    for (int j = 0; j < 3; ++j) raw[j] = *reinterpret_cast<const uint2*>(src + (size_t)j * prm.conv_ld);
-                } else if (prm.conv_state) {
-                    // cache column c holds token c - 4: tokens -3 .. -1 are columns 1 .. 3
-                    const __nv_bfloat16* cs = prm.conv_state + ((size_t)it.seq * prm.conv_ld + ch) * 4;
-                    uint2 q[4];
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) q[c] = *reinterpret_cast<const uint2*>(cs + c * 4);
-#pragma unroll
-                    for (int j = 0; j < 3; ++j)
-                        raw[j] = make_uint2(bf16_bits(q[0], j + 1) | (bf16_bits(q[1], j + 1) << 16),
-                                            bf16_bits(q[2], j + 1) | (bf16_bits(q[3], j + 1) << 16));
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 3; ++j) raw[j] = make_uint2(0u, 0u);
-                }
-            }
-            float wt[4][4];   // [tap][channel]
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const float4 q = sConvW[ccg * 4 + c];
-                wt[0][c] = q.x; wt[1][c] = q.y; wt[2][c] = q.z; wt[3][c] = q.w;
-            }
-            const float4 bs4 = reinterpret_cast<const float4*>(sConvB)[ccg];
-            const float bs[4] = {bs4.x, bs4.y, bs4.z, bs4.w};
-            float in[7][4];   // the raw tokens as float32 (bf16 widening is exact)
-#pragma unroll
-            for (int j = 0; j < 7; ++j) {
-                in[j][0] = __uint_as_float(raw[j].x << 16);
-                in[j][1] = __uint_as_float(raw[j].x & 0xffff0000u);
-                in[j][2] = __uint_as_float(raw[j].y << 16);
-                in[j][3] = __uint_as_float(raw[j].y & 0xffff0000u);
-            }
-            // scalar fused multiply-adds: each lane of the conv kernel's
-            // packed form is the same IEEE operation in the same order
-            uint2 o[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                float a[4];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    a[c] = bs[c];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) a[c] = fmaf(wt[j][c], in[u + j][c], a[c]);
-                    a[c] = silu_half_tanh(a[c]);
-                }
-                o[u] = make_uint2(pack_bf16x2(make_float2(a[0], a[1])), pack_bf16x2(make_float2(a[2], a[3])));
-            }
-            named_bar_sync(kEwBarrier, kEwThreads);   // every raw token has been read
-            if (ctg == kQ / 4 - 1) {
-                // tokens 125 .. 127 raw: the next chunk's left context
-#pragma unroll
-                for (int j = 0; j < 3; ++j) *reinterpret_cast<uint2*>(halo + j * 128 + ccg * 8) = raw[4 + j];
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) st_shared_u2(xbase + (uint32_t)(u + 3) * 128u + (xk ^ ((uint32_t)((u + 4) & 7) << 4)), o[u]);
-            named_bar_sync(kEwBarrier, kEwThreads);   // the tile is convolved
-        };
-        // The conv cache's x columns after the sequence: column j = token
-        // L - 4 + j, from xBC, or for L < 4 the old column L + j.  Only this
-        // thread reads or writes these cache entries after the sequence's
-        // first chunk.
-        auto conv_state_out = [&](const Item& it) {
-            const int ch = it.h * kP + ccg * 4;
-            __nv_bfloat16* cs = prm.conv_state + ((size_t)it.seq * prm.conv_ld + ch) * 4;
-            uint2 old[4], tok[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) old[c] = L < 4 ? *reinterpret_cast<const uint2*>(cs + c * 4) : make_uint2(0u, 0u);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                tok[j] = L - 4 + j >= 0
-                             ? *reinterpret_cast<const uint2*>(prm.xin + ((size_t)it.seq * L + L - 4 + j) * prm.conv_ld + ch)
-                             : make_uint2(0u, 0u);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t e[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) e[j] = L - 4 + j >= 0 ? bf16_bits(tok[j], c) : bf16_bits(old[c], L + j);
-                *reinterpret_cast<uint2*>(cs + c * 4) = make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16));
-            }
-        };
-
         float prev_cl_i = 0.0f;
         int hint = rg.sB0;
         for (int idx = 0; idx < rg.count; ++idx) {
@@ -989,7 +810,6 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 tmem_st16(tH, hv);
             }
             mbar_wait_bounded(bar_ldx + (idx & 1), (uint32_t)(idx >> 1) & 1u, kWaitNs, aborted, prm.status);
-            if constexpr (kConv) conv_x(it, st + kStX);   // (fused conv) x convolved in place
             {
                 const float wj = ex2_approx(cl_last - cl_i) * cv.dt[row];
 #pragma unroll
@@ -1089,9 +909,6 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
 #pragma unroll
                     for (int p = 0; p < 16; ++p) dst[(size_t)(p0 + p) * kN + row] = hv[p];
                 }
-                if constexpr (kConv) {
-                    if (!it.publish && prm.conv_state && ctg == 0) conv_state_out(it);
-                }
             }
             prev_cl_i = cl_i;
             if constexpr (kRagged) {
@@ -1178,19 +995,14 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t s)
 {
     CUtensorMap tmX, tmB, tmC;
     const uint64_t rb = (uint64_t)a.row_stride * 2;
-    const uint64_t rbc = (uint64_t)(a.bc_row_stride ? a.bc_row_stride : a.row_stride) * 2;
     cudaError_t e;
     if ((e = make_map(&tmX, a.x, (uint64_t)a.H * a.P, a.L, a.b, rb)) != cudaSuccess) return e;
-    if ((e = make_map(&tmB, a.B, (uint64_t)a.G * a.N, a.L, a.b, rbc)) != cudaSuccess) return e;
-    if ((e = make_map(&tmC, a.C, (uint64_t)a.G * a.N, a.L, a.b, rbc)) != cudaSuccess) return e;
+    if ((e = make_map(&tmB, a.B, (uint64_t)a.G * a.N, a.L, a.b, rb)) != cudaSuccess) return e;
+    if ((e = make_map(&tmC, a.C, (uint64_t)a.G * a.N, a.L, a.b, rb)) != cudaSuccess) return e;
     CUtensorMap tmY;
     if ((e = make_map(&tmY, a.y, (uint64_t)a.H * a.P, a.L, a.b, (uint64_t)a.H * a.P * 2)) != cudaSuccess) return e;
-    const bool fused = a.conv_w != nullptr;
-    if (fused && a.cu_seqlens) return cudaErrorInvalidValue;   // the fused conv is built for dense batches
-    auto kernel = a.cu_seqlens ? chunk_scan_tc_kernel<true, false>
-                               : (fused ? chunk_scan_tc_kernel<false, true> : chunk_scan_tc_kernel<false, false>);
-    const int smem_bytes = fused ? kSmemBytesConv : kSmemBytes;
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+    auto kernel = a.cu_seqlens ? chunk_scan_tc_kernel<true> : chunk_scan_tc_kernel<false>;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     const int slots = tc_slots(a);
     const size_t ctrl = kWsCtrlBytes(slots);
@@ -1233,12 +1045,7 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t s)
     prm.ws_hdr = ragged ? reinterpret_cast<const int*>(ws) : nullptr;
     prm.nseq = ragged ? a.nseq : a.b;
     prm.status = a.status;
-    prm.xin = fused ? static_cast<const __nv_bfloat16*>(a.x) : nullptr;
-    prm.conv_ld = a.row_stride;
-    prm.conv_w = a.conv_w;
-    prm.conv_bias = a.conv_bias;
-    prm.conv_state = static_cast<__nv_bfloat16*>(a.conv_state);
-    kernel<<<slots, kThreads, smem_bytes, s>>>(tmX, tmB, tmC, tmY, prm);
+    kernel<<<slots, kThreads, kSmemBytes, s>>>(tmX, tmB, tmC, tmY, prm);
     return cudaGetLastError();
 }
 

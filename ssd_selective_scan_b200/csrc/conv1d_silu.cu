@@ -15,13 +15,6 @@
 //
 // The cache is read and rewritten by the thread that owns token tile 0 of a
 // channel group, so an in-place cache update never races with a reader.
-//
-// The kernel runs over a channel range of the rows: `nch` channels starting
-// at the given pointers, input rows `ld_in` elements apart, output rows
-// `ld_out` apart and cache rows (one sequence's [channels][K] block)
-// `ld_state` apart.  A whole-row call passes conv_dim for all three (times K
-// for the cache); the fused prefill path convolves only the B and C channels
-// here, into a compact buffer.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -129,7 +122,7 @@ struct CacheBlock {
 // new column j is old column j + S for j < K - S, else token L - K + j.
 // S is a template parameter so every register index is static.
 template <typename T, int K, int S>
-__device__ inline void roll_cache(T* cs, const T* xb, int L, int64_t ld_in)
+__device__ inline void roll_cache(T* cs, const T* xb, int L, int conv_dim)
 {
     CacheBlock<T, K> blk;
     if (S < K) blk.load(cs);
@@ -140,7 +133,7 @@ __device__ inline void roll_cache(T* cs, const T* xb, int L, int64_t ld_in)
             for (int c = 0; c < kCpt; ++c) blk.set(c, j, blk.get(c, j + S));
         } else {
             float v[kCpt];
-            Vec4<T>::decode(Vec4<T>::load(xb + (size_t)(L - K + j) * ld_in), v);
+            Vec4<T>::decode(Vec4<T>::load(xb + (size_t)(L - K + j) * conv_dim), v);
 #pragma unroll
             for (int c = 0; c < kCpt; ++c) blk.set(c, j, v[c]);
         }
@@ -150,19 +143,19 @@ __device__ inline void roll_cache(T* cs, const T* xb, int L, int64_t ld_in)
 
 template <typename T, int K>
 __global__ void __launch_bounds__(kConvThreads)
-conv1d_silu_kernel(const T* __restrict__ xBC, int64_t ld_in, T* __restrict__ out, int64_t ld_out,
+conv1d_silu_kernel(const T* __restrict__ xBC, T* __restrict__ out,
                    const float* __restrict__ w, const float* __restrict__ bias,
-                   T* __restrict__ conv_state, int64_t ld_state, int L, int nch)
+                   T* __restrict__ conv_state, int L, int conv_dim)
 {
     using V4 = Vec4<T>;
-    const int ngroups = nch / kCpt;
+    const int ngroups = conv_dim / kCpt;
     const int cg = blockIdx.x * kConvThreads + threadIdx.x;
     if (cg >= ngroups) return;
     const int c0 = cg * kCpt;
     const int t0 = blockIdx.y * kConvTile;
     const int bi = blockIdx.z;
-    const T* xb = xBC + (size_t)bi * L * ld_in + c0;
-    T* ob = out + (size_t)bi * L * ld_out + c0;
+    const T* xb = xBC + (size_t)bi * L * conv_dim + c0;
+    T* ob = out + (size_t)bi * L * conv_dim + c0;
 
     // taps of the thread's 4 channels: 4*K contiguous floats
     float wt[K][kCpt];
@@ -189,7 +182,7 @@ conv1d_silu_kernel(const T* __restrict__ xBC, int64_t ld_in, T* __restrict__ out
         if (conv_state) {
             // cache layout [b][conv_dim][K]: column j = time j - K
             CacheBlock<T, K> blk;
-            blk.load(conv_state + (size_t)bi * ld_state + (size_t)c0 * K);
+            blk.load(conv_state + ((size_t)bi * conv_dim + c0) * K);
 #pragma unroll
             for (int c = 0; c < kCpt; ++c)
 #pragma unroll
@@ -202,7 +195,7 @@ conv1d_silu_kernel(const T* __restrict__ xBC, int64_t ld_in, T* __restrict__ out
         }
     } else {
 #pragma unroll
-        for (int j = 0; j < K - 1; ++j) V4::decode(V4::load(xb + (size_t)(t0 - (K - 1) + j) * ld_in), hist[j]);
+        for (int j = 0; j < K - 1; ++j) V4::decode(V4::load(xb + (size_t)(t0 - (K - 1) + j) * conv_dim), hist[j]);
     }
 
     const int t1 = min(L, t0 + kConvTile);
@@ -210,7 +203,7 @@ conv1d_silu_kernel(const T* __restrict__ xBC, int64_t ld_in, T* __restrict__ out
         typename V4::raw raw[kGroup];
 #pragma unroll
         for (int u = 0; u < kGroup; ++u)
-            if (tb + u < t1) raw[u] = V4::load(xb + (size_t)(tb + u) * ld_in);
+            if (tb + u < t1) raw[u] = V4::load(xb + (size_t)(tb + u) * conv_dim);
 #pragma unroll
         for (int u = 0; u < kGroup; ++u) {
             if (tb + u < t1) {
@@ -225,7 +218,7 @@ conv1d_silu_kernel(const T* __restrict__ xBC, int64_t ld_in, T* __restrict__ out
                 a01 = V4::act2(a01);
                 a23 = V4::act2(a23);
                 const float o[kCpt] = {a01.x, a01.y, a23.x, a23.y};
-                V4::store(ob + (size_t)(tb + u) * ld_out, o);
+                V4::store(ob + (size_t)(tb + u) * conv_dim, o);
 #pragma unroll
                 for (int j = 0; j < K - 1; ++j)
 #pragma unroll
@@ -238,48 +231,45 @@ conv1d_silu_kernel(const T* __restrict__ xBC, int64_t ld_in, T* __restrict__ out
         // New cache column j = input at time L - K + j of (old cache | xBC).
         // Times < 0 come from the old cache, which this thread alone reads
         // and writes.
-        T* cs = conv_state + (size_t)bi * ld_state + (size_t)c0 * K;
+        T* cs = conv_state + ((size_t)bi * conv_dim + c0) * K;
         constexpr int S2 = K < 2 ? K : 2, S3 = K < 3 ? K : 3;
-        if (L >= K) roll_cache<T, K, K>(cs, xb, L, ld_in);
-        else if (L == 1) roll_cache<T, K, 1>(cs, xb, L, ld_in);
-        else if (L == 2) roll_cache<T, K, S2>(cs, xb, L, ld_in);
-        else roll_cache<T, K, S3>(cs, xb, L, ld_in);
+        if (L >= K) roll_cache<T, K, K>(cs, xb, L, conv_dim);
+        else if (L == 1) roll_cache<T, K, 1>(cs, xb, L, conv_dim);
+        else if (L == 2) roll_cache<T, K, S2>(cs, xb, L, conv_dim);
+        else roll_cache<T, K, S3>(cs, xb, L, conv_dim);
     }
 }
 
 template <typename T, int K>
-static cudaError_t launch_conv_k(const ConvSlice& c, cudaStream_t s)
+static cudaError_t launch_conv_k(const void* xBC, void* out, const float* w, const float* bias,
+                                 void* conv_state, int b, int L, int conv_dim, cudaStream_t s)
 {
-    const int ngroups = c.nch / kCpt;
-    dim3 grid((ngroups + kConvThreads - 1) / kConvThreads, (c.L + kConvTile - 1) / kConvTile, c.b);
+    const int ngroups = conv_dim / kCpt;
+    dim3 grid((ngroups + kConvThreads - 1) / kConvThreads, (L + kConvTile - 1) / kConvTile, b);
     conv1d_silu_kernel<T, K><<<grid, kConvThreads, 0, s>>>(
-        static_cast<const T*>(c.in), c.ld_in, static_cast<T*>(c.out), c.ld_out, c.w, c.bias,
-        static_cast<T*>(c.state), c.ld_state, c.L, c.nch);
+        static_cast<const T*>(xBC), static_cast<T*>(out), w, bias, static_cast<T*>(conv_state),
+        L, conv_dim);
     return cudaGetLastError();
 }
 
 template <typename T>
-static cudaError_t launch_conv_t(const ConvSlice& c, cudaStream_t s)
+static cudaError_t launch_conv_t(const void* xBC, void* out, const float* w, const float* bias,
+                                 void* conv_state, int b, int L, int conv_dim, int k, cudaStream_t s)
 {
-    switch (c.k) {
-        case 2: return launch_conv_k<T, 2>(c, s);
-        case 3: return launch_conv_k<T, 3>(c, s);
-        case 4: return launch_conv_k<T, 4>(c, s);
+    switch (k) {
+        case 2: return launch_conv_k<T, 2>(xBC, out, w, bias, conv_state, b, L, conv_dim, s);
+        case 3: return launch_conv_k<T, 3>(xBC, out, w, bias, conv_state, b, L, conv_dim, s);
+        case 4: return launch_conv_k<T, 4>(xBC, out, w, bias, conv_state, b, L, conv_dim, s);
         default: return cudaErrorInvalidValue;
     }
-}
-
-cudaError_t launch_conv1d_silu_slice(const ConvSlice& c, cudaStream_t s)
-{
-    return c.bf16 ? launch_conv_t<__nv_bfloat16>(c, s) : launch_conv_t<float>(c, s);
 }
 
 cudaError_t launch_conv1d_silu(const void* xBC, void* out, const float* w, const float* bias,
                                void* conv_state, int b, int L, int conv_dim, int k, bool bf16,
                                cudaStream_t s)
 {
-    ConvSlice c{xBC, conv_dim, out, conv_dim, w, bias, conv_state, (int64_t)conv_dim * k, b, L, conv_dim, k, bf16};
-    return launch_conv1d_silu_slice(c, s);
+    return bf16 ? launch_conv_t<__nv_bfloat16>(xBC, out, w, bias, conv_state, b, L, conv_dim, k, s)
+                : launch_conv_t<float>(xBC, out, w, bias, conv_state, b, L, conv_dim, k, s);
 }
 
 }  // namespace ssd

@@ -30,16 +30,6 @@ struct ScanArgs {
     // of one packed token dimension of L tokens (b = 1 then); nseq sequences.
     const int* cu_seqlens = nullptr;
     int nseq = 0;
-    // B and C rows may have their own token stride (0: row_stride).
-    int64_t bc_row_stride = 0;
-    // Fused conv1d+SiLU of the x channels (tensor-core path, dense batches,
-    // width 4): x is then the raw conv input xBC (row_stride = conv_dim) and
-    // B, C are already convolved.  conv_w [conv_dim][4], conv_bias
-    // [conv_dim] or null, conv_state [b][conv_dim][4] in the I/O dtype or
-    // null (its x channels are read and rewritten here).
-    const float* conv_w = nullptr;
-    const float* conv_bias = nullptr;
-    void* conv_state = nullptr;
 };
 
 // Workspace of a ragged scan: a header (hdr[0] = invalid cu_seqlens flag,
@@ -55,23 +45,6 @@ cudaError_t launch_varlen_prep(const int* cu_seqlens, int nseq, int T, int H, in
 cudaError_t launch_conv1d_silu(const void* xBC, void* out, const float* w, const float* bias,
                                void* conv_state, int b, int L, int conv_dim, int k, bool bf16,
                                cudaStream_t s);
-
-// conv1d+SiLU over a range of nch channels (pointers at its first channel):
-// input rows ld_in elements apart, output rows ld_out apart, one sequence's
-// cache block [nch][k] at state + s * ld_state (channel-major, k columns).
-struct ConvSlice {
-    const void* in;
-    int64_t ld_in;
-    void* out;
-    int64_t ld_out;
-    const float* w;      // [nch][k]
-    const float* bias;   // [nch] or null
-    void* state;         // or null
-    int64_t ld_state;
-    int b, L, nch, k;
-    bool bf16;
-};
-cudaError_t launch_conv1d_silu_slice(const ConvSlice& c, cudaStream_t s);
 
 bool state_update_supports_n(int N);
 cudaError_t launch_state_update(float* state, const void* x, const void* B, const void* C,

@@ -216,8 +216,8 @@ def conv_scan_fwd(xBC: torch.Tensor, w: torch.Tensor, dt_raw: torch.Tensor, A: t
                   final_state: torch.Tensor | bool | None = True,
                   workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
                   stream=None):
-    """Fused prefill: conv1d+SiLU of xBC [b, L, conv_dim], then the chunked
-    scan of its x | B | C channels, without writing the conv output.  w
+    """The prefill layer in one call: conv1d+SiLU of xBC [b, L, conv_dim] into
+    the workspace, then the chunked scan of its x | B | C channels.  w
     [conv_dim, k] f32; conv_state [b, conv_dim, k] (I/O dtype) is updated in
     place.  Returns (y [b, L, H, P], final_state [b, H, P, N] f32 or None)."""
     if xBC.dim() != 3 or not xBC.is_contiguous():
@@ -256,8 +256,8 @@ def layer_prefill(xBC, w, dt_raw, A, H, P, G, N, *, bias=None, conv_state=None, 
                   D=None, init_state=None, Q=128, y=None, final_state=True, workspace=None,
                   stream=None):
     """The prefill layer (conv1d+SiLU, then the chunked scan) through the
-    fused call.  Returns (y, final_state); conv_state, if given, is updated
-    in place."""
+    one-call entry point.  Returns (y, final_state); conv_state, if given, is
+    updated in place."""
     return conv_scan_fwd(xBC, w, dt_raw, A, H, P, G, N, bias=bias, conv_state=conv_state,
                          dt_bias=dt_bias, D=D, init_state=init_state, Q=Q, y=y,
                          final_state=final_state, workspace=workspace, stream=stream)

@@ -207,11 +207,9 @@ def test_conv_scan_validation():
     assert cs(workspace=fake(6)) == INV                                # workspace overlaps final state
     assert cs(final_state=fake(3, 64)) == INV                          # final state overlaps dt_raw
     assert cs(k=5) == UNS and cs(k=1) == UNS
-    # the fused tensor-core path keeps B and C only (2 G N per token); others the whole conv output
-    fused = libssd.ssd_conv_scan_workspace_bytes(2, 256, 40, 64, 128, 8, 128, 4, BF16)
+    # the conv output (b L conv_dim elements, 256-byte rounded), then the scan's own
     scan = libssd.ssd_chunk_scan_workspace_bytes(2, 256, 40, 64, 128, 8, 128, BF16)
-    assert fused == 2 * 256 * 2 * 8 * 128 * 2 + scan
-    assert libssd.ssd_conv_scan_workspace_bytes(2, 256, 40, 64, 128, 8, 128, 3, BF16) == \
+    assert libssd.ssd_conv_scan_workspace_bytes(2, 256, 40, 64, 128, 8, 128, 4, BF16) == \
         2 * 256 * 4608 * 2 + scan
     assert libssd.ssd_conv_scan_workspace_bytes(1, 256, 4, 64, 16, 1, 64, 4, F32) == 256 * 288 * 4
     assert libssd.ssd_conv_scan_workspace_bytes(0, 256, 4, 64, 16, 1, 64, 4, F32) == 0

@@ -1,11 +1,8 @@
-"""GPU parity of the fused prefill call (conv1d+SiLU and the chunked scan in
-one entry point, ssd_conv_scan_fwd) against the fp64 oracle run from the raw
-xBC, called through the C ABI.
-
-The fused tensor-core path convolves the x channels inside the scan kernel
-with the stand-alone conv kernel's arithmetic, so its y, final state and conv
-cache must also equal the two-call path (conv1d_silu, then chunk_scan_fwd on
-its output) bit for bit: a second check that needs no tolerance."""
+"""GPU parity of the one-call prefill layer (conv1d+SiLU, then the chunked
+scan: ssd_conv_scan_fwd) against the fp64 oracle run from the raw xBC,
+called through the C ABI.  Its y, final state and conv cache must also equal
+the two separate calls (conv1d_silu, then chunk_scan_fwd on its output) bit
+for bit."""
 import numpy as np
 import pytest
 import torch
@@ -65,7 +62,6 @@ CASES = {
     "short_L3_cache": (BF16.with_(b=2, L=3, H=8, G=2), dict(conv_state=True)),
     "L129_one_token_chunk": (BF16.with_(b=2, L=129, H=8, G=2), dict(conv_state=True)),
     # more chains than the persistent grid has CTAs: chains cut between CTAs
-    # (a chunk's left context and the cache then cross a hand-off)
     "many_chains_handoff": (BF16.with_(b=4, L=520, H=40), dict(conv_state=True, init_state=True)),
     "h128_g8": (BF16.with_(b=2, L=300, H=128), dict(conv_state=True)),
     "g1_long_memory": (BF16.with_(b=1, L=640, H=6, G=1), dict(a_range=(0.01, 2.0), conv_state=True)),
@@ -86,8 +82,8 @@ def test_conv_scan_matches_oracle_and_two_calls(name):
 
 
 @pytest.mark.parametrize("name,s", [
-    ("tiny_fp32", synth.CONFIGS[0]),                        # float32: conv output in the workspace
-    ("bf16_k3", BF16.with_(b=2, L=300, H=8, G=2, k=3)),     # width 3: not the fused kernel
+    ("tiny_fp32", synth.CONFIGS[0]),                        # float32, general scan kernel
+    ("bf16_k3", BF16.with_(b=2, L=300, H=8, G=2, k=3)),     # conv width 3
     ("bf16_n16", BF16.with_(b=1, L=200, H=4, N=16, G=1)),   # general scan kernel
     ("bf16_q64", BF16.with_(b=1, L=200, H=4, G=2, Q=64)),
 ])
