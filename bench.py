@@ -12,7 +12,8 @@ JSON line.  Next to the headline prefill number the line carries:
                 launch / its CUDA-event duration) against the measured peak;
   scan_only     tokens/s of the scan kernel alone;
   decode        one decode step of the 256-sequence, 128-head workload
-                (conv-cache roll + state update), state-update GB/s;
+                (conv-cache roll, conv + SiLU and state update in one
+                kernel), its GB/s; the two-kernel form beside it;
   e2e           the same prefill step through the public one-call entry point
                 (ssd_conv_scan_fwd) with the step's inputs copied from pinned
                 host memory and y + final state copied back, inside the timed
@@ -70,6 +71,12 @@ def conv_bytes_per_token(s) -> int:
 def decode_state_update_bytes(s) -> int:
     """fp32 state read + written, x/B/C/dt read, y written."""
     return 8 * s.b * s.H * s.P * s.N + s.elem_bytes * s.b * (s.H * s.P + 2 * s.G * s.N + s.H + s.H * s.P)
+
+
+def decode_step_bytes(s) -> int:
+    """The one-kernel decode step: fp32 state read + written, conv cache read +
+    written (k columns), the token's xBC and dt read, y written."""
+    return 8 * s.b * s.H * s.P * s.N + s.elem_bytes * s.b * (2 * s.k * s.conv_dim + s.conv_dim + s.H + s.H * s.P)
 
 
 def load_peaks():
@@ -252,6 +259,12 @@ class DecodeStep:
         self.layer.state_update(d["state"], x, B, C, d["dt_raw"], d["A"], d["dt_bias"], d["D"],
                                 y=self.y)
 
+    def __call__(self):
+        """One decode token per sequence through the one-kernel decode step."""
+        d, s = self.d, self.s
+        self.layer.decode_step(d["xBC"], d["w"], d["conv_state"], d["state"], d["dt_raw"], d["A"],
+                               s.H, s.P, s.G, s.N, dt_bias=d["dt_bias"], D=d["D"], y=self.y)
+
 
 def _events(n):
     return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
@@ -305,22 +318,34 @@ def run_ours(args, rank, world, dev):
     conv_ms = max_over_ranks(conv_ms)
     tokens = s.b * s.L
 
-    # decode: conv-cache roll + state update, one token per sequence
+    # decode: one token per sequence through the one-kernel decode step (the
+    # state is rewritten in place, so consecutive steps are valid work)
     for _ in range(max(3, args.warmup)):
-        dec.conv(); dec.update()
+        dec()
     KD = max(10, K)
-    ev_u = _events(2 * KD)
     d0, d1 = _events(2)
     barrier()
     d0.record()
+    for _ in range(KD):
+        dec()
+    d1.record()
+    barrier()
+    dec_ms = max_over_ranks(d0.elapsed_time(d1) / KD)
+    # the same step as two kernels (conv roll, then the state update alone), for comparison
+    for _ in range(3):
+        dec.conv(); dec.update()
+    ev_u = _events(2 * KD)
+    d2, d3 = _events(2)
+    barrier()
+    d2.record()
     for i in range(KD):
         dec.conv()
         ev_u[2 * i].record()
         dec.update()
         ev_u[2 * i + 1].record()
-    d1.record()
+    d3.record()
     barrier()
-    dec_ms = max_over_ranks(d0.elapsed_time(d1) / KD)
+    two_ms = max_over_ranks(d2.elapsed_time(d3) / KD)
     upd_ms = max_over_ranks(statistics.mean(ev_u[2 * i].elapsed_time(ev_u[2 * i + 1]) for i in range(KD)))
 
     # end to end through the public API: H2D inputs, the layer, D2H results
@@ -385,13 +410,17 @@ def run_ours(args, rank, world, dev):
         "scan_only": {"tokens_per_s": tokens / (scan_ms * 1e-3), "ms": scan_ms},
         "conv": {"ms": conv_ms, "GB/s": conv_bytes_per_token(s) * tokens / (conv_ms * 1e-3) / 1e9,
                  "frac_hbm": conv_bytes_per_token(s) * tokens / (conv_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
-        "decode": {"workload": DECODE.name, "ms_per_step": dec_ms, "state_update_ms": upd_ms,
-                   "state_update_GB/s": decode_state_update_bytes(DECODE) / (upd_ms * 1e-3) / 1e9,
-                   "frac_hbm": decode_state_update_bytes(DECODE) / (upd_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                   "tokens_per_s": world * DECODE.b / (dec_ms * 1e-3)},
+        "decode": {"workload": DECODE.name,
+                   "kernel": "decode_step (conv-cache roll, conv + SiLU, state update: one launch)",
+                   "ms_per_step": dec_ms,
+                   "GB/s": decode_step_bytes(DECODE) / (dec_ms * 1e-3) / 1e9,
+                   "frac_hbm": decode_step_bytes(DECODE) / (dec_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                   "tokens_per_s": world * DECODE.b / (dec_ms * 1e-3),
+                   "two_kernel_ms_per_step": two_ms, "state_update_ms": upd_ms,
+                   "state_update_GB/s": decode_state_update_bytes(DECODE) / (upd_ms * 1e-3) / 1e9},
         "e2e": {"value": shard.aggregate_tokens_per_s(tokens, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": 2 * K,
+        "gpu_launches": 2 * K,   # conv + scan per timed prefill step
         "clocks": clocks,
     }
     return line
@@ -459,9 +488,7 @@ def run_reference(args):
 def run_one_kernel(args, dev):
     """Launch one kernel of the bench workloads alone (for ncu captures)."""
     if args.kernel == "decode":
-        st = DecodeStep(DECODE, synth.config_seed(4), dev)
-        st.conv()
-        fn = st.update
+        fn = DecodeStep(DECODE, synth.config_seed(4), dev)
     else:
         st = PrefillStep(PREFILL, synth.config_seed(1), dev)
         st.conv()

@@ -294,6 +294,32 @@ SSD_API ssd_status_t ssd_state_update(float* state, const void* x, const void* B
                               cudaStream_t stream);
 
 /*
+ * The decode step of the layer in one kernel: ssd_conv1d_silu with L = 1 and
+ * a cache (roll the cache, convolve the new token, SiLU), then
+ * ssd_state_update on its output (the Mamba cache of "Hybrid Architectures
+ * for Language Models", summary page, appendix C: the conv cache and the
+ * state are the per-layer decode state).  The conv outputs never leave the
+ * chip; the results equal those of the two calls bit for bit.
+ *
+ *   state      [b][H][P][N]       float32, read and rewritten in place
+ *   conv_state [b][conv_dim][k]   dtype, REQUIRED, rolled in place (as for
+ *                                 ssd_conv1d_silu), conv_dim = H*P + 2*G*N
+ *   xBC        [b][conv_dim]      dtype, the new token's x | B | C inputs
+ *   w [conv_dim][k], bias [conv_dim] (may be NULL)   float32
+ *   dt_raw [b][H] dtype; dt_bias [H], A [H], D [H] float32 (dt_bias, D may be NULL)
+ *   y          [b][H][P]          dtype, written
+ * One CTA per (sequence, group) convolves the group's B and C channels once
+ * and the x channels of its H/G heads, then updates those heads' states.
+ * Requirements: 2 <= k <= 4 and N a multiple of 4 with N <= 256 (else
+ * SSD_ERR_UNSUPPORTED); H % G == 0; state 16-byte aligned; no buffer may
+ * overlap another.
+ */
+SSD_API ssd_status_t ssd_decode_step(float* state, void* conv_state, const void* xBC, const float* w,
+                                     const float* bias, const void* dt_raw, const float* dt_bias,
+                                     const float* A, const float* D, void* y, int b, int H, int P,
+                                     int N, int G, int k, ssd_dtype_t dtype, cudaStream_t stream);
+
+/*
  * Self-test of the bounded device waits (failure detection without a fault).
  * Every wait of the tensor-core scan gives up after a time limit, records
  * SSD_ERR_TIMEOUT in the call's status word and lets the kernel run to its

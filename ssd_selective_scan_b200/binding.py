@@ -42,6 +42,8 @@ SIGNATURES = {
     "ssd_chunk_scan_fwd_varlen": (_i, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                        _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp, _vp]),
     "ssd_conv_scan_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),
+    "ssd_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                             _i, _i, _i, _i, _i, _i, _i, _vp]),
     "ssd_conv_scan_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp, _vp]),
 }
@@ -131,6 +133,12 @@ def ssd_conv_scan_fwd(xBC, w, bias, conv_state, dt_raw, dt_bias, A, D, init_stat
     return load().ssd_conv_scan_fwd(xBC, w, bias, conv_state, dt_raw, dt_bias, A, D, init_state, y,
                                     final_state, b, L, H, P, N, G, Q, k, dtype, workspace,
                                     workspace_bytes, status, stream)
+
+
+def ssd_decode_step(state, conv_state, xBC, w, bias, dt_raw, dt_bias, A, D, y, b, H, P, N, G, k,
+                    dtype, stream) -> int:
+    return load().ssd_decode_step(state, conv_state, xBC, w, bias, dt_raw, dt_bias, A, D, y, b, H, P,
+                                  N, G, k, dtype, stream)
 
 
 def ssd_selftest_bounded_wait(status, limit_ns, stream) -> int:

@@ -4,6 +4,7 @@
 #include "ssd.h"
 
 #include "kernels.h"
+#include "decode.h"
 
 namespace {
 
@@ -347,6 +348,42 @@ ssd_status_t ssd_state_update(float* state, const void* x, const void* B, const 
     if (b == 0) return SSD_OK;
     return from_cuda(ssd::launch_state_update(state, x, B, C, row_stride, dt_raw, dt_bias, A, D, y,
                                               b, H, P, N, G, dtype == SSD_BF16, stream));
+}
+
+ssd_status_t ssd_decode_step(float* state, void* conv_state, const void* xBC, const float* w,
+                             const float* bias, const void* dt_raw, const float* dt_bias, const float* A,
+                             const float* D, void* y, int b, int H, int P, int N, int G, int k,
+                             ssd_dtype_t dtype, cudaStream_t stream)
+{
+    if (!valid_dtype(dtype) || b < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || k <= 0 || H % G)
+        return SSD_ERR_INVALID_ARG;
+    if (N % 4) return SSD_ERR_INVALID_ARG;
+    if ((int64_t)H * P + 2 * (int64_t)G * N > 0x7fffffffLL) return SSD_ERR_INVALID_ARG;
+    if (b == 0) return SSD_OK;
+    if (!state || !conv_state || !xBC || !w || !dt_raw || !A || !y) return SSD_ERR_INVALID_ARG;
+    const int e = elem_bytes(dtype);
+    if (!aligned(state, 16) || !aligned(conv_state, e) || !aligned(xBC, e) || !aligned(dt_raw, e) ||
+        !aligned(y, e) || !aligned(w, 4) || !aligned(A, 4) || (bias && !aligned(bias, 4)) ||
+        (dt_bias && !aligned(dt_bias, 4)) || (D && !aligned(D, 4)))
+        return SSD_ERR_INVALID_ARG;
+    const int64_t conv_dim = (int64_t)H * P + 2 * (int64_t)G * N;
+    const Range rs = span(state, (int64_t)b * H * P * N * 4);
+    const Range rcs = span(conv_state, (int64_t)b * conv_dim * k * e);
+    const Range rx = span(xBC, (int64_t)b * conv_dim * e);
+    const Range rw = span(w, conv_dim * k * 4);
+    const Range rdt = span(dt_raw, (int64_t)b * H * e);
+    const Range ry = span(y, (int64_t)b * H * P * e);
+    for (Range in : {rcs, rx, rw, rdt, ry})
+        if (overlap(rs, in)) return SSD_ERR_INVALID_ARG;
+    for (Range in : {rx, rw, rdt, ry})
+        if (overlap(rcs, in)) return SSD_ERR_INVALID_ARG;
+    for (Range in : {rx, rw, rdt})
+        if (overlap(ry, in)) return SSD_ERR_INVALID_ARG;
+    if (k < 2 || k > 4 || !ssd::state_update_supports_n(N)) return SSD_ERR_UNSUPPORTED;
+    if ((int64_t)b * G > 0x7fffffffLL) return SSD_ERR_UNSUPPORTED;
+    if (ssd::decode_step_smem_bytes(H, P, N, G) > (size_t)max_optin_smem()) return SSD_ERR_UNSUPPORTED;
+    return from_cuda(ssd::launch_decode_step(state, conv_state, xBC, w, bias, dt_raw, dt_bias, A, D, y, b, H, P,
+                                             N, G, k, dtype == SSD_BF16, stream));
 }
 
 }  // extern "C"

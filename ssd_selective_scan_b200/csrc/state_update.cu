@@ -15,6 +15,7 @@
 // The y reduction over N is a butterfly over the TPR lanes of a row.
 #include "common.cuh"
 #include "kernels.h"
+#include "decode.h"
 
 namespace ssd {
 
@@ -121,6 +122,206 @@ static cudaError_t launch_su_t(float* state, const void* x, const void* B, const
     }
 #undef SSD_SU_CASE
     return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// The decode step in one kernel: the conv-cache roll, conv (width K) and
+// SiLU of the new token, then the state update.  One CTA per (sequence,
+// group): it convolves the group's B and C channels once and the x channels
+// of the group's H / G heads, rewrites exactly those channels' cache columns
+// (so no two CTAs touch the same cache entry and the in-place roll cannot
+// race), keeps the conv outputs in shared memory, then streams the heads'
+// states.  Every value is computed as by conv1d_silu_kernel (L = 1, with a
+// cache) followed by state_update_kernel: the conv outputs are rounded to
+// the I/O type, and each state row uses the same lane layout and reduction
+// order, so the results are equal bit for bit.
+// ---------------------------------------------------------------------------
+constexpr int kDecThreads = 256;
+
+template <typename T> __device__ inline float conv_act(float v);
+template <> __device__ inline float conv_act<float>(float v) { return silu_f(v); }
+template <> __device__ inline float conv_act<__nv_bfloat16>(float v)
+{
+    // the conv kernel's bf16 form: v/2 + (v/2) tanh(v/2)
+    const float hv = v * 0.5f;
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(hv));
+    return fmaf(hv, t, hv);
+}
+
+template <typename T, int N, int K>
+__global__ void __launch_bounds__(kDecThreads)
+decode_step_kernel(float* __restrict__ state, T* __restrict__ conv_state, const T* __restrict__ xBC,
+                   const float* __restrict__ w, const float* __restrict__ bias,
+                   const T* __restrict__ dt_raw, const float* __restrict__ dt_bias,
+                   const float* __restrict__ A, const float* __restrict__ D, T* __restrict__ y,
+                   int H, int P, int G)
+{
+    // shared: x of the group's heads [hpg * P], B [N], C [N], then per head dt, exp(dt A), D
+    extern __shared__ float sU[];
+    constexpr int NV = N / 4;
+    constexpr int TPR = NV < 32 ? NV : 32;
+    constexpr int VPL = NV / TPR;
+    constexpr int RPW = 32 / TPR;
+    constexpr int ROWS = 8;
+    constexpr int kWarps = kDecThreads / 32;
+
+    const int g = blockIdx.x % G;
+    const int bi = blockIdx.x / G;
+    const int hpg = H / G;
+    const int conv_dim = H * P + 2 * G * N;
+    const int nx = hpg * P;
+    float* sDt = sU + nx + 2 * N;
+    float* sDA = sDt + hpg;
+    float* sD = sDA + hpg;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sub = lane / TPR, li = lane % TPR;
+    const int rows_per_iter = kWarps * RPW * ROWS;
+
+    // the first rows of the first head's state are requested before the
+    // conv, so that their latency overlaps it
+    float4 st[ROWS][VPL];
+    int prow[ROWS];
+    auto load_rows = [&](const float* sh, int p0) {
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) {
+            prow[r] = p0 + (r * kWarps + warp) * RPW + sub;
+            if (prow[r] < P) {
+#pragma unroll
+                for (int v = 0; v < VPL; ++v)
+                    st[r][v] = __ldcs(reinterpret_cast<const float4*>(sh + (size_t)prow[r] * N) + v * TPR + li);
+            }
+        }
+    };
+    load_rows(state + ((size_t)bi * H + g * hpg) * (size_t)P * N, 0);
+
+    // 1. conv + SiLU of the group's channels, the cache roll, and each
+    //    head's dt terms
+    for (int i = threadIdx.x; i < nx + 2 * N; i += kDecThreads) {
+        const int c = i < nx ? g * nx + i : (i < nx + N ? H * P + g * N + (i - nx) : H * P + G * N + g * N + (i - nx - N));
+        T* cs = conv_state + ((size_t)bi * conv_dim + c) * K;
+        float win[K];
+#pragma unroll
+        for (int j = 0; j + 1 < K; ++j) win[j] = ld_f(cs + j + 1);
+        win[K - 1] = ld_f(xBC + (size_t)bi * conv_dim + c);
+        float acc = bias ? bias[c] : 0.0f;
+#pragma unroll
+        for (int j = 0; j < K; ++j) acc = fmaf(w[(size_t)c * K + j], win[j], acc);
+        sU[i] = io<T>::to_f(io<T>::from_f(conv_act<T>(acc)));
+#pragma unroll
+        for (int j = 0; j < K; ++j) cs[j] = io<T>::from_f(win[j]);
+    }
+    for (int hl = threadIdx.x; hl < hpg; hl += kDecThreads) {
+        const int h = g * hpg + hl;
+        const float dt = softplus_f(ld_f(dt_raw + (size_t)bi * H + h) + (dt_bias ? dt_bias[h] : 0.0f));
+        sDt[hl] = dt;
+        sDA[hl] = expf(dt * A[h]);
+        sD[hl] = D ? D[h] : 0.0f;
+    }
+    __syncthreads();
+
+    // 2. the state update of each head of the group
+    const float* Bs = sU + nx;
+    const float* Cs = sU + nx + N;
+    float bv[VPL][4], cvv[VPL][4];
+#pragma unroll
+    for (int v = 0; v < VPL; ++v)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int n = (v * TPR + li) * 4 + e;
+            bv[v][e] = Bs[n];
+            cvv[v][e] = Cs[n];
+        }
+    for (int hl = 0; hl < hpg; ++hl) {
+        const int h = g * hpg + hl;
+        const float dt = sDt[hl], dA = sDA[hl], Dh = sD[hl];
+        const float* xs = sU + hl * P;
+        float* sh = state + ((size_t)bi * H + h) * (size_t)P * N;
+        T* yr = y + ((size_t)bi * H + h) * P;
+        for (int p0 = 0; p0 < P; p0 += rows_per_iter) {
+            if (hl > 0 || p0 > 0) load_rows(sh, p0);
+#pragma unroll
+            for (int r = 0; r < ROWS; ++r) {
+                const bool ok = prow[r] < P;
+                const float xp = ok ? xs[prow[r]] : 0.0f;
+                const float dtx = dt * xp;
+                float acc = 0.0f;
+                if (ok) {
+#pragma unroll
+                    for (int v = 0; v < VPL; ++v) {
+                        float4 q = st[r][v];
+                        q.x = fmaf(dA, q.x, dtx * bv[v][0]);
+                        q.y = fmaf(dA, q.y, dtx * bv[v][1]);
+                        q.z = fmaf(dA, q.z, dtx * bv[v][2]);
+                        q.w = fmaf(dA, q.w, dtx * bv[v][3]);
+                        acc = fmaf(cvv[v][0], q.x, acc);
+                        acc = fmaf(cvv[v][1], q.y, acc);
+                        acc = fmaf(cvv[v][2], q.z, acc);
+                        acc = fmaf(cvv[v][3], q.w, acc);
+                        __stcs(reinterpret_cast<float4*>(sh + (size_t)prow[r] * N) + v * TPR + li, q);
+                    }
+                }
+#pragma unroll
+                for (int o = TPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+                if (ok && li == 0) yr[prow[r]] = io<T>::from_f(fmaf(Dh, xp, acc));
+            }
+        }
+    }
+}
+
+size_t decode_step_smem_bytes(int H, int P, int N, int G) { return ((size_t)(H / G) * (P + 3) + 2 * (size_t)N) * 4; }
+
+template <typename T, int K>
+static cudaError_t launch_dec_k(float* state, void* conv_state, const void* xBC, const float* w,
+                                const float* bias, const void* dt_raw, const float* dt_bias, const float* A,
+                                const float* D, void* y, int b, int H, int P, int N, int G, cudaStream_t s)
+{
+    const dim3 grid((unsigned)((int64_t)b * G));
+    const size_t smem = decode_step_smem_bytes(H, P, N, G);
+#define SSD_DEC_CASE(NN)                                                                                   \
+    case NN: {                                                                                             \
+        auto kern = decode_step_kernel<T, NN, K>;                                                          \
+        if (smem > 48 * 1024) {                                                                            \
+            const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                                       (int)smem);                                         \
+            if (e != cudaSuccess) return e;                                                                \
+        }                                                                                                  \
+        kern<<<grid, kDecThreads, smem, s>>>(state, static_cast<T*>(conv_state), static_cast<const T*>(xBC), \
+                                            w, bias, static_cast<const T*>(dt_raw), dt_bias, A, D,         \
+                                            static_cast<T*>(y), H, P, G);                                  \
+        break;                                                                                             \
+    }
+    switch (N) {
+        SSD_DEC_CASE(4) SSD_DEC_CASE(8) SSD_DEC_CASE(16) SSD_DEC_CASE(32)
+        SSD_DEC_CASE(64) SSD_DEC_CASE(128) SSD_DEC_CASE(256)
+        default: return cudaErrorInvalidValue;
+    }
+#undef SSD_DEC_CASE
+    return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_dec_t(float* state, void* conv_state, const void* xBC, const float* w,
+                                const float* bias, const void* dt_raw, const float* dt_bias, const float* A,
+                                const float* D, void* y, int b, int H, int P, int N, int G, int k, cudaStream_t s)
+{
+    switch (k) {
+        case 2: return launch_dec_k<T, 2>(state, conv_state, xBC, w, bias, dt_raw, dt_bias, A, D, y, b, H, P, N, G, s);
+        case 3: return launch_dec_k<T, 3>(state, conv_state, xBC, w, bias, dt_raw, dt_bias, A, D, y, b, H, P, N, G, s);
+        case 4: return launch_dec_k<T, 4>(state, conv_state, xBC, w, bias, dt_raw, dt_bias, A, D, y, b, H, P, N, G, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_decode_step(float* state, void* conv_state, const void* xBC, const float* w,
+                               const float* bias, const void* dt_raw, const float* dt_bias, const float* A,
+                               const float* D, void* y, int b, int H, int P, int N, int G, int k, bool bf16,
+                               cudaStream_t s)
+{
+    return bf16 ? launch_dec_t<__nv_bfloat16>(state, conv_state, xBC, w, bias, dt_raw, dt_bias, A, D, y, b, H, P,
+                                              N, G, k, s)
+                : launch_dec_t<float>(state, conv_state, xBC, w, bias, dt_raw, dt_bias, A, D, y, b, H, P, N, G, k,
+                                      s);
 }
 
 bool state_update_supports_n(int N)

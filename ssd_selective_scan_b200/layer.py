@@ -264,11 +264,30 @@ def layer_prefill(xBC, w, dt_raw, A, H, P, G, N, *, bias=None, conv_state=None, 
 
 
 def decode_step(xBC, w, conv_state, state, dt_raw, A, H, P, G, N, *, bias=None, dt_bias=None,
-                D=None, u=None, y=None, stream=None):
-    """One token per sequence: conv-cache roll + conv + SiLU, then the state
-    update.  xBC [b, conv_dim]; conv_state and state updated in place.  Returns y."""
+                D=None, y=None, stream=None):
+    """One token per sequence in one kernel: conv-cache roll, conv + SiLU,
+    then the state update.  xBC [b, conv_dim]; conv_state [b, conv_dim, k]
+    and state [b, H, P, N] f32 updated in place.  Returns y [b, H, P]."""
+    if xBC.dim() != 2 or not xBC.is_contiguous():
+        raise ValueError("xBC must be a contiguous [b, conv_dim] tensor")
     b, cd = xBC.shape
-    u = conv1d_silu(xBC.view(b, 1, cd), w, bias, conv_state,
-                    out=None if u is None else u.view(b, 1, cd), stream=stream).view(b, cd)
-    x, B, C = split_channels(u, H, P, G, N)
-    return state_update(state, x, B, C, dt_raw, A, dt_bias, D, y=y, stream=stream)
+    if cd != H * P + 2 * G * N:
+        raise ValueError(f"xBC has {cd} channels, expected H*P + 2*G*N = {H * P + 2 * G * N}")
+    k = w.shape[1]
+    if w.shape != (cd, k):
+        raise ValueError("w must be [conv_dim, k]")
+    if conv_state.shape != (b, cd, k) or conv_state.dtype != xBC.dtype or not conv_state.is_contiguous():
+        raise ValueError("conv_state must be a contiguous [b, conv_dim, k] tensor of xBC's dtype")
+    if state.shape != (b, H, P, N):
+        raise ValueError("state must be [b, H, P, N]")
+    _f32(state, "state")
+    if dt_raw.shape != (b, H) or dt_raw.dtype != xBC.dtype or not dt_raw.is_contiguous():
+        raise ValueError("dt_raw must be a contiguous [b, H] tensor of xBC's dtype")
+    if y is None:
+        y = torch.empty((b, H, P), dtype=xBC.dtype, device=xBC.device)
+    st = libssd.ssd_decode_step(_ptr(state), _ptr(conv_state), _ptr(xBC), _ptr(_f32(w, "w")),
+                                _ptr(_f32(bias, "bias")), _ptr(dt_raw), _ptr(_f32(dt_bias, "dt_bias")),
+                                _ptr(_f32(A, "A")), _ptr(_f32(D, "D")), _ptr(y), b, H, P, N, G, k,
+                                _dtype_code(xBC), _stream(stream))
+    libssd.check("ssd_decode_step", st)
+    return y

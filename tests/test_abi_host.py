@@ -36,7 +36,7 @@ def test_header_declares_the_entry_points():
         "ssd_abi_version", "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_static",
         "ssd_chunk_scan_fwd_varlen", "ssd_chunk_scan_varlen_workspace_bytes",
         "ssd_chunk_scan_workspace_bytes", "ssd_conv1d_silu", "ssd_conv_scan_fwd",
-        "ssd_conv_scan_workspace_bytes", "ssd_selftest_bounded_wait",
+        "ssd_conv_scan_workspace_bytes", "ssd_decode_step", "ssd_selftest_bounded_wait",
         "ssd_state_update", "ssd_status_string"])
 
 
@@ -213,3 +213,24 @@ def test_conv_scan_validation():
         2 * 256 * 4608 * 2 + scan
     assert libssd.ssd_conv_scan_workspace_bytes(1, 256, 4, 64, 16, 1, 64, 4, F32) == 256 * 288 * 4
     assert libssd.ssd_conv_scan_workspace_bytes(0, 256, 4, 64, 16, 1, 64, 4, F32) == 0
+
+
+def dec(**kw):
+    a = dict(state=fake(1), conv_state=fake(2), xBC=fake(3), w=fake(4), bias=None, dt_raw=fake(5),
+             dt_bias=None, A=fake(6), D=None, y=fake(7), b=256, H=128, P=64, N=128, G=8, k=4,
+             dtype=BF16, stream=None)
+    a.update(kw)
+    return libssd.ssd_decode_step(**a)
+
+
+def test_decode_step_validation():
+    # every call here fails validation (or is empty work) before any launch
+    assert dec(b=0) == OK
+    for k in ("state", "conv_state", "xBC", "w", "dt_raw", "A", "y"):
+        assert dec(**{k: None}) == INV, k
+    assert dec(G=3) == INV and dec(N=6) == INV and dec(P=0) == INV and dec(dtype=9) == INV
+    assert dec(state=fake(1, 8)) == INV                          # state not 16-byte aligned
+    assert dec(xBC=fake(3, 1)) == INV                            # xBC not element aligned
+    assert dec(y=fake(3, 64)) == INV                             # y overlaps xBC
+    assert dec(conv_state=fake(1, 4096)) == INV                  # cache overlaps the state
+    assert dec(k=5) == UNS and dec(k=1) == UNS and dec(N=512) == UNS

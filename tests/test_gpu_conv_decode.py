@@ -115,3 +115,46 @@ def test_decode_step_full_layer_matches_oracle():
     # state comparison at 1e-5 is test_state_update_matches_oracle
     assert norm_max_abs(state, st_ref) <= 2e-2
     assert_output(y, y_ref, "bf16", "decode-step y")
+
+
+@pytest.mark.parametrize("b,H,P,N,G,k,dtype,bias", [
+    (256, 128, 64, 128, 8, 4, "bf16", False),   # the decode workload at full size
+    (3, 8, 64, 128, 2, 4, "bf16", True),
+    (5, 4, 64, 16, 1, 4, "f32", True),
+    (4, 6, 24, 32, 3, 3, "f32", False),
+    (2, 2, 8, 256, 1, 2, "bf16", True),
+    (7, 12, 16, 64, 4, 4, "f32", True),
+])
+def test_decode_step_kernel_matches_oracle_and_two_calls(b, H, P, N, G, k, dtype, bias):
+    """The one-kernel decode step against the oracle (conv from the raw
+    token, then the recurrence step) and, bit for bit, against the two calls
+    it fuses (conv1d_silu with L = 1, then state_update)."""
+    s = synth.LayerShape("decode", b, 1, H, P, N, G, 128, k, dtype)
+    inp = synth.decode_inputs(s, 7700 + b + N + k)
+    cd = s.conv_dim
+    bs = torch.randn(cd, generator=torch.Generator().manual_seed(b + k)) * 0.3 if bias else None
+    u_ref, cs_ref = oracle.conv1d_silu(f64(inp["xBC"]).reshape(b, 1, cd), f64(inp["w"]),
+                                       None if bs is None else f64(bs), f64(inp["conv_state"]))
+    u_ref = u_ref.reshape(b, cd)
+    y_ref, st_ref = oracle.state_update(
+        f64(inp["state"]), u_ref[:, : H * P].reshape(b, H, P), u_ref[:, H * P: H * P + G * N].reshape(b, G, N),
+        u_ref[:, H * P + G * N:].reshape(b, G, N), f64(inp["dt_raw"]), f64(inp["A"]), f64(inp["dt_bias"]),
+        f64(inp["D"]))
+    args = dict(bias=cuda(bs), dt_bias=cuda(inp["dt_bias"]), D=cuda(inp["D"]))
+    cs1, st1 = cuda(inp["conv_state"]), cuda(inp["state"])
+    y1 = layer.decode_step(cuda(inp["xBC"]), cuda(inp["w"]), cs1, st1, cuda(inp["dt_raw"]), cuda(inp["A"]),
+                           H, P, G, N, **args)
+    # the two calls
+    cs2, st2 = cuda(inp["conv_state"]), cuda(inp["state"])
+    u = layer.conv1d_silu(cuda(inp["xBC"]).view(b, 1, cd), cuda(inp["w"]), cuda(bs), cs2).view(b, cd)
+    xd, Bd, Cd = layer.split_channels(u, H, P, G, N)
+    y2 = layer.state_update(st2, xd, Bd, Cd, cuda(inp["dt_raw"]), cuda(inp["A"]), args["dt_bias"], args["D"])
+    torch.cuda.synchronize()
+    assert np.array_equal(f64(cs1), cs_ref), "conv cache roll"
+    assert torch.equal(cs1, cs2) and torch.equal(st1, st2) and torch.equal(y1, y2), "differs from the two calls"
+    # float32 conv outputs are within 1e-6 of the oracle's, so the state keeps
+    # its 1e-5 bound; bf16-rounded ones move the state at the bf16 bound
+    tol_state = TOL_STATE_F32 if dtype == "f32" else 2e-2
+    e_state = norm_max_abs(st1, st_ref)
+    assert e_state <= tol_state, f"decode state error {e_state:.3e}"
+    assert_output(y1, y_ref, dtype, "decode-step y")
