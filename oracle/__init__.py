@@ -49,6 +49,8 @@ def open_library(path: str):
     lib.oracle_selective_scan.restype = ctypes.c_int
     lib.oracle_state_update.argtypes = [d] * 9 + [i64] * 5 + [ctypes.c_int]
     lib.oracle_state_update.restype = ctypes.c_int
+    lib.oracle_selective_scan_bwd.argtypes = [d] * 18 + [i64] * 6 + [ctypes.c_int]
+    lib.oracle_selective_scan_bwd.restype = ctypes.c_int
     return lib
 
 
@@ -204,6 +206,36 @@ def state_update(state, x, B, C, dt_raw, A, dt_bias=None, D=None, nthreads: int 
     if rc != 0:
         raise ValueError("oracle_state_update: bad sizes")
     return y, st
+
+
+def selective_scan_bwd(x, B, C, dt_raw, A, dy, dt_bias=None, D=None, init_state=None, dfinal=None,
+                       nthreads: int | None = None):
+    """Gradient of sum(dy * y) + sum(dfinal * final_state) through
+    selective_scan, by the reverse-mode token loop of ssd_oracle.c.
+
+    Shapes as for selective_scan; dy [b, L, H, P], dfinal [b, H, P, N] or None.
+    Returns a dict of float64 arrays: dx, dB, dC, ddt_raw, dA, dD, ddt_bias,
+    dinit (the gradient with respect to the initial state, also when none
+    was given: the state is then zero)."""
+    x = _f64(x)
+    b, L, H, P = x.shape
+    B = _f64(B)
+    G, N = B.shape[2], B.shape[3]
+    C = _f64(C, B.shape)
+    dt_raw = _f64(dt_raw, (b, L, H))
+    dy = _f64(dy, (b, L, H, P))
+    out = dict(dx=np.empty((b, L, H, P)), dB=np.empty((b, L, G, N)), dC=np.empty((b, L, G, N)),
+               ddt_raw=np.empty((b, L, H)), dA=np.empty(H), dD=np.empty(H), ddt_bias=np.empty(H),
+               dinit=np.empty((b, H, P, N)))
+    rc = _load().oracle_selective_scan_bwd(
+        _ptr(x), _ptr(B), _ptr(C), _ptr(dt_raw), _ptr(_f64(dt_bias, (H,))), _ptr(_f64(A, (H,))),
+        _ptr(_f64(D, (H,))), _ptr(_f64(init_state, (b, H, P, N))), _ptr(dy),
+        _ptr(_f64(dfinal, (b, H, P, N))), _ptr(out["dx"]), _ptr(out["dB"]), _ptr(out["dC"]),
+        _ptr(out["ddt_raw"]), _ptr(out["dA"]), _ptr(out["dD"]), _ptr(out["ddt_bias"]), _ptr(out["dinit"]),
+        b, L, H, P, N, G, nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_selective_scan_bwd: bad sizes")
+    return out
 
 
 def split_xBC(u, H, P, G, N):

@@ -19,7 +19,11 @@ with ``oracle.using_library``) disagrees with:
 * invariants: linearity of y - D x in x, causality, state hand-off between
   calls, prefill(L) + one decode step = prefill(L + 1), conv-state hand-off;
 * the Mamba cache-size formula of the same page's appendix C, which fixes the
-  element counts of the conv state and the SSM state.
+  element counts of the conv state and the SSM state;
+* for the backward pass: central finite differences of the forward oracle for
+  every input element (brute force on a tiny problem), the closed form of dD,
+  the dt -> 0 limit, linearity in the output gradients, and independence of
+  the thread count.
 
 All inputs are small and seeded so the whole set runs in seconds on a CPU.
 """
@@ -372,6 +376,102 @@ def check_varlen_chunked_prefill():
     _close(fb, fs, 1e-13, "chunked prefill final state")
 
 
+# ----------------------------------------------------------------------------
+# backward pass
+# ----------------------------------------------------------------------------
+
+def _loss(inp, dy, dfinal):
+    y, fs = oracle.selective_scan(inp["x"], inp["B"], inp["C"], inp["dt_raw"], inp["A"], inp["dt_bias"],
+                                  inp["D"], inp["init_state"], nthreads=1)
+    return float(np.sum(dy * y) + np.sum(dfinal * fs))
+
+
+def _bwd(inp, dy, dfinal, nthreads=2):
+    return oracle.selective_scan_bwd(inp["x"], inp["B"], inp["C"], inp["dt_raw"], inp["A"], dy,
+                                     inp["dt_bias"], inp["D"], inp["init_state"], dfinal, nthreads=nthreads)
+
+
+def check_bwd_finite_differences():
+    """Every gradient element against a central difference of the forward
+    oracle's loss sum(dy * y) + sum(dfinal * final_state), step 1e-6 (error
+    O(1e-12) from the step, O(1e-10) from rounding)."""
+    rng = _rng(31)
+    inp = _random_scan_inputs(rng, b=2, L=7, H=4, P=3, N=4, G=2)
+    y, fs = _scan(inp)
+    dy = rng.standard_normal(y.shape)
+    dfinal = rng.standard_normal(fs.shape)
+    grads = _bwd(inp, dy, dfinal)
+    names = {"x": "dx", "B": "dB", "C": "dC", "dt_raw": "ddt_raw", "A": "dA", "D": "dD",
+             "dt_bias": "ddt_bias", "init_state": "dinit"}
+    eps = 1e-6
+    for key, gname in names.items():
+        base = inp[key]
+        fd = np.empty_like(base)
+        for i in np.ndindex(base.shape):
+            orig = base[i]
+            base[i] = orig + eps
+            lp = _loss(inp, dy, dfinal)
+            base[i] = orig - eps
+            lm = _loss(inp, dy, dfinal)
+            base[i] = orig
+            fd[i] = (lp - lm) / (2 * eps)
+        _close(grads[gname], fd, 1e-7, f"gradient {gname} vs finite differences")
+
+
+def check_bwd_dD_closed_form():
+    """y depends on D only through D x: dLoss/dD_h = sum over (b, t, p) of dy x."""
+    rng = _rng(32)
+    inp = _random_scan_inputs(rng, b=2, L=20, H=4, P=5, N=6, G=2)
+    dy = rng.standard_normal(inp["x"].shape)
+    g = _bwd(inp, dy, None)
+    _close(g["dD"], np.einsum("blhp,blhp->h", dy, inp["x"]), 1e-12, "dD closed form")
+
+
+def check_bwd_dt_to_zero():
+    """dt -> 0: the state stays h0, so dx = D dy, dB = 0,
+    dC_t[g] = sum over the group's heads of h0^T dy_t, and dinit = dfinal +
+    sum_t C_t dy_t^T."""
+    rng = _rng(33)
+    inp = _random_scan_inputs(rng, b=1, L=9, H=4, P=3, N=5, G=2)
+    inp["dt_raw"] = np.full_like(inp["dt_raw"], -40.0)
+    inp["dt_bias"] = np.zeros_like(inp["dt_bias"])
+    dy = rng.standard_normal(inp["x"].shape)
+    dfinal = rng.standard_normal(inp["init_state"].shape)
+    g = _bwd(inp, dy, dfinal)
+    H, G = 4, 2
+    grp = np.arange(H) // (H // G)
+    _close(g["dx"], inp["D"][None, None, :, None] * dy, 1e-12, "dt->0 dx")
+    _close(g["dB"], np.zeros_like(g["dB"]), 1e-12, "dt->0 dB")
+    dC = np.zeros_like(g["dC"])
+    for h in range(H):
+        dC[:, :, grp[h], :] += np.einsum("blp,bpn->bln", dy[:, :, h, :], inp["init_state"][:, h])
+    _close(g["dC"], dC, 1e-12, "dt->0 dC")
+    Cg = inp["C"][:, :, grp, :]
+    _close(g["dinit"], dfinal + np.einsum("blhp,blhn->bhpn", dy, Cg), 1e-12, "dt->0 dinit")
+
+
+def check_bwd_linear_in_output_gradients():
+    """The gradients are linear in (dy, dfinal)."""
+    rng = _rng(34)
+    inp = _random_scan_inputs(rng, b=1, L=15, H=2, P=4, N=3, G=1)
+    y, fs = _scan(inp)
+    d1, d2 = rng.standard_normal(y.shape), rng.standard_normal(y.shape)
+    f1, f2 = rng.standard_normal(fs.shape), rng.standard_normal(fs.shape)
+    g1, g2 = _bwd(inp, d1, f1), _bwd(inp, d2, f2)
+    g12 = _bwd(inp, 2.0 * d1 - 0.5 * d2, 2.0 * f1 - 0.5 * f2)
+    for k in g1:
+        _close(g12[k], 2.0 * g1[k] - 0.5 * g2[k], 1e-12, f"linearity {k}")
+
+
+def check_bwd_thread_count_invariance():
+    rng = _rng(35)
+    inp = _random_scan_inputs(rng, b=3, L=11, H=4, P=3, N=4, G=2)
+    dy = rng.standard_normal(inp["x"].shape)
+    a, b = _bwd(inp, dy, None, nthreads=1), _bwd(inp, dy, None, nthreads=5)
+    for k in a:
+        assert np.array_equal(a[k], b[k]), f"{k} depends on the thread count"
+
+
 ALL_CHECKS = [
     check_dt_to_zero,
     check_geometric_series,
@@ -388,4 +488,9 @@ ALL_CHECKS = [
     check_cache_size_formula,
     check_varlen_matches_each_sequence_alone,
     check_varlen_chunked_prefill,
+    check_bwd_finite_differences,
+    check_bwd_dD_closed_form,
+    check_bwd_dt_to_zero,
+    check_bwd_linear_in_output_gradients,
+    check_bwd_thread_count_invariance,
 ]

@@ -37,6 +37,15 @@ MUTANTS = {
     "conv_cache_shift": ("conv_state[(bi * conv_dim + c) * k + j] = hist[L + j];",
                          "conv_state[(bi * conv_dim + c) * k + j] = hist[L + j - (j > 0)];"),
     "conv_bias_dropped": ("double acc = bias ? bias[c] : 0.0;", "double acc = 0.0;"),
+    # backward pass
+    "bwd_output_term_dropped": ("g[p * N + n] += dyt[p] * Ct[n];", "g[p * N + n] += 0.0 * Ct[n];"),
+    "bwd_dC_from_previous_state": ("acc += dyt[p] * ht[p * N + n];", "acc += dyt[p] * hprev[p * N + n];"),
+    "bwd_dB_missing_dt": ("dBt[n] += dt * acc;", "dBt[n] += acc;"),
+    "bwd_ddt_decay_term_dropped": ("const double ddt = xgb + A * a * gh;", "const double ddt = xgb;"),
+    "bwd_sigmoid_sign": ("const double dv = ddt * sigmoid(v);", "const double dv = ddt * sigmoid(-v);"),
+    "bwd_dA_missing_dt": ("dA += dt * a * gh;", "dA += a * gh;"),
+    "bwd_state_gradient_not_decayed": ("for (int64_t i = 0; i < PN; ++i) g[i] *= a;",
+                                       "for (int64_t i = 0; i < PN; ++i) g[i] *= 1.0;"),
 }
 
 
