@@ -463,6 +463,97 @@ def check_bwd_linear_in_output_gradients():
         _close(g12[k], 2.0 * g1[k] - 0.5 * g2[k], 1e-12, f"linearity {k}")
 
 
+def _chunked_bwd(inp, dy, dfinal, Q):
+    """The backward pass evaluated chunk by chunk in matrix form (state-space
+    duality applied to the gradient; written independently of the oracle's
+    token loop).  Per chunk with entering state h0 and incoming state
+    gradient g_end, cum = inclusive cumsum of dt A, Lm[i, j] = exp(cum_i -
+    cum_j) for j <= i:
+      dC  = diag(e^cum) dY h0 + (Lm o dt_j o dY X^T) B
+      gB  = diag(e^(cum_last - cum)) B g_end^T + (Lm^T o (C B^T)^T) dY      (g_j B_j per token)
+      U   = diag(e^(cum_last - cum)) X g_end + (Lm^T o (dY X^T)^T) C         (g_j^T x_j per token)
+      dX  = D dY + diag(dt) gB,   dB = diag(dt) U,   ddt_explicit_j = U_j . B_j
+      <g_t, exp(dt_t A) h_{t-1}> = <g_t, h_t> - dt_t U_t . B_t with
+      <g_t, h_t> = e^cum_last <g_end, h0> + sum_{j<=t} e^(cum_last - cum_j) dt_j x_j^T g_end B_j
+                   + sum_{k>=t} e^cum_k dy_k^T h0 C_k + sum_{k>=t, j<=t} W[k, j],
+      W = Lm o dt_j o (dY X^T) o (C B^T), the last sum by a running update
+    and the entering state's gradient e^cum_last g_end + sum_k e^cum_k dy_k C_k^T
+    becomes the previous chunk's g_end."""
+    x, B, C, dt_raw, A, Dv = inp["x"], inp["B"], inp["C"], inp["dt_raw"], inp["A"], inp["D"]
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    grp = np.arange(H) // (H // G)
+    v = dt_raw + inp["dt_bias"][None, None, :]
+    dt = np.logaddexp(0.0, v)
+    sig = 1.0 / (1.0 + np.exp(-v))
+    out = dict(dx=np.zeros_like(x), dB=np.zeros_like(B), dC=np.zeros_like(C), ddt_raw=np.zeros_like(dt_raw),
+               dA=np.zeros(H), dD=np.zeros(H), ddt_bias=np.zeros(H), dinit=np.zeros((b, H, P, N)))
+    starts = list(range(0, L, Q))
+    for bi in range(b):
+        for h in range(H):
+            g_ = grp[h]
+            h0s = []
+            hcur = inp["init_state"][bi, h].copy() if inp["init_state"] is not None else np.zeros((P, N))
+            for s0 in starts:                          # forward: the state entering each chunk
+                h0s.append(hcur)
+                sl = slice(s0, min(L, s0 + Q))
+                cum = np.cumsum(dt[bi, sl, h] * A[h])
+                w = np.exp(cum[-1] - cum) * dt[bi, sl, h]
+                hcur = np.exp(cum[-1]) * hcur + (x[bi, sl, h].T * w) @ B[bi, sl, g_]
+            gend = dfinal[bi, h].copy() if dfinal is not None else np.zeros((P, N))
+            for ci in reversed(range(len(starts))):   # backward over chunks
+                sl = slice(starts[ci], min(L, starts[ci] + Q))
+                h0 = h0s[ci]
+                X, Bc, Cc, dY, dtc = x[bi, sl, h], B[bi, sl, g_], C[bi, sl, g_], dy[bi, sl, h], dt[bi, sl, h]
+                cum = np.cumsum(dtc * A[h])
+                q = len(dtc)
+                Lm = np.tril(np.exp(cum[:, None] - cum[None, :]))
+                YX = dY @ X.T
+                CB = Cc @ Bc.T
+                el = np.exp(cum[-1] - cum)
+                dCc = np.exp(cum)[:, None] * (dY @ h0) + (Lm * dtc[None, :] * YX) @ Bc
+                gB = el[:, None] * (Bc @ gend.T) + (Lm.T * CB.T) @ dY
+                U = el[:, None] * (X @ gend) + (Lm.T * YX.T) @ Cc
+                dX = Dv[h] * dY + dtc[:, None] * gB
+                W = Lm * dtc[None, :] * YX * CB
+                S = np.empty(q)
+                run = 0.0
+                for t in range(q):                     # sum over k >= t, j <= t of W[k, j]
+                    run += W[t:, t].sum() - (W[t - 1, :t].sum() if t > 0 else 0.0)
+                    S[t] = run
+                t1 = np.exp(cum[-1]) * np.sum(gend * h0)
+                t2 = np.cumsum(el * dtc * np.einsum("jp,pn,jn->j", X, gend, Bc))
+                t3 = np.cumsum((np.exp(cum) * np.einsum("kp,pn,kn->k", dY, h0, Cc))[::-1])[::-1]
+                ub = np.einsum("jn,jn->j", U, Bc)
+                r = t1 + t2 + t3 + S - dtc * ub
+                ddt = ub + A[h] * r
+                out["dx"][bi, sl, h] = dX
+                out["dB"][bi, sl, g_] += dtc[:, None] * U
+                out["dC"][bi, sl, g_] += dCc
+                out["ddt_raw"][bi, sl, h] = ddt * sig[bi, sl, h]
+                out["dA"][h] += np.sum(dtc * r)
+                out["dD"][h] += np.sum(dY * X)
+                gend = np.exp(cum[-1]) * gend + (dY.T * np.exp(cum)) @ Cc
+            out["dinit"][bi, h] = gend
+    out["ddt_bias"] = out["ddt_raw"].sum(axis=(0, 1))
+    return out
+
+
+def check_bwd_chunked_matrix_form():
+    """The oracle's token-loop gradients equal the chunked matrix form at
+    chunk lengths 1, 3, 8 and L (the dual evaluation of the backward pass)."""
+    rng = _rng(36)
+    inp = _random_scan_inputs(rng, b=2, L=17, H=4, P=3, N=5, G=2)
+    y, fs = _scan(inp)
+    dy = rng.standard_normal(y.shape)
+    dfinal = rng.standard_normal(fs.shape)
+    ref = _bwd(inp, dy, dfinal)
+    for Q in (1, 3, 8, 17):
+        got = _chunked_bwd(inp, dy, dfinal, Q)
+        for k in ref:
+            _close(ref[k], got[k], 1e-11, f"chunk {Q}: {k}")
+
+
 def check_bwd_thread_count_invariance():
     rng = _rng(35)
     inp = _random_scan_inputs(rng, b=3, L=11, H=4, P=3, N=4, G=2)
@@ -493,4 +584,5 @@ ALL_CHECKS = [
     check_bwd_dt_to_zero,
     check_bwd_linear_in_output_gradients,
     check_bwd_thread_count_invariance,
+    check_bwd_chunked_matrix_form,
 ]
