@@ -320,6 +320,47 @@ SSD_API ssd_status_t ssd_decode_step(float* state, void* conv_state, const void*
                                      int N, int G, int k, ssd_dtype_t dtype, cudaStream_t stream);
 
 /*
+ * Backward pass of the chunked scan: the gradients of a loss
+ * Loss(y, final_state) through ssd_chunk_scan_fwd, given dy = dLoss/dy and
+ * dfinal = dLoss/d(final_state), for training (the Nemotron feasibility
+ * report plans forward and backward tests of the Mamba-2 layer, sections
+ * 3.2 and 3.3).  The gradients follow the recurrence h_t = exp(dt_t A)
+ * h_{t-1} + dt_t x_t B_t^T, y_t = h_t C_t + D x_t of "Hybrid Architectures for
+ * Language Models" (summary page, section 2 Background) with dt =
+ * softplus(dt_raw + dt_bias).
+ *
+ *   x, B, C, row_stride, dt_raw, dt_bias, A, D, init_state
+ *                 the forward call's inputs, same layouts (init_state may be
+ *                 NULL: zero)
+ *   dy            [b][L][H][P]   dtype
+ *   dfinal        [b][H][P][N]   float32, may be NULL (zero)
+ *   dx            [b][L][H][P]   dtype, written
+ *   dB, dC        [b][L][G][N]   dtype, written (summed over each group's heads)
+ *   ddt_raw       [b][L][H]      dtype, written
+ *   dA, dD, ddt_bias [H]         float32, written (summed over the batch)
+ *   dinit         [b][H][P][N]   float32, may be NULL (not wanted)
+ *   workspace     ssd_chunk_scan_bwd_workspace_bytes(...) bytes: each chunk's
+ *                 entering state and per-head dB, dC (float32), caller-owned
+ * float32 arithmetic on the CUDA cores, chunks of 32 tokens in matrix form;
+ * deterministic.  Requirements: H % G == 0; the shared memory of one CTA,
+ * about 4 (2 P N + 64 P + 160 N + 3.8 K) bytes, within the device limit
+ * (else SSD_ERR_UNSUPPORTED; P = 64, N = 128 takes 179 KB); element-aligned
+ * I/O pointers; no output may overlap an input or another output.
+ */
+SSD_API size_t ssd_chunk_scan_bwd_workspace_bytes(int b, int L, int H, int P, int N, int G,
+                                                  ssd_dtype_t dtype);
+
+SSD_API ssd_status_t ssd_chunk_scan_bwd(const void* x, const void* B, const void* C,
+                                        int64_t row_stride, const void* dt_raw,
+                                        const float* dt_bias, const float* A, const float* D,
+                                        const float* init_state, const void* dy,
+                                        const float* dfinal, void* dx, void* dB, void* dC,
+                                        void* ddt_raw, float* dA, float* dD, float* ddt_bias,
+                                        float* dinit, int b, int L, int H, int P, int N, int G,
+                                        ssd_dtype_t dtype, void* workspace,
+                                        size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Self-test of the bounded device waits (failure detection without a fault).
  * Every wait of the tensor-core scan gives up after a time limit, records
  * SSD_ERR_TIMEOUT in the call's status word and lets the kernel run to its

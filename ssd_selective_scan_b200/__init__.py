@@ -6,12 +6,12 @@ ctypes binding and ``layer`` the torch-facing calls.  The library is loaded
 on first use and there is no fallback path: without libssd.so every call
 raises.
 """
-from .layer import (chunk_scan_fwd, chunk_scan_fwd_varlen, chunk_scan_varlen_workspace_bytes,
+from .layer import (chunk_scan_bwd, chunk_scan_bwd_workspace_bytes, chunk_scan_fwd, chunk_scan_fwd_varlen, chunk_scan_varlen_workspace_bytes,
                     chunk_scan_workspace_bytes, conv1d_silu, conv_scan_fwd, conv_scan_workspace_bytes,
                     decode_step, layer_prefill, split_channels, state_update)
 from .binding import SsdError
 
-__all__ = ["chunk_scan_fwd", "chunk_scan_fwd_varlen", "chunk_scan_varlen_workspace_bytes",
+__all__ = ["chunk_scan_bwd", "chunk_scan_bwd_workspace_bytes", "chunk_scan_fwd", "chunk_scan_fwd_varlen", "chunk_scan_varlen_workspace_bytes",
            "chunk_scan_workspace_bytes", "conv1d_silu", "conv_scan_fwd", "conv_scan_workspace_bytes",
            "decode_step",
            "layer_prefill", "split_channels", "state_update", "SsdError"]

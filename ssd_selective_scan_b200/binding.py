@@ -44,6 +44,10 @@ SIGNATURES = {
     "ssd_conv_scan_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),
     "ssd_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                              _i, _i, _i, _i, _i, _i, _i, _vp]),
+    "ssd_chunk_scan_bwd_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "ssd_chunk_scan_bwd": (_i, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "ssd_conv_scan_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp, _vp]),
 }
@@ -139,6 +143,18 @@ def ssd_decode_step(state, conv_state, xBC, w, bias, dt_raw, dt_bias, A, D, y, b
                     dtype, stream) -> int:
     return load().ssd_decode_step(state, conv_state, xBC, w, bias, dt_raw, dt_bias, A, D, y, b, H, P,
                                   N, G, k, dtype, stream)
+
+
+def ssd_chunk_scan_bwd_workspace_bytes(b, L, H, P, N, G, dtype) -> int:
+    return load().ssd_chunk_scan_bwd_workspace_bytes(b, L, H, P, N, G, dtype)
+
+
+def ssd_chunk_scan_bwd(x, B, C, row_stride, dt_raw, dt_bias, A, D, init_state, dy, dfinal, dx, dB, dC,
+                       ddt_raw, dA, dD, ddt_bias, dinit, b, L, H, P, N, G, dtype, workspace,
+                       workspace_bytes, stream) -> int:
+    return load().ssd_chunk_scan_bwd(x, B, C, row_stride, dt_raw, dt_bias, A, D, init_state, dy, dfinal,
+                                     dx, dB, dC, ddt_raw, dA, dD, ddt_bias, dinit, b, L, H, P, N, G,
+                                     dtype, workspace, workspace_bytes, stream)
 
 
 def ssd_selftest_bounded_wait(status, limit_ns, stream) -> int:

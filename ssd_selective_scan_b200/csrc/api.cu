@@ -5,6 +5,7 @@
 
 #include "kernels.h"
 #include "decode.h"
+#include "scan_bwd.h"
 
 namespace {
 
@@ -384,6 +385,78 @@ ssd_status_t ssd_decode_step(float* state, void* conv_state, const void* xBC, co
     if (ssd::decode_step_smem_bytes(H, P, N, G) > (size_t)max_optin_smem()) return SSD_ERR_UNSUPPORTED;
     return from_cuda(ssd::launch_decode_step(state, conv_state, xBC, w, bias, dt_raw, dt_bias, A, D, y, b, H, P,
                                              N, G, k, dtype == SSD_BF16, stream));
+}
+
+size_t ssd_chunk_scan_bwd_workspace_bytes(int b, int L, int H, int P, int N, int G, ssd_dtype_t dtype)
+{
+    if (b <= 0 || L <= 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || !valid_dtype(dtype)) return 0;
+    return ssd::scan_bwd_workspace_bytes(b, L, H, P, N);
+}
+
+ssd_status_t ssd_chunk_scan_bwd(const void* x, const void* B, const void* C, int64_t row_stride, const void* dt_raw,
+                                const float* dt_bias, const float* A, const float* D, const float* init_state,
+                                const void* dy, const float* dfinal, void* dx, void* dB, void* dC, void* ddt_raw,
+                                float* dA, float* dD, float* ddt_bias, float* dinit, int b, int L, int H, int P,
+                                int N, int G, ssd_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                                cudaStream_t stream)
+{
+    if (!valid_dtype(dtype) || b < 0 || L < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || H % G)
+        return SSD_ERR_INVALID_ARG;
+    if (!A || !dA || !dD || !ddt_bias) return SSD_ERR_INVALID_ARG;
+    const bool tokens = b > 0 && L > 0;
+    if (tokens && (!x || !B || !C || !dt_raw || !dy || !dx || !dB || !dC || !ddt_raw)) return SSD_ERR_INVALID_ARG;
+    if (row_stride < (int64_t)H * P || row_stride < (int64_t)G * N) return SSD_ERR_INVALID_ARG;
+    const int e = elem_bytes(dtype);
+    const void* io_ptrs[] = {x, B, C, dt_raw, dy, dx, dB, dC, ddt_raw};
+    for (const void* q : io_ptrs)
+        if (q && !aligned(q, e)) return SSD_ERR_INVALID_ARG;
+    const void* f32_ptrs[] = {dt_bias, A, D, init_state, dfinal, dA, dD, ddt_bias, dinit, workspace};
+    for (const void* q : f32_ptrs)
+        if (q && !aligned(q, 4)) return SSD_ERR_INVALID_ARG;
+    const size_t need_ws = ssd_chunk_scan_bwd_workspace_bytes(b, L, H, P, N, G, dtype);
+    if (workspace_bytes < need_ws || (need_ws && !workspace)) return SSD_ERR_INVALID_ARG;
+
+    const int64_t rows = (int64_t)b * L;
+    const int64_t row_bytes = row_stride * e;
+    const Range rx = span(x, rows ? (rows - 1) * row_bytes + (int64_t)H * P * e : 0);
+    const Range rB = span(B, rows ? (rows - 1) * row_bytes + (int64_t)G * N * e : 0);
+    const Range rC = span(C, rows ? (rows - 1) * row_bytes + (int64_t)G * N * e : 0);
+    const Range rdt = span(dt_raw, rows * H * e);
+    const Range rdy = span(dy, rows * H * P * e);
+    const int64_t st_bytes = (int64_t)b * H * P * N * 4;
+    const Range ri = span(init_state, init_state ? st_bytes : 0);
+    const Range rfin = span(dfinal, dfinal ? st_bytes : 0);
+    const Range rdx = span(dx, rows * H * P * e);
+    const Range rdB = span(dB, rows * G * N * e);
+    const Range rdC = span(dC, rows * G * N * e);
+    const Range rddt = span(ddt_raw, rows * H * e);
+    const Range rdA = span(dA, (int64_t)H * 4), rdD = span(dD, (int64_t)H * 4), rdb = span(ddt_bias, (int64_t)H * 4);
+    const Range rdi = span(dinit, dinit ? st_bytes : 0);
+    const Range rws = span(workspace, (int64_t)workspace_bytes);
+    const Range ins[] = {rx, rB, rC, rdt, rdy, ri, rfin, span(A, (int64_t)H * 4)};
+    const Range outs[] = {rdx, rdB, rdC, rddt, rdA, rdD, rdb, rdi, rws};
+    for (int i = 0; i < 9; ++i) {
+        for (const Range& in : ins)
+            if (overlap(outs[i], in)) return SSD_ERR_INVALID_ARG;
+        for (int j = i + 1; j < 9; ++j)
+            if (overlap(outs[i], outs[j])) return SSD_ERR_INVALID_ARG;
+    }
+    if (!tokens) {
+        // no tokens: the parameter gradients are zero and the initial
+        // state's gradient is the final state's (or zero)
+        cudaError_t err = cudaMemsetAsync(dA, 0, (size_t)H * 4, stream);
+        if (err == cudaSuccess) err = cudaMemsetAsync(dD, 0, (size_t)H * 4, stream);
+        if (err == cudaSuccess) err = cudaMemsetAsync(ddt_bias, 0, (size_t)H * 4, stream);
+        if (err == cudaSuccess && dinit && b > 0)
+            err = dfinal ? cudaMemcpyAsync(dinit, dfinal, (size_t)st_bytes, cudaMemcpyDeviceToDevice, stream)
+                         : cudaMemsetAsync(dinit, 0, (size_t)st_bytes, stream);
+        return from_cuda(err);
+    }
+    if ((int64_t)b * H > 0x7fffffffLL) return SSD_ERR_UNSUPPORTED;
+    if (ssd::scan_bwd_smem_bytes(P, N) > (size_t)max_optin_smem()) return SSD_ERR_UNSUPPORTED;
+    ssd::ScanBwdArgs a{x, B, C, row_stride, dt_raw, dt_bias, A, D, init_state, dy, dfinal, dx, dB, dC, ddt_raw,
+                       dA, dD, ddt_bias, dinit, b, L, H, P, N, G, dtype == SSD_BF16, workspace};
+    return from_cuda(ssd::launch_scan_bwd(a, stream));
 }
 
 }  // extern "C"

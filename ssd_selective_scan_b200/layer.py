@@ -194,6 +194,55 @@ def state_update(state: torch.Tensor, x: torch.Tensor, B: torch.Tensor, C: torch
     return y
 
 
+def chunk_scan_bwd_workspace_bytes(b, L, H, P, N, G, dtype: torch.dtype) -> int:
+    return int(libssd.ssd_chunk_scan_bwd_workspace_bytes(b, L, H, P, N, G, _DT[dtype]))
+
+
+def chunk_scan_bwd(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor, dt_raw: torch.Tensor,
+                   A: torch.Tensor, dy: torch.Tensor, dt_bias: torch.Tensor | None = None,
+                   D: torch.Tensor | None = None, init_state: torch.Tensor | None = None,
+                   dfinal: torch.Tensor | None = None, want_dinit: bool = True,
+                   workspace: torch.Tensor | None = None, stream=None) -> dict:
+    """Gradients through chunk_scan_fwd.  x, B, C, dt_raw, A, dt_bias, D,
+    init_state as for the forward call; dy [b, L, H, P] (I/O dtype), dfinal
+    [b, H, P, N] f32 or None.  Returns dict(dx, dB, dC, ddt_raw, dA, dD,
+    ddt_bias, dinit): dB, dC [b, L, G, N] and ddt_raw in the I/O dtype, the
+    parameter gradients f32 [H], dinit f32 [b, H, P, N] (None if not wanted)."""
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    if b * L == 0:
+        rs = -(-max(H * P, G * N) // 8) * 8
+    else:
+        rs = _row_view_stride(x, "x")
+        if _row_view_stride(B, "B") != rs or _row_view_stride(C, "C") != rs:
+            raise ValueError("x, B and C must share one token stride")
+    if dy.shape != (b, L, H, P) or dy.dtype != x.dtype or not dy.is_contiguous():
+        raise ValueError("dy must be a contiguous [b, L, H, P] tensor of x's dtype")
+    if dt_raw.shape != (b, L, H) or dt_raw.dtype != x.dtype or not dt_raw.is_contiguous():
+        raise ValueError("dt_raw must be a contiguous [b, L, H] tensor of x's dtype")
+    dev, dt = x.device, x.dtype
+    out = dict(dx=torch.empty((b, L, H, P), dtype=dt, device=dev),
+               dB=torch.empty((b, L, G, N), dtype=dt, device=dev),
+               dC=torch.empty((b, L, G, N), dtype=dt, device=dev),
+               ddt_raw=torch.empty((b, L, H), dtype=dt, device=dev),
+               dA=torch.empty(H, dtype=torch.float32, device=dev),
+               dD=torch.empty(H, dtype=torch.float32, device=dev),
+               ddt_bias=torch.empty(H, dtype=torch.float32, device=dev),
+               dinit=torch.empty((b, H, P, N), dtype=torch.float32, device=dev) if want_dinit else None)
+    need = chunk_scan_bwd_workspace_bytes(b, L, H, P, N, G, dt)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = libssd.ssd_chunk_scan_bwd(
+        _ptr(x), _ptr(B), _ptr(C), rs, _ptr(dt_raw), _ptr(_f32(dt_bias, "dt_bias")), _ptr(_f32(A, "A")),
+        _ptr(_f32(D, "D")), _ptr(_f32(init_state, "init_state")), _ptr(dy), _ptr(_f32(dfinal, "dfinal")),
+        _ptr(out["dx"]), _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["ddt_raw"]), _ptr(out["dA"]),
+        _ptr(out["dD"]), _ptr(out["ddt_bias"]), _ptr(out["dinit"]), b, L, H, P, N, G, _dtype_code(x),
+        _ptr(workspace), ws_bytes, _stream(stream))
+    libssd.check("ssd_chunk_scan_bwd", st)
+    return out
+
+
 def split_channels(u: torch.Tensor, H: int, P: int, G: int, N: int):
     """[.., conv_dim] -> views x [.., H, P], B [.., G, N], C [.., G, N]."""
     lead = u.shape[:-1]

@@ -33,7 +33,8 @@ def declared_entry_points():
 
 def test_header_declares_the_entry_points():
     assert declared_entry_points() == sorted([
-        "ssd_abi_version", "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_static",
+        "ssd_abi_version", "ssd_chunk_scan_bwd", "ssd_chunk_scan_bwd_workspace_bytes",
+        "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_static",
         "ssd_chunk_scan_fwd_varlen", "ssd_chunk_scan_varlen_workspace_bytes",
         "ssd_chunk_scan_workspace_bytes", "ssd_conv1d_silu", "ssd_conv_scan_fwd",
         "ssd_conv_scan_workspace_bytes", "ssd_decode_step", "ssd_selftest_bounded_wait",
@@ -234,3 +235,30 @@ def test_decode_step_validation():
     assert dec(y=fake(3, 64)) == INV                             # y overlaps xBC
     assert dec(conv_state=fake(1, 4096)) == INV                  # cache overlaps the state
     assert dec(k=5) == UNS and dec(k=1) == UNS and dec(N=512) == UNS
+
+
+def bwd(**kw):
+    a = dict(x=fake(1), B=fake(1, 2560 * 2), C=fake(1, (2560 + 1024) * 2), row_stride=4608, dt_raw=fake(2),
+             dt_bias=None, A=fake(3), D=None, init_state=None, dy=fake(4), dfinal=None, dx=fake(5), dB=fake(6),
+             dC=fake(7), ddt_raw=fake(8), dA=fake(9), dD=fake(9, 256), ddt_bias=fake(9, 512), dinit=None,
+             b=2, L=256, H=40, P=64, N=128, G=8, dtype=BF16, workspace=fake(10), workspace_bytes=1 << 33,
+             stream=None)
+    a.update(kw)
+    return libssd.ssd_chunk_scan_bwd(**a)
+
+
+def test_scan_bwd_validation():
+    # every call here fails validation before any launch
+    for k in ("x", "B", "C", "dt_raw", "A", "dy", "dx", "dB", "dC", "ddt_raw", "dA", "dD", "ddt_bias"):
+        assert bwd(**{k: None}) == INV, k
+    assert bwd(G=7) == INV and bwd(dtype=4) == INV and bwd(L=-1) == INV
+    assert bwd(row_stride=100) == INV                          # shorter than H*P
+    assert bwd(x=fake(1, 1)) == INV and bwd(dA=fake(9, 2)) == INV   # misaligned
+    assert bwd(dx=fake(4, 64)) == INV                          # dx overlaps dy
+    assert bwd(dD=fake(9, 64)) == INV                          # dD overlaps dA
+    assert bwd(workspace=fake(5)) == INV                       # workspace overlaps dx
+    assert bwd(workspace_bytes=100) == INV
+    need = libssd.ssd_chunk_scan_bwd_workspace_bytes(2, 256, 40, 64, 128, 8, BF16)
+    assert need > 2 * 40 * 8 * 64 * 128 * 4                    # the chunks' entering states, at least
+    assert libssd.ssd_chunk_scan_bwd_workspace_bytes(0, 256, 40, 64, 128, 8, BF16) == 0
+    assert bwd(N=1024, G=1, workspace_bytes=1 << 40) == UNS   # one CTA's shared memory would not fit
