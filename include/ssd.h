@@ -15,7 +15,11 @@
  *     (same section: state space duality recasts the scan as hardware-
  *     efficient matrix multiplication; chunk length 128 in the feasibility
  *     report, sections 1.4 and 2.6);
- *   - the single-token decode update of the same recurrence.
+ *   - the single-token decode update of the same recurrence;
+ *   - entry points built from these: the prefill layer in one call (conv,
+ *     then scan), ragged prefill over packed sequences (cu_seqlens), the
+ *     decode step in one kernel (cache roll, conv, update), and the scan's
+ *     backward pass (gradients for training).
  * Discretisation (the pages leave it open; this is the Mamba-2 reading):
  *   dt = softplus(dt_raw + dt_bias), Abar = exp(dt * A), Bbar = dt * B.
  *
@@ -26,8 +30,9 @@
  * Conventions shared by every call:
  *   - Every tensor argument is a DEVICE pointer owned by the caller.  The
  *     library never allocates or frees device memory, never synchronises the
- *     device or the stream, and keeps no mutable global state; calls are
- *     thread-safe.  All work is enqueued on `stream` (0 = legacy default).
+ *     device or the stream, and keeps no mutable global state (the one
+ *     exception, ssd_chunk_scan_fwd_static, says so); calls are thread-safe.
+ *     All work is enqueued on `stream` (0 = legacy default).
  *   - I/O tensors (xBC, x, B, C, dt_raw, y, conv_state) have the element
  *     type given by `dtype`; parameters (w, bias, A, D, dt_bias) and SSM
  *     states are float32.  Accumulation is float32; bf16 outputs are
@@ -45,9 +50,13 @@
  *     cudaSuccess; the error is cleared).  Asynchronous faults surface at the
  *     caller's next synchronisation, as for any CUDA work.
  *   - Empty work (b == 0 or L == 0) returns SSD_OK and launches no kernel;
- *     the token tensors are then never touched and may be NULL.  The one
- *     exception is ssd_chunk_scan_fwd with b > 0, L == 0 and a final_state:
- *     it enqueues a copy of init_state (or zeros) into final_state.
+ *     the token tensors are then never touched and may be NULL.  The
+ *     exceptions write what a sequence of no tokens still defines:
+ *     ssd_chunk_scan_fwd and ssd_conv_scan_fwd with b > 0, L == 0 and a
+ *     final_state enqueue a copy of init_state (or zeros) into final_state;
+ *     ssd_chunk_scan_fwd_varlen with empty sequences writes their final
+ *     states; ssd_chunk_scan_bwd zeroes dA, dD and ddt_bias and copies
+ *     dfinal (or zeros) into dinit.
  */
 #ifndef SSD_H_
 #define SSD_H_
