@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import oracle
-from parity_util import assert_output, cuda, f64, norm_max_abs
+from parity_util import assert_output, assert_state, cuda, f64, norm_max_abs
 from ssd_selective_scan_b200 import layer, synth
 
 pytestmark = pytest.mark.gpu
@@ -44,9 +44,7 @@ def _check_oracle(got, ref, s, what):
     (y, fs, cs), (y_ref, fs_ref, cs_ref) = got, ref
     torch.cuda.synchronize()
     assert_output(y, y_ref, s.dtype, f"{what} y")
-    tol = 1e-4 if s.dtype == "f32" else 2e-2
-    es = norm_max_abs(fs, fs_ref)
-    assert es <= tol, f"{what} final state: normalised error {es:.3e} > {tol}"
+    assert_state(fs, fs_ref, s.dtype, f"{what} final state")
     if cs is not None:
         assert np.array_equal(f64(cs), cs_ref), f"{what}: conv cache differs (its columns are copies)"
 
@@ -64,6 +62,9 @@ CASES = {
     # more chains than the persistent grid has CTAs: chains cut between CTAs
     "many_chains_handoff": (BF16.with_(b=4, L=520, H=40), dict(conv_state=True, init_state=True)),
     "h128_g8": (BF16.with_(b=2, L=300, H=128), dict(conv_state=True)),
+    # one head per group, and two, on the tensor-core scan
+    "tc_g_eq_h": (BF16.with_(b=2, L=300, H=8, G=8), dict(conv_state=True, init_state=True)),
+    "tc_two_heads_per_group": (BF16.with_(b=2, L=300, H=8, G=4), dict(conv_state=True, conv_bias=True)),
     "g1_long_memory": (BF16.with_(b=1, L=640, H=6, G=1), dict(a_range=(0.01, 2.0), conv_state=True)),
 }
 

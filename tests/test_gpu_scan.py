@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import oracle
-from parity_util import assert_output, cuda, f64, norm_max_abs
+from parity_util import assert_output, assert_state, cuda, f64, norm_max_abs
 from ssd_selective_scan_b200 import layer, synth
 
 pytestmark = pytest.mark.gpu
@@ -42,9 +42,7 @@ def _gpu_scan(inp, s, u=None, L=None, init_state="inp", final_state=True):
 def _check(y, fs, y_ref, fs_ref, s, what):
     torch.cuda.synchronize()
     e = assert_output(y, y_ref, s.dtype, f"{what} y")
-    tol = 1e-4 if s.dtype == "f32" else 2e-2
-    es = norm_max_abs(fs, fs_ref)
-    assert es <= tol, f"{what} final state: normalised error {es:.3e} > {tol}"
+    es = assert_state(fs, fs_ref, s.dtype, f"{what} final state")
     return e, es
 
 
@@ -53,6 +51,10 @@ CASES = {
     "f32_ragged_n128": (synth.CONFIGS[0].with_(b=2, L=200, H=4, N=128, G=2), dict(init_state=True)),
     "bf16_ragged_q128": (synth.CONFIGS[1].with_(b=2, L=300, H=8, G=2), dict(init_state=True)),
     "bf16_q64_g_eq_h": (synth.CONFIGS[1].with_(b=1, L=200, H=4, G=4, Q=64), {}),
+    # the tensor-core path (bf16, P 64, N 128, Q 128) with one head per group
+    # and with two: every head runs its own recurrence on its group's B and C
+    "bf16_tc_g_eq_h": (synth.CONFIGS[1].with_(b=2, L=300, H=8, G=8), dict(init_state=True)),
+    "bf16_tc_two_heads_per_group": (synth.CONFIGS[1].with_(b=2, L=300, H=8, G=4), dict(dt_bias=True)),
     "bf16_g1": (synth.CONFIGS[1].with_(b=1, L=256, H=6, G=1), dict(dt_bias=True)),
     "bf16_long_memory": (synth.CONFIGS[1].with_(b=1, L=640, H=4, G=2),
                          dict(a_range=(0.01, 2.0), init_state=True)),
