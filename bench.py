@@ -2,23 +2,29 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = one prefill layer call over one batch of the FRANKENSTALLM-H 3B
-layer shape (batch 8 x 2048 tokens, 40 heads x 64, d_state 128, 8 groups,
-chunk 128, conv 4, bf16 I/O, fp32 state): causal conv1d+SiLU, then the
-chunked SSD scan (dt softplus, chunk cumsum, C.B^T o L times X, chunk states,
-state passing, C.h + D.x), with inputs resident in HBM.  Rank 0 prints one
-JSON line.  Next to the headline prefill number the line carries:
-  roofline      the scan kernel's achieved HBM GB/s (algorithmic bytes per
-                launch / its CUDA-event duration) against the measured peak;
-  scan_only     tokens/s of the scan kernel alone;
+One step = one prefill layer call over one batch of the Nemotron-3-Nano-shaped
+long-context workload (1 sequence x 262144 tokens, 64 heads x 64, d_state 128,
+8 groups, chunk 128, conv 4, bf16 I/O, fp32 state): causal conv1d+SiLU, then
+the chunked SSD scan (dt softplus, chunk cumsum, C.B^T o L times X, chunk
+states, state passing, C.h + D.x), with inputs resident in HBM.  Rank 0
+prints one JSON line.  Next to the headline prefill number the line carries:
+  roofline      the scan kernel's achieved HBM GB/s on the headline workload
+                (algorithmic bytes per launch / its CUDA-event duration)
+                against the measured peak;
+  prefill       the same measurement (layer tokens/s, scan and conv rooflines)
+                for each prefill workload: the FRANKENSTALLM-H 3B layer (8 x
+                2048 tokens, 40 heads), the Nemotron-H 8B layer (4 x 4096
+                tokens, 128 heads) and the headline one;
   decode        one decode step of the 256-sequence, 128-head workload
                 (conv-cache roll, conv + SiLU and state update in one
                 kernel), its GB/s; the two-kernel form beside it;
-  e2e           the same prefill step through the public one-call entry point
-                (ssd_conv_scan_fwd) with the step's inputs copied from pinned
-                host memory and y + final state copied back, inside the timed
-                region;
-  cpu_baseline  the fp64 oracle timed on this host's cores on a bounded sample.
+  backward      the scan's backward pass on the 3B layer;
+  e2e           the headline prefill step through the public one-call entry
+                point (ssd_conv_scan_fwd) with the step's inputs copied from
+                pinned host memory and y + final state copied back, inside the
+                timed region;
+  cpu_baseline  the fp64 oracle timed on this host's cores on a bounded sample
+                (a 4096-token prefix of the headline workload).
 Multi-GPU: one process per GPU (torchrun); each rank runs its own batch
 (independent sequences, no data-path collective): weak scaling.
 ``--impl reference`` times the fp64 CPU oracle instead (rank 0 only).
@@ -45,8 +51,12 @@ import torch  # noqa: E402
 from ssd_selective_scan_b200 import shard, synth  # noqa: E402
 
 METRIC = "SSD prefill scan tokens/s/layer & % roofline; decode state-update HBM GB/s"
-PREFILL = synth.CONFIGS[1]
+HEADLINE = 3                      # the largest single-GPU prefill workload
+PREFILL_CONFIGS = (1, 2, 3)
+PREFILL = synth.CONFIGS[HEADLINE]
+BWD = synth.CONFIGS[1]            # the backward pass is timed on the 3B layer
 DECODE = synth.CONFIGS[4]
+ORACLE_PREFIX = 4096              # tokens of the headline workload the oracle times
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
 
@@ -71,6 +81,11 @@ def conv_bytes_per_token(s) -> int:
 def decode_state_update_bytes(s) -> int:
     """fp32 state read + written, x/B/C/dt read, y written."""
     return 8 * s.b * s.H * s.P * s.N + s.elem_bytes * s.b * (s.H * s.P + 2 * s.G * s.N + s.H + s.H * s.P)
+
+
+def scan_bwd_bytes_per_token(s) -> int:
+    """Backward pass: x, B, C, dt, dy read; dx, dB, dC, ddt written."""
+    return s.elem_bytes * (3 * s.H * s.P + 4 * s.G * s.N + 2 * s.H)
 
 
 def decode_step_bytes(s) -> int:
@@ -197,7 +212,7 @@ class ClockSampler:
 # ----------------------------------------------------------------------------
 
 class PrefillStep:
-    def __init__(self, s, seed, dev):
+    def __init__(self, s, seed, dev, layer_call: bool = False):
         from ssd_selective_scan_b200 import layer
         self.layer = layer
         self.s = s
@@ -211,8 +226,10 @@ class PrefillStep:
         self.views = layer.split_channels(self.u, s.H, s.P, s.G, s.N)
         need = layer.chunk_scan_workspace_bytes(s.b, s.L, s.H, s.P, s.N, s.G, s.Q, s.torch_dtype)
         self.ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev) if need else None
-        need = layer.conv_scan_workspace_bytes(s.b, s.L, s.H, s.P, s.N, s.G, s.Q, s.k, s.torch_dtype)
-        self.ws_layer = torch.empty(need, dtype=torch.uint8, device=dev)
+        self.ws_layer = None
+        if layer_call:
+            need = layer.conv_scan_workspace_bytes(s.b, s.L, s.H, s.P, s.N, s.G, s.Q, s.k, s.torch_dtype)
+            self.ws_layer = torch.empty(need, dtype=torch.uint8, device=dev)
 
     def conv(self):
         d = self.d
@@ -235,6 +252,28 @@ class PrefillStep:
                                  bias=d["bias"], conv_state=self.conv_state, dt_bias=d["dt_bias"],
                                  D=d["D"], Q=s.Q, y=self.y, final_state=self.fs,
                                  workspace=self.ws_layer)
+
+
+class BackwardStep:
+    """The scan's backward pass on the scan inputs of a prefill workload."""
+
+    def __init__(self, s, seed, dev):
+        from ssd_selective_scan_b200 import layer
+        self.layer = layer
+        self.s = s
+        inp = synth.scan_inputs(s, seed)
+        self.d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+        g = torch.Generator().manual_seed(seed + 1)
+        self.dy = torch.randn(s.b, s.L, s.H, s.P, generator=g).to(s.torch_dtype).to(dev)
+        self.views = layer.split_channels(self.d["u"], s.H, s.P, s.G, s.N)
+        need = layer.chunk_scan_bwd_workspace_bytes(s.b, s.L, s.H, s.P, s.N, s.G, s.torch_dtype)
+        self.ws = torch.empty(need, dtype=torch.uint8, device=dev)
+
+    def __call__(self):
+        d, s = self.d, self.s
+        x, B, C = self.views
+        self.layer.chunk_scan_bwd(x, B, C, d["dt_raw"], d["A"], self.dy, d["dt_bias"], d["D"], None,
+                                  None, want_dinit=False, workspace=self.ws)
 
 
 class DecodeStep:
@@ -270,11 +309,57 @@ def _events(n):
     return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
 
 
+def workload_config(s) -> dict:
+    """The `config` block of a prefill workload (the same in both arms)."""
+    return {"workload": s.name, "batch": s.b, "seq_len": s.L, "heads": s.H, "head_dim": s.P,
+            "d_state": s.N, "groups": s.G, "chunk": s.Q, "conv": s.k, "state_dtype": "f32",
+            "per_rank_batch": s.b,
+            "l2": f"inputs larger than L2 (xBC {s.b * s.L * s.conv_dim * s.elem_bytes / 1e6:.0f} MB, "
+                  f"conv output the same, per step)",
+            "step": "conv1d+SiLU then chunked SSD scan (one prefill layer)"}
+
+
+def scan_roofline(s, scan_ms: float, peaks: dict, traffic) -> dict:
+    tokens = s.b * s.L
+    scan_bytes = scan_bytes_per_token(s) * tokens
+    flops = scan_flops_per_token(s) * tokens
+    achieved = scan_bytes / (scan_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": "chunk_scan", "achieved": achieved,
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+            "traffic": traffic, "algorithmic_bytes_per_launch": scan_bytes,
+            "algorithmic_flops_per_launch": flops,
+            "tensor_frac": flops / (scan_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "peak_source": peaks["source"], "launch_ms": scan_ms}
+
+
+def time_prefill(step, K, W, barrier, max_over_ranks):
+    """W untimed steps, then K timed steps with per-kernel CUDA events on the
+    launching stream.  Returns (ms per step, mean conv ms, mean scan ms), each
+    the max over ranks."""
+    for _ in range(W):
+        step()
+    ev_scan = _events(2 * K)
+    ev_conv = _events(2 * K)
+    t0, t1 = _events(2)
+    barrier()
+    t0.record()
+    for i in range(K):
+        ev_conv[2 * i].record()
+        step.conv()
+        ev_conv[2 * i + 1].record()
+        ev_scan[2 * i].record()
+        step.scan()
+        ev_scan[2 * i + 1].record()
+    t1.record()
+    barrier()
+    ms_step = max_over_ranks(t0.elapsed_time(t1) / K)
+    scan_ms = max_over_ranks(statistics.mean(ev_scan[2 * i].elapsed_time(ev_scan[2 * i + 1]) for i in range(K)))
+    conv_ms = max_over_ranks(statistics.mean(ev_conv[2 * i].elapsed_time(ev_conv[2 * i + 1]) for i in range(K)))
+    return ms_step, conv_ms, scan_ms
+
+
 def run_ours(args, rank, world, dev):
     import torch.distributed as dist
-    s = PREFILL
-    step = PrefillStep(s, shard.rank_seed(synth.config_seed(1), rank), dev)
-    dec = DecodeStep(DECODE, shard.rank_seed(synth.config_seed(4), rank), dev)
 
     def barrier():
         if world > 1:
@@ -284,42 +369,80 @@ def run_ours(args, rank, world, dev):
     def max_over_ranks(v: float) -> float:
         return shard.max_over_ranks(v, dev)
 
-    for _ in range(args.warmup):
-        step()
     K = args.steps
-    ev_scan = _events(2 * K)
-    ev_conv = _events(2 * K)
-    t0, t1 = _events(2)
+    peaks = load_peaks()
+
+    # the other prefill workloads, each measured the same way
+    blocks = {}
+    for cfg in PREFILL_CONFIGS:
+        if cfg == HEADLINE:
+            continue
+        s = synth.CONFIGS[cfg]
+        st = PrefillStep(s, shard.rank_seed(synth.config_seed(cfg), rank), dev)
+        ms_step, conv_ms, scan_ms = time_prefill(st, K, args.warmup, barrier, max_over_ranks)
+        tokens = s.b * s.L
+        blocks[s.name] = {
+            "tokens_per_s": shard.aggregate_tokens_per_s(tokens, world, ms_step), "ms_per_step": ms_step,
+            "scan": scan_roofline(s, scan_ms, peaks, scan_kernel_traffic(f"chunk_scan@{s.name}")),
+            "conv": {"ms": conv_ms, "GB/s": conv_bytes_per_token(s) * tokens / (conv_ms * 1e-3) / 1e9,
+                     "frac_hbm": conv_bytes_per_token(s) * tokens / (conv_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}}
+        del st
+        torch.cuda.empty_cache()
+
+    # the headline workload, with the clocks sampled over its timed region
+    s = PREFILL
+    step = PrefillStep(s, shard.rank_seed(synth.config_seed(HEADLINE), rank), dev, layer_call=True)
     barrier()
     with ClockSampler(dev) as clk:
-        t0.record()
-        for i in range(K):
-            ev_conv[2 * i].record()
-            step.conv()
-            ev_conv[2 * i + 1].record()
-            ev_scan[2 * i].record()
-            step.scan()
-            ev_scan[2 * i + 1].record()
-        t1.record()
-        barrier()
+        ms_step, conv_ms, scan_ms = time_prefill(step, K, args.warmup, barrier, max_over_ranks)
         # keep the sampler alive over a longer stretch of identical work so the
         # clock record has enough samples (not part of the timed number)
-        t_end = time.time() + max(0.0, 1.5 - t0.elapsed_time(t1) / 1e3)
+        t_end = time.time() + max(0.0, 1.5 - ms_step * K / 1e3)
         while time.time() < t_end:
-            for _ in range(20):
+            for _ in range(5):
                 step()
             torch.cuda.synchronize()
     clocks = clk.summary()
-    ms_total = max_over_ranks(t0.elapsed_time(t1))
-    ms_step = ms_total / K
-    scan_ms = statistics.mean(ev_scan[2 * i].elapsed_time(ev_scan[2 * i + 1]) for i in range(K))
-    conv_ms = statistics.mean(ev_conv[2 * i].elapsed_time(ev_conv[2 * i + 1]) for i in range(K))
-    scan_ms = max_over_ranks(scan_ms)
-    conv_ms = max_over_ranks(conv_ms)
     tokens = s.b * s.L
+    head_roof = scan_roofline(s, scan_ms, peaks, scan_kernel_traffic(f"chunk_scan@{s.name}"))
+    blocks[s.name] = {
+        "tokens_per_s": shard.aggregate_tokens_per_s(tokens, world, ms_step), "ms_per_step": ms_step,
+        "scan": head_roof,
+        "conv": {"ms": conv_ms, "GB/s": conv_bytes_per_token(s) * tokens / (conv_ms * 1e-3) / 1e9,
+                 "frac_hbm": conv_bytes_per_token(s) * tokens / (conv_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}}
+
+    # end to end through the public API: H2D inputs, the layer, D2H results
+    pin_x = step.host["xBC"].pin_memory()
+    pin_dt = step.host["dt_raw"].pin_memory()
+    out_y = torch.empty(step.y.shape, dtype=step.y.dtype, pin_memory=True)
+    out_fs = torch.empty(step.fs.shape, dtype=torch.float32, pin_memory=True)
+    KE = max(3, min(10, K // 4))
+
+    def e2e_step():
+        step.d["xBC"].copy_(pin_x, non_blocking=True)
+        step.d["dt_raw"].copy_(pin_dt, non_blocking=True)
+        step.layer_call()
+        out_y.copy_(step.y, non_blocking=True)
+        out_fs.copy_(step.fs, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    e0, e1 = _events(2)
+    barrier()
+    e0.record()
+    for _ in range(KE):
+        e2e_step()
+    e1.record()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / KE)
+    h2d = pin_x.numel() * pin_x.element_size() + pin_dt.numel() * pin_dt.element_size()
+    d2h = out_y.numel() * out_y.element_size() + out_fs.numel() * 4
+    del step, pin_x, pin_dt, out_y, out_fs
+    torch.cuda.empty_cache()
 
     # decode: one token per sequence through the one-kernel decode step (the
     # state is rewritten in place, so consecutive steps are valid work)
+    dec = DecodeStep(DECODE, shard.rank_seed(synth.config_seed(4), rank), dev)
     for _ in range(max(3, args.warmup)):
         dec()
     KD = max(10, K)
@@ -347,40 +470,28 @@ def run_ours(args, rank, world, dev):
     barrier()
     two_ms = max_over_ranks(d2.elapsed_time(d3) / KD)
     upd_ms = max_over_ranks(statistics.mean(ev_u[2 * i].elapsed_time(ev_u[2 * i + 1]) for i in range(KD)))
+    del dec
+    torch.cuda.empty_cache()
 
-    # end to end through the public API: H2D inputs, the layer, D2H results
-    pin_x = step.host["xBC"].pin_memory()
-    pin_dt = step.host["dt_raw"].pin_memory()
-    out_y = torch.empty(step.y.shape, dtype=step.y.dtype, pin_memory=True)
-    out_fs = torch.empty(step.fs.shape, dtype=torch.float32, pin_memory=True)
-    KE = max(3, K // 4)
-
-    def e2e_step():
-        step.d["xBC"].copy_(pin_x, non_blocking=True)
-        step.d["dt_raw"].copy_(pin_dt, non_blocking=True)
-        step.layer_call()
-        out_y.copy_(step.y, non_blocking=True)
-        out_fs.copy_(step.fs, non_blocking=True)
-
-    for _ in range(2):
-        e2e_step()
-    e0, e1 = _events(2)
+    # the backward pass of the scan on the 3B layer
+    bwd = BackwardStep(BWD, shard.rank_seed(synth.config_seed(1), rank), dev)
+    for _ in range(3):
+        bwd()
+    KB = max(3, min(20, K))
+    b0, b1 = _events(2)
     barrier()
-    e0.record()
-    for _ in range(KE):
-        e2e_step()
-    e1.record()
+    b0.record()
+    for _ in range(KB):
+        bwd()
+    b1.record()
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / KE)
-    h2d = pin_x.numel() * pin_x.element_size() + pin_dt.numel() * pin_dt.element_size()
-    d2h = out_y.numel() * out_y.element_size() + out_fs.numel() * 4
+    bwd_ms = max_over_ranks(b0.elapsed_time(b1) / KB)
+    del bwd
+    torch.cuda.empty_cache()
 
     if rank != 0:
         return None
-    peaks = load_peaks()
-    scan_bytes = scan_bytes_per_token(s) * tokens
-    achieved = scan_bytes / (scan_ms * 1e-3) / 1e9
-    traffic = scan_kernel_traffic("chunk_scan")
+    btok = BWD.b * BWD.L
     line = {
         "metric": METRIC,
         "value": shard.aggregate_tokens_per_s(tokens, world, ms_step),
@@ -394,22 +505,11 @@ def run_ours(args, rank, world, dev):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": s.name, "batch": s.b, "seq_len": s.L, "heads": s.H,
-                   "head_dim": s.P, "d_state": s.N, "groups": s.G, "chunk": s.Q, "conv": s.k,
-                   "state_dtype": "f32", "per_rank_batch": s.b,
-                   "l2": "inputs larger than L2 (xBC 151 MB, conv output 151 MB per step)",
-                   "step": "conv1d+SiLU then chunked SSD scan (one prefill layer)"},
-        "roofline": {"bound": "hbm", "kernel": "chunk_scan", "achieved": achieved,
-                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                     "algorithmic_bytes_per_launch": scan_bytes,
-                     "algorithmic_flops_per_launch": scan_flops_per_token(s) * tokens,
-                     "tensor_frac": scan_flops_per_token(s) * tokens / (scan_ms * 1e-3) / 1e12 /
-                                    peaks["bf16_tflops"],
-                     "peak_source": peaks["source"], "launch_ms": scan_ms},
+        "config": workload_config(s),
+        "roofline": head_roof,
         "scan_only": {"tokens_per_s": tokens / (scan_ms * 1e-3), "ms": scan_ms},
-        "conv": {"ms": conv_ms, "GB/s": conv_bytes_per_token(s) * tokens / (conv_ms * 1e-3) / 1e9,
-                 "frac_hbm": conv_bytes_per_token(s) * tokens / (conv_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "conv": blocks[s.name]["conv"],
+        "prefill": blocks,
         "decode": {"workload": DECODE.name,
                    "kernel": "decode_step (conv-cache roll, conv + SiLU, state update: one launch)",
                    "ms_per_step": dec_ms,
@@ -417,7 +517,13 @@ def run_ours(args, rank, world, dev):
                    "frac_hbm": decode_step_bytes(DECODE) / (dec_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                    "tokens_per_s": world * DECODE.b / (dec_ms * 1e-3),
                    "two_kernel_ms_per_step": two_ms, "state_update_ms": upd_ms,
-                   "state_update_GB/s": decode_state_update_bytes(DECODE) / (upd_ms * 1e-3) / 1e9},
+                   "state_update_GB/s": decode_state_update_bytes(DECODE) / (upd_ms * 1e-3) / 1e9,
+                   "state_update_frac_hbm": decode_state_update_bytes(DECODE) / (upd_ms * 1e-3) / 1e9 /
+                                            peaks["hbm_gbs"]},
+        "backward": {"workload": BWD.name, "kernel": "chunk_scan_bwd (CUDA cores, fp32 arithmetic)",
+                     "ms": bwd_ms, "tokens_per_s": world * btok / (bwd_ms * 1e-3),
+                     "GB/s": scan_bwd_bytes_per_token(BWD) * btok / (bwd_ms * 1e-3) / 1e9,
+                     "frac_hbm": scan_bwd_bytes_per_token(BWD) * btok / (bwd_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
         "e2e": {"value": shard.aggregate_tokens_per_s(tokens, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": 2 * K,   # conv + scan per timed prefill step
@@ -430,57 +536,60 @@ def run_ours(args, rank, world, dev):
 # the fp64 oracle on the host (cpu_baseline and the reference arm)
 # ----------------------------------------------------------------------------
 
-def oracle_sample(seqs: int = 1):
-    """One oracle prefill-layer call on `seqs` sequences of the bench workload."""
-    import numpy as np
+def oracle_sample(tokens: int = ORACLE_PREFIX):
+    """One oracle prefill-layer call on the first `tokens` tokens of the
+    headline workload (the same seeded inputs, cut to a prefix)."""
     import oracle
-    s = PREFILL.with_(b=seqs)
-    inp = synth.layer_inputs(s, synth.config_seed(1))
-    f = lambda t: None if t is None else t.to(torch.float64).numpy()
-    args = (f(inp["xBC"]), f(inp["w"]), f(inp["bias"]), None, f(inp["dt_raw"]), f(inp["A"]),
-            f(inp["dt_bias"]), f(inp["D"]), None, s.H, s.P, s.G, s.N)
+    s = PREFILL
+    inp = synth.layer_inputs(s, synth.config_seed(HEADLINE))
+    f = lambda t: None if t is None else t[:, :tokens].to(torch.float64).numpy()
+    g = lambda t: None if t is None else t.to(torch.float64).numpy()
+    args = (f(inp["xBC"]), g(inp["w"]), g(inp["bias"]), None, f(inp["dt_raw"]), g(inp["A"]),
+            g(inp["dt_bias"]), g(inp["D"]), None, s.H, s.P, s.G, s.N)
+    del inp
     threads = min(oracle.default_threads(), s.b * s.H)
 
     def run():
         t = time.perf_counter()
         oracle.layer_prefill(*args, nthreads=threads)
         return time.perf_counter() - t
-    return s, run, threads
+    return s.b * tokens, run, threads
 
 
-def cpu_baseline(seqs: int = PREFILL.b, min_seconds: float = 10.0, max_runs: int = 50):
-    """The oracle on the bench batch, repeated until about `min_seconds` of
-    CPU time have passed (a bounded sample: at most `max_runs` runs)."""
-    s, run, threads = oracle_sample(seqs)
+def cpu_baseline(min_seconds: float = 10.0, max_runs: int = 50):
+    """The oracle on a 4096-token prefix of the headline workload, repeated
+    until about `min_seconds` of CPU time have passed (a bounded sample: at
+    most `max_runs` runs)."""
+    ntok, run, threads = oracle_sample()
     run()  # warm (compile, page in)
     secs, runs = 0.0, 0
     while secs < min_seconds and runs < max_runs:
         secs += run()
         runs += 1
-    return {"value": runs * s.b * s.L / secs, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{runs} runs of {s.b} of {PREFILL.b} sequences x {s.L} tokens of the bench "
-                      f"workload, conv1d+SiLU and token-by-token scan in fp64, {threads} threads",
+    return {"value": runs * ntok / secs, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{runs} runs of the first {ORACLE_PREFIX} of {PREFILL.L} tokens of the headline "
+                      f"workload ({PREFILL.H} heads), conv1d+SiLU and token-by-token scan in fp64, "
+                      f"{threads} threads",
             "seconds": secs}
 
 
 def run_reference(args):
-    s, run, threads = oracle_sample(1)
+    ntok, run, threads = oracle_sample()
     for _ in range(args.warmup):
         run()
     secs = [run() for _ in range(args.steps)]
     total = sum(secs)
-    v = args.steps * s.b * s.L / total
+    v = args.steps * ntok / total
     return {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": PREFILL.name, "batch": PREFILL.b, "seq_len": PREFILL.L,
-                   "heads": PREFILL.H, "head_dim": PREFILL.P, "d_state": PREFILL.N,
-                   "groups": PREFILL.G, "chunk": PREFILL.Q, "conv": PREFILL.k,
-                   "step": "fp64 oracle: conv1d+SiLU then token-by-token recurrence, one sequence"},
+        "config": workload_config(PREFILL),
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                         "sample": f"1 of {PREFILL.b} sequences x {PREFILL.L} tokens per step"},
+                         "sample": f"each step: the fp64 oracle (conv1d+SiLU, token-by-token "
+                                   f"recurrence) on the first {ORACLE_PREFIX} of the workload's "
+                                   f"{PREFILL.L} tokens, {threads} threads"},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -489,8 +598,14 @@ def run_one_kernel(args, dev):
     """Launch one kernel of the bench workloads alone (for ncu captures)."""
     if args.kernel == "decode":
         fn = DecodeStep(DECODE, synth.config_seed(4), dev)
+    elif args.kernel == "bwd":
+        s = BWD if args.seq_len is None else BWD.with_(L=args.seq_len)
+        fn = BackwardStep(s, synth.config_seed(1), dev)
     else:
-        st = PrefillStep(PREFILL, synth.config_seed(1), dev)
+        s = synth.CONFIGS[args.workload]
+        if args.seq_len is not None:
+            s = s.with_(L=args.seq_len)
+        st = PrefillStep(s, synth.config_seed(args.workload), dev)
         st.conv()
         fn = st.scan if args.kernel == "scan" else st.conv
     for _ in range(args.warmup):
@@ -502,20 +617,24 @@ def run_one_kernel(args, dev):
         fn()
     e1.record()
     torch.cuda.synchronize()
-    print(json.dumps({"kernel": args.kernel, "launches": args.steps,
-                      "ms_per_launch": e0.elapsed_time(e1) / args.steps}), flush=True)
+    print(json.dumps({"kernel": args.kernel, "workload": args.workload, "seq_len": args.seq_len,
+                      "launches": args.steps, "ms_per_launch": e0.elapsed_time(e1) / args.steps}), flush=True)
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["scan", "conv", "decode"],
-                    help="launch only this kernel (warmup + steps launches on the bench "
-                         "workload) and print its mean CUDA-event time; for profiler captures")
+    ap.add_argument("--kernel", choices=["scan", "conv", "decode", "bwd"],
+                    help="launch only this kernel (warmup + steps launches) and print its mean "
+                         "CUDA-event time; for profiler captures")
+    ap.add_argument("--workload", type=int, choices=PREFILL_CONFIGS, default=HEADLINE,
+                    help="prefill workload of --kernel scan|conv")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="--kernel only: a shorter sequence of the same workload (small captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
