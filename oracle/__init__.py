@@ -256,3 +256,62 @@ def layer_prefill(xBC, w, bias, conv_state, dt_raw, A, dt_bias, D, init_state, H
     x, B, C = split_xBC(u, H, P, G, N)
     y, fs = selective_scan(x, B, C, dt_raw, A, dt_bias, D, init_state, nthreads)
     return y, fs, cs
+
+
+# ---------------------------------------------------------------------------
+# The Mamba-2 mixer around the path: in_proj, conv1d+SiLU, the scan, the
+# gated RMSNorm and out_proj (Nemotron feasibility report, section 3.2: the
+# block is x + Mamba2(RMSNorm(x)); section 3.3: in_proj / out_proj are
+# linear layers, the scan stays bf16/fp32).  The pages fix neither the order
+# of the in_proj outputs nor the gate; the readings taken are: output rows
+# z (H*P) | xBC (H*P + 2*G*N) | dt_raw (H); the gate y * SiLU(z); then an
+# RMSNorm over each of `groups` equal slices of every token's H*P vector
+# (one slice by default), times a weight.
+# ---------------------------------------------------------------------------
+
+def silu(v):
+    """SiLU(v) = v / (1 + e^-v) in float64 (v -> -inf gives -0)."""
+    v = np.asarray(v, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return v / (1.0 + np.exp(-v))
+
+
+def rmsnorm_gated(y, z, weight, groups: int = 1, eps: float = 1e-5):
+    """g = y * SiLU(z); every token's vector (last axis) is cut into `groups`
+    equal contiguous slices, each divided by sqrt(mean of its squares + eps),
+    then the whole vector is multiplied elementwise by weight."""
+    g = np.asarray(y, dtype=np.float64) * silu(z)
+    shp = g.shape
+    d = shp[-1]
+    if d % groups:
+        raise ValueError("rmsnorm_gated: groups must divide the vector length")
+    gs = g.reshape(*shp[:-1], groups, d // groups)
+    ms = np.mean(gs * gs, axis=-1, keepdims=True)
+    return (gs / np.sqrt(ms + eps)).reshape(shp) * np.asarray(weight, dtype=np.float64)
+
+
+def mixer_forward(hidden, W_in, conv_w, conv_bias, dt_bias, A, D, norm_w, W_out, H, P, G, N, *,
+                  norm_groups: int = 1, eps: float = 1e-5, conv_state=None, init_state=None,
+                  nthreads: int | None = None):
+    """The Mamba-2 mixer in float64.
+
+    hidden [b, L, d_model]; W_in [2 H P + 2 G N + H, d_model] (rows: z, xBC,
+    dt_raw); conv_w [conv_dim, k], conv_bias [conv_dim] or None; dt_bias, A,
+    D [H]; norm_w [H P]; W_out [d_model, H P].  Returns (out [b, L, d_model],
+    final_state [b, H, P, N], conv_state_out [b, conv_dim, k])."""
+    hidden = _f64(hidden)
+    b, L, _ = hidden.shape
+    d_inner = H * P
+    conv_dim = d_inner + 2 * G * N
+    W_in = _f64(W_in)
+    if W_in.shape[0] != d_inner + conv_dim + H:
+        raise ValueError("mixer_forward: W_in must have 2 H P + 2 G N + H rows")
+    zxbcdt = hidden @ W_in.T
+    z = zxbcdt[..., :d_inner]
+    xBC = np.ascontiguousarray(zxbcdt[..., d_inner:d_inner + conv_dim])
+    dt_raw = np.ascontiguousarray(zxbcdt[..., d_inner + conv_dim:])
+    y, fs, cs = layer_prefill(xBC, conv_w, conv_bias, conv_state, dt_raw, A, dt_bias, D, init_state,
+                              H, P, G, N, nthreads)
+    n = rmsnorm_gated(y.reshape(b, L, d_inner), z, norm_w, norm_groups, eps)
+    out = n @ _f64(W_out).T
+    return out, fs, cs

@@ -23,7 +23,12 @@ with ``oracle.using_library``) disagrees with:
 * for the backward pass: central finite differences of the forward oracle for
   every input element (brute force on a tiny problem), the closed form of dD,
   the dt -> 0 limit, linearity in the output gradients, and independence of
-  the thread count.
+  the thread count;
+* for the mixer around the path (in_proj, the path, gated RMSNorm, out_proj):
+  a hand-worked gated norm, SiLU against the library logistic function,
+  the unit mean square and scale invariance of the norm, the slice-wise
+  definition of a grouped norm, and the wiring of both projections against
+  explicit index loops on a tiny layer.
 
 All inputs are small and seeded so the whole set runs in seconds on a CPU.
 """
@@ -563,6 +568,92 @@ def check_bwd_thread_count_invariance():
         assert np.array_equal(a[k], b[k]), f"{k} depends on the thread count"
 
 
+# ----------------------------------------------------------------------------
+# the mixer: gated RMSNorm and the two projections
+# ----------------------------------------------------------------------------
+
+def check_gated_norm_hand_worked():
+    """y = (3, 4), z = (1, -1), weight (1, 2), eps 0:
+    SiLU(1) = 1/(1 + e^-1), SiLU(-1) = -1/(1 + e); g = y SiLU(z);
+    n = g / sqrt((g0^2 + g1^2) / 2) times the weight."""
+    s1 = 1.0 / (1.0 + math.exp(-1.0))
+    sm1 = -1.0 / (1.0 + math.e)
+    g0, g1 = 3.0 * s1, 4.0 * sm1
+    r = math.sqrt((g0 * g0 + g1 * g1) / 2.0)
+    want = np.array([g0 / r, 2.0 * g1 / r])
+    got = oracle.rmsnorm_gated(np.array([3.0, 4.0]), np.array([1.0, -1.0]), np.array([1.0, 2.0]), 1, 0.0)
+    _close(got, want, 1e-14, "gated norm, hand-worked")
+
+
+def check_silu_matches_library_logistic():
+    from scipy.special import expit
+    v = np.linspace(-30.0, 30.0, 1201)
+    _close(oracle.silu(v), v * expit(v), 1e-15, "SiLU vs v * expit(v)")
+
+
+def check_gated_norm_invariants():
+    rng = _rng(41)
+    y = rng.standard_normal((3, 5, 24))
+    z = rng.standard_normal((3, 5, 24))
+    ones = np.ones(24)
+    # unit mean square per slice (weight 1, eps 0), whatever the grouping
+    for groups in (1, 3, 8):
+        n = oracle.rmsnorm_gated(y, z, ones, groups, 0.0).reshape(3, 5, groups, 24 // groups)
+        _close(np.mean(n * n, axis=-1), np.ones((3, 5, groups)), 1e-13, f"unit mean square, {groups} groups")
+    # scale invariance in y (eps 0)
+    w = rng.standard_normal(24)
+    _close(oracle.rmsnorm_gated(7.5 * y, z, w, 4, 0.0), oracle.rmsnorm_gated(y, z, w, 4, 0.0), 1e-13,
+           "scale invariance")
+    # a grouped norm is the one-group norm of each slice, with the library norm
+    g = y * oracle.silu(z)
+    eps = 1e-2
+    want = np.concatenate([g[..., k:k + 8] / np.sqrt(np.linalg.norm(g[..., k:k + 8], axis=-1, keepdims=True) ** 2 / 8
+                                                        + eps) for k in range(0, 24, 8)], axis=-1) * w
+    _close(oracle.rmsnorm_gated(y, z, w, 3, eps), want, 1e-13, "grouped norm vs slices")
+
+
+def _tiny_mixer(rng, b=2, L=40, d_model=7, H=2, P=3, G=1, N=4, k=4):
+    d_inner = H * P
+    conv_dim = d_inner + 2 * G * N
+    return dict(hidden=rng.standard_normal((b, L, d_model)),
+                W_in=rng.standard_normal((d_inner + conv_dim + H, d_model)) / math.sqrt(d_model),
+                conv_w=rng.standard_normal((conv_dim, k)) * 0.5, conv_bias=rng.standard_normal(conv_dim) * 0.3,
+                dt_bias=rng.standard_normal(H) * 0.5 - 1.0, A=-np.exp(rng.uniform(0.0, 2.0, H)),
+                D=rng.standard_normal(H), norm_w=rng.standard_normal(d_inner),
+                W_out=rng.standard_normal((d_model, d_inner)) / math.sqrt(d_inner), H=H, P=P, G=G, N=N)
+
+
+def check_mixer_projection_wiring():
+    """in_proj with a permutation matrix must hand the path the permuted input
+    columns (z, then xBC, then dt_raw, read by explicit indexing), and
+    out_proj must be out[m] = sum_k n[k] W_out[m][k] (an explicit loop)."""
+    rng = _rng(43)
+    H, P, G, N = 2, 3, 1, 4
+    d_inner, conv_dim = H * P, H * P + 2 * G * N
+    dproj = d_inner + conv_dim + H
+    t = _tiny_mixer(rng, d_model=dproj, H=H, P=P, G=G, N=N)
+    perm = rng.permutation(dproj)
+    W_in = np.zeros((dproj, dproj))
+    W_in[np.arange(dproj), perm] = 1.0          # row j picks input column perm[j]
+    t["W_in"] = W_in
+    hid = t["hidden"]
+    cs0 = rng.standard_normal((hid.shape[0], conv_dim, 4))
+    zxbcdt = hid[..., perm]
+    z, xBC, dt_raw = zxbcdt[..., :d_inner], zxbcdt[..., d_inner:d_inner + conv_dim], zxbcdt[..., -H:]
+    y, fs, cs = oracle.layer_prefill(np.ascontiguousarray(xBC), t["conv_w"], t["conv_bias"], cs0,
+                                     np.ascontiguousarray(dt_raw), t["A"], t["dt_bias"], t["D"], None, H, P, G, N)
+    n = oracle.rmsnorm_gated(y.reshape(y.shape[0], y.shape[1], d_inner), z, t["norm_w"])
+    want = np.zeros(hid.shape[:2] + (dproj,))
+    for m in range(dproj):
+        for kk in range(d_inner):
+            want[..., m] += n[..., kk] * t["W_out"][m, kk]
+    out, fs2, cs2 = oracle.mixer_forward(hid, W_in, t["conv_w"], t["conv_bias"], t["dt_bias"], t["A"], t["D"],
+                                         t["norm_w"], t["W_out"], H, P, G, N, conv_state=cs0)
+    _close(out, want, 1e-12, "mixer output vs explicit wiring")
+    _close(fs2, fs, 1e-13, "mixer final state")
+    _close(cs2, cs, 0.0, "mixer conv state")
+
+
 ALL_CHECKS = [
     check_dt_to_zero,
     check_geometric_series,
@@ -585,4 +676,8 @@ ALL_CHECKS = [
     check_bwd_linear_in_output_gradients,
     check_bwd_thread_count_invariance,
     check_bwd_chunked_matrix_form,
+    check_gated_norm_hand_worked,
+    check_silu_matches_library_logistic,
+    check_gated_norm_invariants,
+    check_mixer_projection_wiring,
 ]

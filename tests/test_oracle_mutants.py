@@ -96,3 +96,42 @@ def test_pins_catch_planted_ragged_mistake(mutant, monkeypatch):
     monkeypatch.setattr(oracle, "selective_scan_varlen", mutant)
     with pytest.raises(AssertionError):
         oracle_checks.check_varlen_matches_each_sequence_alone()
+
+
+# Planted mistakes in the mixer around the path (gated RMSNorm and the two
+# projections, written in numpy in oracle/__init__.py): the edited module is
+# executed apart and its mixer functions are routed to for the checks.
+PY_SRC = os.path.join(os.path.dirname(oracle.__file__), "__init__.py")
+
+MIXER_MUTANTS = {
+    "gate_sigmoid_not_silu": ("return v / (1.0 + np.exp(-v))", "return 1.0 / (1.0 + np.exp(-v))"),
+    "norm_sum_not_mean": ("ms = np.mean(gs * gs, axis=-1, keepdims=True)", "ms = np.sum(gs * gs, axis=-1, keepdims=True)"),
+    "norm_groups_interleaved": ("gs = g.reshape(*shp[:-1], groups, d // groups)",
+                                "gs = g.reshape(*shp[:-1], d // groups, groups).swapaxes(-1, -2)"),
+    "norm_eps_outside_sqrt": ("return (gs / np.sqrt(ms + eps)).reshape(shp)",
+                              "return (gs / (np.sqrt(ms) + eps)).reshape(shp)"),
+    "dt_from_the_front": ("dt_raw = np.ascontiguousarray(zxbcdt[..., d_inner + conv_dim:])",
+                          "dt_raw = np.ascontiguousarray(zxbcdt[..., :H])"),
+    "xBC_offset_by_z": ("xBC = np.ascontiguousarray(zxbcdt[..., d_inner:d_inner + conv_dim])",
+                        "xBC = np.ascontiguousarray(zxbcdt[..., :conv_dim])"),
+    "in_proj_not_transposed": ("zxbcdt = hidden @ W_in.T", "zxbcdt = hidden @ W_in"),
+    "out_proj_not_transposed": ("out = n @ _f64(W_out).T", "out = n @ _f64(W_out)"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MIXER_MUTANTS))
+def test_pins_catch_planted_mixer_mistake(name, monkeypatch):
+    old, new = MIXER_MUTANTS[name]
+    src = open(PY_SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not unique in the oracle module"
+    ns = {"__name__": "oracle_mutant", "__file__": PY_SRC}
+    exec(compile(src.replace(old, new), "oracle_mutant", "exec"), ns)
+    for fn in ("silu", "rmsnorm_gated", "mixer_forward"):
+        monkeypatch.setattr(oracle, fn, ns[fn])
+    caught = []
+    for check in oracle_checks.ALL_CHECKS:
+        try:
+            check()
+        except Exception:   # a wrong value, or a shape that no longer fits
+            caught.append(check.__name__)
+    assert caught, f"planted mistake {name!r} passed every pin"
