@@ -51,6 +51,22 @@
 // SSD_ERR_TIMEOUT in the optional status word and runs to its end without
 // waiting again.
 //
+// Long chains (fewer chains than SMs, e.g. one 262144-token sequence of 64
+// heads): the grid still takes one CTA per SM, so ranges fall inside
+// chains, and a CTA whose range starts inside a chain rebuilds its starting
+// state itself instead of waiting for the CTA before it.  The state entering
+// chunk c0 is sum over earlier chunks c of 2^(decay from c's end to c0) S_c,
+// plus the initial state decayed from the chain's start.  Walking back over
+// at most kPreMax chunks, the decay 2^(sum of cl_last) from the end of each
+// one to c0 is folded into its weights, w'_j = 2^(Lrun + cl_last - cl_j) dt_j,
+// so all of them accumulate into one TMEM accumulator, S += B^T (w' o X),
+// with no per-chunk decay step (the "state-only" items: B and X loaded, no
+// C, no y).  If the walk reaches the chain's start, the decayed initial
+// state is added; if instead the accumulated decay has fallen below 2^-64,
+// older tokens weigh less than 2^-64 of their own size, far under float32
+// rounding, and are dropped.  Otherwise (a long-memory head) the CTA falls
+// back to the published state of its predecessor.
+//
 // Token rows past the end of the sequence are zero-filled by TMA and get
 // dt = 0, so a ragged last chunk needs no special case.
 #include <cudaTypedefs.h>
@@ -75,6 +91,9 @@ constexpr int kVecWarp = kEwWarps + 2;   // chunk vectors (dt, cumulative decay)
 constexpr int kThreads = kEwThreads + 96;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr int kPreMax = 32;            // chunks a range's starting state is rebuilt from, at most
+constexpr int kMinRangeLong = 32;      // units per CTA at least, when chains are split across CTAs
+constexpr float kPreCutLog2 = -64.0f;  // accumulated log2 decay below which older tokens are dropped
 constexpr int kEwBarrier = 1;    // named barrier among the elementwise warps
 
 // Shared-memory layout, offsets from a 1024-byte aligned base.  Tiles are
@@ -272,15 +291,21 @@ __device__ inline int seq_of_unit(const Params& p, const Tabs& tb, int u)
 //       published state.
 // A range that starts and ends inside one chain is a single C segment that
 // is published at its end too.
+//   P = (long chains only) npre state-only items, chunks startC - 1 down to
+//       startC - npre of chain chC, run just before C to rebuild its
+//       starting state.
 struct Range {
     int chA, lenA;
     int uB0, nB, sB0;   // B: units [uB0, uB0 + nB); sB0 = sequence of uB0
     int chC, startC, lenC;
     bool pubC;
+    int npre;           // state-only items before C
     int count;
+    __device__ int pre_begin() const { return lenA + nB; }
+    __device__ bool is_pre(int idx) const { return idx >= lenA + nB && idx < lenA + nB + npre; }
 };
 
-template <bool kRagged>
+template <bool kRagged, bool kLong>
 __device__ inline Range make_range(const Params& p, const Tabs& tb, int t, int units)
 {
     Range r{};
@@ -299,7 +324,8 @@ __device__ inline Range make_range(const Params& p, const Tabs& tb, int t, int u
         r.startC = a.chunk;
         r.lenC = b.chunk - a.chunk;
         r.pubC = true;
-        r.count = r.lenC;
+        r.npre = kLong ? min(r.startC, kPreMax) : 0;
+        r.count = r.npre + r.lenC;
         return r;
     }
     r.chA = b.chain;
@@ -312,7 +338,8 @@ __device__ inline Range make_range(const Params& p, const Tabs& tb, int t, int u
     r.uB0 = a.chunk > 0 ? u0 + (a.ncc - a.chunk) : u0;
     r.nB = (u1 - b.chunk) - r.uB0;
     r.sB0 = kRagged && r.nB > 0 ? seq_of_unit(p, tb, r.uB0) : 0;
-    r.count = r.lenA + r.nB + r.lenC;
+    r.npre = kLong && r.lenC > 0 ? min(r.startC, kPreMax) : 0;
+    r.count = r.lenA + r.nB + r.npre + r.lenC;
     return r;
 }
 
@@ -324,12 +351,15 @@ struct Item {
     int bi;            // coordinate along the batch dimension (0 for a ragged batch)
     bool seg_start, seg_end, publish, depend;
     bool direct_y;     // y written row by row (a ragged batch's last, partial chunk)
+    bool pre;          // state-only item (long chains): rebuilds C's starting state
+    bool pre_first, pre_last;
 };
 
-template <bool kRagged>
+template <bool kRagged, bool kLong>
 __device__ inline Item item_at(const Params& p, const Tabs& tb, const Range& r, int idx, int& hint)
 {
     Item it;
+    it.pre = it.pre_first = it.pre_last = false;
     if (idx < r.lenA) {
         it.chain = r.chA;
         it.chunk = idx;
@@ -345,8 +375,16 @@ __device__ inline Item item_at(const Params& p, const Tabs& tb, const Range& r, 
         it.seg_end = l.chunk == l.ncc - 1;
         it.publish = false;
         it.depend = false;
+    } else if (kLong && idx - r.lenA - r.nB < r.npre) {
+        const int k = idx - r.lenA - r.nB;   // walking back from chunk startC - 1
+        it.chain = r.chC;
+        it.chunk = r.startC - 1 - k;
+        it.seg_start = it.seg_end = it.publish = it.depend = false;
+        it.pre = true;
+        it.pre_first = k == 0;
+        it.pre_last = k == r.npre - 1;
     } else {
-        const int k = idx - r.lenA - r.nB;
+        const int k = idx - r.lenA - r.nB - r.npre;
         it.chain = r.chC;
         it.chunk = r.startC + k;
         it.seg_start = k == 0;
@@ -384,7 +422,9 @@ __device__ inline void tmem_ld8(uint32_t taddr, float (&v)[8])
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-template <bool kRagged>
+// kLong: ranges inside chains rebuild their starting state (state-only
+// items); without it that code is compiled out.
+template <bool kRagged, bool kLong>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY,
@@ -453,7 +493,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             tabs = Tabs{scu, ssu};
         }
     }
-    const Range rg = make_range<kRagged>(prm, tabs, ticket, units);
+    const Range rg = make_range<kRagged, kLong>(prm, tabs, ticket, units);
     auto group_of = [&](const Item& it) { return (int)prm.fHG.div((uint32_t)it.h); };
     auto stage = [&](int idx) { return smem + kOffStage + (idx & 1) * kStageBytes; };
 
@@ -482,34 +522,44 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 umma_commit(bar_m1);
             };
 
-            wait_ld(0);
-            tc_fence_after_sync();
-            mma_G(0);
+            // A state-only item (long chains) runs only the state product,
+            // the first of them without accumulating; the commits stay, so
+            // every barrier keeps its phase.
+            auto next_G = [&](int idx) {
+                wait_ld(idx);
+                tc_fence_after_sync();
+                if (kLong && rg.is_pre(idx)) umma_commit(bar_m1);
+                else mma_G(idx);
+            };
+            next_G(0);
             for (int idx = 0; idx < rg.count; ++idx) {
                 const uint32_t ph = (uint32_t)idx & 1u;
                 const uint64_t so = (idx & 1) ? kStageStep : 0;
                 const uint64_t dC = dCk0 + so, dBmn = dBmn0 + so, dXmn = dXmn0 + so;
+                const bool pre = kLong && rg.is_pre(idx);
+                const uint32_t acc0 = pre && idx == rg.pre_begin() ? 0u : 1u;
                 mbar_wait_bounded(bar_sready, ph, kWaitNs, aborted, prm.status);
                 tc_fence_after_sync();
-                const uint32_t dYo = tmem + kColYo + (uint32_t)(idx & 1) * 64u;
+                if (!pre) {
+                    const uint32_t dYo = tmem + kColYo + (uint32_t)(idx & 1) * 64u;
 #pragma unroll
-                for (int k = 0; k < 8; ++k)   // Yo = C h^T
-                    umma_bf16(dYo, dC + kstep_k(k), dHB + kstep_mn(k), kIdYo, k > 0);
+                    for (int k = 0; k < 8; ++k)   // Yo = C h^T
+                        umma_bf16(dYo, dC + kstep_k(k), dHB + kstep_mn(k), kIdYo, k > 0);
+                }
 #pragma unroll
                 for (int k = 0; k < 8; ++k)   // h += B^T (w o X)   (h already decayed)
-                    umma_bf16(tmem + kColH, dBmn + kstep_mn(k), dWX + kstep_mn(k), kIdS, 1);
+                    umma_bf16(tmem + kColH, dBmn + kstep_mn(k), dWX + kstep_mn(k), kIdS, k > 0 ? 1u : acc0);
                 umma_commit(bar_m4 + (idx & 1));
                 mbar_wait_bounded(bar_mready, ph, kWaitNs, aborted, prm.status);
                 tc_fence_after_sync();
+                if (!pre) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k)   // Yd = M X, M from TMEM
-                    umma_bf16_tmem_a(tmem + kColYd, tmem + kColM + (uint32_t)k * 8u, dXmn + kstep_mn(k), kIdYd, k > 0);
-                umma_commit(bar_m2);
-                if (idx + 1 < rg.count) {   // the next item's C B^T (G was read: mready)
-                    wait_ld(idx + 1);
-                    tc_fence_after_sync();
-                    mma_G(idx + 1);
+                    for (int k = 0; k < 8; ++k)   // Yd = M X, M from TMEM
+                        umma_bf16_tmem_a(tmem + kColYd, tmem + kColM + (uint32_t)k * 8u, dXmn + kstep_mn(k), kIdYd,
+                                         k > 0);
                 }
+                umma_commit(bar_m2);
+                if (idx + 1 < rg.count) next_G(idx + 1);   // the next item's C B^T (G was read: mready)
             }
         }
         __syncwarp();
@@ -522,26 +572,29 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             // prefetch) and passed along a rotation of items idx .. idx + 3.
             struct Co {
                 int g, h, tok0, bi;
-                bool direct_y;
+                bool direct_y, pre;
             };
             int hint = rg.sB0;   // items are visited in increasing order
             auto coord = [&](int idx) {
-                Co c{0, 0, 0, 0, false};
+                Co c{0, 0, 0, 0, false, false};
                 if (idx < rg.count) {
-                    const Item it = item_at<kRagged>(prm, tabs, rg, idx, hint);
-                    c = Co{group_of(it), it.h, it.tok0, it.bi, it.direct_y};
+                    const Item it = item_at<kRagged, kLong>(prm, tabs, rg, idx, hint);
+                    c = Co{group_of(it), it.h, it.tok0, it.bi, it.direct_y, kLong && it.pre};
                 }
                 return c;
             };
-            // B and C of item idx into its stage (G = C B^T needs only these)
+            // B and C of item idx into its stage (G = C B^T needs only these;
+            // a state-only item needs B alone)
             auto issue_bc = [&](int idx, const Co& c) {
                 uint8_t* st = stage(idx);
                 uint64_t* bar = bar_ld + (idx & 1);
-                mbar_arrive_expect_tx(bar, kBytesBC);
+                mbar_arrive_expect_tx(bar, kLong && c.pre ? kBytesBC / 2 : kBytesBC);
                 tma_load_3d(st + kStB, &tmB, c.g * kN, c.tok0, c.bi, bar);
                 tma_load_3d(st + kStB + kTileHalf, &tmB, c.g * kN + 64, c.tok0, c.bi, bar);
-                tma_load_3d(st + kStC, &tmC, c.g * kN, c.tok0, c.bi, bar);
-                tma_load_3d(st + kStC + kTileHalf, &tmC, c.g * kN + 64, c.tok0, c.bi, bar);
+                if (!(kLong && c.pre)) {
+                    tma_load_3d(st + kStC, &tmC, c.g * kN, c.tok0, c.bi, bar);
+                    tma_load_3d(st + kStC + kTileHalf, &tmC, c.g * kN + 64, c.tok0, c.bi, bar);
+                }
             };
             // X of item idx into its stage (the buffer that held y of item idx - 2)
             auto issue_x = [&](int idx, const Co& c) {
@@ -552,8 +605,10 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             auto prefetch_l2 = [&](const Co& c) {
                 tma_prefetch_l2_3d(&tmB, c.g * kN, c.tok0, c.bi);
                 tma_prefetch_l2_3d(&tmB, c.g * kN + 64, c.tok0, c.bi);
-                tma_prefetch_l2_3d(&tmC, c.g * kN, c.tok0, c.bi);
-                tma_prefetch_l2_3d(&tmC, c.g * kN + 64, c.tok0, c.bi);
+                if (!(kLong && c.pre)) {
+                    tma_prefetch_l2_3d(&tmC, c.g * kN, c.tok0, c.bi);
+                    tma_prefetch_l2_3d(&tmC, c.g * kN + 64, c.tok0, c.bi);
+                }
                 tma_prefetch_l2_3d(&tmX, c.h * kP, c.tok0, c.bi);
             };
             prefetch_tensormap(&tmX);
@@ -576,7 +631,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 // y of item idx is staged in its X buffer: store it, then
                 // reload the buffer once the store has read it
                 mbar_wait_bounded(bar_ystaged + (idx & 1), sph, kWaitNs, aborted, prm.status);
-                if (!c0.direct_y) {   // (a partial ragged chunk's rows went out directly)
+                if (!c0.direct_y && !(kLong && c0.pre)) {   // (a partial ragged chunk's rows went out directly;
+                                                 //  a state-only item has no y)
                     tma_store_3d(&tmY, stage(idx) + kStX, c0.h * kP, c0.tok0, c0.bi);
                     bulk_commit_group();
                     bulk_wait_group_read0();
@@ -601,17 +657,20 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         struct DtIn {
             float a2, bias;
             int nvalid;   // tokens 4*lane + k with k < nvalid lie inside the sequence
+            bool pre, pre_first;
             __nv_bfloat16 dt[4];
         };
         // raw inputs of item idx for tokens 4*lane .. 4*lane+3
         int hint = rg.sB0;
         auto load_dt = [&](int idx) {
             DtIn in;
-            const Item it = item_at<kRagged>(prm, tabs, rg, idx, hint);
+            const Item it = item_at<kRagged, kLong>(prm, tabs, rg, idx, hint);
             in.a2 = prm.A[it.h] * 1.4426950408889634f;   // A * log2(e)
             in.bias = prm.dt_bias ? prm.dt_bias[it.h] : 0.0f;
             const __nv_bfloat16* dp = prm.dt_raw + ((size_t)it.bi * L + it.tok0 + lane * 4) * H + it.h;
             in.nvalid = it.nvalid - lane * 4;
+            in.pre = it.pre;
+            in.pre_first = it.pre_first;
 #pragma unroll
             for (int k = 0; k < 4; ++k) in.dt[k] = k < in.nvalid ? dp[(size_t)k * H] : __float2bfloat16_rn(0.0f);
             return in;
@@ -619,7 +678,12 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         // dt (0 past the sequence end), the inclusive cumulative log2 decay
         // (local sums, then a warp scan) and the off-diagonal column factor
         // 2^(cl_e - cl) dt, e the last token of the 32-token block.
+        // A state-only item publishes instead, in the dt slot, its weights
+        // w'_j = 2^(lrun + cl_last - cl_j) dt_j, lrun the log2 decay over the
+        // chunks between it and the rebuilt state (walked back from there),
+        // and in the v slot lrun including its own chunk.
         float vcl[4], vdt[4], vv[4];
+        float lrun = 0.0f;
         auto compute_vecs = [&](const DtIn& in) {
             float run = 0.0f;
 #pragma unroll
@@ -637,6 +701,16 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             const float excl = incl - run;
 #pragma unroll
             for (int k = 0; k < 4; ++k) vcl[k] += excl;
+            if (kLong && in.pre) {
+                if (in.pre_first) lrun = 0.0f;
+                const float cl_last = __shfl_sync(0xffffffffu, vcl[3], 31);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) vdt[k] = ex2_approx(lrun + cl_last - vcl[k]) * vdt[k];
+                lrun += cl_last;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) vv[k] = lrun;
+                return;
+            }
             const float cl_e = __shfl_sync(0xffffffffu, vcl[3], lane | 7);
 #pragma unroll
             for (int k = 0; k < 4; ++k) vv[k] = ex2_approx(cl_e - vcl[k]) * vdt[k];
@@ -685,34 +759,47 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const uint32_t tH = tmem + kColH + (uint32_t)p0 + lane_off;
 
-        // state entering a segment: the initial state, the predecessor
-        // CTA's published state (a dependent segment), or zero
-        auto segment_state = [&](const Item& it, float (&hv)[16]) {
-            const int bi = (int)prm.fH.div((uint32_t)it.chain), h = it.chain - bi * H;
-            const float* src = nullptr;
-            bool cg = false;
-            if (it.depend) {
-                const int* flag = prm.ws_ctrl + 16 + (ticket - 1);
-                if (tid == 0 && !*aborted) {
-                    const uint64_t t0 = globaltimer_ns();
-                    while (ld_acquire_gpu(flag) == 0) {
-                        if (globaltimer_ns() - t0 > kWaitNs) {
-                            *aborted = 1;
-                            if (prm.status) atomicExch(reinterpret_cast<int*>(prm.status), 4);
-                            break;
-                        }
+        // the initial state of chain ch's sequence and head (16 columns p of
+        // state column n = row), or zeros
+        auto load_init = [&](int ch, float (&hv)[16]) {
+            const float* src = prm.init_state ? prm.init_state + (size_t)ch * (kP * kN) : nullptr;
+#pragma unroll
+            for (int p = 0; p < 16; ++p) hv[p] = src ? src[(size_t)(p0 + p) * kN + row] : 0.0f;
+        };
+        // the state published by the predecessor CTA (bounded wait on its flag)
+        auto load_published = [&](float (&hv)[16]) {
+            const int* flag = prm.ws_ctrl + 16 + (ticket - 1);
+            if (tid == 0 && !*aborted) {
+                const uint64_t t0 = globaltimer_ns();
+                while (ld_acquire_gpu(flag) == 0) {
+                    if (globaltimer_ns() - t0 > kWaitNs) {
+                        *aborted = 1;
+                        if (prm.status) atomicExch(reinterpret_cast<int*>(prm.status), 4);
+                        break;
                     }
                 }
-                named_bar_sync(kEwBarrier, kEwThreads);
-                src = prm.ws_states + (size_t)(ticket - 1) * (kP * kN);
-                cg = true;
-            } else if (prm.init_state) {
-                src = prm.init_state + ((size_t)bi * H + h) * (size_t)(kP * kN);
             }
+            named_bar_sync(kEwBarrier, kEwThreads);
+            const float* src = prm.ws_states + (size_t)(ticket - 1) * (kP * kN);
 #pragma unroll
-            for (int p = 0; p < 16; ++p) {
-                const float* q = src + (size_t)(p0 + p) * kN + row;
-                hv[p] = src ? (cg ? __ldcg(q) : *q) : 0.0f;
+            for (int p = 0; p < 16; ++p) hv[p] = __ldcg(src + (size_t)(p0 + p) * kN + row);
+        };
+        // the state-only items (long chains) left a valid starting state in
+        // the TMEM state columns
+        bool pre_ok = false;
+
+        // state entering a segment: the initial state, the rebuilt state,
+        // the predecessor CTA's published state (a dependent segment), or zero
+        auto segment_state = [&](const Item& it, float (&hv)[16]) {
+            if (it.depend) {
+                if (kLong && pre_ok) {
+                    tmem_ld16(tH, hv);
+                    tmem_wait_ld();
+                } else {
+                    load_published(hv);
+                }
+            } else {
+                load_init(it.chain, hv);
             }
         };
 
@@ -720,11 +807,16 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         // is in Yd through M's diagonal), written over x in the item's X
         // buffer for the producer's TMA store.  M X of item j (the X
         // buffer's last reader) is done once bar_m2 has completed for it.
+        // A state-only item has no y: its barriers are still passed.
         // the previous item's row placement (ragged batches only)
         int prev_tok0 = 0, prev_nvalid = 0, prev_h = 0;
-        bool prev_direct = false;
+        bool prev_direct = false, prev_pre = false;
         auto y_epilogue = [&](int j, float cl_i) {
             mbar_wait_bounded(bar_m2, (uint32_t)j & 1u, kWaitNs, aborted, prm.status);
+            if (kLong && prev_pre) {
+                mbar_arrive(bar_ystaged + (j & 1));
+                return;
+            }
             tc_fence_after_sync();
             uint8_t* xs = stage(j) + kStX;
             const float sc = ex2_approx(cl_i);
@@ -770,11 +862,73 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         float prev_cl_i = 0.0f;
         int hint = rg.sB0;
         for (int idx = 0; idx < rg.count; ++idx) {
-            const Item it = item_at<kRagged>(prm, tabs, rg, idx, hint);
+            const Item it = item_at<kRagged, kLong>(prm, tabs, rg, idx, hint);
             const int bi = it.seq, h = it.h;
-            const float Dh = prm.D ? prm.D[h] : 0.0f;
             uint8_t* st = stage(idx);
+            float cl_i = 0.0f;
 
+            if (kLong && it.pre) {
+                // ----------------------------------------------------------
+                // state-only item: w' o X for S += B^T (w' o X), no state
+                // carried in TMEM between these items (the MMAs accumulate)
+                // ----------------------------------------------------------
+                mbar_wait_bounded(bar_vec, (uint32_t)idx & 1u, kWaitNs, aborted, prm.status);
+                const ChunkVecs cv = chunk_vecs(smem, idx & 1);
+                const float wj = cv.dt[row];
+                const float lsum = cv.v[0];   // log2 decay from this chunk's start to the rebuilt state
+                // the previous item's state product, which reads the w o X
+                // buffer, is done
+                if (idx > 0)
+                    mbar_wait_bounded(bar_m4 + ((idx - 1) & 1), (uint32_t)((idx - 1) >> 1) & 1u, kWaitNs, aborted,
+                                      prm.status);
+                mbar_wait_bounded(bar_ldx + (idx & 1), (uint32_t)(idx >> 1) & 1u, kWaitNs, aborted, prm.status);
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    float v[8];
+                    unpack_bf16x8(*reinterpret_cast<const uint4*>(st + kStX + sw128(row, quarter * 2 + q)), v);
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) {
+                        const float2 r = mul2(make_float2(v[e], v[e + 1]), make_float2(wj, wj));
+                        v[e] = r.x;
+                        v[e + 1] = r.y;
+                    }
+                    *reinterpret_cast<uint4*>(sWX + sw128(row, quarter * 2 + q)) = pack_bf16x8(v);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before_sync();
+                mbar_arrive(bar_sready);   // the state product can start
+                if (idx > 0) y_epilogue(idx - 1, prev_cl_i);
+                mbar_wait_bounded(bar_m1, (uint32_t)idx & 1u, kWaitNs, aborted, prm.status);
+                tc_fence_before_sync();
+                mbar_arrive(bar_mready);   // (no masked tile)
+                if (it.pre_last) {
+                    // the walk is over: the rebuilt state is exact when it
+                    // reached the chain's start (plus the decayed initial
+                    // state), or when the accumulated decay is below 2^-64
+                    // (the last state product is waited for either way: the
+                    // next item rewrites the state columns)
+                    const bool from_start = rg.startC - rg.npre == 0;
+                    pre_ok = from_start || lsum <= kPreCutLog2;
+                    mbar_wait_bounded(bar_m4 + (idx & 1), (uint32_t)(idx >> 1) & 1u, kWaitNs, aborted, prm.status);
+                    tc_fence_after_sync();
+                    if (from_start && prm.init_state) {
+                        float hs[16], h0[16];
+                        tmem_ld16(tH, hs);
+                        load_init(it.chain, h0);
+                        tmem_wait_ld();
+                        const float d0 = ex2_approx(lsum);
+#pragma unroll
+                        for (int p = 0; p < 16; ++p) hs[p] = fmaf(d0, h0[p], hs[p]);
+                        tmem_st16(tH, hs);
+                        tmem_wait_st();
+                    }
+                }
+                prev_pre = true;
+                prev_cl_i = 0.0f;
+                continue;
+            }
+
+            const float Dh = prm.D ? prm.D[h] : 0.0f;
             // 1. the state entering item idx (fp32, state column n = row)
             float hv[16];
             if (it.seg_start) {
@@ -797,7 +951,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             //    accumulates onto it) and w o X, w_j = 2^(cl_last - cl_j) dt_j
             mbar_wait_bounded(bar_vec, (uint32_t)idx & 1u, kWaitNs, aborted, prm.status);
             const ChunkVecs cv = chunk_vecs(smem, idx & 1);
-            const float cl_i = cv.cl[row];
+            cl_i = cv.cl[row];
             const float cl_last = cv.cl[kQ - 1];
             {
                 const float decay = ex2_approx(cl_last);
@@ -911,6 +1065,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 }
             }
             prev_cl_i = cl_i;
+            prev_pre = false;
             if constexpr (kRagged) {
                 prev_tok0 = it.tok0;
                 prev_nvalid = it.nvalid;
@@ -961,15 +1116,28 @@ cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t channels, uint64
 }
 
 
-int tc_slots(const ScanArgs& a)
+// CTAs of the persistent grid (one per SM at most).  With at least as many
+// chains as SMs every SM gets work from whole chains and their cuts.  With
+// fewer chains, long ones are split further, into ranges of at least
+// kMinRangeLong units, and the ranges that start inside a chain rebuild
+// their starting state (*long_chains).  A ragged batch's unit count is
+// known on the device only; H times the chunks of its packed tokens stands
+// in for it here.
+int tc_slots(const ScanArgs& a, bool* long_chains = nullptr)
 {
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
         sms = 148;
     const long long chains = (long long)(a.cu_seqlens ? a.nseq : a.b) * a.H;
-    const long long slots = sms;   // one CTA per SM
-    return (int)(chains < slots ? chains : slots);
+    const long long nc = (a.L + kQ - 1) / kQ;
+    const long long units = a.cu_seqlens ? (long long)a.H * nc : chains * nc;
+    long long slots = chains < sms ? chains : sms;
+    const long long split = units / kMinRangeLong;
+    const bool split_chains = chains < sms && split > chains;
+    if (split_chains) slots = split < sms ? split : sms;
+    if (long_chains) *long_chains = split_chains;
+    return (int)slots;
 }
 
 }  // namespace
@@ -1001,10 +1169,12 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t s)
     if ((e = make_map(&tmC, a.C, (uint64_t)a.G * a.N, a.L, a.b, rb)) != cudaSuccess) return e;
     CUtensorMap tmY;
     if ((e = make_map(&tmY, a.y, (uint64_t)a.H * a.P, a.L, a.b, (uint64_t)a.H * a.P * 2)) != cudaSuccess) return e;
-    auto kernel = a.cu_seqlens ? chunk_scan_tc_kernel<true> : chunk_scan_tc_kernel<false>;
+    bool long_chains = false;
+    const int slots = tc_slots(a, &long_chains);
+    auto kernel = a.cu_seqlens ? (long_chains ? chunk_scan_tc_kernel<true, true> : chunk_scan_tc_kernel<true, false>)
+                               : (long_chains ? chunk_scan_tc_kernel<false, true> : chunk_scan_tc_kernel<false, false>);
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    const int slots = tc_slots(a);
     const size_t ctrl = kWsCtrlBytes(slots);
     const bool ragged = a.cu_seqlens != nullptr;
     const size_t table = ragged ? varlen_table_bytes(a.nseq) : 0;

@@ -89,8 +89,11 @@ def test_scan_full_size_matches_oracle(cfg):
 def test_long_context_prefix_causality_and_handoff():
     """262144 tokens: the oracle checks a 4096-token prefix (y and state from a
     separate 4096-token call); the full call must reproduce that prefix's y
-    bit for bit (causality, same chunking), and a hand-off at token 131072
-    through init_state must reproduce the full call's second half."""
+    bit for bit (causality, same chunking: no range of the full call starts
+    inside its first 4096 tokens), two sampled heads of the full call match
+    the oracle over all 262144 tokens (the full call cuts every chain into
+    ranges that rebuild their starting states), and a hand-off at token
+    131072 through init_state must reproduce the full call's second half."""
     s = synth.CONFIGS[3]
     inp = synth.scan_inputs(s, synth.config_seed(3))
     Lp = 4096
@@ -101,6 +104,17 @@ def test_long_context_prefix_causality_and_handoff():
     y, fs = _gpu_scan(inp, s, u=ud)
     torch.cuda.synchronize()
     assert torch.equal(y[:, :Lp], yp), "full call's prefix differs from the prefix call"
+    # heads 5 and 42 (groups 0 and 5) over the whole sequence, one by one
+    heads, hpg = [5, 42], s.H // s.G
+    x, B, C = synth.split_channels(inp["u"], s)
+    x = x.reshape(s.b, s.L, s.H, s.P)[:, :, heads]
+    B = B.reshape(s.b, s.L, s.G, s.N)[:, :, [h // hpg for h in heads]]
+    C = C.reshape(s.b, s.L, s.G, s.N)[:, :, [h // hpg for h in heads]]
+    ys_ref, fss_ref = oracle.selective_scan(
+        f64(x), f64(B), f64(C), f64(inp["dt_raw"][:, :, heads]), f64(inp["A"][heads]),
+        f64(inp["dt_bias"][heads]), f64(inp["D"][heads]), None)
+    del x, B, C
+    _check(y[:, :, heads], fs[:, heads], ys_ref, fss_ref, s, "sampled heads, full length")
     half = s.L // 2
     _, f_half = _gpu_scan(inp, s, u=ud[:, :half], L=half)
     inp2 = dict(inp, dt_raw=inp["dt_raw"][:, half:])
@@ -109,6 +123,37 @@ def test_long_context_prefix_causality_and_handoff():
     assert norm_max_abs(y2, y[:, half:]) <= 1e-2
     assert norm_max_abs(fs2, fs) <= 1e-3
     assert torch.isfinite(y).all()
+
+
+LONG = {
+    # fewer chains than SMs: each chain is cut into ranges of >= 32 chunks,
+    # and each range after the first rebuilds its starting state from the 32
+    # chunks before it (2 chains of 157 chunks -> 9 ranges)
+    "rebuilt_start": (synth.CONFIGS[1].with_(b=1, L=20000, H=2, G=1), dict(init_state=True)),
+    # the second range starts at chunk 32: the walk back reaches the chain's
+    # start and adds the decayed initial state
+    "walk_reaches_chain_start": (synth.CONFIGS[1].with_(b=1, L=40000, H=2, G=2),
+                                 dict(init_state=True, dt_bias=True)),
+    # long-memory heads (|A| down to 0.01): over 32 chunks their decay stays
+    # above 2^-64, so those ranges wait for the state published before them;
+    # the other heads rebuild theirs
+    "long_memory_falls_back": (synth.CONFIGS[1].with_(b=2, L=30000, H=4, G=2),
+                               dict(a_range=(0.01, 2.0), init_state=True)),
+}
+
+
+@pytest.mark.parametrize("name", sorted(LONG))
+def test_long_chains_match_oracle(name):
+    s, kw = LONG[name]
+    inp = synth.scan_inputs(s, 61000 + len(name), **kw)
+    y_ref, fs_ref = _oracle_scan(inp, s)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ud = cuda(inp["u"])
+    x, B, C = layer.split_channels(ud, s.H, s.P, s.G, s.N)
+    y, fs = layer.chunk_scan_fwd(x, B, C, cuda(inp["dt_raw"]), cuda(inp["A"]), cuda(inp["dt_bias"]),
+                                 cuda(inp["D"]), cuda(inp["init_state"]), Q=s.Q, status=status)
+    _check(y, fs, y_ref, fs_ref, s, name)
+    assert int(status.item()) == 0, "a bounded wait gave up"
 
 
 def test_split_prefill_and_decode_extend_prefill():

@@ -102,8 +102,9 @@ def test_varlen_many_short_sequences():
 
 
 def test_varlen_ranges_inside_one_chain():
-    # 2 heads x (157 + 1 + 1) chunks over 6 CTAs: the long chains are split
-    # across CTAs, some of whose ranges start and end inside one chain
+    # 2 heads x (157 + 1 + 1) chunks over 9 CTAs (fewer chains than SMs, so
+    # the long chains are split): ranges start and end inside one chain and
+    # rebuild their starting states from the chunks before them
     lens = [20000, 5, 7]
     s, d = _ragged(BF16.with_(H=2, G=1), lens, 504)
     y, fs, st = _run(s, d)
