@@ -18,8 +18,9 @@
  *   - the single-token decode update of the same recurrence;
  *   - entry points built from these: the prefill layer in one call (conv,
  *     then scan), ragged prefill over packed sequences (cu_seqlens), the
- *     decode step in one kernel (cache roll, conv, update), and the scan's
- *     backward pass (gradients for training).
+ *     decode step in one kernel (cache roll, conv, update), the scan's
+ *     backward pass (gradients for training), and the whole Mamba-2 mixer
+ *     (in_proj, the path, gated RMSNorm, out_proj) with its linear layers.
  * Discretisation (the pages leave it open; this is the Mamba-2 reading):
  *   dt = softplus(dt_raw + dt_bias), Abar = exp(dt * A), Bbar = dt * B.
  *
@@ -368,6 +369,66 @@ SSD_API ssd_status_t ssd_chunk_scan_bwd(const void* x, const void* B, const void
                                         float* dinit, int b, int L, int H, int P, int N, int G,
                                         ssd_dtype_t dtype, void* workspace,
                                         size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Linear layer on the tensor cores, y = x W^T: the Mamba-2 mixer's in_proj
+ * and out_proj (Nemotron feasibility report, section 3.3: the projections
+ * around the scan are linear layers; section 3.2: the mixer module).
+ *
+ *   y[m][n] = sum_k x[m][k] * w[n][k]      bf16 operands, float32 accumulation,
+ *                                          bf16 result (round to nearest even)
+ *   x   [M][ldx]  bf16, row m's K inputs at x[m*ldx .. m*ldx + K)
+ *   w   [N][ldw]  bf16, output n's K weights at w[n*ldw ..)
+ *   y   [M][ldy]  bf16, written (columns < N); must not overlap x or w
+ *   status        optional device int32, set to SSD_ERR_TIMEOUT if a bounded
+ *                 device wait gave up (the result is then invalid)
+ * Requirements: N, K, ldx, ldw, ldy multiples of 8 (16-byte rows); all
+ * pointers 16-byte aligned.  M == 0 does nothing.
+ */
+SSD_API ssd_status_t ssd_linear_bf16(const void* x, int64_t ldx, const void* w, int64_t ldw, void* y,
+                                     int64_t ldy, int M, int N, int K, int32_t* status,
+                                     cudaStream_t stream);
+
+/*
+ * The Mamba-2 mixer forward in one call: in_proj, the hot path (conv1d +
+ * SiLU, chunked scan), the gated RMSNorm and out_proj (the block of the
+ * Nemotron feasibility report, section 3.2, computes x + Mamba2(RMSNorm(x));
+ * this is the Mamba2(.) part).  The pages fix neither the order of in_proj's
+ * outputs nor the gate; this follows the readings also taken by the oracle:
+ *
+ *   zxbcdt = hidden W_in^T, rows of W_in: z (H*P) | xBC (H*P + 2*G*N) | dt_raw (H)
+ *   u      = conv1d + SiLU of xBC (as ssd_conv1d_silu, conv_state rolled in place)
+ *   y      = the chunked scan of u's x | B | C with dt_raw (as ssd_chunk_scan_fwd)
+ *   g      = y * SiLU(z); n = g / sqrt(mean(g^2) + eps) * norm_w, the mean taken
+ *            over each of norm_groups equal slices of a token's H*P vector
+ *   out    = n W_out^T
+ *
+ *   hidden  [b][L][d_model] bf16     W_in [2*H*P + 2*G*N + H][d_model] bf16
+ *   conv_w  [conv_dim][k] float32, conv_bias [conv_dim] float32 or NULL
+ *   conv_state [b][conv_dim][k] bf16 or NULL (read, then rewritten in place)
+ *   dt_bias, A, D [H] float32 (dt_bias, D may be NULL); norm_w [H*P] float32
+ *   W_out   [d_model][H*P] bf16
+ *   init_state, final_state [b][H][P][N] float32 or NULL (may alias)
+ *   out     [b][L][d_model] bf16, written
+ *   workspace  ssd_mixer_workspace_bytes(...) bytes of device scratch,
+ *              caller-owned, no initial contents required
+ *   status  optional device int32 (SSD_ERR_TIMEOUT from a bounded wait)
+ * Requirements: dtype SSD_BF16 (else SSD_ERR_UNSUPPORTED); those of
+ * ssd_chunk_scan_fwd and ssd_conv1d_silu; d_model and H multiples of 8;
+ * (H*P / norm_groups) a multiple of 8; eps >= 0; no output may overlap an
+ * input or the workspace.  b == 0 or L == 0 writes only final_state (the
+ * initial state, or zeros) and leaves conv_state unchanged.
+ */
+SSD_API size_t ssd_mixer_workspace_bytes(int b, int L, int d_model, int H, int P, int N, int G, int Q,
+                                         int k, ssd_dtype_t dtype);
+
+SSD_API ssd_status_t ssd_mixer_fwd(const void* hidden, const void* W_in, const float* conv_w,
+                                   const float* conv_bias, void* conv_state, const float* dt_bias,
+                                   const float* A, const float* D, const float* norm_w, const void* W_out,
+                                   const float* init_state, void* out, float* final_state, int b, int L,
+                                   int d_model, int H, int P, int N, int G, int Q, int k, int norm_groups,
+                                   float eps, ssd_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                                   int32_t* status, cudaStream_t stream);
 
 /*
  * Self-test of the bounded device waits (failure detection without a fault).

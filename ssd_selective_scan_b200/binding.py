@@ -50,6 +50,10 @@ SIGNATURES = {
                                 _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "ssd_conv_scan_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp, _vp]),
+    "ssd_linear_bf16": (_i, [_vp, _i64, _vp, _i64, _vp, _i64, _i, _i, _i, _vp, _vp]),
+    "ssd_mixer_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i, _i, _i]),
+    "ssd_mixer_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                           _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, ctypes.c_float, _i, _vp, _sz, _vp, _vp]),
 }
 
 _lock = threading.Lock()
@@ -164,3 +168,19 @@ def ssd_selftest_bounded_wait(status, limit_ns, stream) -> int:
 def check(fn: str, status: int) -> None:
     if status != SSD_OK:
         raise SsdError(fn, status)
+
+
+def ssd_linear_bf16(x, ldx, w, ldw, y, ldy, M, N, K, status, stream) -> int:
+    return load().ssd_linear_bf16(x, ldx, w, ldw, y, ldy, M, N, K, status, stream)
+
+
+def ssd_mixer_workspace_bytes(b, L, d_model, H, P, N, G, Q, k, dtype) -> int:
+    return load().ssd_mixer_workspace_bytes(b, L, d_model, H, P, N, G, Q, k, dtype)
+
+
+def ssd_mixer_fwd(hidden, W_in, conv_w, conv_bias, conv_state, dt_bias, A, D, norm_w, W_out, init_state, out,
+                  final_state, b, L, d_model, H, P, N, G, Q, k, norm_groups, eps, dtype, workspace,
+                  workspace_bytes, status, stream) -> int:
+    return load().ssd_mixer_fwd(hidden, W_in, conv_w, conv_bias, conv_state, dt_bias, A, D, norm_w, W_out,
+                                init_state, out, final_state, b, L, d_model, H, P, N, G, Q, k, norm_groups, eps,
+                                dtype, workspace, workspace_bytes, status, stream)

@@ -3,6 +3,8 @@
 // synchronisation, no global mutable state.
 #include "ssd.h"
 
+#include <cuda_bf16.h>
+
 #include "kernels.h"
 #include "decode.h"
 #include "scan_bwd.h"
@@ -385,6 +387,142 @@ ssd_status_t ssd_decode_step(float* state, void* conv_state, const void* xBC, co
     if (ssd::decode_step_smem_bytes(H, P, N, G) > (size_t)max_optin_smem()) return SSD_ERR_UNSUPPORTED;
     return from_cuda(ssd::launch_decode_step(state, conv_state, xBC, w, bias, dt_raw, dt_bias, A, D, y, b, H, P,
                                              N, G, k, dtype == SSD_BF16, stream));
+}
+
+ssd_status_t ssd_linear_bf16(const void* x, int64_t ldx, const void* w, int64_t ldw, void* y, int64_t ldy, int M,
+                             int N, int K, int32_t* status, cudaStream_t stream)
+{
+    if (M < 0 || N <= 0 || K <= 0) return SSD_ERR_INVALID_ARG;
+    if (M == 0) return SSD_OK;
+    if (!x || !w || !y) return SSD_ERR_INVALID_ARG;
+    if (ldx < K || ldw < K || ldy < N || ldx % 8 || ldw % 8 || ldy % 8 || N % 8 || K % 8) return SSD_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(w, 16) || !aligned(y, 16) || (status && !aligned(status, 4)))
+        return SSD_ERR_INVALID_ARG;
+    const Range rx = span(x, ((int64_t)(M - 1) * ldx + K) * 2), rw = span(w, ((int64_t)(N - 1) * ldw + K) * 2);
+    const Range ry = span(y, ((int64_t)(M - 1) * ldy + N) * 2);
+    if (overlap(ry, rx) || overlap(ry, rw)) return SSD_ERR_INVALID_ARG;
+    if (!ssd::gemm_bf16_tn_supported(M, N, K, ldx, ldw, 0)) return SSD_ERR_UNSUPPORTED;
+    return from_cuda(ssd::launch_gemm_bf16_tn(x, ldx, w, ldw, y, ldy, nullptr, 0, M, N, K, 0, status, stream));
+}
+
+namespace {
+
+// Workspace of the mixer: in_proj's z | xBC columns and its dt columns, the
+// conv output (later reused for the normed y), the scan's y, then the scan's
+// own workspace.  Byte offsets, each region 256-byte aligned.
+struct MixerWs {
+    size_t zxbc, dt, u, y, scan, total;
+};
+
+MixerWs mixer_ws(int b, int L, int H, int P, int N, int G, int Q)
+{
+    const size_t M = (size_t)b * L;
+    const size_t d_inner = (size_t)H * P, conv_dim = d_inner + 2 * (size_t)G * N;
+    MixerWs w{};
+    w.zxbc = 0;
+    w.dt = w.zxbc + round_up_256(M * (d_inner + conv_dim) * 2);
+    w.u = w.dt + round_up_256(M * (size_t)H * 2);
+    w.y = w.u + round_up_256(M * conv_dim * 2);
+    w.scan = w.y + round_up_256(M * d_inner * 2);
+    w.total = w.scan + ssd_chunk_scan_workspace_bytes(b, L, H, P, N, G, Q, SSD_BF16);
+    return w;
+}
+
+}  // namespace
+
+size_t ssd_mixer_workspace_bytes(int b, int L, int d_model, int H, int P, int N, int G, int Q, int k,
+                                 ssd_dtype_t dtype)
+{
+    if (b <= 0 || L <= 0 || d_model <= 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || k <= 0 || dtype != SSD_BF16)
+        return 0;
+    return mixer_ws(b, L, H, P, N, G, Q).total;
+}
+
+ssd_status_t ssd_mixer_fwd(const void* hidden, const void* W_in, const float* conv_w, const float* conv_bias,
+                           void* conv_state, const float* dt_bias, const float* A, const float* D,
+                           const float* norm_w, const void* W_out, const float* init_state, void* out,
+                           float* final_state, int b, int L, int d_model, int H, int P, int N, int G, int Q, int k,
+                           int norm_groups, float eps, ssd_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                           int32_t* status, cudaStream_t stream)
+{
+    if (!valid_dtype(dtype) || b < 0 || L < 0 || d_model <= 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || k <= 0 ||
+        norm_groups <= 0 || !(eps >= 0.0f))
+        return SSD_ERR_INVALID_ARG;
+    if (H % G || P % 8 || N % 8 || (Q != 64 && Q != 128) || d_model % 8) return SSD_ERR_INVALID_ARG;
+    const int64_t d_inner = (int64_t)H * P, conv_dim = d_inner + 2 * (int64_t)G * N;
+    if (d_inner + conv_dim + H > 0x7fffffffLL || d_inner % norm_groups || (d_inner / norm_groups) % 8)
+        return SSD_ERR_INVALID_ARG;
+    if (dtype != SSD_BF16 || H % 8) return SSD_ERR_UNSUPPORTED;   // bf16 projections; 16-byte dt rows
+    if (k < 2 || k > 4) return SSD_ERR_UNSUPPORTED;
+    if (b == 0 || L == 0) {
+        // no tokens: the conv cache is unchanged and the final state is the initial one
+        return ssd_chunk_scan_fwd(nullptr, nullptr, nullptr, conv_dim, nullptr, dt_bias, A, D, init_state, nullptr,
+                                  final_state, b, L, H, P, N, G, Q, dtype, nullptr, 0, status, stream);
+    }
+    if (!hidden || !W_in || !conv_w || !A || !norm_w || !W_out || !out) return SSD_ERR_INVALID_ARG;
+    const void* ptrs16[] = {hidden, W_in, conv_w, conv_state, norm_w, W_out, init_state, out, final_state, workspace};
+    for (const void* p : ptrs16)
+        if (p && !aligned(p, 16)) return SSD_ERR_INVALID_ARG;
+    if ((conv_bias && !aligned(conv_bias, 4)) || (dt_bias && !aligned(dt_bias, 4)) || !aligned(A, 4) ||
+        (D && !aligned(D, 4)) || (status && !aligned(status, 4)))
+        return SSD_ERR_INVALID_ARG;
+    const MixerWs ws = mixer_ws(b, L, H, P, N, G, Q);
+    if (!workspace || workspace_bytes < ws.total) return SSD_ERR_INVALID_ARG;
+    const int64_t M = (int64_t)b * L;
+    const int64_t nproj = d_inner + conv_dim + H;
+    const Range rh = span(hidden, M * d_model * 2), rwi = span(W_in, nproj * d_model * 2);
+    const Range rwo = span(W_out, (int64_t)d_model * d_inner * 2), ro = span(out, M * d_model * 2);
+    const Range rcs = span(conv_state, conv_state ? (int64_t)b * conv_dim * k * 2 : 0);
+    const int64_t st_bytes = (int64_t)b * H * P * N * 4;
+    const Range ri = span(init_state, init_state ? st_bytes : 0), rf = span(final_state, final_state ? st_bytes : 0);
+    const Range rws = span(workspace, (int64_t)workspace_bytes);
+    for (Range in : {rh, rwi, rwo, rcs, ri, rws})
+        if (overlap(ro, in)) return SSD_ERR_INVALID_ARG;
+    for (Range in : {rh, rwi, rwo, rcs, ro, rws})
+        if (overlap(rf, in)) return SSD_ERR_INVALID_ARG;
+    if (final_state && init_state && final_state != init_state && overlap(rf, ri)) return SSD_ERR_INVALID_ARG;
+    for (Range in : {rh, rwi, rwo, ri})
+        if (overlap(rws, in) || overlap(rcs, in)) return SSD_ERR_INVALID_ARG;
+    if (overlap(rws, rcs)) return SSD_ERR_INVALID_ARG;
+    if (M > 0x7fffffffLL || b > 65535 || (L + 31) / 32 > 65535) return SSD_ERR_UNSUPPORTED;
+    if ((int64_t)b * H * ((L + Q - 1) / Q) > 0x7fffffffLL) return SSD_ERR_UNSUPPORTED;
+    if (!ssd::gemm_bf16_tn_supported((int)M, (int)nproj, d_model, d_model, d_model, (int)(d_inner + conv_dim)) ||
+        !ssd::gemm_bf16_tn_supported((int)M, d_model, (int)d_inner, d_inner, d_inner, 0))
+        return SSD_ERR_UNSUPPORTED;
+
+    uint8_t* wsb = static_cast<uint8_t*>(workspace);
+    auto* zxbc = reinterpret_cast<__nv_bfloat16*>(wsb + ws.zxbc);
+    auto* dt = reinterpret_cast<__nv_bfloat16*>(wsb + ws.dt);
+    auto* u = reinterpret_cast<__nv_bfloat16*>(wsb + ws.u);
+    auto* ybuf = reinterpret_cast<__nv_bfloat16*>(wsb + ws.y);
+    const int64_t ldz = d_inner + conv_dim;
+    // 1. in_proj: z | xBC into one buffer, dt into another
+    cudaError_t e = ssd::launch_gemm_bf16_tn(hidden, d_model, W_in, d_model, zxbc, ldz, dt, H, (int)M, (int)nproj,
+                                             d_model, (int)ldz, status, stream);
+    // 2. conv1d + SiLU of the xBC columns
+    if (e == cudaSuccess)
+        e = ssd::launch_conv1d_silu(zxbc + d_inner, u, conv_w, conv_bias, conv_state, b, L, (int)conv_dim, k, true,
+                                    stream, ldz);
+    // 3. the chunked scan
+    if (e == cudaSuccess) {
+        ScanArgs a{u, u + d_inner, u + d_inner + (int64_t)G * N, conv_dim, dt, dt_bias, A, D, init_state, ybuf,
+                   final_state, b, L, H, P, N, G, Q, true, wsb + ws.scan, workspace_bytes - ws.scan, status};
+        if (ssd::chunk_scan_tc_supported(a)) {
+            e = ssd::launch_chunk_scan_tc(a, stream);
+        } else {
+            if (ssd::chunk_scan_simt_smem_bytes(P, N) > (size_t)max_optin_smem()) return SSD_ERR_UNSUPPORTED;
+            e = ssd::launch_chunk_scan_simt(a, stream);
+        }
+    }
+    // 4. the gated RMSNorm, into the (now free) conv-output buffer
+    if (e == cudaSuccess)
+        e = ssd::launch_rmsnorm_gated(ybuf, d_inner, zxbc, ldz, norm_w, u, d_inner, (int)M, (int)d_inner, norm_groups,
+                                      eps, stream);
+    // 5. out_proj
+    if (e == cudaSuccess)
+        e = ssd::launch_gemm_bf16_tn(u, d_inner, W_out, d_inner, out, d_model, nullptr, 0, (int)M, d_model,
+                                     (int)d_inner, 0, status, stream);
+    return from_cuda(e);
 }
 
 size_t ssd_chunk_scan_bwd_workspace_bytes(int b, int L, int H, int P, int N, int G, ssd_dtype_t dtype)

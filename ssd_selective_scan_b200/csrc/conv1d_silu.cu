@@ -15,6 +15,8 @@
 //
 // The cache is read and rewritten by the thread that owns token tile 0 of a
 // channel group, so an in-place cache update never races with a reader.
+// The input rows may be wider than conv_dim (in_stride elements apart: the
+// xBC columns of the in_projection's output); the output is dense.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -122,7 +124,7 @@ struct CacheBlock {
 // new column j is old column j + S for j < K - S, else token L - K + j.
 // S is a template parameter so every register index is static.
 template <typename T, int K, int S>
-__device__ inline void roll_cache(T* cs, const T* xb, int L, int conv_dim)
+__device__ inline void roll_cache(T* cs, const T* xb, int L, int64_t in_stride)
 {
     CacheBlock<T, K> blk;
     if (S < K) blk.load(cs);
@@ -133,7 +135,7 @@ __device__ inline void roll_cache(T* cs, const T* xb, int L, int conv_dim)
             for (int c = 0; c < kCpt; ++c) blk.set(c, j, blk.get(c, j + S));
         } else {
             float v[kCpt];
-            Vec4<T>::decode(Vec4<T>::load(xb + (size_t)(L - K + j) * conv_dim), v);
+            Vec4<T>::decode(Vec4<T>::load(xb + (int64_t)(L - K + j) * in_stride), v);
 #pragma unroll
             for (int c = 0; c < kCpt; ++c) blk.set(c, j, v[c]);
         }
@@ -145,7 +147,7 @@ template <typename T, int K>
 __global__ void __launch_bounds__(kConvThreads)
 conv1d_silu_kernel(const T* __restrict__ xBC, T* __restrict__ out,
                    const float* __restrict__ w, const float* __restrict__ bias,
-                   T* __restrict__ conv_state, int L, int conv_dim)
+                   T* __restrict__ conv_state, int L, int conv_dim, int64_t in_stride)
 {
     using V4 = Vec4<T>;
     const int ngroups = conv_dim / kCpt;
@@ -154,7 +156,7 @@ conv1d_silu_kernel(const T* __restrict__ xBC, T* __restrict__ out,
     const int c0 = cg * kCpt;
     const int t0 = blockIdx.y * kConvTile;
     const int bi = blockIdx.z;
-    const T* xb = xBC + (size_t)bi * L * conv_dim + c0;
+    const T* xb = xBC + (int64_t)bi * L * in_stride + c0;
     T* ob = out + (size_t)bi * L * conv_dim + c0;
 
     // taps of the thread's 4 channels: 4*K contiguous floats
@@ -195,7 +197,7 @@ conv1d_silu_kernel(const T* __restrict__ xBC, T* __restrict__ out,
         }
     } else {
 #pragma unroll
-        for (int j = 0; j < K - 1; ++j) V4::decode(V4::load(xb + (size_t)(t0 - (K - 1) + j) * conv_dim), hist[j]);
+        for (int j = 0; j < K - 1; ++j) V4::decode(V4::load(xb + (int64_t)(t0 - (K - 1) + j) * in_stride), hist[j]);
     }
 
     const int t1 = min(L, t0 + kConvTile);
@@ -203,7 +205,7 @@ conv1d_silu_kernel(const T* __restrict__ xBC, T* __restrict__ out,
         typename V4::raw raw[kGroup];
 #pragma unroll
         for (int u = 0; u < kGroup; ++u)
-            if (tb + u < t1) raw[u] = V4::load(xb + (size_t)(tb + u) * conv_dim);
+            if (tb + u < t1) raw[u] = V4::load(xb + (int64_t)(tb + u) * in_stride);
 #pragma unroll
         for (int u = 0; u < kGroup; ++u) {
             if (tb + u < t1) {
@@ -233,43 +235,45 @@ conv1d_silu_kernel(const T* __restrict__ xBC, T* __restrict__ out,
         // and writes.
         T* cs = conv_state + ((size_t)bi * conv_dim + c0) * K;
         constexpr int S2 = K < 2 ? K : 2, S3 = K < 3 ? K : 3;
-        if (L >= K) roll_cache<T, K, K>(cs, xb, L, conv_dim);
-        else if (L == 1) roll_cache<T, K, 1>(cs, xb, L, conv_dim);
-        else if (L == 2) roll_cache<T, K, S2>(cs, xb, L, conv_dim);
-        else roll_cache<T, K, S3>(cs, xb, L, conv_dim);
+        if (L >= K) roll_cache<T, K, K>(cs, xb, L, in_stride);
+        else if (L == 1) roll_cache<T, K, 1>(cs, xb, L, in_stride);
+        else if (L == 2) roll_cache<T, K, S2>(cs, xb, L, in_stride);
+        else roll_cache<T, K, S3>(cs, xb, L, in_stride);
     }
 }
 
 template <typename T, int K>
 static cudaError_t launch_conv_k(const void* xBC, void* out, const float* w, const float* bias,
-                                 void* conv_state, int b, int L, int conv_dim, cudaStream_t s)
+                                 void* conv_state, int b, int L, int conv_dim, int64_t in_stride, cudaStream_t s)
 {
     const int ngroups = conv_dim / kCpt;
     dim3 grid((ngroups + kConvThreads - 1) / kConvThreads, (L + kConvTile - 1) / kConvTile, b);
     conv1d_silu_kernel<T, K><<<grid, kConvThreads, 0, s>>>(
         static_cast<const T*>(xBC), static_cast<T*>(out), w, bias, static_cast<T*>(conv_state),
-        L, conv_dim);
+        L, conv_dim, in_stride);
     return cudaGetLastError();
 }
 
 template <typename T>
 static cudaError_t launch_conv_t(const void* xBC, void* out, const float* w, const float* bias,
-                                 void* conv_state, int b, int L, int conv_dim, int k, cudaStream_t s)
+                                 void* conv_state, int b, int L, int conv_dim, int64_t in_stride, int k,
+                                 cudaStream_t s)
 {
     switch (k) {
-        case 2: return launch_conv_k<T, 2>(xBC, out, w, bias, conv_state, b, L, conv_dim, s);
-        case 3: return launch_conv_k<T, 3>(xBC, out, w, bias, conv_state, b, L, conv_dim, s);
-        case 4: return launch_conv_k<T, 4>(xBC, out, w, bias, conv_state, b, L, conv_dim, s);
+        case 2: return launch_conv_k<T, 2>(xBC, out, w, bias, conv_state, b, L, conv_dim, in_stride, s);
+        case 3: return launch_conv_k<T, 3>(xBC, out, w, bias, conv_state, b, L, conv_dim, in_stride, s);
+        case 4: return launch_conv_k<T, 4>(xBC, out, w, bias, conv_state, b, L, conv_dim, in_stride, s);
         default: return cudaErrorInvalidValue;
     }
 }
 
 cudaError_t launch_conv1d_silu(const void* xBC, void* out, const float* w, const float* bias,
                                void* conv_state, int b, int L, int conv_dim, int k, bool bf16,
-                               cudaStream_t s)
+                               cudaStream_t s, int64_t in_stride)
 {
-    return bf16 ? launch_conv_t<__nv_bfloat16>(xBC, out, w, bias, conv_state, b, L, conv_dim, k, s)
-                : launch_conv_t<float>(xBC, out, w, bias, conv_state, b, L, conv_dim, k, s);
+    if (in_stride <= 0) in_stride = conv_dim;
+    return bf16 ? launch_conv_t<__nv_bfloat16>(xBC, out, w, bias, conv_state, b, L, conv_dim, in_stride, k, s)
+                : launch_conv_t<float>(xBC, out, w, bias, conv_state, b, L, conv_dim, in_stride, k, s);
 }
 
 }  // namespace ssd

@@ -42,9 +42,22 @@ cudaError_t launch_varlen_prep(const int* cu_seqlens, int nseq, int T, int H, in
                                int* ctrl, int ctrl_ints, const float* init_state, float* final_state,
                                long long state_elems_per_seq, int32_t* status, cudaStream_t s);
 
+// in_stride: elements between consecutive input tokens (0: conv_dim)
 cudaError_t launch_conv1d_silu(const void* xBC, void* out, const float* w, const float* bias,
                                void* conv_state, int b, int L, int conv_dim, int k, bool bf16,
-                               cudaStream_t s);
+                               cudaStream_t s, int64_t in_stride = 0);
+
+// C0/C1 [M][.] = A[M][K] B[N][K]^T, bf16 in and out, fp32 accumulation
+// (tensor cores); output columns >= n_split (a multiple of 8; 0: none) go to
+// C1 at column - n_split.
+bool gemm_bf16_tn_supported(int M, int N, int K, int64_t lda, int64_t ldb, int n_split);
+cudaError_t launch_gemm_bf16_tn(const void* A, int64_t lda, const void* B, int64_t ldb, void* C0, int64_t ldc0,
+                                void* C1, int64_t ldc1, int M, int N, int K, int n_split, int32_t* status,
+                                cudaStream_t s);
+
+// n[M][d] = RMSNorm over `groups` slices of (y * SiLU(z)) times w, bf16 in/out
+cudaError_t launch_rmsnorm_gated(const void* y, int64_t ldy, const void* z, int64_t ldz, const float* w, void* n,
+                                 int64_t ldn, int M, int d, int groups, float eps, cudaStream_t s);
 
 bool state_update_supports_n(int N);
 cudaError_t launch_state_update(float* state, const void* x, const void* B, const void* C,

@@ -340,3 +340,73 @@ def decode_step(xBC, w, conv_state, state, dt_raw, A, H, P, G, N, *, bias=None, 
                                 _dtype_code(xBC), _stream(stream))
     libssd.check("ssd_decode_step", st)
     return y
+
+
+def linear(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor | None = None, status: torch.Tensor | None = None,
+           stream=None) -> torch.Tensor:
+    """y = x w^T on the tensor cores (bf16 in and out, fp32 accumulation).
+    x [..., K] with a dense last dimension, w [N, K]; returns y [..., N]."""
+    if x.dtype != torch.bfloat16 or w.dtype != torch.bfloat16:
+        raise TypeError("linear: bf16 operands expected")
+    K = x.shape[-1]
+    N = w.shape[0]
+    if w.shape != (N, K) or w.stride(1) != 1 or x.stride(-1) != 1:
+        raise ValueError("linear: x [..., K] and w [N, K] with contiguous rows expected")
+    x2 = x.reshape(-1, K)
+    M = x2.shape[0]
+    if y is None:
+        y = torch.empty((*x.shape[:-1], N), dtype=torch.bfloat16, device=x.device)
+    y2 = y.view(-1, N)
+    st = libssd.ssd_linear_bf16(_ptr(x2), x2.stride(0) if M else K, _ptr(w), w.stride(0), _ptr(y2),
+                                y2.stride(0) if M else N, M, N, K, _ptr(status), _stream(stream))
+    libssd.check("ssd_linear_bf16", st)
+    return y
+
+
+def mixer_workspace_bytes(b, L, d_model, H, P, N, G, Q, k) -> int:
+    return int(libssd.ssd_mixer_workspace_bytes(b, L, d_model, H, P, N, G, Q, k, libssd.SSD_BF16))
+
+
+def mixer_forward(hidden: torch.Tensor, W_in: torch.Tensor, conv_w: torch.Tensor, dt_bias: torch.Tensor | None,
+                  A: torch.Tensor, D: torch.Tensor | None, norm_w: torch.Tensor, W_out: torch.Tensor,
+                  H: int, P: int, G: int, N: int, *, conv_bias: torch.Tensor | None = None,
+                  conv_state: torch.Tensor | None = None, init_state: torch.Tensor | None = None,
+                  Q: int = 128, norm_groups: int = 1, eps: float = 1e-5, out: torch.Tensor | None = None,
+                  final_state: torch.Tensor | bool | None = True, workspace: torch.Tensor | None = None,
+                  status: torch.Tensor | None = None, stream=None):
+    """The Mamba-2 mixer forward in one call (in_proj, conv1d+SiLU, chunked
+    scan, gated RMSNorm, out_proj).  hidden [b, L, d_model] bf16; W_in
+    [2HP + 2GN + H, d_model] bf16; conv_w [conv_dim, k] f32; norm_w [H P] f32;
+    W_out [d_model, H P] bf16; conv_state [b, conv_dim, k] bf16 (updated in
+    place).  Returns (out [b, L, d_model] bf16, final_state [b, H, P, N] f32
+    or None)."""
+    if hidden.dim() != 3 or not hidden.is_contiguous() or hidden.dtype != torch.bfloat16:
+        raise ValueError("hidden must be a contiguous bf16 [b, L, d_model] tensor")
+    b, L, d_model = hidden.shape
+    d_inner = H * P
+    conv_dim = d_inner + 2 * G * N
+    k = conv_w.shape[1]
+    if W_in.shape != (d_inner + conv_dim + H, d_model) or not W_in.is_contiguous():
+        raise ValueError("W_in must be a contiguous [2HP + 2GN + H, d_model] tensor")
+    if W_out.shape != (d_model, d_inner) or not W_out.is_contiguous():
+        raise ValueError("W_out must be a contiguous [d_model, H P] tensor")
+    if conv_state is not None and (conv_state.shape != (b, conv_dim, k) or conv_state.dtype != torch.bfloat16
+                                   or not conv_state.is_contiguous()):
+        raise ValueError("conv_state must be a contiguous bf16 [b, conv_dim, k] tensor")
+    if out is None:
+        out = torch.empty((b, L, d_model), dtype=torch.bfloat16, device=hidden.device)
+    if final_state is True:
+        final_state = torch.empty((b, H, P, N), dtype=torch.float32, device=hidden.device)
+    elif final_state is False:
+        final_state = None
+    need = mixer_workspace_bytes(b, L, d_model, H, P, N, G, Q, k)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=hidden.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = libssd.ssd_mixer_fwd(
+        _ptr(hidden), _ptr(W_in), _ptr(_f32(conv_w, "conv_w")), _ptr(_f32(conv_bias, "conv_bias")), _ptr(conv_state),
+        _ptr(_f32(dt_bias, "dt_bias")), _ptr(_f32(A, "A")), _ptr(_f32(D, "D")), _ptr(_f32(norm_w, "norm_w")),
+        _ptr(W_out), _ptr(_f32(init_state, "init_state")), _ptr(out), _ptr(final_state), b, L, d_model, H, P, N, G,
+        Q, k, norm_groups, eps, libssd.SSD_BF16, _ptr(workspace), ws_bytes, _ptr(status), _stream(stream))
+    libssd.check("ssd_mixer_fwd", st)
+    return out, final_state

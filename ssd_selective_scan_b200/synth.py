@@ -165,3 +165,34 @@ def split_channels(u: torch.Tensor, shape: LayerShape):
     B = u[..., s.d_inner: s.d_inner + s.G * s.N]
     C = u[..., s.d_inner + s.G * s.N:]
     return x, B, C
+
+
+def mixer_inputs(shape: LayerShape, d_model: int, seed: int, *, conv_bias: bool = False,
+                 conv_state: bool = False, init_state: bool = False) -> dict:
+    """Inputs of the whole mixer (in_proj, the path, gated RMSNorm, out_proj),
+    host tensors: hidden [b, L, d_model] ~ N(0, 1) (the block's pre-norm makes
+    its input unit-scale), W_in [2HP + 2GN + H, d_model] bf16 whose rows give
+    z and x ~ N(0, 1), B and C ~ N(0, 1)/sqrt(N) and dt_raw ~ N(0, 1/4)
+    (the scan inputs' scales), dt_bias = -2.5 (dt around softplus(-2.5) =
+    0.08, inside the scan workloads' dt range), W_out [d_model, HP] bf16 with
+    N(0, 1/HP) entries, norm_w ~ 1 + N(0, 0.01), and the conv, A and D of the
+    scan workloads."""
+    g = _gen(seed)
+    s = shape
+    d_inner = s.H * s.P
+    out = {}
+    out["hidden"] = torch.randn(s.b, s.L, d_model, generator=g).to(torch.bfloat16)
+    scale = torch.cat([torch.ones(d_inner + d_inner), torch.full((2 * s.G * s.N,), 1.0 / math.sqrt(s.N)),
+                       torch.full((s.H,), 0.5)])
+    W_in = torch.randn(2 * d_inner + 2 * s.G * s.N + s.H, d_model, generator=g) / math.sqrt(d_model)
+    out["W_in"] = (W_in * scale[:, None]).to(torch.bfloat16)
+    out["conv_w"] = torch.randn(s.conv_dim, s.k, generator=g) * 0.5
+    out["conv_bias"] = (torch.randn(s.conv_dim, generator=g) * math.sqrt(0.1)) if conv_bias else None
+    out["dt_bias"] = torch.full((s.H,), -2.5)
+    out["A"] = _a_log_uniform(s.H, 1.0, 16.0, g)
+    out["D"] = torch.randn(s.H, generator=g)
+    out["norm_w"] = 1.0 + torch.randn(d_inner, generator=g) * 0.1
+    out["W_out"] = (torch.randn(d_model, d_inner, generator=g) / math.sqrt(d_inner)).to(torch.bfloat16)
+    out["conv_state"] = (_xbc(s, (s.b, s.k), g).transpose(1, 2).contiguous().to(torch.bfloat16)) if conv_state else None
+    out["init_state"] = (torch.randn(s.b, s.H, s.P, s.N, generator=g) * math.sqrt(0.1)) if init_state else None
+    return out

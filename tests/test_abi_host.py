@@ -37,8 +37,8 @@ def test_header_declares_the_entry_points():
         "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_static",
         "ssd_chunk_scan_fwd_varlen", "ssd_chunk_scan_varlen_workspace_bytes",
         "ssd_chunk_scan_workspace_bytes", "ssd_conv1d_silu", "ssd_conv_scan_fwd",
-        "ssd_conv_scan_workspace_bytes", "ssd_decode_step", "ssd_selftest_bounded_wait",
-        "ssd_state_update", "ssd_status_string"])
+        "ssd_conv_scan_workspace_bytes", "ssd_decode_step", "ssd_linear_bf16", "ssd_mixer_fwd",
+        "ssd_mixer_workspace_bytes", "ssd_selftest_bounded_wait", "ssd_state_update", "ssd_status_string"])
 
 
 def test_library_exports_every_declared_symbol():
@@ -262,3 +262,41 @@ def test_scan_bwd_validation():
     assert need > 2 * 40 * 8 * 64 * 128 * 4                    # the chunks' entering states, at least
     assert libssd.ssd_chunk_scan_bwd_workspace_bytes(0, 256, 40, 64, 128, 8, BF16) == 0
     assert bwd(N=1024, G=1, workspace_bytes=1 << 40) == UNS   # one CTA's shared memory would not fit
+
+
+def test_linear_validation():
+    P_ = 1 << 20   # any 16-byte aligned non-null address (nothing is launched)
+    f = libssd.ssd_linear_bf16
+    assert f(P_, 64, P_ + (1 << 16), 64, P_ + (1 << 18), 64, 0, 64, 64, None, None) == OK   # no rows
+    assert f(P_, 64, P_ + (1 << 16), 64, P_ + (1 << 18), 64, -1, 64, 64, None, None) == INV
+    assert f(None, 64, P_ + (1 << 16), 64, P_ + (1 << 18), 64, 4, 64, 64, None, None) == INV
+    assert f(P_, 64, P_ + (1 << 16), 64, P_ + (1 << 18), 64, 4, 60, 64, None, None) == INV   # N % 8
+    assert f(P_, 64, P_ + (1 << 16), 64, P_ + (1 << 18), 64, 4, 64, 60, None, None) == INV   # K % 8
+    assert f(P_, 32, P_ + (1 << 16), 64, P_ + (1 << 18), 64, 4, 64, 64, None, None) == INV   # ldx < K
+    assert f(P_ + 2, 64, P_ + (1 << 16), 64, P_ + (1 << 18), 64, 4, 64, 64, None, None) == INV   # alignment
+    assert f(P_, 64, P_ + (1 << 16), 64, P_, 64, 4, 64, 64, None, None) == INV   # y overlaps x
+
+
+def test_mixer_validation():
+    P_ = 1 << 20
+    ws = libssd.ssd_mixer_workspace_bytes(2, 300, 256, 8, 64, 128, 2, 128, 4, BF16)
+    assert ws > 2 * 300 * (2 * 512 + 512 + 8) * 2   # in_proj output alone
+    assert libssd.ssd_mixer_workspace_bytes(2, 300, 256, 8, 64, 128, 2, 128, 4, F32) == 0
+
+    def call(**kw):
+        a = dict(hidden=P_, W_in=P_ + (1 << 22), conv_w=P_ + (2 << 22), conv_bias=None, conv_state=None,
+                 dt_bias=None, A=P_ + (3 << 22), D=None, norm_w=P_ + (4 << 22), W_out=P_ + (5 << 22),
+                 init_state=None, out=P_ + (6 << 22), final_state=None, b=2, L=300, d_model=256, H=8, P=64,
+                 N=128, G=2, Q=128, k=4, norm_groups=1, eps=1e-5, dtype=BF16, workspace=P_ + (8 << 22),
+                 workspace_bytes=ws, status=None, stream=None)
+        a.update(kw)
+        return libssd.ssd_mixer_fwd(*a.values())
+    assert call(d_model=250) == INV          # d_model % 8
+    assert call(H=6, G=3) == UNS             # H % 8: the dt rows are not 16-byte rows
+    assert call(dtype=F32) == UNS            # bf16 projections only
+    assert call(norm_groups=3) == INV        # H*P not divisible
+    assert call(eps=-1.0) == INV
+    assert call(k=5) == UNS
+    assert call(hidden=None) == INV
+    assert call(workspace_bytes=ws - 256) == INV
+    assert call(out=P_ + 16) == INV          # out overlaps hidden
