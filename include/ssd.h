@@ -159,7 +159,10 @@ SSD_API size_t ssd_chunk_scan_workspace_bytes(int b, int L, int H, int P, int N,
  *              ignored; only this call uses it while it runs
  *   status     optional device int32: set to SSD_ERR_TIMEOUT by the kernels
  *              if a bounded wait gave up (the results are then invalid);
- *              never cleared by the library
+ *              never cleared by the library.  With status NULL a wait that
+ *              gave up goes unreported: callers that cannot rule out long
+ *              stalls (a GPU shared with other work, the tensor-core path's
+ *              cross-CTA hand-offs) should pass one and check it
  * Requirements: P a multiple of 8, N a multiple of 8, H % G == 0, Q in
  * {64, 128}; row_stride a multiple of 8 elements (16 bytes); all pointers
  * 16-byte aligned.
