@@ -41,7 +41,7 @@ namespace {
 template <typename T>
 __device__ inline void store_f(T* p, float v) { *p = io<T>::from_f(v); }
 
-constexpr int kBwdThreads = 256;
+constexpr int kBwdThreads = 1024;
 constexpr int kBwdQ = 32;   // chunk length of the backward pass
 
 struct BwdParams {
@@ -66,11 +66,20 @@ struct BwdParams {
     int L, H, P, N, G;
 };
 
-// shared-memory floats of one CTA
+// Shared-memory rows are padded by one float (row strides P+1, N+1, Q+1):
+// the phases that give each lane of a warp its own row (the Gram tiles, dx,
+// the per-token scalars) then hit 32 different banks instead of one.
 __host__ __device__ inline int bwd_smem_floats(int P, int N)
 {
-    const int Q = kBwdQ;
-    return 2 * P * N + 2 * Q * P + 2 * Q * N + 3 * Q * Q + 3 * Q * N + 15 * Q + kBwdThreads;
+    const int Q = kBwdQ, PS = P + 1, NS = N + 1, QS = Q + 1;
+    return 2 * P * NS + 2 * Q * PS + 2 * Q * NS + 3 * Q * QS + 3 * Q * NS + 15 * Q + kBwdThreads / 32;
+}
+
+__device__ inline float warp_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
 }
 
 template <typename T>
@@ -79,26 +88,27 @@ scan_bwd_chain_kernel(const BwdParams p)
 {
     extern __shared__ float sm[];
     const int P = p.P, N = p.N, L = p.L, H = p.H;
-    const int Q = kBwdQ;
+    const int Q = kBwdQ, PS = P + 1, NS = N + 1, QS = Q + 1;
     const int tid = threadIdx.x, nt = blockDim.x;
+    const int warp = tid >> 5, lane = tid & 31, nwarps = nt >> 5;
     const int chain = blockIdx.x;
     const int bi = chain / H, h = chain - bi * H;
     const int grp = h / (H / p.G);
     const int nchunks = (L + Q - 1) / Q;
 
-    float* sH0 = sm;                 // [P][N] entering state of the chunk
-    float* sG = sH0 + P * N;         // [P][N] state gradient at the chunk's end
-    float* sX = sG + P * N;          // [Q][P]
-    float* sDY = sX + Q * P;         // [Q][P]
-    float* sB = sDY + Q * P;         // [Q][N]
-    float* sC = sB + Q * N;          // [Q][N]
-    float* sYX = sC + Q * N;         // [Q][Q] dy_i . x_j
-    float* sCB = sYX + Q * Q;        // [Q][Q] C_i . B_j
-    float* sLm = sCB + Q * Q;        // [Q][Q] exp(cum_i - cum_j), j <= i (else 0)
-    float* sT1 = sLm + Q * Q;        // [Q][N] dY h0
-    float* sT2 = sT1 + Q * N;        // [Q][N] X g_end
-    float* sU = sT2 + Q * N;         // [Q][N] U
-    float* sDt = sU + Q * N;         // [Q]
+    float* sH0 = sm;                 // [P][NS] entering state of the chunk
+    float* sG = sH0 + P * NS;        // [P][NS] state gradient at the chunk's end
+    float* sX = sG + P * NS;         // [Q][PS]
+    float* sDY = sX + Q * PS;        // [Q][PS]
+    float* sB = sDY + Q * PS;        // [Q][NS]
+    float* sC = sB + Q * NS;         // [Q][NS]
+    float* sYX = sC + Q * NS;        // [Q][QS] dy_i . x_j
+    float* sCB = sYX + Q * QS;       // [Q][QS] C_i . B_j
+    float* sLm = sCB + Q * QS;       // [Q][QS] exp(cum_i - cum_j), j <= i (else 0)
+    float* sT1 = sLm + Q * QS;       // [Q][NS] dY h0
+    float* sT2 = sT1 + Q * NS;       // [Q][NS] X g_end
+    float* sU = sT2 + Q * NS;        // [Q][NS] U
+    float* sDt = sU + Q * NS;        // [Q]
     float* sCum = sDt + Q;           // [Q] inclusive cumsum of dt A
     float* sSig = sCum + Q;          // [Q] sigmoid(dt_raw + dt_bias)
     float* sXgB = sSig + Q;          // [Q] x_j^T g_end B_j
@@ -111,7 +121,7 @@ scan_bwd_chain_kernel(const BwdParams p)
     float* sEc = sEl + Q;            // [Q] exp(cum_j)
     float* sE = sEc + Q;             // [1]: exp(cum_last)
     float* sMisc = sE + Q;           // [3 Q]: scratch of the sequential step
-    float* sRed = sMisc + 3 * Q;     // [nthreads] block reduction
+    float* sRed = sMisc + 3 * Q;     // [nwarps] block reduction
 
     const T* xg = static_cast<const T*>(p.x);
     const T* Bg = static_cast<const T*>(p.B);
@@ -130,14 +140,14 @@ scan_bwd_chain_kernel(const BwdParams p)
         for (int i = tid; i < Q * P; i += nt) {
             const int j = i / P, pp = i - j * P;
             const size_t t = tok0 + s0 + j;
-            sX[i] = j < q ? ld_f(xg + t * p.row_stride + (size_t)h * P + pp) : 0.0f;
-            if (with_dy) sDY[i] = j < q ? ld_f(dyg + (t * H + h) * P + pp) : 0.0f;
+            sX[j * PS + pp] = j < q ? ld_f(xg + t * p.row_stride + (size_t)h * P + pp) : 0.0f;
+            if (with_dy) sDY[j * PS + pp] = j < q ? ld_f(dyg + (t * H + h) * P + pp) : 0.0f;
         }
         for (int i = tid; i < Q * N; i += nt) {
             const int j = i / N, n = i - j * N;
             const size_t t = tok0 + s0 + j;
-            sB[i] = j < q ? ld_f(Bg + t * p.row_stride + (size_t)grp * N + n) : 0.0f;
-            if (with_dy) sC[i] = j < q ? ld_f(Cg + t * p.row_stride + (size_t)grp * N + n) : 0.0f;
+            sB[j * NS + n] = j < q ? ld_f(Bg + t * p.row_stride + (size_t)grp * N + n) : 0.0f;
+            if (with_dy) sC[j * NS + n] = j < q ? ld_f(Cg + t * p.row_stride + (size_t)grp * N + n) : 0.0f;
         }
         for (int j = tid; j < Q; j += nt) {
             const float v = j < q ? ld_f(dtr + (tok0 + s0 + j) * H + h) + dtb : 0.0f;
@@ -157,11 +167,16 @@ scan_bwd_chain_kernel(const BwdParams p)
     };
 
     // ---------------- forward: the state entering every chunk ----------------
-    for (int i = tid; i < P * N; i += nt)
-        sH0[i] = p.init_state ? p.init_state[(size_t)chain * P * N + i] : 0.0f;
+    for (int i = tid; i < P * N; i += nt) {
+        const int pp = i / N, n = i - pp * N;
+        sH0[pp * NS + n] = p.init_state ? p.init_state[(size_t)chain * P * N + i] : 0.0f;
+    }
     __syncthreads();
     for (int c = 0; c < nchunks; ++c) {
-        for (int i = tid; i < P * N; i += nt) h0s[(size_t)c * P * N + i] = sH0[i];
+        for (int i = tid; i < P * N; i += nt) {
+            const int pp = i / N, n = i - pp * N;
+            h0s[(size_t)c * P * N + i] = sH0[pp * NS + n];
+        }
         const int q = load_chunk(c, false);
         const float cl = sCum[q - 1];
         for (int j = tid; j < Q; j += nt) sEl[j] = j < q ? expf(cl - sCum[j]) * sDt[j] : 0.0f;
@@ -169,19 +184,25 @@ scan_bwd_chain_kernel(const BwdParams p)
         const float ecl = expf(cl);
         for (int i = tid; i < P * N; i += nt) {
             const int pp = i / N, n = i - pp * N;
-            float acc = ecl * sH0[i];
-            for (int j = 0; j < q; ++j) acc += sX[j * P + pp] * sEl[j] * sB[j * N + n];
-            sH0[i] = acc;
+            float acc = ecl * sH0[pp * NS + n];
+            for (int j = 0; j < q; ++j) acc += sX[j * PS + pp] * sEl[j] * sB[j * NS + n];
+            sH0[pp * NS + n] = acc;
         }
         __syncthreads();
     }
 
     // ---------------- backward over the chunks ----------------
-    for (int i = tid; i < P * N; i += nt) sG[i] = p.dfinal ? p.dfinal[(size_t)chain * P * N + i] : 0.0f;
+    for (int i = tid; i < P * N; i += nt) {
+        const int pp = i / N, n = i - pp * N;
+        sG[pp * NS + n] = p.dfinal ? p.dfinal[(size_t)chain * P * N + i] : 0.0f;
+    }
     float accA = 0.0f, accD = 0.0f, accBias = 0.0f;   // thread 0's sums
     for (int c = nchunks - 1; c >= 0; --c) {
         const int s0 = c * Q;
-        for (int i = tid; i < P * N; i += nt) sH0[i] = h0s[(size_t)c * P * N + i];
+        for (int i = tid; i < P * N; i += nt) {
+            const int pp = i / N, n = i - pp * N;
+            sH0[pp * NS + n] = h0s[(size_t)c * P * N + i];
+        }
         const int q = load_chunk(c, true);
         const float cl = sCum[q - 1];
 
@@ -189,11 +210,11 @@ scan_bwd_chain_kernel(const BwdParams p)
         for (int i = tid; i < Q * Q; i += nt) {
             const int a = i / Q, bb = i - a * Q;
             float yx = 0.0f, cb = 0.0f;
-            for (int pp = 0; pp < P; ++pp) yx += sDY[a * P + pp] * sX[bb * P + pp];
-            for (int n = 0; n < N; ++n) cb += sC[a * N + n] * sB[bb * N + n];
-            sYX[i] = yx;
-            sCB[i] = cb;
-            sLm[i] = (bb <= a && a < q) ? expf(sCum[a] - sCum[bb]) : 0.0f;
+            for (int pp = 0; pp < P; ++pp) yx += sDY[a * PS + pp] * sX[bb * PS + pp];
+            for (int n = 0; n < N; ++n) cb += sC[a * NS + n] * sB[bb * NS + n];
+            sYX[a * QS + bb] = yx;
+            sCB[a * QS + bb] = cb;
+            sLm[a * QS + bb] = (bb <= a && a < q) ? expf(sCum[a] - sCum[bb]) : 0.0f;
         }
         for (int j = tid; j < Q; j += nt) {
             sEl[j] = j < q ? expf(cl - sCum[j]) : 0.0f;
@@ -204,17 +225,21 @@ scan_bwd_chain_kernel(const BwdParams p)
             const int k = i / N, n = i - k * N;
             float t1 = 0.0f, t2 = 0.0f;
             for (int pp = 0; pp < P; ++pp) {
-                t1 += sDY[k * P + pp] * sH0[pp * N + n];
-                t2 += sX[k * P + pp] * sG[pp * N + n];
+                t1 += sDY[k * PS + pp] * sH0[pp * NS + n];
+                t2 += sX[k * PS + pp] * sG[pp * NS + n];
             }
-            sT1[i] = t1;
-            sT2[i] = t2;
+            sT1[k * NS + n] = t1;
+            sT2[k * NS + n] = t2;
         }
-        // <g_end, h0>, per-thread partials
+        // <g_end, h0>: per-thread partials, then one per warp
         {
             float part = 0.0f;
-            for (int i = tid; i < P * N; i += nt) part += sG[i] * sH0[i];
-            sRed[tid] = part;
+            for (int i = tid; i < P * N; i += nt) {
+                const int pp = i / N, n = i - pp * N;
+                part += sG[pp * NS + n] * sH0[pp * NS + n];
+            }
+            part = warp_sum(part);
+            if (lane == 0) sRed[warp] = part;
         }
         __syncthreads();
 
@@ -223,58 +248,67 @@ scan_bwd_chain_kernel(const BwdParams p)
             const int r = i / N, n = i - r * N;
             float dc = 0.0f, u = 0.0f;
             if (r < q) {
-                dc = sEc[r] * sT1[i];
-                for (int j = 0; j <= r; ++j) dc += sLm[r * Q + j] * sDt[j] * sYX[r * Q + j] * sB[j * N + n];
-                u = sEl[r] * sT2[i];
-                for (int k = r; k < q; ++k) u += sLm[k * Q + r] * sYX[k * Q + r] * sC[k * N + n];
+                dc = sEc[r] * sT1[r * NS + n];
+                for (int j = 0; j <= r; ++j) dc += sLm[r * QS + j] * sDt[j] * sYX[r * QS + j] * sB[j * NS + n];
+                u = sEl[r] * sT2[r * NS + n];
+                for (int k = r; k < q; ++k) u += sLm[k * QS + r] * sYX[k * QS + r] * sC[k * NS + n];
                 const size_t t = tok0 + s0 + r;
                 p.ws_dC[(t * H + h) * N + n] = dc;
                 p.ws_dB[(t * H + h) * N + n] = sDt[r] * u;
             }
-            sU[i] = u;
+            sU[r * NS + n] = u;
         }
         for (int i = tid; i < Q * P; i += nt) {
             const int j = i / P, pp = i - j * P;
             if (j < q) {
                 float gb = 0.0f;
-                for (int n = 0; n < N; ++n) gb += sB[j * N + n] * sG[pp * N + n];
+                for (int n = 0; n < N; ++n) gb += sB[j * NS + n] * sG[pp * NS + n];
                 gb *= sEl[j];
-                for (int k = j; k < q; ++k) gb += sLm[k * Q + j] * sCB[k * Q + j] * sDY[k * P + pp];
-                const float dxv = Dh * sDY[i] + sDt[j] * gb;
+                for (int k = j; k < q; ++k) gb += sLm[k * QS + j] * sCB[k * QS + j] * sDY[k * PS + pp];
+                const float dxv = Dh * sDY[j * PS + pp] + sDt[j] * gb;
                 store_f(static_cast<T*>(p.dx) + ((tok0 + s0 + j) * H + h) * P + pp, dxv);
             }
         }
         __syncthreads();
 
-        // 3. per-token scalars: x^T g_end B, dy^T h0 C, U.B, dy.x, the
-        //    masked pair tile's column and row sums
-        for (int j = tid; j < Q; j += nt) {
+        // 3. per-token scalars, one warp per token: x^T g_end B, dy^T h0 C,
+        //    U.B, dy.x, the masked pair tile's column and row sums
+        for (int j = warp; j < Q; j += nwarps) {
             float xgb = 0.0f, yhc = 0.0f, ub = 0.0f, dd = 0.0f, col = 0.0f, row = 0.0f;
             if (j < q) {
-                for (int n = 0; n < N; ++n) {
-                    xgb += sT2[j * N + n] * sB[j * N + n];
-                    yhc += sT1[j * N + n] * sC[j * N + n];
-                    ub += sU[j * N + n] * sB[j * N + n];
+                for (int n = lane; n < N; n += 32) {
+                    const float b = sB[j * NS + n];
+                    xgb += sT2[j * NS + n] * b;
+                    yhc += sT1[j * NS + n] * sC[j * NS + n];
+                    ub += sU[j * NS + n] * b;
                 }
-                for (int pp = 0; pp < P; ++pp) dd += sDY[j * P + pp] * sX[j * P + pp];
-                for (int k = j; k < q; ++k)   // W[k][j], k >= j
-                    col += sLm[k * Q + j] * sDt[j] * sYX[k * Q + j] * sCB[k * Q + j];
-                for (int i2 = 0; i2 <= j; ++i2)   // W[j][i2], i2 <= j
-                    row += sLm[j * Q + i2] * sDt[i2] * sYX[j * Q + i2] * sCB[j * Q + i2];
+                for (int pp = lane; pp < P; pp += 32) dd += sDY[j * PS + pp] * sX[j * PS + pp];
+                for (int k = j + lane; k < q; k += 32)   // W[k][j], k >= j
+                    col += sLm[k * QS + j] * sDt[j] * sYX[k * QS + j] * sCB[k * QS + j];
+                for (int i2 = lane; i2 <= j; i2 += 32)   // W[j][i2], i2 <= j
+                    row += sLm[j * QS + i2] * sDt[i2] * sYX[j * QS + i2] * sCB[j * QS + i2];
             }
-            sXgB[j] = xgb;
-            sYhC[j] = yhc;
-            sUB[j] = ub;
-            sDD[j] = dd;
-            sCol[j] = col;
-            sRow[j] = row;
+            xgb = warp_sum(xgb);
+            yhc = warp_sum(yhc);
+            ub = warp_sum(ub);
+            dd = warp_sum(dd);
+            col = warp_sum(col);
+            row = warp_sum(row);
+            if (lane == 0) {
+                sXgB[j] = xgb;
+                sYhC[j] = yhc;
+                sUB[j] = ub;
+                sDD[j] = dd;
+                sCol[j] = col;
+                sRow[j] = row;
+            }
         }
         __syncthreads();
 
         // 4. the decay gradient and ddt (sequential over the chunk's tokens)
         if (tid == 0) {
             float gh0 = 0.0f;
-            for (int i = 0; i < nt; ++i) gh0 += sRed[i];
+            for (int w = 0; w < nwarps; ++w) gh0 += sRed[w];
             const float t1 = sE[0] * gh0;
             float* t3 = sMisc;   // suffix sums of e^cum_k dy_k^T h0 C_k
             float suf = 0.0f;
@@ -298,14 +332,17 @@ scan_bwd_chain_kernel(const BwdParams p)
         // 5. the entering state's gradient, the previous chunk's g_end
         for (int i = tid; i < P * N; i += nt) {
             const int pp = i / N, n = i - pp * N;
-            float g = sE[0] * sG[i];
-            for (int k = 0; k < q; ++k) g += sEc[k] * sDY[k * P + pp] * sC[k * N + n];
-            sG[i] = g;
+            float g = sE[0] * sG[pp * NS + n];
+            for (int k = 0; k < q; ++k) g += sEc[k] * sDY[k * PS + pp] * sC[k * NS + n];
+            sG[pp * NS + n] = g;
         }
         __syncthreads();
     }
     if (p.dinit)
-        for (int i = tid; i < P * N; i += nt) p.dinit[(size_t)chain * P * N + i] = sG[i];
+        for (int i = tid; i < P * N; i += nt) {
+            const int pp = i / N, n = i - pp * N;
+            p.dinit[(size_t)chain * P * N + i] = sG[pp * NS + n];
+        }
     if (tid == 0) {
         const int nch = (int)gridDim.x;
         p.ws_part[chain] = accA;
