@@ -528,7 +528,11 @@ ssd_status_t ssd_mixer_fwd(const void* hidden, const void* W_in, const float* co
 size_t ssd_chunk_scan_bwd_workspace_bytes(int b, int L, int H, int P, int N, int G, ssd_dtype_t dtype)
 {
     if (b <= 0 || L <= 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || !valid_dtype(dtype)) return 0;
-    return ssd::scan_bwd_workspace_bytes(b, L, H, P, N);
+    const size_t general = ssd::scan_bwd_workspace_bytes(b, L, H, P, N);
+    // a tensor-core shape may still take the general path (unaligned pointers)
+    if (ssd::scan_bwd_tc_shape(P, N, dtype == SSD_BF16))
+        return std::max(general, ssd::scan_bwd_tc_workspace_bytes(b, L, H));
+    return general;
 }
 
 ssd_status_t ssd_chunk_scan_bwd(const void* x, const void* B, const void* C, int64_t row_stride, const void* dt_raw,
@@ -591,9 +595,10 @@ ssd_status_t ssd_chunk_scan_bwd(const void* x, const void* B, const void* C, int
         return from_cuda(err);
     }
     if ((int64_t)b * H > 0x7fffffffLL) return SSD_ERR_UNSUPPORTED;
-    if (ssd::scan_bwd_smem_bytes(P, N) > (size_t)max_optin_smem()) return SSD_ERR_UNSUPPORTED;
     ssd::ScanBwdArgs a{x, B, C, row_stride, dt_raw, dt_bias, A, D, init_state, dy, dfinal, dx, dB, dC, ddt_raw,
                        dA, dD, ddt_bias, dinit, b, L, H, P, N, G, dtype == SSD_BF16, workspace};
+    if (ssd::scan_bwd_tc_supported(a)) return from_cuda(ssd::launch_scan_bwd_tc(a, stream));
+    if (ssd::scan_bwd_smem_bytes(P, N) > (size_t)max_optin_smem()) return SSD_ERR_UNSUPPORTED;
     return from_cuda(ssd::launch_scan_bwd(a, stream));
 }
 

@@ -37,8 +37,20 @@ struct ScanBwdArgs {
     void* workspace;
 };
 
+// General path (scan_bwd.cu): float32 on the CUDA cores, any P and N whose
+// shared-memory footprint fits one CTA.
 size_t scan_bwd_smem_bytes(int P, int N);
 size_t scan_bwd_workspace_bytes(int b, int L, int H, int P, int N);
 cudaError_t launch_scan_bwd(const ScanBwdArgs& a, cudaStream_t s);
+
+// Tensor-core path (scan_bwd_tc.cu): bf16 I/O with P = 64, N = 128.
+// scan_bwd_tc_shape: the dtype and shape qualify (the workspace is sized for
+// both paths then); scan_bwd_tc_supported: the call also meets the TMA and
+// vector-store alignment (16-byte pointers, row_stride % 8 == 0) and size
+// limits, else the general path runs.
+bool scan_bwd_tc_shape(int P, int N, bool bf16);
+bool scan_bwd_tc_supported(const ScanBwdArgs& a);
+size_t scan_bwd_tc_workspace_bytes(int b, int L, int H);
+cudaError_t launch_scan_bwd_tc(const ScanBwdArgs& a, cudaStream_t s);
 
 }  // namespace ssd

@@ -1,0 +1,1066 @@
+// scan_bwd_tc.cu -- backward pass of the chunked SSD scan on the 5th-
+// generation tensor cores (tcgen05 + TMEM): bf16 I/O, fp32 accumulation,
+// chunks of Q = 128 tokens, head dim P = 64, state size N = 128.
+//
+// The gradients of the recurrence of "Hybrid Architectures for Language
+// Models" (summary page, section 2 Background: h_t = exp(dt_t A) h_{t-1} +
+// dt_t x_t B_t^T, y_t = h_t C_t + D x_t) in the chunked matrix form of
+// scan_bwd.cu, reorganised so that each chunk is independent once its
+// entering state h0 and the state gradient at its end g are known.  In log2
+// units, l_t = dt_t A log2(e), cum = inclusive cumsum of l inside a chunk, cl
+// its last value, Ec_k = 2^cum_k, El_j = 2^(cl - cum_j), Lm[i][j] =
+// 2^(cum_i - cum_j) for j <= i (else 0):
+//
+// 1. bwd_states_kernel (tensor cores), per chunk and head:
+//      S^T  = B^T (w o X),  w_j = El_j dt_j      the chunk's own end state
+//      dS^T = C^T (Ec o dY)                     its part of the entering
+//                                               state's gradient
+// 2. bwd_pass_kernel (CUDA cores), per (sequence, head), chunk after chunk:
+//      h0_{c+1} = 2^cl_c h0_c + S_c,   g_{c-1} = 2^cl_c g_c + dS_c,
+//      t1_c = 2^cl_c <g_c, h0_c>;   the initial state's gradient is g_{-1}.
+// 3. bwd_chunk_kernel (tensor cores), per chunk and head:
+//      YX = dY X^T,  CB = C B^T                              (Q x Q)
+//      M1 = Lm o dt_j o YX,  M2 = Lm o YX,  M3 = Lm o CB      (bf16 tiles)
+//      dC = (Ec o dY) h0 + M1 B                              (Q x N)
+//      U  = (El o X) g + M2^T C,    dB = dt o U               (Q x N)
+//      gB = El o (B g^T) + M3^T dY, dx = D dy + dt o gB       (Q x P)
+//    The decay gradient r_t = <g_t, exp(dt_t A) h_{t-1}> has a closed form
+//    in the tiles' row sums (U.B = El x^T g B + sum_k M2 CB and
+//    dC.C = Ec dy^T h0 C + W, W_k = sum_j M1[k][j] CB[k][j]):
+//      r_t = t1 - sum_k W_k + sum_{j<t} dt_j U_j.B_j + sum_{k>=t} dC_k.C_k,
+//    then ddt = U.B + A r, ddt_raw = ddt sigmoid(dt_raw + dt_bias),
+//    dA = sum dt r, dD = sum dy.x, ddt_bias = sum ddt_raw.  The products
+//    take M1 and M2 rounded to bf16 while W is summed in fp32, so the
+//    rounding is compensated exactly: r_t gains sum_{j<t} colD_j -
+//    sum_{k>=t} rowD_k, rowD_k = sum_j (bf16(M1) - M1)[k][j] CB[k][j],
+//    colD_j = dt_j sum_k (M2 - bf16(M2))[k][j] CB[k][j].  (Without it the
+//    large sums of the closed form amplify the bf16 rounding of the tiles.)
+// dB and dC of a group are sums over its heads: one CTA takes the heads of a
+// group in order and keeps the sums in registers.  dA, dD and ddt_bias are
+// summed over sequences, chunks and row quarters in a fixed order by a last
+// kernel, so the result is deterministic.
+//
+// Kernels 1 and 3: one CTA per (chunk, sequence, group), a TMA producer
+// warp, an MMA warp (one thread issues tcgen05.mma; TMEM allocation) and
+// elementwise warps that serve TMEM lanes 32*(warp%4).. (token rows, or
+// state columns n).  Tiles are 128-byte swizzled, loaded by TMA without
+// multicast.  Every mbarrier wait is bounded (1 s); a CTA that gives up
+// sets the timeout flag in the workspace's first word and ends.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "scan_bwd.h"
+#include "sm100.cuh"
+
+namespace ssd {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kQ = 128, kP = 64, kN = 128;
+constexpr uint32_t kTileHalf = 16384;        // 128 rows x 64 bf16, swizzled
+constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kPassSlices = 8;               // CTAs per chain in the passing kernel
+constexpr int kPassThreads = 256;            // 4 state elements per thread
+constexpr int kParts = 4;                    // dA / dD / ddt_bias partials per (chain, chunk)
+
+constexpr uint32_t kStatesDim = kN * kP;     // floats of one chunk state
+
+__device__ inline uint32_t sw128(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
+
+__device__ inline uint4 pack8(const float* v)
+{
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        w[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__device__ inline void unpack8(uint4 q, float* v)
+{
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+// K-major operand, 128 rows, K up to 128 as 64-wide halves: K-step k (16 elements)
+__device__ inline uint64_t desc_k(uint32_t base, int k)
+{
+    return umma_desc_sw128(base + (uint32_t)(k >> 2) * kTileHalf + (uint32_t)(k & 3) * 32u, 16u, 1024u);
+}
+
+// MN-major operand with K along rows: K-step k (16 rows); 64-wide M/N blocks kTileHalf apart
+__device__ inline uint64_t desc_mn(uint32_t base, int k)
+{
+    return umma_desc_sw128(base + (uint32_t)k * 2048u, kTileHalf, 1024u);
+}
+
+// A wait that ignores the abort flag: used once at the end to let this
+// CTA's own TMA loads land before shared memory is released.
+__device__ inline void drain_wait(uint64_t* bar, uint32_t parity)
+{
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer_ns() - t0 > kWaitNs) break;
+}
+
+// Named barrier among n threads that also ORs a flag over them: every
+// participant gets the same answer, so a give-up seen by any thread ends
+// the loop of all of them at the same barrier.
+__device__ inline bool named_bar_any(int id, int n, bool v)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "barrier.red.or.pred p, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
+
+__device__ inline float warp_incl_scan(float v, int lane)
+{
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+    }
+    return v;
+}
+
+// Column sums over a warp's 32 rows of 16 values per lane: lane l (and
+// l + 16) receives the sum of column l & 15 (31 shuffles, fixed order).
+__device__ inline float warp_colsum16(float (&v)[16], int lane)
+{
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v[k] += __shfl_xor_sync(0xffffffffu, v[k], 16);
+#pragma unroll
+    for (int off = 8; off >= 1; off >>= 1) {
+        const bool up = (lane & off) != 0;
+#pragma unroll
+        for (int k = 0; k < off; ++k) {
+            const float send = up ? v[k] : v[k + off];
+            const float keep = up ? v[k + off] : v[k];
+            v[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+    return v[0];
+}
+
+__device__ inline float bf16_round(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
+
+__device__ inline float warp_total(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+struct TcParams {
+    const __nv_bfloat16* dt_raw;   // [b][L][H]
+    const float* dt_bias;
+    const float* A;
+    const float* D;
+    const float* init_state;       // [b][H][P][N]
+    const float* dfinal;           // [b][H][P][N]
+    __nv_bfloat16* dx;             // [b][L][H][P]
+    __nv_bfloat16* dB;             // [b][L][G][N]
+    __nv_bfloat16* dC;
+    __nv_bfloat16* ddt_raw;        // [b][L][H]
+    float* dA;
+    float* dD;
+    float* ddt_bias;
+    float* dinit;                  // [b][H][P][N]
+    int32_t* status;               // workspace word 0: timeout flag
+    float* ws_S;                   // [chains][nc][N][P] fp32: S, then h0
+    float* ws_dS;                  // [chains][nc][N][P] fp32
+    __nv_bfloat16* ws_hb;          // [chains][nc][N][P] bf16 h0
+    __nv_bfloat16* ws_gb;          // [chains][nc][N][P] bf16 g
+    float* ws_cl;                  // [chains][nc]
+    float* ws_t1;                  // [chains][nc][kPassSlices]
+    float* ws_part;                // [3][chains][nc][kParts]
+    int b, L, H, G, nc;
+};
+
+// dt_t and sigmoid(dt_raw + dt_bias) of chunk row i (0 past the sequence's end)
+__device__ inline void row_dt(const TcParams& p, int bi, int h, int t, bool valid, float& dt, float& sig)
+{
+    float v = 0.0f;
+    if (valid) v = __bfloat162float(p.dt_raw[((size_t)bi * p.L + t) * p.H + h]) + (p.dt_bias ? p.dt_bias[h] : 0.0f);
+    dt = valid ? softplus_f(v) : 0.0f;
+    sig = 1.0f / (1.0f + __expf(-v));
+}
+
+// Inclusive cumsum of l over the 128 rows held by 4 warps (one row per
+// thread, warp w%4 = quadrant): warp scans, then the lower quadrants' totals.
+// `tot` is 4 floats of shared memory; `bar_id` a named barrier of the 128 threads.
+__device__ inline float block_cumsum128(float l, int quad, int lane, float* tot, int bar_id)
+{
+    const float inc = warp_incl_scan(l, lane);
+    if (lane == 31) tot[quad] = inc;
+    named_bar_sync(bar_id, 128);
+    float off = 0.0f;
+    for (int q = 0; q < quad; ++q) off += tot[q];
+    return inc + off;
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 1: chunk states S^T = B^T (w o X) and dS^T = C^T (Ec o dY)
+// ---------------------------------------------------------------------------
+namespace k1 {
+constexpr int kEwWarps = 4;
+constexpr int kThreads = (kEwWarps + 2) * 32;   // warp 0 producer, 1 MMA, 2..5 rows
+constexpr int kOffB = 0, kOffC = 32768, kOffX = 65536, kOffDY = 81920, kOffWX = 98304, kOffWDY = 114688;
+constexpr int kOffVec = 131072;                 // tot[4]
+constexpr int kOffBar = kOffVec + 64;
+constexpr int kOffMisc = kOffBar + 8 * 8;
+constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+constexpr uint32_t kTmemCols = 128;             // S^T [0,64), dS^T [64,128)
+constexpr uint32_t kIdS = umma_idesc_bf16(128, 64, true, true);   // B^T (MN) x wX (MN)
+}  // namespace k1
+
+__global__ void __launch_bounds__(k1::kThreads, 1)
+bwd_states_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
+                  const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmDY,
+                  const TcParams p)
+{
+    using namespace k1;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x;
+    const int bi = blockIdx.y / p.G, g = blockIdx.y - bi * p.G;
+    const int hpg = p.H / p.G;
+    const int t0 = c * kQ;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+    uint64_t* bar_ld = bars + 0;     // X, dY (and B, C for the first head) landed
+    uint64_t* bar_w = bars + 1;      // w o X and Ec o dY written (row warps)
+    uint64_t* bar_xfree = bars + 2;  // X, dY read (row warps)
+    uint64_t* bar_mma = bars + 3;    // S^T, dS^T in TMEM
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+    volatile int* aborted = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+    float* tot = reinterpret_cast<float*>(smem + kOffVec);
+
+    if (tid == 0) {
+        *aborted = 0;
+        mbar_init(bar_ld, 1);
+        mbar_init(bar_w, kEwWarps * 32);
+        mbar_init(bar_xfree, kEwWarps * 32);
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tensormap(&tmX);
+            prefetch_tensormap(&tmB);
+            prefetch_tensormap(&tmC);
+            prefetch_tensormap(&tmDY);
+            int issued = 0;
+            for (int hh = 0; hh < hpg; ++hh) {
+                const int h = g * hpg + hh;
+                if (hh > 0 && !mbar_wait_bounded(bar_xfree, (uint32_t)(hh - 1) & 1u, kWaitNs, aborted, p.status))
+                    break;
+                mbar_arrive_expect_tx(bar_ld, hh == 0 ? 6 * kTileHalf : 2 * kTileHalf);
+                tma_load_3d(smem + kOffX, &tmX, h * kP, t0, bi, bar_ld);
+                tma_load_3d(smem + kOffDY, &tmDY, h * kP, t0, bi, bar_ld);
+                if (hh == 0) {
+                    tma_load_3d(smem + kOffB, &tmB, g * kN, t0, bi, bar_ld);
+                    tma_load_3d(smem + kOffB + kTileHalf, &tmB, g * kN + 64, t0, bi, bar_ld);
+                    tma_load_3d(smem + kOffC, &tmC, g * kN, t0, bi, bar_ld);
+                    tma_load_3d(smem + kOffC + kTileHalf, &tmC, g * kN + 64, t0, bi, bar_ld);
+                }
+                ++issued;
+            }
+            if (issued > 0) drain_wait(bar_ld, (uint32_t)(issued - 1) & 1u);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t sB = smem_u32(smem + kOffB), sC = smem_u32(smem + kOffC);
+            const uint32_t sWX = smem_u32(smem + kOffWX), sWDY = smem_u32(smem + kOffWDY);
+            int committed = 0;
+            for (int hh = 0; hh < hpg; ++hh) {
+                const uint32_t ph = (uint32_t)hh & 1u;
+                // (the row warps waited for the loads before arriving here; a
+                // second waiter on bar_ld could fall two phases behind it)
+                if (!mbar_wait_bounded(bar_w, ph, kWaitNs, aborted, p.status)) break;
+                tc_fence_after_sync();
+#pragma unroll
+                for (int k = 0; k < 8; ++k) umma_bf16(tmem, desc_mn(sB, k), desc_mn(sWX, k), kIdS, k > 0);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) umma_bf16(tmem + 64, desc_mn(sC, k), desc_mn(sWDY, k), kIdS, k > 0);
+                umma_commit(bar_mma);
+                ++committed;
+            }
+            if (committed > 0) drain_wait(bar_mma, (uint32_t)(committed - 1) & 1u);
+        }
+        __syncwarp();
+    } else {
+        // row warps: thread = token row i (weights), then state row n = i (epilogue)
+        const int quad = warp & 3;
+        const int i = quad * 32 + lane;
+        const int t = t0 + i;
+        const bool valid = t < p.L;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        bool ok = true;
+        for (int hh = 0; hh < hpg; ++hh) {
+            const int h = g * hpg + hh;
+            const int chain = bi * p.H + h;
+            const uint32_t ph = (uint32_t)hh & 1u;
+            float dt, sig;
+            row_dt(p, bi, h, t, valid, dt, sig);
+            // tot[] of the previous head read; a give-up anywhere ends all rows here
+            if (named_bar_any(1, 128, !ok)) break;
+            const float cum = block_cumsum128(dt * p.A[h] * kLog2e, quad, lane, tot, 1);
+            const float cl = tot[0] + tot[1] + tot[2] + tot[3];
+            const float w = ex2_approx(cl - cum) * dt;
+            const float e = ex2_approx(cum);
+            if (i == 0) p.ws_cl[(size_t)chain * p.nc + c] = cl;
+            // (after a give-up the head runs on without waiting, so that
+            // every row reaches the next barrier)
+            ok = mbar_wait_bounded(bar_ld, ph, kWaitNs, aborted, p.status) && ok;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                float v[8];
+                const uint32_t o = sw128(i, ch);
+                unpack8(*reinterpret_cast<const uint4*>(smem + kOffX + o), v);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) v[k] *= w;
+                *reinterpret_cast<uint4*>(smem + kOffWX + o) = pack8(v);
+                unpack8(*reinterpret_cast<const uint4*>(smem + kOffDY + o), v);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) v[k] *= e;
+                *reinterpret_cast<uint4*>(smem + kOffWDY + o) = pack8(v);
+            }
+            mbar_arrive(bar_xfree);
+            fence_proxy_async_smem();
+            mbar_arrive(bar_w);
+            ok = mbar_wait_bounded(bar_mma, ph, kWaitNs, aborted, p.status) && ok;
+            tc_fence_after_sync();
+            // state row n = i: S^T[n][0..63], dS^T[n][0..63]
+            float* dS = p.ws_S + ((size_t)chain * p.nc + c) * kStatesDim + (size_t)i * kP;
+            float* ddS = p.ws_dS + ((size_t)chain * p.nc + c) * kStatesDim + (size_t)i * kP;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float v[32];
+                tmem_ld32(tmem + lane_off + (uint32_t)(half * 32), v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < 32; k += 4)
+                    *reinterpret_cast<float4*>(dS + half * 32 + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+                tmem_ld32(tmem + lane_off + 64u + (uint32_t)(half * 32), v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < 32; k += 4)
+                    *reinterpret_cast<float4*>(ddS + half * 32 + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+            }
+            tc_fence_before_sync();
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 2: entering states forward, state gradients backward
+// ---------------------------------------------------------------------------
+// Grid (chains, kPassSlices); thread j of slice s owns state elements
+// e = s*1024 + 4j .. +3 of the [n][p] layout (one n, four p).
+__global__ void __launch_bounds__(kPassThreads)
+bwd_pass_kernel(const TcParams p)
+{
+    __shared__ float red[kPassThreads / 32];
+    const int chain = blockIdx.x, s = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int e0 = s * (kStatesDim / kPassSlices) + tid * 4;
+    const int n = e0 / kP, p0 = e0 - n * kP;
+    const int nc = p.nc;
+    const size_t base = (size_t)chain * nc * kStatesDim + e0;
+    const float* cl = p.ws_cl + (size_t)chain * nc;
+
+    // forward: h0 of every chunk (fp32 in place of S, bf16 copy)
+    float h[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        h[k] = p.init_state ? p.init_state[(size_t)chain * kStatesDim + (size_t)(p0 + k) * kN + n] : 0.0f;
+    float4 Snext = *reinterpret_cast<const float4*>(p.ws_S + base);
+    for (int c = 0; c < nc; ++c) {
+        const float4 S = Snext;
+        if (c + 1 < nc) Snext = *reinterpret_cast<const float4*>(p.ws_S + base + (size_t)(c + 1) * kStatesDim);
+        const size_t o = base + (size_t)c * kStatesDim;
+        *reinterpret_cast<float4*>(p.ws_S + o) = make_float4(h[0], h[1], h[2], h[3]);
+        __nv_bfloat162 lo = __floats2bfloat162_rn(h[0], h[1]), hi = __floats2bfloat162_rn(h[2], h[3]);
+        *reinterpret_cast<uint2*>(p.ws_hb + o) =
+            make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+        const float d = ex2_approx(cl[c]);
+        h[0] = d * h[0] + S.x;
+        h[1] = d * h[1] + S.y;
+        h[2] = d * h[2] + S.z;
+        h[3] = d * h[3] + S.w;
+    }
+
+    // backward: g at the end of every chunk (bf16), t1 partials, dinit
+    float gv[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        gv[k] = p.dfinal ? p.dfinal[(size_t)chain * kStatesDim + (size_t)(p0 + k) * kN + n] : 0.0f;
+    for (int c = nc - 1; c >= 0; --c) {
+        const size_t o = base + (size_t)c * kStatesDim;
+        const float4 h0 = *reinterpret_cast<const float4*>(p.ws_S + o);
+        const float4 dS = *reinterpret_cast<const float4*>(p.ws_dS + o);
+        __nv_bfloat162 lo = __floats2bfloat162_rn(gv[0], gv[1]), hi = __floats2bfloat162_rn(gv[2], gv[3]);
+        *reinterpret_cast<uint2*>(p.ws_gb + o) =
+            make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+        const float d = ex2_approx(cl[c]);
+        float part = gv[0] * h0.x + gv[1] * h0.y + gv[2] * h0.z + gv[3] * h0.w;
+        part = warp_total(part);
+        if (lane == 0) red[warp] = part;
+        __syncthreads();
+        if (tid == 0) {
+            float t = 0.0f;
+            for (int w = 0; w < kPassThreads / 32; ++w) t += red[w];
+            p.ws_t1[((size_t)chain * nc + c) * kPassSlices + s] = d * t;
+        }
+        __syncthreads();
+        gv[0] = d * gv[0] + dS.x;
+        gv[1] = d * gv[1] + dS.y;
+        gv[2] = d * gv[2] + dS.z;
+        gv[3] = d * gv[3] + dS.w;
+    }
+    if (p.dinit) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) p.dinit[(size_t)chain * kStatesDim + (size_t)(p0 + k) * kN + n] = gv[k];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 3: the chunk's gradients
+// ---------------------------------------------------------------------------
+namespace k3 {
+constexpr int kEwWarps = 16;                    // 4 lane quadrants x 4 column quarters
+constexpr int kEwThreads = kEwWarps * 32;
+constexpr int kThreads = kEwThreads + 64;       // warp 0 producer, 1 MMA, 2..17 elementwise
+// shared memory (1024-aligned); region R holds X, h0, Ec o dY, El o X in
+// the first phase and the tiles M1, M2, M3 in the second
+constexpr int kOffB = 0, kOffC = 32768, kOffDY = 65536, kOffG = 81920, kOffR = 98304;
+constexpr int kOffX = kOffR, kOffH = kOffR + 16384, kOffEDY = kOffR + 32768, kOffEX = kOffR + 49152;
+constexpr int kOffM1 = kOffR, kOffM2 = kOffR + 32768, kOffM3 = kOffR + 65536;
+constexpr int kOffVec = kOffR + 98304;          // floats: cum, dt, sig [128] each, partials [6][4][128], tot [8]
+constexpr int kVecFloats = 3 * kQ + 24 * kQ + 8;
+constexpr int kOffBar = kOffVec + ((kVecFloats * 4 + 63) / 64) * 64;
+constexpr int kNumBars = 6;
+constexpr int kOffMisc = kOffBar + 8 * kNumBars;
+constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+constexpr uint32_t kTmemCols = 512;
+// TMEM columns
+constexpr uint32_t kColYX = 0;     // YX [0,128); after the tiles are built: gB [0,64), B g^T [64,128)
+constexpr uint32_t kColGB = 0, kColBG = 64;
+constexpr uint32_t kColCB = 128;   // CB (kept across the group's heads)
+constexpr uint32_t kColDC = 256;   // dC
+constexpr uint32_t kColU = 384;    // U
+constexpr uint32_t kIdKK128 = umma_idesc_bf16(128, 128, false, false);
+constexpr uint32_t kIdKM128 = umma_idesc_bf16(128, 128, false, true);
+constexpr uint32_t kIdMM128 = umma_idesc_bf16(128, 128, true, true);
+constexpr uint32_t kIdMM64 = umma_idesc_bf16(128, 64, true, true);
+constexpr uint32_t kIdKM64 = umma_idesc_bf16(128, 64, false, true);
+constexpr int kBarEw = 1, kBarRows = 2;         // named barriers: all elementwise warps; the 4 row warps
+}  // namespace k3
+
+__global__ void __launch_bounds__(k3::kThreads, 1)
+bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
+                 const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmDY,
+                 const __grid_constant__ CUtensorMap tmHb, const __grid_constant__ CUtensorMap tmGb, const TcParams p)
+{
+    using namespace k3;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x;
+    const int bi = blockIdx.y / p.G, g = blockIdx.y - bi * p.G;
+    const int hpg = p.H / p.G;
+    const int t0 = c * kQ;
+    const int q = min(kQ, p.L - t0);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+    uint64_t* bar_ld = bars + 0;   // X, dY, h0, g (and B, C for the first head) landed
+    uint64_t* bar_e0 = bars + 1;   // Ec o dY, El o X written
+    uint64_t* bar_p1 = bars + 2;   // YX, CB, dC and U's first products done
+    uint64_t* bar_e1 = bars + 3;   // M1, M2, M3 written; YX read
+    uint64_t* bar_p2 = bars + 4;   // dC, U, gB, B g^T done
+    uint64_t* bar_e2 = bars + 5;   // the head's epilogue done (dY, g, M tiles free)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+    volatile int* aborted = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+    float* sCum = reinterpret_cast<float*>(smem + kOffVec);
+    float* sDt = sCum + kQ;
+    float* sSig = sDt + kQ;
+    float* sRow = sSig + kQ;        // [4 quarters][128]: W partials
+    float* sDD = sRow + 4 * kQ;     // dy.x partials
+    float* sDCC = sDD + 4 * kQ;     // dC.C partials
+    float* sUB = sDCC + 4 * kQ;     // U.B partials
+    float* sRowD = sUB + 4 * kQ;    // rowD partials [column quarter][row]
+    float* sColD = sRowD + 4 * kQ;  // colD partials [lane quadrant][column] (without dt)
+    float* tot = sColD + 4 * kQ;    // [8] scan scratch
+
+    if (tid == 0) {
+        *aborted = 0;
+        mbar_init(bar_ld, 1);
+        mbar_init(bar_e0, kEwThreads);
+        mbar_init(bar_p1, 1);
+        mbar_init(bar_e1, kEwThreads);
+        mbar_init(bar_p2, 1);
+        mbar_init(bar_e2, kEwThreads);
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        if (lane == 0) {
+            prefetch_tensormap(&tmX);
+            prefetch_tensormap(&tmB);
+            prefetch_tensormap(&tmC);
+            prefetch_tensormap(&tmDY);
+            prefetch_tensormap(&tmHb);
+            prefetch_tensormap(&tmGb);
+            int issued = 0;
+            for (int hh = 0; hh < hpg; ++hh) {
+                const int h = g * hpg + hh;
+                const int row = ((bi * p.H + h) * p.nc + c) * kN;   // state rows of this (chain, chunk)
+                if (hh > 0 && !mbar_wait_bounded(bar_e2, (uint32_t)(hh - 1) & 1u, kWaitNs, aborted, p.status))
+                    break;
+                mbar_arrive_expect_tx(bar_ld, hh == 0 ? 8 * kTileHalf : 4 * kTileHalf);
+                tma_load_3d(smem + kOffX, &tmX, h * kP, t0, bi, bar_ld);
+                tma_load_3d(smem + kOffDY, &tmDY, h * kP, t0, bi, bar_ld);
+                tma_load_3d(smem + kOffH, &tmHb, 0, row, 0, bar_ld);
+                tma_load_3d(smem + kOffG, &tmGb, 0, row, 0, bar_ld);
+                if (hh == 0) {
+                    tma_load_3d(smem + kOffB, &tmB, g * kN, t0, bi, bar_ld);
+                    tma_load_3d(smem + kOffB + kTileHalf, &tmB, g * kN + 64, t0, bi, bar_ld);
+                    tma_load_3d(smem + kOffC, &tmC, g * kN, t0, bi, bar_ld);
+                    tma_load_3d(smem + kOffC + kTileHalf, &tmC, g * kN + 64, t0, bi, bar_ld);
+                }
+                ++issued;
+            }
+            if (issued > 0) drain_wait(bar_ld, (uint32_t)(issued - 1) & 1u);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------- MMA issue ----------------
+        if (lane == 0) {
+            const uint32_t sB = smem_u32(smem + kOffB), sC = smem_u32(smem + kOffC);
+            const uint32_t sDY = smem_u32(smem + kOffDY), sG = smem_u32(smem + kOffG);
+            const uint32_t sX = smem_u32(smem + kOffX), sH = smem_u32(smem + kOffH);
+            const uint32_t sEDY = smem_u32(smem + kOffEDY), sEX = smem_u32(smem + kOffEX);
+            const uint32_t sM1 = smem_u32(smem + kOffM1), sM2 = smem_u32(smem + kOffM2), sM3 = smem_u32(smem + kOffM3);
+            int committed = 0;
+            for (int hh = 0; hh < hpg; ++hh) {
+                const uint32_t ph = (uint32_t)hh & 1u;
+                if (!mbar_wait_bounded(bar_ld, ph, kWaitNs, aborted, p.status)) break;
+                // the previous head's epilogue has read gB and B g^T (YX's columns)
+                if (hh > 0 && !mbar_wait_bounded(bar_e2, ph ^ 1u, kWaitNs, aborted, p.status)) break;
+                tc_fence_after_sync();
+#pragma unroll
+                for (int k = 0; k < 4; ++k)   // YX = dY X^T (K = P)
+                    umma_bf16(tmem + kColYX, desc_k(sDY, k), desc_k(sX, k), kIdKK128, k > 0);
+                if (hh == 0) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)   // CB = C B^T (K = N)
+                        umma_bf16(tmem + kColCB, desc_k(sC, k), desc_k(sB, k), kIdKK128, k > 0);
+                }
+                if (!mbar_wait_bounded(bar_e0, ph, kWaitNs, aborted, p.status)) break;
+                tc_fence_after_sync();
+#pragma unroll
+                for (int k = 0; k < 4; ++k)   // dC (+)= (Ec o dY) h0   (h0 as [n][p], K = P; summed over heads)
+                    umma_bf16(tmem + kColDC, desc_k(sEDY, k), desc_k(sH, k), kIdKK128, (hh > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)   // U = (El o X) g
+                    umma_bf16(tmem + kColU, desc_k(sEX, k), desc_k(sG, k), kIdKK128, k > 0);
+                umma_commit(bar_p1);
+                ++committed;
+                if (!mbar_wait_bounded(bar_e1, ph, kWaitNs, aborted, p.status)) break;
+                tc_fence_after_sync();
+#pragma unroll
+                for (int k = 0; k < 8; ++k)   // dC += M1 B              (K = Q)
+                    umma_bf16(tmem + kColDC, desc_k(sM1, k), desc_mn(sB, k), kIdKM128, 1u);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)   // U += M2^T C
+                    umma_bf16(tmem + kColU, desc_mn(sM2, k), desc_mn(sC, k), kIdMM128, 1u);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)   // gB = M3^T dY
+                    umma_bf16(tmem + kColGB, desc_mn(sM3, k), desc_mn(sDY, k), kIdMM64, k > 0);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)   // B g^T                    (g as [n][p], K = N)
+                    umma_bf16(tmem + kColBG, desc_k(sB, k), desc_mn(sG, k), kIdKM64, k > 0);
+                umma_commit(bar_p2);
+                ++committed;
+            }
+            if (committed > 0) drain_wait((committed & 1) ? bar_p1 : bar_p2, (uint32_t)((committed - 1) >> 1) & 1u);
+        }
+        __syncwarp();
+    } else {
+        // ---------------- elementwise warps ----------------
+        const int ew = warp - 2;
+        const int quad = warp & 3;           // TMEM lane quadrant: rows 32*quad ..
+        const int qs = ew >> 2;              // column quarter
+        const int i = quad * 32 + lane;      // token row
+        const int t = t0 + i;
+        const bool valid = i < q;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        // dB of the group (this row, 32 columns) summed over its heads; dC's
+        // sum stays in TMEM (its accumulator runs on across the heads), and a
+        // head's dC.C is the difference of consecutive running dots
+        float accdB[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) accdB[k] = 0.0f;
+        float prev_dcc = 0.0f;
+        bool ok = true;
+        for (int hh = 0; hh < hpg; ++hh) {
+            const int h = g * hpg + hh;
+            const int chain = bi * p.H + h;
+            const uint32_t ph = (uint32_t)hh & 1u;
+            const float Ah = p.A[h];
+            const float Dh = p.D ? p.D[h] : 0.0f;
+
+            // E0: dt, cumulative decay (row warps), then the scaled copies.
+            // The barrier also ends the loop of every warp at once after a
+            // give-up (inside a head nobody leaves early, so that every
+            // warp reaches every barrier).
+            if (named_bar_any(kBarEw, kEwThreads, !ok)) {
+                ok = false;
+                break;
+            }
+            if (qs == 0) {
+                float dt, sig;
+                row_dt(p, bi, h, t, valid, dt, sig);
+                const float cum = block_cumsum128(dt * Ah * kLog2e, quad, lane, tot, kBarRows);
+                sCum[i] = cum;
+                sDt[i] = dt;
+                sSig[i] = sig;
+            }
+            named_bar_sync(kBarEw, kEwThreads);
+            const float cum_i = sCum[i], dt_i = sDt[i];
+            const float cl = sCum[kQ - 1];
+            const float Ec = ex2_approx(cum_i), El = ex2_approx(cl - cum_i);
+            ok = mbar_wait_bounded(bar_ld, ph, kWaitNs, aborted, p.status) && ok;
+            {
+                float dd = 0.0f;
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const uint32_t o = sw128(i, qs * 2 + cc);
+                    float y[8], xv[8];
+                    unpack8(*reinterpret_cast<const uint4*>(smem + kOffDY + o), y);
+                    unpack8(*reinterpret_cast<const uint4*>(smem + kOffX + o), xv);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) dd = fmaf(y[k], xv[k], dd);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        y[k] *= Ec;
+                        xv[k] *= El;
+                    }
+                    *reinterpret_cast<uint4*>(smem + kOffEDY + o) = pack8(y);
+                    *reinterpret_cast<uint4*>(smem + kOffEX + o) = pack8(xv);
+                }
+                sDD[qs * kQ + i] = dd;
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(bar_e0);
+
+            // E1: the masked tiles M1, M2, M3 from YX and CB, and W's row partials
+            ok = mbar_wait_bounded(bar_p1, ph, kWaitNs, aborted, p.status) && ok;
+            tc_fence_after_sync();
+            {
+                float w = 0.0f, rowd = 0.0f;
+                const uint32_t half = (uint32_t)(qs >> 1) * kTileHalf;
+#pragma unroll
+                for (int sub = 0; sub < 2; ++sub) {   // 16 columns at a time
+                    float yx[16], cb[16], cold[16];
+                    tmem_ld16(tmem + kColYX + lane_off + (uint32_t)(qs * 32 + sub * 16), yx);
+                    tmem_ld16(tmem + kColCB + lane_off + (uint32_t)(qs * 32 + sub * 16), cb);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        float m1[8], m2[8], m3[8];
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const int jj = cc * 8 + k;
+                            const int j = qs * 32 + sub * 16 + jj;
+                            const float lm = j <= i ? ex2_approx(cum_i - sCum[j]) : 0.0f;
+                            const float v2 = lm * yx[jj];
+                            const float v1 = v2 * sDt[j];
+                            m2[k] = bf16_round(v2);
+                            m1[k] = bf16_round(v1);
+                            m3[k] = lm * cb[jj];
+                            w = fmaf(v1, cb[jj], w);
+                            rowd = fmaf(m1[k] - v1, cb[jj], rowd);
+                            cold[jj] = (v2 - m2[k]) * cb[jj];
+                        }
+                        const uint32_t o = half + sw128(i, (qs & 1) * 4 + sub * 2 + cc);
+                        *reinterpret_cast<uint4*>(smem + kOffM1 + o) = pack8(m1);
+                        *reinterpret_cast<uint4*>(smem + kOffM2 + o) = pack8(m2);
+                        *reinterpret_cast<uint4*>(smem + kOffM3 + o) = pack8(m3);
+                    }
+                    const float cs = warp_colsum16(cold, lane);
+                    if (lane < 16) sColD[quad * kQ + qs * 32 + sub * 16 + lane] = cs;
+                }
+                sRowD[qs * kQ + i] = rowd;
+                sRow[qs * kQ + i] = w;
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            mbar_arrive(bar_e1);
+
+            // E2: dC, dB (summed over heads), dx, and the row dots
+            ok = mbar_wait_bounded(bar_p2, ph, kWaitNs, aborted, p.status) && ok;
+            tc_fence_after_sync();
+            {
+                const uint32_t half = (uint32_t)(qs >> 1) * kTileHalf;
+                float dcc = 0.0f, ub = 0.0f;
+#pragma unroll
+                for (int sub = 0; sub < 2; ++sub) {   // 16 columns at a time
+                    float v[16], u[16];
+                    tmem_ld16(tmem + kColDC + lane_off + (uint32_t)(qs * 32 + sub * 16), v);
+                    tmem_ld16(tmem + kColU + lane_off + (uint32_t)(qs * 32 + sub * 16), u);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const uint32_t o = half + sw128(i, (qs & 1) * 4 + sub * 2 + cc);
+                        float cr[8], br[8];
+                        unpack8(*reinterpret_cast<const uint4*>(smem + kOffC + o), cr);
+                        unpack8(*reinterpret_cast<const uint4*>(smem + kOffB + o), br);
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const int jj = cc * 8 + k;
+                            dcc = fmaf(v[jj], cr[k], dcc);
+                            ub = fmaf(u[jj], br[k], ub);
+                            accdB[sub * 16 + jj] = fmaf(dt_i, u[jj], accdB[sub * 16 + jj]);
+                        }
+                    }
+                }
+                {   // this head's share of the running dot
+                    const float run = dcc;
+                    dcc = run - prev_dcc;
+                    prev_dcc = run;
+                }
+                float gb[16], bg[16];
+                tmem_ld16(tmem + kColGB + lane_off + (uint32_t)(qs * 16), gb);
+                tmem_ld16(tmem + kColBG + lane_off + (uint32_t)(qs * 16), bg);
+                tmem_wait_ld();
+                float dxv[16];
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    float y[8];
+                    unpack8(*reinterpret_cast<const uint4*>(smem + kOffDY + sw128(i, qs * 2 + cc)), y);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        dxv[cc * 8 + k] = fmaf(Dh, y[k], dt_i * fmaf(El, bg[cc * 8 + k], gb[cc * 8 + k]));
+                }
+                if (valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(p.dx + (((size_t)bi * p.L + t) * p.H + h) * kP + qs * 16);
+                    dst[0] = pack8(dxv);
+                    dst[1] = pack8(dxv + 8);
+                }
+                sDCC[qs * kQ + i] = dcc;
+                sUB[qs * kQ + i] = ub;
+            }
+            tc_fence_before_sync();
+            named_bar_sync(kBarEw, kEwThreads);
+
+            // the row warps: per-token scalars, the decay gradient, ddt
+            if (qs == 0) {
+                const float dcc_h = sDCC[i] + sDCC[kQ + i] + sDCC[2 * kQ + i] + sDCC[3 * kQ + i];
+                const float ub = sUB[i] + sUB[kQ + i] + sUB[2 * kQ + i] + sUB[3 * kQ + i];
+                const float wr = sRow[i] + sRow[kQ + i] + sRow[2 * kQ + i] + sRow[3 * kQ + i];
+                const float dd = sDD[i] + sDD[kQ + i] + sDD[2 * kQ + i] + sDD[3 * kQ + i];
+                const float rowd = sRowD[i] + sRowD[kQ + i] + sRowD[2 * kQ + i] + sRowD[3 * kQ + i];
+                const float cold = dt_i * (sColD[i] + sColD[kQ + i] + sColD[2 * kQ + i] + sColD[3 * kQ + i]);
+                const float a = fmaf(dt_i, ub, cold);
+                const float dcc = dcc_h - rowd;
+                // exclusive prefix of a, inclusive suffix of dcc, total of wr
+                const float ia = warp_incl_scan(a, lane);
+                const float idc = warp_incl_scan(dcc, lane);
+                const float tw = warp_total(wr);
+                if (lane == 31) {
+                    tot[quad] = ia;
+                    tot[4 + quad] = idc;
+                }
+                named_bar_sync(kBarRows, 128);
+                float offa = 0.0f, offc = 0.0f, alldc = 0.0f;
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    if (qq < quad) {
+                        offa += tot[qq];
+                        offc += tot[4 + qq];
+                    }
+                    alldc += tot[4 + qq];
+                }
+                // W total: reduce the four warp totals through shared memory
+                named_bar_sync(kBarRows, 128);
+                if (lane == 0) tot[quad] = tw;
+                named_bar_sync(kBarRows, 128);
+                const float wsum = tot[0] + tot[1] + tot[2] + tot[3];
+                const float* t1p = p.ws_t1 + ((size_t)chain * p.nc + c) * kPassSlices;
+                float t1 = 0.0f;
+#pragma unroll
+                for (int s = 0; s < kPassSlices; ++s) t1 += t1p[s];
+                const float pre = offa + ia - a;                  // sum_{j<i} a_j
+                const float suf = alldc - (offc + idc - dcc);     // sum_{k>=i} dcc_k
+                const float r = t1 - wsum + pre + suf;            // (a and dcc carry the rounding terms)
+                float ra = 0.0f, rd = 0.0f, rb = 0.0f;
+                if (valid) {
+                    const float ddt = ub + Ah * r;
+                    const float dv = ddt * sSig[i];
+                    const __nv_bfloat16 dvb = __float2bfloat16_rn(dv);
+                    p.ddt_raw[((size_t)bi * p.L + t) * p.H + h] = dvb;
+                    ra = dt_i * r;
+                    rd = dd;
+                    rb = dv;
+                }
+                ra = warp_total(ra);
+                rd = warp_total(rd);
+                rb = warp_total(rb);
+                if (lane == 0) {
+                    const size_t nparts = (size_t)p.b * p.H * p.nc * kParts;
+                    const size_t o = ((size_t)chain * p.nc + c) * kParts + quad;
+                    p.ws_part[o] = ra;
+                    p.ws_part[nparts + o] = rd;
+                    p.ws_part[2 * nparts + o] = rb;
+                }
+                named_bar_sync(kBarRows, 128);   // tot[] read before the next head's scan
+            }
+            mbar_arrive(bar_e2);
+        }
+        // dB, dC of the group: this thread's row and 32 columns (the last
+        // head's products are complete: its epilogue waited for them)
+        if (ok) {
+            tc_fence_after_sync();
+            float v[32];
+            tmem_ld32(tmem + kColDC + lane_off + (uint32_t)(qs * 32), v);
+            tmem_wait_ld();
+            if (valid) {
+                const size_t o = (((size_t)bi * p.L + t) * p.G + g) * kN + qs * 32;
+                uint4* db = reinterpret_cast<uint4*>(p.dB + o);
+                uint4* dc = reinterpret_cast<uint4*>(p.dC + o);
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    db[cc] = pack8(accdB + cc * 8);
+                    dc[cc] = pack8(v + cc * 8);
+                }
+            }
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// dA, dD, ddt_bias [H]: one CTA per head sums its (sequence, chunk, quarter)
+// partials in a fixed order (thread-strided, then a fixed tree).
+__global__ void __launch_bounds__(256)
+bwd_head_sum_kernel(const float* __restrict__ part, float* __restrict__ dA, float* __restrict__ dD,
+                    float* __restrict__ dbias, int b, int H, int nc)
+{
+    __shared__ float red[3][256];
+    const int h = blockIdx.x, tid = threadIdx.x;
+    const size_t per_chain = (size_t)nc * kParts;
+    const size_t nparts = (size_t)b * H * per_chain;
+    float a = 0.0f, d = 0.0f, s = 0.0f;
+    for (int bi = 0; bi < b; ++bi) {
+        const size_t o = (size_t)(bi * H + h) * per_chain;
+        for (size_t k = tid; k < per_chain; k += 256) {
+            a += part[o + k];
+            d += part[nparts + o + k];
+            s += part[2 * nparts + o + k];
+        }
+    }
+    red[0][tid] = a;
+    red[1][tid] = d;
+    red[2][tid] = s;
+    __syncthreads();
+    for (int w = 128; w > 0; w >>= 1) {
+        if (tid < w) {
+            red[0][tid] += red[0][tid + w];
+            red[1][tid] += red[1][tid + w];
+            red[2][tid] += red[2][tid + w];
+        }
+        __syncthreads();
+    }
+    if (tid == 0) {
+        dA[h] = red[0][0];
+        dD[h] = red[1][0];
+        dbias[h] = red[2][0];
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult qr{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr) != cudaSuccess ||
+            qr != cudaDriverEntryPointSuccess)
+            ptr = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }();
+    return fn;
+}
+
+// 3-D bf16 map: dim0 channels (contiguous), dim1 rows (row_bytes apart),
+// dim2 sequences (rows * row_bytes apart); box 64 x 128 x 1, 128-byte
+// swizzle; rows past the end read as zero.
+cudaError_t map3d(CUtensorMap* m, const void* base, uint64_t channels, uint64_t rows, uint64_t seqs,
+                  uint64_t row_bytes)
+{
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[3] = {channels, rows, seqs};
+    const cuuint64_t strides[2] = {row_bytes, row_bytes * rows};
+    const cuuint32_t box[3] = {64, (cuuint32_t)kQ, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+size_t al256(size_t n) { return (n + 255) / 256 * 256; }
+
+struct TcWs {
+    size_t ctrl, S, dS, hb, gb, cl, t1, part, total;
+};
+
+TcWs tc_ws_layout(int b, int L, int H)
+{
+    const size_t chains = (size_t)b * H;
+    const size_t nc = (size_t)(L + kQ - 1) / kQ;
+    TcWs w{};
+    size_t o = 0;
+    w.ctrl = o;
+    o += 256;
+    w.S = o;
+    o += al256(chains * nc * kStatesDim * 4);
+    w.dS = o;
+    o += al256(chains * nc * kStatesDim * 4);
+    w.hb = o;
+    o += al256(chains * nc * kStatesDim * 2);
+    w.gb = o;
+    o += al256(chains * nc * kStatesDim * 2);
+    w.cl = o;
+    o += al256(chains * nc * 4);
+    w.t1 = o;
+    o += al256(chains * nc * kPassSlices * 4);
+    w.part = o;
+    o += al256(3 * chains * nc * kParts * 4);
+    w.total = o;
+    return w;
+}
+
+bool a16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
+
+}  // namespace
+
+bool scan_bwd_tc_shape(int P, int N, bool bf16) { return bf16 && P == kP && N == kN; }
+
+bool scan_bwd_tc_supported(const ScanBwdArgs& a)
+{
+    return scan_bwd_tc_shape(a.P, a.N, a.bf16) && a.b > 0 && a.L > 0 && (int64_t)a.b * a.G < 65536 &&
+           a.row_stride % 8 == 0 && a16(a.x) &&
+           a16(a.B) && a16(a.C) && a16(a.dy) && a16(a.dx) && a16(a.dB) && a16(a.dC) && a16(a.workspace) &&
+           (size_t)a.b * a.H * ((a.L + kQ - 1) / kQ) * kN < 0x7fffffffULL;
+}
+
+size_t scan_bwd_tc_workspace_bytes(int b, int L, int H)
+{
+    if (b <= 0 || L <= 0) return 0;
+    return tc_ws_layout(b, L, H).total;
+}
+
+cudaError_t launch_scan_bwd_tc(const ScanBwdArgs& a, cudaStream_t s)
+{
+    const int nc = (a.L + kQ - 1) / kQ;
+    const TcWs w = tc_ws_layout(a.b, a.L, a.H);
+    uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+    TcParams p{};
+    p.dt_raw = static_cast<const __nv_bfloat16*>(a.dt_raw);
+    p.dt_bias = a.dt_bias;
+    p.A = a.A;
+    p.D = a.D;
+    p.init_state = a.init_state;
+    p.dfinal = a.dfinal;
+    p.dx = static_cast<__nv_bfloat16*>(a.dx);
+    p.dB = static_cast<__nv_bfloat16*>(a.dB);
+    p.dC = static_cast<__nv_bfloat16*>(a.dC);
+    p.ddt_raw = static_cast<__nv_bfloat16*>(a.ddt_raw);
+    p.dA = a.dA;
+    p.dD = a.dD;
+    p.ddt_bias = a.ddt_bias;
+    p.dinit = a.dinit;
+    p.status = reinterpret_cast<int32_t*>(ws + w.ctrl);
+    p.ws_S = reinterpret_cast<float*>(ws + w.S);
+    p.ws_dS = reinterpret_cast<float*>(ws + w.dS);
+    p.ws_hb = reinterpret_cast<__nv_bfloat16*>(ws + w.hb);
+    p.ws_gb = reinterpret_cast<__nv_bfloat16*>(ws + w.gb);
+    p.ws_cl = reinterpret_cast<float*>(ws + w.cl);
+    p.ws_t1 = reinterpret_cast<float*>(ws + w.t1);
+    p.ws_part = reinterpret_cast<float*>(ws + w.part);
+    p.b = a.b;
+    p.L = a.L;
+    p.H = a.H;
+    p.G = a.G;
+    p.nc = nc;
+
+    const uint64_t rb = (uint64_t)a.row_stride * 2;
+    const uint64_t state_rows = (uint64_t)a.b * a.H * nc * kN;
+    CUtensorMap tmX, tmB, tmC, tmDY, tmHb, tmGb;
+    cudaError_t e;
+    if ((e = map3d(&tmX, a.x, (uint64_t)a.H * kP, a.L, a.b, rb)) != cudaSuccess) return e;
+    if ((e = map3d(&tmB, a.B, (uint64_t)a.G * kN, a.L, a.b, rb)) != cudaSuccess) return e;
+    if ((e = map3d(&tmC, a.C, (uint64_t)a.G * kN, a.L, a.b, rb)) != cudaSuccess) return e;
+    if ((e = map3d(&tmDY, a.dy, (uint64_t)a.H * kP, a.L, a.b, (uint64_t)a.H * kP * 2)) != cudaSuccess) return e;
+    if ((e = map3d(&tmHb, p.ws_hb, kP, state_rows, 1, kP * 2)) != cudaSuccess) return e;
+    if ((e = map3d(&tmGb, p.ws_gb, kP, state_rows, 1, kP * 2)) != cudaSuccess) return e;
+
+    if ((e = cudaMemsetAsync(p.status, 0, 4, s)) != cudaSuccess) return e;
+    const dim3 grid((unsigned)nc, (unsigned)(a.b * a.G));
+    if ((e = cudaFuncSetAttribute(bwd_states_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, k1::kSmemBytes)) !=
+        cudaSuccess)
+        return e;
+    bwd_states_kernel<<<grid, k1::kThreads, k1::kSmemBytes, s>>>(tmX, tmB, tmC, tmDY, p);
+    bwd_pass_kernel<<<dim3((unsigned)(a.b * a.H), kPassSlices), kPassThreads, 0, s>>>(p);
+    if ((e = cudaFuncSetAttribute(bwd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, k3::kSmemBytes)) !=
+        cudaSuccess)
+        return e;
+    bwd_chunk_kernel<<<grid, k3::kThreads, k3::kSmemBytes, s>>>(tmX, tmB, tmC, tmDY, tmHb, tmGb, p);
+    bwd_head_sum_kernel<<<a.H, 256, 0, s>>>(p.ws_part, a.dA, a.dD, a.ddt_bias, a.b, a.H, nc);
+    return cudaGetLastError();
+}
+
+}  // namespace ssd
