@@ -15,16 +15,18 @@
 //      S^T  = B^T (w o X),  w_j = El_j dt_j      the chunk's own end state
 //      dS^T = C^T (Ec o dY)                     its part of the entering
 //                                               state's gradient
-// 2. bwd_pass_kernel (CUDA cores), per (sequence, head), chunk after chunk:
-//      h0_{c+1} = 2^cl_c h0_c + S_c,   g_{c-1} = 2^cl_c g_c + dS_c,
-//      t1_c = 2^cl_c <g_c, h0_c>;   the initial state's gradient is g_{-1}.
+// 2. bwd_pass_kernel (CUDA cores), per (sequence, head), chunk after chunk,
+//    the two directions independently (fp32 sums of bf16 S and dS):
+//      h0_{c+1} = 2^cl_c h0_c + S_c,   g_{c-1} = 2^cl_c g_c + dS_c;
+//    the initial state's gradient is g_{-1}.
 // 3. bwd_chunk_kernel (tensor cores), per chunk and head:
 //      YX = dY X^T,  CB = C B^T                              (Q x Q)
 //      M1 = Lm o dt_j o YX,  M2 = Lm o YX,  M3 = Lm o CB      (bf16 tiles)
 //      dC = (Ec o dY) h0 + M1 B                              (Q x N)
 //      U  = (El o X) g + M2^T C,    dB = dt o U               (Q x N)
 //      gB = El o (B g^T) + M3^T dY, dx = D dy + dt o gB       (Q x P)
-//    The decay gradient r_t = <g_t, exp(dt_t A) h_{t-1}> has a closed form
+//    With t1 = 2^cl <g, h0> (from the bf16 tiles of h0 and g),
+//    the decay gradient r_t = <g_t, exp(dt_t A) h_{t-1}> has a closed form
 //    in the tiles' row sums (U.B = El x^T g B + sum_k M2 CB and
 //    dC.C = Ec dy^T h0 C + W, W_k = sum_j M1[k][j] CB[k][j]):
 //      r_t = t1 - sum_k W_k + sum_{j<t} dt_j U_j.B_j + sum_{k>=t} dC_k.C_k,
@@ -64,7 +66,7 @@ constexpr int kQ = 128, kP = 64, kN = 128;
 constexpr uint32_t kTileHalf = 16384;        // 128 rows x 64 bf16, swizzled
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kPassSlices = 8;               // CTAs per chain in the passing kernel
+constexpr int kPassSlices = 8;               // CTAs per chain and direction in the passing kernel
 constexpr int kPassThreads = 256;            // 4 state elements per thread
 constexpr int kParts = 4;                    // dA / dD / ddt_bias partials per (chain, chunk)
 
@@ -171,6 +173,7 @@ __device__ inline float warp_total(float v)
 
 struct TcParams {
     const __nv_bfloat16* dt_raw;   // [b][L][H]
+    const __nv_bfloat16* dy;       // [b][L][H][P]
     const float* dt_bias;
     const float* A;
     const float* D;
@@ -185,12 +188,11 @@ struct TcParams {
     float* ddt_bias;
     float* dinit;                  // [b][H][P][N]
     int32_t* status;               // workspace word 0: timeout flag
-    float* ws_S;                   // [chains][nc][N][P] fp32: S, then h0
-    float* ws_dS;                  // [chains][nc][N][P] fp32
+    __nv_bfloat16* ws_S;           // [chains][nc][N][P] bf16 S
+    __nv_bfloat16* ws_dS;          // [chains][nc][N][P] bf16 dS
     __nv_bfloat16* ws_hb;          // [chains][nc][N][P] bf16 h0
     __nv_bfloat16* ws_gb;          // [chains][nc][N][P] bf16 g
     float* ws_cl;                  // [chains][nc]
-    float* ws_t1;                  // [chains][nc][kPassSlices]
     float* ws_part;                // [3][chains][nc][kParts]
     int b, L, H, G, nc;
 };
@@ -356,22 +358,20 @@ bwd_states_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             mbar_arrive(bar_w);
             ok = mbar_wait_bounded(bar_mma, ph, kWaitNs, aborted, p.status) && ok;
             tc_fence_after_sync();
-            // state row n = i: S^T[n][0..63], dS^T[n][0..63]
-            float* dS = p.ws_S + ((size_t)chain * p.nc + c) * kStatesDim + (size_t)i * kP;
-            float* ddS = p.ws_dS + ((size_t)chain * p.nc + c) * kStatesDim + (size_t)i * kP;
+            // state row n = i: S^T[n][0..63], dS^T[n][0..63], in bf16
+            uint4* dS = reinterpret_cast<uint4*>(p.ws_S + ((size_t)chain * p.nc + c) * kStatesDim + (size_t)i * kP);
+            uint4* ddS = reinterpret_cast<uint4*>(p.ws_dS + ((size_t)chain * p.nc + c) * kStatesDim + (size_t)i * kP);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                float v[32];
+                float v[32], u[32];
                 tmem_ld32(tmem + lane_off + (uint32_t)(half * 32), v);
+                tmem_ld32(tmem + lane_off + 64u + (uint32_t)(half * 32), u);
                 tmem_wait_ld();
 #pragma unroll
-                for (int k = 0; k < 32; k += 4)
-                    *reinterpret_cast<float4*>(dS + half * 32 + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
-                tmem_ld32(tmem + lane_off + 64u + (uint32_t)(half * 32), v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int k = 0; k < 32; k += 4)
-                    *reinterpret_cast<float4*>(ddS + half * 32 + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+                for (int k = 0; k < 4; ++k) {
+                    dS[half * 4 + k] = pack8(v + 8 * k);
+                    ddS[half * 4 + k] = pack8(u + 8 * k);
+                }
             }
             tc_fence_before_sync();
         }
@@ -387,72 +387,55 @@ bwd_states_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 // ---------------------------------------------------------------------------
 // Kernel 2: entering states forward, state gradients backward
 // ---------------------------------------------------------------------------
-// Grid (chains, kPassSlices); thread j of slice s owns state elements
-// e = s*1024 + 4j .. +3 of the [n][p] layout (one n, four p).
+// Grid (chains, kPassSlices, 2): thread j of slice s owns state elements
+// e = s*1024 + 4j .. +3 of the [n][p] layout (one n, four p); z = 0 walks
+// the entering states forward, z = 1 the state gradients backward.
+__device__ inline void ld_bf16x4(const __nv_bfloat16* src, float (&v)[4])
+{
+    const uint2 q = *reinterpret_cast<const uint2*>(src);
+    v[0] = __uint_as_float(q.x << 16);
+    v[1] = __uint_as_float(q.x & 0xffff0000u);
+    v[2] = __uint_as_float(q.y << 16);
+    v[3] = __uint_as_float(q.y & 0xffff0000u);
+}
+
+__device__ inline void st_bf16x4(__nv_bfloat16* dst, const float (&v)[4])
+{
+    __nv_bfloat162 lo = __floats2bfloat162_rn(v[0], v[1]), hi = __floats2bfloat162_rn(v[2], v[3]);
+    *reinterpret_cast<uint2*>(dst) = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+}
+
 __global__ void __launch_bounds__(kPassThreads)
 bwd_pass_kernel(const TcParams p)
 {
-    __shared__ float red[kPassThreads / 32];
     const int chain = blockIdx.x, s = blockIdx.y;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int e0 = s * (kStatesDim / kPassSlices) + tid * 4;
+    const bool fwd = blockIdx.z == 0;
+    const int e0 = s * (kStatesDim / kPassSlices) + threadIdx.x * 4;
     const int n = e0 / kP, p0 = e0 - n * kP;
     const int nc = p.nc;
     const size_t base = (size_t)chain * nc * kStatesDim + e0;
     const float* cl = p.ws_cl + (size_t)chain * nc;
-
-    // forward: h0 of every chunk (fp32 in place of S, bf16 copy)
-    float h[4];
+    const float* start = fwd ? p.init_state : p.dfinal;
+    const __nv_bfloat16* inc = fwd ? p.ws_S : p.ws_dS;
+    __nv_bfloat16* out = fwd ? p.ws_hb : p.ws_gb;
+    float v[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-        h[k] = p.init_state ? p.init_state[(size_t)chain * kStatesDim + (size_t)(p0 + k) * kN + n] : 0.0f;
-    float4 Snext = *reinterpret_cast<const float4*>(p.ws_S + base);
-    for (int c = 0; c < nc; ++c) {
-        const float4 S = Snext;
-        if (c + 1 < nc) Snext = *reinterpret_cast<const float4*>(p.ws_S + base + (size_t)(c + 1) * kStatesDim);
+    for (int k = 0; k < 4; ++k) v[k] = start ? start[(size_t)chain * kStatesDim + (size_t)(p0 + k) * kN + n] : 0.0f;
+    // forward: out[c] = h0_c, h0_{c+1} = 2^cl_c h0_c + S_c;
+    // backward: out[c] = g_c, g_{c-1} = 2^cl_c g_c + dS_c
+    for (int k = 0; k < nc; ++k) {
+        const int c = fwd ? k : nc - 1 - k;
         const size_t o = base + (size_t)c * kStatesDim;
-        *reinterpret_cast<float4*>(p.ws_S + o) = make_float4(h[0], h[1], h[2], h[3]);
-        __nv_bfloat162 lo = __floats2bfloat162_rn(h[0], h[1]), hi = __floats2bfloat162_rn(h[2], h[3]);
-        *reinterpret_cast<uint2*>(p.ws_hb + o) =
-            make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+        float a[4];
+        ld_bf16x4(inc + o, a);
+        st_bf16x4(out + o, v);
         const float d = ex2_approx(cl[c]);
-        h[0] = d * h[0] + S.x;
-        h[1] = d * h[1] + S.y;
-        h[2] = d * h[2] + S.z;
-        h[3] = d * h[3] + S.w;
-    }
-
-    // backward: g at the end of every chunk (bf16), t1 partials, dinit
-    float gv[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-        gv[k] = p.dfinal ? p.dfinal[(size_t)chain * kStatesDim + (size_t)(p0 + k) * kN + n] : 0.0f;
-    for (int c = nc - 1; c >= 0; --c) {
-        const size_t o = base + (size_t)c * kStatesDim;
-        const float4 h0 = *reinterpret_cast<const float4*>(p.ws_S + o);
-        const float4 dS = *reinterpret_cast<const float4*>(p.ws_dS + o);
-        __nv_bfloat162 lo = __floats2bfloat162_rn(gv[0], gv[1]), hi = __floats2bfloat162_rn(gv[2], gv[3]);
-        *reinterpret_cast<uint2*>(p.ws_gb + o) =
-            make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
-        const float d = ex2_approx(cl[c]);
-        float part = gv[0] * h0.x + gv[1] * h0.y + gv[2] * h0.z + gv[3] * h0.w;
-        part = warp_total(part);
-        if (lane == 0) red[warp] = part;
-        __syncthreads();
-        if (tid == 0) {
-            float t = 0.0f;
-            for (int w = 0; w < kPassThreads / 32; ++w) t += red[w];
-            p.ws_t1[((size_t)chain * nc + c) * kPassSlices + s] = d * t;
-        }
-        __syncthreads();
-        gv[0] = d * gv[0] + dS.x;
-        gv[1] = d * gv[1] + dS.y;
-        gv[2] = d * gv[2] + dS.z;
-        gv[3] = d * gv[3] + dS.w;
+        for (int e = 0; e < 4; ++e) v[e] = fmaf(d, v[e], a[e]);
     }
-    if (p.dinit) {
+    if (!fwd && p.dinit) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) p.dinit[(size_t)chain * kStatesDim + (size_t)(p0 + k) * kN + n] = gv[k];
+        for (int k = 0; k < 4; ++k) p.dinit[(size_t)chain * kStatesDim + (size_t)(p0 + k) * kN + n] = v[k];
     }
 }
 
@@ -468,8 +451,8 @@ constexpr int kThreads = kEwThreads + 64;       // warp 0 producer, 1 MMA, 2..17
 constexpr int kOffB = 0, kOffC = 32768, kOffDY = 65536, kOffG = 81920, kOffR = 98304;
 constexpr int kOffX = kOffR, kOffH = kOffR + 16384, kOffEDY = kOffR + 32768, kOffEX = kOffR + 49152;
 constexpr int kOffM1 = kOffR, kOffM2 = kOffR + 32768, kOffM3 = kOffR + 65536;
-constexpr int kOffVec = kOffR + 98304;          // floats: cum, dt, sig [128] each, partials [6][4][128], tot [8]
-constexpr int kVecFloats = 3 * kQ + 24 * kQ + 8;
+constexpr int kOffVec = kOffR + 98304;          // floats: cum, dt, sig [128] each, partials [6][4][128], tot [8], t1 [16]
+constexpr int kVecFloats = 3 * kQ + 24 * kQ + 8 + 16;
 constexpr int kOffBar = kOffVec + ((kVecFloats * 4 + 63) / 64) * 64;
 constexpr int kNumBars = 6;
 constexpr int kOffMisc = kOffBar + 8 * kNumBars;
@@ -522,6 +505,7 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     float* sRowD = sUB + 4 * kQ;    // rowD partials [column quarter][row]
     float* sColD = sRowD + 4 * kQ;  // colD partials [lane quadrant][column] (without dt)
     float* tot = sColD + 4 * kQ;    // [8] scan scratch
+    float* sT1 = tot + 8;           // [16] <g, h0> partials, one per elementwise warp
 
     if (tid == 0) {
         *aborted = 0;
@@ -552,7 +536,9 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             for (int hh = 0; hh < hpg; ++hh) {
                 const int h = g * hpg + hh;
                 const int row = ((bi * p.H + h) * p.nc + c) * kN;   // state rows of this (chain, chunk)
-                if (hh > 0 && !mbar_wait_bounded(bar_e2, (uint32_t)(hh - 1) & 1u, kWaitNs, aborted, p.status))
+                // the previous head's products are done: X, h0, dY, g and the
+                // M tiles are free (its epilogue reads dy from global memory)
+                if (hh > 0 && !mbar_wait_bounded(bar_p2, (uint32_t)(hh - 1) & 1u, kWaitNs, aborted, p.status))
                     break;
                 mbar_arrive_expect_tx(bar_ld, hh == 0 ? 8 * kTileHalf : 4 * kTileHalf);
                 tma_load_3d(smem + kOffX, &tmX, h * kP, t0, bi, bar_ld);
@@ -687,6 +673,19 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     *reinterpret_cast<uint4*>(smem + kOffEX + o) = pack8(xv);
                 }
                 sDD[qs * kQ + i] = dd;
+                // <g, h0> over the two bf16 tiles (same layout): 2 chunks per thread
+                float gh = 0.0f;
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const uint32_t o = (uint32_t)((ew * 32 + lane) * 2 + cc) * 16u;
+                    float hv[8], gv[8];
+                    unpack8(*reinterpret_cast<const uint4*>(smem + kOffH + o), hv);
+                    unpack8(*reinterpret_cast<const uint4*>(smem + kOffG + o), gv);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) gh = fmaf(hv[k], gv[k], gh);
+                }
+                gh = warp_total(gh);
+                if (lane == 0) sT1[ew] = gh;
             }
             fence_proxy_async_smem();
             mbar_arrive(bar_e0);
@@ -772,10 +771,12 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 tmem_ld16(tmem + kColBG + lane_off + (uint32_t)(qs * 16), bg);
                 tmem_wait_ld();
                 float dxv[16];
+                const uint4* dyr = reinterpret_cast<const uint4*>(p.dy + (((size_t)bi * p.L + min(t, p.L - 1)) * p.H + h) * kP +
+                                                                  qs * 16);
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     float y[8];
-                    unpack8(*reinterpret_cast<const uint4*>(smem + kOffDY + sw128(i, qs * 2 + cc)), y);
+                    unpack8(dyr[cc], y);
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
                         dxv[cc * 8 + k] = fmaf(Dh, y[k], dt_i * fmaf(El, bg[cc * 8 + k], gb[cc * 8 + k]));
@@ -824,10 +825,10 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 if (lane == 0) tot[quad] = tw;
                 named_bar_sync(kBarRows, 128);
                 const float wsum = tot[0] + tot[1] + tot[2] + tot[3];
-                const float* t1p = p.ws_t1 + ((size_t)chain * p.nc + c) * kPassSlices;
                 float t1 = 0.0f;
 #pragma unroll
-                for (int s = 0; s < kPassSlices; ++s) t1 += t1p[s];
+                for (int w2 = 0; w2 < kEwWarps; ++w2) t1 += sT1[w2];
+                t1 *= ex2_approx(sCum[kQ - 1]);
                 const float pre = offa + ia - a;                  // sum_{j<i} a_j
                 const float suf = alldc - (offc + idc - dcc);     // sum_{k>=i} dcc_k
                 const float r = t1 - wsum + pre + suf;            // (a and dcc carry the rounding terms)
@@ -954,7 +955,7 @@ cudaError_t map3d(CUtensorMap* m, const void* base, uint64_t channels, uint64_t 
 size_t al256(size_t n) { return (n + 255) / 256 * 256; }
 
 struct TcWs {
-    size_t ctrl, S, dS, hb, gb, cl, t1, part, total;
+    size_t ctrl, S, dS, hb, gb, cl, part, total;
 };
 
 TcWs tc_ws_layout(int b, int L, int H)
@@ -966,17 +967,15 @@ TcWs tc_ws_layout(int b, int L, int H)
     w.ctrl = o;
     o += 256;
     w.S = o;
-    o += al256(chains * nc * kStatesDim * 4);
+    o += al256(chains * nc * kStatesDim * 2);
     w.dS = o;
-    o += al256(chains * nc * kStatesDim * 4);
+    o += al256(chains * nc * kStatesDim * 2);
     w.hb = o;
     o += al256(chains * nc * kStatesDim * 2);
     w.gb = o;
     o += al256(chains * nc * kStatesDim * 2);
     w.cl = o;
     o += al256(chains * nc * 4);
-    w.t1 = o;
-    o += al256(chains * nc * kPassSlices * 4);
     w.part = o;
     o += al256(3 * chains * nc * kParts * 4);
     w.total = o;
@@ -1010,6 +1009,7 @@ cudaError_t launch_scan_bwd_tc(const ScanBwdArgs& a, cudaStream_t s)
     uint8_t* ws = static_cast<uint8_t*>(a.workspace);
     TcParams p{};
     p.dt_raw = static_cast<const __nv_bfloat16*>(a.dt_raw);
+    p.dy = static_cast<const __nv_bfloat16*>(a.dy);
     p.dt_bias = a.dt_bias;
     p.A = a.A;
     p.D = a.D;
@@ -1024,12 +1024,11 @@ cudaError_t launch_scan_bwd_tc(const ScanBwdArgs& a, cudaStream_t s)
     p.ddt_bias = a.ddt_bias;
     p.dinit = a.dinit;
     p.status = reinterpret_cast<int32_t*>(ws + w.ctrl);
-    p.ws_S = reinterpret_cast<float*>(ws + w.S);
-    p.ws_dS = reinterpret_cast<float*>(ws + w.dS);
+    p.ws_S = reinterpret_cast<__nv_bfloat16*>(ws + w.S);
+    p.ws_dS = reinterpret_cast<__nv_bfloat16*>(ws + w.dS);
     p.ws_hb = reinterpret_cast<__nv_bfloat16*>(ws + w.hb);
     p.ws_gb = reinterpret_cast<__nv_bfloat16*>(ws + w.gb);
     p.ws_cl = reinterpret_cast<float*>(ws + w.cl);
-    p.ws_t1 = reinterpret_cast<float*>(ws + w.t1);
     p.ws_part = reinterpret_cast<float*>(ws + w.part);
     p.b = a.b;
     p.L = a.L;
@@ -1054,7 +1053,7 @@ cudaError_t launch_scan_bwd_tc(const ScanBwdArgs& a, cudaStream_t s)
         cudaSuccess)
         return e;
     bwd_states_kernel<<<grid, k1::kThreads, k1::kSmemBytes, s>>>(tmX, tmB, tmC, tmDY, p);
-    bwd_pass_kernel<<<dim3((unsigned)(a.b * a.H), kPassSlices), kPassThreads, 0, s>>>(p);
+    bwd_pass_kernel<<<dim3((unsigned)(a.b * a.H), kPassSlices, 2), kPassThreads, 0, s>>>(p);
     if ((e = cudaFuncSetAttribute(bwd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, k3::kSmemBytes)) !=
         cudaSuccess)
         return e;
