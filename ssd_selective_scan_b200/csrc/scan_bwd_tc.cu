@@ -21,24 +21,23 @@
 //    the initial state's gradient is g_{-1}.
 // 3. bwd_chunk_kernel (tensor cores), per chunk and head:
 //      YX = dY X^T,  CB = C B^T                              (Q x Q)
-//      M1 = Lm o dt_j o YX,  M2 = Lm o YX,  M3 = Lm o CB      (bf16 tiles)
+//      M2 = Lm o YX,  M1 = dt_j o M2,  M3 = Lm o CB           (M1, M3 bf16 tiles)
 //      dC = (Ec o dY) h0 + M1 B                              (Q x N)
-//      U  = (El o X) g + M2^T C,    dB = dt o U               (Q x N)
+//      dB = dt o U = (dt o El o X) g + M1^T C                (Q x N)
 //      gB = El o (B g^T) + M3^T dY, dx = D dy + dt o gB       (Q x P)
-//    With t1 = 2^cl <g, h0> (from the bf16 tiles of h0 and g),
-//    the decay gradient r_t = <g_t, exp(dt_t A) h_{t-1}> has a closed form
-//    in the tiles' row sums (U.B = El x^T g B + sum_k M2 CB and
-//    dC.C = Ec dy^T h0 C + W, W_k = sum_j M1[k][j] CB[k][j]):
-//      r_t = t1 - sum_k W_k + sum_{j<t} dt_j U_j.B_j + sum_{k>=t} dC_k.C_k,
+//    and, in fp32, U_j.B_j = El_j x_j.(B g^T)_j + sum_k M2[k][j] CB[k][j].
+//    With t1 = 2^cl <g, h0> (from the bf16 tiles of h0 and g), the decay
+//    gradient r_t = <g_t, exp(dt_t A) h_{t-1}> has a closed form in the
+//    tiles' sums (dt_j U_j.B_j = dt_j El_j x_j^T g B_j + sum_k W[k][j] and
+//    dC_k.C_k = Ec_k dy_k^T h0 C_k + sum_j W[k][j], W = M1 o CB):
+//      r_t = t1 - sum W + sum_{j<t} dt_j U_j.B_j + sum_{k>=t} dC_k.C_k,
 //    then ddt = U.B + A r, ddt_raw = ddt sigmoid(dt_raw + dt_bias),
-//    dA = sum dt r, dD = sum dy.x, ddt_bias = sum ddt_raw.  The products
-//    take M1 and M2 rounded to bf16 while W is summed in fp32, so the
-//    rounding is compensated exactly: r_t gains sum_{j<t} colD_j -
-//    sum_{k>=t} rowD_k, rowD_k = sum_j (bf16(M1) - M1)[k][j] CB[k][j],
-//    colD_j = dt_j sum_k (M2 - bf16(M2))[k][j] CB[k][j].  (Without it the
-//    large sums of the closed form amplify the bf16 rounding of the tiles.)
+//    dA = sum dt r, dD = sum dy.x, ddt_bias = sum ddt_raw.  dC takes M1
+//    rounded to bf16 while W is summed in fp32, so that rounding is taken
+//    out exactly: dC_k.C_k - sum_j (bf16(M1) - M1)[k][j] CB[k][j].  (Without
+//    it the large sums of the closed form amplify the rounding.)
 // dB and dC of a group are sums over its heads: one CTA takes the heads of a
-// group in order and keeps the sums in registers.  dA, dD and ddt_bias are
+// group in order and its accumulators run on across them in TMEM.  dA, dD and ddt_bias are
 // summed over sequences, chunks and row quarters in a fixed order by a last
 // kernel, so the result is deterministic.
 //
@@ -174,6 +173,8 @@ __device__ inline float warp_total(float v)
 struct TcParams {
     const __nv_bfloat16* dt_raw;   // [b][L][H]
     const __nv_bfloat16* dy;       // [b][L][H][P]
+    const __nv_bfloat16* x;        // token rows row_stride apart
+    int64_t row_stride;
     const float* dt_bias;
     const float* A;
     const float* D;
@@ -446,12 +447,12 @@ namespace k3 {
 constexpr int kEwWarps = 16;                    // 4 lane quadrants x 4 column quarters
 constexpr int kEwThreads = kEwWarps * 32;
 constexpr int kThreads = kEwThreads + 64;       // warp 0 producer, 1 MMA, 2..17 elementwise
-// shared memory (1024-aligned); region R holds X, h0, Ec o dY, El o X in
-// the first phase and the tiles M1, M2, M3 in the second
+// shared memory (1024-aligned); region R holds X, h0, Ec o dY, dt o El o X
+// in the first phase and the tiles M1, M3 in the second
 constexpr int kOffB = 0, kOffC = 32768, kOffDY = 65536, kOffG = 81920, kOffR = 98304;
 constexpr int kOffX = kOffR, kOffH = kOffR + 16384, kOffEDY = kOffR + 32768, kOffEX = kOffR + 49152;
-constexpr int kOffM1 = kOffR, kOffM2 = kOffR + 32768, kOffM3 = kOffR + 65536;
-constexpr int kOffVec = kOffR + 98304;          // floats: cum, dt, sig [128] each, partials [6][4][128], tot [8], t1 [16]
+constexpr int kOffM1 = kOffR, kOffM3 = kOffR + 32768;
+constexpr int kOffVec = kOffR + 65536;          // floats: cum, dt, sig [128] each, partials [6][4][128], tot [8], t1 [16]
 constexpr int kVecFloats = 3 * kQ + 24 * kQ + 8 + 16;
 constexpr int kOffBar = kOffVec + ((kVecFloats * 4 + 63) / 64) * 64;
 constexpr int kNumBars = 6;
@@ -462,8 +463,8 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColYX = 0;     // YX [0,128); after the tiles are built: gB [0,64), B g^T [64,128)
 constexpr uint32_t kColGB = 0, kColBG = 64;
 constexpr uint32_t kColCB = 128;   // CB (kept across the group's heads)
-constexpr uint32_t kColDC = 256;   // dC
-constexpr uint32_t kColU = 384;    // U
+constexpr uint32_t kColDC = 256;   // dC, summed over the group's heads
+constexpr uint32_t kColDB = 384;   // dB, summed over the group's heads
 constexpr uint32_t kIdKK128 = umma_idesc_bf16(128, 128, false, false);
 constexpr uint32_t kIdKM128 = umma_idesc_bf16(128, 128, false, true);
 constexpr uint32_t kIdMM128 = umma_idesc_bf16(128, 128, true, true);
@@ -488,23 +489,23 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     const int q = min(kQ, p.L - t0);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
     uint64_t* bar_ld = bars + 0;   // X, dY, h0, g (and B, C for the first head) landed
-    uint64_t* bar_e0 = bars + 1;   // Ec o dY, El o X written
-    uint64_t* bar_p1 = bars + 2;   // YX, CB, dC and U's first products done
-    uint64_t* bar_e1 = bars + 3;   // M1, M2, M3 written; YX read
-    uint64_t* bar_p2 = bars + 4;   // dC, U, gB, B g^T done
-    uint64_t* bar_e2 = bars + 5;   // the head's epilogue done (dY, g, M tiles free)
+    uint64_t* bar_e0 = bars + 1;   // Ec o dY, dt o El o X written
+    uint64_t* bar_p1 = bars + 2;   // YX, CB and the first products of dC, dB done
+    uint64_t* bar_e1 = bars + 3;   // M1, M3 written; YX read
+    uint64_t* bar_p2 = bars + 4;   // dC, dB, gB, B g^T done
+    uint64_t* bar_e2 = bars + 5;   // the head's epilogue has read gB, B g^T and dC
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* aborted = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
     float* sCum = reinterpret_cast<float*>(smem + kOffVec);
     float* sDt = sCum + kQ;
     float* sSig = sDt + kQ;
-    float* sRow = sSig + kQ;        // [4 quarters][128]: W partials
-    float* sDD = sRow + 4 * kQ;     // dy.x partials
+    float* sRow = sSig + kQ;        // [column quarter][row]: W partials
+    float* sRowD = sRow + 4 * kQ;   // rowD partials
+    float* sDD = sRowD + 4 * kQ;    // dy.x partials
     float* sDCC = sDD + 4 * kQ;     // dC.C partials
-    float* sUB = sDCC + 4 * kQ;     // U.B partials
-    float* sRowD = sUB + 4 * kQ;    // rowD partials [column quarter][row]
-    float* sColD = sRowD + 4 * kQ;  // colD partials [lane quadrant][column] (without dt)
-    float* tot = sColD + 4 * kQ;    // [8] scan scratch
+    float* sXGB = sDCC + 4 * kQ;    // x^T g B partials
+    float* sCol = sXGB + 4 * kQ;    // [lane quadrant][column]: sum_k M2 CB partials
+    float* tot = sCol + 4 * kQ;     // [8] scan scratch
     float* sT1 = tot + 8;           // [16] <g, h0> partials, one per elementwise warp
 
     if (tid == 0) {
@@ -537,7 +538,7 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 const int h = g * hpg + hh;
                 const int row = ((bi * p.H + h) * p.nc + c) * kN;   // state rows of this (chain, chunk)
                 // the previous head's products are done: X, h0, dY, g and the
-                // M tiles are free (its epilogue reads dy from global memory)
+                // M tiles are free (its epilogue reads x and dy from global memory)
                 if (hh > 0 && !mbar_wait_bounded(bar_p2, (uint32_t)(hh - 1) & 1u, kWaitNs, aborted, p.status))
                     break;
                 mbar_arrive_expect_tx(bar_ld, hh == 0 ? 8 * kTileHalf : 4 * kTileHalf);
@@ -563,12 +564,13 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             const uint32_t sDY = smem_u32(smem + kOffDY), sG = smem_u32(smem + kOffG);
             const uint32_t sX = smem_u32(smem + kOffX), sH = smem_u32(smem + kOffH);
             const uint32_t sEDY = smem_u32(smem + kOffEDY), sEX = smem_u32(smem + kOffEX);
-            const uint32_t sM1 = smem_u32(smem + kOffM1), sM2 = smem_u32(smem + kOffM2), sM3 = smem_u32(smem + kOffM3);
+            const uint32_t sM1 = smem_u32(smem + kOffM1), sM3 = smem_u32(smem + kOffM3);
             int committed = 0;
             for (int hh = 0; hh < hpg; ++hh) {
                 const uint32_t ph = (uint32_t)hh & 1u;
+                const uint32_t acc = hh > 0 ? 1u : 0u;   // dC, dB: sums over the group's heads
                 if (!mbar_wait_bounded(bar_ld, ph, kWaitNs, aborted, p.status)) break;
-                // the previous head's epilogue has read gB and B g^T (YX's columns)
+                // the previous head's epilogue has read gB, B g^T (YX's columns) and dC
                 if (hh > 0 && !mbar_wait_bounded(bar_e2, ph ^ 1u, kWaitNs, aborted, p.status)) break;
                 tc_fence_after_sync();
 #pragma unroll
@@ -582,26 +584,26 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 if (!mbar_wait_bounded(bar_e0, ph, kWaitNs, aborted, p.status)) break;
                 tc_fence_after_sync();
 #pragma unroll
-                for (int k = 0; k < 4; ++k)   // dC (+)= (Ec o dY) h0   (h0 as [n][p], K = P; summed over heads)
-                    umma_bf16(tmem + kColDC, desc_k(sEDY, k), desc_k(sH, k), kIdKK128, (hh > 0 || k > 0) ? 1u : 0u);
+                for (int k = 0; k < 4; ++k)   // dC (+)= (Ec o dY) h0      (h0 as [n][p], K = P)
+                    umma_bf16(tmem + kColDC, desc_k(sEDY, k), desc_k(sH, k), kIdKK128, k > 0 ? 1u : acc);
 #pragma unroll
-                for (int k = 0; k < 4; ++k)   // U = (El o X) g
-                    umma_bf16(tmem + kColU, desc_k(sEX, k), desc_k(sG, k), kIdKK128, k > 0);
+                for (int k = 0; k < 4; ++k)   // dB (+)= (dt o El o X) g
+                    umma_bf16(tmem + kColDB, desc_k(sEX, k), desc_k(sG, k), kIdKK128, k > 0 ? 1u : acc);
                 umma_commit(bar_p1);
                 ++committed;
                 if (!mbar_wait_bounded(bar_e1, ph, kWaitNs, aborted, p.status)) break;
                 tc_fence_after_sync();
 #pragma unroll
-                for (int k = 0; k < 8; ++k)   // dC += M1 B              (K = Q)
+                for (int k = 0; k < 8; ++k)   // dC += M1 B                 (K = Q)
                     umma_bf16(tmem + kColDC, desc_k(sM1, k), desc_mn(sB, k), kIdKM128, 1u);
 #pragma unroll
-                for (int k = 0; k < 8; ++k)   // U += M2^T C
-                    umma_bf16(tmem + kColU, desc_mn(sM2, k), desc_mn(sC, k), kIdMM128, 1u);
+                for (int k = 0; k < 8; ++k)   // dB += M1^T C  (M1 = dt_j o M2)
+                    umma_bf16(tmem + kColDB, desc_mn(sM1, k), desc_mn(sC, k), kIdMM128, 1u);
 #pragma unroll
                 for (int k = 0; k < 8; ++k)   // gB = M3^T dY
                     umma_bf16(tmem + kColGB, desc_mn(sM3, k), desc_mn(sDY, k), kIdMM64, k > 0);
 #pragma unroll
-                for (int k = 0; k < 8; ++k)   // B g^T                    (g as [n][p], K = N)
+                for (int k = 0; k < 8; ++k)   // B g^T                       (g as [n][p], K = N)
                     umma_bf16(tmem + kColBG, desc_k(sB, k), desc_mn(sG, k), kIdKM64, k > 0);
                 umma_commit(bar_p2);
                 ++committed;
@@ -617,13 +619,10 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         const int i = quad * 32 + lane;      // token row
         const int t = t0 + i;
         const bool valid = i < q;
+        const size_t trow = (size_t)bi * p.L + min(t, p.L - 1);   // (a valid row for addressing)
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        // dB of the group (this row, 32 columns) summed over its heads; dC's
-        // sum stays in TMEM (its accumulator runs on across the heads), and a
-        // head's dC.C is the difference of consecutive running dots
-        float accdB[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) accdB[k] = 0.0f;
+        // dC and dB accumulate over the group's heads in TMEM; a head's dC.C
+        // is the difference of consecutive running dots
         float prev_dcc = 0.0f;
         bool ok = true;
         for (int hh = 0; hh < hpg; ++hh) {
@@ -656,6 +655,7 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             ok = mbar_wait_bounded(bar_ld, ph, kWaitNs, aborted, p.status) && ok;
             {
                 float dd = 0.0f;
+                const float wx = dt_i * El;
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     const uint32_t o = sw128(i, qs * 2 + cc);
@@ -667,7 +667,7 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         y[k] *= Ec;
-                        xv[k] *= El;
+                        xv[k] *= wx;
                     }
                     *reinterpret_cast<uint4*>(smem + kOffEDY + o) = pack8(y);
                     *reinterpret_cast<uint4*>(smem + kOffEX + o) = pack8(xv);
@@ -690,7 +690,8 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             fence_proxy_async_smem();
             mbar_arrive(bar_e0);
 
-            // E1: the masked tiles M1, M2, M3 from YX and CB, and W's row partials
+            // E1: the masked tiles M1, M3 from YX and CB; W's row partials,
+            // the rounding of M1 (rowD) and the column sums of M2 o CB
             ok = mbar_wait_bounded(bar_p1, ph, kWaitNs, aborted, p.status) && ok;
             tc_fence_after_sync();
             {
@@ -698,13 +699,13 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 const uint32_t half = (uint32_t)(qs >> 1) * kTileHalf;
 #pragma unroll
                 for (int sub = 0; sub < 2; ++sub) {   // 16 columns at a time
-                    float yx[16], cb[16], cold[16];
+                    float yx[16], cb[16], col[16];
                     tmem_ld16(tmem + kColYX + lane_off + (uint32_t)(qs * 32 + sub * 16), yx);
                     tmem_ld16(tmem + kColCB + lane_off + (uint32_t)(qs * 32 + sub * 16), cb);
                     tmem_wait_ld();
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
-                        float m1[8], m2[8], m3[8];
+                        float m1[8], m3[8];
 #pragma unroll
                         for (int k = 0; k < 8; ++k) {
                             const int jj = cc * 8 + k;
@@ -712,53 +713,45 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                             const float lm = j <= i ? ex2_approx(cum_i - sCum[j]) : 0.0f;
                             const float v2 = lm * yx[jj];
                             const float v1 = v2 * sDt[j];
-                            m2[k] = bf16_round(v2);
                             m1[k] = bf16_round(v1);
                             m3[k] = lm * cb[jj];
                             w = fmaf(v1, cb[jj], w);
                             rowd = fmaf(m1[k] - v1, cb[jj], rowd);
-                            cold[jj] = (v2 - m2[k]) * cb[jj];
+                            col[jj] = v2 * cb[jj];
                         }
                         const uint32_t o = half + sw128(i, (qs & 1) * 4 + sub * 2 + cc);
                         *reinterpret_cast<uint4*>(smem + kOffM1 + o) = pack8(m1);
-                        *reinterpret_cast<uint4*>(smem + kOffM2 + o) = pack8(m2);
                         *reinterpret_cast<uint4*>(smem + kOffM3 + o) = pack8(m3);
                     }
-                    const float cs = warp_colsum16(cold, lane);
-                    if (lane < 16) sColD[quad * kQ + qs * 32 + sub * 16 + lane] = cs;
+                    const float cs = warp_colsum16(col, lane);
+                    if (lane < 16) sCol[quad * kQ + qs * 32 + sub * 16 + lane] = cs;
                 }
-                sRowD[qs * kQ + i] = rowd;
                 sRow[qs * kQ + i] = w;
+                sRowD[qs * kQ + i] = rowd;
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
             mbar_arrive(bar_e1);
 
-            // E2: dC, dB (summed over heads), dx, and the row dots
+            // E2: dx, this head's dC.C and x^T g B partials
             ok = mbar_wait_bounded(bar_p2, ph, kWaitNs, aborted, p.status) && ok;
             tc_fence_after_sync();
             {
                 const uint32_t half = (uint32_t)(qs >> 1) * kTileHalf;
-                float dcc = 0.0f, ub = 0.0f;
+                float dcc = 0.0f;
 #pragma unroll
                 for (int sub = 0; sub < 2; ++sub) {   // 16 columns at a time
-                    float v[16], u[16];
+                    float v[16];
                     tmem_ld16(tmem + kColDC + lane_off + (uint32_t)(qs * 32 + sub * 16), v);
-                    tmem_ld16(tmem + kColU + lane_off + (uint32_t)(qs * 32 + sub * 16), u);
                     tmem_wait_ld();
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
-                        const uint32_t o = half + sw128(i, (qs & 1) * 4 + sub * 2 + cc);
-                        float cr[8], br[8];
-                        unpack8(*reinterpret_cast<const uint4*>(smem + kOffC + o), cr);
-                        unpack8(*reinterpret_cast<const uint4*>(smem + kOffB + o), br);
+                        float cr[8];
+                        unpack8(*reinterpret_cast<const uint4*>(smem + kOffC + half +
+                                                                sw128(i, (qs & 1) * 4 + sub * 2 + cc)),
+                                cr);
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            const int jj = cc * 8 + k;
-                            dcc = fmaf(v[jj], cr[k], dcc);
-                            ub = fmaf(u[jj], br[k], ub);
-                            accdB[sub * 16 + jj] = fmaf(dt_i, u[jj], accdB[sub * 16 + jj]);
-                        }
+                        for (int k = 0; k < 8; ++k) dcc = fmaf(v[cc * 8 + k], cr[k], dcc);
                     }
                 }
                 {   // this head's share of the running dot
@@ -770,9 +763,9 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 tmem_ld16(tmem + kColGB + lane_off + (uint32_t)(qs * 16), gb);
                 tmem_ld16(tmem + kColBG + lane_off + (uint32_t)(qs * 16), bg);
                 tmem_wait_ld();
-                float dxv[16];
-                const uint4* dyr = reinterpret_cast<const uint4*>(p.dy + (((size_t)bi * p.L + min(t, p.L - 1)) * p.H + h) * kP +
-                                                                  qs * 16);
+                const size_t rowp = (trow * p.H + h) * kP + qs * 16;
+                const uint4* dyr = reinterpret_cast<const uint4*>(p.dy + rowp);
+                float dxv[16], xgb = 0.0f;
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     float y[8];
@@ -781,27 +774,37 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     for (int k = 0; k < 8; ++k)
                         dxv[cc * 8 + k] = fmaf(Dh, y[k], dt_i * fmaf(El, bg[cc * 8 + k], gb[cc * 8 + k]));
                 }
+                const uint4* xr = reinterpret_cast<const uint4*>(p.x + trow * p.row_stride + (size_t)h * kP + qs * 16);
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    float xv[8];
+                    unpack8(xr[cc], xv);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) xgb = fmaf(xv[k], bg[cc * 8 + k], xgb);
+                }
                 if (valid) {
-                    uint4* dst = reinterpret_cast<uint4*>(p.dx + (((size_t)bi * p.L + t) * p.H + h) * kP + qs * 16);
+                    uint4* dst = reinterpret_cast<uint4*>(p.dx + rowp);
                     dst[0] = pack8(dxv);
                     dst[1] = pack8(dxv + 8);
                 }
                 sDCC[qs * kQ + i] = dcc;
-                sUB[qs * kQ + i] = ub;
+                sXGB[qs * kQ + i] = xgb;
             }
             tc_fence_before_sync();
+            mbar_arrive(bar_e2);   // gB, B g^T and dC read: the next head's products may start
             named_bar_sync(kBarEw, kEwThreads);
 
             // the row warps: per-token scalars, the decay gradient, ddt
             if (qs == 0) {
                 const float dcc_h = sDCC[i] + sDCC[kQ + i] + sDCC[2 * kQ + i] + sDCC[3 * kQ + i];
-                const float ub = sUB[i] + sUB[kQ + i] + sUB[2 * kQ + i] + sUB[3 * kQ + i];
+                const float xgb = sXGB[i] + sXGB[kQ + i] + sXGB[2 * kQ + i] + sXGB[3 * kQ + i];
+                const float col = sCol[i] + sCol[kQ + i] + sCol[2 * kQ + i] + sCol[3 * kQ + i];
                 const float wr = sRow[i] + sRow[kQ + i] + sRow[2 * kQ + i] + sRow[3 * kQ + i];
-                const float dd = sDD[i] + sDD[kQ + i] + sDD[2 * kQ + i] + sDD[3 * kQ + i];
                 const float rowd = sRowD[i] + sRowD[kQ + i] + sRowD[2 * kQ + i] + sRowD[3 * kQ + i];
-                const float cold = dt_i * (sColD[i] + sColD[kQ + i] + sColD[2 * kQ + i] + sColD[3 * kQ + i]);
-                const float a = fmaf(dt_i, ub, cold);
-                const float dcc = dcc_h - rowd;
+                const float dd = sDD[i] + sDD[kQ + i] + sDD[2 * kQ + i] + sDD[3 * kQ + i];
+                const float ub = fmaf(El, xgb, col);   // U_i . B_i
+                const float a = dt_i * ub;
+                const float dcc = dcc_h - rowd;        // dC.C with M1's rounding taken out
                 // exclusive prefix of a, inclusive suffix of dcc, total of wr
                 const float ia = warp_incl_scan(a, lane);
                 const float idc = warp_incl_scan(dcc, lane);
@@ -828,16 +831,15 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 float t1 = 0.0f;
 #pragma unroll
                 for (int w2 = 0; w2 < kEwWarps; ++w2) t1 += sT1[w2];
-                t1 *= ex2_approx(sCum[kQ - 1]);
+                t1 *= ex2_approx(cl);
                 const float pre = offa + ia - a;                  // sum_{j<i} a_j
                 const float suf = alldc - (offc + idc - dcc);     // sum_{k>=i} dcc_k
-                const float r = t1 - wsum + pre + suf;            // (a and dcc carry the rounding terms)
+                const float r = t1 - wsum + pre + suf;
                 float ra = 0.0f, rd = 0.0f, rb = 0.0f;
                 if (valid) {
                     const float ddt = ub + Ah * r;
                     const float dv = ddt * sSig[i];
-                    const __nv_bfloat16 dvb = __float2bfloat16_rn(dv);
-                    p.ddt_raw[((size_t)bi * p.L + t) * p.H + h] = dvb;
+                    p.ddt_raw[trow * p.H + h] = __float2bfloat16_rn(dv);
                     ra = dt_i * r;
                     rd = dd;
                     rb = dv;
@@ -854,23 +856,23 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 }
                 named_bar_sync(kBarRows, 128);   // tot[] read before the next head's scan
             }
-            mbar_arrive(bar_e2);
         }
         // dB, dC of the group: this thread's row and 32 columns (the last
         // head's products are complete: its epilogue waited for them)
         if (ok) {
             tc_fence_after_sync();
-            float v[32];
-            tmem_ld32(tmem + kColDC + lane_off + (uint32_t)(qs * 32), v);
+            float vc[32], vb[32];
+            tmem_ld32(tmem + kColDC + lane_off + (uint32_t)(qs * 32), vc);
+            tmem_ld32(tmem + kColDB + lane_off + (uint32_t)(qs * 32), vb);
             tmem_wait_ld();
             if (valid) {
-                const size_t o = (((size_t)bi * p.L + t) * p.G + g) * kN + qs * 32;
+                const size_t o = ((trow * p.G) + g) * kN + qs * 32;
                 uint4* db = reinterpret_cast<uint4*>(p.dB + o);
                 uint4* dc = reinterpret_cast<uint4*>(p.dC + o);
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
-                    db[cc] = pack8(accdB + cc * 8);
-                    dc[cc] = pack8(v + cc * 8);
+                    db[cc] = pack8(vb + cc * 8);
+                    dc[cc] = pack8(vc + cc * 8);
                 }
             }
         }
@@ -1010,6 +1012,8 @@ cudaError_t launch_scan_bwd_tc(const ScanBwdArgs& a, cudaStream_t s)
     TcParams p{};
     p.dt_raw = static_cast<const __nv_bfloat16*>(a.dt_raw);
     p.dy = static_cast<const __nv_bfloat16*>(a.dy);
+    p.x = static_cast<const __nv_bfloat16*>(a.x);
+    p.row_stride = a.row_stride;
     p.dt_bias = a.dt_bias;
     p.A = a.A;
     p.D = a.D;
