@@ -198,11 +198,17 @@ struct TcParams {
     int b, L, H, G, nc;
 };
 
-// dt_t and sigmoid(dt_raw + dt_bias) of chunk row i (0 past the sequence's end)
-__device__ inline void row_dt(const TcParams& p, int bi, int h, int t, bool valid, float& dt, float& sig)
+// dt_raw of token row t for head h (0 past the sequence's end); loaded a
+// head ahead of its use so that its latency hides behind the head before
+__device__ inline float row_dt_raw(const TcParams& p, int bi, int h, int t, bool valid)
 {
-    float v = 0.0f;
-    if (valid) v = __bfloat162float(p.dt_raw[((size_t)bi * p.L + t) * p.H + h]) + (p.dt_bias ? p.dt_bias[h] : 0.0f);
+    return valid ? __bfloat162float(p.dt_raw[((size_t)bi * p.L + t) * p.H + h]) : 0.0f;
+}
+
+// dt_t and sigmoid(dt_raw + dt_bias) from the raw value (dt = 0 past the end)
+__device__ inline void row_dt(const TcParams& p, int h, float raw, bool valid, float& dt, float& sig)
+{
+    const float v = valid ? raw + (p.dt_bias ? p.dt_bias[h] : 0.0f) : 0.0f;
     dt = valid ? softplus_f(v) : 0.0f;
     sig = 1.0f / (1.0f + __expf(-v));
 }
@@ -224,18 +230,19 @@ __device__ inline float block_cumsum128(float l, int quad, int lane, float* tot,
 // Kernel 1: chunk states S^T = B^T (w o X) and dS^T = C^T (Ec o dY)
 // ---------------------------------------------------------------------------
 namespace k1 {
-constexpr int kEwWarps = 4;
-constexpr int kThreads = (kEwWarps + 2) * 32;   // warp 0 producer, 1 MMA, 2..5 rows
-constexpr int kOffB = 0, kOffC = 32768, kOffX = 65536, kOffDY = 81920, kOffWX = 98304, kOffWDY = 114688;
-constexpr int kOffVec = 131072;                 // tot[4]
-constexpr int kOffBar = kOffVec + 64;
+constexpr int kEwWarps = 8;                     // two per TMEM lane quadrant
+constexpr int kThreads = (kEwWarps + 2) * 32;   // warp 0 producer, 1 MMA, 2..9 rows
+// X and dY are scaled in place (w o X, Ec o dY); 2 CTAs fit on an SM
+constexpr int kOffB = 0, kOffC = 32768, kOffX = 65536, kOffDY = 81920;
+constexpr int kOffVec = 98304;                  // floats: tot[4], w[128], Ec[128]
+constexpr int kOffBar = kOffVec + 1088;
 constexpr int kOffMisc = kOffBar + 8 * 8;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;
 constexpr uint32_t kTmemCols = 128;             // S^T [0,64), dS^T [64,128)
 constexpr uint32_t kIdS = umma_idesc_bf16(128, 64, true, true);   // B^T (MN) x wX (MN)
 }  // namespace k1
 
-__global__ void __launch_bounds__(k1::kThreads, 1)
+__global__ void __launch_bounds__(k1::kThreads, 2)
 bwd_states_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmDY,
                   const TcParams p)
@@ -250,9 +257,8 @@ bwd_states_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     const int t0 = c * kQ;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
     uint64_t* bar_ld = bars + 0;     // X, dY (and B, C for the first head) landed
-    uint64_t* bar_w = bars + 1;      // w o X and Ec o dY written (row warps)
-    uint64_t* bar_xfree = bars + 2;  // X, dY read (row warps)
-    uint64_t* bar_mma = bars + 3;    // S^T, dS^T in TMEM
+    uint64_t* bar_w = bars + 1;      // w o X and Ec o dY written in place (row warps)
+    uint64_t* bar_mma = bars + 2;    // S^T, dS^T in TMEM (X and dY free)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* aborted = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
     float* tot = reinterpret_cast<float*>(smem + kOffVec);
@@ -261,7 +267,6 @@ bwd_states_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         *aborted = 0;
         mbar_init(bar_ld, 1);
         mbar_init(bar_w, kEwWarps * 32);
-        mbar_init(bar_xfree, kEwWarps * 32);
         mbar_init(bar_mma, 1);
         fence_mbar_init();
     }
@@ -280,7 +285,8 @@ bwd_states_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             int issued = 0;
             for (int hh = 0; hh < hpg; ++hh) {
                 const int h = g * hpg + hh;
-                if (hh > 0 && !mbar_wait_bounded(bar_xfree, (uint32_t)(hh - 1) & 1u, kWaitNs, aborted, p.status))
+                // the previous head's products have read its X and dY
+                if (hh > 0 && !mbar_wait_bounded(bar_mma, (uint32_t)(hh - 1) & 1u, kWaitNs, aborted, p.status))
                     break;
                 mbar_arrive_expect_tx(bar_ld, hh == 0 ? 6 * kTileHalf : 2 * kTileHalf);
                 tma_load_3d(smem + kOffX, &tmX, h * kP, t0, bi, bar_ld);
@@ -299,7 +305,7 @@ bwd_states_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t sB = smem_u32(smem + kOffB), sC = smem_u32(smem + kOffC);
-            const uint32_t sWX = smem_u32(smem + kOffWX), sWDY = smem_u32(smem + kOffWDY);
+            const uint32_t sWX = smem_u32(smem + kOffX), sWDY = smem_u32(smem + kOffDY);   // scaled in place
             int committed = 0;
             for (int hh = 0; hh < hpg; ++hh) {
                 const uint32_t ph = (uint32_t)hh & 1u;
@@ -318,61 +324,69 @@ bwd_states_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         }
         __syncwarp();
     } else {
-        // row warps: thread = token row i (weights), then state row n = i (epilogue)
+        // elementwise warps, two per lane quadrant (part 0, 1): thread = token
+        // row i (weights; part p scales chunks 4p..4p+3 of X and dY), then
+        // state row n = i (epilogue: part 0 writes S^T, part 1 dS^T)
+        const int ew = warp - 2;
         const int quad = warp & 3;
+        const int part = ew >> 2;
         const int i = quad * 32 + lane;
         const int t = t0 + i;
         const bool valid = t < p.L;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        float* sW = tot + 4;   // [128] w_i = El_i dt_i
+        float* sE = sW + kQ;   // [128] Ec_i
         bool ok = true;
+        float raw_next = part == 0 ? row_dt_raw(p, bi, g * hpg, t, valid) : 0.0f;
         for (int hh = 0; hh < hpg; ++hh) {
             const int h = g * hpg + hh;
             const int chain = bi * p.H + h;
             const uint32_t ph = (uint32_t)hh & 1u;
-            float dt, sig;
-            row_dt(p, bi, h, t, valid, dt, sig);
-            // tot[] of the previous head read; a give-up anywhere ends all rows here
-            if (named_bar_any(1, 128, !ok)) break;
-            const float cum = block_cumsum128(dt * p.A[h] * kLog2e, quad, lane, tot, 1);
-            const float cl = tot[0] + tot[1] + tot[2] + tot[3];
-            const float w = ex2_approx(cl - cum) * dt;
-            const float e = ex2_approx(cum);
-            if (i == 0) p.ws_cl[(size_t)chain * p.nc + c] = cl;
+            const float raw = raw_next;
+            if (part == 0 && hh + 1 < hpg) raw_next = row_dt_raw(p, bi, h + 1, t, valid);
+            // the previous head's weights read; a give-up anywhere ends all rows here
+            if (named_bar_any(2, kEwWarps * 32, !ok)) break;
+            if (part == 0) {
+                float dt, sig;
+                row_dt(p, h, raw, valid, dt, sig);
+                const float cum = block_cumsum128(dt * p.A[h] * kLog2e, quad, lane, tot, 1);
+                const float cl = tot[0] + tot[1] + tot[2] + tot[3];
+                sW[i] = ex2_approx(cl - cum) * dt;
+                sE[i] = ex2_approx(cum);
+                if (i == 0) p.ws_cl[(size_t)chain * p.nc + c] = cl;
+            }
+            named_bar_sync(2, kEwWarps * 32);
+            const float w = sW[i], e = sE[i];
             // (after a give-up the head runs on without waiting, so that
             // every row reaches the next barrier)
             ok = mbar_wait_bounded(bar_ld, ph, kWaitNs, aborted, p.status) && ok;
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
+            for (int cc = 0; cc < 4; ++cc) {
                 float v[8];
-                const uint32_t o = sw128(i, ch);
+                const uint32_t o = sw128(i, part * 4 + cc);
                 unpack8(*reinterpret_cast<const uint4*>(smem + kOffX + o), v);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) v[k] *= w;
-                *reinterpret_cast<uint4*>(smem + kOffWX + o) = pack8(v);
+                *reinterpret_cast<uint4*>(smem + kOffX + o) = pack8(v);
                 unpack8(*reinterpret_cast<const uint4*>(smem + kOffDY + o), v);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) v[k] *= e;
-                *reinterpret_cast<uint4*>(smem + kOffWDY + o) = pack8(v);
+                *reinterpret_cast<uint4*>(smem + kOffDY + o) = pack8(v);
             }
-            mbar_arrive(bar_xfree);
             fence_proxy_async_smem();
             mbar_arrive(bar_w);
             ok = mbar_wait_bounded(bar_mma, ph, kWaitNs, aborted, p.status) && ok;
             tc_fence_after_sync();
-            // state row n = i: S^T[n][0..63], dS^T[n][0..63], in bf16
-            uint4* dS = reinterpret_cast<uint4*>(p.ws_S + ((size_t)chain * p.nc + c) * kStatesDim + (size_t)i * kP);
-            uint4* ddS = reinterpret_cast<uint4*>(p.ws_dS + ((size_t)chain * p.nc + c) * kStatesDim + (size_t)i * kP);
+            // state row n = i of S^T (part 0) or dS^T (part 1), in bf16
+            uint4* dst = reinterpret_cast<uint4*>((part == 0 ? p.ws_S : p.ws_dS) +
+                                                  ((size_t)chain * p.nc + c) * kStatesDim + (size_t)i * kP);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                float v[32], u[32];
-                tmem_ld32(tmem + lane_off + (uint32_t)(half * 32), v);
-                tmem_ld32(tmem + lane_off + 64u + (uint32_t)(half * 32), u);
+                float v[32];
+                tmem_ld32(tmem + lane_off + (uint32_t)(part * 64 + half * 32), v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    dS[half * 4 + k] = pack8(v + 8 * k);
-                    ddS[half * 4 + k] = pack8(u + 8 * k);
-                }
+                for (int k = 0; k < 4; ++k) dst[half * 4 + k] = pack8(v + 8 * k);
             }
             tc_fence_before_sync();
         }
@@ -452,8 +466,11 @@ constexpr int kThreads = kEwThreads + 64;       // warp 0 producer, 1 MMA, 2..17
 constexpr int kOffB = 0, kOffC = 32768, kOffDY = 65536, kOffG = 81920, kOffR = 98304;
 constexpr int kOffX = kOffR, kOffH = kOffR + 16384, kOffEDY = kOffR + 32768, kOffEX = kOffR + 49152;
 constexpr int kOffM1 = kOffR, kOffM3 = kOffR + 32768;
-constexpr int kOffVec = kOffR + 65536;          // floats: cum, dt, sig [128] each, partials [6][4][128], tot [8], t1 [16]
-constexpr int kVecFloats = 3 * kQ + 24 * kQ + 8 + 16;
+// floats, two sets by head parity: cum, dt, sig [128] each, partials
+// [6][4][128], t1 [16]; then scan scratch [16]
+constexpr int kOffVec = kOffR + 65536;
+constexpr int kVecSet = 3 * kQ + 24 * kQ + 16;
+constexpr int kVecFloats = 2 * kVecSet + 16;
 constexpr int kOffBar = kOffVec + ((kVecFloats * 4 + 63) / 64) * 64;
 constexpr int kNumBars = 6;
 constexpr int kOffMisc = kOffBar + 8 * kNumBars;
@@ -496,17 +513,29 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     uint64_t* bar_e2 = bars + 5;   // the head's epilogue has read gB, B g^T and dC
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* aborted = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
-    float* sCum = reinterpret_cast<float*>(smem + kOffVec);
-    float* sDt = sCum + kQ;
-    float* sSig = sDt + kQ;
-    float* sRow = sSig + kQ;        // [column quarter][row]: W partials
-    float* sRowD = sRow + 4 * kQ;   // rowD partials
-    float* sDD = sRowD + 4 * kQ;    // dy.x partials
-    float* sDCC = sDD + 4 * kQ;     // dC.C partials
-    float* sXGB = sDCC + 4 * kQ;    // x^T g B partials
-    float* sCol = sXGB + 4 * kQ;    // [lane quadrant][column]: sum_k M2 CB partials
-    float* tot = sCol + 4 * kQ;     // [8] scan scratch
-    float* sT1 = tot + 8;           // [16] <g, h0> partials, one per elementwise warp
+    // per-head vectors and partial sums, by head parity (a head's last step
+    // runs while the next head is under way)
+    struct Vec {
+        float *cum, *dt, *sig;
+        float *row, *rowd, *dd, *dcc, *xgb, *col;   // [4][128] partials
+        float* t1;                                   // [16] <g, h0> partials
+    };
+    auto vec = [&](int parity) {
+        float* b = reinterpret_cast<float*>(smem + kOffVec) + parity * kVecSet;
+        Vec v;
+        v.cum = b;
+        v.dt = b + kQ;
+        v.sig = b + 2 * kQ;
+        v.row = b + 3 * kQ;       // [column quarter][row]: W partials
+        v.rowd = v.row + 4 * kQ;  // rowD partials
+        v.dd = v.rowd + 4 * kQ;   // dy.x partials
+        v.dcc = v.dd + 4 * kQ;    // dC.C partials
+        v.xgb = v.dcc + 4 * kQ;   // x^T g B partials
+        v.col = v.xgb + 4 * kQ;   // [lane quadrant][column]: sum_k M2 CB partials
+        v.t1 = v.col + 4 * kQ;
+        return v;
+    };
+    float* tot = reinterpret_cast<float*>(smem + kOffVec) + 2 * kVecSet;   // [4] cumsum, [8] row scans
 
     if (tid == 0) {
         *aborted = 0;
@@ -625,32 +654,109 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         // is the difference of consecutive running dots
         float prev_dcc = 0.0f;
         bool ok = true;
-        for (int hh = 0; hh < hpg; ++hh) {
+        float raw_next = qs == 0 ? row_dt_raw(p, bi, g * hpg, t, valid) : 0.0f;
+
+        // The last step of head hh, on the row warps (qs == 0): per-token
+        // scalars, the decay gradient, ddt_raw and the partial sums of dA,
+        // dD, ddt_bias.  It runs one head late, while the next head's second
+        // products are on the tensor cores.
+        auto row_step = [&](int hh) {
+            const Vec v = vec(hh & 1);
             const int h = g * hpg + hh;
             const int chain = bi * p.H + h;
+            const float cl = v.cum[kQ - 1];
+            const float dt_i = v.dt[i];
+            const float El = ex2_approx(cl - v.cum[i]);
+            const float dcc_h = v.dcc[i] + v.dcc[kQ + i] + v.dcc[2 * kQ + i] + v.dcc[3 * kQ + i];
+            const float xgb = v.xgb[i] + v.xgb[kQ + i] + v.xgb[2 * kQ + i] + v.xgb[3 * kQ + i];
+            const float col = v.col[i] + v.col[kQ + i] + v.col[2 * kQ + i] + v.col[3 * kQ + i];
+            const float wr = v.row[i] + v.row[kQ + i] + v.row[2 * kQ + i] + v.row[3 * kQ + i];
+            const float rowd = v.rowd[i] + v.rowd[kQ + i] + v.rowd[2 * kQ + i] + v.rowd[3 * kQ + i];
+            const float dd = v.dd[i] + v.dd[kQ + i] + v.dd[2 * kQ + i] + v.dd[3 * kQ + i];
+            const float ub = fmaf(El, xgb, col);   // U_i . B_i
+            const float a = dt_i * ub;
+            const float dcc = dcc_h - rowd;        // dC.C with M1's rounding taken out
+            // exclusive prefix of a, inclusive suffix of dcc, total of wr
+            const float ia = warp_incl_scan(a, lane);
+            const float idc = warp_incl_scan(dcc, lane);
+            const float tw = warp_total(wr);
+            float* ts = tot + 4;
+            named_bar_sync(kBarRows, 128);   // ts[] of the previous step read
+            if (lane == 31) {
+                ts[quad] = ia;
+                ts[4 + quad] = idc;
+            }
+            named_bar_sync(kBarRows, 128);
+            float offa = 0.0f, offc = 0.0f, alldc = 0.0f;
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+                if (qq < quad) {
+                    offa += ts[qq];
+                    offc += ts[4 + qq];
+                }
+                alldc += ts[4 + qq];
+            }
+            named_bar_sync(kBarRows, 128);
+            if (lane == 0) ts[quad] = tw;
+            named_bar_sync(kBarRows, 128);
+            const float wsum = ts[0] + ts[1] + ts[2] + ts[3];
+            float t1 = 0.0f;
+#pragma unroll
+            for (int w2 = 0; w2 < kEwWarps; ++w2) t1 += v.t1[w2];
+            t1 *= ex2_approx(cl);
+            const float pre = offa + ia - a;                  // sum_{j<i} a_j
+            const float suf = alldc - (offc + idc - dcc);     // sum_{k>=i} dcc_k
+            const float r = t1 - wsum + pre + suf;
+            float ra = 0.0f, rd = 0.0f, rb = 0.0f;
+            if (valid) {
+                const float ddt = ub + p.A[h] * r;
+                const float dv = ddt * v.sig[i];
+                p.ddt_raw[trow * p.H + h] = __float2bfloat16_rn(dv);
+                ra = dt_i * r;
+                rd = dd;
+                rb = dv;
+            }
+            ra = warp_total(ra);
+            rd = warp_total(rd);
+            rb = warp_total(rb);
+            if (lane == 0) {
+                const size_t nparts = (size_t)p.b * p.H * p.nc * kParts;
+                const size_t o = ((size_t)chain * p.nc + c) * kParts + quad;
+                p.ws_part[o] = ra;
+                p.ws_part[nparts + o] = rd;
+                p.ws_part[2 * nparts + o] = rb;
+            }
+        };
+
+        for (int hh = 0; hh < hpg; ++hh) {
+            const int h = g * hpg + hh;
             const uint32_t ph = (uint32_t)hh & 1u;
+            const Vec v = vec(hh & 1);
             const float Ah = p.A[h];
             const float Dh = p.D ? p.D[h] : 0.0f;
+            const float raw = raw_next;
+            if (qs == 0 && hh + 1 < hpg) raw_next = row_dt_raw(p, bi, h + 1, t, valid);
 
             // E0: dt, cumulative decay (row warps), then the scaled copies.
             // The barrier also ends the loop of every warp at once after a
             // give-up (inside a head nobody leaves early, so that every
-            // warp reaches every barrier).
+            // warp reaches every barrier), and it orders the previous
+            // head's partial sums before their use.
             if (named_bar_any(kBarEw, kEwThreads, !ok)) {
                 ok = false;
                 break;
             }
             if (qs == 0) {
                 float dt, sig;
-                row_dt(p, bi, h, t, valid, dt, sig);
+                row_dt(p, h, raw, valid, dt, sig);
                 const float cum = block_cumsum128(dt * Ah * kLog2e, quad, lane, tot, kBarRows);
-                sCum[i] = cum;
-                sDt[i] = dt;
-                sSig[i] = sig;
+                v.cum[i] = cum;
+                v.dt[i] = dt;
+                v.sig[i] = sig;
             }
             named_bar_sync(kBarEw, kEwThreads);
-            const float cum_i = sCum[i], dt_i = sDt[i];
-            const float cl = sCum[kQ - 1];
+            const float cum_i = v.cum[i], dt_i = v.dt[i];
+            const float cl = v.cum[kQ - 1];
             const float Ec = ex2_approx(cum_i), El = ex2_approx(cl - cum_i);
             ok = mbar_wait_bounded(bar_ld, ph, kWaitNs, aborted, p.status) && ok;
             {
@@ -672,7 +778,7 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     *reinterpret_cast<uint4*>(smem + kOffEDY + o) = pack8(y);
                     *reinterpret_cast<uint4*>(smem + kOffEX + o) = pack8(xv);
                 }
-                sDD[qs * kQ + i] = dd;
+                v.dd[qs * kQ + i] = dd;
                 // <g, h0> over the two bf16 tiles (same layout): 2 chunks per thread
                 float gh = 0.0f;
 #pragma unroll
@@ -685,7 +791,7 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     for (int k = 0; k < 8; ++k) gh = fmaf(hv[k], gv[k], gh);
                 }
                 gh = warp_total(gh);
-                if (lane == 0) sT1[ew] = gh;
+                if (lane == 0) v.t1[ew] = gh;
             }
             fence_proxy_async_smem();
             mbar_arrive(bar_e0);
@@ -710,9 +816,9 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                         for (int k = 0; k < 8; ++k) {
                             const int jj = cc * 8 + k;
                             const int j = qs * 32 + sub * 16 + jj;
-                            const float lm = j <= i ? ex2_approx(cum_i - sCum[j]) : 0.0f;
+                            const float lm = j <= i ? ex2_approx(cum_i - v.cum[j]) : 0.0f;
                             const float v2 = lm * yx[jj];
-                            const float v1 = v2 * sDt[j];
+                            const float v1 = v2 * v.dt[j];
                             m1[k] = bf16_round(v1);
                             m3[k] = lm * cb[jj];
                             w = fmaf(v1, cb[jj], w);
@@ -724,14 +830,17 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                         *reinterpret_cast<uint4*>(smem + kOffM3 + o) = pack8(m3);
                     }
                     const float cs = warp_colsum16(col, lane);
-                    if (lane < 16) sCol[quad * kQ + qs * 32 + sub * 16 + lane] = cs;
+                    if (lane < 16) v.col[quad * kQ + qs * 32 + sub * 16 + lane] = cs;
                 }
-                sRow[qs * kQ + i] = w;
-                sRowD[qs * kQ + i] = rowd;
+                v.row[qs * kQ + i] = w;
+                v.rowd[qs * kQ + i] = rowd;
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
             mbar_arrive(bar_e1);
+
+            // the previous head's last step, while the products run
+            if (qs == 0 && hh > 0) row_step(hh - 1);
 
             // E2: dx, this head's dC.C and x^T g B partials
             ok = mbar_wait_bounded(bar_p2, ph, kWaitNs, aborted, p.status) && ok;
@@ -741,8 +850,8 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 float dcc = 0.0f;
 #pragma unroll
                 for (int sub = 0; sub < 2; ++sub) {   // 16 columns at a time
-                    float v[16];
-                    tmem_ld16(tmem + kColDC + lane_off + (uint32_t)(qs * 32 + sub * 16), v);
+                    float vv[16];
+                    tmem_ld16(tmem + kColDC + lane_off + (uint32_t)(qs * 32 + sub * 16), vv);
                     tmem_wait_ld();
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
@@ -751,7 +860,7 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                                                                 sw128(i, (qs & 1) * 4 + sub * 2 + cc)),
                                 cr);
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) dcc = fmaf(v[cc * 8 + k], cr[k], dcc);
+                        for (int k = 0; k < 8; ++k) dcc = fmaf(vv[cc * 8 + k], cr[k], dcc);
                     }
                 }
                 {   // this head's share of the running dot
@@ -787,76 +896,16 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     dst[0] = pack8(dxv);
                     dst[1] = pack8(dxv + 8);
                 }
-                sDCC[qs * kQ + i] = dcc;
-                sXGB[qs * kQ + i] = xgb;
+                v.dcc[qs * kQ + i] = dcc;
+                v.xgb[qs * kQ + i] = xgb;
             }
             tc_fence_before_sync();
             mbar_arrive(bar_e2);   // gB, B g^T and dC read: the next head's products may start
-            named_bar_sync(kBarEw, kEwThreads);
-
-            // the row warps: per-token scalars, the decay gradient, ddt
-            if (qs == 0) {
-                const float dcc_h = sDCC[i] + sDCC[kQ + i] + sDCC[2 * kQ + i] + sDCC[3 * kQ + i];
-                const float xgb = sXGB[i] + sXGB[kQ + i] + sXGB[2 * kQ + i] + sXGB[3 * kQ + i];
-                const float col = sCol[i] + sCol[kQ + i] + sCol[2 * kQ + i] + sCol[3 * kQ + i];
-                const float wr = sRow[i] + sRow[kQ + i] + sRow[2 * kQ + i] + sRow[3 * kQ + i];
-                const float rowd = sRowD[i] + sRowD[kQ + i] + sRowD[2 * kQ + i] + sRowD[3 * kQ + i];
-                const float dd = sDD[i] + sDD[kQ + i] + sDD[2 * kQ + i] + sDD[3 * kQ + i];
-                const float ub = fmaf(El, xgb, col);   // U_i . B_i
-                const float a = dt_i * ub;
-                const float dcc = dcc_h - rowd;        // dC.C with M1's rounding taken out
-                // exclusive prefix of a, inclusive suffix of dcc, total of wr
-                const float ia = warp_incl_scan(a, lane);
-                const float idc = warp_incl_scan(dcc, lane);
-                const float tw = warp_total(wr);
-                if (lane == 31) {
-                    tot[quad] = ia;
-                    tot[4 + quad] = idc;
-                }
-                named_bar_sync(kBarRows, 128);
-                float offa = 0.0f, offc = 0.0f, alldc = 0.0f;
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    if (qq < quad) {
-                        offa += tot[qq];
-                        offc += tot[4 + qq];
-                    }
-                    alldc += tot[4 + qq];
-                }
-                // W total: reduce the four warp totals through shared memory
-                named_bar_sync(kBarRows, 128);
-                if (lane == 0) tot[quad] = tw;
-                named_bar_sync(kBarRows, 128);
-                const float wsum = tot[0] + tot[1] + tot[2] + tot[3];
-                float t1 = 0.0f;
-#pragma unroll
-                for (int w2 = 0; w2 < kEwWarps; ++w2) t1 += sT1[w2];
-                t1 *= ex2_approx(cl);
-                const float pre = offa + ia - a;                  // sum_{j<i} a_j
-                const float suf = alldc - (offc + idc - dcc);     // sum_{k>=i} dcc_k
-                const float r = t1 - wsum + pre + suf;
-                float ra = 0.0f, rd = 0.0f, rb = 0.0f;
-                if (valid) {
-                    const float ddt = ub + Ah * r;
-                    const float dv = ddt * sSig[i];
-                    p.ddt_raw[trow * p.H + h] = __float2bfloat16_rn(dv);
-                    ra = dt_i * r;
-                    rd = dd;
-                    rb = dv;
-                }
-                ra = warp_total(ra);
-                rd = warp_total(rd);
-                rb = warp_total(rb);
-                if (lane == 0) {
-                    const size_t nparts = (size_t)p.b * p.H * p.nc * kParts;
-                    const size_t o = ((size_t)chain * p.nc + c) * kParts + quad;
-                    p.ws_part[o] = ra;
-                    p.ws_part[nparts + o] = rd;
-                    p.ws_part[2 * nparts + o] = rb;
-                }
-                named_bar_sync(kBarRows, 128);   // tot[] read before the next head's scan
-            }
         }
+        // the last head's last step (its partial sums complete after this
+        // barrier, which also makes the decision the same for every warp)
+        if (named_bar_any(kBarEw, kEwThreads, !ok)) ok = false;
+        if (ok && qs == 0) row_step(hpg - 1);
         // dB, dC of the group: this thread's row and 32 columns (the last
         // head's products are complete: its epilogue waited for them)
         if (ok) {
