@@ -68,6 +68,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kPassSlices = 8;               // CTAs per chain and direction in the passing kernel
 constexpr int kPassThreads = 256;            // 4 state elements per thread
 constexpr int kParts = 4;                    // dA / dD / ddt_bias partials per (chain, chunk)
+constexpr int kMaxHpg = 256;                 // heads per group (per-head scalars kept in shared memory)
 
 constexpr uint32_t kStatesDim = kN * kP;     // floats of one chunk state
 
@@ -206,9 +207,9 @@ __device__ inline float row_dt_raw(const TcParams& p, int bi, int h, int t, bool
 }
 
 // dt_t and sigmoid(dt_raw + dt_bias) from the raw value (dt = 0 past the end)
-__device__ inline void row_dt(const TcParams& p, int h, float raw, bool valid, float& dt, float& sig)
+__device__ inline void row_dt(float bias, float raw, bool valid, float& dt, float& sig)
 {
-    const float v = valid ? raw + (p.dt_bias ? p.dt_bias[h] : 0.0f) : 0.0f;
+    const float v = valid ? raw + bias : 0.0f;
     dt = valid ? softplus_f(v) : 0.0f;
     sig = 1.0f / (1.0f + __expf(-v));
 }
@@ -234,8 +235,8 @@ constexpr int kEwWarps = 8;                     // two per TMEM lane quadrant
 constexpr int kThreads = (kEwWarps + 2) * 32;   // warp 0 producer, 1 MMA, 2..9 rows
 // X and dY are scaled in place (w o X, Ec o dY); 2 CTAs fit on an SM
 constexpr int kOffB = 0, kOffC = 32768, kOffX = 65536, kOffDY = 81920;
-constexpr int kOffVec = 98304;                  // floats: tot[4], w[128], Ec[128]
-constexpr int kOffBar = kOffVec + 1088;
+constexpr int kOffVec = 98304;                  // floats: tot[4], w[128], Ec[128], A and dt_bias [kMaxHpg]
+constexpr int kOffBar = kOffVec + 1088 + 8 * kMaxHpg;
 constexpr int kOffMisc = kOffBar + 8 * 8;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;
 constexpr uint32_t kTmemCols = 128;             // S^T [0,64), dS^T [64,128)
@@ -262,6 +263,12 @@ bwd_states_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* aborted = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
     float* tot = reinterpret_cast<float*>(smem + kOffVec);
+    float* sA = tot + 4 + 2 * kQ;      // [hpg] A of the group's heads
+    float* sBias = sA + kMaxHpg;       // [hpg] dt_bias
+    for (int k = tid; k < hpg; k += kThreads) {
+        sA[k] = p.A[g * hpg + k];
+        sBias[k] = p.dt_bias ? p.dt_bias[g * hpg + k] : 0.0f;
+    }
 
     if (tid == 0) {
         *aborted = 0;
@@ -348,8 +355,8 @@ bwd_states_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             if (named_bar_any(2, kEwWarps * 32, !ok)) break;
             if (part == 0) {
                 float dt, sig;
-                row_dt(p, h, raw, valid, dt, sig);
-                const float cum = block_cumsum128(dt * p.A[h] * kLog2e, quad, lane, tot, 1);
+                row_dt(sBias[hh], raw, valid, dt, sig);
+                const float cum = block_cumsum128(dt * sA[hh] * kLog2e, quad, lane, tot, 1);
                 const float cl = tot[0] + tot[1] + tot[2] + tot[3];
                 sW[i] = ex2_approx(cl - cum) * dt;
                 sE[i] = ex2_approx(cum);
@@ -467,10 +474,10 @@ constexpr int kOffB = 0, kOffC = 32768, kOffDY = 65536, kOffG = 81920, kOffR = 9
 constexpr int kOffX = kOffR, kOffH = kOffR + 16384, kOffEDY = kOffR + 32768, kOffEX = kOffR + 49152;
 constexpr int kOffM1 = kOffR, kOffM3 = kOffR + 32768;
 // floats, two sets by head parity: cum, dt, sig [128] each, partials
-// [6][4][128], t1 [16]; then scan scratch [16]
+// [6][4][128], t1 [16]; then scan scratch [16]; A, D, dt_bias [kMaxHpg]
 constexpr int kOffVec = kOffR + 65536;
 constexpr int kVecSet = 3 * kQ + 24 * kQ + 16;
-constexpr int kVecFloats = 2 * kVecSet + 16;
+constexpr int kVecFloats = 2 * kVecSet + 16 + 3 * kMaxHpg;
 constexpr int kOffBar = kOffVec + ((kVecFloats * 4 + 63) / 64) * 64;
 constexpr int kNumBars = 6;
 constexpr int kOffMisc = kOffBar + 8 * kNumBars;
@@ -536,6 +543,14 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         return v;
     };
     float* tot = reinterpret_cast<float*>(smem + kOffVec) + 2 * kVecSet;   // [4] cumsum, [8] row scans
+    float* sA = tot + 16;              // [hpg] per-head scalars of the group
+    float* sD = sA + kMaxHpg;
+    float* sBias = sD + kMaxHpg;
+    for (int k = tid; k < hpg; k += kThreads) {
+        sA[k] = p.A[g * hpg + k];
+        sD[k] = p.D ? p.D[g * hpg + k] : 0.0f;
+        sBias[k] = p.dt_bias ? p.dt_bias[g * hpg + k] : 0.0f;
+    }
 
     if (tid == 0) {
         *aborted = 0;
@@ -709,7 +724,7 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             const float r = t1 - wsum + pre + suf;
             float ra = 0.0f, rd = 0.0f, rb = 0.0f;
             if (valid) {
-                const float ddt = ub + p.A[h] * r;
+                const float ddt = ub + sA[hh] * r;
                 const float dv = ddt * v.sig[i];
                 p.ddt_raw[trow * p.H + h] = __float2bfloat16_rn(dv);
                 ra = dt_i * r;
@@ -732,8 +747,8 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             const int h = g * hpg + hh;
             const uint32_t ph = (uint32_t)hh & 1u;
             const Vec v = vec(hh & 1);
-            const float Ah = p.A[h];
-            const float Dh = p.D ? p.D[h] : 0.0f;
+            const float Ah = sA[hh];
+            const float Dh = sD[hh];
             const float raw = raw_next;
             if (qs == 0 && hh + 1 < hpg) raw_next = row_dt_raw(p, bi, h + 1, t, valid);
 
@@ -748,7 +763,7 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             }
             if (qs == 0) {
                 float dt, sig;
-                row_dt(p, h, raw, valid, dt, sig);
+                row_dt(sBias[hh], raw, valid, dt, sig);
                 const float cum = block_cumsum128(dt * Ah * kLog2e, quad, lane, tot, kBarRows);
                 v.cum[i] = cum;
                 v.dt[i] = dt;
@@ -842,7 +857,12 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             // the previous head's last step, while the products run
             if (qs == 0 && hh > 0) row_step(hh - 1);
 
-            // E2: dx, this head's dC.C and x^T g B partials
+            // E2: dx, this head's dC.C and x^T g B partials (the dy and x
+            // rows are loaded before the wait for the products)
+            const size_t rowp = (trow * p.H + h) * kP + qs * 16;
+            const uint4* dyr = reinterpret_cast<const uint4*>(p.dy + rowp);
+            const uint4* xr = reinterpret_cast<const uint4*>(p.x + trow * p.row_stride + (size_t)h * kP + qs * 16);
+            const uint4 dy0 = dyr[0], dy1 = dyr[1], x0 = xr[0], x1 = xr[1];
             ok = mbar_wait_bounded(bar_p2, ph, kWaitNs, aborted, p.status) && ok;
             tc_fence_after_sync();
             {
@@ -872,22 +892,19 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 tmem_ld16(tmem + kColGB + lane_off + (uint32_t)(qs * 16), gb);
                 tmem_ld16(tmem + kColBG + lane_off + (uint32_t)(qs * 16), bg);
                 tmem_wait_ld();
-                const size_t rowp = (trow * p.H + h) * kP + qs * 16;
-                const uint4* dyr = reinterpret_cast<const uint4*>(p.dy + rowp);
                 float dxv[16], xgb = 0.0f;
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     float y[8];
-                    unpack8(dyr[cc], y);
+                    unpack8(cc ? dy1 : dy0, y);
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
                         dxv[cc * 8 + k] = fmaf(Dh, y[k], dt_i * fmaf(El, bg[cc * 8 + k], gb[cc * 8 + k]));
                 }
-                const uint4* xr = reinterpret_cast<const uint4*>(p.x + trow * p.row_stride + (size_t)h * kP + qs * 16);
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     float xv[8];
-                    unpack8(xr[cc], xv);
+                    unpack8(cc ? x1 : x0, xv);
 #pragma unroll
                     for (int k = 0; k < 8; ++k) xgb = fmaf(xv[k], bg[cc * 8 + k], xgb);
                 }
@@ -1042,6 +1059,7 @@ bool scan_bwd_tc_shape(int P, int N, bool bf16) { return bf16 && P == kP && N ==
 bool scan_bwd_tc_supported(const ScanBwdArgs& a)
 {
     return scan_bwd_tc_shape(a.P, a.N, a.bf16) && a.b > 0 && a.L > 0 && (int64_t)a.b * a.G < 65536 &&
+           a.H / a.G <= kMaxHpg &&
            a.row_stride % 8 == 0 && a16(a.x) &&
            a16(a.B) && a16(a.C) && a16(a.dy) && a16(a.dx) && a16(a.dB) && a16(a.dC) && a16(a.workspace) &&
            (size_t)a.b * a.H * ((a.L + kQ - 1) / kQ) * kN < 0x7fffffffULL;
