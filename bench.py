@@ -93,6 +93,13 @@ def scan_bwd_bytes_per_token(s) -> int:
     return s.elem_bytes * (3 * s.H * s.P + 4 * s.G * s.N + 2 * s.H)
 
 
+def scan_bwd_flops_per_token(s) -> int:
+    """Backward pass, the chunked matrix form: causal C.B^T (G*Q*N), causal
+    dY.X^T and M3^T.dY (2*H*Q*P), causal M1.B and M1^T.C (2*H*Q*N), and the
+    five state products S, dS, (Ec o dY).h0, (El o X).g, B.g^T (10*H*P*N)."""
+    return s.G * s.Q * s.N + 2 * s.H * s.Q * s.P + 2 * s.H * s.Q * s.N + 10 * s.H * s.P * s.N
+
+
 def linear_flops(M, N, K) -> int:
     return 2 * M * N * K
 
@@ -583,10 +590,14 @@ def run_ours(args, rank, world, dev):
                    "state_update_GB/s": decode_state_update_bytes(DECODE) / (upd_ms * 1e-3) / 1e9,
                    "state_update_frac_hbm": decode_state_update_bytes(DECODE) / (upd_ms * 1e-3) / 1e9 /
                                             peaks["hbm_gbs"]},
-        "backward": {"workload": BWD.name, "kernel": "chunk_scan_bwd (CUDA cores, fp32 arithmetic)",
+        "backward": {"workload": BWD.name,
+                     "kernels": "chunk states (tcgen05), state passing, chunk gradients (tcgen05), head sums",
                      "ms": bwd_ms, "tokens_per_s": world * btok / (bwd_ms * 1e-3),
                      "GB/s": scan_bwd_bytes_per_token(BWD) * btok / (bwd_ms * 1e-3) / 1e9,
-                     "frac_hbm": scan_bwd_bytes_per_token(BWD) * btok / (bwd_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+                     "frac_hbm": scan_bwd_bytes_per_token(BWD) * btok / (bwd_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "TFLOP/s": scan_bwd_flops_per_token(BWD) * btok / (bwd_ms * 1e-3) / 1e12,
+                     "frac_bf16_peak": scan_bwd_flops_per_token(BWD) * btok / (bwd_ms * 1e-3) / 1e12 /
+                                       peaks["bf16_tflops"]},
         "mixer": {"workload": MIXER.name, "d_model": MIXER_D_MODEL,
                   "kernels": "in_proj (tcgen05 linear), conv1d+SiLU, chunk scan, gated RMSNorm, out_proj",
                   "ms": mix_ms, "tokens_per_s": world * mtok / (mix_ms * 1e-3),
