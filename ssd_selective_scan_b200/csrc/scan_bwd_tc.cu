@@ -246,6 +246,7 @@ constexpr uint32_t kIdS = umma_idesc_bf16(128, 64, true, true);   // B^T (MN) x 
 __global__ void __launch_bounds__(k1::kThreads, 2)
 bwd_states_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmDY,
+                  const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmdS,
                   const TcParams p)
 {
     using namespace k1;
@@ -260,6 +261,7 @@ bwd_states_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     uint64_t* bar_ld = bars + 0;     // X, dY (and B, C for the first head) landed
     uint64_t* bar_w = bars + 1;      // w o X and Ec o dY written in place (row warps)
     uint64_t* bar_mma = bars + 2;    // S^T, dS^T in TMEM (X and dY free)
+    uint64_t* bar_staged = bars + 3; // S^T, dS^T staged in bf16 over X and dY (row warps)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* aborted = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
     float* tot = reinterpret_cast<float*>(smem + kOffVec);
@@ -275,6 +277,7 @@ bwd_states_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         mbar_init(bar_ld, 1);
         mbar_init(bar_w, kEwWarps * 32);
         mbar_init(bar_mma, 1);
+        mbar_init(bar_staged, kEwWarps * 32);
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
@@ -289,12 +292,24 @@ bwd_states_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             prefetch_tensormap(&tmB);
             prefetch_tensormap(&tmC);
             prefetch_tensormap(&tmDY);
+            prefetch_tensormap(&tmS);
+            prefetch_tensormap(&tmdS);
+            // the staged S^T and dS^T tiles of head hh go out by TMA store;
+            // X and dY are reloaded once the store has read them
+            auto store_states = [&](int hh) {
+                const int row = ((bi * p.H + g * hpg + hh) * p.nc + c) * kN;
+                tma_store_3d(&tmS, smem + kOffX, 0, row, 0);
+                tma_store_3d(&tmdS, smem + kOffDY, 0, row, 0);
+                bulk_commit_group();
+                bulk_wait_group_read0();
+            };
             int issued = 0;
             for (int hh = 0; hh < hpg; ++hh) {
                 const int h = g * hpg + hh;
-                // the previous head's products have read its X and dY
-                if (hh > 0 && !mbar_wait_bounded(bar_mma, (uint32_t)(hh - 1) & 1u, kWaitNs, aborted, p.status))
-                    break;
+                if (hh > 0) {
+                    if (!mbar_wait_bounded(bar_staged, (uint32_t)(hh - 1) & 1u, kWaitNs, aborted, p.status)) break;
+                    store_states(hh - 1);
+                }
                 mbar_arrive_expect_tx(bar_ld, hh == 0 ? 6 * kTileHalf : 2 * kTileHalf);
                 tma_load_3d(smem + kOffX, &tmX, h * kP, t0, bi, bar_ld);
                 tma_load_3d(smem + kOffDY, &tmDY, h * kP, t0, bi, bar_ld);
@@ -306,7 +321,10 @@ bwd_states_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 }
                 ++issued;
             }
+            if (issued == hpg && mbar_wait_bounded(bar_staged, (uint32_t)(hpg - 1) & 1u, kWaitNs, aborted, p.status))
+                store_states(hpg - 1);
             if (issued > 0) drain_wait(bar_ld, (uint32_t)(issued - 1) & 1u);
+            bulk_wait_group0();
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -384,18 +402,21 @@ bwd_states_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             mbar_arrive(bar_w);
             ok = mbar_wait_bounded(bar_mma, ph, kWaitNs, aborted, p.status) && ok;
             tc_fence_after_sync();
-            // state row n = i of S^T (part 0) or dS^T (part 1), in bf16
-            uint4* dst = reinterpret_cast<uint4*>((part == 0 ? p.ws_S : p.ws_dS) +
-                                                  ((size_t)chain * p.nc + c) * kStatesDim + (size_t)i * kP);
+            // state row n = i of S^T (part 0) or dS^T (part 1), in bf16, staged
+            // (swizzled as the store's tensor map expects) over X or dY
+            uint8_t* stg = smem + (part == 0 ? kOffX : kOffDY);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 float v[32];
                 tmem_ld32(tmem + lane_off + (uint32_t)(part * 64 + half * 32), v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int k = 0; k < 4; ++k) dst[half * 4 + k] = pack8(v + 8 * k);
+                for (int k = 0; k < 4; ++k) *reinterpret_cast<uint4*>(stg + sw128(i, half * 4 + k)) = pack8(v + 8 * k);
             }
             tc_fence_before_sync();
+            fence_proxy_async_smem();
+            mbar_arrive(bar_staged);
+            (void)chain;
         }
     }
     tc_fence_before_sync();
@@ -412,15 +433,6 @@ bwd_states_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 // Grid (chains, kPassSlices, 2): thread j of slice s owns state elements
 // e = s*1024 + 4j .. +3 of the [n][p] layout (one n, four p); z = 0 walks
 // the entering states forward, z = 1 the state gradients backward.
-__device__ inline void ld_bf16x4(const __nv_bfloat16* src, float (&v)[4])
-{
-    const uint2 q = *reinterpret_cast<const uint2*>(src);
-    v[0] = __uint_as_float(q.x << 16);
-    v[1] = __uint_as_float(q.x & 0xffff0000u);
-    v[2] = __uint_as_float(q.y << 16);
-    v[3] = __uint_as_float(q.y & 0xffff0000u);
-}
-
 __device__ inline void st_bf16x4(__nv_bfloat16* dst, const float (&v)[4])
 {
     __nv_bfloat162 lo = __floats2bfloat162_rn(v[0], v[1]), hi = __floats2bfloat162_rn(v[2], v[3]);
@@ -444,16 +456,42 @@ bwd_pass_kernel(const TcParams p)
 #pragma unroll
     for (int k = 0; k < 4; ++k) v[k] = start ? start[(size_t)chain * kStatesDim + (size_t)(p0 + k) * kN + n] : 0.0f;
     // forward: out[c] = h0_c, h0_{c+1} = 2^cl_c h0_c + S_c;
-    // backward: out[c] = g_c, g_{c-1} = 2^cl_c g_c + dS_c
-    for (int k = 0; k < nc; ++k) {
-        const int c = fwd ? k : nc - 1 - k;
-        const size_t o = base + (size_t)c * kStatesDim;
-        float a[4];
-        ld_bf16x4(inc + o, a);
-        st_bf16x4(out + o, v);
-        const float d = ex2_approx(cl[c]);
+    // backward: out[c] = g_c, g_{c-1} = 2^cl_c g_c + dS_c.
+    // The chunk states and decays are loaded kAhead chunks ahead (a ring
+    // of registers with static indices), so the walk is not one load
+    // latency per chunk.
+    constexpr int kAhead = 4;
+    uint2 ring[kAhead];
+    float dring[kAhead];
+    auto chunk_of = [&](int k) { return fwd ? k : nc - 1 - k; };
 #pragma unroll
-        for (int e = 0; e < 4; ++e) v[e] = fmaf(d, v[e], a[e]);
+    for (int r = 0; r < kAhead; ++r) {
+        if (r < nc) {
+            const int c = chunk_of(r);
+            ring[r] = *reinterpret_cast<const uint2*>(inc + base + (size_t)c * kStatesDim);
+            dring[r] = cl[c];
+        }
+    }
+    for (int k0 = 0; k0 < nc; k0 += kAhead) {
+#pragma unroll
+        for (int r = 0; r < kAhead; ++r) {
+            const int k = k0 + r;
+            if (k < nc) {
+                const int c = chunk_of(k);
+                const uint2 q = ring[r];
+                const float d = ex2_approx(dring[r]);
+                if (k + kAhead < nc) {
+                    const int cn = chunk_of(k + kAhead);
+                    ring[r] = *reinterpret_cast<const uint2*>(inc + base + (size_t)cn * kStatesDim);
+                    dring[r] = cl[cn];
+                }
+                st_bf16x4(out + base + (size_t)c * kStatesDim, v);
+                const float a[4] = {__uint_as_float(q.x << 16), __uint_as_float(q.x & 0xffff0000u),
+                                    __uint_as_float(q.y << 16), __uint_as_float(q.y & 0xffff0000u)};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) v[e] = fmaf(d, v[e], a[e]);
+            }
+        }
     }
     if (!fwd && p.dinit) {
 #pragma unroll
@@ -1109,7 +1147,7 @@ cudaError_t launch_scan_bwd_tc(const ScanBwdArgs& a, cudaStream_t s)
 
     const uint64_t rb = (uint64_t)a.row_stride * 2;
     const uint64_t state_rows = (uint64_t)a.b * a.H * nc * kN;
-    CUtensorMap tmX, tmB, tmC, tmDY, tmHb, tmGb;
+    CUtensorMap tmX, tmB, tmC, tmDY, tmHb, tmGb, tmS, tmdS;
     cudaError_t e;
     if ((e = map3d(&tmX, a.x, (uint64_t)a.H * kP, a.L, a.b, rb)) != cudaSuccess) return e;
     if ((e = map3d(&tmB, a.B, (uint64_t)a.G * kN, a.L, a.b, rb)) != cudaSuccess) return e;
@@ -1117,13 +1155,15 @@ cudaError_t launch_scan_bwd_tc(const ScanBwdArgs& a, cudaStream_t s)
     if ((e = map3d(&tmDY, a.dy, (uint64_t)a.H * kP, a.L, a.b, (uint64_t)a.H * kP * 2)) != cudaSuccess) return e;
     if ((e = map3d(&tmHb, p.ws_hb, kP, state_rows, 1, kP * 2)) != cudaSuccess) return e;
     if ((e = map3d(&tmGb, p.ws_gb, kP, state_rows, 1, kP * 2)) != cudaSuccess) return e;
+    if ((e = map3d(&tmS, p.ws_S, kP, state_rows, 1, kP * 2)) != cudaSuccess) return e;
+    if ((e = map3d(&tmdS, p.ws_dS, kP, state_rows, 1, kP * 2)) != cudaSuccess) return e;
 
     if ((e = cudaMemsetAsync(p.status, 0, 4, s)) != cudaSuccess) return e;
     const dim3 grid((unsigned)nc, (unsigned)(a.b * a.G));
     if ((e = cudaFuncSetAttribute(bwd_states_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, k1::kSmemBytes)) !=
         cudaSuccess)
         return e;
-    bwd_states_kernel<<<grid, k1::kThreads, k1::kSmemBytes, s>>>(tmX, tmB, tmC, tmDY, p);
+    bwd_states_kernel<<<grid, k1::kThreads, k1::kSmemBytes, s>>>(tmX, tmB, tmC, tmDY, tmS, tmdS, p);
     bwd_pass_kernel<<<dim3((unsigned)(a.b * a.H), kPassSlices, 2), kPassThreads, 0, s>>>(p);
     if ((e = cudaFuncSetAttribute(bwd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, k3::kSmemBytes)) !=
         cudaSuccess)
