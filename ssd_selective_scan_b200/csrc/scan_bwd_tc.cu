@@ -511,10 +511,10 @@ constexpr int kThreads = kEwThreads + 64;       // warp 0 producer, 1 MMA, 2..17
 constexpr int kOffB = 0, kOffC = 32768, kOffDY = 65536, kOffG = 81920, kOffR = 98304;
 constexpr int kOffX = kOffR, kOffH = kOffR + 16384, kOffEDY = kOffR + 32768, kOffEX = kOffR + 49152;
 constexpr int kOffM1 = kOffR, kOffM3 = kOffR + 32768;
-// floats, two sets by head parity: cum, dt, sig [128] each, partials
+// floats, two sets by head parity: cum, dt, sig, v [128] each, partials
 // [6][4][128], t1 [16]; then scan scratch [16]; A, D, dt_bias [kMaxHpg]
 constexpr int kOffVec = kOffR + 65536;
-constexpr int kVecSet = 3 * kQ + 24 * kQ + 16;
+constexpr int kVecSet = 4 * kQ + 24 * kQ + 16;
 constexpr int kVecFloats = 2 * kVecSet + 16 + 3 * kMaxHpg;
 constexpr int kOffBar = kOffVec + ((kVecFloats * 4 + 63) / 64) * 64;
 constexpr int kNumBars = 6;
@@ -562,6 +562,7 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     // runs while the next head is under way)
     struct Vec {
         float *cum, *dt, *sig;
+        float* v;                                    // 2^(cum_e - cum_j), e = last column of j's 32-block
         float *row, *rowd, *dd, *dcc, *xgb, *col;   // [4][128] partials
         float* t1;                                   // [16] <g, h0> partials
     };
@@ -571,7 +572,8 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         v.cum = b;
         v.dt = b + kQ;
         v.sig = b + 2 * kQ;
-        v.row = b + 3 * kQ;       // [column quarter][row]: W partials
+        v.v = b + 3 * kQ;
+        v.row = b + 4 * kQ;       // [column quarter][row]: W partials
         v.rowd = v.row + 4 * kQ;  // rowD partials
         v.dd = v.rowd + 4 * kQ;   // dy.x partials
         v.dcc = v.dd + 4 * kQ;    // dC.C partials
@@ -806,6 +808,8 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 v.cum[i] = cum;
                 v.dt[i] = dt;
                 v.sig[i] = sig;
+                // (this warp holds the 32-block of row i: its last row is lane 31)
+                v.v[i] = ex2_approx(__shfl_sync(0xffffffffu, cum, 31) - cum);
             }
             named_bar_sync(kBarEw, kEwThreads);
             const float cum_i = v.cum[i], dt_i = v.dt[i];
@@ -854,35 +858,75 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             ok = mbar_wait_bounded(bar_p1, ph, kWaitNs, aborted, p.status) && ok;
             tc_fence_after_sync();
             {
+                // Column block qs against the row block quad: above the
+                // diagonal the tiles are zero; below it the decay factors
+                // as 2^(cum_i - cum_e) 2^(cum_e - cum_j) (e = the block's
+                // last column, both factors <= 1); on the diagonal one
+                // exponential per element.
                 float w = 0.0f, rowd = 0.0f;
                 const uint32_t half = (uint32_t)(qs >> 1) * kTileHalf;
+                const bool above = qs > quad, below = qs < quad;
+                const float u = below ? ex2_approx(cum_i - v.cum[qs * 32 + 31]) : 0.0f;
 #pragma unroll
                 for (int sub = 0; sub < 2; ++sub) {   // 16 columns at a time
-                    float yx[16], cb[16], col[16];
-                    tmem_ld16(tmem + kColYX + lane_off + (uint32_t)(qs * 32 + sub * 16), yx);
-                    tmem_ld16(tmem + kColCB + lane_off + (uint32_t)(qs * 32 + sub * 16), cb);
-                    tmem_wait_ld();
+                    float cs = 0.0f;
+                    if (above) {
+                        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-                    for (int cc = 0; cc < 2; ++cc) {
-                        float m1[8], m3[8];
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            const int jj = cc * 8 + k;
-                            const int j = qs * 32 + sub * 16 + jj;
-                            const float lm = j <= i ? ex2_approx(cum_i - v.cum[j]) : 0.0f;
-                            const float v2 = lm * yx[jj];
-                            const float v1 = v2 * v.dt[j];
-                            m1[k] = bf16_round(v1);
-                            m3[k] = lm * cb[jj];
-                            w = fmaf(v1, cb[jj], w);
-                            rowd = fmaf(m1[k] - v1, cb[jj], rowd);
-                            col[jj] = v2 * cb[jj];
+                        for (int cc = 0; cc < 2; ++cc) {
+                            const uint32_t o = half + sw128(i, (qs & 1) * 4 + sub * 2 + cc);
+                            *reinterpret_cast<uint4*>(smem + kOffM1 + o) = z;
+                            *reinterpret_cast<uint4*>(smem + kOffM3 + o) = z;
                         }
-                        const uint32_t o = half + sw128(i, (qs & 1) * 4 + sub * 2 + cc);
-                        *reinterpret_cast<uint4*>(smem + kOffM1 + o) = pack8(m1);
-                        *reinterpret_cast<uint4*>(smem + kOffM3 + o) = pack8(m3);
+                    } else {
+                        float yx[16], cb[16], col[16];
+                        tmem_ld16(tmem + kColYX + lane_off + (uint32_t)(qs * 32 + sub * 16), yx);
+                        tmem_ld16(tmem + kColCB + lane_off + (uint32_t)(qs * 32 + sub * 16), cb);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int cc = 0; cc < 2; ++cc) {
+                            const int j0 = qs * 32 + sub * 16 + cc * 8;
+                            float lm[8];
+                            if (below) {
+                                const float4 va = reinterpret_cast<const float4*>(v.v + j0)[0];
+                                const float4 vb = reinterpret_cast<const float4*>(v.v + j0)[1];
+                                const float vv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+                                for (int k = 0; k < 8; ++k) lm[k] = u * vv[k];
+                            } else {
+                                const float4 ca = reinterpret_cast<const float4*>(v.cum + j0)[0];
+                                const float4 cb4 = reinterpret_cast<const float4*>(v.cum + j0)[1];
+                                const float cj[8] = {ca.x, ca.y, ca.z, ca.w, cb4.x, cb4.y, cb4.z, cb4.w};
+#pragma unroll
+                                for (int k = 0; k < 8; ++k) lm[k] = j0 + k <= i ? ex2_approx(cum_i - cj[k]) : 0.0f;
+                            }
+                            const float4 da = reinterpret_cast<const float4*>(v.dt + j0)[0];
+                            const float4 db = reinterpret_cast<const float4*>(v.dt + j0)[1];
+                            const float dj[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+                            float m1[8], m3[8];
+#pragma unroll
+                            for (int k = 0; k < 8; k += 2) {
+                                const int jj = cc * 8 + k;
+                                const float2 v2 = mul2(make_float2(lm[k], lm[k + 1]), make_float2(yx[jj], yx[jj + 1]));
+                                const float2 v1 = mul2(v2, make_float2(dj[k], dj[k + 1]));
+                                const float2 c2 = make_float2(cb[jj], cb[jj + 1]);
+                                m1[k] = bf16_round(v1.x);
+                                m1[k + 1] = bf16_round(v1.y);
+                                const float2 m3p = mul2(make_float2(lm[k], lm[k + 1]), c2);
+                                m3[k] = m3p.x;
+                                m3[k + 1] = m3p.y;
+                                w = fmaf(v1.x, c2.x, fmaf(v1.y, c2.y, w));
+                                rowd = fmaf(m1[k] - v1.x, c2.x, fmaf(m1[k + 1] - v1.y, c2.y, rowd));
+                                const float2 cl2 = mul2(v2, c2);
+                                col[jj] = cl2.x;
+                                col[jj + 1] = cl2.y;
+                            }
+                            const uint32_t o = half + sw128(i, (qs & 1) * 4 + sub * 2 + cc);
+                            *reinterpret_cast<uint4*>(smem + kOffM1 + o) = pack8(m1);
+                            *reinterpret_cast<uint4*>(smem + kOffM3 + o) = pack8(m3);
+                        }
+                        cs = warp_colsum16(col, lane);
                     }
-                    const float cs = warp_colsum16(col, lane);
                     if (lane < 16) v.col[quad * kQ + qs * 32 + sub * 16 + lane] = cs;
                 }
                 v.row[qs * kQ + i] = w;
