@@ -517,7 +517,7 @@ constexpr int kOffVec = kOffR + 65536;
 constexpr int kVecSet = 4 * kQ + 24 * kQ + 16;
 constexpr int kVecFloats = 2 * kVecSet + 16 + 3 * kMaxHpg;
 constexpr int kOffBar = kOffVec + ((kVecFloats * 4 + 63) / 64) * 64;
-constexpr int kNumBars = 6;
+constexpr int kNumBars = 7;
 constexpr int kOffMisc = kOffBar + 8 * kNumBars;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;
 constexpr uint32_t kTmemCols = 512;
@@ -556,6 +556,7 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     uint64_t* bar_e1 = bars + 3;   // M1, M3 written; YX read
     uint64_t* bar_p2 = bars + 4;   // dC, dB, gB, B g^T done
     uint64_t* bar_e2 = bars + 5;   // the head's epilogue has read gB, B g^T and dC
+    uint64_t* bar_p2a = bars + 6;  // gB, B g^T done (the rest of the second products still running)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* aborted = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
     // per-head vectors and partial sums, by head parity (a head's last step
@@ -600,6 +601,7 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         mbar_init(bar_e1, kEwThreads);
         mbar_init(bar_p2, 1);
         mbar_init(bar_e2, kEwThreads);
+        mbar_init(bar_p2a, 1);
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
@@ -678,17 +680,18 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 if (!mbar_wait_bounded(bar_e1, ph, kWaitNs, aborted, p.status)) break;
                 tc_fence_after_sync();
 #pragma unroll
-                for (int k = 0; k < 8; ++k)   // dC += M1 B                 (K = Q)
-                    umma_bf16(tmem + kColDC, desc_k(sM1, k), desc_mn(sB, k), kIdKM128, 1u);
-#pragma unroll
-                for (int k = 0; k < 8; ++k)   // dB += M1^T C  (M1 = dt_j o M2)
-                    umma_bf16(tmem + kColDB, desc_mn(sM1, k), desc_mn(sC, k), kIdMM128, 1u);
-#pragma unroll
                 for (int k = 0; k < 8; ++k)   // gB = M3^T dY
                     umma_bf16(tmem + kColGB, desc_mn(sM3, k), desc_mn(sDY, k), kIdMM64, k > 0);
 #pragma unroll
                 for (int k = 0; k < 8; ++k)   // B g^T                       (g as [n][p], K = N)
                     umma_bf16(tmem + kColBG, desc_k(sB, k), desc_mn(sG, k), kIdKM64, k > 0);
+                umma_commit(bar_p2a);         // dx can start
+#pragma unroll
+                for (int k = 0; k < 8; ++k)   // dC += M1 B                 (K = Q)
+                    umma_bf16(tmem + kColDC, desc_k(sM1, k), desc_mn(sB, k), kIdKM128, 1u);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)   // dB += M1^T C  (M1 = dt_j o M2)
+                    umma_bf16(tmem + kColDB, desc_mn(sM1, k), desc_mn(sC, k), kIdMM128, 1u);
                 umma_commit(bar_p2);
                 ++committed;
             }
@@ -945,31 +948,11 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             const uint4* dyr = reinterpret_cast<const uint4*>(p.dy + rowp);
             const uint4* xr = reinterpret_cast<const uint4*>(p.x + trow * p.row_stride + (size_t)h * kP + qs * 16);
             const uint4 dy0 = dyr[0], dy1 = dyr[1], x0 = xr[0], x1 = xr[1];
-            ok = mbar_wait_bounded(bar_p2, ph, kWaitNs, aborted, p.status) && ok;
+            ok = mbar_wait_bounded(bar_p2a, ph, kWaitNs, aborted, p.status) && ok;
             tc_fence_after_sync();
             {
-                const uint32_t half = (uint32_t)(qs >> 1) * kTileHalf;
-                float dcc = 0.0f;
-#pragma unroll
-                for (int sub = 0; sub < 2; ++sub) {   // 16 columns at a time
-                    float vv[16];
-                    tmem_ld16(tmem + kColDC + lane_off + (uint32_t)(qs * 32 + sub * 16), vv);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int cc = 0; cc < 2; ++cc) {
-                        float cr[8];
-                        unpack8(*reinterpret_cast<const uint4*>(smem + kOffC + half +
-                                                                sw128(i, (qs & 1) * 4 + sub * 2 + cc)),
-                                cr);
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) dcc = fmaf(vv[cc * 8 + k], cr[k], dcc);
-                    }
-                }
-                {   // this head's share of the running dot
-                    const float run = dcc;
-                    dcc = run - prev_dcc;
-                    prev_dcc = run;
-                }
+                // dx and x^T g B from gB and B g^T, while dC and dB are still
+                // on the tensor cores
                 float gb[16], bg[16];
                 tmem_ld16(tmem + kColGB + lane_off + (uint32_t)(qs * 16), gb);
                 tmem_ld16(tmem + kColBG + lane_off + (uint32_t)(qs * 16), bg);
@@ -977,26 +960,41 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 float dxv[16], xgb = 0.0f;
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
-                    float y[8];
+                    float y[8], xv[8];
                     unpack8(cc ? dy1 : dy0, y);
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        dxv[cc * 8 + k] = fmaf(Dh, y[k], dt_i * fmaf(El, bg[cc * 8 + k], gb[cc * 8 + k]));
-                }
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    float xv[8];
                     unpack8(cc ? x1 : x0, xv);
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) xgb = fmaf(xv[k], bg[cc * 8 + k], xgb);
+                    for (int k = 0; k < 8; ++k) {
+                        dxv[cc * 8 + k] = fmaf(Dh, y[k], dt_i * fmaf(El, bg[cc * 8 + k], gb[cc * 8 + k]));
+                        xgb = fmaf(xv[k], bg[cc * 8 + k], xgb);
+                    }
                 }
                 if (valid) {
                     uint4* dst = reinterpret_cast<uint4*>(p.dx + rowp);
                     dst[0] = pack8(dxv);
                     dst[1] = pack8(dxv + 8);
                 }
-                v.dcc[qs * kQ + i] = dcc;
                 v.xgb[qs * kQ + i] = xgb;
+            }
+            ok = mbar_wait_bounded(bar_p2, ph, kWaitNs, aborted, p.status) && ok;
+            tc_fence_after_sync();
+            {
+                // this head's dC.C: the difference of consecutive running dots
+                const uint32_t half = (uint32_t)(qs >> 1) * kTileHalf;
+                float vv[32];
+                tmem_ld32(tmem + kColDC + lane_off + (uint32_t)(qs * 32), vv);
+                tmem_wait_ld();
+                float dcc = 0.0f;
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    float cr[8];
+                    unpack8(*reinterpret_cast<const uint4*>(smem + kOffC + half + sw128(i, (qs & 1) * 4 + cc)), cr);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) dcc = fmaf(vv[cc * 8 + k], cr[k], dcc);
+                }
+                const float run = dcc;
+                v.dcc[qs * kQ + i] = run - prev_dcc;
+                prev_dcc = run;
             }
             tc_fence_before_sync();
             mbar_arrive(bar_e2);   // gB, B g^T and dC read: the next head's products may start
