@@ -73,6 +73,10 @@ CASES = {
     "bf16_tc_weak_decay": (synth.CONFIGS[1].with_(b=1, L=1000, H=4, G=2), dict(a_range=(0.01, 2.0))),
     "bf16_tc_strong_decay": (synth.CONFIGS[1].with_(b=1, L=600, H=4, G=2), dict(a_range=(8.0, 64.0),
                                                                                 dt_range=(-1.0, 1.0))),
+    # the 8B layer's 16 heads per group (the longest head loop), two groups
+    "bf16_tc_group16": (synth.CONFIGS[2].with_(b=1, L=300, H=32, G=2), {}),
+    # one group of 16 heads over 47 chunks (the state passing walks a long chain)
+    "bf16_tc_long_chain_g1": (synth.CONFIGS[1].with_(b=1, L=6000, H=16, G=1), dict(a_range=(0.01, 2.0))),
     # the general (CUDA-core) path in bf16: a state size the tensor-core path does not take
     "bf16_general_n64": (synth.CONFIGS[1].with_(b=2, L=300, H=4, G=2, N=64), {}),
 }
