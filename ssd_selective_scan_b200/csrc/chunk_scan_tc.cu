@@ -46,8 +46,9 @@
 // boundary is finished by the next CTA, which starts from the state the
 // previous CTA published in the workspace.  Each CTA first runs the
 // segment it must publish, last the segment that depends on its
-// predecessor, so the hand-off wait is normally zero.  Every wait (mbarrier
-// or hand-off flag) is bounded (1 s); a CTA that gives up records
+// predecessor, so the hand-off wait is normally zero.  Every wait is
+// bounded: an mbarrier wait by 1 s, a hand-off wait by 1 s plus 16 us per
+// chunk of the chain before the range; a CTA that gives up records
 // SSD_ERR_TIMEOUT in the optional status word and runs to its end without
 // waiting again.
 //
@@ -91,6 +92,7 @@ constexpr int kVecWarp = kEwWarps + 2;   // chunk vectors (dt, cumulative decay)
 constexpr int kThreads = kEwThreads + 96;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr uint64_t kWaitPerChunkNs = 16000;   // hand-off waits: + 16 us per chunk before the range
 constexpr int kPreMax = 32;            // chunks a range's starting state is rebuilt from, at most
 constexpr int kMinRangeLong = 32;      // units per CTA at least, when chains are split across CTAs
 constexpr float kPreCutLog2 = -64.0f;  // accumulated log2 decay below which older tokens are dropped
@@ -766,13 +768,17 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
 #pragma unroll
             for (int p = 0; p < 16; ++p) hv[p] = src ? src[(size_t)(p0 + p) * kN + row] : 0.0f;
         };
-        // the state published by the predecessor CTA (bounded wait on its flag)
+        // the state published by the predecessor CTA (bounded wait on its
+        // flag).  The ranges of a long-memory chain publish one after
+        // another, so the bound allows for the chain's chunks before this
+        // range as well.
         auto load_published = [&](float (&hv)[16]) {
             const int* flag = prm.ws_ctrl + 16 + (ticket - 1);
+            const uint64_t limit = kWaitNs + (uint64_t)rg.startC * kWaitPerChunkNs;
             if (tid == 0 && !*aborted) {
                 const uint64_t t0 = globaltimer_ns();
                 while (ld_acquire_gpu(flag) == 0) {
-                    if (globaltimer_ns() - t0 > kWaitNs) {
+                    if (globaltimer_ns() - t0 > limit) {
                         *aborted = 1;
                         if (prm.status) atomicExch(reinterpret_cast<int*>(prm.status), 4);
                         break;
