@@ -140,6 +140,10 @@ LONG = {
     # the other heads rebuild theirs
     "long_memory_falls_back": (synth.CONFIGS[1].with_(b=2, L=30000, H=4, G=2),
                                dict(a_range=(0.01, 2.0), init_state=True)),
+    # 32 chains of 256 chunks (32 heads in 4 groups): 4 aligned ranges per
+    # chain, 128 CTAs, with an initial state and dt_bias
+    "aligned_ranges_32_heads": (synth.CONFIGS[1].with_(b=1, L=32768, H=32, G=4),
+                                dict(init_state=True, dt_bias=True)),
 }
 
 
