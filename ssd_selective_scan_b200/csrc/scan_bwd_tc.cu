@@ -37,16 +37,19 @@
 //    out exactly: dC_k.C_k - sum_j (bf16(M1) - M1)[k][j] CB[k][j].  (Without
 //    it the large sums of the closed form amplify the rounding.)
 // dB and dC of a group are sums over its heads: one CTA takes the heads of a
-// group in order and its accumulators run on across them in TMEM.  dA, dD and ddt_bias are
-// summed over sequences, chunks and row quarters in a fixed order by a last
-// kernel, so the result is deterministic.
+// group in order and its accumulators run on across them in TMEM.  dA, dD
+// and ddt_bias are summed over sequences, chunks and row quarters in a
+// fixed order by a last kernel, so the result is deterministic.
 //
 // Kernels 1 and 3: one CTA per (chunk, sequence, group), a TMA producer
 // warp, an MMA warp (one thread issues tcgen05.mma; TMEM allocation) and
 // elementwise warps that serve TMEM lanes 32*(warp%4).. (token rows, or
 // state columns n).  Tiles are 128-byte swizzled, loaded by TMA without
-// multicast.  Every mbarrier wait is bounded (1 s); a CTA that gives up
-// sets the timeout flag in the workspace's first word and ends.
+// multicast; kernel 1 writes its bf16 state tiles by TMA store.  In kernel
+// 3 the next head's loads start once the current head's products are done,
+// and a head's per-token step runs while the next head's second products
+// are on the tensor cores.  Every mbarrier wait is bounded (1 s); a CTA that
+// gives up sets the timeout flag in the workspace's first word and ends.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -416,7 +419,6 @@ bwd_states_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             tc_fence_before_sync();
             fence_proxy_async_smem();
             mbar_arrive(bar_staged);
-            (void)chain;
         }
     }
     tc_fence_before_sync();
