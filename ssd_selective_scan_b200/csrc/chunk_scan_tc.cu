@@ -604,7 +604,15 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 mbar_arrive_expect_tx(bar, kBytesX);
                 tma_load_3d(stage(idx) + kStX, &tmX, c.h * kP, c.tok0, c.bi, bar);
             };
+            // (long chains: the heads of a group walk the same chunks in step,
+            // so B and C come from L2 and only X is prefetched; the B and C
+            // prefetches there cost more TMA issue time than they save:
+            // 2.66 -> 2.49 ms on 1 x 262144 tokens, 64 heads)
             auto prefetch_l2 = [&](const Co& c) {
+                if constexpr (kLong) {
+                    tma_prefetch_l2_3d(&tmX, c.h * kP, c.tok0, c.bi);
+                    return;
+                }
                 tma_prefetch_l2_3d(&tmB, c.g * kN, c.tok0, c.bi);
                 tma_prefetch_l2_3d(&tmB, c.g * kN + 64, c.tok0, c.bi);
                 if (!(kLong && c.pre)) {
