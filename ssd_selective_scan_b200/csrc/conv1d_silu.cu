@@ -4,7 +4,7 @@
 // and SiLU from the Nemotron feasibility report, section 1.4).
 //
 // HBM-bound streaming kernel.  Each thread owns 4 adjacent channels (an
-// 8-byte bf16 or 16-byte float vector) and walks a tile of 32 tokens,
+// 8-byte bf16 or 16-byte float vector) and walks a tile of 32 tokens (64 for long sequences),
 // keeping the k-1 previous inputs in registers; the k-1 halo tokens before
 // its tile are re-read (they were just read by the neighbouring tile, so
 // they come from L2).  Tokens move in groups of 8 whose loads are all issued
@@ -24,6 +24,8 @@ namespace ssd {
 
 constexpr int kConvThreads = 128;
 constexpr int kConvTile = 32;   // tokens per thread
+constexpr int kConvTileLong = 64;       // ... for long sequences (fewer halo re-reads, fewer CTAs)
+constexpr int kConvLongTokens = 65536;  // L from which the long tile is used
 constexpr int kGroup = 8;       // tokens loaded together
 constexpr int kCpt = 4;         // channels per thread
 
@@ -143,7 +145,7 @@ __device__ inline void roll_cache(T* cs, const T* xb, int L, int64_t in_stride)
     blk.store(cs);
 }
 
-template <typename T, int K>
+template <typename T, int K, int kTile>
 __global__ void __launch_bounds__(kConvThreads)
 conv1d_silu_kernel(const T* __restrict__ xBC, T* __restrict__ out,
                    const float* __restrict__ w, const float* __restrict__ bias,
@@ -154,7 +156,7 @@ conv1d_silu_kernel(const T* __restrict__ xBC, T* __restrict__ out,
     const int cg = blockIdx.x * kConvThreads + threadIdx.x;
     if (cg >= ngroups) return;
     const int c0 = cg * kCpt;
-    const int t0 = blockIdx.y * kConvTile;
+    const int t0 = blockIdx.y * kTile;
     const int bi = blockIdx.z;
     const T* xb = xBC + (int64_t)bi * L * in_stride + c0;
     T* ob = out + (size_t)bi * L * conv_dim + c0;
@@ -200,7 +202,7 @@ conv1d_silu_kernel(const T* __restrict__ xBC, T* __restrict__ out,
         for (int j = 0; j < K - 1; ++j) V4::decode(V4::load(xb + (int64_t)(t0 - (K - 1) + j) * in_stride), hist[j]);
     }
 
-    const int t1 = min(L, t0 + kConvTile);
+    const int t1 = min(L, t0 + kTile);
     for (int tb = t0; tb < t1; tb += kGroup) {
         typename V4::raw raw[kGroup];
 #pragma unroll
@@ -247,10 +249,19 @@ static cudaError_t launch_conv_k(const void* xBC, void* out, const float* w, con
                                  void* conv_state, int b, int L, int conv_dim, int64_t in_stride, cudaStream_t s)
 {
     const int ngroups = conv_dim / kCpt;
-    dim3 grid((ngroups + kConvThreads - 1) / kConvThreads, (L + kConvTile - 1) / kConvTile, b);
-    conv1d_silu_kernel<T, K><<<grid, kConvThreads, 0, s>>>(
-        static_cast<const T*>(xBC), static_cast<T*>(out), w, bias, static_cast<T*>(conv_state),
-        L, conv_dim, in_stride);
+    // Long sequences take 64-token tiles: 4% faster on 1 x 262144 tokens,
+    // 3% slower on 8 x 2048 (same-GPU A/B)
+    if (L >= kConvLongTokens) {
+        dim3 grid((ngroups + kConvThreads - 1) / kConvThreads, (L + kConvTileLong - 1) / kConvTileLong, b);
+        conv1d_silu_kernel<T, K, kConvTileLong><<<grid, kConvThreads, 0, s>>>(
+            static_cast<const T*>(xBC), static_cast<T*>(out), w, bias, static_cast<T*>(conv_state),
+            L, conv_dim, in_stride);
+    } else {
+        dim3 grid((ngroups + kConvThreads - 1) / kConvThreads, (L + kConvTile - 1) / kConvTile, b);
+        conv1d_silu_kernel<T, K, kConvTile><<<grid, kConvThreads, 0, s>>>(
+            static_cast<const T*>(xBC), static_cast<T*>(out), w, bias, static_cast<T*>(conv_state),
+            L, conv_dim, in_stride);
+    }
     return cudaGetLastError();
 }
 

@@ -31,6 +31,8 @@ def _conv_case(b, L, cd, k, dtype, bias, state, seed):
     (2, 3, 16, 4, False, True),          # call shorter than the conv width
     (1, 37, 24, 3, True, True),
     (2, 70, 32, 2, True, False),
+    # long sequences take 64-token tiles; a ragged last tile, cache in and out
+    (2, 65600, 64, 4, True, True),
 ])
 def test_conv1d_silu_matches_oracle(dtype, b, L, cd, k, bias, state):
     xbc, w, bs, st = _conv_case(b, L, cd, k, dtype, bias, state, seed=1000 + L + cd + k)
