@@ -137,6 +137,7 @@ static cudaError_t launch_su_t(float* state, const void* x, const void* B, const
 // order, so the results are equal bit for bit.
 // ---------------------------------------------------------------------------
 constexpr int kDecThreads = 256;
+constexpr int kDecBlocksPerSm = 3;
 
 template <typename T> __device__ inline float conv_act(float v);
 template <> __device__ inline float conv_act<float>(float v) { return silu_f(v); }
@@ -150,7 +151,7 @@ template <> __device__ inline float conv_act<__nv_bfloat16>(float v)
 }
 
 template <typename T, int N, int K>
-__global__ void __launch_bounds__(kDecThreads)
+__global__ void __launch_bounds__(kDecThreads, kDecBlocksPerSm)
 decode_step_kernel(float* __restrict__ state, T* __restrict__ conv_state, const T* __restrict__ xBC,
                    const float* __restrict__ w, const float* __restrict__ bias,
                    const T* __restrict__ dt_raw, const float* __restrict__ dt_bias,
@@ -163,7 +164,7 @@ decode_step_kernel(float* __restrict__ state, T* __restrict__ conv_state, const 
     constexpr int TPR = NV < 32 ? NV : 32;
     constexpr int VPL = NV / TPR;
     constexpr int RPW = 32 / TPR;
-    constexpr int ROWS = 8;
+    constexpr int ROWS = 8 / VPL;   // 128 bytes of state in flight per thread
     constexpr int kWarps = kDecThreads / 32;
 
     const int g = blockIdx.x % G;
@@ -178,18 +179,20 @@ decode_step_kernel(float* __restrict__ state, T* __restrict__ conv_state, const 
     const int sub = lane / TPR, li = lane % TPR;
     const int rows_per_iter = kWarps * RPW * ROWS;
 
+    // A thread's rows in one pass are p = p0 + r * kRowStep + prow0,
+    // r < ROWS: one base address and compile-time offsets.
+    constexpr int kRowStep = kWarps * RPW;
+    const int prow0 = warp * RPW + sub;
     // the first rows of the first head's state are requested before the
     // conv, so that their latency overlaps it
     float4 st[ROWS][VPL];
-    int prow[ROWS];
     auto load_rows = [&](const float* sh, int p0) {
+        const float4* src = reinterpret_cast<const float4*>(sh + (size_t)(p0 + prow0) * N) + li;
 #pragma unroll
         for (int r = 0; r < ROWS; ++r) {
-            prow[r] = p0 + (r * kWarps + warp) * RPW + sub;
-            if (prow[r] < P) {
+            if (p0 + prow0 + r * kRowStep < P) {
 #pragma unroll
-                for (int v = 0; v < VPL; ++v)
-                    st[r][v] = __ldcs(reinterpret_cast<const float4*>(sh + (size_t)prow[r] * N) + v * TPR + li);
+                for (int v = 0; v < VPL; ++v) st[r][v] = __ldcs(src + r * kRowStep * NV + v * TPR);
             }
         }
     };
@@ -240,10 +243,12 @@ decode_step_kernel(float* __restrict__ state, T* __restrict__ conv_state, const 
         T* yr = y + ((size_t)bi * H + h) * P;
         for (int p0 = 0; p0 < P; p0 += rows_per_iter) {
             if (hl > 0 || p0 > 0) load_rows(sh, p0);
+            float4* dst = reinterpret_cast<float4*>(sh + (size_t)(p0 + prow0) * N) + li;
 #pragma unroll
             for (int r = 0; r < ROWS; ++r) {
-                const bool ok = prow[r] < P;
-                const float xp = ok ? xs[prow[r]] : 0.0f;
+                const int prow = p0 + prow0 + r * kRowStep;
+                const bool ok = prow < P;
+                const float xp = ok ? xs[prow] : 0.0f;
                 const float dtx = dt * xp;
                 float acc = 0.0f;
                 if (ok) {
@@ -258,12 +263,12 @@ decode_step_kernel(float* __restrict__ state, T* __restrict__ conv_state, const 
                         acc = fmaf(cvv[v][1], q.y, acc);
                         acc = fmaf(cvv[v][2], q.z, acc);
                         acc = fmaf(cvv[v][3], q.w, acc);
-                        __stcs(reinterpret_cast<float4*>(sh + (size_t)prow[r] * N) + v * TPR + li, q);
+                        __stcs(dst + r * kRowStep * NV + v * TPR, q);
                     }
                 }
 #pragma unroll
                 for (int o = TPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-                if (ok && li == 0) yr[prow[r]] = io<T>::from_f(fmaf(Dh, xp, acc));
+                if (ok && li == 0) yr[prow] = io<T>::from_f(fmaf(Dh, xp, acc));
             }
         }
     }
