@@ -322,6 +322,10 @@ bwd_states_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     tma_load_3d(smem + kOffC, &tmC, g * kN, t0, bi, bar_ld);
                     tma_load_3d(smem + kOffC + kTileHalf, &tmC, g * kN + 64, t0, bi, bar_ld);
                 }
+                if (hh + 1 < hpg) {   // the next head's tiles into L2 meanwhile
+                    tma_prefetch_l2_3d(&tmX, (h + 1) * kP, t0, bi);
+                    tma_prefetch_l2_3d(&tmDY, (h + 1) * kP, t0, bi);
+                }
                 ++issued;
             }
             if (issued == hpg && mbar_wait_bounded(bar_staged, (uint32_t)(hpg - 1) & 1u, kWaitNs, aborted, p.status))
@@ -639,6 +643,12 @@ bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     tma_load_3d(smem + kOffB + kTileHalf, &tmB, g * kN + 64, t0, bi, bar_ld);
                     tma_load_3d(smem + kOffC, &tmC, g * kN, t0, bi, bar_ld);
                     tma_load_3d(smem + kOffC + kTileHalf, &tmC, g * kN + 64, t0, bi, bar_ld);
+                }
+                if (hh + 1 < hpg) {   // the next head's tiles into L2 while this head computes
+                    tma_prefetch_l2_3d(&tmX, (h + 1) * kP, t0, bi);
+                    tma_prefetch_l2_3d(&tmDY, (h + 1) * kP, t0, bi);
+                    tma_prefetch_l2_3d(&tmHb, 0, row + p.nc * kN, 0);
+                    tma_prefetch_l2_3d(&tmGb, 0, row + p.nc * kN, 0);
                 }
                 ++issued;
             }
