@@ -219,6 +219,7 @@ struct Params {
     __nv_bfloat16* y;
     float* final_state;
     int L, H, G, nc, nslots;   // L: tokens per sequence (dense) or in the packed dimension (ragged)
+    int Hf;                    // heads per sequence (H counts head pairs in the pair kernel)
     int units;                 // dense batches: units in the list
     FastDiv fnc, fH, fHG;      // division by nc, H, H / G
     int* ws_ctrl;        // [0] ticket, [16 + t] hand-off flag of boundary t
@@ -1098,6 +1099,668 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     }
 }
 
+// ---------------------------------------------------------------------------
+// Head pairs.  When a group has an even number of heads, an item is two
+// heads h, h + 1 of one group over one chunk.  They share B, C and G, so B
+// and C are loaded and C B^T computed once per pair, and their states sit
+// side by side in TMEM (lane n, columns [h p | h+1 p]), so that both state
+// products are one N = 128 MMA chain and so are both C h^T.  The elementwise
+// warps run one chain of steps per pair rather than one per head.
+//   TMEM: G [0,128); M of the two heads [128,256) (bf16 pairs); Y of the two
+//   heads [256,384): C h^T, scaled in place by 2^(cl_i) by the elementwise
+//   warps, then M X accumulated onto it, so Y = y; the state pair [384,512).
+//   Shared memory: one B/C buffer, reloaded once the item's last product
+//   reading it (C h^T) is done; two X stages holding both heads' tiles, over
+//   which y is staged; the bf16 state pair; w o X of both heads.
+// Per item the MMA warp issues the state product once the state is
+// released, C h^T once the previous item's y has been read from TMEM, both
+// heads' M X once the masked tiles and the scaled C h^T are in TMEM, then
+// the next item's G.  The elementwise warps release the state, read the
+// previous y, build both masked tiles from one read of G and scale C h^T.
+// Elementwise warp w serves TMEM lanes 32*(w%4).. and column quarter w/4:
+// for the state, w o X and y, quarter q is head q/2, columns p of
+// 32*(q%2)..; for the masked tiles, 8 columns of every 32-token block, for
+// both heads.
+// ---------------------------------------------------------------------------
+namespace pr {
+constexpr int kStB = 0, kStC = 32768;       // the B/C buffer, two 16 KB halves each
+constexpr int kOffX = 65536;                 // two X stages [128 tok][h p | h+1 p]
+constexpr int kXStage = 32768;
+constexpr int kOffHB = kOffX + 2 * kXStage;  // bf16 state pair [128 n][h p | h+1 p]
+constexpr int kOffWX = kOffHB + 32768;       // w o X of both heads [128 tok][h p | h+1 p]
+constexpr int kOffVec = kOffWX + 32768;      // per parity and head: cl, dt, v (float[128] each)
+constexpr int kVecHead = 3 * kQ, kVecSet = 2 * kVecHead;
+constexpr int kOffBar = kOffVec + 2 * kVecSet * 4;
+constexpr int kNumBars = 13;
+constexpr int kOffMisc = kOffBar + 8 * kNumBars;
+constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+constexpr uint32_t kColG = 0, kColM = 128, kColY = 256, kColH = 384;
+constexpr uint32_t kIdYo = umma_idesc_bf16(128, 128, false, true);   // C (K-maj) x state pair (MN-maj)
+constexpr uint32_t kIdS = umma_idesc_bf16(128, 128, true, true);     // B^T (MN-maj) x (w o X) pair (MN-maj)
+static_assert(kSmemBytes <= 232448, "shared memory");
+}  // namespace pr
+
+template <bool kLong>
+__global__ void __launch_bounds__(kThreads, 1)
+chunk_scan_tc_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
+                          const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY,
+                          const Params prm)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + pr::kOffBar);
+    uint64_t* bar_ld = bars + 0;        // B (and C) landed in the B/C buffer (TMA)
+    uint64_t* bar_ldx = bars + 1;       // [2]: stage's X landed (TMA)
+    uint64_t* bar_vec = bars + 3;       // chunk vectors published (vector warp)
+    uint64_t* bar_sready = bars + 4;    // bf16 state, w o X and decayed state ready (elementwise warps)
+    uint64_t* bar_m4 = bars + 5;        // state product done
+    uint64_t* bar_yread = bars + 6;     // previous item's y read from TMEM (elementwise warps)
+    uint64_t* bar_myo = bars + 7;       // C h^T done, and every earlier product: the B/C buffer is free
+    uint64_t* bar_m1 = bars + 8;        // G done
+    uint64_t* bar_mready = bars + 9;    // masked tiles and scaled C h^T in TMEM; G read (elementwise warps)
+    uint64_t* bar_m2 = bars + 10;       // M X done: y in TMEM
+    uint64_t* bar_ystaged = bars + 11;  // [2]: y staged in the stage's X buffer (elementwise warps)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + pr::kOffMisc);
+    volatile int* aborted = reinterpret_cast<volatile int*>(smem + pr::kOffMisc + 4);
+    int* ticket_slot = reinterpret_cast<int*>(smem + pr::kOffMisc + 8);
+    const int L = prm.L, Hf = prm.Hf;
+
+    if (tid == 0) {
+        *aborted = 0;
+        mbar_init(bar_ld, 1);
+        mbar_init(bar_ldx, 1);
+        mbar_init(bar_ldx + 1, 1);
+        mbar_init(bar_vec, 1);
+        mbar_init(bar_sready, kEwThreads);
+        mbar_init(bar_m4, 1);
+        mbar_init(bar_yread, kEwThreads);
+        mbar_init(bar_myo, 1);
+        mbar_init(bar_m1, 1);
+        mbar_init(bar_mready, kEwThreads);
+        mbar_init(bar_m2, 1);
+        mbar_init(bar_ystaged, kEwThreads);
+        mbar_init(bar_ystaged + 1, kEwThreads);
+        fence_mbar_init();
+        *ticket_slot = atomicAdd(prm.ws_ctrl, 1);
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const int ticket = *ticket_slot;
+    const Tabs tabs{nullptr, nullptr};
+    const Range rg = make_range<false, kLong>(prm, tabs, ticket, prm.units);
+    auto group_of = [&](const Item& it) { return (int)prm.fHG.div((uint32_t)it.h); };
+    auto xstage = [&](int idx) { return smem + pr::kOffX + (idx & 1) * pr::kXStage; };
+    // per parity and head: cl, dt, v
+    auto vecs = [&](int parity, int hd) {
+        return reinterpret_cast<float*>(smem + pr::kOffVec) + parity * pr::kVecSet + hd * pr::kVecHead;
+    };
+
+    if (warp == kMmaWarp) {
+        // ------------------------------------------------------------------
+        // MMA warp (one thread)
+        // ------------------------------------------------------------------
+        if (lane == 0 && rg.count > 0) {
+            const uint32_t sbc = smem_u32(smem);
+            const uint64_t dCk = desc_kmajor(sbc + pr::kStC, 0), dBk = desc_kmajor(sbc + pr::kStB, 0);
+            const uint64_t dBmn = desc_mnmajor(sbc + pr::kStB, 0);
+            const uint64_t dHB = desc_mnmajor(smem_u32(smem + pr::kOffHB), 0);
+            const uint64_t dWX = desc_mnmajor(smem_u32(smem + pr::kOffWX), 0);
+            const uint64_t dX0 = desc_mnmajor(smem_u32(smem + pr::kOffX), 0);
+            constexpr uint64_t kXStep = (uint64_t)(pr::kXStage >> 4), kHalfStep = (uint64_t)(kTileHalf >> 4);
+            auto kstep_k = [](int k) -> uint64_t { return (uint64_t)(((k >> 2) * kTileHalf + (k & 3) * 32u) >> 4); };
+            auto kstep_mn = [](int k) -> uint64_t { return (uint64_t)((k * 2048u) >> 4); };
+            // G = C B^T of item idx (a state-only item has none; the commit stays)
+            auto next_G = [&](int idx) {
+                mbar_wait_bounded(bar_ld, (uint32_t)idx & 1u, kWaitNs, aborted, prm.status);
+                tc_fence_after_sync();
+                if (!(kLong && rg.is_pre(idx))) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        umma_bf16(tmem + pr::kColG, dCk + kstep_k(k), dBk + kstep_k(k), kIdG, k > 0);
+                }
+                umma_commit(bar_m1);
+            };
+            next_G(0);
+            for (int idx = 0; idx < rg.count; ++idx) {
+                const uint32_t ph = (uint32_t)idx & 1u;
+                const bool pre = kLong && rg.is_pre(idx);
+                const uint32_t acc0 = pre && idx == rg.pre_begin() ? 0u : 1u;
+                mbar_wait_bounded(bar_sready, ph, kWaitNs, aborted, prm.status);
+                tc_fence_after_sync();
+#pragma unroll
+                for (int k = 0; k < 8; ++k)   // [h | h+1] += B^T (w o X)   (the states already decayed)
+                    umma_bf16(tmem + pr::kColH, dBmn + kstep_mn(k), dWX + kstep_mn(k), pr::kIdS, k > 0 ? 1u : acc0);
+                umma_commit(bar_m4);
+                mbar_wait_bounded(bar_yread, ph, kWaitNs, aborted, prm.status);
+                tc_fence_after_sync();
+                if (!pre) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)   // Y = C [h | h+1]^T
+                        umma_bf16(tmem + pr::kColY, dCk + kstep_k(k), dHB + kstep_mn(k), pr::kIdYo, k > 0);
+                }
+                umma_commit(bar_myo);
+                mbar_wait_bounded(bar_mready, ph, kWaitNs, aborted, prm.status);
+                tc_fence_after_sync();
+                if (!pre) {
+                    const uint64_t dX = dX0 + (idx & 1) * kXStep;
+#pragma unroll
+                    for (int hd = 0; hd < 2; ++hd)
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)   // Y += M X, per head (M from TMEM)
+                            umma_bf16_tmem_a(tmem + pr::kColY + (uint32_t)hd * 64u,
+                                             tmem + pr::kColM + (uint32_t)hd * 64u + (uint32_t)k * 8u,
+                                             dX + (uint64_t)hd * kHalfStep + kstep_mn(k), kIdYd, 1u);
+                }
+                umma_commit(bar_m2);
+                if (idx + 1 < rg.count) next_G(idx + 1);
+            }
+        }
+        __syncwarp();
+    } else if (warp == kProdWarp) {
+        // ------------------------------------------------------------------
+        // producer warp (one thread)
+        // ------------------------------------------------------------------
+        if (lane == 0 && rg.count > 0) {
+            struct Co {
+                int g, h, tok0, bi;   // h: the pair's first head
+                bool pre;
+            };
+            int hint = rg.sB0;
+            auto coord = [&](int idx) {
+                Co c{0, 0, 0, 0, false};
+                if (idx < rg.count) {
+                    const Item it = item_at<false, kLong>(prm, tabs, rg, idx, hint);
+                    c = Co{group_of(it), 2 * it.h, it.tok0, it.bi, kLong && it.pre};
+                }
+                return c;
+            };
+            auto issue_bc = [&](const Co& c) {
+                mbar_arrive_expect_tx(bar_ld, c.pre ? kBytesBC / 2 : kBytesBC);
+                tma_load_3d(smem + pr::kStB, &tmB, c.g * kN, c.tok0, c.bi, bar_ld);
+                tma_load_3d(smem + pr::kStB + kTileHalf, &tmB, c.g * kN + 64, c.tok0, c.bi, bar_ld);
+                if (!c.pre) {
+                    tma_load_3d(smem + pr::kStC, &tmC, c.g * kN, c.tok0, c.bi, bar_ld);
+                    tma_load_3d(smem + pr::kStC + kTileHalf, &tmC, c.g * kN + 64, c.tok0, c.bi, bar_ld);
+                }
+            };
+            auto issue_x = [&](int idx, const Co& c) {
+                uint64_t* bar = bar_ldx + (idx & 1);
+                mbar_arrive_expect_tx(bar, 2 * kBytesX);
+                tma_load_3d(xstage(idx), &tmX, c.h * kP, c.tok0, c.bi, bar);
+                tma_load_3d(xstage(idx) + kTileHalf, &tmX, c.h * kP + kP, c.tok0, c.bi, bar);
+            };
+            // (long chains: a group's pairs walk the same chunks in step, so
+            // B and C come from L2 and only X is prefetched)
+            auto prefetch_l2 = [&](const Co& c) {
+                tma_prefetch_l2_3d(&tmX, c.h * kP, c.tok0, c.bi);
+                tma_prefetch_l2_3d(&tmX, c.h * kP + kP, c.tok0, c.bi);
+                if constexpr (!kLong) {
+                    tma_prefetch_l2_3d(&tmB, c.g * kN, c.tok0, c.bi);
+                    tma_prefetch_l2_3d(&tmB, c.g * kN + 64, c.tok0, c.bi);
+                    tma_prefetch_l2_3d(&tmC, c.g * kN, c.tok0, c.bi);
+                    tma_prefetch_l2_3d(&tmC, c.g * kN + 64, c.tok0, c.bi);
+                }
+            };
+            prefetch_tensormap(&tmX);
+            prefetch_tensormap(&tmB);
+            prefetch_tensormap(&tmC);
+            prefetch_tensormap(&tmY);
+            Co c0 = coord(0), c1 = coord(1), c2 = coord(2), c3 = coord(3);   // items idx .. idx + 3
+            issue_bc(c0);
+            issue_x(0, c0);
+            if (rg.count > 1) {
+                issue_x(1, c1);
+                prefetch_l2(c1);
+            }
+            if (rg.count > 2) prefetch_l2(c2);
+            for (int idx = 0; idx < rg.count; ++idx) {
+                const uint32_t sph = (uint32_t)(idx >> 1) & 1u;
+                // C h^T of item idx, the last product reading B and C, is done
+                mbar_wait_bounded(bar_myo, (uint32_t)idx & 1u, kWaitNs, aborted, prm.status);
+                if (idx + 1 < rg.count) issue_bc(c1);
+                // y of item idx is staged in its X stage: store it, then
+                // reload the stage once the stores have read it
+                mbar_wait_bounded(bar_ystaged + (idx & 1), sph, kWaitNs, aborted, prm.status);
+                if (!c0.pre) {
+                    tma_store_3d(&tmY, xstage(idx), c0.h * kP, c0.tok0, c0.bi);
+                    tma_store_3d(&tmY, xstage(idx) + kTileHalf, c0.h * kP + kP, c0.tok0, c0.bi);
+                    bulk_commit_group();
+                    bulk_wait_group_read0();
+                }
+                if (idx + 2 < rg.count) issue_x(idx + 2, c2);
+                if (idx + 3 < rg.count) prefetch_l2(c3);
+                c0 = c1;
+                c1 = c2;
+                c2 = c3;
+                c3 = coord(idx + 4);
+            }
+            bulk_wait_group0();
+        }
+        __syncwarp();
+    } else if (warp == kVecWarp) {
+        // ------------------------------------------------------------------
+        // vector warp: both heads' dt, cumulative decay and off-diagonal
+        // column factors (as in the one-head kernel), one chunk ahead
+        // ------------------------------------------------------------------
+        struct DtIn {
+            float a2[2], bias[2];
+            int nvalid;
+            bool pre, pre_first;
+            __nv_bfloat16 dt[2][4];
+        };
+        int hint = rg.sB0;
+        auto load_dt = [&](int idx) {
+            DtIn in;
+            const Item it = item_at<false, kLong>(prm, tabs, rg, idx, hint);
+            const int h0 = 2 * it.h;
+#pragma unroll
+            for (int hd = 0; hd < 2; ++hd) {
+                in.a2[hd] = prm.A[h0 + hd] * 1.4426950408889634f;
+                in.bias[hd] = prm.dt_bias ? prm.dt_bias[h0 + hd] : 0.0f;
+            }
+            const __nv_bfloat16* dp = prm.dt_raw + ((size_t)it.bi * L + it.tok0 + lane * 4) * Hf + h0;
+            in.nvalid = it.nvalid - lane * 4;
+            in.pre = it.pre;
+            in.pre_first = it.pre_first;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+                for (int hd = 0; hd < 2; ++hd)
+                    in.dt[hd][k] = k < in.nvalid ? dp[(size_t)k * Hf + hd] : __float2bfloat16_rn(0.0f);
+            return in;
+        };
+        float vcl[2][4], vdt[2][4], vv[2][4];
+        float lrun[2] = {0.0f, 0.0f};
+        auto compute_vecs = [&](const DtIn& in) {
+#pragma unroll
+            for (int hd = 0; hd < 2; ++hd) {
+                float run = 0.0f;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    vdt[hd][k] = k < in.nvalid ? softplus_fast(__bfloat162float(in.dt[hd][k]) + in.bias[hd]) : 0.0f;
+                    run += vdt[hd][k] * in.a2[hd];
+                    vcl[hd][k] = run;
+                }
+                float incl = run;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float v = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += v;
+                }
+                const float excl = incl - run;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) vcl[hd][k] += excl;
+                if (kLong && in.pre) {
+                    if (in.pre_first) lrun[hd] = 0.0f;
+                    const float cl_last = __shfl_sync(0xffffffffu, vcl[hd][3], 31);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) vdt[hd][k] = ex2_approx(lrun[hd] + cl_last - vcl[hd][k]) * vdt[hd][k];
+                    lrun[hd] += cl_last;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) vv[hd][k] = lrun[hd];
+                    continue;
+                }
+                const float cl_e = __shfl_sync(0xffffffffu, vcl[hd][3], lane | 7);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) vv[hd][k] = ex2_approx(cl_e - vcl[hd][k]) * vdt[hd][k];
+            }
+        };
+        auto publish_vecs = [&](int idx) {
+#pragma unroll
+            for (int hd = 0; hd < 2; ++hd) {
+                float* b = vecs(idx & 1, hd);
+                reinterpret_cast<float4*>(b)[lane] = make_float4(vcl[hd][0], vcl[hd][1], vcl[hd][2], vcl[hd][3]);
+                reinterpret_cast<float4*>(b + kQ)[lane] = make_float4(vdt[hd][0], vdt[hd][1], vdt[hd][2], vdt[hd][3]);
+                reinterpret_cast<float4*>(b + 2 * kQ)[lane] = make_float4(vv[hd][0], vv[hd][1], vv[hd][2], vv[hd][3]);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_vec);
+        };
+        if (rg.count > 0) {
+            DtIn in = load_dt(0);
+            compute_vecs(in);
+            publish_vecs(0);
+            if (rg.count > 1) {
+                in = load_dt(1);
+                compute_vecs(in);
+            }
+            if (rg.count > 2) in = load_dt(2);
+            for (int idx = 0; idx + 1 < rg.count; ++idx) {
+                // vectors idx - 1 were last read before the masked tiles of
+                // item idx - 1 were ready, earlier than this item's release
+                if (lane == 0) mbar_wait_bounded(bar_sready, (uint32_t)idx & 1u, kWaitNs, aborted, prm.status);
+                __syncwarp();
+                publish_vecs(idx + 1);
+                if (idx + 2 < rg.count) {
+                    compute_vecs(in);
+                    if (idx + 3 < rg.count) in = load_dt(idx + 3);
+                }
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------------
+        // elementwise warps
+        // ------------------------------------------------------------------
+        const int quad = warp & 3;          // TMEM lane quadrant
+        const int quarter = warp >> 2;      // column quarter
+        const int row = quad * 32 + lane;   // token row i / state column n
+        const int hd = quarter >> 1;        // this thread's head of the pair (state, w o X, y)
+        const int pq = (quarter & 1) * 32;  // its 32 columns p of that head
+        const int ch0 = pq >> 3;            // their first 16-byte chunk in a 128-byte row
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const uint32_t tH = tmem + pr::kColH + (uint32_t)(hd * 64 + pq) + lane_off;
+        const uint32_t tY = tmem + pr::kColY + (uint32_t)(hd * 64 + pq) + lane_off;
+        uint8_t* sHB = smem + pr::kOffHB + hd * kTileHalf;
+        uint8_t* sWX = smem + pr::kOffWX + hd * kTileHalf;
+        constexpr size_t kPN = (size_t)kP * kN;
+
+        // the initial state of this thread's head of pair chain ch (32
+        // columns p of state column n = row), or zeros
+        auto load_init = [&](int ch, float (&hv)[32]) {
+            const int seq = (int)prm.fH.div((uint32_t)ch);
+            const int h = 2 * (ch - seq * prm.H) + hd;
+            const float* src = prm.init_state ? prm.init_state + ((size_t)seq * Hf + h) * kPN : nullptr;
+#pragma unroll
+            for (int p = 0; p < 32; ++p) hv[p] = src ? src[(size_t)(pq + p) * kN + row] : 0.0f;
+        };
+        auto load_published = [&](float (&hv)[32]) {
+            const int* flag = prm.ws_ctrl + 16 + (ticket - 1);
+            const uint64_t limit = kWaitNs + (uint64_t)rg.startC * kWaitPerChunkNs;
+            if (tid == 0 && !*aborted) {
+                const uint64_t t0 = globaltimer_ns();
+                while (ld_acquire_gpu(flag) == 0) {
+                    if (globaltimer_ns() - t0 > limit) {
+                        *aborted = 1;
+                        if (prm.status) atomicExch(reinterpret_cast<int*>(prm.status), 4);
+                        break;
+                    }
+                }
+            }
+            named_bar_sync(kEwBarrier, kEwThreads);
+            const float* src = prm.ws_states + ((size_t)(ticket - 1) * 2 + hd) * kPN;
+#pragma unroll
+            for (int p = 0; p < 32; ++p) hv[p] = __ldcg(src + (size_t)(pq + p) * kN + row);
+        };
+        bool pre_ok = false;
+        auto segment_state = [&](const Item& it, float (&hv)[32]) {
+            if (it.depend) {
+                if (kLong && pre_ok) {
+                    tmem_ld32(tH, hv);
+                    tmem_wait_ld();
+                } else {
+                    load_published(hv);
+                }
+            } else {
+                load_init(it.chain, hv);
+            }
+        };
+        // y of item j (Y, this thread's head and columns), staged over the
+        // item's X tiles for the producer's TMA stores; then (unless it is
+        // the last) the arrival that lets C h^T of the next item into Y
+        bool prev_pre = false;
+        auto y_epilogue = [&](int j, bool release) {
+            mbar_wait_bounded(bar_m2, (uint32_t)j & 1u, kWaitNs, aborted, prm.status);
+            if (kLong && prev_pre) {
+                mbar_arrive(bar_ystaged + (j & 1));
+                if (release) mbar_arrive(bar_yread);
+                return;
+            }
+            tc_fence_after_sync();
+            float yv[32];
+            tmem_ld32(tY, yv);
+            tmem_wait_ld();
+            if (release) {
+                tc_fence_before_sync();
+                mbar_arrive(bar_yread);
+            }
+            uint8_t* xs = xstage(j) + hd * kTileHalf;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(xs + sw128(row, ch0 + q)) = pack_bf16x8(&yv[q * 8]);
+            fence_proxy_async_smem();
+            mbar_arrive(bar_ystaged + (j & 1));
+        };
+
+        int hint = rg.sB0;
+        for (int idx = 0; idx < rg.count; ++idx) {
+            const Item it = item_at<false, kLong>(prm, tabs, rg, idx, hint);
+            const int h0 = 2 * it.h;
+            const uint32_t ph = (uint32_t)idx & 1u;
+            uint8_t* xs = xstage(idx) + hd * kTileHalf;
+            const float* cv = vecs(idx & 1, hd);
+
+            if (kLong && it.pre) {
+                // ----------------------------------------------------------
+                // state-only item: w' o X of both heads
+                // ----------------------------------------------------------
+                mbar_wait_bounded(bar_vec, ph, kWaitNs, aborted, prm.status);
+                const float wj = cv[kQ + row];
+                const float lsum = cv[2 * kQ];   // this head's log2 decay from the chunk's start to the rebuilt state
+                const bool both_cut = vecs(idx & 1, 0)[2 * kQ] <= kPreCutLog2 && vecs(idx & 1, 1)[2 * kQ] <= kPreCutLog2;
+                if (idx > 0)
+                    mbar_wait_bounded(bar_m4, (uint32_t)(idx - 1) & 1u, kWaitNs, aborted, prm.status);
+                mbar_wait_bounded(bar_ldx + (idx & 1), (uint32_t)(idx >> 1) & 1u, kWaitNs, aborted, prm.status);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float v[8];
+                    unpack_bf16x8(*reinterpret_cast<const uint4*>(xs + sw128(row, ch0 + q)), v);
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) {
+                        const float2 r = mul2(make_float2(v[e], v[e + 1]), make_float2(wj, wj));
+                        v[e] = r.x;
+                        v[e + 1] = r.y;
+                    }
+                    *reinterpret_cast<uint4*>(sWX + sw128(row, ch0 + q)) = pack_bf16x8(v);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before_sync();
+                mbar_arrive(bar_sready);
+                if (idx > 0) y_epilogue(idx - 1, true);
+                else mbar_arrive(bar_yread);
+                mbar_wait_bounded(bar_m1, ph, kWaitNs, aborted, prm.status);
+                mbar_wait_bounded(bar_myo, ph, kWaitNs, aborted, prm.status);
+                tc_fence_before_sync();
+                mbar_arrive(bar_mready);   // (no masked tiles)
+                if (it.pre_last) {
+                    const bool from_start = rg.startC - rg.npre == 0;
+                    pre_ok = from_start || both_cut;
+                    mbar_wait_bounded(bar_m4, ph, kWaitNs, aborted, prm.status);
+                    tc_fence_after_sync();
+                    if (from_start && prm.init_state) {
+                        // + the initial state decayed over the walk, 16 columns at a time
+                        const int seq = (int)prm.fH.div((uint32_t)it.chain);
+                        const float* src =
+                            prm.init_state + ((size_t)seq * Hf + 2 * (it.chain - seq * prm.H) + hd) * kPN;
+                        const float d0 = ex2_approx(lsum);
+#pragma unroll 1
+                        for (int hp = 0; hp < 32; hp += 16) {
+                            float hs[16];
+                            tmem_ld16(tH + (uint32_t)hp, hs);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int p = 0; p < 16; ++p) hs[p] = fmaf(d0, src[(size_t)(pq + hp + p) * kN + row], hs[p]);
+                            tmem_st16(tH + (uint32_t)hp, hs);
+                            tmem_wait_st();
+                        }
+                    }
+                }
+                prev_pre = true;
+                continue;
+            }
+
+            // 1. the state entering item idx (fp32; this thread's head, 32
+            //    columns p of state column n = row)
+            float hv[32];
+            if (it.seg_start) {
+                segment_state(it, hv);
+            } else {
+                // the previous state product is done (w o X is free), and
+                // so is its C h^T (waited for before its masked tiles were
+                // released), so the bf16 state may be rewritten
+                mbar_wait_bounded(bar_m4, (uint32_t)(idx - 1) & 1u, kWaitNs, aborted, prm.status);
+                tc_fence_after_sync();
+                tmem_ld32(tH, hv);
+                tmem_wait_ld();
+            }
+            // 2. its bf16 copy for C h^T
+#pragma unroll
+            for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(sHB + sw128(row, ch0 + q)) = pack_bf16x8(&hv[q * 8]);
+            // 3. the decayed state back into TMEM and w o X
+            mbar_wait_bounded(bar_vec, ph, kWaitNs, aborted, prm.status);
+            const float cl_i = cv[row];
+            const float cl_last = cv[kQ - 1];
+            {
+                const float decay = ex2_approx(cl_last);
+#pragma unroll
+                for (int p = 0; p < 32; p += 2) {
+                    const float2 r = mul2(make_float2(hv[p], hv[p + 1]), make_float2(decay, decay));
+                    hv[p] = r.x;
+                    hv[p + 1] = r.y;
+                }
+                tmem_st32(tH, hv);
+            }
+            mbar_wait_bounded(bar_ldx + (idx & 1), (uint32_t)(idx >> 1) & 1u, kWaitNs, aborted, prm.status);
+            {
+                const float wj = ex2_approx(cl_last - cl_i) * cv[kQ + row];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float v[8];
+                    unpack_bf16x8(*reinterpret_cast<const uint4*>(xs + sw128(row, ch0 + q)), v);
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) {
+                        const float2 r = mul2(make_float2(v[e], v[e + 1]), make_float2(wj, wj));
+                        v[e] = r.x;
+                        v[e + 1] = r.y;
+                    }
+                    *reinterpret_cast<uint4*>(sWX + sw128(row, ch0 + q)) = pack_bf16x8(v);
+                }
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            mbar_arrive(bar_sready);   // the state product can start
+
+            // 4. y of the previous item; then C h^T of this one may go into Y
+            if (idx > 0) y_epilogue(idx - 1, true);
+            else mbar_arrive(bar_yread);
+
+            // 5. both heads' masked tiles from one read of G (column block jb
+            //    is zero above the row quadrant's diagonal block; of every
+            //    block, column quarter `quarter` takes 8 columns)
+            mbar_wait_bounded(bar_m1, ph, kWaitNs, aborted, prm.status);
+            tc_fence_after_sync();
+            {
+                float gv[4][8];
+#pragma unroll
+                for (int jb = 0; jb < 4; ++jb)
+                    if (jb <= quad) tmem_ld8(tmem + pr::kColG + lane_off + (uint32_t)(jb * 32 + quarter * 8), gv[jb]);
+                tmem_wait_ld();
+#pragma unroll 1
+                for (int hm = 0; hm < 2; ++hm) {
+                    const float* cm = vecs(idx & 1, hm);
+                    const float cl_m = cm[row];
+                    const float Dm = prm.D ? prm.D[h0 + hm] : 0.0f;
+#pragma unroll
+                    for (int jb = 0; jb < 4; ++jb) {
+                        const int j0 = jb * 32 + quarter * 8;
+                        uint32_t w[4] = {0u, 0u, 0u, 0u};
+                        if (jb < quad) {
+                            const float u = ex2_approx(cl_m - cm[jb * 32 + 31]);
+                            const float4 va = reinterpret_cast<const float4*>(cm + 2 * kQ + j0)[0];
+                            const float4 vb = reinterpret_cast<const float4*>(cm + 2 * kQ + j0)[1];
+                            const float vv8[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 uv = mul2(make_float2(u, u), make_float2(vv8[2 * e], vv8[2 * e + 1]));
+                                const float2 m = mul2(make_float2(gv[jb][2 * e], gv[jb][2 * e + 1]), uv);
+                                __nv_bfloat162 b2 = __floats2bfloat162_rn(m.x, m.y);
+                                w[e] = *reinterpret_cast<uint32_t*>(&b2);
+                            }
+                        } else if (jb == quad) {
+                            const float4 ca = reinterpret_cast<const float4*>(cm + j0)[0];
+                            const float4 cb = reinterpret_cast<const float4*>(cm + j0)[1];
+                            const float4 da = reinterpret_cast<const float4*>(cm + kQ + j0)[0];
+                            const float4 db = reinterpret_cast<const float4*>(cm + kQ + j0)[1];
+                            const float cc[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+                            const float dd[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+                            float m[8];
+#pragma unroll
+                            for (int e = 0; e < 8; e += 2) {
+                                const float2 f = mul2(make_float2(ex2_approx(cl_m - cc[e]), ex2_approx(cl_m - cc[e + 1])),
+                                                      make_float2(dd[e], dd[e + 1]));
+                                const float2 v = mul2(make_float2(gv[jb][e], gv[jb][e + 1]), f);
+                                m[e] = (j0 + e < row) ? v.x : (j0 + e == row ? v.x + Dm : 0.0f);
+                                m[e + 1] = (j0 + e + 1 < row) ? v.y : (j0 + e + 1 == row ? v.y + Dm : 0.0f);
+                            }
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                __nv_bfloat162 b2 = __floats2bfloat162_rn(m[2 * e], m[2 * e + 1]);
+                                w[e] = *reinterpret_cast<uint32_t*>(&b2);
+                            }
+                        }
+                        tmem_st4(tmem + pr::kColM + (uint32_t)hm * 64u + lane_off + (uint32_t)(j0 >> 1), w[0], w[1], w[2],
+                                 w[3]);
+                    }
+                }
+            }
+            // 6. C h^T of this thread's head and columns scaled by 2^(cl_i)
+            //    in place: M X accumulates onto it
+            mbar_wait_bounded(bar_myo, ph, kWaitNs, aborted, prm.status);
+            tc_fence_after_sync();
+            {
+                float yo[32];
+                tmem_ld32(tY, yo);
+                tmem_wait_ld();
+                const float sc = ex2_approx(cl_i);
+#pragma unroll
+                for (int p = 0; p < 32; p += 2) {
+                    const float2 r = mul2(make_float2(yo[p], yo[p + 1]), make_float2(sc, sc));
+                    yo[p] = r.x;
+                    yo[p + 1] = r.y;
+                }
+                tmem_st32(tY, yo);
+            }
+            tmem_wait_st();
+            tc_fence_before_sync();
+            mbar_arrive(bar_mready);   // M X can start
+
+            // 7. end of a segment: the states leave the chip
+            if (it.seg_end) {
+                mbar_wait_bounded(bar_m4, ph, kWaitNs, aborted, prm.status);
+                tc_fence_after_sync();
+                tmem_ld32(tH, hv);
+                tmem_wait_ld();
+                if (it.publish) {
+                    float* dst = prm.ws_states + ((size_t)ticket * 2 + hd) * kPN;
+#pragma unroll
+                    for (int p = 0; p < 32; ++p) __stcg(dst + (size_t)(pq + p) * kN + row, hv[p]);
+                    __threadfence();
+                    named_bar_sync(kEwBarrier, kEwThreads);
+                    if (tid == 0) st_release_gpu(prm.ws_ctrl + 16 + ticket, 1);
+                } else if (prm.final_state) {
+                    float* dst = prm.final_state + ((size_t)it.seq * Hf + h0 + hd) * kPN;
+#pragma unroll
+                    for (int p = 0; p < 32; ++p) dst[(size_t)(pq + p) * kN + row] = hv[p];
+                }
+            }
+            prev_pre = false;
+        }
+        if (rg.count > 0) y_epilogue(rg.count - 1, false);
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_tiled_fn()
 {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
@@ -1141,13 +1804,17 @@ cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t channels, uint64
 // 64-head workload: 128 CTAs, 12% faster than 148 unaligned ones).  A ragged
 // batch's chain lengths are known on the device only: it takes ranges of at
 // least kMinRangeLong units over H times the chunks of its packed tokens.
+// Dense batches whose groups hold an even number of heads run the head-pair
+// kernel, whose chains are (sequence, head pair).
+bool tc_pairs(const ScanArgs& a) { return !a.cu_seqlens && a.G > 0 && (a.H / a.G) % 2 == 0; }
+
 int tc_slots(const ScanArgs& a, bool* long_chains = nullptr)
 {
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
         sms = 148;
-    const long long chains = (long long)(a.cu_seqlens ? a.nseq : a.b) * a.H;
+    const long long chains = (long long)(a.cu_seqlens ? a.nseq : a.b) * (tc_pairs(a) ? a.H / 2 : a.H);
     const long long nc = (a.L + kQ - 1) / kQ;
     const long long units = a.cu_seqlens ? (long long)a.H * nc : chains * nc;
     long long slots = chains < sms ? chains : sms;
@@ -1182,7 +1849,7 @@ size_t chunk_scan_tc_workspace_bytes(const ScanArgs& a)
     }
     if (a.b <= 0 || a.L <= 0) return 0;
     const int slots = tc_slots(a);
-    return kWsCtrlBytes(slots) + (size_t)slots * kStateBytes;
+    return kWsCtrlBytes(slots) + (size_t)slots * kStateBytes * (tc_pairs(a) ? 2 : 1);
 }
 
 cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t s)
@@ -1197,14 +1864,20 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t s)
     if ((e = make_map(&tmY, a.y, (uint64_t)a.H * a.P, a.L, a.b, (uint64_t)a.H * a.P * 2)) != cudaSuccess) return e;
     bool long_chains = false;
     const int slots = tc_slots(a, &long_chains);
-    auto kernel = a.cu_seqlens ? (long_chains ? chunk_scan_tc_kernel<true, true> : chunk_scan_tc_kernel<true, false>)
-                               : (long_chains ? chunk_scan_tc_kernel<false, true> : chunk_scan_tc_kernel<false, false>);
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    const bool pairs = tc_pairs(a);
+    const int hunits = pairs ? a.H / 2 : a.H;   // chains per sequence
+    auto kernel = pairs ? (long_chains ? chunk_scan_tc_pair_kernel<true> : chunk_scan_tc_pair_kernel<false>)
+                  : a.cu_seqlens
+                      ? (long_chains ? chunk_scan_tc_kernel<true, true> : chunk_scan_tc_kernel<true, false>)
+                      : (long_chains ? chunk_scan_tc_kernel<false, true> : chunk_scan_tc_kernel<false, false>);
+    const int smem_bytes = pairs ? pr::kSmemBytes : kSmemBytes;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
     if (e != cudaSuccess) return e;
     const size_t ctrl = kWsCtrlBytes(slots);
     const bool ragged = a.cu_seqlens != nullptr;
     const size_t table = ragged ? varlen_table_bytes(a.nseq) : 0;
-    if (!a.workspace || a.workspace_bytes < table + ctrl + (size_t)slots * kStateBytes) return cudaErrorInvalidValue;
+    if (!a.workspace || a.workspace_bytes < table + ctrl + (size_t)slots * kStateBytes * (pairs ? 2 : 1))
+        return cudaErrorInvalidValue;
     uint8_t* ws = static_cast<uint8_t*>(a.workspace);
     int* ws_ctrl = reinterpret_cast<int*>(ws + table);
     // ticket counter and hand-off flags start at zero on every call (a
@@ -1226,14 +1899,15 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t s)
     prm.y = static_cast<__nv_bfloat16*>(a.y);
     prm.final_state = a.final_state;
     prm.L = a.L;
-    prm.H = a.H;
+    prm.H = hunits;
+    prm.Hf = a.H;
     prm.G = a.G;
     prm.nc = ragged ? 1 : (a.L + kQ - 1) / kQ;   // (a ragged batch's chunk counts vary)
     prm.nslots = slots;
-    prm.units = ragged ? 0 : a.b * a.H * prm.nc;
+    prm.units = ragged ? 0 : a.b * hunits * prm.nc;
     prm.fnc = FastDiv::make((uint32_t)prm.nc);
-    prm.fH = FastDiv::make((uint32_t)a.H);
-    prm.fHG = FastDiv::make((uint32_t)(a.H / a.G));
+    prm.fH = FastDiv::make((uint32_t)hunits);
+    prm.fHG = FastDiv::make((uint32_t)(hunits / a.G));
     prm.ws_ctrl = ws_ctrl;
     prm.ws_states = reinterpret_cast<float*>(ws + table + ctrl);
     prm.cu_seqlens = a.cu_seqlens;
@@ -1241,7 +1915,7 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t s)
     prm.ws_hdr = ragged ? reinterpret_cast<const int*>(ws) : nullptr;
     prm.nseq = ragged ? a.nseq : a.b;
     prm.status = a.status;
-    kernel<<<slots, kThreads, kSmemBytes, s>>>(tmX, tmB, tmC, tmY, prm);
+    kernel<<<slots, kThreads, smem_bytes, s>>>(tmX, tmB, tmC, tmY, prm);
     return cudaGetLastError();
 }
 
