@@ -11,7 +11,10 @@ general path (fp32); empty sequences inside and at the end of the batch;
 lengths 1, 127/128/129 around a chunk; many short sequences (many chains,
 tails of 1 token); one long sequence next to short ones, so that scheduling
 ranges start and end inside one chain; equal lengths, which must give the
-dense call's result bit for bit; a prompt prefilled as two calls with the
+dense call's result bit for bit where both calls take the one-head kernel
+(an odd number of heads per group; with an even number the dense call runs
+head pairs, whose y is summed in another order, and the two agree within
+the bf16 bound); a prompt prefilled as two calls with the
 state handed over; and an invalid cu_seqlens, which must write nothing and
 report SSD_ERR_INVALID_ARG.
 """
@@ -111,17 +114,22 @@ def test_varlen_ranges_inside_one_chain():
     _check(s, d, y, fs, st, "bf16")
 
 
-def test_varlen_equal_lengths_match_the_dense_call_bit_for_bit():
+@pytest.mark.parametrize("hpg", [3, 4], ids=["one_head_kernel", "head_pairs"])
+def test_varlen_equal_lengths_match_the_dense_call(hpg):
     b, L = 3, 300
-    s, d = _ragged(BF16, [L] * b, 505)
+    s, d = _ragged(BF16.with_(H=2 * hpg, G=2), [L] * b, 505)
     y, fs, st = _run(s, d)
     assert st == 0
     yd, fsd = layer.chunk_scan_fwd(d["x"].view(b, L, s.H, s.P), d["B"].view(b, L, s.G, s.N),
                                    d["C"].view(b, L, s.G, s.N), d["dt_raw"].view(b, L, s.H), d["A"],
                                    d["dt_bias"], d["D"], d["init_state"], Q=s.Q)
     torch.cuda.synchronize()
-    assert torch.equal(y.view(b, L, s.H, s.P), yd)
-    assert torch.equal(fs, fsd)
+    if hpg % 2:   # the same kernel on both calls
+        assert torch.equal(y.view(b, L, s.H, s.P), yd)
+        assert torch.equal(fs, fsd)
+    else:         # the dense call runs head pairs
+        assert norm_max_abs(y.view(b, L, s.H, s.P), yd) <= TOL_BF16_NMA
+        assert norm_max_abs(fs, fsd) <= TOL_BF16_NMA
 
 
 def test_varlen_chunked_prefill_hands_the_state_over():
