@@ -3,7 +3,11 @@ the fp64 oracle on identical seeded inputs, called through the C ABI.
 
 Sizes span several chunks and a ragged last chunk; the full-size workloads
 are checked element by element (configs 0-2) or on a 4096-token prefix plus
-size-independent properties (the 262144-token one)."""
+size-independent properties (the 262144-token one).  Both tensor-core
+kernels are covered: dense batches whose groups hold an even number of
+heads run head pairs (e.g. 2, 4, 6, 8 and 16 heads per group below, the
+8B and long-context workloads), the others one head per item (1, 3 and 5
+heads per group, the 3B workload); each in its dense and long-chain forms."""
 import math
 
 import numpy as np
@@ -144,6 +148,16 @@ LONG = {
     # chain, 128 CTAs, with an initial state and dt_bias
     "aligned_ranges_32_heads": (synth.CONFIGS[1].with_(b=1, L=32768, H=32, G=4),
                                 dict(init_state=True, dt_bias=True)),
+    # head pairs (2 heads per group): 2 pair chains of 64 chunks -> 2 ranges
+    # each; the second range's walk reaches the chain's start and adds both
+    # heads' decayed initial states
+    "pairs_walk_reaches_chain_start": (synth.CONFIGS[1].with_(b=1, L=8100, H=4, G=2),
+                                       dict(init_state=True, dt_bias=True)),
+    # one head per item (3 heads per group) with long-memory heads: 6 chains
+    # of 157 chunks, 4 ranges each, some rebuilt and some waiting for the
+    # published state
+    "odd_groups_long_memory": (synth.CONFIGS[1].with_(b=1, L=20000, H=6, G=2),
+                               dict(a_range=(0.01, 2.0), init_state=True)),
 }
 
 
