@@ -1140,6 +1140,32 @@ constexpr uint32_t kIdS = umma_idesc_bf16(128, 128, true, true);     // B^T (MN-
 static_assert(kSmemBytes <= 232448, "shared memory");
 }  // namespace pr
 
+// 32 TMEM columns of a lane as two 16-column accesses: in the pair kernel
+// this is 2% faster on the 8B layer than one 32-column access and gives the
+// same values (the register allocator places two short vectors more freely).
+__device__ inline void pair_ld32(uint32_t taddr, float (&v)[32])
+{
+    float a[16], b[16];
+    tmem_ld16(taddr, a);
+    tmem_ld16(taddr + 16u, b);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        v[i] = a[i];
+        v[16 + i] = b[i];
+    }
+}
+__device__ inline void pair_st32(uint32_t taddr, const float (&v)[32])
+{
+    float a[16], b[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        a[i] = v[i];
+        b[i] = v[16 + i];
+    }
+    tmem_st16(taddr, a);
+    tmem_st16(taddr + 16u, b);
+}
+
 template <bool kLong>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_scan_tc_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
@@ -1491,7 +1517,7 @@ chunk_scan_tc_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_
         auto segment_state = [&](const Item& it, float (&hv)[32]) {
             if (it.depend) {
                 if (kLong && pre_ok) {
-                    tmem_ld32(tH, hv);
+                    pair_ld32(tH, hv);
                     tmem_wait_ld();
                 } else {
                     load_published(hv);
@@ -1513,7 +1539,7 @@ chunk_scan_tc_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_
             }
             tc_fence_after_sync();
             float yv[32];
-            tmem_ld32(tY, yv);
+            pair_ld32(tY, yv);
             tmem_wait_ld();
             if (release) {
                 tc_fence_before_sync();
@@ -1604,7 +1630,7 @@ chunk_scan_tc_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_
                 // released), so the bf16 state may be rewritten
                 mbar_wait_bounded(bar_m4, (uint32_t)(idx - 1) & 1u, kWaitNs, aborted, prm.status);
                 tc_fence_after_sync();
-                tmem_ld32(tH, hv);
+                pair_ld32(tH, hv);
                 tmem_wait_ld();
             }
             // 2. its bf16 copy for C h^T
@@ -1622,7 +1648,7 @@ chunk_scan_tc_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_
                     hv[p] = r.x;
                     hv[p + 1] = r.y;
                 }
-                tmem_st32(tH, hv);
+                pair_st32(tH, hv);
             }
             mbar_wait_bounded(bar_ldx + (idx & 1), (uint32_t)(idx >> 1) & 1u, kWaitNs, aborted, prm.status);
             {
@@ -1714,7 +1740,7 @@ chunk_scan_tc_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_
             tc_fence_after_sync();
             {
                 float yo[32];
-                tmem_ld32(tY, yo);
+                pair_ld32(tY, yo);
                 tmem_wait_ld();
                 const float sc = ex2_approx(cl_i);
 #pragma unroll
@@ -1723,7 +1749,7 @@ chunk_scan_tc_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_
                     yo[p] = r.x;
                     yo[p + 1] = r.y;
                 }
-                tmem_st32(tY, yo);
+                pair_st32(tY, yo);
             }
             tmem_wait_st();
             tc_fence_before_sync();
@@ -1733,7 +1759,7 @@ chunk_scan_tc_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_
             if (it.seg_end) {
                 mbar_wait_bounded(bar_m4, ph, kWaitNs, aborted, prm.status);
                 tc_fence_after_sync();
-                tmem_ld32(tH, hv);
+                pair_ld32(tH, hv);
                 tmem_wait_ld();
                 if (it.publish) {
                     float* dst = prm.ws_states + ((size_t)ticket * 2 + hd) * kPN;
