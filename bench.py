@@ -336,6 +336,7 @@ class DecodeStep:
         self.u = torch.empty(s.b, s.conv_dim, dtype=s.torch_dtype, device=dev)
         self.y = torch.empty(s.b, s.H, s.P, dtype=s.torch_dtype, device=dev)
         self.views = layer.split_channels(self.u, s.H, s.P, s.G, s.N)
+        self.ws = layer.decode_step_workspace(s.b, s.G, dev)
 
     def conv(self):
         d, s = self.d, self.s
@@ -349,7 +350,14 @@ class DecodeStep:
                                 y=self.y)
 
     def __call__(self):
-        """One decode token per sequence through the one-kernel decode step."""
+        """One decode token per sequence through the one-kernel decode step,
+        one CTA per (sequence, head) with its workspace of arrival counters."""
+        d, s = self.d, self.s
+        self.layer.decode_step(d["xBC"], d["w"], d["conv_state"], d["state"], d["dt_raw"], d["A"],
+                               s.H, s.P, s.G, s.N, dt_bias=d["dt_bias"], D=d["D"], y=self.y, workspace=self.ws)
+
+    def per_group(self):
+        """The same step, one CTA per (sequence, group), no workspace."""
         d, s = self.d, self.s
         self.layer.decode_step(d["xBC"], d["w"], d["conv_state"], d["state"], d["dt_raw"], d["A"],
                                s.H, s.P, s.G, s.N, dt_bias=d["dt_bias"], D=d["D"], y=self.y)
@@ -541,6 +549,17 @@ def run_ours(args, rank, world, dev):
     d1.record()
     barrier()
     dec_ms = max_over_ranks(d0.elapsed_time(d1) / KD)
+    # the one-kernel step without the workspace (one CTA per sequence and group)
+    for _ in range(3):
+        dec.per_group()
+    d4, d5 = _events(2)
+    barrier()
+    d4.record()
+    for _ in range(KD):
+        dec.per_group()
+    d5.record()
+    barrier()
+    grp_ms = max_over_ranks(d4.elapsed_time(d5) / KD)
     # the same step as two kernels (conv roll, then the state update alone), for comparison
     for _ in range(3):
         dec.conv(); dec.update()
@@ -620,11 +639,13 @@ def run_ours(args, rank, world, dev):
         "conv": blocks[s.name]["conv"],
         "prefill": blocks,
         "decode": {"workload": DECODE.name,
-                   "kernel": "decode_step (conv-cache roll, conv + SiLU, state update: one launch)",
+                   "kernel": "decode_step_head (conv-cache roll, conv + SiLU, state update: one launch, "
+                             "one CTA per sequence and head, ssd_decode_step_ws)",
                    "ms_per_step": dec_ms,
                    "GB/s": decode_step_bytes(DECODE) / (dec_ms * 1e-3) / 1e9,
                    "frac_hbm": decode_step_bytes(DECODE) / (dec_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                    "tokens_per_s": world * DECODE.b / (dec_ms * 1e-3),
+                   "per_group_kernel_ms_per_step": grp_ms,
                    "two_kernel_ms_per_step": two_ms, "state_update_ms": upd_ms,
                    "state_update_GB/s": decode_state_update_bytes(DECODE) / (upd_ms * 1e-3) / 1e9,
                    "state_update_frac_hbm": decode_state_update_bytes(DECODE) / (upd_ms * 1e-3) / 1e9 /

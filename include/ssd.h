@@ -333,6 +333,28 @@ SSD_API ssd_status_t ssd_decode_step(float* state, void* conv_state, const void*
                                      int N, int G, int k, ssd_dtype_t dtype, cudaStream_t stream);
 
 /*
+ * The same decode step in one kernel with a small workspace, so that it can
+ * run one CTA per (sequence, head) and keep HBM as busy as ssd_state_update
+ * does: every CTA convolves its head's x channels and its group's B and C
+ * channels, and the group's B and C cache columns, which its heads share,
+ * are rolled by whichever of the group's CTAs finishes reading them last (an
+ * atomic count per (sequence, group); no CTA waits for another).  Same
+ * arguments, layouts and results as ssd_decode_step (bit for bit), plus
+ *   workspace        int32 [b][G], caller-owned, ZERO before the first call
+ *                    on it; every call leaves it zero.  Calls that may run
+ *                    at the same time need separate workspaces.
+ *   workspace_bytes  at least ssd_decode_step_workspace_bytes(b, G)
+ * Errors as ssd_decode_step, SSD_ERR_INVALID_ARG for a NULL, unaligned,
+ * short or overlapping workspace, and SSD_ERR_UNSUPPORTED for P > 256.
+ */
+SSD_API size_t ssd_decode_step_workspace_bytes(int b, int G);
+SSD_API ssd_status_t ssd_decode_step_ws(float* state, void* conv_state, const void* xBC, const float* w,
+                                        const float* bias, const void* dt_raw, const float* dt_bias,
+                                        const float* A, const float* D, void* y, int b, int H, int P,
+                                        int N, int G, int k, ssd_dtype_t dtype, void* workspace,
+                                        size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Backward pass of the chunked scan: the gradients of a loss
  * Loss(y, final_state) through ssd_chunk_scan_fwd, given dy = dLoss/dy and
  * dfinal = dLoss/d(final_state), for training (the Nemotron feasibility

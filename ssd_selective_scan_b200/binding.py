@@ -44,6 +44,9 @@ SIGNATURES = {
     "ssd_conv_scan_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),
     "ssd_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                              _i, _i, _i, _i, _i, _i, _i, _vp]),
+    "ssd_decode_step_workspace_bytes": (_sz, [_i, _i]),
+    "ssd_decode_step_ws": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "ssd_chunk_scan_bwd_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "ssd_chunk_scan_bwd": (_i, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                 _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -147,6 +150,16 @@ def ssd_decode_step(state, conv_state, xBC, w, bias, dt_raw, dt_bias, A, D, y, b
                     dtype, stream) -> int:
     return load().ssd_decode_step(state, conv_state, xBC, w, bias, dt_raw, dt_bias, A, D, y, b, H, P,
                                   N, G, k, dtype, stream)
+
+
+def ssd_decode_step_workspace_bytes(b, G) -> int:
+    return load().ssd_decode_step_workspace_bytes(b, G)
+
+
+def ssd_decode_step_ws(state, conv_state, xBC, w, bias, dt_raw, dt_bias, A, D, y, b, H, P, N, G, k,
+                       dtype, workspace, workspace_bytes, stream) -> int:
+    return load().ssd_decode_step_ws(state, conv_state, xBC, w, bias, dt_raw, dt_bias, A, D, y, b, H, P,
+                                     N, G, k, dtype, workspace, workspace_bytes, stream)
 
 
 def ssd_chunk_scan_bwd_workspace_bytes(b, L, H, P, N, G, dtype) -> int:

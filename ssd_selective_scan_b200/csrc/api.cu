@@ -353,16 +353,23 @@ ssd_status_t ssd_state_update(float* state, const void* x, const void* B, const 
                                               b, H, P, N, G, dtype == SSD_BF16, stream));
 }
 
-ssd_status_t ssd_decode_step(float* state, void* conv_state, const void* xBC, const float* w,
-                             const float* bias, const void* dt_raw, const float* dt_bias, const float* A,
-                             const float* D, void* y, int b, int H, int P, int N, int G, int k,
-                             ssd_dtype_t dtype, cudaStream_t stream)
+// Arguments of the decode step (both forms): SSD_OK, or the error to return
+// (with b == 0 reported as SSD_OK and *nothing set).
+static ssd_status_t decode_step_check(float* state, void* conv_state, const void* xBC, const float* w,
+                                      const float* bias, const void* dt_raw, const float* dt_bias, const float* A,
+                                      const float* D, void* y, int b, int H, int P, int N, int G, int k,
+                                      ssd_dtype_t dtype, const void* workspace, size_t workspace_bytes,
+                                      bool with_workspace, bool* nothing)
 {
+    *nothing = false;
     if (!valid_dtype(dtype) || b < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || k <= 0 || H % G)
         return SSD_ERR_INVALID_ARG;
     if (N % 4) return SSD_ERR_INVALID_ARG;
     if ((int64_t)H * P + 2 * (int64_t)G * N > 0x7fffffffLL) return SSD_ERR_INVALID_ARG;
-    if (b == 0) return SSD_OK;
+    if (b == 0) {
+        *nothing = true;
+        return SSD_OK;
+    }
     if (!state || !conv_state || !xBC || !w || !dt_raw || !A || !y) return SSD_ERR_INVALID_ARG;
     const int e = elem_bytes(dtype);
     if (!aligned(state, 16) || !aligned(conv_state, e) || !aligned(xBC, e) || !aligned(dt_raw, e) ||
@@ -382,11 +389,50 @@ ssd_status_t ssd_decode_step(float* state, void* conv_state, const void* xBC, co
         if (overlap(rcs, in)) return SSD_ERR_INVALID_ARG;
     for (Range in : {rx, rw, rdt})
         if (overlap(ry, in)) return SSD_ERR_INVALID_ARG;
+    if (with_workspace) {
+        if (!workspace || !aligned(workspace, 4) || workspace_bytes < (size_t)b * G * 4) return SSD_ERR_INVALID_ARG;
+        const Range rws = span(workspace, (int64_t)b * G * 4);
+        for (Range in : {rs, rcs, rx, rw, rdt, ry})
+            if (overlap(rws, in)) return SSD_ERR_INVALID_ARG;
+    }
     if (k < 2 || k > 4 || !ssd::state_update_supports_n(N)) return SSD_ERR_UNSUPPORTED;
-    if ((int64_t)b * G > 0x7fffffffLL) return SSD_ERR_UNSUPPORTED;
-    if (ssd::decode_step_smem_bytes(H, P, N, G) > (size_t)max_optin_smem()) return SSD_ERR_UNSUPPORTED;
+    if (with_workspace && P > ssd::decode_step_head_max_p()) return SSD_ERR_UNSUPPORTED;
+    if ((int64_t)b * (with_workspace ? H : G) > 0x7fffffffLL) return SSD_ERR_UNSUPPORTED;
+    const size_t smem = with_workspace ? ssd::decode_step_head_smem_bytes(P, N) : ssd::decode_step_smem_bytes(H, P, N, G);
+    if (smem > (size_t)max_optin_smem()) return SSD_ERR_UNSUPPORTED;
+    return SSD_OK;
+}
+
+ssd_status_t ssd_decode_step(float* state, void* conv_state, const void* xBC, const float* w,
+                             const float* bias, const void* dt_raw, const float* dt_bias, const float* A,
+                             const float* D, void* y, int b, int H, int P, int N, int G, int k,
+                             ssd_dtype_t dtype, cudaStream_t stream)
+{
+    bool nothing = false;
+    const ssd_status_t st = decode_step_check(state, conv_state, xBC, w, bias, dt_raw, dt_bias, A, D, y, b, H, P, N,
+                                              G, k, dtype, nullptr, 0, false, &nothing);
+    if (st != SSD_OK || nothing) return st;
     return from_cuda(ssd::launch_decode_step(state, conv_state, xBC, w, bias, dt_raw, dt_bias, A, D, y, b, H, P,
                                              N, G, k, dtype == SSD_BF16, stream));
+}
+
+size_t ssd_decode_step_workspace_bytes(int b, int G)
+{
+    return b > 0 && G > 0 ? (size_t)b * G * 4 : 0;
+}
+
+ssd_status_t ssd_decode_step_ws(float* state, void* conv_state, const void* xBC, const float* w,
+                                const float* bias, const void* dt_raw, const float* dt_bias, const float* A,
+                                const float* D, void* y, int b, int H, int P, int N, int G, int k,
+                                ssd_dtype_t dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    bool nothing = false;
+    const ssd_status_t st = decode_step_check(state, conv_state, xBC, w, bias, dt_raw, dt_bias, A, D, y, b, H, P, N,
+                                              G, k, dtype, workspace, workspace_bytes, true, &nothing);
+    if (st != SSD_OK || nothing) return st;
+    return from_cuda(ssd::launch_decode_step_head(state, conv_state, xBC, w, bias, dt_raw, dt_bias, A, D, y,
+                                                  static_cast<int*>(workspace), b, H, P, N, G, k, dtype == SSD_BF16,
+                                                  stream));
 }
 
 ssd_status_t ssd_linear_bf16(const void* x, int64_t ldx, const void* w, int64_t ldw, void* y, int64_t ldy, int M,

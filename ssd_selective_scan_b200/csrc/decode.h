@@ -16,4 +16,13 @@ cudaError_t launch_decode_step(float* state, void* conv_state, const void* xBC, 
                                const float* D, void* y, int b, int H, int P, int N, int G, int k, bool bf16,
                                cudaStream_t s);
 
+// The decode step in one kernel, one CTA per (sequence, head); arrivals:
+// int32 [b][G], zero on entry and left zero.
+size_t decode_step_head_smem_bytes(int P, int N);
+int decode_step_head_max_p();   // largest head dim of the per-head form
+cudaError_t launch_decode_step_head(float* state, void* conv_state, const void* xBC, const float* w,
+                                    const float* bias, const void* dt_raw, const float* dt_bias, const float* A,
+                                    const float* D, void* y, int* arrivals, int b, int H, int P, int N, int G, int k,
+                                    bool bf16, cudaStream_t s);
+
 }  // namespace ssd

@@ -313,10 +313,14 @@ def layer_prefill(xBC, w, dt_raw, A, H, P, G, N, *, bias=None, conv_state=None, 
 
 
 def decode_step(xBC, w, conv_state, state, dt_raw, A, H, P, G, N, *, bias=None, dt_bias=None,
-                D=None, y=None, stream=None):
+                D=None, y=None, workspace=None, stream=None):
     """One token per sequence in one kernel: conv-cache roll, conv + SiLU,
     then the state update.  xBC [b, conv_dim]; conv_state [b, conv_dim, k]
-    and state [b, H, P, N] f32 updated in place.  Returns y [b, H, P]."""
+    and state [b, H, P, N] f32 updated in place.  Returns y [b, H, P].
+    With `workspace` (int32, at least b * G elements, zero before its first
+    use; the call leaves it zero) the step runs one CTA per (sequence, head)
+    (ssd_decode_step_ws), else one per (sequence, group) (ssd_decode_step);
+    the results are the same."""
     if xBC.dim() != 2 or not xBC.is_contiguous():
         raise ValueError("xBC must be a contiguous [b, conv_dim] tensor")
     b, cd = xBC.shape
@@ -334,12 +338,27 @@ def decode_step(xBC, w, conv_state, state, dt_raw, A, H, P, G, N, *, bias=None, 
         raise ValueError("dt_raw must be a contiguous [b, H] tensor of xBC's dtype")
     if y is None:
         y = torch.empty((b, H, P), dtype=xBC.dtype, device=xBC.device)
+    if workspace is not None:
+        if workspace.dtype != torch.int32 or not workspace.is_contiguous() or workspace.device != xBC.device:
+            raise ValueError("workspace must be a contiguous int32 tensor on xBC's device")
+        st = libssd.ssd_decode_step_ws(_ptr(state), _ptr(conv_state), _ptr(xBC), _ptr(_f32(w, "w")),
+                                       _ptr(_f32(bias, "bias")), _ptr(dt_raw), _ptr(_f32(dt_bias, "dt_bias")),
+                                       _ptr(_f32(A, "A")), _ptr(_f32(D, "D")), _ptr(y), b, H, P, N, G, k,
+                                       _dtype_code(xBC), _ptr(workspace), workspace.numel() * 4, _stream(stream))
+        libssd.check("ssd_decode_step_ws", st)
+        return y
     st = libssd.ssd_decode_step(_ptr(state), _ptr(conv_state), _ptr(xBC), _ptr(_f32(w, "w")),
                                 _ptr(_f32(bias, "bias")), _ptr(dt_raw), _ptr(_f32(dt_bias, "dt_bias")),
                                 _ptr(_f32(A, "A")), _ptr(_f32(D, "D")), _ptr(y), b, H, P, N, G, k,
                                 _dtype_code(xBC), _stream(stream))
     libssd.check("ssd_decode_step", st)
     return y
+
+
+def decode_step_workspace(b: int, G: int, device) -> torch.Tensor:
+    """A zeroed workspace for decode_step(..., workspace=...)."""
+    n = libssd.ssd_decode_step_workspace_bytes(b, G) // 4
+    return torch.zeros(max(n, 1), dtype=torch.int32, device=device)
 
 
 def linear(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor | None = None, status: torch.Tensor | None = None,

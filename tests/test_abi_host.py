@@ -37,7 +37,8 @@ def test_header_declares_the_entry_points():
         "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_static",
         "ssd_chunk_scan_fwd_varlen", "ssd_chunk_scan_varlen_workspace_bytes",
         "ssd_chunk_scan_workspace_bytes", "ssd_conv1d_silu", "ssd_conv_scan_fwd",
-        "ssd_conv_scan_workspace_bytes", "ssd_decode_step", "ssd_linear_bf16", "ssd_mixer_fwd",
+        "ssd_conv_scan_workspace_bytes", "ssd_decode_step", "ssd_decode_step_workspace_bytes",
+        "ssd_decode_step_ws", "ssd_linear_bf16", "ssd_mixer_fwd",
         "ssd_mixer_workspace_bytes", "ssd_selftest_bounded_wait", "ssd_state_update", "ssd_status_string"])
 
 
@@ -235,6 +236,29 @@ def test_decode_step_validation():
     assert dec(y=fake(3, 64)) == INV                             # y overlaps xBC
     assert dec(conv_state=fake(1, 4096)) == INV                  # cache overlaps the state
     assert dec(k=5) == UNS and dec(k=1) == UNS and dec(N=512) == UNS
+
+
+def dec_ws(**kw):
+    a = dict(state=fake(1), conv_state=fake(2), xBC=fake(3), w=fake(4), bias=None, dt_raw=fake(5),
+             dt_bias=None, A=fake(6), D=None, y=fake(7), b=256, H=128, P=64, N=128, G=8, k=4,
+             dtype=BF16, workspace=fake(8), workspace_bytes=256 * 8 * 4, stream=None)
+    a.update(kw)
+    return libssd.ssd_decode_step_ws(**a)
+
+
+def test_decode_step_ws_validation():
+    # every call here fails validation (or is empty work) before any launch
+    assert libssd.ssd_decode_step_workspace_bytes(256, 8) == 256 * 8 * 4
+    assert libssd.ssd_decode_step_workspace_bytes(0, 8) == 0
+    assert dec_ws(b=0) == OK
+    for k in ("state", "conv_state", "xBC", "w", "dt_raw", "A", "y", "workspace"):
+        assert dec_ws(**{k: None}) == INV, k
+    assert dec_ws(workspace_bytes=256 * 8 * 4 - 4) == INV       # short
+    assert dec_ws(workspace=fake(8, 2)) == INV                   # not 4-byte aligned
+    assert dec_ws(workspace=fake(7, 64)) == INV                  # overlaps y
+    assert dec_ws(G=3) == INV and dec_ws(N=6) == INV and dec_ws(dtype=9) == INV
+    assert dec_ws(conv_state=fake(1, 4096)) == INV               # cache overlaps the state
+    assert dec_ws(k=5) == UNS and dec_ws(N=512) == UNS and dec_ws(P=320, b=1) == UNS
 
 
 def bwd(**kw):

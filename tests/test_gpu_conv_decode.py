@@ -127,10 +127,13 @@ def test_decode_step_full_layer_matches_oracle():
     (2, 2, 8, 256, 1, 2, "bf16", True),
     (7, 12, 16, 64, 4, 4, "f32", True),
 ])
-def test_decode_step_kernel_matches_oracle_and_two_calls(b, H, P, N, G, k, dtype, bias):
-    """The one-kernel decode step against the oracle (conv from the raw
-    token, then the recurrence step) and, bit for bit, against the two calls
-    it fuses (conv1d_silu with L = 1, then state_update)."""
+@pytest.mark.parametrize("form", ["per_group", "per_head_ws"])
+def test_decode_step_kernel_matches_oracle_and_two_calls(b, H, P, N, G, k, dtype, bias, form):
+    """The one-kernel decode step, in both forms (one CTA per group; one per
+    head with the workspace of arrival counters), against the oracle (conv
+    from the raw token, then the recurrence step) and, bit for bit, against
+    the two calls it fuses (conv1d_silu with L = 1, then state_update).  The
+    workspace form must leave its counters at zero."""
     s = synth.LayerShape("decode", b, 1, H, P, N, G, 128, k, dtype)
     inp = synth.decode_inputs(s, 7700 + b + N + k)
     cd = s.conv_dim
@@ -144,8 +147,9 @@ def test_decode_step_kernel_matches_oracle_and_two_calls(b, H, P, N, G, k, dtype
         f64(inp["D"]))
     args = dict(bias=cuda(bs), dt_bias=cuda(inp["dt_bias"]), D=cuda(inp["D"]))
     cs1, st1 = cuda(inp["conv_state"]), cuda(inp["state"])
+    ws = layer.decode_step_workspace(b, G, "cuda") if form == "per_head_ws" else None
     y1 = layer.decode_step(cuda(inp["xBC"]), cuda(inp["w"]), cs1, st1, cuda(inp["dt_raw"]), cuda(inp["A"]),
-                           H, P, G, N, **args)
+                           H, P, G, N, workspace=ws, **args)
     # the two calls
     cs2, st2 = cuda(inp["conv_state"]), cuda(inp["state"])
     u = layer.conv1d_silu(cuda(inp["xBC"]).view(b, 1, cd), cuda(inp["w"]), cuda(bs), cs2).view(b, cd)
@@ -154,9 +158,38 @@ def test_decode_step_kernel_matches_oracle_and_two_calls(b, H, P, N, G, k, dtype
     torch.cuda.synchronize()
     assert np.array_equal(f64(cs1), cs_ref), "conv cache roll"
     assert torch.equal(cs1, cs2) and torch.equal(st1, st2) and torch.equal(y1, y2), "differs from the two calls"
+    if ws is not None:
+        assert int(ws.abs().sum()) == 0, "arrival counters not left at zero"
     # float32 conv outputs are within 1e-6 of the oracle's, so the state keeps
     # its 1e-5 bound; bf16-rounded ones move the state at the bf16 bound
     tol_state = TOL_STATE_F32 if dtype == "f32" else 2e-2
     e_state = norm_max_abs(st1, st_ref)
     assert e_state <= tol_state, f"decode state error {e_state:.3e}"
     assert_output(y1, y_ref, dtype, "decode-step y")
+
+
+def test_decode_step_ws_successive_steps_equal_the_two_calls():
+    """Three decode steps in a row through the workspace form (the arrival
+    counters reset by each call are reused by the next) equal three steps of
+    the two calls bit for bit: the group's shared B and C cache columns are
+    rolled exactly once per step."""
+    b, H, P, N, G, k = 6, 16, 64, 128, 2, 4
+    s = synth.LayerShape("decode", b, 1, H, P, N, G, 128, k, "bf16")
+    inp = synth.decode_inputs(s, 7811)
+    cd = s.conv_dim
+    ws = layer.decode_step_workspace(b, G, "cuda")
+    cs1, st1 = cuda(inp["conv_state"]), cuda(inp["state"])
+    cs2, st2 = cuda(inp["conv_state"]), cuda(inp["state"])
+    g = torch.Generator().manual_seed(5)
+    for step in range(3):
+        xBC = (torch.randn(b, cd, generator=g) * 0.5).to(torch.bfloat16).cuda()
+        dt_raw = (torch.rand(b, H, generator=g) * -3 - 1).to(torch.bfloat16).cuda()
+        y1 = layer.decode_step(xBC, cuda(inp["w"]), cs1, st1, dt_raw, cuda(inp["A"]), H, P, G, N,
+                               dt_bias=cuda(inp["dt_bias"]), D=cuda(inp["D"]), workspace=ws)
+        u = layer.conv1d_silu(xBC.view(b, 1, cd), cuda(inp["w"]), None, cs2).view(b, cd)
+        xd, Bd, Cd = layer.split_channels(u, H, P, G, N)
+        y2 = layer.state_update(st2, xd, Bd, Cd, dt_raw, cuda(inp["A"]), cuda(inp["dt_bias"]), cuda(inp["D"]))
+        torch.cuda.synchronize()
+        assert torch.equal(cs1, cs2) and torch.equal(st1, st2) and torch.equal(y1, y2), f"step {step}"
+    assert int(ws.abs().sum()) == 0
+
