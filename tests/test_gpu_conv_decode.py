@@ -126,6 +126,7 @@ def test_decode_step_full_layer_matches_oracle():
     (4, 6, 24, 32, 3, 3, "f32", False),
     (2, 2, 8, 256, 1, 2, "bf16", True),
     (7, 12, 16, 64, 4, 4, "f32", True),
+    (3, 4, 64, 128, 4, 4, "bf16", False),       # one head per group: every CTA is its group's last
 ])
 @pytest.mark.parametrize("form", ["per_group", "per_head_ws"])
 def test_decode_step_kernel_matches_oracle_and_two_calls(b, H, P, N, G, k, dtype, bias, form):
