@@ -1005,19 +1005,21 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             // 5. the masked tile M = G o L of item idx into TMEM (bf16
             //    pairs), the A operand of M X.  Column block jb (32 tokens)
             //    is zero above the row quadrant's diagonal block; of every
-            //    block, column quarter `quarter` takes 8 columns.
+            //    block, column quarter `quarter` takes 8 columns.  One block
+            //    at a time, in a loop that is not unrolled: the smaller code
+            //    is faster (3B layer 0.0963 -> 0.0943 ms).
             mbar_wait_bounded(bar_m1, (uint32_t)idx & 1u, kWaitNs, aborted, prm.status);
             tc_fence_after_sync();
             {
-                float gv[4][8];
-#pragma unroll
-                for (int jb = 0; jb < 4; ++jb)
-                    if (jb <= quad) tmem_ld8(tmem + kColG + lane_off + (uint32_t)(jb * 32 + quarter * 8), gv[jb]);
-                tmem_wait_ld();
-#pragma unroll
+#pragma unroll 1
                 for (int jb = 0; jb < 4; ++jb) {
                     const int j0 = jb * 32 + quarter * 8;
                     uint32_t w[4] = {0u, 0u, 0u, 0u};
+                    float gb[8];
+                    if (jb <= quad) {
+                        tmem_ld8(tmem + kColG + lane_off + (uint32_t)j0, gb);
+                        tmem_wait_ld();
+                    }
                     if (jb < quad) {
                         const float u = ex2_approx(cl_i - cv.cl[jb * 32 + 31]);
                         const float4 va = reinterpret_cast<const float4*>(cv.v + j0)[0];
@@ -1026,7 +1028,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const float2 uv = mul2(make_float2(u, u), make_float2(vv[2 * e], vv[2 * e + 1]));
-                            const float2 m = mul2(make_float2(gv[jb][2 * e], gv[jb][2 * e + 1]), uv);
+                            const float2 m = mul2(make_float2(gb[2 * e], gb[2 * e + 1]), uv);
                             __nv_bfloat162 b2 = __floats2bfloat162_rn(m.x, m.y);
                             w[e] = *reinterpret_cast<uint32_t*>(&b2);
                         }
@@ -1043,7 +1045,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                         for (int e = 0; e < 8; e += 2) {
                             const float2 f = mul2(make_float2(ex2_approx(cl_i - cc[e]), ex2_approx(cl_i - cc[e + 1])),
                                                   make_float2(dd[e], dd[e + 1]));
-                            const float2 v = mul2(make_float2(gv[jb][e], gv[jb][e + 1]), f);
+                            const float2 v = mul2(make_float2(gb[e], gb[e + 1]), f);
                             m[e] = (j0 + e < row) ? v.x : (j0 + e == row ? v.x + Dh : 0.0f);
                             m[e + 1] = (j0 + e + 1 < row) ? v.y : (j0 + e + 1 == row ? v.y + Dh : 0.0f);
                         }
