@@ -25,7 +25,7 @@ namespace ssd {
 constexpr int kConvThreads = 128;
 constexpr int kConvTile = 32;   // tokens per thread
 constexpr int kConvTileLong = 64;       // ... for long sequences (fewer halo re-reads, fewer CTAs)
-constexpr int kConvLongTokens = 65536;  // L from which the long tile is used
+constexpr int kConvLongTokens = 4096;   // L from which the long tile is used (shorter: more CTAs pay)
 constexpr int kGroup = 8;       // tokens loaded together
 constexpr int kCpt = 4;         // channels per thread
 
