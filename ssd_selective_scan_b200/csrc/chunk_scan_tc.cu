@@ -158,14 +158,16 @@ __device__ inline uint4 pack_bf16x8(const float* v)
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-__device__ inline void unpack_bf16x8(uint4 q, float* v)
+// Eight bf16 values times w, in bf16 pairs: w is rounded to bf16 once
+// (relative error 2^-9, like the product's own rounding), then each product
+// is rounded to bf16 as the packed fp32 form did.  Half the instructions of
+// unpack, fp32 multiply and pack.
+__device__ inline uint4 scale_bf16x8(uint4 q, __nv_bfloat162 w)
 {
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&q);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        v[2 * i] = __uint_as_float(w[i] << 16);
-        v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-    }
+    for (int i = 0; i < 4; ++i) h[i] = __hmul2(h[i], w);
+    return q;
 }
 
 // K-major operand, 128 rows, K = 128 as two 64-wide halves: descriptor of
@@ -897,18 +899,11 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                     mbar_wait_bounded(bar_m4 + ((idx - 1) & 1), (uint32_t)((idx - 1) >> 1) & 1u, kWaitNs, aborted,
                                       prm.status);
                 mbar_wait_bounded(bar_ldx + (idx & 1), (uint32_t)(idx >> 1) & 1u, kWaitNs, aborted, prm.status);
+                const __nv_bfloat162 w2 = __floats2bfloat162_rn(wj, wj);
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    float v[8];
-                    unpack_bf16x8(*reinterpret_cast<const uint4*>(st + kStX + sw128(row, quarter * 2 + q)), v);
-#pragma unroll
-                    for (int e = 0; e < 8; e += 2) {
-                        const float2 r = mul2(make_float2(v[e], v[e + 1]), make_float2(wj, wj));
-                        v[e] = r.x;
-                        v[e + 1] = r.y;
-                    }
-                    *reinterpret_cast<uint4*>(sWX + sw128(row, quarter * 2 + q)) = pack_bf16x8(v);
-                }
+                for (int q = 0; q < 2; ++q)
+                    *reinterpret_cast<uint4*>(sWX + sw128(row, quarter * 2 + q)) =
+                        scale_bf16x8(*reinterpret_cast<const uint4*>(st + kStX + sw128(row, quarter * 2 + q)), w2);
                 fence_proxy_async_smem();
                 tc_fence_before_sync();
                 mbar_arrive(bar_sready);   // the state product can start
@@ -981,18 +976,11 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             mbar_wait_bounded(bar_ldx + (idx & 1), (uint32_t)(idx >> 1) & 1u, kWaitNs, aborted, prm.status);
             {
                 const float wj = ex2_approx(cl_last - cl_i) * cv.dt[row];
+                const __nv_bfloat162 w2 = __floats2bfloat162_rn(wj, wj);
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    float v[8];
-                    unpack_bf16x8(*reinterpret_cast<const uint4*>(st + kStX + sw128(row, quarter * 2 + q)), v);
-#pragma unroll
-                    for (int e = 0; e < 8; e += 2) {
-                        const float2 r = mul2(make_float2(v[e], v[e + 1]), make_float2(wj, wj));
-                        v[e] = r.x;
-                        v[e + 1] = r.y;
-                    }
-                    *reinterpret_cast<uint4*>(sWX + sw128(row, quarter * 2 + q)) = pack_bf16x8(v);
-                }
+                for (int q = 0; q < 2; ++q)
+                    *reinterpret_cast<uint4*>(sWX + sw128(row, quarter * 2 + q)) =
+                        scale_bf16x8(*reinterpret_cast<const uint4*>(st + kStX + sw128(row, quarter * 2 + q)), w2);
             }
             tmem_wait_st();
             fence_proxy_async_smem();
@@ -1573,18 +1561,11 @@ chunk_scan_tc_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_
                 if (idx > 0)
                     mbar_wait_bounded(bar_m4, (uint32_t)(idx - 1) & 1u, kWaitNs, aborted, prm.status);
                 mbar_wait_bounded(bar_ldx + (idx & 1), (uint32_t)(idx >> 1) & 1u, kWaitNs, aborted, prm.status);
+                const __nv_bfloat162 w2 = __floats2bfloat162_rn(wj, wj);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float v[8];
-                    unpack_bf16x8(*reinterpret_cast<const uint4*>(xs + sw128(row, ch0 + q)), v);
-#pragma unroll
-                    for (int e = 0; e < 8; e += 2) {
-                        const float2 r = mul2(make_float2(v[e], v[e + 1]), make_float2(wj, wj));
-                        v[e] = r.x;
-                        v[e + 1] = r.y;
-                    }
-                    *reinterpret_cast<uint4*>(sWX + sw128(row, ch0 + q)) = pack_bf16x8(v);
-                }
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4*>(sWX + sw128(row, ch0 + q)) =
+                        scale_bf16x8(*reinterpret_cast<const uint4*>(xs + sw128(row, ch0 + q)), w2);
                 fence_proxy_async_smem();
                 tc_fence_before_sync();
                 mbar_arrive(bar_sready);
@@ -1655,18 +1636,11 @@ chunk_scan_tc_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_
             mbar_wait_bounded(bar_ldx + (idx & 1), (uint32_t)(idx >> 1) & 1u, kWaitNs, aborted, prm.status);
             {
                 const float wj = ex2_approx(cl_last - cl_i) * cv[kQ + row];
+                const __nv_bfloat162 w2 = __floats2bfloat162_rn(wj, wj);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float v[8];
-                    unpack_bf16x8(*reinterpret_cast<const uint4*>(xs + sw128(row, ch0 + q)), v);
-#pragma unroll
-                    for (int e = 0; e < 8; e += 2) {
-                        const float2 r = mul2(make_float2(v[e], v[e + 1]), make_float2(wj, wj));
-                        v[e] = r.x;
-                        v[e + 1] = r.y;
-                    }
-                    *reinterpret_cast<uint4*>(sWX + sw128(row, ch0 + q)) = pack_bf16x8(v);
-                }
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4*>(sWX + sw128(row, ch0 + q)) =
+                        scale_bf16x8(*reinterpret_cast<const uint4*>(xs + sw128(row, ch0 + q)), w2);
             }
             tmem_wait_st();
             fence_proxy_async_smem();
