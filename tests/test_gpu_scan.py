@@ -69,6 +69,14 @@ CASES = {
     "bf16_many_chains_handoff": (synth.CONFIGS[1].with_(b=3, L=300, H=128, G=8), dict(init_state=True)),
     "bf16_many_chains_long_memory": (synth.CONFIGS[1].with_(b=5, L=520, H=64, G=8),
                                      dict(a_range=(0.01, 2.0))),
+    # strong decay (|A| 12 to 50, dt 0.7 to 2.1: the state keeps between
+    # 2^-12 and 2^-153 of itself per token), so the decay factors of
+    # masked-out columns overflow and those of early columns underflow; head
+    # pairs and one head per item
+    "bf16_tc_strong_decay_pairs": (synth.CONFIGS[1].with_(b=2, L=300, H=8, G=4),
+                                   dict(a_range=(8.0, 64.0), dt_range=(0.0, 2.0), init_state=True)),
+    "bf16_tc_strong_decay_one_head": (synth.CONFIGS[1].with_(b=2, L=300, H=6, G=2),
+                                      dict(a_range=(8.0, 64.0), dt_range=(0.0, 2.0), init_state=True)),
 }
 
 
@@ -158,6 +166,10 @@ LONG = {
     # published state
     "odd_groups_long_memory": (synth.CONFIGS[1].with_(b=1, L=20000, H=6, G=2),
                                dict(a_range=(0.01, 2.0), init_state=True)),
+    # head pairs with strong decay: every rebuilding walk stops after its
+    # first chunk, whose decay already falls below 2^-64 for both heads
+    "pairs_strong_decay_cut": (synth.CONFIGS[1].with_(b=1, L=8100, H=4, G=2),
+                               dict(a_range=(8.0, 64.0), dt_range=(0.0, 2.0), init_state=True)),
 }
 
 
