@@ -8,7 +8,7 @@ sequence alone in fp64 on the exact values the GPU consumed.
 
 Covered: the tensor-core path (bf16, P = 64, N = 128, Q = 128) and the
 general path (fp32); empty sequences inside and at the end of the batch;
-lengths 1, 127/128/129 around a chunk; many short sequences (many chains,
+lengths 1, 127/128/129 around a chunk; strong decay; many short sequences (many chains,
 tails of 1 token); one long sequence next to short ones, so that scheduling
 ranges start and end inside one chain; equal lengths, which must give the
 dense call's result bit for bit where both calls take the one-head kernel
@@ -29,15 +29,15 @@ from ssd_selective_scan_b200 import binding, layer, synth
 pytestmark = pytest.mark.gpu
 
 
-def _ragged(shape, lens, seed, init=True, dt_bias=True):
+def _ragged(shape, lens, seed, init=True, dt_bias=True, **decay):
     """Packed inputs of a ragged batch: x [T, H, P], B, C [T, G, N] (views of
     one [T, conv_dim] tensor), dt_raw [T, H], cu_seqlens, per-sequence init.
     dt_bias ~ N(0, 0.5) exercises the bias; dt_bias=False is the workloads'
     recipe (bias 0), which keeps the fp32 cumulative decays in the range the
-    1e-4 bound is set for."""
+    1e-4 bound is set for.  `decay` passes a_range / dt_range on."""
     T = int(sum(lens))
     s = shape.with_(b=1, L=max(T, 1))
-    inp = synth.scan_inputs(s, seed, dt_bias=dt_bias)
+    inp = synth.scan_inputs(s, seed, dt_bias=dt_bias, **decay)
     u = inp["u"][0, :T].cuda()
     x = u[:, : s.H * s.P].view(T, s.H, s.P)
     B = u[:, s.H * s.P: s.H * s.P + s.G * s.N].view(T, s.G, s.N)
@@ -100,6 +100,16 @@ def test_varlen_many_short_sequences():
     rng = np.random.default_rng(503)
     lens = list(rng.integers(0, 8, size=300))
     s, d = _ragged(BF16, lens, 503)
+    y, fs, st = _run(s, d)
+    _check(s, d, y, fs, st, "bf16")
+
+
+def test_varlen_strong_decay():
+    # |A| 12 to 50 and dt 0.7 to 2.1 (no bias): each token keeps between
+    # 2^-12 and 2^-153 of the state, so masked-out decay factors overflow
+    # and early columns underflow, in full and partial chunks
+    lens = [300, 1, 129, 0, 257]
+    s, d = _ragged(BF16, lens, 505, dt_bias=False, a_range=(8.0, 64.0), dt_range=(0.0, 2.0))
     y, fs, st = _run(s, d)
     _check(s, d, y, fs, st, "bf16")
 
