@@ -234,6 +234,7 @@ struct Params {
     const int* cu_seqlens;
     const int* seq_units;
     const int* ws_hdr;
+    int4* unit_desc;         // per unit: {chain, chunk, first token, end of its sequence}
     int nseq;
 };
 
@@ -248,7 +249,20 @@ struct Loc {
 struct Tabs {
     const int* cu;
     const int* su;
+    const int4* desc;   // per-unit descriptors (global memory)
 };
+
+// A unit descriptor written earlier in this kernel by this CTA (a plain
+// coherent load, never the read-only path).
+__device__ inline int4 ld_desc(const int4* p)
+{
+    int4 v;
+    asm volatile("ld.global.v4.s32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p)
+                 : "memory");
+    return v;
+}
 
 // `hint` is a sequence at or before u's; callers that visit units in
 // increasing order keep it and the search costs O(1) per call.
@@ -302,6 +316,8 @@ __device__ inline int seq_of_unit(const Params& p, const Tabs& tb, int u)
 struct Range {
     int chA, lenA;
     int uB0, nB, sB0;   // B: units [uB0, uB0 + nB); sB0 = sequence of uB0
+    int uA0, uC0;       // first units of A and of C (C's state-only items precede uC0)
+    int uEnd;           // one past the range's last unit
     int chC, startC, lenC;
     bool pubC;
     int npre;           // state-only items before C
@@ -324,6 +340,8 @@ __device__ inline Range make_range(const Params& p, const Tabs& tb, int t, int u
         int hint1 = kRagged ? seq_of_unit(p, tb, u1) : 0;
         b = locate<kRagged>(p, tb, u1, hint1);
     }
+    r.uC0 = u0;
+    r.uEnd = u1;
     if (a.chunk > 0 && b.chain == a.chain) {   // inside one chain
         r.chC = a.chain;
         r.startC = a.chunk;
@@ -335,6 +353,7 @@ __device__ inline Range make_range(const Params& p, const Tabs& tb, int t, int u
     }
     r.chA = b.chain;
     r.lenA = b.chunk;
+    r.uA0 = u1 - b.chunk;
     if (a.chunk > 0) {
         r.chC = a.chain;
         r.startC = a.chunk;
@@ -365,6 +384,46 @@ __device__ inline Item item_at(const Params& p, const Tabs& tb, const Range& r, 
 {
     Item it;
     it.pre = it.pre_first = it.pre_last = false;
+    if constexpr (kRagged) {
+        // the item's unit, then its descriptor
+        int u;
+        it.publish = it.depend = false;
+        if (idx < r.lenA) {
+            u = r.uA0 + idx;
+            it.seg_start = idx == 0;
+            it.seg_end = it.publish = idx == r.lenA - 1;
+        } else if (idx - r.lenA < r.nB) {
+            u = r.uB0 + (idx - r.lenA);
+        } else if (kLong && idx - r.lenA - r.nB < r.npre) {
+            const int k = idx - r.lenA - r.nB;   // walking back from chunk startC - 1
+            u = r.uC0 - 1 - k;
+            it.seg_start = it.seg_end = false;
+            it.pre = true;
+            it.pre_first = k == 0;
+            it.pre_last = k == r.npre - 1;
+        } else {
+            const int k = idx - r.lenA - r.nB - r.npre;
+            u = r.uC0 + k;
+            it.seg_start = it.depend = k == 0;
+            it.seg_end = k == r.lenC - 1;
+            it.publish = it.seg_end && r.pubC;
+        }
+        const int4 d = ld_desc(tb.desc + u);   // (written by this CTA in its prologue)
+        it.chain = d.x;
+        it.chunk = d.y;
+        it.tok0 = d.z;
+        it.nvalid = min(kQ, d.w - d.z);
+        if (idx >= r.lenA && idx - r.lenA < r.nB) {   // B: whole chains
+            it.seg_start = d.y == 0;
+            it.seg_end = d.w - d.z <= kQ;
+        }
+        it.seq = (int)p.fH.div((uint32_t)it.chain);
+        it.h = it.chain - it.seq * p.H;
+        it.bi = 0;
+        it.direct_y = it.nvalid < kQ;
+        (void)hint;
+        return it;
+    }
     if (idx < r.lenA) {
         it.chain = r.chA;
         it.chunk = idx;
@@ -484,7 +543,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     const int ticket = *ticket_slot;
     // a ragged batch reads its unit count (0 if cu_seqlens was invalid)
     const int units = kRagged ? (prm.ws_hdr[0] ? 0 : prm.ws_hdr[1]) : prm.units;
-    Tabs tabs{prm.cu_seqlens, prm.seq_units};
+    Tabs tabs{prm.cu_seqlens, prm.seq_units, prm.unit_desc};
     if constexpr (kRagged) {
         // the ragged tables into shared memory when they fit
         if (prm.nseq <= kMaxSeqSmem && units > 0) {
@@ -495,10 +554,27 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 ssu[i] = prm.seq_units[i];
             }
             __syncthreads();
-            tabs = Tabs{scu, ssu};
+            tabs = Tabs{scu, ssu, prm.unit_desc};
         }
     }
     const Range rg = make_range<kRagged, kLong>(prm, tabs, ticket, units);
+    if constexpr (kRagged) {
+        // the descriptors of this range's units (its state-only items'
+        // included), so that every role finds an item with one load; a
+        // unit shared with the range before is written by both CTAs with
+        // the same value
+        if (rg.count > 0) {
+            for (int u = rg.uC0 - rg.npre + tid; u < rg.uEnd; u += kThreads) {
+                const int sq = seq_of_unit(prm, tabs, u);
+                const int base = tabs.su[sq];
+                const int ncs = (tabs.su[sq + 1] - base) / prm.H;
+                const int h = (u - base) / ncs;
+                const int c = u - base - h * ncs;
+                prm.unit_desc[u] = make_int4(sq * prm.H + h, c, tabs.cu[sq] + c * kQ, tabs.cu[sq + 1]);
+            }
+        }
+        __syncthreads();
+    }
     auto group_of = [&](const Item& it) { return (int)prm.fHG.div((uint32_t)it.h); };
     auto stage = [&](int idx) { return smem + kOffStage + (idx & 1) * kStageBytes; };
 
@@ -1207,7 +1283,7 @@ chunk_scan_tc_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     const int ticket = *ticket_slot;
-    const Tabs tabs{nullptr, nullptr};
+    const Tabs tabs{nullptr, nullptr, nullptr};
     const Range rg = make_range<false, kLong>(prm, tabs, ticket, prm.units);
     auto group_of = [&](const Item& it) { return (int)prm.fHG.div((uint32_t)it.h); };
     auto xstage = [&](int idx) { return smem + pr::kOffX + (idx & 1) * pr::kXStage; };
@@ -1856,7 +1932,8 @@ size_t chunk_scan_tc_workspace_bytes(const ScanArgs& a)
     if (a.cu_seqlens) {   // ragged: the unit table comes first
         if (a.nseq <= 0) return 0;
         const int slots = tc_slots(a);
-        return varlen_table_bytes(a.nseq) + kWsCtrlBytes(slots) + (size_t)slots * kStateBytes;
+        return varlen_table_bytes(a.nseq) + varlen_desc_bytes(a.nseq, a.L, a.H, kQ) + kWsCtrlBytes(slots) +
+               (size_t)slots * kStateBytes;
     }
     if (a.b <= 0 || a.L <= 0) return 0;
     const int slots = tc_slots(a);
@@ -1886,7 +1963,9 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t s)
     if (e != cudaSuccess) return e;
     const size_t ctrl = kWsCtrlBytes(slots);
     const bool ragged = a.cu_seqlens != nullptr;
-    const size_t table = ragged ? varlen_table_bytes(a.nseq) : 0;
+    // a ragged batch: header and sequence table, then the unit descriptors
+    const size_t vtab = ragged ? varlen_table_bytes(a.nseq) : 0;
+    const size_t table = ragged ? vtab + varlen_desc_bytes(a.nseq, a.L, a.H, kQ) : 0;
     if (!a.workspace || a.workspace_bytes < table + ctrl + (size_t)slots * kStateBytes * (pairs ? 2 : 1))
         return cudaErrorInvalidValue;
     uint8_t* ws = static_cast<uint8_t*>(a.workspace);
@@ -1924,6 +2003,7 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t s)
     prm.cu_seqlens = a.cu_seqlens;
     prm.seq_units = ragged ? reinterpret_cast<const int*>(ws + kVarlenUnitsOffset) : nullptr;
     prm.ws_hdr = ragged ? reinterpret_cast<const int*>(ws) : nullptr;
+    prm.unit_desc = ragged ? reinterpret_cast<int4*>(ws + vtab) : nullptr;
     prm.nseq = ragged ? a.nseq : a.b;
     prm.status = a.status;
     kernel<<<slots, kThreads, smem_bytes, s>>>(tmX, tmB, tmC, tmY, prm);

@@ -42,6 +42,16 @@ cudaError_t launch_varlen_prep(const int* cu_seqlens, int nseq, int T, int H, in
                                int* ctrl, int ctrl_ints, const float* init_state, float* final_state,
                                long long state_elems_per_seq, int32_t* status, cudaStream_t s);
 
+// Per-unit descriptors of a ragged batch's unit list (the tensor-core scan;
+// each CTA writes those of its own range): unit u -> {chain s * H + h,
+// chunk c, first token cu[s] + c * Q, end of the sequence cu[s + 1]}.  A
+// batch has at most H * (ceil(T / Q) + nseq) units.
+inline size_t varlen_desc_bytes(int nseq, long long T, int H, int Q)
+{
+    const long long units = (long long)H * ((T + Q - 1) / Q + nseq);
+    return ((size_t)units * 16 + 255) / 256 * 256;
+}
+
 // in_stride: elements between consecutive input tokens (0: conv_dim)
 cudaError_t launch_conv1d_silu(const void* xBC, void* out, const float* w, const float* bias,
                                void* conv_state, int b, int L, int conv_dim, int k, bool bf16,
