@@ -62,6 +62,7 @@ BWD = synth.CONFIGS[1]            # the backward pass is timed on the 3B layer
 MIXER = synth.CONFIGS[1]          # the whole mixer is timed on the 3B layer ...
 MIXER_D_MODEL = 2560              # ... with its d_model
 DECODE = synth.CONFIGS[4]
+RAGGED = synth.CONFIGS[1]         # ragged prefill: the 3B layer's tokens packed as prompts of mixed lengths
 ORACLE_PREFIX = 4096              # tokens of the headline workload the oracle times
 E2E_PIECES = 8                    # the end-to-end leg streams the sequence in this many pieces
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
@@ -324,6 +325,39 @@ class MixerStep:
 
     def in_proj(self):
         self.layer.linear(self.d["hidden"].view(-1, self.d_model), self.d["W_in"], y=self.zx)
+
+
+class RaggedStep:
+    """The ragged scan (ssd_chunk_scan_fwd_varlen) on a prefill workload's
+    tokens packed as a batch of prompts: a seeded length mix, or the
+    workload's own equal lengths."""
+
+    def __init__(self, s, seed, dev, lens=None):
+        from ssd_selective_scan_b200 import layer
+        self.layer = layer
+        T = s.b * s.L
+        self.lens = synth.ragged_lengths(T, seed) if lens is None else list(lens)
+        self.s = s.with_(b=1, L=T)
+        inp = synth.scan_inputs(self.s, seed)
+        u = inp["u"][0].to(dev)
+        x, B, C = layer.split_channels(u, s.H, s.P, s.G, s.N)
+        self.x, self.B, self.C = x.view(T, s.H, s.P), B.view(T, s.G, s.N), C.view(T, s.G, s.N)
+        self.dt = inp["dt_raw"][0].contiguous().to(dev)
+        self.A, self.dtb, self.D = inp["A"].to(dev), inp["dt_bias"].to(dev), inp["D"].to(dev)
+        offs = [0]
+        for n in self.lens:
+            offs.append(offs[-1] + n)
+        self.cu = torch.tensor(offs, dtype=torch.int32, device=dev)
+        self.y = torch.empty(T, s.H, s.P, dtype=s.torch_dtype, device=dev)
+        self.fs = torch.empty(len(self.lens), s.H, s.P, s.N, dtype=torch.float32, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        need = layer.chunk_scan_varlen_workspace_bytes(len(self.lens), T, s.H, s.P, s.N, s.G, s.Q, s.torch_dtype)
+        self.ws = torch.empty(need, dtype=torch.uint8, device=dev)
+
+    def __call__(self):
+        self.layer.chunk_scan_fwd_varlen(self.x, self.B, self.C, self.dt, self.A, self.cu, self.dtb, self.D, None,
+                                         Q=self.s.Q, y=self.y, final_state=self.fs, workspace=self.ws,
+                                         status=self.status)
 
 
 class DecodeStep:
@@ -615,10 +649,26 @@ def run_ours(args, rank, world, dev):
     del mx
     torch.cuda.empty_cache()
 
+    # the ragged scan: the 3B layer's 16384 tokens as a mix of prompt
+    # lengths, and as its own 8 equal sequences (against the dense call)
+    rag = RaggedStep(RAGGED, shard.rank_seed(synth.config_seed(1), rank), dev)
+    rag_ms = time_fn(rag, KM)
+    rag_lens = rag.lens
+    rag_status = int(rag.status.item())
+    del rag
+    req = RaggedStep(RAGGED, shard.rank_seed(synth.config_seed(1), rank), dev, lens=[RAGGED.L] * RAGGED.b)
+    req_ms = time_fn(req, KM)
+    del req
+    torch.cuda.empty_cache()
+    if rag_status != 0:
+        raise RuntimeError(f"ragged scan reported status {rag_status}")
+
     if rank != 0:
         return None
     btok = BWD.b * BWD.L
     mtok = MIXER.b * MIXER.L
+    rtok = RAGGED.b * RAGGED.L
+    rbytes = scan_bytes_per_token(RAGGED) * rtok
     nproj = 2 * MIXER.H * MIXER.P + 2 * MIXER.G * MIXER.N + MIXER.H
     line = {
         "metric": METRIC,
@@ -658,6 +708,15 @@ def run_ours(args, rank, world, dev):
                      "TFLOP/s": scan_bwd_flops_per_token(BWD) * btok / (bwd_ms * 1e-3) / 1e12,
                      "frac_bf16_peak": scan_bwd_flops_per_token(BWD) * btok / (bwd_ms * 1e-3) / 1e12 /
                                        peaks["bf16_tflops"]},
+        "ragged": {"workload": f"{RAGGED.name} tokens as {len(rag_lens)} prompts of 64-4096 tokens "
+                               "(seeded log-uniform mix)",
+                   "kernel": "ssd_chunk_scan_fwd_varlen (preparation kernel + tensor-core scan, one head per item)",
+                   "tokens": rtok, "nseq": len(rag_lens), "ms": rag_ms,
+                   "tokens_per_s": world * rtok / (rag_ms * 1e-3),
+                   "GB/s": rbytes / (rag_ms * 1e-3) / 1e9,
+                   "frac_hbm": rbytes / (rag_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                   "equal_lengths_ms": req_ms,
+                   "dense_scan_ms": blocks[RAGGED.name]["scan"]["launch_ms"]},
         "mixer": {"workload": MIXER.name, "d_model": MIXER_D_MODEL,
                   "kernels": "in_proj (tcgen05 linear), conv1d+SiLU, chunk scan, gated RMSNorm, out_proj",
                   "ms": mix_ms, "tokens_per_s": world * mtok / (mix_ms * 1e-3),

@@ -196,3 +196,19 @@ def mixer_inputs(shape: LayerShape, d_model: int, seed: int, *, conv_bias: bool 
     out["conv_state"] = (_xbc(s, (s.b, s.k), g).transpose(1, 2).contiguous().to(torch.bfloat16)) if conv_state else None
     out["init_state"] = (torch.randn(s.b, s.H, s.P, s.N, generator=g) * math.sqrt(0.1)) if init_state else None
     return out
+
+
+def ragged_lengths(total: int, seed: int, lo: int = 64, hi: int = 4096) -> list:
+    """A serving-like prefill batch of `total` packed tokens: prompt lengths
+    drawn log-uniformly from [lo, hi] until the next one would overflow the
+    total, the last prompt taking what is left (the pages give no length
+    mix; this one spans a chunk's 128 tokens on both sides)."""
+    g = _gen(seed)
+    lens, left = [], total
+    while left > 0:
+        u = float(torch.rand(1, generator=g))
+        n = int(round(math.exp(math.log(lo) + u * (math.log(hi) - math.log(lo)))))
+        n = min(n, left) if left - n >= lo else left
+        lens.append(n)
+        left -= n
+    return lens

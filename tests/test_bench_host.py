@@ -1,6 +1,7 @@
 """The benchmark's algorithmic work per token and per step (CPU only): the
 byte and FLOP counts behind every roofline fraction, checked against their
-definitions worked out by hand for the bench workloads."""
+definitions worked out by hand for the bench workloads, and the seeded
+prompt-length mix of the ragged block."""
 import bench
 from ssd_selective_scan_b200 import synth
 
@@ -30,3 +31,13 @@ def test_peaks_fallback_is_labelled(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))   # no MEASURED_PEAKS.json there
     p = bench.load_peaks()
     assert p["source"] == "fallback" and p["hbm_gbs"] == 6650.0 and p["bf16_tflops"] == 1590.0
+
+
+def test_ragged_length_mix():
+    from ssd_selective_scan_b200 import synth
+    a = synth.ragged_lengths(16384, 11)
+    assert a == synth.ragged_lengths(16384, 11), "not reproducible from its seed"
+    assert sum(a) == 16384 and len(a) > 1
+    assert all(64 <= n < 4096 + 64 for n in a)
+    assert synth.ragged_lengths(16384, 12) != a
+    assert synth.ragged_lengths(100, 3) == [100]

@@ -8,7 +8,8 @@ sequence alone in fp64 on the exact values the GPU consumed.
 
 Covered: the tensor-core path (bf16, P = 64, N = 128, Q = 128) and the
 general path (fp32); empty sequences inside and at the end of the batch;
-lengths 1, 127/128/129 around a chunk; strong decay; many short sequences (many chains,
+lengths 1, 127/128/129 around a chunk; strong decay; the benchmark's prompt-length
+mix; many short sequences (many chains,
 tails of 1 token); one long sequence next to short ones, so that scheduling
 ranges start and end inside one chain; equal lengths, which must give the
 dense call's result bit for bit where both calls take the one-head kernel
@@ -110,6 +111,15 @@ def test_varlen_strong_decay():
     # and early columns underflow, in full and partial chunks
     lens = [300, 1, 129, 0, 257]
     s, d = _ragged(BF16, lens, 505, dt_bias=False, a_range=(8.0, 64.0), dt_range=(0.0, 2.0))
+    y, fs, st = _run(s, d)
+    _check(s, d, y, fs, st, "bf16")
+
+
+def test_varlen_prompt_length_mix():
+    # the benchmark's recipe of prompt lengths (log-uniform 64-4096 tokens)
+    lens = synth.ragged_lengths(6000, 77)
+    assert len(lens) > 2
+    s, d = _ragged(BF16, lens, 506)
     y, fs, st = _run(s, d)
     _check(s, d, y, fs, st, "bf16")
 
