@@ -486,13 +486,20 @@ __device__ inline void tmem_ld8(uint32_t taddr, float (&v)[8])
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// y tensor maps with boxes of 64, 32, 16 and 8 rows: a ragged batch's
+// partial last chunk stores its first rows (a multiple of 8) with at most
+// four of them, never reaching the next sequence's rows.
+struct YBoxes {
+    CUtensorMap m[4];
+};
+
 // kLong: ranges inside chains rebuild their starting state (state-only
 // items); without it that code is compiled out.
 template <bool kRagged, bool kLong>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY,
-                     const Params prm)
+                     const __grid_constant__ YBoxes ypart, const Params prm)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -652,15 +659,15 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             // The coordinates of an item, computed once (for its L2
             // prefetch) and passed along a rotation of items idx .. idx + 3.
             struct Co {
-                int g, h, tok0, bi;
+                int g, h, tok0, bi, nvalid;
                 bool direct_y, pre;
             };
             int hint = rg.sB0;   // items are visited in increasing order
             auto coord = [&](int idx) {
-                Co c{0, 0, 0, 0, false, false};
+                Co c{0, 0, 0, 0, 0, false, false};
                 if (idx < rg.count) {
                     const Item it = item_at<kRagged, kLong>(prm, tabs, rg, idx, hint);
-                    c = Co{group_of(it), it.h, it.tok0, it.bi, it.direct_y, kLong && it.pre};
+                    c = Co{group_of(it), it.h, it.tok0, it.bi, it.nvalid, it.direct_y, kLong && it.pre};
                 }
                 return c;
             };
@@ -720,9 +727,26 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 // y of item idx is staged in its X buffer: store it, then
                 // reload the buffer once the store has read it
                 mbar_wait_bounded(bar_ystaged + (idx & 1), sph, kWaitNs, aborted, prm.status);
-                if (!c0.direct_y && !(kLong && c0.pre)) {   // (a partial ragged chunk's rows went out directly;
-                                                 //  a state-only item has no y)
-                    tma_store_3d(&tmY, stage(idx) + kStX, c0.h * kP, c0.tok0, c0.bi);
+                if (!(kLong && c0.pre)) {   // (a state-only item has no y)
+                    if (!c0.direct_y) {
+                        tma_store_3d(&tmY, stage(idx) + kStX, c0.h * kP, c0.tok0, c0.bi);
+                    } else if constexpr (kRagged) {
+                        // a partial last chunk: its rows up to the last
+                        // multiple of 8 in boxes of 64, 32, 16, 8 rows (each
+                        // starting on a whole swizzle atom); the rest went
+                        // out row by row from the elementwise warps
+                        const int nfull = c0.nvalid & ~7;
+                        int off = 0;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const int rows = 64 >> q;
+                            if (nfull & rows) {
+                                tma_store_3d(&ypart.m[q], stage(idx) + kStX + off * 128, c0.h * kP, c0.tok0 + off,
+                                             c0.bi);
+                                off += rows;
+                            }
+                        }
+                    }
                     bulk_commit_group();
                     bulk_wait_group_read0();
                 }
@@ -930,24 +954,19 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 }
                 packed[q] = pack_bf16x8(o);
             }
-            bool staged = true;
             if constexpr (kRagged) {
-                if (prev_direct) {
-                    // a ragged batch's partial last chunk: its rows past the
-                    // sequence's end belong to the next sequence, so the rows
-                    // go out one by one instead of as a 128-row TMA box
-                    staged = false;
-                    if (row < prev_nvalid) {
-                        __nv_bfloat16* yr = prm.y + ((size_t)(prev_tok0 + row) * H + prev_h) * kP + p0;
-                        reinterpret_cast<uint4*>(yr)[0] = packed[0];
-                        reinterpret_cast<uint4*>(yr)[1] = packed[1];
-                    }
+                // a ragged batch's partial last chunk: its rows past the
+                // sequence's end belong to the next sequence, so no 128-row
+                // box goes out; the producer stores the rows up to the last
+                // multiple of 8 in smaller boxes, and the rest go out here
+                if (prev_direct && row >= (prev_nvalid & ~7) && row < prev_nvalid) {
+                    __nv_bfloat16* yr = prm.y + ((size_t)(prev_tok0 + row) * H + prev_h) * kP + p0;
+                    reinterpret_cast<uint4*>(yr)[0] = packed[0];
+                    reinterpret_cast<uint4*>(yr)[1] = packed[1];
                 }
             }
-            if (staged) {
 #pragma unroll
-                for (int q = 0; q < 2; ++q) *reinterpret_cast<uint4*>(xs + sw128(row, quarter * 2 + q)) = packed[q];
-            }
+            for (int q = 0; q < 2; ++q) *reinterpret_cast<uint4*>(xs + sw128(row, quarter * 2 + q)) = packed[q];
             fence_proxy_async_smem();
             mbar_arrive(bar_ystaged + (j & 1));
         };
@@ -1236,7 +1255,7 @@ template <bool kLong>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_scan_tc_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY,
-                          const Params prm)
+                          const __grid_constant__ YBoxes ypart, const Params prm)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1865,13 +1884,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled_fn()
 // dim1 = tokens (stride row_bytes), dim2 = sequences (stride L * row_bytes);
 // box 64 channels x 128 tokens x 1, 128-byte swizzle, zero fill out of range.
 cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t channels, uint64_t L, uint64_t b,
-                     uint64_t row_bytes)
+                     uint64_t row_bytes, uint32_t box_rows = kQ)
 {
     auto fn = encode_tiled_fn();
     if (!fn) return cudaErrorNotSupported;
     const cuuint64_t dims[3] = {channels, L, b};
     const cuuint64_t strides[2] = {row_bytes, row_bytes * L};
-    const cuuint32_t box[3] = {64, (cuuint32_t)kQ, 1};
+    const cuuint32_t box[3] = {64, box_rows, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1950,6 +1969,13 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t s)
     if ((e = make_map(&tmC, a.C, (uint64_t)a.G * a.N, a.L, a.b, rb)) != cudaSuccess) return e;
     CUtensorMap tmY;
     if ((e = make_map(&tmY, a.y, (uint64_t)a.H * a.P, a.L, a.b, (uint64_t)a.H * a.P * 2)) != cudaSuccess) return e;
+    YBoxes ypart{};   // (used by ragged batches only)
+    if (a.cu_seqlens) {   // a ragged batch's partial last chunks
+        for (int q = 0; q < 4; ++q)
+            if ((e = make_map(&ypart.m[q], a.y, (uint64_t)a.H * a.P, a.L, a.b, (uint64_t)a.H * a.P * 2,
+                              (uint32_t)(64 >> q))) != cudaSuccess)
+                return e;
+    }
     bool long_chains = false;
     const int slots = tc_slots(a, &long_chains);
     const bool pairs = tc_pairs(a);
@@ -2006,7 +2032,7 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t s)
     prm.unit_desc = ragged ? reinterpret_cast<int4*>(ws + vtab) : nullptr;
     prm.nseq = ragged ? a.nseq : a.b;
     prm.status = a.status;
-    kernel<<<slots, kThreads, smem_bytes, s>>>(tmX, tmB, tmC, tmY, prm);
+    kernel<<<slots, kThreads, smem_bytes, s>>>(tmX, tmB, tmC, tmY, ypart, prm);
     return cudaGetLastError();
 }
 
