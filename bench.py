@@ -808,6 +808,8 @@ def run_one_kernel(args, dev):
     elif args.kernel == "bwd":
         s = BWD if args.seq_len is None else BWD.with_(L=args.seq_len)
         fn = BackwardStep(s, synth.config_seed(1), dev)
+    elif args.kernel == "ragged":
+        fn = RaggedStep(RAGGED, synth.config_seed(1), dev)
     else:
         s = synth.CONFIGS[args.workload]
         if args.seq_len is not None:
@@ -824,7 +826,9 @@ def run_one_kernel(args, dev):
         fn()
     e1.record()
     torch.cuda.synchronize()
-    print(json.dumps({"kernel": args.kernel, "workload": args.workload, "seq_len": args.seq_len,
+    workload = {"decode": DECODE.name, "mixer": MIXER.name, "linear": MIXER.name, "bwd": BWD.name,
+                "ragged": RAGGED.name + " as a prompt-length mix"}.get(args.kernel, args.workload)
+    print(json.dumps({"kernel": args.kernel, "workload": workload, "seq_len": args.seq_len,
                       "launches": args.steps, "ms_per_launch": e0.elapsed_time(e1) / args.steps}), flush=True)
 
 
@@ -835,7 +839,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["scan", "conv", "decode", "bwd", "mixer", "linear"],
+    ap.add_argument("--kernel", choices=["scan", "conv", "decode", "bwd", "mixer", "linear", "ragged"],
                     help="launch only this kernel (warmup + steps launches) and print its mean "
                          "CUDA-event time; for profiler captures")
     ap.add_argument("--workload", type=int, choices=PREFILL_CONFIGS, default=HEADLINE,
