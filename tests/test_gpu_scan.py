@@ -7,7 +7,9 @@ size-independent properties (the 262144-token one).  Both tensor-core
 kernels are covered: dense batches whose groups hold an even number of
 heads run head pairs (e.g. 2, 4, 6, 8 and 16 heads per group below, the
 8B and long-context workloads), the others one head per item (1, 3 and 5
-heads per group, the 3B workload); each in its dense and long-chain forms."""
+heads per group, the 3B workload); each in its dense and long-chain forms,
+with long-memory heads (|A| down to 0.01) and with strong decay (|A| up to
+50, dt up to 2.1), where the decay factors of masked-out columns overflow."""
 import math
 
 import numpy as np
